@@ -1,0 +1,350 @@
+#!/usr/bin/env python
+"""Benchmark of the Naju scan hot path (fwd + bwd) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one forward (fused conv + scan + readout + SiLU(z) modulation) and
+one backward over one batch of the workload's synthetic inputs, all resident
+in HBM.  Prints one JSON line (rank 0).  Under torchrun each rank runs its own
+replica of the workload (batch elements are independent; weak scaling, no
+collective on the data path); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from discrete_selective_ssm_b200.workloads import WORKLOADS, make_inputs, scaled  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def alg_bytes(w, E):
+    """Algorithmic HBM bytes of one fwd and one bwd over workload w with
+    activation element size E (inputs read once, outputs written once)."""
+    T = w.batch * w.seqlen
+    d, N = w.d_inner, w.d_state
+    fwd = T * (5 * E * d + 2 * E * N) + w.batch * d * N * 4
+    bwd = T * (9 * E * d + 4 * E * N) + w.batch * d * N * 4
+    return fwd, bwd
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_oracle_step(w, t, n_batch=1):
+    """One fwd + bwd of the fp64 oracle over the first n_batch batch elements
+    of the workload.  Returns (seconds, tokens, threads)."""
+    import oracle
+    sl = {k: (v[:n_batch] if k in ("u", "a", "b", "B", "C", "z", "dout") else v)
+          for k, v in t.items()}
+    t0 = time.perf_counter()
+    oracle.block_fwd(sl["u"], sl["conv_w"], sl["conv_b"], sl["a"], sl["b"], sl["B"], sl["C"],
+                     sl["z"], sl["D"])
+    oracle.block_bwd(sl["u"], sl["conv_w"], sl["conv_b"], sl["a"], sl["b"], sl["B"], sl["C"],
+                     sl["z"], sl["D"], None, sl["dout"])
+    return time.perf_counter() - t0, n_batch * w.seqlen, oracle.num_threads()
+
+
+def cpu_sample_workload(w):
+    """Bounded CPU sample: one batch element, the sequence cut to keep the
+    oracle's fwd+bwd around 10-20 s on a few host cores."""
+    per_tok = w.d_inner * w.d_state  # state updates per token
+    L = max(64, min(w.seqlen, int(6e8 / per_tok)))
+    return scaled(w, batch=1, seqlen=L)
+
+
+def run_reference(args, w, rank, world):
+    """The oracle as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    ws = cpu_sample_workload(w)
+    t = make_inputs(ws, which=("u", "a", "b", "B", "C", "z", "D", "conv_w", "conv_b", "dout"))
+    for _ in range(max(0, min(args.warmup, 1))):
+        cpu_oracle_step(ws, t)
+    times = []
+    for _ in range(args.steps):
+        dt, toks, thr = cpu_oracle_step(ws, t)
+        times.append(dt)
+    ms = 1e3 * statistics.mean(times)
+    val = ws.batch * ws.seqlen / (ms / 1e3)
+    sample = (f"oracle fwd+bwd on batch 1 x L={ws.seqlen} x d_inner={ws.d_inner} x "
+              f"d_state={ws.d_state} (slice of {w.name})")
+    print(json.dumps({
+        "metric": "naju_scan_fwd_bwd_tokens_per_s", "value": val, "unit": "tokens/s",
+        "impl": "reference", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                   "d_inner": w.d_inner, "d_state": w.d_state, "dtype_inputs": w.dtype},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="throughput_train", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+    if w.decode_steps:
+        raise SystemExit("decode workloads are parity cases; bench a training workload")
+
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+
+    import discrete_selective_ssm_b200 as naju
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    t_host = make_inputs(w, which=("u", "a", "b", "B", "C", "z", "D", "conv_w", "conv_b", "dout"))
+    t = {k: v.to(dev) for k, v in t_host.items()}
+    E = 2 if w.dtype == "bf16" else 4
+    out_dt = naju.BF16 if w.dtype == "bf16" else naju.F32
+    dims = naju.make_dims(w.batch, w.seqlen, w.d_inner, w.d_state,
+                          naju.BF16 if w.dtype == "bf16" else naju.F32, out_dt)
+    ws = naju.alloc_workspace(dims, dev)
+    y = torch.empty((w.batch, w.seqlen, w.d_inner), dtype=w.torch_dtype, device=dev)
+    ot = w.torch_dtype
+    shp = (w.batch, w.seqlen, w.d_inner)
+    grads = {"dhu": torch.empty(shp, dtype=ot, device=dev),
+             "da": torch.empty(shp, dtype=ot, device=dev),
+             "db": torch.empty(shp, dtype=ot, device=dev),
+             "dz": torch.empty(shp, dtype=ot, device=dev),
+             "dB": torch.empty((w.batch, w.seqlen, w.d_state), dtype=ot, device=dev),
+             "dC": torch.empty((w.batch, w.seqlen, w.d_state), dtype=ot, device=dev),
+             "dD": torch.empty(w.d_inner, dtype=torch.float32, device=dev),
+             "dconv_w": torch.empty_like(t["conv_w"]),
+             "dconv_b": torch.empty(w.d_inner, dtype=torch.float32, device=dev),
+             "dx0": None}
+    stream = torch.cuda.current_stream()
+
+    def step(inp, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        naju.scan_fwd(inp["u"], inp["a"], inp["b"], inp["B"], inp["C"], conv_w=inp["conv_w"],
+                      conv_b=inp["conv_b"], z=inp["z"], D=inp["D"], out_dtype=out_dt,
+                      workspace=ws, want_final=False, y=y)
+        if ev is not None:
+            ev[1].record(stream)
+        naju.scan_bwd(inp["dout"], inp["u"], inp["a"], inp["b"], inp["B"], inp["C"], ws,
+                      conv_w=inp["conv_w"], conv_b=inp["conv_b"], z=inp["z"], D=inp["D"],
+                      out_dtype=out_dt, grads=grads)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step(t)
+    torch.cuda.synchronize()
+    if naju.last_device_status(ws) != 0:
+        raise SystemExit("device status not OK after warm-up")
+
+    # ---------------------------------------------------------- timed region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(t, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = clk.stop()
+    ms_total = start.elapsed_time(end)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    if naju.last_device_status(ws) != 0:
+        raise SystemExit("device status not OK after the timed region")
+    if dist is not None:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    tokens = w.batch * w.seqlen
+    value = world * tokens / (ms_step / 1e3)
+
+    # -------------------------------------------------------------- e2e leg
+    pinned = {k: v.pin_memory() for k, v in t_host.items()}
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    outs = [y] + [v for v in grads.values() if v is not None]
+    host_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    dev_in = {k: torch.empty_like(v) for k, v in t.items()}
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        step(dev_in)
+        for ho, o in zip(host_outs, outs):
+            ho.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = s2.elapsed_time(e2) / args.e2e_steps
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_val = world * tokens / (e2e_ms / 1e3)
+
+    # ---------------------------------------------------------------- roofline
+    pk, pk_kind = peaks()
+    fwd_b, bwd_b = alg_bytes(w, E)
+    dom_is_bwd = bwd_ms >= fwd_ms
+    dom_ms = bwd_ms if dom_is_bwd else fwd_ms
+    dom_b = bwd_b if dom_is_bwd else fwd_b
+    achieved = dom_b / (dom_ms / 1e3) / 1e9
+    peak = float(pk["hbm_gbs"])
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")
+    if os.path.exists(prof):
+        with open(prof) as fh:
+            tr = json.load(fh)
+        traffic = tr.get("bwd" if dom_is_bwd else "fwd")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ws_cpu = cpu_sample_workload(w)
+        tc = make_inputs(ws_cpu, which=("u", "a", "b", "B", "C", "z", "D", "conv_w", "conv_b",
+                                        "dout"))
+        dt, toks, thr = cpu_oracle_step(ws_cpu, tc)
+        cpu = {"value": toks / dt, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+               "sample": f"oracle fwd+bwd, batch 1 x L={ws_cpu.seqlen} slice of {w.name}, "
+                         f"{dt:.1f} s"}
+
+    if rank == 0:
+        print(json.dumps({
+            "metric": "naju_scan_fwd_bwd_tokens_per_s", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                       "d_inner": w.d_inner, "d_state": w.d_state, "conv_width": 4,
+                       "fused_conv": True, "gating": True, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (no flush)",
+                       "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+                       "fwd_gbs": fwd_b / (fwd_ms / 1e3) / 1e9,
+                       "bwd_gbs": bwd_b / (bwd_ms / 1e3) / 1e9,
+                       "fwd_frac_hbm": fwd_b / (fwd_ms / 1e3) / 1e9 / peak,
+                       "bwd_frac_hbm": bwd_b / (bwd_ms / 1e3) / 1e9 / peak},
+            "roofline": {"bound": "hbm", "kernel": "scan_bwd" if dom_is_bwd else "scan_fwd",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "alg_bytes": dom_b, "peak_kind": pk_kind},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 5 * args.steps,
+            "clocks": clocks,
+        }), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,271 @@
+// C ABI of the Naju scan library: argument checks, workspace layout and
+// kernel launches.  See include/naju.h for the contract of each entry point.
+#include <stdint.h>
+#include <string.h>
+
+#include <cmath>
+
+#include "naju.h"
+#include "naju_common.cuh"
+#include "naju_kernels.h"
+#include "naju_testing.h"
+
+using namespace naju;
+
+namespace {
+
+constexpr int kSMs = 148;
+constexpr int kTck = 128;          // tokens per forward checkpoint segment
+constexpr long long kDefaultWait = 1LL << 21;
+
+long long g_wait_limit = kDefaultWait;
+int g_skip_publish = 0;
+int g_fwd_groups = 0;
+
+inline bool aligned(const void* ptr, size_t a) {
+    return (reinterpret_cast<uintptr_t>(ptr) % a) == 0;
+}
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+naju_status check_dims(const naju_dims* dm) {
+    if (!dm) return NAJU_ERR_INVALID_ARG;
+    if (dm->batch < 1 || dm->seqlen < 1 || dm->d_inner < 1 || dm->reserved != 0)
+        return NAJU_ERR_INVALID_ARG;
+    if (dm->batch > (1 << 20) || dm->seqlen > (1LL << 26) || dm->d_inner > (1 << 20))
+        return NAJU_ERR_INVALID_ARG;
+    if (dm->batch * dm->seqlen * dm->d_inner > (1LL << 40)) return NAJU_ERR_INVALID_ARG;
+    if (dm->d_state != 16 && dm->d_state != 32 && dm->d_state != 64 && dm->d_state != 128)
+        return NAJU_ERR_UNSUPPORTED;
+    if (dm->dtype != NAJU_F32 && dm->dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
+    if (dm->out_dtype != NAJU_F32 && dm->out_dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
+    if (dm->dtype == NAJU_F32 && dm->out_dtype != NAJU_F32) return NAJU_ERR_UNSUPPORTED;
+    return NAJU_OK;
+}
+
+// Workspace layout (every region 256-byte aligned).
+struct Layout {
+    int nck, ngroups, seg_per_group, ntiles_f;
+    int nsub, nclus, ntiles_b;
+    size_t off_fflags, off_bflags, off_ckpt, off_carry, off_dbc, off_chan, off_edge, total;
+};
+
+int auto_groups(const naju_dims* dm, int nck, int ntiles_f) {
+    if (g_fwd_groups > 0) return g_fwd_groups < nck ? g_fwd_groups : nck;
+    const int64_t items = dm->batch * (int64_t)ntiles_f;
+    const int64_t want = 3 * kSMs;
+    if (items >= want) return 1;
+    int64_t g = cdiv(want, items);
+    return (int)(g < nck ? g : nck);
+}
+
+Layout layout(const naju_dims* dm) {
+    Layout l{};
+    const int64_t Bt = dm->batch, L = dm->seqlen, d = dm->d_inner, N = dm->d_state;
+    l.nck = (int)cdiv(L, kTck);
+    l.ntiles_f = (int)cdiv(d, fwd_channels_per_block(N));
+    int g = auto_groups(dm, l.nck, l.ntiles_f);
+    l.seg_per_group = (int)cdiv(l.nck, g);
+    l.ngroups = (int)cdiv(l.nck, l.seg_per_group);
+    l.nsub = (int)cdiv(L, kBwdSub);
+    const int tiles_b = (int)cdiv(d, bwd_channels_per_block(N));
+    l.nclus = (int)cdiv(tiles_b, bwd_cluster_size());
+    l.ntiles_b = l.nclus * bwd_cluster_size();
+    size_t off = sizeof(WsHeader);
+    l.off_fflags = off;
+    off = up256(off + sizeof(int) * (size_t)l.ngroups * Bt * l.ntiles_f);
+    l.off_bflags = off;
+    off = up256(off + sizeof(int) * (size_t)l.nsub * Bt * l.ntiles_b);
+    l.off_ckpt = off;
+    off = up256(off + sizeof(float) * (size_t)Bt * (l.nck + 1) * d * N);
+    l.off_carry = off;
+    off = up256(off + sizeof(float) * (size_t)l.nsub * Bt * d * N);
+    l.off_dbc = off;
+    off = up256(off + sizeof(float) * (size_t)l.nclus * Bt * L * 2 * N);
+    l.off_chan = off;
+    off = up256(off + sizeof(float) * (size_t)Bt * l.nsub * d * 8);
+    l.off_edge = off;
+    off = up256(off + sizeof(float) * (size_t)Bt * l.nsub * 2 * 3 * d);
+    l.total = off;
+    return l;
+}
+
+inline naju_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NAJU_OK : NAJU_ERR_CUDA; }
+
+#define NAJU_REQUIRE(cond) \
+    do {                   \
+        if (!(cond)) return NAJU_ERR_INVALID_ARG; \
+    } while (0)
+
+inline bool ok_act(const void* p) { return p && aligned(p, 16); }
+inline bool ok_opt(const void* p) { return !p || aligned(p, 16); }
+
+}  // namespace
+
+extern "C" {
+
+size_t naju_scan_workspace_bytes(const naju_dims* dims) {
+    if (check_dims(dims) != NAJU_OK) return 0;
+    return layout(dims).total;
+}
+
+naju_status naju_conv_silu_fwd(const naju_dims* dims, const void* u, const float* conv_w,
+                               const float* conv_b, void* h, void* stream) {
+    naju_status st = check_dims(dims);
+    if (st != NAJU_OK) return st;
+    if (dims->conv_width != 4) return NAJU_ERR_UNSUPPORTED;
+    NAJU_REQUIRE(ok_act(u) && ok_act(h) && conv_w && ok_opt(conv_b));
+    return cuda_status(launch_conv_fwd(dims->batch, dims->seqlen, dims->d_inner, u, conv_w,
+                                       conv_b, h, dims->dtype, dims->out_dtype,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+naju_status naju_conv_silu_bwd(const naju_dims* dims, const void* u, const float* conv_w,
+                               const float* conv_b, const void* dh, void* du, float* dconv_w,
+                               float* dconv_b, void* stream) {
+    naju_status st = check_dims(dims);
+    if (st != NAJU_OK) return st;
+    if (dims->conv_width != 4) return NAJU_ERR_UNSUPPORTED;
+    if (dims->dtype != dims->out_dtype) return NAJU_ERR_UNSUPPORTED;  // dh arrives in dtype
+    NAJU_REQUIRE(ok_act(u) && ok_act(dh) && ok_act(du) && conv_w && dconv_w);
+    return cuda_status(launch_conv_bwd(dims->batch, dims->seqlen, dims->d_inner, u, conv_w,
+                                       conv_b, dh, du, dconv_w, dconv_b, dims->dtype,
+                                       dims->out_dtype, static_cast<cudaStream_t>(stream)));
+}
+
+naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* conv_w,
+                          const float* conv_b, const void* a, const void* b, const void* B,
+                          const void* C, const void* z, const float* D, const float* x0,
+                          void* y, float* x_final, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    naju_status st = check_dims(dims);
+    if (st != NAJU_OK) return st;
+    if (conv_w && dims->conv_width != 4) return NAJU_ERR_UNSUPPORTED;
+    NAJU_REQUIRE(ok_act(hu) && ok_act(a) && ok_act(b) && ok_act(B) && ok_act(C) && ok_act(y));
+    NAJU_REQUIRE(ok_opt(z) && ok_opt(x0) && ok_opt(x_final));
+    NAJU_REQUIRE(workspace && aligned(workspace, 256));
+    const Layout l = layout(dims);
+    NAJU_REQUIRE(workspace_bytes >= l.total);
+    NAJU_REQUIRE((int64_t)l.ngroups * dims->batch * l.ntiles_f < (1LL << 31));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+    cudaError_t e = cudaMemsetAsync(&hdr->fwd_ticket, 0, sizeof(int), s);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(ws + l.off_fflags, 0,
+                            sizeof(int) * (size_t)l.ngroups * dims->batch * l.ntiles_f, s);
+    if (e != cudaSuccess) return NAJU_ERR_CUDA;
+    FwdParams p{};
+    p.hu = hu; p.conv_w = conv_w; p.conv_b = conv_b; p.a = a; p.b = b; p.B = B; p.C = C;
+    p.z = z; p.D = D; p.x0 = x0; p.y = y; p.x_final = x_final;
+    p.ckpt = reinterpret_cast<float*>(ws + l.off_ckpt);
+    p.flags = reinterpret_cast<int*>(ws + l.off_fflags);
+    p.hdr = hdr;
+    p.Bt = dims->batch; p.L = dims->seqlen; p.d = dims->d_inner; p.N = dims->d_state;
+    p.T_ck = kTck; p.nck = l.nck; p.seg_per_group = l.seg_per_group; p.ngroups = l.ngroups;
+    p.ntiles = l.ntiles_f;
+    p.scale = 1.0f / std::sqrt((float)dims->d_state);
+    p.wait_limit = g_wait_limit;
+    p.fault_skip_publish = g_skip_publish;
+    return cuda_status(launch_scan_fwd(p, dims->dtype, dims->out_dtype, s));
+}
+
+naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* conv_w,
+                          const float* conv_b, const void* a, const void* b, const void* B,
+                          const void* C, const void* z, const float* D, const float* x0,
+                          const void* dy, const float* dx_final, void* dhu, void* da, void* db,
+                          void* dB, void* dC, void* dz, float* dD, float* dconv_w,
+                          float* dconv_b, float* dx0, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    (void)x0;  // the forward's checkpoint 0 holds the initial state
+    naju_status st = check_dims(dims);
+    if (st != NAJU_OK) return st;
+    if (conv_w && dims->conv_width != 4) return NAJU_ERR_UNSUPPORTED;
+    NAJU_REQUIRE(ok_act(hu) && ok_act(a) && ok_act(b) && ok_act(B) && ok_act(C) && ok_act(dy));
+    NAJU_REQUIRE(ok_act(dhu) && ok_act(da) && ok_act(db) && ok_act(dB) && ok_act(dC));
+    NAJU_REQUIRE(ok_opt(z) && ok_opt(dx_final) && ok_opt(dx0));
+    NAJU_REQUIRE(!z || ok_act(dz));
+    NAJU_REQUIRE(!conv_w || dconv_w);
+    NAJU_REQUIRE(workspace && aligned(workspace, 256));
+    const Layout l = layout(dims);
+    NAJU_REQUIRE(workspace_bytes >= l.total);
+    NAJU_REQUIRE((int64_t)l.nsub * dims->batch * l.ntiles_b < (1LL << 31));
+    NAJU_REQUIRE(l.nsub <= 65535 && dims->batch <= 65535);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+    cudaError_t e = cudaMemsetAsync(&hdr->bwd_ticket, 0, sizeof(int), s);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(ws + l.off_bflags, 0,
+                            sizeof(int) * (size_t)l.nsub * dims->batch * l.ntiles_b, s);
+    if (e != cudaSuccess) return NAJU_ERR_CUDA;
+    BwdParams p{};
+    p.hu = hu; p.conv_w = conv_w; p.conv_b = conv_b; p.a = a; p.b = b; p.B = B; p.C = C;
+    p.z = z; p.D = D; p.dy = dy; p.dx_final = dx_final;
+    p.dhu = dhu; p.da = da; p.db = db; p.dz = dz; p.dx0 = dx0;
+    p.ckpt = reinterpret_cast<const float*>(ws + l.off_ckpt);
+    p.carry = reinterpret_cast<float*>(ws + l.off_carry);
+    p.flags = reinterpret_cast<int*>(ws + l.off_bflags);
+    p.dBCp = reinterpret_cast<float*>(ws + l.off_dbc);
+    p.chan_part = reinterpret_cast<float*>(ws + l.off_chan);
+    p.conv_edge = reinterpret_cast<float*>(ws + l.off_edge);
+    p.hdr = hdr;
+    p.Bt = dims->batch; p.L = dims->seqlen; p.d = dims->d_inner; p.N = dims->d_state;
+    p.T_ck = kTck; p.nck = l.nck; p.nsub = l.nsub; p.ntiles = l.ntiles_b; p.nclus = l.nclus;
+    p.scale = 1.0f / std::sqrt((float)dims->d_state);
+    p.wait_limit = g_wait_limit;
+    p.fault_skip_publish = g_skip_publish;
+    return cuda_status(launch_scan_bwd(p, dims->dtype, dims->out_dtype, dB, dC, dD, dconv_w,
+                                       dconv_b, s));
+}
+
+naju_status naju_scan_step(int64_t batch, int64_t d_inner, int64_t d_state, int32_t dtype,
+                           const void* h, const void* a, const void* b, const void* B,
+                           const void* C, const void* z, const float* D, float* state, void* y,
+                           void* stream) {
+    if (batch < 1 || d_inner < 1 || batch > 65535) return NAJU_ERR_INVALID_ARG;
+    if (d_state != 16 && d_state != 32 && d_state != 64 && d_state != 128)
+        return NAJU_ERR_UNSUPPORTED;
+    if (dtype != NAJU_F32 && dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
+    NAJU_REQUIRE(ok_act(h) && ok_act(a) && ok_act(b) && ok_act(B) && ok_act(C) && ok_act(y));
+    NAJU_REQUIRE(ok_opt(z) && ok_act(state));
+    return cuda_status(launch_scan_step(batch, d_inner, d_state, h, a, b, B, C, z, D, state, y,
+                                        dtype, static_cast<cudaStream_t>(stream)));
+}
+
+naju_status naju_last_device_status(void* workspace, void* stream) {
+    if (!workspace || !aligned(workspace, 256)) return NAJU_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NAJU_ERR_CUDA;
+    int v = 0;
+    WsHeader* hdr = static_cast<WsHeader*>(workspace);
+    if (cudaMemcpy(&v, &hdr->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return NAJU_ERR_CUDA;
+    if (cudaMemset(&hdr->status, 0, sizeof(int)) != cudaSuccess) return NAJU_ERR_CUDA;
+    if (v & (1 << NAJU_ERR_TIMEOUT)) return NAJU_ERR_TIMEOUT;
+    return NAJU_OK;
+}
+
+const char* naju_status_string(naju_status s) {
+    switch (s) {
+        case NAJU_OK: return "ok";
+        case NAJU_ERR_INVALID_ARG: return "invalid argument";
+        case NAJU_ERR_UNSUPPORTED: return "unsupported configuration";
+        case NAJU_ERR_CUDA: return "CUDA error";
+        case NAJU_ERR_TIMEOUT: return "inter-block wait timed out";
+    }
+    return "unknown status";
+}
+
+void naju_testing_set_wait_limit(int64_t polls) {
+    g_wait_limit = polls > 0 ? (long long)polls : kDefaultWait;
+}
+void naju_testing_set_skip_publish(int32_t skip) { g_skip_publish = skip ? 1 : 0; }
+void naju_testing_set_fwd_groups(int32_t groups) { g_fwd_groups = groups > 0 ? groups : 0; }
+int32_t naju_testing_fwd_groups(const void* dims) {
+    const naju_dims* dm = static_cast<const naju_dims*>(dims);
+    if (check_dims(dm) != NAJU_OK) return 0;
+    return layout(dm).ngroups;
+}
+
+}  // extern "C"

@@ -1,0 +1,93 @@
+// Internal launch interface between the C ABI layer and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace naju {
+
+struct WsHeader;
+
+constexpr int kFwdChunk = 32;   // tokens staged per forward chunk
+constexpr int kBwdSub = 64;     // tokens per backward work item
+constexpr int kBwdChunk = 16;   // tokens per backward contraction block
+
+struct FwdParams {
+    const void* hu;
+    const float* conv_w;
+    const float* conv_b;
+    const void* a;
+    const void* b;
+    const void* B;
+    const void* C;
+    const void* z;
+    const float* D;
+    const float* x0;
+    void* y;
+    float* x_final;
+    float* ckpt;        // [Bt][nck+1][d][N] fp32 state at segment starts (+ final)
+    int* flags;         // [ngroups][Bt][ntiles]
+    WsHeader* hdr;
+    int64_t Bt, L, d, N;
+    int T_ck;           // tokens per checkpoint segment
+    int nck;            // number of segments = ceil(L / T_ck)
+    int seg_per_group;  // segments per sequence group
+    int ngroups;
+    int ntiles;         // channel tiles = ceil(d / P)
+    float scale;        // 1 / sqrt(N)
+    long long wait_limit;
+    int fault_skip_publish;
+};
+
+struct BwdParams {
+    const void* hu;
+    const float* conv_w;
+    const float* conv_b;
+    const void* a;
+    const void* b;
+    const void* B;
+    const void* C;
+    const void* z;
+    const float* D;
+    const void* dy;
+    const float* dx_final;
+    void* dhu;
+    void* da;
+    void* db;
+    void* dz;
+    float* dx0;
+    const float* ckpt;     // written by the forward
+    float* carry;          // [nsub][Bt][d][N] adjoint carries between items
+    int* flags;            // [nsub][Bt][ntiles]
+    float* dBCp;           // [nclus][Bt][L][2][N] partial dB, dC over channel clusters
+    float* chan_part;      // [Bt*nsub][d][8] partial dD, dconv_w[4], dconv_b
+    float* conv_edge;      // [Bt][nsub][2][3][d]: first 3 dp / last 3 partial du
+    WsHeader* hdr;
+    int64_t Bt, L, d, N;
+    int T_ck, nck;
+    int nsub;              // ceil(L / kBwdSub)
+    int ntiles;
+    int nclus;             // ceil(ntiles / cluster size)
+    float scale;
+    long long wait_limit;
+    int fault_skip_publish;
+};
+
+int fwd_channels_per_block(int64_t N);
+int bwd_channels_per_block(int64_t N);
+int bwd_cluster_size();
+
+cudaError_t launch_scan_fwd(const FwdParams& p, int dtype, int out_dtype, cudaStream_t st);
+cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, int out_dtype, void* dB, void* dC,
+                            float* dD, float* dconv_w, float* dconv_b, cudaStream_t st);
+cudaError_t launch_conv_fwd(int64_t Bt, int64_t L, int64_t d, const void* u, const float* w,
+                            const float* bias, void* h, int dtype, int out_dtype,
+                            cudaStream_t st);
+cudaError_t launch_conv_bwd(int64_t Bt, int64_t L, int64_t d, const void* u, const float* w,
+                            const float* bias, const void* dh, void* du, float* dw,
+                            float* dbias, int dtype, int out_dtype, cudaStream_t st);
+cudaError_t launch_scan_step(int64_t Bt, int64_t d, int64_t N, const void* h, const void* a,
+                             const void* b, const void* B, const void* C, const void* z,
+                             const float* D, float* state, void* y, int dtype,
+                             cudaStream_t st);
+
+}  // namespace naju

@@ -1,0 +1,742 @@
+// Naju backward scan on CUDA cores (sm_100a).
+//
+// Reverse-mode gradient of the forward in naju_scan_fwd.cu, derived by hand
+// from the recurrence of the Naju reproduction README ("Core equations").
+// For one (batch, channel) row, with G_t = dLoss/dx_t and s = 1/sqrt(N):
+//   dy_t   = dout_t SiLU(z_t),   dz_t = dout_t y_t SiLU'(z_t)
+//   G_t    = s dy_t C_t + f_{t+1} G_{t+1}          (the last G also gets dx_final)
+//   GB_t   = G_t . B_t
+//   dh_t   = D dy_t + i_t GB_t,  db_t = h_t GB_t i_t (1 - i_t)
+//   da_t   = (f_t df_t)(1 - f_t) with
+//   f_t df_t = G_t . (f_t x_{t-1}) = sum_{t' >= t} dL_{t'} + dx_final . x_L,
+//   dL_t   = s dy_t (x_t . C_t) - i_t h_t GB_t
+//   dB_t   = sum_d G_t[d] i_t[d] h_t[d],   dC_t = s sum_d dy_t[d] x_t[d]
+//   dD     = sum dy h,   dx0 = f_0 G_0,    conv: dp = dh SiLU'(p), du, dw, dbias.
+//
+// Work decomposition.  One work item = (batch b, tile of P channels, block k
+// of 64 tokens).  Items are taken from an atomic ticket from the end of the
+// sequence backwards.  An item:
+//  0. recomputes its start state from the forward's nearest checkpoint;
+//  1. (0 < k < last) runs a local reverse pass with a zero carry to get the
+//     block's own adjoint contribution and decay product;
+//  2. waits (bounded) for item k+1 to publish the adjoint carry entering its
+//     end, publishes the carry leaving its start (decoupled look-back);
+//  3. sweeps forward over 16-token sub-blocks: the state readout (kept for
+//     dz and dL) and, per sub-block, dC as a contraction over the block's
+//     channels: dC_t = s[(dy E)_t X_b + sum_{m<=t} A[t,m] B_m], where X_b is
+//     the state entering the sub-block, E_t the decay since then and
+//     A[t,m] = sum_d dy_t E_t/E_m i_m h_m;
+//  4. sweeps backward: the adjoint G, per-channel gradients, and per
+//     sub-block dB_m = s sum_{t>=m} A[t,m] C_t + (i h F)_m H_e, with H_e the
+//     carry entering the sub-block's end and F_m the decay to that end.
+// dB/dC partial sums over the P channels are summed across the thread-block
+// cluster (consecutive channel tiles) through distributed shared memory and
+// written once per cluster; small kernels then sum clusters, the per-channel
+// partials (dD, dconv) and the conv's block-boundary terms.
+#include <cooperative_groups.h>
+
+#include "naju_common.cuh"
+#include "naju_kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace naju {
+
+constexpr float kRenormB = 18446744073709551616.0f;  // 2^64
+constexpr float kLogFloor = -10.0f;  // per-token log f floor inside the pivot factors of A
+constexpr int kCluster = 8;
+
+template <int N> struct BwdShape;
+template <> struct BwdShape<16> { static constexpr int NS = 16, S = 1; };
+template <> struct BwdShape<32> { static constexpr int NS = 32, S = 1; };
+template <> struct BwdShape<64> { static constexpr int NS = 32, S = 2; };
+template <> struct BwdShape<128> { static constexpr int NS = 32, S = 4; };
+
+int bwd_channels_per_block(int64_t N) { return N <= 32 ? 128 : (N == 64 ? 64 : 32); }
+int bwd_cluster_size() { return kCluster; }
+
+template <int N, int P>
+struct BwdSmem {
+    static constexpr int T = kBwdChunk;   // 16
+    static constexpr int K = kBwdSub;     // 64
+    float f[T][P], q[T][P], v[T][P], dy[T][P];
+    float lg[T][P], E[T][P];              // clamped log-prefix / true decay prefix
+    float fa[T][P], fb[T][P];             // A factors (dy side / i h side)
+    float gb[T][P], fdf[T][P], dp[T + 3][P];
+    float ys[K][P];                       // unscaled readout x_t . C_t
+    float Bm[T][N], Cm[T][N];
+    float snap[P][N];                     // X_b (forward) or H_e (backward)
+    float A[K / T][T][T];                 // per sub-block contraction matrix
+    float acc[K][2][N];                   // dB (0) and dC (1) partials of the item
+    int item;
+};
+
+template <typename Tin, typename Tout, int N, bool CONV>
+__global__ void __launch_bounds__(128, 1)
+scan_bwd_kernel(const BwdParams p) {
+    constexpr int NS = BwdShape<N>::NS, S = BwdShape<N>::S;
+    constexpr int NT = 128, P = NT / S;
+    constexpr int T = kBwdChunk, K = kBwdSub, NSUB = K / T;
+    constexpr int R = T / S;              // prep run length per thread
+    using Sm = BwdSmem<N, P>;
+    extern __shared__ float4 smem4[];
+    Sm& sm = *reinterpret_cast<Sm*>(smem4);
+    cg::cluster_group cluster = cg::this_cluster();
+    const int crank = (int)cluster.block_rank();
+
+    const int tid = threadIdx.x;
+    const int js = tid % S, pl = tid / S;
+    const int pp = tid % P, rr = tid / P;
+    const int64_t Bt = p.Bt, L = p.L, d = p.d;
+    const float s = p.scale;
+
+    // ---------------------------------------------------- work item
+    if (crank == 0 && tid == 0) sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
+    cluster.sync();
+    const int item = *cluster.map_shared_rank(&sm.item, 0);
+    const int per_k = (int)(Bt * p.nclus);
+    const int k = p.nsub - 1 - item / per_k;
+    const int bb = (item % per_k) / p.nclus;
+    const int cgi = item % p.nclus;
+    const int tile = cgi * kCluster + crank;
+    const int64_t c0 = (int64_t)tile * P;
+    const int64_t c = c0 + pl;
+    const bool cvalid = c < d;
+    const int64_t cp = c0 + pp;
+    const bool cpvalid = cp < d;
+    const int64_t tb = (int64_t)k * K;
+    const int64_t te = min64(L, tb + K);
+    const bool last = (k == p.nsub - 1);
+
+    const Tin* hu = static_cast<const Tin*>(p.hu);
+    const Tin* ga = static_cast<const Tin*>(p.a);
+    const Tin* gbp = static_cast<const Tin*>(p.b);
+    const Tin* gB = static_cast<const Tin*>(p.B);
+    const Tin* gC = static_cast<const Tin*>(p.C);
+    const Tin* gz = static_cast<const Tin*>(p.z);
+    const Tin* gdy = static_cast<const Tin*>(p.dy);
+
+    float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, wb = 0.f, Dc = 0.f;
+    if (cpvalid) {
+        if (CONV) {
+            w0 = p.conv_w[cp * 4]; w1 = p.conv_w[cp * 4 + 1];
+            w2 = p.conv_w[cp * 4 + 2]; w3 = p.conv_w[cp * 4 + 3];
+            wb = p.conv_b ? p.conv_b[cp] : 0.f;
+        }
+        Dc = p.D ? p.D[cp] : 0.f;
+    }
+
+    // Stage one sub-block [t0, t0+T) of per-(token, channel) scalars and B, C.
+    auto stage = [&](int64_t t0, int64_t tlim) {
+        for (int e = tid; e < T * N; e += NT) {
+            const int tt = e / N;
+            const int64_t t = t0 + tt;
+            float vb = 0.f, vc = 0.f;
+            if (t < tlim) {
+                vb = to_f(gB[((int64_t)bb * L + t) * N + (e % N)]);
+                vc = to_f(gC[((int64_t)bb * L + t) * N + (e % N)]);
+            }
+            sm.Bm[tt][e % N] = vb;
+            sm.Cm[tt][e % N] = vc;
+        }
+        const int64_t tr = t0 + rr * R;
+        float u0 = 0.f, u1 = 0.f, u2 = 0.f;
+        if (CONV && cpvalid) {
+            const Tin* col = hu + (int64_t)bb * L * d + cp;
+            if (tr >= 3 && tr - 3 < L) u0 = to_f(col[(tr - 3) * d]);
+            if (tr >= 2 && tr - 2 < L) u1 = to_f(col[(tr - 2) * d]);
+            if (tr >= 1 && tr - 1 < L) u2 = to_f(col[(tr - 1) * d]);
+        }
+        for (int kk = 0; kk < R; ++kk) {
+            const int tt = rr * R + kk;
+            const int64_t t = tr + kk;
+            float f = 1.f, q = 1.f, v = 0.f, dyv = 0.f;
+            if (cpvalid && t < tlim) {
+                const int64_t e = ((int64_t)bb * L + t) * d + cp;
+                float h;
+                if (CONV) {
+                    const float u3 = to_f(hu[e]);
+                    h = siluf_(wb + w0 * u0 + w1 * u1 + w2 * u2 + w3 * u3);
+                    u0 = u1; u1 = u2; u2 = u3;
+                } else {
+                    h = to_f(hu[e]);
+                }
+                q = 1.f + __expf(-to_f(ga[e]));
+                f = 1.f / q;
+                v = sigmoidf_(to_f(gbp[e])) * h;
+                dyv = to_f(gdy[e]);
+                if (gz) dyv *= siluf_(to_f(gz[e]));
+            }
+            sm.f[tt][pp] = f; sm.q[tt][pp] = q; sm.v[tt][pp] = v; sm.dy[tt][pp] = dyv;
+        }
+    };
+
+    // ----------------------------------------------------- register state
+    float xs[NS], gs[NS];
+    float Q = 1.f, iQ = 1.f;   // forward: x = xs * iQ
+    float Rr = 1.f, iR = 1.f;  // backward: G = gs * iR
+    float logF = 0.f;          // log of decay folded out of the backward state
+
+    auto load_rows = [&](float* dst, const float* src, bool cg_) {
+#pragma unroll
+        for (int m = 0; m < NS / 4; ++m) {
+            float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (src && cvalid) {
+                const float4* s4 = reinterpret_cast<const float4*>(src + c * N) + m * S + js;
+                v4 = cg_ ? __ldcg(s4) : *s4;
+            }
+            dst[4 * m] = v4.x; dst[4 * m + 1] = v4.y; dst[4 * m + 2] = v4.z; dst[4 * m + 3] = v4.w;
+        }
+    };
+    auto red = [&](float v) {
+#pragma unroll
+        for (int o = 1; o < S; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        return v;
+    };
+    // Forward token: xs <- xs + (v Q) B (rescaled), optional readout.
+    auto fstep = [&](int tt, bool read) -> float {
+        const float qv = sm.q[tt][pl], fv = sm.f[tt][pl], vv = sm.v[tt][pl];
+        float Qn = Q * qv, iQn = iQ * fv;
+        if (__any_sync(0xffffffffu, !(Qn <= kRenormB))) {
+#pragma unroll
+            for (int j = 0; j < NS; ++j) xs[j] *= iQn;
+            Qn = 1.f; iQn = 1.f;
+        }
+        Q = Qn; iQ = iQn;
+        const float wv = vv * Q;
+        const float4* b4 = reinterpret_cast<const float4*>(sm.Bm[tt]);
+        const float4* c4 = reinterpret_cast<const float4*>(sm.Cm[tt]);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int m = 0; m < NS / 4; ++m) {
+            const float4 bv = b4[m * S + js];
+            xs[4 * m] = fmaf(wv, bv.x, xs[4 * m]);
+            xs[4 * m + 1] = fmaf(wv, bv.y, xs[4 * m + 1]);
+            xs[4 * m + 2] = fmaf(wv, bv.z, xs[4 * m + 2]);
+            xs[4 * m + 3] = fmaf(wv, bv.w, xs[4 * m + 3]);
+            if (read) {
+                const float4 cv = c4[m * S + js];
+                a0 = fmaf(xs[4 * m], cv.x, a0);
+                a1 = fmaf(xs[4 * m + 1], cv.y, a1);
+                a2 = fmaf(xs[4 * m + 2], cv.z, a2);
+                a3 = fmaf(xs[4 * m + 3], cv.w, a3);
+            }
+        }
+        return ((a0 + a1) + (a2 + a3)) * iQ;
+    };
+    // Backward token t (after the carry from t+1 is in gs): G_t = G + s dy C.
+    // The decay f_{t+1} was folded in by bdecay() of the later token.
+    auto bstep = [&](int tt, bool dotB) -> float {
+        const float wv = s * sm.dy[tt][pl] * Rr;
+        const float4* b4 = reinterpret_cast<const float4*>(sm.Bm[tt]);
+        const float4* c4 = reinterpret_cast<const float4*>(sm.Cm[tt]);
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int m = 0; m < NS / 4; ++m) {
+            const float4 cv = c4[m * S + js];
+            gs[4 * m] = fmaf(wv, cv.x, gs[4 * m]);
+            gs[4 * m + 1] = fmaf(wv, cv.y, gs[4 * m + 1]);
+            gs[4 * m + 2] = fmaf(wv, cv.z, gs[4 * m + 2]);
+            gs[4 * m + 3] = fmaf(wv, cv.w, gs[4 * m + 3]);
+            if (dotB) {
+                const float4 bv = b4[m * S + js];
+                a0 = fmaf(gs[4 * m], bv.x, a0);
+                a1 = fmaf(gs[4 * m + 1], bv.y, a1);
+                a2 = fmaf(gs[4 * m + 2], bv.z, a2);
+                a3 = fmaf(gs[4 * m + 3], bv.w, a3);
+            }
+        }
+        return ((a0 + a1) + (a2 + a3)) * iR;
+    };
+    // Multiply the backward state by f_t (moving from t to t-1).
+    auto bdecay = [&](int tt) {
+        const float qv = sm.q[tt][pl], fv = sm.f[tt][pl];
+        float Rn = Rr * qv, iRn = iR * fv;
+        if (__any_sync(0xffffffffu, !(Rn <= kRenormB))) {
+            logF += __logf(iRn);
+#pragma unroll
+            for (int j = 0; j < NS; ++j) gs[j] *= iRn;
+            Rn = 1.f; iRn = 1.f;
+        }
+        Rr = Rn; iR = iRn;
+    };
+
+    // --------------------------------------- 0. state entering the block
+    {
+        const int kc = (int)(tb / p.T_ck);
+        const float* ck = p.ckpt + ((int64_t)bb * (p.nck + 1) + kc) * d * N;
+        load_rows(xs, ck, false);
+        Q = 1.f; iQ = 1.f;
+        for (int64_t t0 = (int64_t)kc * p.T_ck; t0 < tb; t0 += T) {
+            stage(t0, tb);
+            __syncthreads();
+            for (int tt = 0; tt < T; ++tt) fstep(tt, false);
+            __syncthreads();
+        }
+#pragma unroll
+        for (int j = 0; j < NS; ++j) xs[j] *= iQ;
+        Q = 1.f; iQ = 1.f;
+    }
+
+    // ------------------------------------- 1. local adjoint contribution
+    const bool local = (k > 0) && !last;
+    if (local) {
+#pragma unroll
+        for (int j = 0; j < NS; ++j) gs[j] = 0.f;
+        Rr = 1.f; iR = 1.f; logF = 0.f;
+        for (int sb = NSUB - 1; sb >= 0; --sb) {
+            const int64_t t0 = tb + sb * T;
+            stage(t0, te);
+            __syncthreads();
+            for (int tt = T - 1; tt >= 0; --tt) {
+                bstep(tt, false);
+                bdecay(tt);
+            }
+            __syncthreads();
+        }
+    }
+
+    // -------------------------------------------- 2. carry in / publish
+    float* carry_in = p.carry + ((int64_t)k * Bt + bb) * d * N;
+    float* carry_out = k > 0 ? p.carry + ((int64_t)(k - 1) * Bt + bb) * d * N : nullptr;
+    int* flag_in = p.flags + ((int64_t)k * Bt + bb) * p.ntiles + tile;
+    int* flag_out = k > 0 ? p.flags + ((int64_t)(k - 1) * Bt + bb) * p.ntiles + tile : nullptr;
+    float H[NS];
+    {
+        __shared__ int s_ok;
+        if (!last) {
+            if (tid == 0) s_ok = wait_flag(flag_in, &p.hdr->status, p.wait_limit) ? 1 : 0;
+            __syncthreads();
+            load_rows(H, s_ok ? carry_in : nullptr, true);
+        } else {
+            load_rows(H, p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr, false);
+        }
+        if (local) {
+            // carry out = decay(block) * H + local contribution.
+            const float Pf = __expf(logF + __logf(iR));
+            if (cvalid) {
+#pragma unroll
+                for (int m = 0; m < NS / 4; ++m) {
+                    float4 o4 = make_float4(fmaf(Pf, H[4 * m], gs[4 * m] * iR),
+                                            fmaf(Pf, H[4 * m + 1], gs[4 * m + 1] * iR),
+                                            fmaf(Pf, H[4 * m + 2], gs[4 * m + 2] * iR),
+                                            fmaf(Pf, H[4 * m + 3], gs[4 * m + 3] * iR));
+                    reinterpret_cast<float4*>(carry_out + c * N)[m * S + js] = o4;
+                }
+            }
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) st_release(flag_out, 1);
+        }
+    }
+
+    // ---------------------------------------------- 3. forward sweep
+    for (int sb = 0; sb < NSUB; ++sb) {
+        const int64_t t0 = tb + sb * T;
+        stage(t0, te);
+        // Snapshot of the state entering the sub-block (xs is unscaled here).
+        if (cvalid) {
+#pragma unroll
+            for (int m = 0; m < NS / 4; ++m)
+                reinterpret_cast<float4*>(sm.snap[pl])[m * S + js] =
+                    make_float4(xs[4 * m], xs[4 * m + 1], xs[4 * m + 2], xs[4 * m + 3]);
+        } else if (js == 0) {
+            for (int j = 0; j < N; ++j) sm.snap[pl][j] = 0.f;
+        }
+        __syncthreads();
+        float lg = 0.f, E = 1.f;
+        for (int tt = 0; tt < T; ++tt) {
+            const float yv = red(fstep(tt, true));
+            const float fv = sm.f[tt][pl];
+            lg += fmaxf(__logf(fv), kLogFloor);
+            E *= fv;
+            if (js == 0) {
+                sm.ys[sb * T + tt][pl] = yv;
+                sm.lg[tt][pl] = lg;
+                sm.E[tt][pl] = E;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < NS; ++j) xs[j] *= iQ;
+        Q = 1.f; iQ = 1.f;
+        __syncthreads();
+        // Pivot factors of A around token T/2 of the sub-block.
+        for (int kk = 0; kk < R; ++kk) {
+            const int tt = rr * R + kk;
+            const float piv = sm.lg[T / 2][pp];
+            const float l = sm.lg[tt][pp];
+            sm.fa[tt][pp] = sm.dy[tt][pp] * __expf(l - piv);
+            sm.fb[tt][pp] = sm.v[tt][pp] * __expf(piv - l);
+            sm.E[tt][pp] *= sm.dy[tt][pp];  // dy_t E_t
+        }
+        __syncthreads();
+        // A[t][m] = sum_p fa[t][p] fb[m][p] for m <= t.
+        for (int e = tid; e < T * T; e += NT) {
+            const int tt = e / T, mm = e % T;
+            float acc = 0.f;
+            if (mm <= tt) {
+                for (int q2 = 0; q2 < P; ++q2) acc = fmaf(sm.fa[tt][q2], sm.fb[mm][q2], acc);
+            }
+            sm.A[sb][tt][mm] = acc;
+        }
+        __syncthreads();
+        // dC[t][j] = s [ sum_p (dy E)[t][p] X_b[p][j] + sum_{m<=t} A[t][m] B[m][j] ].
+        {
+            constexpr int JB = (N * T) / NT;  // outputs per thread
+            const int tt = tid / (N / JB);
+            const int j0 = (tid % (N / JB)) * JB;
+            float o[JB];
+#pragma unroll
+            for (int r = 0; r < JB; ++r) o[r] = 0.f;
+            for (int q2 = 0; q2 < P; ++q2) {
+                const float a = sm.E[tt][q2];
+#pragma unroll
+                for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.snap[q2][j0 + r], o[r]);
+            }
+            for (int mm = 0; mm <= tt; ++mm) {
+                const float a = sm.A[sb][tt][mm];
+#pragma unroll
+                for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.Bm[mm][j0 + r], o[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < JB; ++r) sm.acc[sb * T + tt][1][j0 + r] = s * o[r];
+        }
+        __syncthreads();
+    }
+
+    // tail of f df: H . x_end (per channel)
+    float tail = 0.f;
+#pragma unroll
+    for (int j = 0; j < NS; ++j) tail = fmaf(H[j], xs[j], tail);
+    tail = red(tail);
+
+    // ---------------------------------------------- 4. backward sweep
+#pragma unroll
+    for (int j = 0; j < NS; ++j) gs[j] = H[j];
+    Rr = 1.f; iR = 1.f; logF = 0.f;
+    float cum = 0.f;  // sum of dL over later tokens of the block
+    float dD_acc = 0.f, dw0 = 0.f, dw1 = 0.f, dw2 = 0.f, dw3 = 0.f, dbias = 0.f;
+    Tout* gdhu = static_cast<Tout*>(p.dhu);
+    Tout* gda = static_cast<Tout*>(p.da);
+    Tout* gdb = static_cast<Tout*>(p.db);
+    Tout* gdz = static_cast<Tout*>(p.dz);
+    float* edge = p.conv_edge + ((int64_t)bb * p.nsub + k) * 2 * 3 * d;
+    if (tid < P) {  // dp beyond the block: zero (next block's terms go via the edge fixup)
+        sm.dp[T][tid] = 0.f; sm.dp[T + 1][tid] = 0.f; sm.dp[T + 2][tid] = 0.f;
+    }
+    for (int sb = NSUB - 1; sb >= 0; --sb) {
+        const int64_t t0 = tb + sb * T;
+        stage(t0, te);
+        // H_e: carry entering the sub-block's end, true scale.
+        if (cvalid) {
+#pragma unroll
+            for (int m = 0; m < NS / 4; ++m)
+                reinterpret_cast<float4*>(sm.snap[pl])[m * S + js] =
+                    make_float4(gs[4 * m] * iR, gs[4 * m + 1] * iR, gs[4 * m + 2] * iR,
+                                gs[4 * m + 3] * iR);
+        } else if (js == 0) {
+            for (int j = 0; j < N; ++j) sm.snap[pl][j] = 0.f;
+        }
+        __syncthreads();
+        float F = 1.f;  // prod f_{m+1..end of sub-block}
+        for (int tt = T - 1; tt >= 0; --tt) {
+            const float gbv = red(bstep(tt, true));
+            const float vv = sm.v[tt][pl];
+            const float dL = s * sm.dy[tt][pl] * sm.ys[sb * T + tt][pl] - vv * gbv;
+            cum += dL;
+            if (js == 0) {
+                sm.gb[tt][pl] = gbv;
+                sm.fdf[tt][pl] = cum + tail;
+                sm.E[tt][pl] = vv * F;  // (i h F)_m
+            }
+            F *= sm.f[tt][pl];
+            bdecay(tt);
+        }
+        __syncthreads();
+        // dB[m][j] = sum_p (i h F)[m][p] H_e[p][j] + s sum_{t>=m} A[t][m] C[t][j].
+        {
+            constexpr int JB = (N * T) / NT;
+            const int mm = tid / (N / JB);
+            const int j0 = (tid % (N / JB)) * JB;
+            float o[JB], o2[JB];
+#pragma unroll
+            for (int r = 0; r < JB; ++r) { o[r] = 0.f; o2[r] = 0.f; }
+            for (int q2 = 0; q2 < P; ++q2) {
+                const float a = sm.E[mm][q2];
+#pragma unroll
+                for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.snap[q2][j0 + r], o[r]);
+            }
+            for (int tt = mm; tt < T; ++tt) {
+                const float a = sm.A[sb][tt][mm];
+#pragma unroll
+                for (int r = 0; r < JB; ++r) o2[r] = fmaf(a, sm.Cm[tt][j0 + r], o2[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < JB; ++r) sm.acc[sb * T + mm][0][j0 + r] = fmaf(s, o2[r], o[r]);
+        }
+        // Per-channel gradients of the sub-block (thread pp, run rr).
+        {
+            const int64_t tr = t0 + rr * R;
+            float u0 = 0.f, u1 = 0.f, u2 = 0.f;
+            if (CONV && cpvalid) {
+                const Tin* col = hu + (int64_t)bb * L * d + cp;
+                if (tr >= 3 && tr - 3 < L) u0 = to_f(col[(tr - 3) * d]);
+                if (tr >= 2 && tr - 2 < L) u1 = to_f(col[(tr - 2) * d]);
+                if (tr >= 1 && tr - 1 < L) u2 = to_f(col[(tr - 1) * d]);
+            }
+            for (int kk = 0; kk < R; ++kk) {
+                const int tt = rr * R + kk;
+                const int64_t t = tr + kk;
+                float dpv = 0.f;
+                if (cpvalid && t < te) {
+                    const int64_t e = ((int64_t)bb * L + t) * d + cp;
+                    float h, pre = 0.f, u3 = 0.f;
+                    if (CONV) {
+                        u3 = to_f(hu[e]);
+                        pre = wb + w0 * u0 + w1 * u1 + w2 * u2 + w3 * u3;
+                        h = siluf_(pre);
+                    } else {
+                        h = to_f(hu[e]);
+                    }
+                    const float fv = sm.f[tt][pp];
+                    const float iv = sigmoidf_(to_f(gbp[e]));
+                    const float gbv = sm.gb[tt][pp];
+                    const float dyv = sm.dy[tt][pp];
+                    const float dh = Dc * dyv + iv * gbv;
+                    gda[e] = from_f<Tout>(sm.fdf[tt][pp] * (1.f - fv));
+                    gdb[e] = from_f<Tout>(h * gbv * iv * (1.f - iv));
+                    if (gz) {
+                        const float zv = to_f(gz[e]);
+                        const float yv = fmaf(s, sm.ys[sb * T + tt][pp], Dc * h);
+                        gdz[e] = from_f<Tout>(to_f(gdy[e]) * yv * dsiluf_(zv));
+                    }
+                    dD_acc = fmaf(dyv, h, dD_acc);
+                    if (CONV) {
+                        dpv = dh * dsiluf_(pre);
+                        dw0 = fmaf(dpv, u0, dw0); dw1 = fmaf(dpv, u1, dw1);
+                        dw2 = fmaf(dpv, u2, dw2); dw3 = fmaf(dpv, u3, dw3);
+                        dbias += dpv;
+                        u0 = u1; u1 = u2; u2 = u3;
+                    } else {
+                        gdhu[e] = from_f<Tout>(dh);
+                    }
+                }
+                if (CONV) sm.dp[tt][pp] = dpv;
+            }
+        }
+        __syncthreads();
+        if (CONV) {
+            // du_t = w3 dp_t + w2 dp_{t+1} + w1 dp_{t+2} + w0 dp_{t+3}
+            for (int kk = 0; kk < R; ++kk) {
+                const int tt = rr * R + kk;
+                const int64_t t = t0 + tt;
+                if (cpvalid && t < te) {
+                    const float duv = w3 * sm.dp[tt][pp] + w2 * sm.dp[tt + 1][pp] +
+                                      w1 * sm.dp[tt + 2][pp] + w0 * sm.dp[tt + 3][pp];
+                    const int64_t e = ((int64_t)bb * L + t) * d + cp;
+                    if (!last && t >= te - 3) {
+                        edge[(3 + (t - (te - 3))) * d + cp] = duv;  // partial, fixed up later
+                    } else {
+                        gdhu[e] = from_f<Tout>(duv);
+                    }
+                    if (sb == 0 && tt < 3) edge[tt * d + cp] = sm.dp[tt][pp];
+                }
+            }
+            __syncthreads();
+            if (tid < P) {  // carry the first three dp rows to the earlier sub-block
+                sm.dp[T][tid] = sm.dp[0][tid];
+                sm.dp[T + 1][tid] = sm.dp[1][tid];
+                sm.dp[T + 2][tid] = sm.dp[2][tid];
+            }
+        }
+        __syncthreads();
+    }
+
+    // ------------------------------------------------ carries and partials
+    if (last && k > 0) {  // publish the carry leaving the block after the full sweep
+        if (cvalid) {
+#pragma unroll
+            for (int m = 0; m < NS / 4; ++m)
+                reinterpret_cast<float4*>(carry_out + c * N)[m * S + js] =
+                    make_float4(gs[4 * m] * iR, gs[4 * m + 1] * iR, gs[4 * m + 2] * iR,
+                                gs[4 * m + 3] * iR);
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && !p.fault_skip_publish) st_release(flag_out, 1);
+    }
+    if (k == 0 && p.dx0 && cvalid) {
+#pragma unroll
+        for (int m = 0; m < NS / 4; ++m)
+            reinterpret_cast<float4*>(p.dx0 + ((int64_t)bb * d + c) * N)[m * S + js] =
+                make_float4(gs[4 * m] * iR, gs[4 * m + 1] * iR, gs[4 * m + 2] * iR,
+                            gs[4 * m + 3] * iR);
+    }
+    // Per-channel partial sums (runs of the same channel add through shared atomics).
+    {
+        float* cpart = p.chan_part + ((int64_t)bb * p.nsub + k) * d * 8;
+        __syncthreads();
+        float* red6 = &sm.fdf[0][0];  // reuse: [6][P]
+        for (int i = tid; i < 6 * P; i += NT) red6[i] = 0.f;
+        __syncthreads();
+        if (cpvalid) {
+            atomicAdd(&red6[0 * P + pp], dD_acc);
+            atomicAdd(&red6[1 * P + pp], dw0);
+            atomicAdd(&red6[2 * P + pp], dw1);
+            atomicAdd(&red6[3 * P + pp], dw2);
+            atomicAdd(&red6[4 * P + pp], dw3);
+            atomicAdd(&red6[5 * P + pp], dbias);
+        }
+        __syncthreads();
+        if (tid < P && c0 + tid < d) {
+#pragma unroll
+            for (int r = 0; r < 6; ++r) cpart[(c0 + tid) * 8 + r] = red6[r * P + tid];
+        }
+    }
+    // Cluster reduction of the dB / dC partials of this block.
+    cluster.sync();
+    {
+        constexpr int ROWS = K / kCluster;
+        const int r0 = crank * ROWS;
+        float* out = p.dBCp + (((int64_t)cgi * Bt + bb) * L) * 2 * N;
+        for (int e = tid; e < ROWS * 2 * N; e += NT) {
+            const int tt = r0 + e / (2 * N);
+            const int rem = e % (2 * N);
+            float acc = 0.f;
+#pragma unroll
+            for (int qr = 0; qr < kCluster; ++qr) {
+                const float* rem_acc = cluster.map_shared_rank(&sm.acc[0][0][0], qr);
+                acc += rem_acc[tt * 2 * N + rem];
+            }
+            const int64_t t = tb + tt;
+            if (t < te) out[t * 2 * N + rem] = acc;
+        }
+    }
+    cluster.sync();
+}
+
+// Sum the cluster partials of dB, dC and write them in the output dtype.
+template <typename Tout>
+__global__ void reduce_dBC_kernel(const float* __restrict__ part, int nclus, int64_t BtL,
+                                  int64_t N, Tout* __restrict__ dB, Tout* __restrict__ dC) {
+    const int64_t n = BtL * N;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t row = i / N, j = i % N;
+        float sb = 0.f, sc = 0.f;
+        for (int q = 0; q < nclus; ++q) {
+            const float* pr = part + ((int64_t)q * BtL + row) * 2 * N;
+            sb += pr[j];
+            sc += pr[N + j];
+        }
+        dB[i] = from_f<Tout>(sb);
+        dC[i] = from_f<Tout>(sc);
+    }
+}
+
+// Sum per-(batch, block) channel partials: dD, dconv_w[4], dconv_b.
+__global__ void reduce_chan_kernel(const float* __restrict__ part, int64_t rows, int64_t d,
+                                   float* dD, float* dw, float* dbias) {
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= d) return;
+    float acc[6] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* pr = part + (r * d + c) * 8;
+#pragma unroll
+        for (int q = 0; q < 6; ++q) acc[q] += pr[q];
+    }
+    if (dD) dD[c] = acc[0];
+    if (dw) {
+        dw[c * 4] = acc[1]; dw[c * 4 + 1] = acc[2]; dw[c * 4 + 2] = acc[3]; dw[c * 4 + 3] = acc[4];
+    }
+    if (dbias) dbias[c] = acc[5];
+}
+
+// du of the last three tokens of each non-final block: the block's own
+// partial plus the terms from the first three dp of the next block.
+template <typename Tout>
+__global__ void conv_edge_kernel(const float* __restrict__ edge, const float* __restrict__ w,
+                                 int64_t Bt, int nsub, int64_t L, int64_t d,
+                                 Tout* __restrict__ du) {
+    const int64_t n = Bt * (int64_t)(nsub - 1) * 3 * d;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t c = i % d;
+        const int r = (int)((i / d) % 3);
+        const int64_t kb = (i / (3 * d)) % (nsub - 1);
+        const int64_t bb = i / (3 * d * (nsub - 1));
+        const int64_t t = (kb + 1) * kBwdSub - 3 + r;
+        const float* mine = edge + ((bb * nsub + kb) * 2 + 1) * 3 * d;
+        const float* next = edge + ((bb * nsub + kb + 1) * 2 + 0) * 3 * d;
+        float v = mine[r * d + c];
+        // du_t += sum_k w[k] dp_{t+3-k} over the next block's tokens.
+        for (int kk = 0; kk < 4; ++kk) {
+            const int64_t ts = t + 3 - kk - (kb + 1) * kBwdSub;
+            if (ts >= 0 && ts < 3) v += w[c * 4 + kk] * next[ts * d + c];
+        }
+        du[(bb * L + t) * d + c] = from_f<Tout>(v);
+    }
+}
+
+template <typename Tin, typename Tout, int N, bool CONV>
+static cudaError_t launch_bwd_t(const BwdParams& p, void* dB, void* dC, float* dD, float* dw,
+                                float* dbias, cudaStream_t st) {
+    constexpr int S = BwdShape<N>::S;
+    constexpr int P = 128 / S;
+    const size_t smem = sizeof(BwdSmem<N, P>);
+    auto kern = scan_bwd_kernel<Tin, Tout, N, CONV>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.nclus * kCluster), (unsigned)p.Bt, (unsigned)p.nsub);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, p);
+    if (e != cudaSuccess) return e;
+    const int64_t BtL = p.Bt * p.L;
+    reduce_dBC_kernel<Tout><<<592, 256, 0, st>>>(p.dBCp, p.nclus, BtL, N,
+                                                  static_cast<Tout*>(dB), static_cast<Tout*>(dC));
+    reduce_chan_kernel<<<(unsigned)((p.d + 127) / 128), 128, 0, st>>>(
+        p.chan_part, p.Bt * p.nsub, p.d, dD, CONV ? dw : nullptr, CONV ? dbias : nullptr);
+    if (CONV && p.nsub > 1)
+        conv_edge_kernel<Tout><<<296, 256, 0, st>>>(p.conv_edge, p.conv_w, p.Bt, p.nsub, p.L,
+                                                     p.d, static_cast<Tout*>(p.dhu));
+    return cudaGetLastError();
+}
+
+template <typename Tin, typename Tout, bool CONV>
+static cudaError_t launch_bwd_n(const BwdParams& p, void* dB, void* dC, float* dD, float* dw,
+                                float* dbias, cudaStream_t st) {
+    switch (p.N) {
+        case 16: return launch_bwd_t<Tin, Tout, 16, CONV>(p, dB, dC, dD, dw, dbias, st);
+        case 32: return launch_bwd_t<Tin, Tout, 32, CONV>(p, dB, dC, dD, dw, dbias, st);
+        case 64: return launch_bwd_t<Tin, Tout, 64, CONV>(p, dB, dC, dD, dw, dbias, st);
+        case 128: return launch_bwd_t<Tin, Tout, 128, CONV>(p, dB, dC, dD, dw, dbias, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, int out_dtype, void* dB, void* dC,
+                            float* dD, float* dw, float* dbias, cudaStream_t st) {
+    const bool conv = p.conv_w != nullptr;
+    if (dtype == NAJU_F32)
+        return conv ? launch_bwd_n<float, float, true>(p, dB, dC, dD, dw, dbias, st)
+                    : launch_bwd_n<float, float, false>(p, dB, dC, dD, dw, dbias, st);
+    if (out_dtype == NAJU_BF16)
+        return conv ? launch_bwd_n<__nv_bfloat16, __nv_bfloat16, true>(p, dB, dC, dD, dw, dbias, st)
+                    : launch_bwd_n<__nv_bfloat16, __nv_bfloat16, false>(p, dB, dC, dD, dw, dbias,
+                                                                         st);
+    return conv ? launch_bwd_n<__nv_bfloat16, float, true>(p, dB, dC, dD, dw, dbias, st)
+                : launch_bwd_n<__nv_bfloat16, float, false>(p, dB, dC, dD, dw, dbias, st);
+}
+
+}  // namespace naju

@@ -1,0 +1,142 @@
+/*
+ * naju.h -- C ABI of the B200 (sm_100a) Naju scan library.
+ *
+ * Naju (arXiv 2607.21000; Naju reproduction README, "Core equations" and the
+ * block flowchart) is a native-discrete selective state-space block.  This
+ * library implements its data-parallel hot path:
+ *
+ *   h_n   = SiLU(causal depthwise conv(u)_n)                    (optional)
+ *   x_n   = f_n (.) x_{n-1} + i_n (.) (h_n B_n^T),  f = sigmoid(a), i = sigmoid(b)
+ *   y_n   = x_n C_n / sqrt(d_state) + D (.) h_n
+ *   out_n = y_n * SiLU(z_n)                                       (optional)
+ *
+ * its gradients, and a single-token decode step on a carried state.
+ *
+ * Shapes (row-major, contiguous; Bt = batch, L = seqlen, d = d_inner,
+ * N = d_state, W = conv_width):
+ *   u or h, a, b, z, y (out), dy, du/dh, da, db, dz : [Bt, L, d]  activation dtype
+ *   B, C, dB, dC                                   : [Bt, L, N]  activation dtype
+ *   x0, x_final, dx_final, dx0, decode state       : [Bt, d, N]  fp32
+ *   D, dD, conv_b, dconv_b                         : [d]         fp32
+ *   conv_w, dconv_w                                : [d, W]      fp32
+ * Gates f, i are per (token, channel) and broadcast over the N state columns;
+ * B and C are one N-vector per (batch, token), shared by all channels.  The
+ * conv is a cross-correlation over the W most recent tokens with zero left
+ * padding: p_t = conv_b + sum_k conv_w[k] u_{t-(W-1)+k}.
+ *
+ * Ownership and ordering.  The caller allocates every device buffer (inputs,
+ * outputs and the workspace); the library never allocates, frees or
+ * synchronises (except naju_last_device_status), and every call is enqueued
+ * on the given CUDA stream (`stream` is a cudaStream_t; NULL = the legacy
+ * default stream).  All pointers are device pointers unless stated.
+ *
+ * Errors.  Every entry point validates its arguments on the host before any
+ * launch and returns NAJU_ERR_INVALID_ARG (null required pointer, bad size,
+ * misaligned pointer: activations need 16-byte alignment) or
+ * NAJU_ERR_UNSUPPORTED (d_state not in {16, 32, 64, 128}, conv_width != 4,
+ * unknown dtype) without touching the GPU.  A failed launch returns
+ * NAJU_ERR_CUDA.  Waits between thread blocks are bounded: when one gives up
+ * it records NAJU_ERR_TIMEOUT in the workspace's status word (read with
+ * naju_last_device_status) and the kernel returns instead of hanging.
+ */
+#ifndef NAJU_H_
+#define NAJU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NAJU_OK = 0,
+    NAJU_ERR_INVALID_ARG = 1,
+    NAJU_ERR_UNSUPPORTED = 2,
+    NAJU_ERR_CUDA = 3,
+    NAJU_ERR_TIMEOUT = 4
+} naju_status;
+
+typedef enum { NAJU_F32 = 0, NAJU_BF16 = 1 } naju_dtype;
+
+typedef struct {
+    int64_t batch;      /* Bt >= 1                                        */
+    int64_t seqlen;     /* L >= 1                                         */
+    int64_t d_inner;    /* d >= 1                                         */
+    int64_t d_state;    /* N in {16, 32, 64, 128}                         */
+    int32_t conv_width; /* W; must be 4 when conv weights are passed      */
+    int32_t dtype;      /* naju_dtype of the activation inputs            */
+    int32_t out_dtype;  /* naju_dtype of y and of the activation grads;
+                           bf16 inputs may write f32 or bf16 outputs,
+                           f32 inputs write f32                            */
+    int32_t reserved;   /* must be 0                                      */
+} naju_dims;
+
+/* Bytes of device workspace that naju_scan_fwd / naju_scan_bwd need for
+ * these dims: state checkpoints written by the forward and read by the
+ * backward, inter-block carry flags, the status word, and the backward's
+ * partial sums.  0 if dims are invalid.  The workspace must be 256-byte
+ * aligned, must not be shared by calls that may run concurrently, and must
+ * be passed unchanged from a forward to the backward of the same inputs. */
+size_t naju_scan_workspace_bytes(const naju_dims* dims);
+
+/* Causal depthwise conv + SiLU (README flowchart, "causal depthwise conv +
+ * SiLU"): h = SiLU(conv(u)).  u, h in dims->dtype (h in out_dtype);
+ * conv_b may be NULL (zero bias).  Uses no workspace. */
+naju_status naju_conv_silu_fwd(const naju_dims* dims, const void* u, const float* conv_w,
+                               const float* conv_b, void* h, void* stream);
+
+/* Gradient of naju_conv_silu_fwd given dh: writes du (out_dtype) and
+ * overwrites dconv_w [d, W], dconv_b [d] (fp32, summed over batch and time;
+ * dconv_b may be NULL). */
+naju_status naju_conv_silu_bwd(const naju_dims* dims, const void* u, const float* conv_w,
+                               const float* conv_b, const void* dh, void* du, float* dconv_w,
+                               float* dconv_b, void* stream);
+
+/* Forward scan (README, "Core equations"), fused with the conv + SiLU that
+ * produces h when conv_w != NULL (then `hu` is u; otherwise `hu` is h) and
+ * with the SiLU(z) output modulation when z != NULL.  D == NULL means no
+ * feedthrough; x0 == NULL means a zero initial state.  Writes y (out_dtype),
+ * optionally x_final, and the state checkpoints the backward needs into the
+ * workspace. */
+naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* conv_w,
+                          const float* conv_b, const void* a, const void* b, const void* B,
+                          const void* C, const void* z, const float* D, const float* x0,
+                          void* y, float* x_final, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Backward of naju_scan_fwd for a loss with gradient dy w.r.t. y and,
+ * optionally, dx_final w.r.t. x_final.  Same inputs as the forward; the
+ * workspace must hold that forward's checkpoints.  Writes dhu (du in fused
+ * mode, dh otherwise), da, db, dB, dC and dz (when z != NULL) in out_dtype,
+ * and overwrites dD (when D != NULL), dconv_w and dconv_b (fused mode) and
+ * dx0 (when not NULL) in fp32. */
+naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* conv_w,
+                          const float* conv_b, const void* a, const void* b, const void* B,
+                          const void* C, const void* z, const float* D, const float* x0,
+                          const void* dy, const float* dx_final, void* dhu, void* da, void* db,
+                          void* dB, void* dC, void* dz, float* dD, float* dconv_w,
+                          float* dconv_b, float* dx0, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* One decode step (README, "Core equations", one token): h, a, b, z, y are
+ * [batch, d_inner] in `dtype` (y too); B, C are [batch, d_state]; state
+ * [batch, d_inner, d_state] fp32 is read and overwritten in place.  h is the
+ * post-conv activation.  z and D may be NULL.  Uses no workspace. */
+naju_status naju_scan_step(int64_t batch, int64_t d_inner, int64_t d_state, int32_t dtype,
+                           const void* h, const void* a, const void* b, const void* B,
+                           const void* C, const void* z, const float* D, float* state, void* y,
+                           void* stream);
+
+/* Synchronises `stream`, reads the workspace's status word (NAJU_OK or
+ * NAJU_ERR_TIMEOUT) and clears it.  Returns NAJU_ERR_CUDA if the stream
+ * itself reports an error. */
+naju_status naju_last_device_status(void* workspace, void* stream);
+
+/* Static description of a status code. */
+const char* naju_status_string(naju_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NAJU_H_ */

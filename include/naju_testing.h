@@ -1,0 +1,39 @@
+/*
+ * naju_testing.h -- process-wide test and tuning hooks of the Naju library.
+ *
+ * These hooks exist so that the library's failure handling can be exercised
+ * without faulting a GPU: a forward whose first sequence group never
+ * publishes its carry makes the next group's bounded wait run out, which must
+ * surface as NAJU_ERR_TIMEOUT from naju_last_device_status() while the kernel
+ * still returns.  They are not part of the numerical interface and default to
+ * off.  Not thread-safe: set them before launching work.
+ */
+#ifndef NAJU_TESTING_H_
+#define NAJU_TESTING_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Polls before an inter-block wait gives up (each poll sleeps <= 0.5 us).
+ * polls <= 0 restores the default (about one second). */
+void naju_testing_set_wait_limit(int64_t polls);
+
+/* skip != 0: the forward's first sequence group and the backward's last
+ * block do not publish their carries (their successors time out). */
+void naju_testing_set_skip_publish(int32_t skip);
+
+/* Forces the number of sequence groups of the forward (<= 0: automatic).
+ * More groups than checkpoint segments are clamped. */
+void naju_testing_set_fwd_groups(int32_t groups);
+
+/* The forward's number of sequence groups for these dims (after the
+ * automatic choice and any forced value). */
+int32_t naju_testing_fwd_groups(const void* dims);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NAJU_TESTING_H_ */

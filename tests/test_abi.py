@@ -1,0 +1,85 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, sizes workspaces, and rejects bad arguments before touching a GPU."""
+import ctypes
+
+import pytest
+
+import discrete_selective_ssm_b200 as naju
+from discrete_selective_ssm_b200 import _native
+
+
+@pytest.fixture(scope="module")
+def L():
+    return naju.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = naju.declared_symbols()
+    assert "naju_scan_fwd" in names and "naju_scan_bwd" in names and "naju_scan_step" in names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+
+
+def test_workspace_bytes(L):
+    d = naju.make_dims(2, 300, 200, 64, naju.BF16)
+    n = naju.workspace_bytes(d)
+    # at least the checkpoints: Bt * (ceil(L/128)+1) * d * N fp32
+    assert n >= 2 * 4 * 200 * 64 * 4
+    assert n % 256 == 0
+    bad = naju.make_dims(2, 300, 200, 48, naju.BF16)
+    assert naju.workspace_bytes(bad) == 0
+    assert L.naju_scan_workspace_bytes(None) == 0
+
+
+def test_rejects_bad_arguments_on_host(L):
+    d = naju.make_dims(1, 8, 8, 16, naju.F32)
+    null = None
+    # null dims / null required pointers -> INVALID_ARG (1), never reaches CUDA
+    assert L.naju_scan_fwd(None, *([null] * 13), 0, null) == 1
+    assert L.naju_scan_fwd(ctypes.byref(d), *([null] * 13), 0, null) == 1
+    assert L.naju_scan_bwd(ctypes.byref(d), *([null] * 23), 0, null) == 1
+    # unsupported d_state -> UNSUPPORTED (2)
+    d2 = naju.make_dims(1, 8, 8, 24, naju.F32)
+    assert L.naju_scan_fwd(ctypes.byref(d2), *([null] * 13), 0, null) == 2
+    # f32 inputs with bf16 outputs -> UNSUPPORTED
+    d3 = naju.make_dims(1, 8, 8, 16, naju.F32, naju.BF16)
+    assert L.naju_scan_fwd(ctypes.byref(d3), *([null] * 13), 0, null) == 2
+    # conv width other than 4 in fused mode -> UNSUPPORTED
+    d4 = naju.make_dims(1, 8, 8, 16, naju.F32, conv_width=3)
+    fake = ctypes.c_void_p(256)
+    assert L.naju_scan_fwd(ctypes.byref(d4), fake, fake, *([null] * 11), 0, null) == 2
+    # misaligned activation pointer -> INVALID_ARG
+    mis = ctypes.c_void_p(258)
+    assert L.naju_scan_fwd(ctypes.byref(d), mis, null, null, fake, fake, fake, fake, null, null,
+                           null, fake, null, fake, 1 << 30, null) == 1
+    # workspace too small -> INVALID_ARG
+    assert L.naju_scan_fwd(ctypes.byref(d), fake, null, null, fake, fake, fake, fake, null, null,
+                           null, fake, null, fake, 16, null) == 1
+    # step: bad d_state / null pointers
+    assert L.naju_scan_step(1, 8, 24, 0, *([null] * 10)) == 2
+    assert L.naju_scan_step(1, 8, 16, 0, *([null] * 10)) == 1
+    assert L.naju_last_device_status(None, None) == 1
+
+
+def test_status_strings(L):
+    for code in range(5):
+        assert L.naju_status_string(code)
+
+
+def test_fwd_group_policy(L):
+    # Few (batch x tile) items split the sequence; many do not.
+    few = naju.make_dims(2, 8192, 2048, 128, naju.BF16)
+    many = naju.make_dims(16, 4096, 2048, 64, naju.BF16)
+    assert naju.testing_fwd_groups(few) > 1
+    assert naju.testing_fwd_groups(many) == 1
+    naju.testing_set_fwd_groups(3)
+    try:
+        assert naju.testing_fwd_groups(many) == 3
+    finally:
+        naju.testing_set_fwd_groups(0)
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        _native._ptr(torch.zeros(4), "x")

@@ -1,0 +1,339 @@
+"""GPU parity: every C-ABI entry point against the fp64 oracle on identical
+seeded inputs, at sizes the oracle finishes in seconds that still span
+several channel tiles, several checkpoint segments and ragged tails."""
+import numpy as np
+import pytest
+import torch
+
+import discrete_selective_ssm_b200 as naju
+import oracle
+from discrete_selective_ssm_b200.workloads import WORKLOADS, make_inputs, scaled
+from naju_check import TOL_BF16, TOL_F32, assert_close, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def wl(N, dtype, Bt=2, L=300, d=200, base="mid_lm", **kw):
+    return scaled(WORKLOADS[base], batch=Bt, seqlen=L, d_inner=d, d_state=N, dtype=dtype, **kw)
+
+
+def gpu(t):
+    return None if t is None else t.to(DEV).contiguous()
+
+
+def inputs(w, conv, use_z=True, use_D=True, use_x0=False, use_dxL=False, seed_offset=0):
+    keys = ["u" if conv else "h", "a", "b", "B", "C", "dout"]
+    if use_z:
+        keys.append("z")
+    if use_D:
+        keys.append("D")
+    if conv:
+        keys += ["conv_w", "conv_b"]
+    if use_x0:
+        keys.append("x0")
+    if use_dxL:
+        keys.append("dxL")
+    return make_inputs(w, which=tuple(keys), seed_offset=seed_offset)
+
+
+def run_fwd(t, conv, out_dtype=None, groups=0):
+    naju.testing_set_fwd_groups(groups)
+    try:
+        hu = t["u"] if conv else t["h"]
+        y, xf, ws = naju.scan_fwd(gpu(hu), gpu(t["a"]), gpu(t["b"]), gpu(t["B"]), gpu(t["C"]),
+                                  conv_w=gpu(t.get("conv_w")), conv_b=gpu(t.get("conv_b")),
+                                  z=gpu(t.get("z")), D=gpu(t.get("D")), x0=gpu(t.get("x0")),
+                                  out_dtype=out_dtype)
+        torch.cuda.synchronize()
+        assert naju.last_device_status(ws) == 0
+    finally:
+        naju.testing_set_fwd_groups(0)
+    return y, xf, ws
+
+
+def oracle_fwd(t, conv):
+    if conv:
+        out, xL, _ = oracle.block_fwd(t["u"], t["conv_w"], t["conv_b"], t["a"], t["b"], t["B"],
+                                      t["C"], t.get("z"), t.get("D"), t.get("x0"))
+    else:
+        out, xL = oracle.scan_fwd(t["h"], t["a"], t["b"], t["B"], t["C"], t.get("z"),
+                                  t.get("D"), t.get("x0"))
+    return out, xL
+
+
+def tol_of(dtype):
+    return TOL_F32 if dtype == "f32" else TOL_BF16
+
+
+# ----------------------------------------------------------------- forward
+@pytest.mark.parametrize("N", [16, 32, 64, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("conv", [True, False])
+def test_fwd_parity(N, dtype, conv):
+    w = wl(N, dtype)
+    t = inputs(w, conv, use_x0=True)
+    out_dt = naju.F32  # bf16 inputs, fp32 outputs: the arithmetic's own error
+    y, xf, _ = run_fwd(t, conv, out_dtype=out_dt)
+    ro, rx = oracle_fwd(t, conv)
+    assert_close(y, ro, tol_of(dtype), name="y")
+    assert_close(xf, rx, tol_of(dtype), name="x_final")
+
+
+@pytest.mark.parametrize("N", [16, 64, 128])
+def test_fwd_bf16_outputs(N):
+    w = wl(N, "bf16", Bt=3, L=257, d=130)
+    t = inputs(w, True)
+    y, xf, _ = run_fwd(t, True, out_dtype=naju.BF16)
+    assert y.dtype == torch.bfloat16
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_BF16, bf16_out=True, name="y")
+    assert_close(xf, rx, TOL_BF16, name="x_final")
+
+
+@pytest.mark.parametrize("groups", [2, 3, 7])
+def test_fwd_sequence_groups(groups):
+    """Splitting the sequence across blocks (look-back carry) changes nothing."""
+    w = wl(64, "f32", Bt=2, L=1000, d=70)
+    t = inputs(w, True, use_x0=True)
+    ro, rx = oracle_fwd(t, True)
+    y, xf, _ = run_fwd(t, True, groups=groups)
+    assert_close(y, ro, TOL_F32, name=f"y groups={groups}")
+    assert_close(xf, rx, TOL_F32, name=f"x_final groups={groups}")
+
+
+@pytest.mark.parametrize("L,d", [(1, 1), (5, 7), (31, 65), (32, 64), (129, 129)])
+def test_fwd_small_and_ragged(L, d):
+    w = wl(32, "f32", Bt=1, L=L, d=d)
+    t = inputs(w, True, use_x0=True)
+    y, xf, _ = run_fwd(t, True)
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_F32, name="y")
+    assert_close(xf, rx, TOL_F32, name="x_final")
+
+
+def test_fwd_no_optional_inputs():
+    w = wl(64, "f32", Bt=2, L=100, d=64)
+    t = inputs(w, False, use_z=False, use_D=False)
+    y, xf, _ = run_fwd(t, False)
+    ro, rx = oracle_fwd(t, False)
+    assert_close(y, ro, TOL_F32, name="y")
+    assert_close(xf, rx, TOL_F32, name="x_final")
+
+
+def test_fwd_extreme_gates():
+    """Forget gates at 0 and 1 (a = -60 / +60) and a long run of tiny f force
+    the rescaled state through many renormalisations."""
+    w = wl(64, "f32", Bt=2, L=400, d=96)
+    t = inputs(w, True, use_x0=True)
+    a = t["a"].clone()
+    a[:, 50:60] = -60.0
+    a[:, 100:300:3] = -25.0
+    a[:, 300:350] = 60.0
+    t["a"] = a
+    y, xf, _ = run_fwd(t, True)
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_F32, name="y")
+    assert_close(xf, rx, TOL_F32, name="x_final")
+
+
+def test_long_retention_overwrite_distribution():
+    """Overwrite events (a ~ N(-4,1), b ~ N(3,1) on 5% of entries)."""
+    w = scaled(WORKLOADS["long_retention"], batch=1, seqlen=700, d_inner=96, d_state=128)
+    t = inputs(w, True)
+    y, xf, ws = run_fwd(t, True, out_dtype=naju.F32)
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_BF16, name="y")
+    assert_close(xf, rx, TOL_BF16, name="x_final")
+
+
+# ---------------------------------------------------------------- backward
+def run_bwd(t, conv, out_dtype=None, groups=0):
+    y, xf, ws = run_fwd(t, conv, out_dtype=out_dtype, groups=groups)
+    hu = t["u"] if conv else t["h"]
+    g = naju.scan_bwd(gpu(t["dout"]), gpu(hu), gpu(t["a"]), gpu(t["b"]), gpu(t["B"]),
+                      gpu(t["C"]), ws, conv_w=gpu(t.get("conv_w")), conv_b=gpu(t.get("conv_b")),
+                      z=gpu(t.get("z")), D=gpu(t.get("D")), x0=gpu(t.get("x0")),
+                      dx_final=gpu(t.get("dxL")), out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert naju.last_device_status(ws) == 0
+    return g
+
+
+def oracle_bwd(t, conv):
+    if conv:
+        return oracle.block_bwd(t["u"], t["conv_w"], t["conv_b"], t["a"], t["b"], t["B"],
+                                t["C"], t.get("z"), t.get("D"), t.get("x0"), t["dout"],
+                                t.get("dxL"))
+    g = oracle.scan_bwd(t["h"], t["a"], t["b"], t["B"], t["C"], t.get("z"), t.get("D"),
+                        t.get("x0"), t["dout"], t.get("dxL"))
+    return g
+
+
+def compare_grads(g, r, conv, tol, bf16_out=False, has_z=True, has_D=True):
+    assert_close(g["dhu"], r["du"] if conv else r["dh"], tol, bf16_out, "du" if conv else "dh")
+    for k in ("da", "db", "dB", "dC"):
+        assert_close(g[k], r[k], tol, bf16_out, k)
+    if has_z:
+        assert_close(g["dz"], r["dz"], tol, bf16_out, "dz")
+    if has_D:
+        assert_close(g["dD"], r["dD"], tol, False, "dD")
+    assert_close(g["dx0"], r["dx0"], tol, False, "dx0")
+    if conv:
+        assert_close(g["dconv_w"], r["dconv_w"], tol, False, "dconv_w")
+        assert_close(g["dconv_b"], r["dconv_b"], tol, False, "dconv_b")
+
+
+@pytest.mark.parametrize("N", [16, 32, 64, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("conv", [True, False])
+def test_bwd_parity(N, dtype, conv):
+    d = {16: 300, 32: 300, 64: 600, 128: 300}[N]
+    w = wl(N, dtype, Bt=2, L=300, d=d)
+    t = inputs(w, conv, use_x0=True, use_dxL=True)
+    g = run_bwd(t, conv, out_dtype=naju.F32)
+    r = oracle_bwd(t, conv)
+    compare_grads(g, r, conv, tol_of(dtype))
+
+
+def test_bwd_bf16_outputs():
+    w = wl(64, "bf16", Bt=2, L=200, d=130)
+    t = inputs(w, True)
+    g = run_bwd(t, True, out_dtype=naju.BF16)
+    r = oracle_bwd(t, True)
+    compare_grads(g, r, True, TOL_BF16, bf16_out=True)
+
+
+@pytest.mark.parametrize("L", [1, 3, 64, 65, 130])
+def test_bwd_lengths(L):
+    w = wl(32, "f32", Bt=2, L=L, d=140)
+    t = inputs(w, True, use_x0=True, use_dxL=True)
+    g = run_bwd(t, True)
+    r = oracle_bwd(t, True)
+    compare_grads(g, r, True, TOL_F32)
+
+
+def test_bwd_no_optional_inputs():
+    w = wl(64, "f32", Bt=1, L=150, d=64)
+    t = inputs(w, False, use_z=False, use_D=False)
+    g = run_bwd(t, False)
+    r = oracle_bwd(t, False)
+    compare_grads(g, r, False, TOL_F32, has_z=False, has_D=False)
+
+
+def test_bwd_extreme_gates():
+    w = wl(64, "f32", Bt=1, L=300, d=64)
+    t = inputs(w, True, use_x0=True, use_dxL=True)
+    a = t["a"].clone()
+    a[:, 40:50] = -60.0
+    a[:, 100:200:3] = -25.0
+    a[:, 220:260] = 60.0
+    t["a"] = a
+    g = run_bwd(t, True)
+    r = oracle_bwd(t, True)
+    compare_grads(g, r, True, TOL_F32)
+
+
+def test_bwd_after_grouped_forward():
+    """Checkpoints written by a sequence-split forward serve the backward."""
+    w = wl(64, "f32", Bt=1, L=700, d=64)
+    t = inputs(w, True, use_x0=True)
+    g = run_bwd(t, True, groups=3)
+    r = oracle_bwd(t, True)
+    compare_grads(g, r, True, TOL_F32)
+
+
+# ------------------------------------------------------------- decode step
+@pytest.mark.parametrize("N", [16, 32, 64, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_step_parity(N, dtype):
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    gen = torch.Generator().manual_seed(N)
+    Bt, d = 5, 77
+    state = torch.randn(Bt, d, N, generator=gen)
+    h, a, b, z = (torch.randn(Bt, d, generator=gen).to(tdt) for _ in range(4))
+    a = (a.float() + 4).to(tdt)
+    B, C = (torch.randn(Bt, N, generator=gen).to(tdt) for _ in range(2))
+    D = torch.randn(d, generator=gen)
+    ro, rs = oracle.scan_step(state, h, a, b, B, C, z, D)
+    st = gpu(state)
+    y = naju.scan_step(st, gpu(h), gpu(a), gpu(b), gpu(B), gpu(C), gpu(z), gpu(D))
+    torch.cuda.synchronize()
+    tol = tol_of(dtype)
+    assert_close(y, ro, tol, bf16_out=(dtype == "bf16"), name="y")
+    assert_close(st, rs, tol, name="state")
+
+
+def test_steps_equal_forward():
+    """L decode steps from x0 reproduce the forward's final state (f32)."""
+    w = wl(64, "f32", Bt=2, L=40, d=48)
+    t = inputs(w, False, use_x0=True)
+    y, xf, _ = run_fwd(t, False)
+    st = gpu(t["x0"])
+    for n in range(40):
+        yn = naju.scan_step(st, gpu(t["h"][:, n]), gpu(t["a"][:, n]), gpu(t["b"][:, n]),
+                            gpu(t["B"][:, n]), gpu(t["C"][:, n]), gpu(t["z"][:, n]),
+                            gpu(t["D"]))
+        assert_close(yn, to_np(y)[:, n], TOL_F32, name=f"y[{n}]")
+    torch.cuda.synchronize()
+    assert_close(st, xf, TOL_F32, name="state")
+
+
+# -------------------------------------------------------------- the conv
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_conv_standalone(dtype):
+    w = wl(16, dtype, Bt=2, L=150, d=100)
+    t = make_inputs(w, which=("u", "conv_w", "conv_b", "dout"))
+    cb = torch.randn(100)
+    h = naju.conv_silu_fwd(gpu(t["u"]), gpu(t["conv_w"]), gpu(cb))
+    rh = oracle.conv_silu_fwd(t["u"], t["conv_w"], cb)
+    assert_close(h, rh, tol_of(dtype), bf16_out=(dtype == "bf16"), name="h")
+    du, dw, db = naju.conv_silu_bwd(gpu(t["u"]), gpu(t["conv_w"]), gpu(cb), gpu(t["dout"]))
+    rdu, rdw, rdb = oracle.conv_silu_bwd(t["u"], t["conv_w"], cb, t["dout"])
+    torch.cuda.synchronize()
+    assert_close(du, rdu, tol_of(dtype), bf16_out=(dtype == "bf16"), name="du")
+    assert_close(dw, rdw, tol_of(dtype), name="dw")
+    assert_close(db, rdb, tol_of(dtype), name="dbias")
+
+
+# ---------------------------------------------------- bounded-wait failure
+def test_forward_wait_timeout_is_reported():
+    """A group that never publishes makes its successor's bounded wait give
+    up: the kernel returns and the status word reports the timeout."""
+    w = wl(32, "f32", Bt=1, L=512, d=64)
+    t = inputs(w, True)
+    naju.testing_set_wait_limit(2000)
+    naju.testing_set_skip_publish(True)
+    naju.testing_set_fwd_groups(4)
+    try:
+        hu = gpu(t["u"])
+        y, xf, ws = naju.scan_fwd(hu, gpu(t["a"]), gpu(t["b"]), gpu(t["B"]), gpu(t["C"]),
+                                  conv_w=gpu(t["conv_w"]), conv_b=gpu(t["conv_b"]))
+        assert naju.last_device_status(ws) == 4
+        assert naju.last_device_status(ws) == 0  # cleared on read
+    finally:
+        naju.testing_set_skip_publish(False)
+        naju.testing_set_wait_limit(0)
+        naju.testing_set_fwd_groups(0)
+    # The context is still usable and the next call is correct.
+    y, xf, _ = run_fwd(t, True)
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_F32, name="y after timeout")
+
+
+def test_backward_wait_timeout_is_reported():
+    w = wl(32, "f32", Bt=1, L=256, d=64)
+    t = inputs(w, True)
+    y, xf, ws = run_fwd(t, True)
+    naju.testing_set_wait_limit(2000)
+    naju.testing_set_skip_publish(True)
+    try:
+        naju.scan_bwd(gpu(t["dout"]), gpu(t["u"]), gpu(t["a"]), gpu(t["b"]), gpu(t["B"]),
+                      gpu(t["C"]), ws, conv_w=gpu(t["conv_w"]), conv_b=gpu(t["conv_b"]))
+        assert naju.last_device_status(ws) == 4
+    finally:
+        naju.testing_set_skip_publish(False)
+        naju.testing_set_wait_limit(0)
+    g = run_bwd(t, True)
+    r = oracle_bwd(t, True)
+    compare_grads(g, r, True, TOL_F32)

@@ -50,9 +50,11 @@ __device__ __forceinline__ void store8(float* p, const float* v) {
 }
 
 // ------------------------------------------------------------ activations
-// CUDA's fast exponential; the accuracy of each use is covered by the
+// CUDA's fast exponential and its round-to-nearest reciprocal (inf -> 0, so
+// sigmoid saturates cleanly); the accuracy of each use is covered by the
 // parity tests against the fp64 oracle.
-__device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + __expf(-v)); }
+__device__ __forceinline__ float rcpf_(float v) { return __frcp_rn(v); }
+__device__ __forceinline__ float sigmoidf_(float v) { return rcpf_(1.0f + __expf(-v)); }
 __device__ __forceinline__ float siluf_(float v) { return v * sigmoidf_(v); }
 // d/dv SiLU(v) = s (1 + v (1 - s)), s = sigmoid(v)
 __device__ __forceinline__ float dsiluf_(float v) {
@@ -99,5 +101,56 @@ struct WsHeader {
     int pad3[32];
 };
 static_assert(sizeof(WsHeader) == 512, "header is two 256-byte blocks");
+
+}  // namespace naju
+
+namespace naju {
+
+// ------------------------------------------------------ async staging
+// 16-byte global -> shared copy; src_bytes = 0 zero-fills the destination
+// (no global bytes are read; `src` must still be a valid address).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N_>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N_) : "memory");
+}
+
+// Stage `rows` rows (token t0 + r, r in [0, rows)) of a [Bt, L, width]
+// tensor, columns [col0, col0 + cols), into dst[rows][cols] (element type T).
+// Rows outside [0, tlim) and columns past `width` are zero.  vec: the 16-byte
+// path is legal (width * sizeof(T) and col0 * sizeof(T) multiples of 16,
+// cols * sizeof(T) multiple of 16); otherwise plain loads are used.
+template <typename T>
+__device__ __forceinline__ void stage_rows(T* dst, const T* src_b, int64_t width, int64_t t0,
+                                           int rows, int64_t tlim, int64_t col0, int cols,
+                                           bool vec, int tid, int nthreads) {
+    constexpr int G = 16 / sizeof(T);  // elements per granule
+    if (vec) {
+        const int gpr = cols / G;      // granules per row
+        for (int e = tid; e < rows * gpr; e += nthreads) {
+            const int r = e / gpr, gi = e % gpr;
+            const int64_t t = t0 + r;
+            const int64_t col = col0 + (int64_t)gi * G;
+            const bool ok = t >= 0 && t < tlim && col < width;
+            const T* s = ok ? src_b + t * width + col : src_b;
+            cp_async16(dst + r * cols + gi * G, s, ok ? 16 : 0);
+        }
+    } else {
+        for (int e = tid; e < rows * cols; e += nthreads) {
+            const int r = e / cols, ci = e % cols;
+            const int64_t t = t0 + r;
+            const int64_t col = col0 + ci;
+            T v = T(0.f);
+            if (t >= 0 && t < tlim && col < width) v = src_b[t * width + col];
+            dst[r * cols + ci] = v;
+        }
+    }
+}
 
 }  // namespace naju

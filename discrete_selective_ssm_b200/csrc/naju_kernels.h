@@ -7,7 +7,7 @@ namespace naju {
 
 struct WsHeader;
 
-constexpr int kFwdChunk = 32;   // tokens staged per forward chunk
+constexpr int kFwdChunk = 16;   // tokens staged per forward chunk
 constexpr int kBwdSub = 64;     // tokens per backward work item
 constexpr int kBwdChunk = 16;   // tokens per backward contraction block
 

@@ -29,6 +29,8 @@
 //  4. sweeps backward: the adjoint G, per-channel gradients, and per
 //     sub-block dB_m = s sum_{t>=m} A[t,m] C_t + (i h F)_m H_e, with H_e the
 //     carry entering the sub-block's end and F_m the decay to that end.
+// Every sub-block's raw inputs are staged by cp.async, and the next
+// sub-block's copy is issued as soon as the current one has been unpacked.
 // dB/dC partial sums over the P channels are summed across the thread-block
 // cluster (consecutive channel tiles) through distributed shared memory and
 // written once per cluster; small kernels then sum clusters, the per-channel
@@ -55,30 +57,36 @@ template <> struct BwdShape<128> { static constexpr int NS = 32, S = 4; };
 int bwd_channels_per_block(int64_t N) { return N <= 32 ? 128 : (N == 64 ? 64 : 32); }
 int bwd_cluster_size() { return kCluster; }
 
-template <int N, int P>
+template <typename Tin, int N, int P>
 struct BwdSmem {
     static constexpr int T = kBwdChunk;   // 16
     static constexpr int K = kBwdSub;     // 64
+    // raw rows of the current sub-block (cp.async destination)
+    Tin u[T + 3][P], a[T][P], b[T][P], z[T][P], dout[T][P];
+    Tin Bm[T][N], Cm[T][N];
+    // unpacked per-(token, channel) values
     float f[T][P], q[T][P], v[T][P], dy[T][P];
-    float lg[T][P], E[T][P];              // clamped log-prefix / true decay prefix
-    float fa[T][P], fb[T][P];             // A factors (dy side / i h side)
-    float gb[T][P], fdf[T][P], dp[T + 3][P];
-    float ys[K][P];                       // unscaled readout x_t . C_t
-    float Bm[T][N], Cm[T][N];
-    float snap[P][N];                     // X_b (forward) or H_e (backward)
-    float A[K / T][T][T];                 // per sub-block contraction matrix
-    float acc[K][2][N];                   // dB (0) and dC (1) partials of the item
-    int item;
+    float x1[T][P];   // forward: clamped log-prefix   backward: G . B
+    float x2[T][P];   // forward: dy * decay prefix    backward: i h * decay to end
+    float x3[T][P];   // forward: A factor (dy side)   backward: f df
+    float x4[T][P];   // forward: A factor (i h side)
+    float dp[T + 3][P];
+    float ys[K][P];   // unscaled readout x_t . C_t of the block
+    float Bf[T][N], Cf[T][N];
+    float snap[P][N]; // X_b (forward) or H_e (backward)
+    float A[K / T][T][T];
+    float acc[K][N];  // dC (forward sweep) then dB (backward sweep) partials
+    int item, ok;
 };
 
 template <typename Tin, typename Tout, int N, bool CONV>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 2)
 scan_bwd_kernel(const BwdParams p) {
     constexpr int NS = BwdShape<N>::NS, S = BwdShape<N>::S;
     constexpr int NT = 128, P = NT / S;
     constexpr int T = kBwdChunk, K = kBwdSub, NSUB = K / T;
     constexpr int R = T / S;              // prep run length per thread
-    using Sm = BwdSmem<N, P>;
+    using Sm = BwdSmem<Tin, N, P>;
     extern __shared__ float4 smem4[];
     Sm& sm = *reinterpret_cast<Sm*>(smem4);
     cg::cluster_group cluster = cg::this_cluster();
@@ -108,13 +116,15 @@ scan_bwd_kernel(const BwdParams p) {
     const int64_t te = min64(L, tb + K);
     const bool last = (k == p.nsub - 1);
 
-    const Tin* hu = static_cast<const Tin*>(p.hu);
-    const Tin* ga = static_cast<const Tin*>(p.a);
-    const Tin* gbp = static_cast<const Tin*>(p.b);
-    const Tin* gB = static_cast<const Tin*>(p.B);
-    const Tin* gC = static_cast<const Tin*>(p.C);
-    const Tin* gz = static_cast<const Tin*>(p.z);
-    const Tin* gdy = static_cast<const Tin*>(p.dy);
+    const int64_t boff = (int64_t)bb * L;
+    const Tin* hu = static_cast<const Tin*>(p.hu) + boff * d;
+    const Tin* ga = static_cast<const Tin*>(p.a) + boff * d;
+    const Tin* gbp = static_cast<const Tin*>(p.b) + boff * d;
+    const Tin* gz = p.z ? static_cast<const Tin*>(p.z) + boff * d : nullptr;
+    const Tin* gdy = static_cast<const Tin*>(p.dy) + boff * d;
+    const Tin* gB = static_cast<const Tin*>(p.B) + boff * N;
+    const Tin* gC = static_cast<const Tin*>(p.C) + boff * N;
+    const bool vec = ((d * (int64_t)sizeof(Tin)) % 16) == 0;
 
     float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, wb = 0.f, Dc = 0.f;
     if (cpvalid) {
@@ -126,48 +136,62 @@ scan_bwd_kernel(const BwdParams p) {
         Dc = p.D ? p.D[cp] : 0.f;
     }
 
-    // Stage one sub-block [t0, t0+T) of per-(token, channel) scalars and B, C.
-    auto stage = [&](int64_t t0, int64_t tlim) {
+    // Stage the raw rows of sub-block [t0, t0+T) (tokens >= tlim are zero).
+    auto issue = [&](int64_t t0, int64_t tlim) {
+        stage_rows(&sm.u[0][0], hu, d, t0 - 3, T + 3, L, c0, P, vec, tid, NT);
+        stage_rows(&sm.a[0][0], ga, d, t0, T, tlim, c0, P, vec, tid, NT);
+        stage_rows(&sm.b[0][0], gbp, d, t0, T, tlim, c0, P, vec, tid, NT);
+        if (gz) stage_rows(&sm.z[0][0], gz, d, t0, T, tlim, c0, P, vec, tid, NT);
+        stage_rows(&sm.dout[0][0], gdy, d, t0, T, tlim, c0, P, vec, tid, NT);
+        stage_rows(&sm.Bm[0][0], gB, N, t0, T, tlim, 0, N, true, tid, NT);
+        stage_rows(&sm.Cm[0][0], gC, N, t0, T, tlim, 0, N, true, tid, NT);
+        cp_async_commit();
+    };
+    // Unpack the staged rows into fp32 per-(token, channel) values.
+    auto prep = [&](int64_t t0, int64_t tlim) {
         for (int e = tid; e < T * N; e += NT) {
-            const int tt = e / N;
-            const int64_t t = t0 + tt;
-            float vb = 0.f, vc = 0.f;
-            if (t < tlim) {
-                vb = to_f(gB[((int64_t)bb * L + t) * N + (e % N)]);
-                vc = to_f(gC[((int64_t)bb * L + t) * N + (e % N)]);
-            }
-            sm.Bm[tt][e % N] = vb;
-            sm.Cm[tt][e % N] = vc;
+            (&sm.Bf[0][0])[e] = to_f((&sm.Bm[0][0])[e]);
+            (&sm.Cf[0][0])[e] = to_f((&sm.Cm[0][0])[e]);
         }
-        const int64_t tr = t0 + rr * R;
-        float u0 = 0.f, u1 = 0.f, u2 = 0.f;
-        if (CONV && cpvalid) {
-            const Tin* col = hu + (int64_t)bb * L * d + cp;
-            if (tr >= 3 && tr - 3 < L) u0 = to_f(col[(tr - 3) * d]);
-            if (tr >= 2 && tr - 2 < L) u1 = to_f(col[(tr - 2) * d]);
-            if (tr >= 1 && tr - 1 < L) u2 = to_f(col[(tr - 1) * d]);
-        }
+#pragma unroll
         for (int kk = 0; kk < R; ++kk) {
             const int tt = rr * R + kk;
-            const int64_t t = tr + kk;
+            const int64_t t = t0 + tt;
             float f = 1.f, q = 1.f, v = 0.f, dyv = 0.f;
             if (cpvalid && t < tlim) {
-                const int64_t e = ((int64_t)bb * L + t) * d + cp;
                 float h;
                 if (CONV) {
-                    const float u3 = to_f(hu[e]);
-                    h = siluf_(wb + w0 * u0 + w1 * u1 + w2 * u2 + w3 * u3);
-                    u0 = u1; u1 = u2; u2 = u3;
+                    h = siluf_(wb + w0 * to_f(sm.u[tt][pp]) + w1 * to_f(sm.u[tt + 1][pp]) +
+                               w2 * to_f(sm.u[tt + 2][pp]) + w3 * to_f(sm.u[tt + 3][pp]));
                 } else {
-                    h = to_f(hu[e]);
+                    h = to_f(sm.u[tt + 3][pp]);
                 }
-                q = 1.f + __expf(-to_f(ga[e]));
-                f = 1.f / q;
-                v = sigmoidf_(to_f(gbp[e])) * h;
-                dyv = to_f(gdy[e]);
-                if (gz) dyv *= siluf_(to_f(gz[e]));
+                q = 1.f + __expf(-to_f(sm.a[tt][pp]));
+                f = rcpf_(q);
+                v = sigmoidf_(to_f(sm.b[tt][pp])) * h;
+                dyv = to_f(sm.dout[tt][pp]);
+                if (gz) dyv *= siluf_(to_f(sm.z[tt][pp]));
             }
             sm.f[tt][pp] = f; sm.q[tt][pp] = q; sm.v[tt][pp] = v; sm.dy[tt][pp] = dyv;
+        }
+    };
+    // Sub-block sequence of a pass: sub-block i starts at t0 + dir * i * T.
+    // The raw buffer is refilled with sub-block i+1 right after sub-block i
+    // is unpacked unless `late` (the body reads raw rows), in which case the
+    // refill follows the body.
+    auto pass = [&](int64_t first, int count, int dir, int64_t tlim, bool late, auto&& body) {
+        if (count <= 0) return;
+        issue(first, tlim);
+        for (int i = 0; i < count; ++i) {
+            const int64_t t0 = first + (int64_t)dir * i * T;
+            cp_async_wait<0>();
+            __syncthreads();
+            prep(t0, tlim);
+            __syncthreads();
+            if (!late && i + 1 < count) issue(t0 + dir * T, tlim);
+            body(i, t0);
+            __syncthreads();
+            if (late && i + 1 < count) issue(t0 + dir * T, tlim);
         }
     };
 
@@ -204,8 +228,8 @@ scan_bwd_kernel(const BwdParams p) {
         }
         Q = Qn; iQ = iQn;
         const float wv = vv * Q;
-        const float4* b4 = reinterpret_cast<const float4*>(sm.Bm[tt]);
-        const float4* c4 = reinterpret_cast<const float4*>(sm.Cm[tt]);
+        const float4* b4 = reinterpret_cast<const float4*>(sm.Bf[tt]);
+        const float4* c4 = reinterpret_cast<const float4*>(sm.Cf[tt]);
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
         for (int m = 0; m < NS / 4; ++m) {
@@ -225,11 +249,10 @@ scan_bwd_kernel(const BwdParams p) {
         return ((a0 + a1) + (a2 + a3)) * iQ;
     };
     // Backward token t (after the carry from t+1 is in gs): G_t = G + s dy C.
-    // The decay f_{t+1} was folded in by bdecay() of the later token.
     auto bstep = [&](int tt, bool dotB) -> float {
         const float wv = s * sm.dy[tt][pl] * Rr;
-        const float4* b4 = reinterpret_cast<const float4*>(sm.Bm[tt]);
-        const float4* c4 = reinterpret_cast<const float4*>(sm.Cm[tt]);
+        const float4* b4 = reinterpret_cast<const float4*>(sm.Bf[tt]);
+        const float4* c4 = reinterpret_cast<const float4*>(sm.Cf[tt]);
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
         for (int m = 0; m < NS / 4; ++m) {
@@ -260,6 +283,24 @@ scan_bwd_kernel(const BwdParams p) {
         }
         Rr = Rn; iR = iRn;
     };
+    // Cluster sum of acc[K][N] into the dB (slot 0) or dC (slot 1) partials.
+    auto cluster_reduce = [&](int slot) {
+        cluster.sync();
+        constexpr int ROWS = K / kCluster;
+        const int r0 = crank * ROWS;
+        float* out = p.dBCp + (((int64_t)cgi * Bt + bb) * L) * 2 * N + slot * N;
+        for (int e = tid; e < ROWS * N; e += NT) {
+            const int tt = r0 + e / N;
+            const int j = e % N;
+            float a = 0.f;
+#pragma unroll
+            for (int qr = 0; qr < kCluster; ++qr)
+                a += cluster.map_shared_rank(&sm.acc[0][0], qr)[tt * N + j];
+            const int64_t t = tb + tt;
+            if (t < te) out[t * 2 * N + j] = a;
+        }
+        cluster.sync();
+    };
 
     // --------------------------------------- 0. state entering the block
     {
@@ -267,12 +308,10 @@ scan_bwd_kernel(const BwdParams p) {
         const float* ck = p.ckpt + ((int64_t)bb * (p.nck + 1) + kc) * d * N;
         load_rows(xs, ck, false);
         Q = 1.f; iQ = 1.f;
-        for (int64_t t0 = (int64_t)kc * p.T_ck; t0 < tb; t0 += T) {
-            stage(t0, tb);
-            __syncthreads();
+        const int64_t t_ck = (int64_t)kc * p.T_ck;
+        pass(t_ck, (int)((tb - t_ck) / T), +1, tb, false, [&](int, int64_t) {
             for (int tt = 0; tt < T; ++tt) fstep(tt, false);
-            __syncthreads();
-        }
+        });
 #pragma unroll
         for (int j = 0; j < NS; ++j) xs[j] *= iQ;
         Q = 1.f; iQ = 1.f;
@@ -284,16 +323,12 @@ scan_bwd_kernel(const BwdParams p) {
 #pragma unroll
         for (int j = 0; j < NS; ++j) gs[j] = 0.f;
         Rr = 1.f; iR = 1.f; logF = 0.f;
-        for (int sb = NSUB - 1; sb >= 0; --sb) {
-            const int64_t t0 = tb + sb * T;
-            stage(t0, te);
-            __syncthreads();
+        pass(tb + (NSUB - 1) * T, NSUB, -1, te, false, [&](int, int64_t) {
             for (int tt = T - 1; tt >= 0; --tt) {
                 bstep(tt, false);
                 bdecay(tt);
             }
-            __syncthreads();
-        }
+        });
     }
 
     // -------------------------------------------- 2. carry in / publish
@@ -303,11 +338,10 @@ scan_bwd_kernel(const BwdParams p) {
     int* flag_out = k > 0 ? p.flags + ((int64_t)(k - 1) * Bt + bb) * p.ntiles + tile : nullptr;
     float H[NS];
     {
-        __shared__ int s_ok;
         if (!last) {
-            if (tid == 0) s_ok = wait_flag(flag_in, &p.hdr->status, p.wait_limit) ? 1 : 0;
+            if (tid == 0) sm.ok = wait_flag(flag_in, &p.hdr->status, p.wait_limit) ? 1 : 0;
             __syncthreads();
-            load_rows(H, s_ok ? carry_in : nullptr, true);
+            load_rows(H, sm.ok ? carry_in : nullptr, true);
         } else {
             load_rows(H, p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr, false);
         }
@@ -331,9 +365,7 @@ scan_bwd_kernel(const BwdParams p) {
     }
 
     // ---------------------------------------------- 3. forward sweep
-    for (int sb = 0; sb < NSUB; ++sb) {
-        const int64_t t0 = tb + sb * T;
-        stage(t0, te);
+    pass(tb, NSUB, +1, te, false, [&](int sb, int64_t t0) {
         // Snapshot of the state entering the sub-block (xs is unscaled here).
         if (cvalid) {
 #pragma unroll
@@ -343,7 +375,6 @@ scan_bwd_kernel(const BwdParams p) {
         } else if (js == 0) {
             for (int j = 0; j < N; ++j) sm.snap[pl][j] = 0.f;
         }
-        __syncthreads();
         float lg = 0.f, E = 1.f;
         for (int tt = 0; tt < T; ++tt) {
             const float yv = red(fstep(tt, true));
@@ -352,8 +383,8 @@ scan_bwd_kernel(const BwdParams p) {
             E *= fv;
             if (js == 0) {
                 sm.ys[sb * T + tt][pl] = yv;
-                sm.lg[tt][pl] = lg;
-                sm.E[tt][pl] = E;
+                sm.x1[tt][pl] = lg;
+                sm.x2[tt][pl] = E;
             }
         }
 #pragma unroll
@@ -363,21 +394,22 @@ scan_bwd_kernel(const BwdParams p) {
         // Pivot factors of A around token T/2 of the sub-block.
         for (int kk = 0; kk < R; ++kk) {
             const int tt = rr * R + kk;
-            const float piv = sm.lg[T / 2][pp];
-            const float l = sm.lg[tt][pp];
-            sm.fa[tt][pp] = sm.dy[tt][pp] * __expf(l - piv);
-            sm.fb[tt][pp] = sm.v[tt][pp] * __expf(piv - l);
-            sm.E[tt][pp] *= sm.dy[tt][pp];  // dy_t E_t
+            const float piv = sm.x1[T / 2][pp];
+            const float l = sm.x1[tt][pp];
+            sm.x3[tt][pp] = sm.dy[tt][pp] * __expf(l - piv);
+            sm.x4[tt][pp] = sm.v[tt][pp] * __expf(piv - l);
+            sm.x2[tt][pp] *= sm.dy[tt][pp];  // dy_t E_t
         }
         __syncthreads();
         // A[t][m] = sum_p fa[t][p] fb[m][p] for m <= t.
         for (int e = tid; e < T * T; e += NT) {
             const int tt = e / T, mm = e % T;
-            float acc = 0.f;
+            float a = 0.f;
             if (mm <= tt) {
-                for (int q2 = 0; q2 < P; ++q2) acc = fmaf(sm.fa[tt][q2], sm.fb[mm][q2], acc);
+#pragma unroll 8
+                for (int q2 = 0; q2 < P; ++q2) a = fmaf(sm.x3[tt][q2], sm.x4[mm][q2], a);
             }
-            sm.A[sb][tt][mm] = acc;
+            sm.A[sb][tt][mm] = a;
         }
         __syncthreads();
         // dC[t][j] = s [ sum_p (dy E)[t][p] X_b[p][j] + sum_{m<=t} A[t][m] B[m][j] ].
@@ -388,21 +420,22 @@ scan_bwd_kernel(const BwdParams p) {
             float o[JB];
 #pragma unroll
             for (int r = 0; r < JB; ++r) o[r] = 0.f;
+#pragma unroll 4
             for (int q2 = 0; q2 < P; ++q2) {
-                const float a = sm.E[tt][q2];
+                const float a = sm.x2[tt][q2];
 #pragma unroll
                 for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.snap[q2][j0 + r], o[r]);
             }
             for (int mm = 0; mm <= tt; ++mm) {
                 const float a = sm.A[sb][tt][mm];
 #pragma unroll
-                for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.Bm[mm][j0 + r], o[r]);
+                for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.Bf[mm][j0 + r], o[r]);
             }
 #pragma unroll
-            for (int r = 0; r < JB; ++r) sm.acc[sb * T + tt][1][j0 + r] = s * o[r];
+            for (int r = 0; r < JB; ++r) sm.acc[sb * T + tt][j0 + r] = s * o[r];
         }
-        __syncthreads();
-    }
+    });
+    cluster_reduce(1);
 
     // tail of f df: H . x_end (per channel)
     float tail = 0.f;
@@ -416,17 +449,16 @@ scan_bwd_kernel(const BwdParams p) {
     Rr = 1.f; iR = 1.f; logF = 0.f;
     float cum = 0.f;  // sum of dL over later tokens of the block
     float dD_acc = 0.f, dw0 = 0.f, dw1 = 0.f, dw2 = 0.f, dw3 = 0.f, dbias = 0.f;
-    Tout* gdhu = static_cast<Tout*>(p.dhu);
-    Tout* gda = static_cast<Tout*>(p.da);
-    Tout* gdb = static_cast<Tout*>(p.db);
-    Tout* gdz = static_cast<Tout*>(p.dz);
+    Tout* gdhu = static_cast<Tout*>(p.dhu) + boff * d;
+    Tout* gda = static_cast<Tout*>(p.da) + boff * d;
+    Tout* gdb = static_cast<Tout*>(p.db) + boff * d;
+    Tout* gdz = p.dz ? static_cast<Tout*>(p.dz) + boff * d : nullptr;
     float* edge = p.conv_edge + ((int64_t)bb * p.nsub + k) * 2 * 3 * d;
     if (tid < P) {  // dp beyond the block: zero (next block's terms go via the edge fixup)
         sm.dp[T][tid] = 0.f; sm.dp[T + 1][tid] = 0.f; sm.dp[T + 2][tid] = 0.f;
     }
-    for (int sb = NSUB - 1; sb >= 0; --sb) {
-        const int64_t t0 = tb + sb * T;
-        stage(t0, te);
+    pass(tb + (NSUB - 1) * T, NSUB, -1, te, true, [&](int i, int64_t t0) {
+        const int sb = NSUB - 1 - i;
         // H_e: carry entering the sub-block's end, true scale.
         if (cvalid) {
 #pragma unroll
@@ -437,7 +469,6 @@ scan_bwd_kernel(const BwdParams p) {
         } else if (js == 0) {
             for (int j = 0; j < N; ++j) sm.snap[pl][j] = 0.f;
         }
-        __syncthreads();
         float F = 1.f;  // prod f_{m+1..end of sub-block}
         for (int tt = T - 1; tt >= 0; --tt) {
             const float gbv = red(bstep(tt, true));
@@ -445,9 +476,9 @@ scan_bwd_kernel(const BwdParams p) {
             const float dL = s * sm.dy[tt][pl] * sm.ys[sb * T + tt][pl] - vv * gbv;
             cum += dL;
             if (js == 0) {
-                sm.gb[tt][pl] = gbv;
-                sm.fdf[tt][pl] = cum + tail;
-                sm.E[tt][pl] = vv * F;  // (i h F)_m
+                sm.x1[tt][pl] = gbv;
+                sm.x3[tt][pl] = cum + tail;
+                sm.x2[tt][pl] = vv * F;  // (i h F)_m
             }
             F *= sm.f[tt][pl];
             bdecay(tt);
@@ -461,83 +492,75 @@ scan_bwd_kernel(const BwdParams p) {
             float o[JB], o2[JB];
 #pragma unroll
             for (int r = 0; r < JB; ++r) { o[r] = 0.f; o2[r] = 0.f; }
+#pragma unroll 4
             for (int q2 = 0; q2 < P; ++q2) {
-                const float a = sm.E[mm][q2];
+                const float a = sm.x2[mm][q2];
 #pragma unroll
                 for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.snap[q2][j0 + r], o[r]);
             }
             for (int tt = mm; tt < T; ++tt) {
                 const float a = sm.A[sb][tt][mm];
 #pragma unroll
-                for (int r = 0; r < JB; ++r) o2[r] = fmaf(a, sm.Cm[tt][j0 + r], o2[r]);
+                for (int r = 0; r < JB; ++r) o2[r] = fmaf(a, sm.Cf[tt][j0 + r], o2[r]);
             }
 #pragma unroll
-            for (int r = 0; r < JB; ++r) sm.acc[sb * T + mm][0][j0 + r] = fmaf(s, o2[r], o[r]);
+            for (int r = 0; r < JB; ++r) sm.acc[sb * T + mm][j0 + r] = fmaf(s, o2[r], o[r]);
         }
         // Per-channel gradients of the sub-block (thread pp, run rr).
-        {
-            const int64_t tr = t0 + rr * R;
-            float u0 = 0.f, u1 = 0.f, u2 = 0.f;
-            if (CONV && cpvalid) {
-                const Tin* col = hu + (int64_t)bb * L * d + cp;
-                if (tr >= 3 && tr - 3 < L) u0 = to_f(col[(tr - 3) * d]);
-                if (tr >= 2 && tr - 2 < L) u1 = to_f(col[(tr - 2) * d]);
-                if (tr >= 1 && tr - 1 < L) u2 = to_f(col[(tr - 1) * d]);
-            }
-            for (int kk = 0; kk < R; ++kk) {
-                const int tt = rr * R + kk;
-                const int64_t t = tr + kk;
-                float dpv = 0.f;
-                if (cpvalid && t < te) {
-                    const int64_t e = ((int64_t)bb * L + t) * d + cp;
-                    float h, pre = 0.f, u3 = 0.f;
-                    if (CONV) {
-                        u3 = to_f(hu[e]);
-                        pre = wb + w0 * u0 + w1 * u1 + w2 * u2 + w3 * u3;
-                        h = siluf_(pre);
-                    } else {
-                        h = to_f(hu[e]);
-                    }
-                    const float fv = sm.f[tt][pp];
-                    const float iv = sigmoidf_(to_f(gbp[e]));
-                    const float gbv = sm.gb[tt][pp];
-                    const float dyv = sm.dy[tt][pp];
-                    const float dh = Dc * dyv + iv * gbv;
-                    gda[e] = from_f<Tout>(sm.fdf[tt][pp] * (1.f - fv));
-                    gdb[e] = from_f<Tout>(h * gbv * iv * (1.f - iv));
-                    if (gz) {
-                        const float zv = to_f(gz[e]);
-                        const float yv = fmaf(s, sm.ys[sb * T + tt][pp], Dc * h);
-                        gdz[e] = from_f<Tout>(to_f(gdy[e]) * yv * dsiluf_(zv));
-                    }
-                    dD_acc = fmaf(dyv, h, dD_acc);
-                    if (CONV) {
-                        dpv = dh * dsiluf_(pre);
-                        dw0 = fmaf(dpv, u0, dw0); dw1 = fmaf(dpv, u1, dw1);
-                        dw2 = fmaf(dpv, u2, dw2); dw3 = fmaf(dpv, u3, dw3);
-                        dbias += dpv;
-                        u0 = u1; u1 = u2; u2 = u3;
-                    } else {
-                        gdhu[e] = from_f<Tout>(dh);
-                    }
+#pragma unroll
+        for (int kk = 0; kk < R; ++kk) {
+            const int tt = rr * R + kk;
+            const int64_t t = t0 + tt;
+            float dpv = 0.f;
+            if (cpvalid && t < te) {
+                float h, pre = 0.f;
+                if (CONV) {
+                    pre = wb + w0 * to_f(sm.u[tt][pp]) + w1 * to_f(sm.u[tt + 1][pp]) +
+                          w2 * to_f(sm.u[tt + 2][pp]) + w3 * to_f(sm.u[tt + 3][pp]);
+                    h = siluf_(pre);
+                } else {
+                    h = to_f(sm.u[tt + 3][pp]);
                 }
-                if (CONV) sm.dp[tt][pp] = dpv;
+                const float fv = sm.f[tt][pp];
+                const float iv = sigmoidf_(to_f(sm.b[tt][pp]));
+                const float gbv = sm.x1[tt][pp];
+                const float dyv = sm.dy[tt][pp];
+                const float dh = Dc * dyv + iv * gbv;
+                gda[t * d + cp] = from_f<Tout>(sm.x3[tt][pp] * (1.f - fv));
+                gdb[t * d + cp] = from_f<Tout>(h * gbv * iv * (1.f - iv));
+                if (gz) {
+                    const float zv = to_f(sm.z[tt][pp]);
+                    const float yv = fmaf(s, sm.ys[sb * T + tt][pp], Dc * h);
+                    gdz[t * d + cp] = from_f<Tout>(to_f(sm.dout[tt][pp]) * yv * dsiluf_(zv));
+                }
+                dD_acc = fmaf(dyv, h, dD_acc);
+                if (CONV) {
+                    dpv = dh * dsiluf_(pre);
+                    dw0 = fmaf(dpv, to_f(sm.u[tt][pp]), dw0);
+                    dw1 = fmaf(dpv, to_f(sm.u[tt + 1][pp]), dw1);
+                    dw2 = fmaf(dpv, to_f(sm.u[tt + 2][pp]), dw2);
+                    dw3 = fmaf(dpv, to_f(sm.u[tt + 3][pp]), dw3);
+                    dbias += dpv;
+                } else {
+                    gdhu[t * d + cp] = from_f<Tout>(dh);
+                }
             }
+            if (CONV) sm.dp[tt][pp] = dpv;
         }
-        __syncthreads();
         if (CONV) {
+            __syncthreads();
             // du_t = w3 dp_t + w2 dp_{t+1} + w1 dp_{t+2} + w0 dp_{t+3}
+#pragma unroll
             for (int kk = 0; kk < R; ++kk) {
                 const int tt = rr * R + kk;
                 const int64_t t = t0 + tt;
                 if (cpvalid && t < te) {
                     const float duv = w3 * sm.dp[tt][pp] + w2 * sm.dp[tt + 1][pp] +
                                       w1 * sm.dp[tt + 2][pp] + w0 * sm.dp[tt + 3][pp];
-                    const int64_t e = ((int64_t)bb * L + t) * d + cp;
                     if (!last && t >= te - 3) {
                         edge[(3 + (t - (te - 3))) * d + cp] = duv;  // partial, fixed up later
                     } else {
-                        gdhu[e] = from_f<Tout>(duv);
+                        gdhu[t * d + cp] = from_f<Tout>(duv);
                     }
                     if (sb == 0 && tt < 3) edge[tt * d + cp] = sm.dp[tt][pp];
                 }
@@ -549,8 +572,8 @@ scan_bwd_kernel(const BwdParams p) {
                 sm.dp[T + 2][tid] = sm.dp[2][tid];
             }
         }
-        __syncthreads();
-    }
+    });
+    cluster_reduce(0);
 
     // ------------------------------------------------ carries and partials
     if (last && k > 0) {  // publish the carry leaving the block after the full sweep
@@ -575,8 +598,8 @@ scan_bwd_kernel(const BwdParams p) {
     // Per-channel partial sums (runs of the same channel add through shared atomics).
     {
         float* cpart = p.chan_part + ((int64_t)bb * p.nsub + k) * d * 8;
+        float* red6 = &sm.x1[0][0];  // reuse: [6][P] (T >= 6)
         __syncthreads();
-        float* red6 = &sm.fdf[0][0];  // reuse: [6][P]
         for (int i = tid; i < 6 * P; i += NT) red6[i] = 0.f;
         __syncthreads();
         if (cpvalid) {
@@ -593,26 +616,6 @@ scan_bwd_kernel(const BwdParams p) {
             for (int r = 0; r < 6; ++r) cpart[(c0 + tid) * 8 + r] = red6[r * P + tid];
         }
     }
-    // Cluster reduction of the dB / dC partials of this block.
-    cluster.sync();
-    {
-        constexpr int ROWS = K / kCluster;
-        const int r0 = crank * ROWS;
-        float* out = p.dBCp + (((int64_t)cgi * Bt + bb) * L) * 2 * N;
-        for (int e = tid; e < ROWS * 2 * N; e += NT) {
-            const int tt = r0 + e / (2 * N);
-            const int rem = e % (2 * N);
-            float acc = 0.f;
-#pragma unroll
-            for (int qr = 0; qr < kCluster; ++qr) {
-                const float* rem_acc = cluster.map_shared_rank(&sm.acc[0][0][0], qr);
-                acc += rem_acc[tt * 2 * N + rem];
-            }
-            const int64_t t = tb + tt;
-            if (t < te) out[t * 2 * N + rem] = acc;
-        }
-    }
-    cluster.sync();
 }
 
 // Sum the cluster partials of dB, dC and write them in the output dtype.
@@ -683,7 +686,7 @@ static cudaError_t launch_bwd_t(const BwdParams& p, void* dB, void* dC, float* d
                                 float* dbias, cudaStream_t st) {
     constexpr int S = BwdShape<N>::S;
     constexpr int P = 128 / S;
-    const size_t smem = sizeof(BwdSmem<N, P>);
+    const size_t smem = sizeof(BwdSmem<Tin, N, P>);
     auto kern = scan_bwd_kernel<Tin, Tout, N, CONV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);

@@ -10,16 +10,18 @@
 // Work decomposition.  A thread block owns P channels of one batch element
 // and one group of consecutive checkpoint segments.  Each channel's d_state
 // row is split over S threads that keep NS state entries in registers.  The
-// sequence is streamed in chunks of T tokens: the block first computes the
-// per-(token, channel) scalars of the chunk into shared memory (conv, gates,
-// feedthrough, modulation), then every thread advances its state slice token
-// by token, and the chunk's outputs are written back coalesced.
+// sequence is streamed in chunks of T tokens through a double-buffered
+// shared-memory stage filled by cp.async (the next chunk's raw rows are in
+// flight while the current chunk is scanned).  Per chunk the block first
+// computes the per-(token, channel) scalars (conv, gates) into shared memory,
+// then every thread advances its state slice token by token, and the
+// chunk's outputs are written back coalesced.
 //
 // Rescaled state.  Each thread keeps xs = x * Q with Q = prod 1/f since the
 // last renormalisation, so one token costs one FMA for the write
-// (xs += (i h Q) B) and one FMA for the readout (y = (xs . C) / Q).  Q only
-// grows (1/f = 1 + e^{-a} >= 1); when it would pass 2^64 in any lane of a
-// warp, the warp folds Q back into its states.
+// (xs += (i h Q) B) and one FMA for the readout (y = (xs . C) / Q); both run
+// as packed two-wide FP32 FMAs.  Q only grows (1/f = 1 + e^{-a} >= 1); when it
+// would pass 2^64 in any lane of a warp, the warp folds Q back into its states.
 //
 // Sequence groups.  When batch x channel tiles alone do not fill the GPU,
 // the sequence is split into G groups handled by different blocks.  A block
@@ -36,8 +38,25 @@ namespace naju {
 
 constexpr float kRenorm = 18446744073709551616.0f;  // 2^64
 
+template <typename Tin, int P, int N>
+struct FwdRaw {
+    static constexpr int T = kFwdChunk;
+    Tin u[T + 3][P];   // rows t0-3 .. t0+T-1 (conv input, or h in rows 3..)
+    Tin a[T][P], b[T][P], z[T][P];
+    Tin Bm[T][N], Cm[T][N];
+};
+
+template <typename Tin, int P, int N>
+struct FwdSmem {
+    static constexpr int T = kFwdChunk;
+    FwdRaw<Tin, P, N> raw[2];
+    float sB[T][N], sC[T][N];
+    float sQ[T][P], sF[T][P], sV[T][P], sH[T][P], sY[T][P];
+    int item, ok;
+};
+
 template <typename Tin, typename Tout, int NS, int S, bool CONV>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 4)
 scan_fwd_kernel(const FwdParams p) {
     constexpr int NT = 128;
     constexpr int P = NT / S;        // channels per block
@@ -45,27 +64,18 @@ scan_fwd_kernel(const FwdParams p) {
     constexpr int T = kFwdChunk;     // tokens per chunk
     constexpr int R = T / S;         // tokens per prep run (NT / P = S runs)
     static_assert(NS % 4 == 0 && T % S == 0, "tile shape");
-
+    using Sm = FwdSmem<Tin, P, N>;
     extern __shared__ float4 smem4[];
-    float* sm = reinterpret_cast<float*>(smem4);
-    float* sB = sm;                  // [T][N]
-    float* sC = sB + T * N;          // [T][N]
-    float* sQ = sC + T * N;          // [T][P]  1/f
-    float* sF = sQ + T * P;          // [T][P]  f
-    float* sV = sF + T * P;          // [T][P]  i*h
-    float* sHD = sV + T * P;         // [T][P]  D*h
-    float* sG = sHD + T * P;         // [T][P]  SiLU(z) (or 1)
-    float* sY = sG + T * P;          // [T][P]  x.C (unscaled readout)
-    __shared__ int s_item;
+    Sm& sm = *reinterpret_cast<Sm*>(smem4);
 
     const int tid = threadIdx.x;
     const int js = tid % S;
     const int pl = tid / S;
     const int64_t Bt = p.Bt, L = p.L, d = p.d;
 
-    if (tid == 0) s_item = atomicAdd(&p.hdr->fwd_ticket, 1);
+    if (tid == 0) sm.item = atomicAdd(&p.hdr->fwd_ticket, 1);
     __syncthreads();
-    const int item = s_item;
+    const int item = sm.item;
     const int per_g = (int)(Bt * p.ntiles);
     const int g = item / per_g;
     const int bb = (item % per_g) / p.ntiles;
@@ -80,13 +90,15 @@ scan_fwd_kernel(const FwdParams p) {
     const int64_t tend = min64(L, (int64_t)seg1 * p.T_ck);
     const bool last_group = (g == p.ngroups - 1);
 
-    const Tin* hu = static_cast<const Tin*>(p.hu);
-    const Tin* ga = static_cast<const Tin*>(p.a);
-    const Tin* gb = static_cast<const Tin*>(p.b);
-    const Tin* gB = static_cast<const Tin*>(p.B);
-    const Tin* gC = static_cast<const Tin*>(p.C);
-    const Tin* gz = static_cast<const Tin*>(p.z);
-    Tout* gy = static_cast<Tout*>(p.y);
+    const int64_t boff = (int64_t)bb * L;
+    const Tin* hu = static_cast<const Tin*>(p.hu) + boff * d;
+    const Tin* ga = static_cast<const Tin*>(p.a) + boff * d;
+    const Tin* gb = static_cast<const Tin*>(p.b) + boff * d;
+    const Tin* gz = p.z ? static_cast<const Tin*>(p.z) + boff * d : nullptr;
+    const Tin* gB = static_cast<const Tin*>(p.B) + boff * N;
+    const Tin* gC = static_cast<const Tin*>(p.C) + boff * N;
+    Tout* gy = static_cast<Tout*>(p.y) + boff * d;
+    const bool vec = ((d * (int64_t)sizeof(Tin)) % 16) == 0;
 
     // Per-thread prep assignment: channel column pp, token run rr.
     const int pp = tid % P;
@@ -107,66 +119,49 @@ scan_fwd_kernel(const FwdParams p) {
 
     float* ck_b = p.ckpt + (int64_t)bb * (p.nck + 1) * d * N;  // [nck+1][d][N]
 
-    // ------------------------------------------------ chunk staging helpers
-    auto prep_chunk = [&](int64_t t0, bool full) {
-        // B, C rows of the chunk -> fp32 smem (zeros past L).
+    // ------------------------------------------------ chunk staging
+    auto issue = [&](int64_t t0, int buf, bool full) {
+        FwdRaw<Tin, P, N>& r = sm.raw[buf];
+        stage_rows(&r.u[0][0], hu, d, t0 - 3, T + 3, L, c0, P, vec, tid, NT);
+        stage_rows(&r.a[0][0], ga, d, t0, T, tend, c0, P, vec, tid, NT);
+        stage_rows(&r.b[0][0], gb, d, t0, T, tend, c0, P, vec, tid, NT);
+        if (full && gz) stage_rows(&r.z[0][0], gz, d, t0, T, tend, c0, P, vec, tid, NT);
+        stage_rows(&r.Bm[0][0], gB, N, t0, T, tend, 0, N, true, tid, NT);
+        if (full) stage_rows(&r.Cm[0][0], gC, N, t0, T, tend, 0, N, true, tid, NT);
+        cp_async_commit();
+    };
+    auto prep = [&](int64_t t0, int buf, bool full) {
+        const FwdRaw<Tin, P, N>& r = sm.raw[buf];
         for (int e = tid; e < T * N; e += NT) {
-            const int tt = e / N;
-            const int64_t t = t0 + tt;
-            float vb = 0.f, vc = 0.f;
-            if (t < tend) {
-                vb = to_f(gB[((int64_t)bb * L + t) * N + (e % N)]);
-                if (full) vc = to_f(gC[((int64_t)bb * L + t) * N + (e % N)]);
-            }
-            sB[e] = vb;
-            sC[e] = vc;
+            (&sm.sB[0][0])[e] = to_f((&r.Bm[0][0])[e]);
+            if (full) (&sm.sC[0][0])[e] = to_f((&r.Cm[0][0])[e]);
         }
-        // Per-(token, channel) scalars; run rr covers tokens [rr*R, rr*R+R).
-        const int64_t tr = t0 + rr * R;
-        float u0 = 0.f, u1 = 0.f, u2 = 0.f;  // u_{t-3}, u_{t-2}, u_{t-1}
-        if (CONV && cpvalid) {
-            const Tin* col = hu + (int64_t)bb * L * d + cp;
-            if (tr - 3 >= 0 && tr - 3 < L) u0 = to_f(col[(tr - 3) * d]);
-            if (tr - 2 >= 0 && tr - 2 < L) u1 = to_f(col[(tr - 2) * d]);
-            if (tr - 1 >= 0 && tr - 1 < L) u2 = to_f(col[(tr - 1) * d]);
-        }
-#pragma unroll 4
+#pragma unroll
         for (int k = 0; k < R; ++k) {
             const int tt = rr * R + k;
-            const int64_t t = tr + k;
-            float q = 1.f, f = 1.f, v = 0.f, hd = 0.f, gg = 1.f;
+            const int64_t t = t0 + tt;
+            float q = 1.f, f = 1.f, v = 0.f, h = 0.f;
             if (cpvalid && t < tend) {
-                const int64_t e = ((int64_t)bb * L + t) * d + cp;
-                float h;
                 if (CONV) {
-                    const float u3 = to_f(hu[e]);
-                    const float pre = wb + w0 * u0 + w1 * u1 + w2 * u2 + w3 * u3;
+                    const float pre = wb + w0 * to_f(r.u[tt][pp]) + w1 * to_f(r.u[tt + 1][pp]) +
+                                      w2 * to_f(r.u[tt + 2][pp]) + w3 * to_f(r.u[tt + 3][pp]);
                     h = siluf_(pre);
-                    u0 = u1; u1 = u2; u2 = u3;
                 } else {
-                    h = to_f(hu[e]);
+                    h = to_f(r.u[tt + 3][pp]);
                 }
-                const float ea = __expf(-to_f(ga[e]));
-                q = 1.f + ea;
-                f = 1.f / q;
-                v = sigmoidf_(to_f(gb[e])) * h;
-                if (full) {
-                    hd = Dc * h;
-                    if (gz) gg = siluf_(to_f(gz[e]));
-                }
+                q = 1.f + __expf(-to_f(r.a[tt][pp]));
+                f = rcpf_(q);
+                v = sigmoidf_(to_f(r.b[tt][pp])) * h;
             }
-            sQ[tt * P + pp] = q;
-            sF[tt * P + pp] = f;
-            sV[tt * P + pp] = v;
-            if (full) {
-                sHD[tt * P + pp] = hd;
-                sG[tt * P + pp] = gg;
-            }
+            sm.sQ[tt][pp] = q;
+            sm.sF[tt][pp] = f;
+            sm.sV[tt][pp] = v;
+            sm.sH[tt][pp] = h;
         }
     };
 
     // ------------------------------------------------------- state in regs
-    float xs[NS];
+    float2 xs[NS / 2];
     float Q = 1.f, invQ = 1.f;      // x = xs * invQ; Q ~ 1/invQ
     float logPf = 0.f;              // log of prod f folded by renormalisation
 
@@ -178,8 +173,8 @@ scan_fwd_kernel(const FwdParams p) {
                 const float4* s4 = reinterpret_cast<const float4*>(src + c * N) + m * S + js;
                 v4 = cg ? __ldcg(s4) : *s4;
             }
-            xs[4 * m + 0] = v4.x; xs[4 * m + 1] = v4.y;
-            xs[4 * m + 2] = v4.z; xs[4 * m + 3] = v4.w;
+            xs[2 * m] = make_float2(v4.x, v4.y);
+            xs[2 * m + 1] = make_float2(v4.z, v4.w);
         }
         Q = 1.f; invQ = 1.f; logPf = 0.f;
     };
@@ -187,63 +182,103 @@ scan_fwd_kernel(const FwdParams p) {
         if (!cvalid) return;
 #pragma unroll
         for (int m = 0; m < NS / 4; ++m) {
-            float4 v4 = make_float4(xs[4 * m] * invQ, xs[4 * m + 1] * invQ,
-                                    xs[4 * m + 2] * invQ, xs[4 * m + 3] * invQ);
+            float4 v4 = make_float4(xs[2 * m].x * invQ, xs[2 * m].y * invQ,
+                                    xs[2 * m + 1].x * invQ, xs[2 * m + 1].y * invQ);
             reinterpret_cast<float4*>(dst + c * N)[m * S + js] = v4;
         }
     };
 
     // One token of the recurrence for this thread's state slice.  Returns the
-    // unscaled readout partial x.C when READ.
+    // readout partial x.C (true scale) when READ.
     auto step = [&](int tt, bool READ) -> float {
-        const float q = sQ[tt * P + pl];
-        const float f = sF[tt * P + pl];
-        const float v = sV[tt * P + pl];
+        const float q = sm.sQ[tt][pl];
+        const float f = sm.sF[tt][pl];
+        const float v = sm.sV[tt][pl];
         float Qn = Q * q;
         float iQn = invQ * f;
-        const bool need = !(Qn <= kRenorm);
-        if (__any_sync(0xffffffffu, need)) {
+        if (__any_sync(0xffffffffu, !(Qn <= kRenorm))) {
             // Fold: xs <- x_{t-1} * f_t, i.e. xs * invQ * f.
             logPf += __logf(iQn);
+            const float2 s2 = make_float2(iQn, iQn);
 #pragma unroll
-            for (int j = 0; j < NS; ++j) xs[j] *= iQn;
+            for (int j = 0; j < NS / 2; ++j) xs[j] = __fmul2_rn(xs[j], s2);
             Qn = 1.f;
             iQn = 1.f;
         }
         Q = Qn;
         invQ = iQn;
         const float wv = v * Q;
-        const float4* b4 = reinterpret_cast<const float4*>(sB + tt * N);
-        const float4* c4 = reinterpret_cast<const float4*>(sC + tt * N);
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        const float2 w2v = make_float2(wv, wv);
+        const float4* b4 = reinterpret_cast<const float4*>(sm.sB[tt]);
+        const float4* c4 = reinterpret_cast<const float4*>(sm.sC[tt]);
+        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int m = 0; m < NS / 4; ++m) {
             const float4 bv = b4[m * S + js];
-            xs[4 * m + 0] = fmaf(wv, bv.x, xs[4 * m + 0]);
-            xs[4 * m + 1] = fmaf(wv, bv.y, xs[4 * m + 1]);
-            xs[4 * m + 2] = fmaf(wv, bv.z, xs[4 * m + 2]);
-            xs[4 * m + 3] = fmaf(wv, bv.w, xs[4 * m + 3]);
+            xs[2 * m] = __ffma2_rn(w2v, make_float2(bv.x, bv.y), xs[2 * m]);
+            xs[2 * m + 1] = __ffma2_rn(w2v, make_float2(bv.z, bv.w), xs[2 * m + 1]);
             if (READ) {
                 const float4 cv = c4[m * S + js];
-                a0 = fmaf(xs[4 * m + 0], cv.x, a0);
-                a1 = fmaf(xs[4 * m + 1], cv.y, a1);
-                a2 = fmaf(xs[4 * m + 2], cv.z, a2);
-                a3 = fmaf(xs[4 * m + 3], cv.w, a3);
+                a0 = __ffma2_rn(xs[2 * m], make_float2(cv.x, cv.y), a0);
+                a1 = __ffma2_rn(xs[2 * m + 1], make_float2(cv.z, cv.w), a1);
             }
         }
-        return (a0 + a1) + (a2 + a3);
+        return ((a0.x + a0.y) + (a1.x + a1.y)) * invQ;
+    };
+
+    // One pass over the group's chunks: FULL = readout, outputs, checkpoints.
+    auto run_pass = [&](bool full) {
+        const int nch = (int)((tend - tbeg + T - 1) / T);
+        issue(tbeg, 0, full);
+        const float scale = p.scale;
+        for (int k = 0; k < nch; ++k) {
+            const int buf = k & 1;
+            const int64_t t0 = tbeg + (int64_t)k * T;
+            if (k + 1 < nch) {
+                issue(t0 + T, buf ^ 1, full);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncthreads();
+            prep(t0, buf, full);
+            __syncthreads();
+            if (full) {
+                for (int tt = 0; tt < T; ++tt) {
+                    float part = step(tt, true);
+#pragma unroll
+                    for (int o = 1; o < S; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                    if (js == 0) sm.sY[tt][pl] = part;
+                }
+                const int64_t tnext = t0 + T;
+                if (tnext < tend && tnext % p.T_ck == 0)
+                    store_state(ck_b + (tnext / p.T_ck) * d * N);
+            } else {
+                for (int tt = 0; tt < T; ++tt) step(tt, false);
+            }
+            __syncthreads();
+            if (full && cpvalid) {
+                const FwdRaw<Tin, P, N>& r = sm.raw[buf];
+#pragma unroll
+                for (int kk = 0; kk < R; ++kk) {
+                    const int tt = rr * R + kk;
+                    const int64_t t = t0 + tt;
+                    if (t < tend) {
+                        float yv = fmaf(scale, sm.sY[tt][pp], Dc * sm.sH[tt][pp]);
+                        if (gz) yv *= siluf_(to_f(r.z[tt][pp]));
+                        gy[t * d + cp] = from_f<Tout>(yv);
+                    }
+                }
+            }
+            __syncthreads();
+        }
     };
 
     // --------------------------------------------- local pass (groups > 0)
     const bool do_local = (g > 0) && !last_group;
     if (do_local) {
         load_state(nullptr, false);
-        for (int64_t t0 = tbeg; t0 < tend; t0 += T) {
-            prep_chunk(t0, false);
-            __syncthreads();
-            for (int tt = 0; tt < T; ++tt) step(tt, false);
-            __syncthreads();
-        }
+        run_pass(false);
     }
     // Local end state (zero start) and log prod f of the group.
     const float logPf_loc = logPf + __logf(invQ);
@@ -254,22 +289,22 @@ scan_fwd_kernel(const FwdParams p) {
     int* flag_mine = p.flags + ((int64_t)g * Bt + bb) * p.ntiles + tile;
     float* ck_start = ck_b + (int64_t)seg0 * d * N;
     float* ck_end = ck_b + (int64_t)seg1 * d * N;
-    __shared__ int s_ok;
     if (g > 0) {
-        if (tid == 0) s_ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
+        if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
         __syncthreads();
+        const bool ok = sm.ok != 0;
         if (do_local) {
             // X_end = prod f * X_start + local state.
             const float Pf = __expf(logPf_loc);
 #pragma unroll
             for (int m = 0; m < NS / 4; ++m) {
                 float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (s_ok && cvalid)
+                if (ok && cvalid)
                     v4 = __ldcg(reinterpret_cast<const float4*>(ck_start + c * N) + m * S + js);
-                xs[4 * m + 0] = fmaf(Pf, v4.x, xs[4 * m + 0] * invQ);
-                xs[4 * m + 1] = fmaf(Pf, v4.y, xs[4 * m + 1] * invQ);
-                xs[4 * m + 2] = fmaf(Pf, v4.z, xs[4 * m + 2] * invQ);
-                xs[4 * m + 3] = fmaf(Pf, v4.w, xs[4 * m + 3] * invQ);
+                xs[2 * m].x = fmaf(Pf, v4.x, xs[2 * m].x * invQ);
+                xs[2 * m].y = fmaf(Pf, v4.y, xs[2 * m].y * invQ);
+                xs[2 * m + 1].x = fmaf(Pf, v4.z, xs[2 * m + 1].x * invQ);
+                xs[2 * m + 1].y = fmaf(Pf, v4.w, xs[2 * m + 1].y * invQ);
             }
             invQ = 1.f;
             store_state(ck_end);
@@ -277,40 +312,14 @@ scan_fwd_kernel(const FwdParams p) {
             __syncthreads();
             if (tid == 0) st_release(flag_mine, 1);
         }
-        load_state(s_ok ? ck_start : nullptr, true);
+        load_state(ok ? ck_start : nullptr, true);
     } else {
         load_state(p.x0 ? p.x0 + (int64_t)bb * d * N : nullptr, false);
         store_state(ck_b);  // checkpoint 0 = initial state
     }
 
     // ------------------------------------------------------- full pass
-    const float scale = p.scale;
-    for (int64_t t0 = tbeg; t0 < tend; t0 += T) {
-        prep_chunk(t0, true);
-        __syncthreads();
-        for (int tt = 0; tt < T; ++tt) {
-            float part = step(tt, true);
-#pragma unroll
-            for (int o = 1; o < S; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-            if (js == 0) sY[tt * P + pl] = part * invQ;
-        }
-        // Interior checkpoints at segment boundaries inside this group.
-        const int64_t tnext = t0 + T;
-        if (tnext < tend && tnext % p.T_ck == 0) store_state(ck_b + (tnext / p.T_ck) * d * N);
-        __syncthreads();
-        // Epilogue: out = (scale * x.C + D h) * SiLU(z), coalesced over channels.
-        if (cpvalid) {
-            for (int k = 0; k < R; ++k) {
-                const int tt = rr * R + k;
-                const int64_t t = t0 + tt;
-                if (t < tend) {
-                    const float yv = fmaf(scale, sY[tt * P + pp], sHD[tt * P + pp]);
-                    gy[((int64_t)bb * L + t) * d + cp] = from_f<Tout>(yv * sG[tt * P + pp]);
-                }
-            }
-        }
-        __syncthreads();
-    }
+    run_pass(true);
 
     // -------------------------------------------------- group end state
     if (g == 0 && p.ngroups > 1) {
@@ -329,8 +338,7 @@ template <typename Tin, typename Tout, int NS, int S, bool CONV>
 static cudaError_t launch_fwd_t(const FwdParams& p, cudaStream_t st) {
     constexpr int P = 128 / S;
     constexpr int N = NS * S;
-    constexpr int T = kFwdChunk;
-    const size_t smem = sizeof(float) * (2 * T * N + 6 * T * P);
+    const size_t smem = sizeof(FwdSmem<Tin, P, N>);
     auto kern = scan_fwd_kernel<Tin, Tout, NS, S, CONV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -344,7 +352,7 @@ template <typename Tin, typename Tout, bool CONV>
 static cudaError_t launch_fwd_n(const FwdParams& p, cudaStream_t st) {
     switch (p.N) {
         case 16: return launch_fwd_t<Tin, Tout, 16, 1, CONV>(p, st);
-        case 32: return launch_fwd_t<Tin, Tout, 32, 1, CONV>(p, st);
+        case 32: return launch_fwd_t<Tin, Tout, 16, 2, CONV>(p, st);
         case 64: return launch_fwd_t<Tin, Tout, 32, 2, CONV>(p, st);
         case 128: return launch_fwd_t<Tin, Tout, 32, 4, CONV>(p, st);
         default: return cudaErrorInvalidValue;
@@ -352,7 +360,7 @@ static cudaError_t launch_fwd_n(const FwdParams& p, cudaStream_t st) {
 }
 
 int fwd_channels_per_block(int64_t N) {
-    return N <= 32 ? 128 : (N == 64 ? 64 : 32);
+    return N == 16 ? 128 : (N <= 64 ? 64 : 32);
 }
 
 cudaError_t launch_scan_fwd(const FwdParams& p, int dtype, int out_dtype, cudaStream_t st) {

@@ -105,6 +105,27 @@ naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* co
                           void* y, float* x_final, void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* Allocation-free forward for callers that cannot allocate device memory
+ * (for example code running where no allocator is available, or a plugin
+ * that is handed only its input and output buffers).  The Naju pages have no
+ * counterpart: this is a library convenience.  Same arguments and results as
+ * naju_scan_fwd (y, optional x_final), but no workspace: the scratch is a
+ * fixed 32 MiB device array inside the library, reserved on every GPU that
+ * loads the library until the process exits.  The whole sequence runs as one
+ * group, so the scratch holds only a work ticket, per-tile flags and the
+ * start and end states: problems needing more than 32 MiB (about
+ * batch * d_inner * d_state * 8 bytes) return NAJU_ERR_UNSUPPORTED before any
+ * launch.  It writes no checkpoints, so naju_scan_bwd cannot follow it.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call shares the one array, and each call clears what must start at
+ * zero; calls that may overlap on the GPU (other streams, other threads) race
+ * on it and must be serialised by the caller. */
+naju_status naju_scan_fwd_noalloc(const naju_dims* dims, const void* hu, const float* conv_w,
+                                  const float* conv_b, const void* a, const void* b,
+                                  const void* B, const void* C, const void* z, const float* D,
+                                  const float* x0, void* y, float* x_final, void* stream);
+
 /* Backward of naju_scan_fwd for a loss with gradient dy w.r.t. y and,
  * optionally, dx_final w.r.t. x_final.  Same inputs as the forward; the
  * workspace must hold that forward's checkpoints.  Writes dhu (du in fused

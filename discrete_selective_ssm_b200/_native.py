@@ -77,6 +77,9 @@ def lib(build_if_missing: bool = True):
             L.naju_testing_set_fwd_groups.argtypes = [i32]
             L.naju_testing_fwd_groups.argtypes = [vp]
             L.naju_testing_fwd_groups.restype = i32
+            L.naju_testing_set_bwd_groups.argtypes = [i32]
+            L.naju_testing_bwd_groups.argtypes = [vp]
+            L.naju_testing_bwd_groups.restype = i32
             for name in ("naju_conv_silu_fwd", "naju_conv_silu_bwd", "naju_scan_fwd",
                          "naju_scan_bwd", "naju_scan_step", "naju_last_device_status"):
                 getattr(L, name).restype = ctypes.c_int
@@ -272,3 +275,11 @@ def testing_set_fwd_groups(groups: int):
 
 def testing_fwd_groups(dims: Dims) -> int:
     return int(lib().naju_testing_fwd_groups(ctypes.byref(dims)))
+
+
+def testing_set_bwd_groups(groups: int):
+    lib().naju_testing_set_bwd_groups(int(groups))
+
+
+def testing_bwd_groups(dims: Dims) -> int:
+    return int(lib().naju_testing_bwd_groups(ctypes.byref(dims)))

@@ -15,12 +15,13 @@ using namespace naju;
 namespace {
 
 constexpr int kSMs = 148;
-constexpr int kTck = 128;          // tokens per forward checkpoint segment
+constexpr int kTck = kBwdSub;      // tokens per forward checkpoint segment (= backward block)
 constexpr long long kDefaultWait = 1LL << 21;
 
 long long g_wait_limit = kDefaultWait;
 int g_skip_publish = 0;
 int g_fwd_groups = 0;
+int g_bwd_groups = 0;
 
 inline bool aligned(const void* ptr, size_t a) {
     return (reinterpret_cast<uintptr_t>(ptr) % a) == 0;
@@ -46,7 +47,7 @@ naju_status check_dims(const naju_dims* dm) {
 // Workspace layout (every region 256-byte aligned).
 struct Layout {
     int nck, ngroups, seg_per_group, ntiles_f;
-    int nsub, nclus, ntiles_b;
+    int nsub, nclus, ntiles_b, bgroups, blk_per_group;
     size_t off_fflags, off_bflags, off_ckpt, off_carry, off_dbc, off_chan, off_edge, total;
 };
 
@@ -71,21 +72,33 @@ Layout layout(const naju_dims* dm) {
     const int tiles_b = (int)cdiv(d, bwd_channels_per_block(N));
     l.nclus = (int)cdiv(tiles_b, bwd_cluster_size());
     l.ntiles_b = l.nclus * bwd_cluster_size();
+    {
+        // Backward blocks hold ~111 KB of shared memory: two per SM.
+        int gb = g_bwd_groups;
+        if (gb <= 0) {
+            const int64_t ctas = Bt * (int64_t)l.ntiles_b;
+            const int64_t want = 4 * kSMs;
+            gb = ctas >= want ? 1 : (int)cdiv(want, ctas);
+        }
+        if (gb > l.nsub) gb = l.nsub;
+        l.blk_per_group = (int)cdiv(l.nsub, gb);
+        l.bgroups = (int)cdiv(l.nsub, l.blk_per_group);
+    }
     size_t off = sizeof(WsHeader);
     l.off_fflags = off;
     off = up256(off + sizeof(int) * (size_t)l.ngroups * Bt * l.ntiles_f);
     l.off_bflags = off;
-    off = up256(off + sizeof(int) * (size_t)l.nsub * Bt * l.ntiles_b);
+    off = up256(off + sizeof(int) * (size_t)l.bgroups * Bt * l.ntiles_b);
     l.off_ckpt = off;
     off = up256(off + sizeof(float) * (size_t)Bt * (l.nck + 1) * d * N);
     l.off_carry = off;
-    off = up256(off + sizeof(float) * (size_t)l.nsub * Bt * d * N);
+    off = up256(off + sizeof(float) * (size_t)l.bgroups * Bt * d * N);
     l.off_dbc = off;
     off = up256(off + sizeof(float) * (size_t)l.nclus * Bt * L * 2 * N);
     l.off_chan = off;
-    off = up256(off + sizeof(float) * (size_t)Bt * l.nsub * d * 8);
+    off = up256(off + sizeof(float) * (size_t)Bt * l.bgroups * d * 8);
     l.off_edge = off;
-    off = up256(off + sizeof(float) * (size_t)Bt * l.nsub * 2 * 3 * d);
+    off = up256(off + sizeof(float) * (size_t)Bt * l.bgroups * 2 * 3 * d);
     l.total = off;
     return l;
 }
@@ -189,15 +202,15 @@ naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* co
     NAJU_REQUIRE(workspace && aligned(workspace, 256));
     const Layout l = layout(dims);
     NAJU_REQUIRE(workspace_bytes >= l.total);
-    NAJU_REQUIRE((int64_t)l.nsub * dims->batch * l.ntiles_b < (1LL << 31));
-    NAJU_REQUIRE(l.nsub <= 65535 && dims->batch <= 65535);
+    NAJU_REQUIRE((int64_t)l.bgroups * dims->batch * l.ntiles_b < (1LL << 31));
+    NAJU_REQUIRE(l.bgroups <= 65535 && dims->batch <= 65535);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     char* ws = static_cast<char*>(workspace);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     cudaError_t e = cudaMemsetAsync(&hdr->bwd_ticket, 0, sizeof(int), s);
     if (e == cudaSuccess)
         e = cudaMemsetAsync(ws + l.off_bflags, 0,
-                            sizeof(int) * (size_t)l.nsub * dims->batch * l.ntiles_b, s);
+                            sizeof(int) * (size_t)l.bgroups * dims->batch * l.ntiles_b, s);
     if (e != cudaSuccess) return NAJU_ERR_CUDA;
     BwdParams p{};
     p.hu = hu; p.conv_w = conv_w; p.conv_b = conv_b; p.a = a; p.b = b; p.B = B; p.C = C;
@@ -212,6 +225,7 @@ naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* co
     p.hdr = hdr;
     p.Bt = dims->batch; p.L = dims->seqlen; p.d = dims->d_inner; p.N = dims->d_state;
     p.T_ck = kTck; p.nck = l.nck; p.nsub = l.nsub; p.ntiles = l.ntiles_b; p.nclus = l.nclus;
+    p.blk_per_group = l.blk_per_group; p.ngroups = l.bgroups;
     p.scale = 1.0f / std::sqrt((float)dims->d_state);
     p.wait_limit = g_wait_limit;
     p.fault_skip_publish = g_skip_publish;
@@ -262,6 +276,12 @@ void naju_testing_set_wait_limit(int64_t polls) {
 }
 void naju_testing_set_skip_publish(int32_t skip) { g_skip_publish = skip ? 1 : 0; }
 void naju_testing_set_fwd_groups(int32_t groups) { g_fwd_groups = groups > 0 ? groups : 0; }
+void naju_testing_set_bwd_groups(int32_t groups) { g_bwd_groups = groups > 0 ? groups : 0; }
+int32_t naju_testing_bwd_groups(const void* dims) {
+    const naju_dims* dm = static_cast<const naju_dims*>(dims);
+    if (check_dims(dm) != NAJU_OK) return 0;
+    return layout(dm).bgroups;
+}
 int32_t naju_testing_fwd_groups(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);
     if (check_dims(dm) != NAJU_OK) return 0;

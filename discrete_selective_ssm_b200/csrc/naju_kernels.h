@@ -55,16 +55,18 @@ struct BwdParams {
     void* db;
     void* dz;
     float* dx0;
-    const float* ckpt;     // written by the forward
-    float* carry;          // [nsub][Bt][d][N] adjoint carries between items
-    int* flags;            // [nsub][Bt][ntiles]
+    const float* ckpt;     // written by the forward, one state per kBwdSub tokens
+    float* carry;          // [ngroups][Bt][d][N] adjoint carries between groups
+    int* flags;            // [ngroups][Bt][ntiles]
     float* dBCp;           // [nclus][Bt][L][2][N] partial dB, dC over channel clusters
-    float* chan_part;      // [Bt*nsub][d][8] partial dD, dconv_w[4], dconv_b
-    float* conv_edge;      // [Bt][nsub][2][3][d]: first 3 dp / last 3 partial du
+    float* chan_part;      // [Bt*ngroups][d][8] partial dD, dconv_w[4], dconv_b
+    float* conv_edge;      // [Bt][ngroups][2][3][d]: first 3 dp / last 3 partial du
     WsHeader* hdr;
     int64_t Bt, L, d, N;
-    int T_ck, nck;
-    int nsub;              // ceil(L / kBwdSub)
+    int T_ck, nck;         // forward checkpoint spacing (== kBwdSub) and count
+    int nsub;              // ceil(L / kBwdSub) blocks
+    int blk_per_group;     // blocks per sequence group
+    int ngroups;
     int ntiles;
     int nclus;             // ceil(ntiles / cluster size)
     float scale;

@@ -13,29 +13,36 @@
 //   dB_t   = sum_d G_t[d] i_t[d] h_t[d],   dC_t = s sum_d dy_t[d] x_t[d]
 //   dD     = sum dy h,   dx0 = f_0 G_0,    conv: dp = dh SiLU'(p), du, dw, dbias.
 //
-// Work decomposition.  One work item = (batch b, tile of P channels, block k
-// of 64 tokens).  Items are taken from an atomic ticket from the end of the
-// sequence backwards.  An item:
-//  0. recomputes its start state from the forward's nearest checkpoint;
-//  1. (0 < k < last) runs a local reverse pass with a zero carry to get the
-//     block's own adjoint contribution and decay product;
-//  2. waits (bounded) for item k+1 to publish the adjoint carry entering its
-//     end, publishes the carry leaving its start (decoupled look-back);
-//  3. sweeps forward over 16-token sub-blocks: the state readout (kept for
-//     dz and dL) and, per sub-block, dC as a contraction over the block's
-//     channels: dC_t = s[(dy E)_t X_b + sum_{m<=t} A[t,m] B_m], where X_b is
-//     the state entering the sub-block, E_t the decay since then and
-//     A[t,m] = sum_d dy_t E_t/E_m i_m h_m;
-//  4. sweeps backward: the adjoint G, per-channel gradients, and per
-//     sub-block dB_m = s sum_{t>=m} A[t,m] C_t + (i h F)_m H_e, with H_e the
-//     carry entering the sub-block's end and F_m the decay to that end.
-// Every sub-block's raw inputs are staged by cp.async, and the next
-// sub-block's copy is issued as soon as the current one has been unpacked.
-// dB/dC partial sums over the P channels are summed across the thread-block
-// cluster (consecutive channel tiles) through distributed shared memory and
-// written once per cluster; small kernels then sum clusters, the per-channel
-// partials (dD, dconv) and the conv's block-boundary terms.
+// Work decomposition.  A thread block owns P channels of one batch element
+// and one sequence group of consecutive 64-token blocks; the blocks of a
+// cluster (consecutive channel tiles) share batch element and group.  The
+// group's blocks are walked from the last to the first with the adjoint
+// carry in registers.  For each block:
+//  * the forward checkpoint at the block start gives its initial state;
+//  * a forward sweep over 16-token sub-blocks recomputes the readout
+//    (kept for dz and dL) and forms dC as a contraction over the block's
+//    channels: dC_t = s[(dy E)_t X_b + sum_{m<=t} A[t,m] B_m], with X_b the
+//    state entering the sub-block, E_t the decay since then and
+//    A[t,m] = sum_d dy_t E_t/E_m i_m h_m;
+//  * a backward sweep runs the adjoint, writes the per-channel gradients and
+//    forms dB_m = s sum_{t>=m} A[t,m] C_t + (i h F)_m H_e, with H_e the
+//    carry entering the sub-block's end and F_m the decay to that end.
+// The dB/dC partial sums over each block's channels are summed across the
+// cluster through distributed shared memory and written once per cluster.
+//
+// Sequence groups.  When batch x channel tiles alone do not fill the GPU,
+// the sequence is split into groups.  The carry entering a group's end comes
+// from the next group: every group with a predecessor first runs a cheap
+// reverse pass (adjoint only) - from dx_final for the last group, from a zero
+// carry for the others, which then wait (bounded) for the carry of the next
+// group - and publishes the carry leaving its start before its main work
+// (a decoupled look-back running backwards in time).  Groups are taken from
+// an atomic ticket starting with the last, so every awaited block has started.
+// Small kernels then sum the cluster partials, the per-channel partials
+// (dD, dconv) and the conv's group-boundary terms.
 #include <cooperative_groups.h>
+
+#include <type_traits>
 
 #include "naju_common.cuh"
 #include "naju_kernels.h"
@@ -66,16 +73,16 @@ struct BwdSmem {
     Tin Bm[T][N], Cm[T][N];
     // unpacked per-(token, channel) values
     float f[T][P], q[T][P], v[T][P], dy[T][P];
-    float x1[T][P];   // forward: clamped log-prefix   backward: G . B
-    float x2[T][P];   // forward: dy * decay prefix    backward: i h * decay to end
-    float x3[T][P];   // forward: A factor (dy side)   backward: f df
-    float x4[T][P];   // forward: A factor (i h side)
+    float x1[T][P];       // forward: clamped log-prefix   backward: G . B
+    float x2[T][P + 1];   // forward: dy * decay prefix    backward: i h * decay to end
+    float x3[T][P + 1];   // forward: A factor (dy side)   backward: f df
+    float x4[T][P + 1];   // forward: A factor (i h side)
     float dp[T + 3][P];
-    float ys[K][P];   // unscaled readout x_t . C_t of the block
+    float ys[K][P];       // unscaled readout x_t . C_t of the block
     float Bf[T][N], Cf[T][N];
-    float snap[P][N]; // X_b (forward) or H_e (backward)
+    float snap[P][N];     // X_b (forward) or H_e (backward)
     float A[K / T][T][T];
-    float acc[K][N];  // dC (forward sweep) then dB (backward sweep) partials
+    float acc[K][N];      // dC (forward sweep) then dB (backward sweep) partials
     int item, ok;
 };
 
@@ -102,9 +109,9 @@ scan_bwd_kernel(const BwdParams p) {
     if (crank == 0 && tid == 0) sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
     cluster.sync();
     const int item = *cluster.map_shared_rank(&sm.item, 0);
-    const int per_k = (int)(Bt * p.nclus);
-    const int k = p.nsub - 1 - item / per_k;
-    const int bb = (item % per_k) / p.nclus;
+    const int per_g = (int)(Bt * p.nclus);
+    const int g = p.ngroups - 1 - item / per_g;
+    const int bb = (item % per_g) / p.nclus;
     const int cgi = item % p.nclus;
     const int tile = cgi * kCluster + crank;
     const int64_t c0 = (int64_t)tile * P;
@@ -112,9 +119,12 @@ scan_bwd_kernel(const BwdParams p) {
     const bool cvalid = c < d;
     const int64_t cp = c0 + pp;
     const bool cpvalid = cp < d;
-    const int64_t tb = (int64_t)k * K;
-    const int64_t te = min64(L, tb + K);
-    const bool last = (k == p.nsub - 1);
+    const int kb0 = g * p.blk_per_group;
+    const int kb1 = min(kb0 + p.blk_per_group, p.nsub);
+    const int64_t tg0 = (int64_t)kb0 * K;
+    const int64_t tg1 = min64(L, (int64_t)kb1 * K);
+    const bool lastg = (g == p.ngroups - 1);
+    const bool firstg = (g == 0);
 
     const int64_t boff = (int64_t)bb * L;
     const Tin* hu = static_cast<const Tin*>(p.hu) + boff * d;
@@ -175,7 +185,7 @@ scan_bwd_kernel(const BwdParams p) {
             sm.f[tt][pp] = f; sm.q[tt][pp] = q; sm.v[tt][pp] = v; sm.dy[tt][pp] = dyv;
         }
     };
-    // Sub-block sequence of a pass: sub-block i starts at t0 + dir * i * T.
+    // Sub-block sequence of a pass: sub-block i starts at first + dir * i * T.
     // The raw buffer is refilled with sub-block i+1 right after sub-block i
     // is unpacked unless `late` (the body reads raw rows), in which case the
     // refill follows the body.
@@ -196,12 +206,12 @@ scan_bwd_kernel(const BwdParams p) {
     };
 
     // ----------------------------------------------------- register state
-    float xs[NS], gs[NS];
+    float2 xs[NS / 2], gs[NS / 2];
     float Q = 1.f, iQ = 1.f;   // forward: x = xs * iQ
     float Rr = 1.f, iR = 1.f;  // backward: G = gs * iR
     float logF = 0.f;          // log of decay folded out of the backward state
 
-    auto load_rows = [&](float* dst, const float* src, bool cg_) {
+    auto load_rows = [&](float2* dst, const float* src, bool cg_) {
 #pragma unroll
         for (int m = 0; m < NS / 4; ++m) {
             float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -209,82 +219,136 @@ scan_bwd_kernel(const BwdParams p) {
                 const float4* s4 = reinterpret_cast<const float4*>(src + c * N) + m * S + js;
                 v4 = cg_ ? __ldcg(s4) : *s4;
             }
-            dst[4 * m] = v4.x; dst[4 * m + 1] = v4.y; dst[4 * m + 2] = v4.z; dst[4 * m + 3] = v4.w;
+            dst[2 * m] = make_float2(v4.x, v4.y);
+            dst[2 * m + 1] = make_float2(v4.z, v4.w);
         }
+    };
+    auto store_rows = [&](float* dst, const float2* src, float sc) {
+        if (!cvalid) return;
+#pragma unroll
+        for (int m = 0; m < NS / 4; ++m)
+            reinterpret_cast<float4*>(dst + c * N)[m * S + js] =
+                make_float4(src[2 * m].x * sc, src[2 * m].y * sc, src[2 * m + 1].x * sc,
+                            src[2 * m + 1].y * sc);
+    };
+    auto snap_rows = [&](const float2* src, float sc) {
+        if (cvalid) {
+#pragma unroll
+            for (int m = 0; m < NS / 4; ++m)
+                reinterpret_cast<float4*>(sm.snap[pl])[m * S + js] =
+                    make_float4(src[2 * m].x * sc, src[2 * m].y * sc, src[2 * m + 1].x * sc,
+                                src[2 * m + 1].y * sc);
+        } else {
+#pragma unroll
+            for (int m = 0; m < NS / 4; ++m)
+                reinterpret_cast<float4*>(sm.snap[pl])[m * S + js] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    auto scale_rows = [&](float2* v, float sc) {
+        const float2 s2 = make_float2(sc, sc);
+#pragma unroll
+        for (int j = 0; j < NS / 2; ++j) v[j] = __fmul2_rn(v[j], s2);
     };
     auto red = [&](float v) {
 #pragma unroll
         for (int o = 1; o < S; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         return v;
     };
-    // Forward token: xs <- xs + (v Q) B (rescaled), optional readout.
-    auto fstep = [&](int tt, bool read) -> float {
+    // Forward token: xs <- xs + (v Q) B (rescaled); returns the readout x.C.
+    // CHECK: test Q against the renormalisation bound (slow path only).
+    auto fstep = [&](int tt, auto check) -> float {
         const float qv = sm.q[tt][pl], fv = sm.f[tt][pl], vv = sm.v[tt][pl];
         float Qn = Q * qv, iQn = iQ * fv;
-        if (__any_sync(0xffffffffu, !(Qn <= kRenormB))) {
-#pragma unroll
-            for (int j = 0; j < NS; ++j) xs[j] *= iQn;
-            Qn = 1.f; iQn = 1.f;
+        if constexpr (decltype(check)::value) {
+            if (__any_sync(0xffffffffu, !(Qn <= kRenormB))) {
+                scale_rows(xs, iQn);
+                Qn = 1.f; iQn = 1.f;
+            }
         }
         Q = Qn; iQ = iQn;
         const float wv = vv * Q;
+        const float2 w2v = make_float2(wv, wv);
         const float4* b4 = reinterpret_cast<const float4*>(sm.Bf[tt]);
         const float4* c4 = reinterpret_cast<const float4*>(sm.Cf[tt]);
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        float2 a[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
         for (int m = 0; m < NS / 4; ++m) {
             const float4 bv = b4[m * S + js];
-            xs[4 * m] = fmaf(wv, bv.x, xs[4 * m]);
-            xs[4 * m + 1] = fmaf(wv, bv.y, xs[4 * m + 1]);
-            xs[4 * m + 2] = fmaf(wv, bv.z, xs[4 * m + 2]);
-            xs[4 * m + 3] = fmaf(wv, bv.w, xs[4 * m + 3]);
-            if (read) {
-                const float4 cv = c4[m * S + js];
-                a0 = fmaf(xs[4 * m], cv.x, a0);
-                a1 = fmaf(xs[4 * m + 1], cv.y, a1);
-                a2 = fmaf(xs[4 * m + 2], cv.z, a2);
-                a3 = fmaf(xs[4 * m + 3], cv.w, a3);
-            }
+            const float4 cv = c4[m * S + js];
+            xs[2 * m] = __ffma2_rn(w2v, make_float2(bv.x, bv.y), xs[2 * m]);
+            xs[2 * m + 1] = __ffma2_rn(w2v, make_float2(bv.z, bv.w), xs[2 * m + 1]);
+            a[(2 * m) & 3] = __ffma2_rn(xs[2 * m], make_float2(cv.x, cv.y), a[(2 * m) & 3]);
+            a[(2 * m + 1) & 3] =
+                __ffma2_rn(xs[2 * m + 1], make_float2(cv.z, cv.w), a[(2 * m + 1) & 3]);
         }
-        return ((a0 + a1) + (a2 + a3)) * iQ;
+        const float2 a01 = __fadd2_rn(a[0], a[1]), a23 = __fadd2_rn(a[2], a[3]);
+        return ((a01.x + a01.y) + (a23.x + a23.y)) * iQ;
     };
     // Backward token t (after the carry from t+1 is in gs): G_t = G + s dy C.
     auto bstep = [&](int tt, bool dotB) -> float {
         const float wv = s * sm.dy[tt][pl] * Rr;
+        const float2 w2v = make_float2(wv, wv);
         const float4* b4 = reinterpret_cast<const float4*>(sm.Bf[tt]);
         const float4* c4 = reinterpret_cast<const float4*>(sm.Cf[tt]);
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        float2 a[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
         for (int m = 0; m < NS / 4; ++m) {
             const float4 cv = c4[m * S + js];
-            gs[4 * m] = fmaf(wv, cv.x, gs[4 * m]);
-            gs[4 * m + 1] = fmaf(wv, cv.y, gs[4 * m + 1]);
-            gs[4 * m + 2] = fmaf(wv, cv.z, gs[4 * m + 2]);
-            gs[4 * m + 3] = fmaf(wv, cv.w, gs[4 * m + 3]);
+            gs[2 * m] = __ffma2_rn(w2v, make_float2(cv.x, cv.y), gs[2 * m]);
+            gs[2 * m + 1] = __ffma2_rn(w2v, make_float2(cv.z, cv.w), gs[2 * m + 1]);
             if (dotB) {
                 const float4 bv = b4[m * S + js];
-                a0 = fmaf(gs[4 * m], bv.x, a0);
-                a1 = fmaf(gs[4 * m + 1], bv.y, a1);
-                a2 = fmaf(gs[4 * m + 2], bv.z, a2);
-                a3 = fmaf(gs[4 * m + 3], bv.w, a3);
+                a[(2 * m) & 3] = __ffma2_rn(gs[2 * m], make_float2(bv.x, bv.y), a[(2 * m) & 3]);
+                a[(2 * m + 1) & 3] =
+                    __ffma2_rn(gs[2 * m + 1], make_float2(bv.z, bv.w), a[(2 * m + 1) & 3]);
             }
         }
-        return ((a0 + a1) + (a2 + a3)) * iR;
+        const float2 a01 = __fadd2_rn(a[0], a[1]), a23 = __fadd2_rn(a[2], a[3]);
+        return ((a01.x + a01.y) + (a23.x + a23.y)) * iR;
     };
     // Multiply the backward state by f_t (moving from t to t-1).
-    auto bdecay = [&](int tt) {
+    auto bdecay = [&](int tt, auto check) {
         const float qv = sm.q[tt][pl], fv = sm.f[tt][pl];
         float Rn = Rr * qv, iRn = iR * fv;
-        if (__any_sync(0xffffffffu, !(Rn <= kRenormB))) {
-            logF += __logf(iRn);
-#pragma unroll
-            for (int j = 0; j < NS; ++j) gs[j] *= iRn;
-            Rn = 1.f; iRn = 1.f;
+        if constexpr (decltype(check)::value) {
+            if (__any_sync(0xffffffffu, !(Rn <= kRenormB))) {
+                logF += __logf(iRn);
+                scale_rows(gs, iRn);
+                Rn = 1.f; iRn = 1.f;
+            }
         }
         Rr = Rn; iR = iRn;
     };
+    // Whether the next T tokens can run without renormalisation checks: the
+    // scale (Q forward, R backward) times the sub-block's product of 1/f stays
+    // below the bound in every lane of the warp.  If not, fold the scale into
+    // the state first and test again; if it still fails (a sub-block whose own
+    // decay exceeds 2^64), the caller takes the checked path.
+    auto fast_fwd = [&]() -> bool {
+        float pq = 1.f;
+#pragma unroll
+        for (int tt = 0; tt < T; ++tt) pq *= sm.q[tt][pl];
+        if (!__any_sync(0xffffffffu, !(Q * pq <= kRenormB))) return true;
+        scale_rows(xs, iQ);
+        Q = 1.f; iQ = 1.f;
+        return !__any_sync(0xffffffffu, !(pq <= kRenormB));
+    };
+    auto fast_bwd = [&]() -> bool {
+        float pq = 1.f;
+#pragma unroll
+        for (int tt = 0; tt < T; ++tt) pq *= sm.q[tt][pl];
+        if (!__any_sync(0xffffffffu, !(Rr * pq <= kRenormB))) return true;
+        logF += __logf(iR);
+        scale_rows(gs, iR);
+        Rr = 1.f; iR = 1.f;
+        return !__any_sync(0xffffffffu, !(pq <= kRenormB));
+    };
+    using Checked = std::integral_constant<bool, true>;
+    using Unchecked = std::integral_constant<bool, false>;
     // Cluster sum of acc[K][N] into the dB (slot 0) or dC (slot 1) partials.
-    auto cluster_reduce = [&](int slot) {
+    auto cluster_reduce = [&](int slot, int64_t tb, int64_t te) {
         cluster.sync();
         constexpr int ROWS = K / kCluster;
         const int r0 = crank * ROWS;
@@ -302,302 +366,288 @@ scan_bwd_kernel(const BwdParams p) {
         cluster.sync();
     };
 
-    // --------------------------------------- 0. state entering the block
-    {
-        const int kc = (int)(tb / p.T_ck);
-        const float* ck = p.ckpt + ((int64_t)bb * (p.nck + 1) + kc) * d * N;
-        load_rows(xs, ck, false);
-        Q = 1.f; iQ = 1.f;
-        const int64_t t_ck = (int64_t)kc * p.T_ck;
-        pass(t_ck, (int)((tb - t_ck) / T), +1, tb, false, [&](int, int64_t) {
-            for (int tt = 0; tt < T; ++tt) fstep(tt, false);
-        });
+    // ------------------------------------ carry entering the group's end
+    float2 H[NS / 2];
+    float* carry_in = p.carry + ((int64_t)g * Bt + bb) * d * N;
+    float* carry_out = g > 0 ? p.carry + ((int64_t)(g - 1) * Bt + bb) * d * N : nullptr;
+    int* flag_in = p.flags + ((int64_t)g * Bt + bb) * p.ntiles + tile;
+    int* flag_out = g > 0 ? p.flags + ((int64_t)(g - 1) * Bt + bb) * p.ntiles + tile : nullptr;
+    if (lastg) load_rows(H, p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr, false);
+    if (!firstg) {
+        // Early reverse pass over the group: adjoint only, to publish the carry
+        // leaving the group's start before the main work.
+        if (lastg) {
 #pragma unroll
-        for (int j = 0; j < NS; ++j) xs[j] *= iQ;
-        Q = 1.f; iQ = 1.f;
-    }
-
-    // ------------------------------------- 1. local adjoint contribution
-    const bool local = (k > 0) && !last;
-    if (local) {
+            for (int j = 0; j < NS / 2; ++j) gs[j] = H[j];
+        } else {
 #pragma unroll
-        for (int j = 0; j < NS; ++j) gs[j] = 0.f;
+            for (int j = 0; j < NS / 2; ++j) gs[j] = make_float2(0.f, 0.f);
+        }
         Rr = 1.f; iR = 1.f; logF = 0.f;
-        pass(tb + (NSUB - 1) * T, NSUB, -1, te, false, [&](int, int64_t) {
-            for (int tt = T - 1; tt >= 0; --tt) {
-                bstep(tt, false);
-                bdecay(tt);
+        const int nsb = (int)((tg1 - tg0 + T - 1) / T);
+        pass(tg0 + (int64_t)(nsb - 1) * T, nsb, -1, tg1, false, [&](int, int64_t) {
+            if (fast_bwd()) {
+#pragma unroll 2
+                for (int tt = T - 1; tt >= 0; --tt) {
+                    bstep(tt, false);
+                    bdecay(tt, Unchecked{});
+                }
+            } else {
+                for (int tt = T - 1; tt >= 0; --tt) {
+                    bstep(tt, false);
+                    bdecay(tt, Checked{});
+                }
             }
         });
-    }
-
-    // -------------------------------------------- 2. carry in / publish
-    float* carry_in = p.carry + ((int64_t)k * Bt + bb) * d * N;
-    float* carry_out = k > 0 ? p.carry + ((int64_t)(k - 1) * Bt + bb) * d * N : nullptr;
-    int* flag_in = p.flags + ((int64_t)k * Bt + bb) * p.ntiles + tile;
-    int* flag_out = k > 0 ? p.flags + ((int64_t)(k - 1) * Bt + bb) * p.ntiles + tile : nullptr;
-    float H[NS];
-    {
-        if (!last) {
+        if (!lastg) {
             if (tid == 0) sm.ok = wait_flag(flag_in, &p.hdr->status, p.wait_limit) ? 1 : 0;
             __syncthreads();
             load_rows(H, sm.ok ? carry_in : nullptr, true);
-        } else {
-            load_rows(H, p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr, false);
-        }
-        if (local) {
-            // carry out = decay(block) * H + local contribution.
+            // carry out = decay(group) * H + local contribution
             const float Pf = __expf(logF + __logf(iR));
-            if (cvalid) {
+            const float2 P2 = make_float2(Pf, Pf);
+            const float2 r2 = make_float2(iR, iR);
 #pragma unroll
-                for (int m = 0; m < NS / 4; ++m) {
-                    float4 o4 = make_float4(fmaf(Pf, H[4 * m], gs[4 * m] * iR),
-                                            fmaf(Pf, H[4 * m + 1], gs[4 * m + 1] * iR),
-                                            fmaf(Pf, H[4 * m + 2], gs[4 * m + 2] * iR),
-                                            fmaf(Pf, H[4 * m + 3], gs[4 * m + 3] * iR));
-                    reinterpret_cast<float4*>(carry_out + c * N)[m * S + js] = o4;
-                }
-            }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) st_release(flag_out, 1);
+            for (int j = 0; j < NS / 2; ++j) gs[j] = __ffma2_rn(P2, H[j], __fmul2_rn(gs[j], r2));
+            iR = 1.f;
         }
+        store_rows(carry_out, gs, iR);
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && !(lastg && p.fault_skip_publish)) st_release(flag_out, 1);
+    } else if (!lastg) {
+        if (tid == 0) sm.ok = wait_flag(flag_in, &p.hdr->status, p.wait_limit) ? 1 : 0;
+        __syncthreads();
+        load_rows(H, sm.ok ? carry_in : nullptr, true);
     }
 
-    // ---------------------------------------------- 3. forward sweep
-    pass(tb, NSUB, +1, te, false, [&](int sb, int64_t t0) {
-        // Snapshot of the state entering the sub-block (xs is unscaled here).
-        if (cvalid) {
+    // ------------------------------------------------ main: blocks in reverse
 #pragma unroll
-            for (int m = 0; m < NS / 4; ++m)
-                reinterpret_cast<float4*>(sm.snap[pl])[m * S + js] =
-                    make_float4(xs[4 * m], xs[4 * m + 1], xs[4 * m + 2], xs[4 * m + 3]);
-        } else if (js == 0) {
-            for (int j = 0; j < N; ++j) sm.snap[pl][j] = 0.f;
-        }
-        float lg = 0.f, E = 1.f;
-        for (int tt = 0; tt < T; ++tt) {
-            const float yv = red(fstep(tt, true));
-            const float fv = sm.f[tt][pl];
-            lg += fmaxf(__logf(fv), kLogFloor);
-            E *= fv;
-            if (js == 0) {
-                sm.ys[sb * T + tt][pl] = yv;
-                sm.x1[tt][pl] = lg;
-                sm.x2[tt][pl] = E;
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < NS; ++j) xs[j] *= iQ;
-        Q = 1.f; iQ = 1.f;
-        __syncthreads();
-        // Pivot factors of A around token T/2 of the sub-block.
-        for (int kk = 0; kk < R; ++kk) {
-            const int tt = rr * R + kk;
-            const float piv = sm.x1[T / 2][pp];
-            const float l = sm.x1[tt][pp];
-            sm.x3[tt][pp] = sm.dy[tt][pp] * __expf(l - piv);
-            sm.x4[tt][pp] = sm.v[tt][pp] * __expf(piv - l);
-            sm.x2[tt][pp] *= sm.dy[tt][pp];  // dy_t E_t
-        }
-        __syncthreads();
-        // A[t][m] = sum_p fa[t][p] fb[m][p] for m <= t.
-        for (int e = tid; e < T * T; e += NT) {
-            const int tt = e / T, mm = e % T;
-            float a = 0.f;
-            if (mm <= tt) {
-#pragma unroll 8
-                for (int q2 = 0; q2 < P; ++q2) a = fmaf(sm.x3[tt][q2], sm.x4[mm][q2], a);
-            }
-            sm.A[sb][tt][mm] = a;
-        }
-        __syncthreads();
-        // dC[t][j] = s [ sum_p (dy E)[t][p] X_b[p][j] + sum_{m<=t} A[t][m] B[m][j] ].
-        {
-            constexpr int JB = (N * T) / NT;  // outputs per thread
-            const int tt = tid / (N / JB);
-            const int j0 = (tid % (N / JB)) * JB;
-            float o[JB];
-#pragma unroll
-            for (int r = 0; r < JB; ++r) o[r] = 0.f;
-#pragma unroll 4
-            for (int q2 = 0; q2 < P; ++q2) {
-                const float a = sm.x2[tt][q2];
-#pragma unroll
-                for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.snap[q2][j0 + r], o[r]);
-            }
-            for (int mm = 0; mm <= tt; ++mm) {
-                const float a = sm.A[sb][tt][mm];
-#pragma unroll
-                for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.Bf[mm][j0 + r], o[r]);
-            }
-#pragma unroll
-            for (int r = 0; r < JB; ++r) sm.acc[sb * T + tt][j0 + r] = s * o[r];
-        }
-    });
-    cluster_reduce(1);
-
-    // tail of f df: H . x_end (per channel)
-    float tail = 0.f;
-#pragma unroll
-    for (int j = 0; j < NS; ++j) tail = fmaf(H[j], xs[j], tail);
-    tail = red(tail);
-
-    // ---------------------------------------------- 4. backward sweep
-#pragma unroll
-    for (int j = 0; j < NS; ++j) gs[j] = H[j];
+    for (int j = 0; j < NS / 2; ++j) gs[j] = H[j];
     Rr = 1.f; iR = 1.f; logF = 0.f;
-    float cum = 0.f;  // sum of dL over later tokens of the block
     float dD_acc = 0.f, dw0 = 0.f, dw1 = 0.f, dw2 = 0.f, dw3 = 0.f, dbias = 0.f;
     Tout* gdhu = static_cast<Tout*>(p.dhu) + boff * d;
     Tout* gda = static_cast<Tout*>(p.da) + boff * d;
     Tout* gdb = static_cast<Tout*>(p.db) + boff * d;
     Tout* gdz = p.dz ? static_cast<Tout*>(p.dz) + boff * d : nullptr;
-    float* edge = p.conv_edge + ((int64_t)bb * p.nsub + k) * 2 * 3 * d;
-    if (tid < P) {  // dp beyond the block: zero (next block's terms go via the edge fixup)
+    float* edge = p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d;
+    if (tid < P) {  // dp beyond the group: zero (the next group's terms go via the edge fixup)
         sm.dp[T][tid] = 0.f; sm.dp[T + 1][tid] = 0.f; sm.dp[T + 2][tid] = 0.f;
     }
-    pass(tb + (NSUB - 1) * T, NSUB, -1, te, true, [&](int i, int64_t t0) {
-        const int sb = NSUB - 1 - i;
-        // H_e: carry entering the sub-block's end, true scale.
-        if (cvalid) {
-#pragma unroll
-            for (int m = 0; m < NS / 4; ++m)
-                reinterpret_cast<float4*>(sm.snap[pl])[m * S + js] =
-                    make_float4(gs[4 * m] * iR, gs[4 * m + 1] * iR, gs[4 * m + 2] * iR,
-                                gs[4 * m + 3] * iR);
-        } else if (js == 0) {
-            for (int j = 0; j < N; ++j) sm.snap[pl][j] = 0.f;
-        }
-        float F = 1.f;  // prod f_{m+1..end of sub-block}
-        for (int tt = T - 1; tt >= 0; --tt) {
-            const float gbv = red(bstep(tt, true));
-            const float vv = sm.v[tt][pl];
-            const float dL = s * sm.dy[tt][pl] * sm.ys[sb * T + tt][pl] - vv * gbv;
-            cum += dL;
-            if (js == 0) {
-                sm.x1[tt][pl] = gbv;
-                sm.x3[tt][pl] = cum + tail;
-                sm.x2[tt][pl] = vv * F;  // (i h F)_m
-            }
-            F *= sm.f[tt][pl];
-            bdecay(tt);
-        }
-        __syncthreads();
-        // dB[m][j] = sum_p (i h F)[m][p] H_e[p][j] + s sum_{t>=m} A[t][m] C[t][j].
-        {
-            constexpr int JB = (N * T) / NT;
-            const int mm = tid / (N / JB);
-            const int j0 = (tid % (N / JB)) * JB;
-            float o[JB], o2[JB];
-#pragma unroll
-            for (int r = 0; r < JB; ++r) { o[r] = 0.f; o2[r] = 0.f; }
-#pragma unroll 4
-            for (int q2 = 0; q2 < P; ++q2) {
-                const float a = sm.x2[mm][q2];
-#pragma unroll
-                for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.snap[q2][j0 + r], o[r]);
-            }
-            for (int tt = mm; tt < T; ++tt) {
-                const float a = sm.A[sb][tt][mm];
-#pragma unroll
-                for (int r = 0; r < JB; ++r) o2[r] = fmaf(a, sm.Cf[tt][j0 + r], o2[r]);
-            }
-#pragma unroll
-            for (int r = 0; r < JB; ++r) sm.acc[sb * T + mm][j0 + r] = fmaf(s, o2[r], o[r]);
-        }
-        // Per-channel gradients of the sub-block (thread pp, run rr).
-#pragma unroll
-        for (int kk = 0; kk < R; ++kk) {
-            const int tt = rr * R + kk;
-            const int64_t t = t0 + tt;
-            float dpv = 0.f;
-            if (cpvalid && t < te) {
-                float h, pre = 0.f;
-                if (CONV) {
-                    pre = wb + w0 * to_f(sm.u[tt][pp]) + w1 * to_f(sm.u[tt + 1][pp]) +
-                          w2 * to_f(sm.u[tt + 2][pp]) + w3 * to_f(sm.u[tt + 3][pp]);
-                    h = siluf_(pre);
-                } else {
-                    h = to_f(sm.u[tt + 3][pp]);
+    for (int k = kb1 - 1; k >= kb0; --k) {
+        const int64_t tb = (int64_t)k * K;
+        const int64_t te = min64(L, tb + K);
+        // carry entering this block's end, true scale (gs is unchanged by the
+        // forward sweep and serves as H in the tail below)
+        scale_rows(gs, iR);
+        Rr = 1.f; iR = 1.f;
+        // state entering the block
+        load_rows(xs, p.ckpt + ((int64_t)bb * (p.nck + 1) + k) * d * N, false);
+        Q = 1.f; iQ = 1.f;
+
+        // --------------------------------------------- forward sweep
+        pass(tb, NSUB, +1, te, false, [&](int sb, int64_t) {
+            snap_rows(xs, 1.f);  // state entering the sub-block (xs unscaled here)
+            float lg = 0.f, E = 1.f;
+            auto tok = [&](int tt, auto check) {
+                const float yv = red(fstep(tt, check));
+                const float fv = sm.f[tt][pl];
+                lg += fmaxf(__logf(fv), kLogFloor);
+                E *= fv;
+                if (js == 0) {
+                    sm.ys[sb * T + tt][pl] = yv;
+                    sm.x1[tt][pl] = lg;
+                    sm.x2[tt][pl] = E;
                 }
-                const float fv = sm.f[tt][pp];
-                const float iv = sigmoidf_(to_f(sm.b[tt][pp]));
-                const float gbv = sm.x1[tt][pp];
-                const float dyv = sm.dy[tt][pp];
-                const float dh = Dc * dyv + iv * gbv;
-                gda[t * d + cp] = from_f<Tout>(sm.x3[tt][pp] * (1.f - fv));
-                gdb[t * d + cp] = from_f<Tout>(h * gbv * iv * (1.f - iv));
-                if (gz) {
-                    const float zv = to_f(sm.z[tt][pp]);
-                    const float yv = fmaf(s, sm.ys[sb * T + tt][pp], Dc * h);
-                    gdz[t * d + cp] = from_f<Tout>(to_f(sm.dout[tt][pp]) * yv * dsiluf_(zv));
-                }
-                dD_acc = fmaf(dyv, h, dD_acc);
-                if (CONV) {
-                    dpv = dh * dsiluf_(pre);
-                    dw0 = fmaf(dpv, to_f(sm.u[tt][pp]), dw0);
-                    dw1 = fmaf(dpv, to_f(sm.u[tt + 1][pp]), dw1);
-                    dw2 = fmaf(dpv, to_f(sm.u[tt + 2][pp]), dw2);
-                    dw3 = fmaf(dpv, to_f(sm.u[tt + 3][pp]), dw3);
-                    dbias += dpv;
-                } else {
-                    gdhu[t * d + cp] = from_f<Tout>(dh);
-                }
+            };
+            if (fast_fwd()) {
+#pragma unroll 2
+                for (int tt = 0; tt < T; ++tt) tok(tt, Unchecked{});
+            } else {
+                for (int tt = 0; tt < T; ++tt) tok(tt, Checked{});
             }
-            if (CONV) sm.dp[tt][pp] = dpv;
-        }
-        if (CONV) {
+            scale_rows(xs, iQ);
+            Q = 1.f; iQ = 1.f;
             __syncthreads();
-            // du_t = w3 dp_t + w2 dp_{t+1} + w1 dp_{t+2} + w0 dp_{t+3}
+            // Pivot factors of A around token T/2 of the sub-block.
+#pragma unroll
+            for (int kk = 0; kk < R; ++kk) {
+                const int tt = rr * R + kk;
+                const float piv = sm.x1[T / 2][pp];
+                const float l = sm.x1[tt][pp];
+                sm.x3[tt][pp] = sm.dy[tt][pp] * __expf(l - piv);
+                sm.x4[tt][pp] = sm.v[tt][pp] * __expf(piv - l);
+                sm.x2[tt][pp] *= sm.dy[tt][pp];  // dy_t E_t
+            }
+            __syncthreads();
+            // A[t][m] = sum_p fa[t][p] fb[m][p] for m <= t (two outputs per thread).
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int e = tid + h2 * NT;
+                const int tt = e / T, mm = e % T;
+                float a = 0.f;
+                if (mm <= tt) {
+#pragma unroll 8
+                    for (int q2 = 0; q2 < P; ++q2) a = fmaf(sm.x3[tt][q2], sm.x4[mm][q2], a);
+                }
+                sm.A[sb][tt][mm] = a;
+            }
+            __syncthreads();
+            // dC[t][j] = s [ sum_p (dy E)[t][p] X_b[p][j] + sum_{m<=t} A[t][m] B[m][j] ].
+            {
+                constexpr int JB = (N * T) / NT;  // outputs per thread
+                const int tt = tid % T;
+                const int j0 = (tid / T) * JB;
+                float o[JB];
+#pragma unroll
+                for (int r = 0; r < JB; ++r) o[r] = 0.f;
+#pragma unroll 4
+                for (int q2 = 0; q2 < P; ++q2) {
+                    const float a = sm.x2[tt][q2];
+#pragma unroll
+                    for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.snap[q2][j0 + r], o[r]);
+                }
+                for (int mm = 0; mm <= tt; ++mm) {
+                    const float a = sm.A[sb][tt][mm];
+#pragma unroll
+                    for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.Bf[mm][j0 + r], o[r]);
+                }
+#pragma unroll
+                for (int r = 0; r < JB; ++r) sm.acc[sb * T + tt][j0 + r] = s * o[r];
+            }
+        });
+        cluster_reduce(1, tb, te);
+
+        // tail of f df over this block: H . x_end (per channel)
+        float tail = 0.f;
+#pragma unroll
+        for (int j = 0; j < NS / 2; ++j) tail = fmaf(gs[j].x, xs[j].x, fmaf(gs[j].y, xs[j].y, tail));
+        tail = red(tail);
+
+        // --------------------------------------------- backward sweep
+        float cum = 0.f;  // sum of dL over later tokens of the block
+        const bool group_end_block = (k == kb1 - 1);
+        pass(tb + (NSUB - 1) * T, NSUB, -1, te, true, [&](int i, int64_t t0) {
+            const int sb = NSUB - 1 - i;
+            snap_rows(gs, iR);  // H_e: carry entering the sub-block's end, true scale
+            float F = 1.f;      // prod f_{m+1..end of sub-block}
+            auto tok = [&](int tt, auto check) {
+                const float gbv = red(bstep(tt, true));
+                const float vv = sm.v[tt][pl];
+                const float dL = s * sm.dy[tt][pl] * sm.ys[sb * T + tt][pl] - vv * gbv;
+                cum += dL;
+                if (js == 0) {
+                    sm.x1[tt][pl] = gbv;
+                    sm.x3[tt][pl] = cum + tail;
+                    sm.x2[tt][pl] = vv * F;  // (i h F)_m
+                }
+                F *= sm.f[tt][pl];
+                bdecay(tt, check);
+            };
+            if (fast_bwd()) {
+#pragma unroll 2
+                for (int tt = T - 1; tt >= 0; --tt) tok(tt, Unchecked{});
+            } else {
+                for (int tt = T - 1; tt >= 0; --tt) tok(tt, Checked{});
+            }
+            __syncthreads();
+            // dB[m][j] = sum_p (i h F)[m][p] H_e[p][j] + s sum_{t>=m} A[t][m] C[t][j].
+            {
+                constexpr int JB = (N * T) / NT;
+                const int mm = tid % T;
+                const int j0 = (tid / T) * JB;
+                float o[JB], o2[JB];
+#pragma unroll
+                for (int r = 0; r < JB; ++r) { o[r] = 0.f; o2[r] = 0.f; }
+#pragma unroll 4
+                for (int q2 = 0; q2 < P; ++q2) {
+                    const float a = sm.x2[mm][q2];
+#pragma unroll
+                    for (int r = 0; r < JB; ++r) o[r] = fmaf(a, sm.snap[q2][j0 + r], o[r]);
+                }
+                for (int tt = mm; tt < T; ++tt) {
+                    const float a = sm.A[sb][tt][mm];
+#pragma unroll
+                    for (int r = 0; r < JB; ++r) o2[r] = fmaf(a, sm.Cf[tt][j0 + r], o2[r]);
+                }
+#pragma unroll
+                for (int r = 0; r < JB; ++r) sm.acc[sb * T + mm][j0 + r] = fmaf(s, o2[r], o[r]);
+            }
+            // Per-channel gradients of the sub-block (thread pp, run rr).
 #pragma unroll
             for (int kk = 0; kk < R; ++kk) {
                 const int tt = rr * R + kk;
                 const int64_t t = t0 + tt;
+                float dpv = 0.f;
                 if (cpvalid && t < te) {
-                    const float duv = w3 * sm.dp[tt][pp] + w2 * sm.dp[tt + 1][pp] +
-                                      w1 * sm.dp[tt + 2][pp] + w0 * sm.dp[tt + 3][pp];
-                    if (!last && t >= te - 3) {
-                        edge[(3 + (t - (te - 3))) * d + cp] = duv;  // partial, fixed up later
+                    float h, pre = 0.f;
+                    if (CONV) {
+                        pre = wb + w0 * to_f(sm.u[tt][pp]) + w1 * to_f(sm.u[tt + 1][pp]) +
+                              w2 * to_f(sm.u[tt + 2][pp]) + w3 * to_f(sm.u[tt + 3][pp]);
+                        h = siluf_(pre);
                     } else {
-                        gdhu[t * d + cp] = from_f<Tout>(duv);
+                        h = to_f(sm.u[tt + 3][pp]);
                     }
-                    if (sb == 0 && tt < 3) edge[tt * d + cp] = sm.dp[tt][pp];
+                    const float fv = sm.f[tt][pp];
+                    const float iv = sigmoidf_(to_f(sm.b[tt][pp]));
+                    const float gbv = sm.x1[tt][pp];
+                    const float dyv = sm.dy[tt][pp];
+                    const float dh = Dc * dyv + iv * gbv;
+                    gda[t * d + cp] = from_f<Tout>(sm.x3[tt][pp] * (1.f - fv));
+                    gdb[t * d + cp] = from_f<Tout>(h * gbv * iv * (1.f - iv));
+                    if (gz) {
+                        const float zv = to_f(sm.z[tt][pp]);
+                        const float yv = fmaf(s, sm.ys[sb * T + tt][pp], Dc * h);
+                        gdz[t * d + cp] = from_f<Tout>(to_f(sm.dout[tt][pp]) * yv * dsiluf_(zv));
+                    }
+                    dD_acc = fmaf(dyv, h, dD_acc);
+                    if (CONV) {
+                        dpv = dh * dsiluf_(pre);
+                        dw0 = fmaf(dpv, to_f(sm.u[tt][pp]), dw0);
+                        dw1 = fmaf(dpv, to_f(sm.u[tt + 1][pp]), dw1);
+                        dw2 = fmaf(dpv, to_f(sm.u[tt + 2][pp]), dw2);
+                        dw3 = fmaf(dpv, to_f(sm.u[tt + 3][pp]), dw3);
+                        dbias += dpv;
+                    } else {
+                        gdhu[t * d + cp] = from_f<Tout>(dh);
+                    }
+                }
+                if (CONV) sm.dp[tt][pp] = dpv;
+            }
+            if (CONV) {
+                __syncthreads();
+                // du_t = w3 dp_t + w2 dp_{t+1} + w1 dp_{t+2} + w0 dp_{t+3}
+#pragma unroll
+                for (int kk = 0; kk < R; ++kk) {
+                    const int tt = rr * R + kk;
+                    const int64_t t = t0 + tt;
+                    if (cpvalid && t < te) {
+                        const float duv = w3 * sm.dp[tt][pp] + w2 * sm.dp[tt + 1][pp] +
+                                          w1 * sm.dp[tt + 2][pp] + w0 * sm.dp[tt + 3][pp];
+                        if (!lastg && group_end_block && t >= te - 3) {
+                            edge[(3 + (t - (te - 3))) * d + cp] = duv;  // partial, fixed up later
+                        } else {
+                            gdhu[t * d + cp] = from_f<Tout>(duv);
+                        }
+                        if (k == kb0 && sb == 0 && tt < 3) edge[tt * d + cp] = sm.dp[tt][pp];
+                    }
+                }
+                __syncthreads();
+                if (tid < P) {  // carry the first three dp rows to the earlier sub-block
+                    sm.dp[T][tid] = sm.dp[0][tid];
+                    sm.dp[T + 1][tid] = sm.dp[1][tid];
+                    sm.dp[T + 2][tid] = sm.dp[2][tid];
                 }
             }
-            __syncthreads();
-            if (tid < P) {  // carry the first three dp rows to the earlier sub-block
-                sm.dp[T][tid] = sm.dp[0][tid];
-                sm.dp[T + 1][tid] = sm.dp[1][tid];
-                sm.dp[T + 2][tid] = sm.dp[2][tid];
-            }
-        }
-    });
-    cluster_reduce(0);
+        });
+        cluster_reduce(0, tb, te);
+    }
 
     // ------------------------------------------------ carries and partials
-    if (last && k > 0) {  // publish the carry leaving the block after the full sweep
-        if (cvalid) {
-#pragma unroll
-            for (int m = 0; m < NS / 4; ++m)
-                reinterpret_cast<float4*>(carry_out + c * N)[m * S + js] =
-                    make_float4(gs[4 * m] * iR, gs[4 * m + 1] * iR, gs[4 * m + 2] * iR,
-                                gs[4 * m + 3] * iR);
-        }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0 && !p.fault_skip_publish) st_release(flag_out, 1);
-    }
-    if (k == 0 && p.dx0 && cvalid) {
-#pragma unroll
-        for (int m = 0; m < NS / 4; ++m)
-            reinterpret_cast<float4*>(p.dx0 + ((int64_t)bb * d + c) * N)[m * S + js] =
-                make_float4(gs[4 * m] * iR, gs[4 * m + 1] * iR, gs[4 * m + 2] * iR,
-                            gs[4 * m + 3] * iR);
-    }
+    if (firstg && p.dx0) store_rows(p.dx0 + (int64_t)bb * d * N, gs, iR);
     // Per-channel partial sums (runs of the same channel add through shared atomics).
     {
-        float* cpart = p.chan_part + ((int64_t)bb * p.nsub + k) * d * 8;
+        float* cpart = p.chan_part + ((int64_t)bb * p.ngroups + g) * d * 8;
         float* red6 = &sm.x1[0][0];  // reuse: [6][P] (T >= 6)
         __syncthreads();
         for (int i = tid; i < 6 * P; i += NT) red6[i] = 0.f;
@@ -655,26 +705,27 @@ __global__ void reduce_chan_kernel(const float* __restrict__ part, int64_t rows,
     if (dbias) dbias[c] = acc[5];
 }
 
-// du of the last three tokens of each non-final block: the block's own
-// partial plus the terms from the first three dp of the next block.
+// du of the last three tokens of each non-final sequence group: the group's
+// own partial plus the terms from the first three dp of the next group.
 template <typename Tout>
 __global__ void conv_edge_kernel(const float* __restrict__ edge, const float* __restrict__ w,
-                                 int64_t Bt, int nsub, int64_t L, int64_t d,
-                                 Tout* __restrict__ du) {
-    const int64_t n = Bt * (int64_t)(nsub - 1) * 3 * d;
+                                 int64_t Bt, int ngroups, int64_t group_tokens, int64_t L,
+                                 int64_t d, Tout* __restrict__ du) {
+    const int64_t n = Bt * (int64_t)(ngroups - 1) * 3 * d;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t c = i % d;
         const int r = (int)((i / d) % 3);
-        const int64_t kb = (i / (3 * d)) % (nsub - 1);
-        const int64_t bb = i / (3 * d * (nsub - 1));
-        const int64_t t = (kb + 1) * kBwdSub - 3 + r;
-        const float* mine = edge + ((bb * nsub + kb) * 2 + 1) * 3 * d;
-        const float* next = edge + ((bb * nsub + kb + 1) * 2 + 0) * 3 * d;
+        const int64_t gb = (i / (3 * d)) % (ngroups - 1);
+        const int64_t bb = i / (3 * d * (ngroups - 1));
+        const int64_t tend = (gb + 1) * group_tokens;
+        const int64_t t = tend - 3 + r;
+        const float* mine = edge + ((bb * ngroups + gb) * 2 + 1) * 3 * d;
+        const float* next = edge + ((bb * ngroups + gb + 1) * 2 + 0) * 3 * d;
         float v = mine[r * d + c];
-        // du_t += sum_k w[k] dp_{t+3-k} over the next block's tokens.
+        // du_t += sum_k w[k] dp_{t+3-k} over the next group's tokens.
         for (int kk = 0; kk < 4; ++kk) {
-            const int64_t ts = t + 3 - kk - (kb + 1) * kBwdSub;
+            const int64_t ts = t + 3 - kk - tend;
             if (ts >= 0 && ts < 3) v += w[c * 4 + kk] * next[ts * d + c];
         }
         du[(bb * L + t) * d + c] = from_f<Tout>(v);
@@ -692,7 +743,7 @@ static cudaError_t launch_bwd_t(const BwdParams& p, void* dB, void* dC, float* d
                                          (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.nclus * kCluster), (unsigned)p.Bt, (unsigned)p.nsub);
+    cfg.gridDim = dim3((unsigned)(p.nclus * kCluster), (unsigned)p.Bt, (unsigned)p.ngroups);
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -709,9 +760,10 @@ static cudaError_t launch_bwd_t(const BwdParams& p, void* dB, void* dC, float* d
     reduce_dBC_kernel<Tout><<<592, 256, 0, st>>>(p.dBCp, p.nclus, BtL, N,
                                                   static_cast<Tout*>(dB), static_cast<Tout*>(dC));
     reduce_chan_kernel<<<(unsigned)((p.d + 127) / 128), 128, 0, st>>>(
-        p.chan_part, p.Bt * p.nsub, p.d, dD, CONV ? dw : nullptr, CONV ? dbias : nullptr);
-    if (CONV && p.nsub > 1)
-        conv_edge_kernel<Tout><<<296, 256, 0, st>>>(p.conv_edge, p.conv_w, p.Bt, p.nsub, p.L,
+        p.chan_part, p.Bt * p.ngroups, p.d, dD, CONV ? dw : nullptr, CONV ? dbias : nullptr);
+    if (CONV && p.ngroups > 1)
+        conv_edge_kernel<Tout><<<296, 256, 0, st>>>(p.conv_edge, p.conv_w, p.Bt, p.ngroups,
+                                                     (int64_t)p.blk_per_group * kBwdSub, p.L,
                                                      p.d, static_cast<Tout*>(p.dhu));
     return cudaGetLastError();
 }

@@ -24,13 +24,16 @@
 // would pass 2^64 in any lane of a warp, the warp folds Q back into its states.
 //
 // Sequence groups.  When batch x channel tiles alone do not fill the GPU,
-// the sequence is split into G groups handled by different blocks.  A block
-// of group g > 0 first runs its group with a zero initial state to get the
-// group's local end state and decay product, then waits (bounded) for group
-// g-1 to publish its end state, publishes its own, and finally runs the group
-// again from the true initial state producing outputs (a decoupled
-// look-back along the sequence).  Work items are taken from an atomic ticket
-// in group order, so every awaited block has already started.
+// the sequence is split into G groups handled by different blocks.  Every
+// group but the last first runs its tokens without readout: group 0 from x0,
+// the others from a zero state, after which they wait (bounded) for group
+// g-1's end state, fold it in with the group's decay product and publish
+// their own end state.  All groups then run their full pass from the true
+// initial state concurrently (a decoupled look-back along the sequence).
+// Work items are taken from an atomic ticket in group order, so every
+// awaited block has already started.
+#include <type_traits>
+
 #include "naju_common.cuh"
 #include "naju_kernels.h"
 
@@ -189,21 +192,24 @@ scan_fwd_kernel(const FwdParams p) {
     };
 
     // One token of the recurrence for this thread's state slice.  Returns the
-    // readout partial x.C (true scale) when READ.
-    auto step = [&](int tt, bool READ) -> float {
+    // readout partial x.C (true scale) when READ.  CHECK tests Q against the
+    // renormalisation bound (slow path only).
+    auto step = [&](int tt, auto read, auto check) -> float {
         const float q = sm.sQ[tt][pl];
         const float f = sm.sF[tt][pl];
         const float v = sm.sV[tt][pl];
         float Qn = Q * q;
         float iQn = invQ * f;
-        if (__any_sync(0xffffffffu, !(Qn <= kRenorm))) {
-            // Fold: xs <- x_{t-1} * f_t, i.e. xs * invQ * f.
-            logPf += __logf(iQn);
-            const float2 s2 = make_float2(iQn, iQn);
+        if constexpr (decltype(check)::value) {
+            if (__any_sync(0xffffffffu, !(Qn <= kRenorm))) {
+                // Fold: xs <- x_{t-1} * f_t, i.e. xs * invQ * f.
+                logPf += __logf(iQn);
+                const float2 s2 = make_float2(iQn, iQn);
 #pragma unroll
-            for (int j = 0; j < NS / 2; ++j) xs[j] = __fmul2_rn(xs[j], s2);
-            Qn = 1.f;
-            iQn = 1.f;
+                for (int j = 0; j < NS / 2; ++j) xs[j] = __fmul2_rn(xs[j], s2);
+                Qn = 1.f;
+                iQn = 1.f;
+            }
         }
         Q = Qn;
         invQ = iQn;
@@ -211,19 +217,40 @@ scan_fwd_kernel(const FwdParams p) {
         const float2 w2v = make_float2(wv, wv);
         const float4* b4 = reinterpret_cast<const float4*>(sm.sB[tt]);
         const float4* c4 = reinterpret_cast<const float4*>(sm.sC[tt]);
-        float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+        float2 a[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
         for (int m = 0; m < NS / 4; ++m) {
             const float4 bv = b4[m * S + js];
             xs[2 * m] = __ffma2_rn(w2v, make_float2(bv.x, bv.y), xs[2 * m]);
             xs[2 * m + 1] = __ffma2_rn(w2v, make_float2(bv.z, bv.w), xs[2 * m + 1]);
-            if (READ) {
+            if constexpr (decltype(read)::value) {
                 const float4 cv = c4[m * S + js];
-                a0 = __ffma2_rn(xs[2 * m], make_float2(cv.x, cv.y), a0);
-                a1 = __ffma2_rn(xs[2 * m + 1], make_float2(cv.z, cv.w), a1);
+                a[(2 * m) & 3] = __ffma2_rn(xs[2 * m], make_float2(cv.x, cv.y), a[(2 * m) & 3]);
+                a[(2 * m + 1) & 3] =
+                    __ffma2_rn(xs[2 * m + 1], make_float2(cv.z, cv.w), a[(2 * m + 1) & 3]);
             }
         }
-        return ((a0.x + a0.y) + (a1.x + a1.y)) * invQ;
+        const float2 a01 = __fadd2_rn(a[0], a[1]), a23 = __fadd2_rn(a[2], a[3]);
+        return ((a01.x + a01.y) + (a23.x + a23.y)) * invQ;
+    };
+    using Yes = std::integral_constant<bool, true>;
+    using No = std::integral_constant<bool, false>;
+    // Whether the chunk's T tokens can run without renormalisation checks
+    // (Q times the chunk's product of 1/f stays below the bound in every lane
+    // of the warp); otherwise fold Q into the state first and test again.
+    auto fast_chunk = [&]() -> bool {
+        float pq = 1.f;
+#pragma unroll
+        for (int tt = 0; tt < T; ++tt) pq *= sm.sQ[tt][pl];
+        if (!__any_sync(0xffffffffu, !(Q * pq <= kRenorm))) return true;
+        logPf += __logf(invQ);
+        const float2 s2 = make_float2(invQ, invQ);
+#pragma unroll
+        for (int j = 0; j < NS / 2; ++j) xs[j] = __fmul2_rn(xs[j], s2);
+        Q = 1.f;
+        invQ = 1.f;
+        return !__any_sync(0xffffffffu, !(pq <= kRenorm));
     };
 
     // One pass over the group's chunks: FULL = readout, outputs, checkpoints.
@@ -243,18 +270,28 @@ scan_fwd_kernel(const FwdParams p) {
             __syncthreads();
             prep(t0, buf, full);
             __syncthreads();
+            const bool fast = fast_chunk();
             if (full) {
-                for (int tt = 0; tt < T; ++tt) {
-                    float part = step(tt, true);
+                auto tok = [&](int tt, auto check) {
+                    float part = step(tt, Yes{}, check);
 #pragma unroll
                     for (int o = 1; o < S; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
                     if (js == 0) sm.sY[tt][pl] = part;
+                };
+                if (fast) {
+#pragma unroll 2
+                    for (int tt = 0; tt < T; ++tt) tok(tt, No{});
+                } else {
+                    for (int tt = 0; tt < T; ++tt) tok(tt, Yes{});
                 }
                 const int64_t tnext = t0 + T;
                 if (tnext < tend && tnext % p.T_ck == 0)
                     store_state(ck_b + (tnext / p.T_ck) * d * N);
+            } else if (fast) {
+#pragma unroll 2
+                for (int tt = 0; tt < T; ++tt) step(tt, No{}, No{});
             } else {
-                for (int tt = 0; tt < T; ++tt) step(tt, false);
+                for (int tt = 0; tt < T; ++tt) step(tt, No{}, Yes{});
             }
             __syncthreads();
             if (full && cpvalid) {
@@ -274,28 +311,26 @@ scan_fwd_kernel(const FwdParams p) {
         }
     };
 
-    // --------------------------------------------- local pass (groups > 0)
-    const bool do_local = (g > 0) && !last_group;
-    if (do_local) {
-        load_state(nullptr, false);
-        run_pass(false);
-    }
-    // Local end state (zero start) and log prod f of the group.
-    const float logPf_loc = logPf + __logf(invQ);
-
-    // ----------------------------------------------- carry in / publish
+    // ------------------------------------------ early pass and carry chain
+    // Every group with a successor first runs its tokens without readout to
+    // get its end state and publishes it, so that all full passes can run
+    // concurrently: group 0 starts from x0, later groups from a zero state
+    // and fold in the predecessor's end state once it is published.
+    const float* x0b = p.x0 ? p.x0 + (int64_t)bb * d * N : nullptr;
     const int* flag_prev = (g > 0) ? p.flags + ((int64_t)(g - 1) * Bt + bb) * p.ntiles + tile
                                    : nullptr;
     int* flag_mine = p.flags + ((int64_t)g * Bt + bb) * p.ntiles + tile;
     float* ck_start = ck_b + (int64_t)seg0 * d * N;
     float* ck_end = ck_b + (int64_t)seg1 * d * N;
-    if (g > 0) {
-        if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
-        __syncthreads();
-        const bool ok = sm.ok != 0;
-        if (do_local) {
-            // X_end = prod f * X_start + local state.
-            const float Pf = __expf(logPf_loc);
+    bool ok = true;
+    if (!last_group) {
+        load_state(g == 0 ? x0b : nullptr, false);
+        run_pass(false);
+        if (g > 0) {
+            const float Pf = __expf(logPf + __logf(invQ));  // prod f over the group
+            if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
+            __syncthreads();
+            ok = sm.ok != 0;
 #pragma unroll
             for (int m = 0; m < NS / 4; ++m) {
                 float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -307,27 +342,25 @@ scan_fwd_kernel(const FwdParams p) {
                 xs[2 * m + 1].y = fmaf(Pf, v4.w, xs[2 * m + 1].y * invQ);
             }
             invQ = 1.f;
-            store_state(ck_end);
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) st_release(flag_mine, 1);
         }
+        store_state(ck_end);
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && !(g == 0 && p.fault_skip_publish)) st_release(flag_mine, 1);
+    } else if (g > 0) {
+        if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
+        __syncthreads();
+        ok = sm.ok != 0;
+    }
+    if (g > 0) {
         load_state(ok ? ck_start : nullptr, true);
     } else {
-        load_state(p.x0 ? p.x0 + (int64_t)bb * d * N : nullptr, false);
+        load_state(x0b, false);
         store_state(ck_b);  // checkpoint 0 = initial state
     }
 
     // ------------------------------------------------------- full pass
     run_pass(true);
-
-    // -------------------------------------------------- group end state
-    if (g == 0 && p.ngroups > 1) {
-        store_state(ck_end);
-        __threadfence();
-        __syncthreads();
-        if (tid == 0 && !p.fault_skip_publish) st_release(flag_mine, 1);
-    }
     if (last_group) {
         store_state(ck_b + (int64_t)p.nck * d * N);
         if (p.x_final) store_state(p.x_final + (int64_t)bb * d * N);

@@ -22,7 +22,7 @@ extern "C" {
 void naju_testing_set_wait_limit(int64_t polls);
 
 /* skip != 0: the forward's first sequence group and the backward's last
- * block do not publish their carries (their successors time out). */
+ * sequence group do not publish their carries (their successors time out). */
 void naju_testing_set_skip_publish(int32_t skip);
 
 /* Forces the number of sequence groups of the forward (<= 0: automatic).
@@ -32,6 +32,13 @@ void naju_testing_set_fwd_groups(int32_t groups);
 /* The forward's number of sequence groups for these dims (after the
  * automatic choice and any forced value). */
 int32_t naju_testing_fwd_groups(const void* dims);
+
+/* Forces the number of sequence groups of the backward (<= 0: automatic);
+ * more groups than 64-token blocks are clamped. */
+void naju_testing_set_bwd_groups(int32_t groups);
+
+/* The backward's number of sequence groups for these dims. */
+int32_t naju_testing_bwd_groups(const void* dims);
 
 #ifdef __cplusplus
 }

@@ -234,6 +234,21 @@ def test_bwd_extreme_gates():
     compare_grads(g, r, True, TOL_F32)
 
 
+@pytest.mark.parametrize("groups", [1, 2, 3, 5])
+def test_bwd_sequence_groups(groups):
+    """Splitting the backward's sequence across blocks (reverse look-back of
+    the adjoint carry, conv terms across group edges) changes nothing."""
+    w = wl(64, "f32", Bt=2, L=600, d=100)
+    t = inputs(w, True, use_x0=True, use_dxL=True)
+    r = oracle_bwd(t, True)
+    naju.testing_set_bwd_groups(groups)
+    try:
+        g = run_bwd(t, True)
+    finally:
+        naju.testing_set_bwd_groups(0)
+    compare_grads(g, r, True, TOL_F32)
+
+
 def test_bwd_after_grouped_forward():
     """Checkpoints written by a sequence-split forward serve the backward."""
     w = wl(64, "f32", Bt=1, L=700, d=64)

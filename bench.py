@@ -311,10 +311,15 @@ def main():
         ws_cpu = cpu_sample_workload(w)
         tc = make_inputs(ws_cpu, which=("u", "a", "b", "B", "C", "z", "D", "conv_w", "conv_b",
                                         "dout"))
-        dt, toks, thr = cpu_oracle_step(ws_cpu, tc)
-        cpu = {"value": toks / dt, "unit": "tokens/s", "cores": thr, "kind": "oracle",
-               "sample": f"oracle fwd+bwd, batch 1 x L={ws_cpu.seqlen} slice of {w.name}, "
-                         f"{dt:.1f} s"}
+        dt_sum, toks_sum, reps = 0.0, 0, 0
+        while dt_sum < 10.0 and reps < 64:  # about 10 s of host work
+            dt, toks, thr = cpu_oracle_step(ws_cpu, tc)
+            dt_sum += dt
+            toks_sum += toks
+            reps += 1
+        cpu = {"value": toks_sum / dt_sum, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+               "sample": f"oracle fwd+bwd, {reps} x (batch 1 x L={ws_cpu.seqlen}) slice of "
+                         f"{w.name}, {dt_sum:.1f} s"}
 
     if rank == 0:
         print(json.dumps({

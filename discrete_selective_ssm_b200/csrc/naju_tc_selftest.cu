@@ -1,0 +1,90 @@
+// Self-test of the tensor-core building block used by the tensor-core scan:
+// D[128 x N] = A[128 x K] * B[N x K]^T with A staged in tensor memory, B in
+// shared memory (no-swizzle K-major core matrices) and D in tensor memory,
+// kind::tf32, K = 8 per instruction.  Exposed through naju_testing.h so the
+// test suite can check the operand conventions against a host product.
+#include "naju.h"
+#include "naju_common.cuh"
+#include "naju_tc.cuh"
+#include "naju_testing.h"
+
+namespace naju {
+
+__global__ void __launch_bounds__(128, 1)
+tc_selftest_kernel(const float* __restrict__ A, const float* __restrict__ B,
+                   float* __restrict__ D, int N, int K, uint32_t ncols, int* status) {
+    extern __shared__ float4 smem4[];
+    unsigned char* sb = reinterpret_cast<unsigned char*>(smem4);
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t taddr_s;
+    const int tid = threadIdx.x, warp = tid / 32;
+
+    if (warp == 0) {
+        tc::tmem_alloc(&taddr_s, ncols);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) tc::mbar_init(&mbar, 1);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = taddr_s;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+
+    // A row `tid` -> TMEM lane `tid`, columns [0, K).
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = A[tid * K + k0 + i];
+        tc::tmem_st16(tbase + lane_off + k0, v);
+    }
+    // B [N x K] -> shared memory, K-major core matrices.
+    for (int e = tid; e < N * K; e += 128) {
+        const int row = e / K, k = e % K;
+        *reinterpret_cast<float*>(sb + tc::kmajor_offset(row, k, K)) = B[e];
+    }
+    tc::tmem_st_wait();
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+        tc::fence_after_sync();
+        const uint32_t idesc = tc::idesc_tf32(128, N);
+        const uint32_t sbase = tc::smem_u32(sb);
+        for (int ks = 0; ks < K / 8; ++ks) {
+            const uint64_t bdesc = tc::sdesc(sbase + ks * 256, 128, 32 * K);
+            tc::mma_tf32_ts(tbase + K, tbase + ks * 8, bdesc, idesc, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&mbar);
+    }
+    const bool done = tc::mbar_wait(&mbar, 0, 1LL << 22);
+    if (!done && tid == 0) atomicOr(status, 1 << NAJU_ERR_TIMEOUT);
+    tc::fence_after_sync();
+    for (int n0 = 0; n0 < N; n0 += 16) {
+        float v[16];
+        tc::tmem_ld16(tbase + lane_off + K + n0, v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) D[tid * N + n0 + i] = done ? v[i] : __int_as_float(0x7fc00000);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, ncols);
+}
+
+}  // namespace naju
+
+extern "C" naju_status naju_testing_tc_mma(int32_t N, int32_t K, const float* A, const float* B,
+                                           float* D, int* status, void* stream) {
+    if (!A || !B || !D || !status) return NAJU_ERR_INVALID_ARG;
+    if (N < 16 || N > 256 || N % 16 != 0 || K < 16 || K % 16 != 0 || K + N > 512)
+        return NAJU_ERR_UNSUPPORTED;
+    uint32_t ncols = 32;
+    while (ncols < (uint32_t)(K + N)) ncols <<= 1;
+    const size_t smem = sizeof(float) * (size_t)N * K;
+    cudaError_t e = cudaFuncSetAttribute(naju::tc_selftest_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return NAJU_ERR_CUDA;
+    naju::tc_selftest_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(A, B, D, N, K,
+                                                                                 ncols, status);
+    return cudaGetLastError() == cudaSuccess ? NAJU_OK : NAJU_ERR_CUDA;
+}

@@ -13,6 +13,8 @@
 
 #include <stdint.h>
 
+#include "naju.h"
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -39,6 +41,15 @@ void naju_testing_set_bwd_groups(int32_t groups);
 
 /* The backward's number of sequence groups for these dims. */
 int32_t naju_testing_bwd_groups(const void* dims);
+
+/* Self-test of the tensor-core building block of the tensor-core scans:
+ * D[128 x N] = A[128 x K] * B[N x K]^T (device pointers, row-major fp32)
+ * computed with A in tensor memory, B in shared memory and kind::tf32 MMAs
+ * (one thread block).  N, K multiples of 16, N <= 256, K + N <= 512.  A
+ * completion wait that runs out sets NAJU_ERR_TIMEOUT in *status (device
+ * int) and writes NaN to D. */
+naju_status naju_testing_tc_mma(int32_t N, int32_t K, const float* A, const float* B, float* D,
+                                int* status, void* stream);
 
 #ifdef __cplusplus
 }

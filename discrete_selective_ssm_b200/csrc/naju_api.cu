@@ -22,6 +22,7 @@ long long g_wait_limit = kDefaultWait;
 int g_skip_publish = 0;
 int g_fwd_groups = 0;
 int g_bwd_groups = 0;
+int g_fwd_impl = 0;  // 0 automatic, 1 CUDA cores, 2 tensor cores
 
 inline bool aligned(const void* ptr, size_t a) {
     return (reinterpret_cast<uintptr_t>(ptr) % a) == 0;
@@ -46,15 +47,23 @@ naju_status check_dims(const naju_dims* dm) {
 
 // Workspace layout (every region 256-byte aligned).
 struct Layout {
+    bool fwd_tc;
     int nck, ngroups, seg_per_group, ntiles_f;
     int nsub, nclus, ntiles_b, bgroups, blk_per_group;
     size_t off_fflags, off_bflags, off_ckpt, off_carry, off_dbc, off_chan, off_edge, total;
 };
 
-int auto_groups(const naju_dims* dm, int nck, int ntiles_f) {
+bool use_fwd_tc(const naju_dims* dm) {
+    if (g_fwd_impl == 1) return false;
+    return fwd_tc_supported(dm->dtype, dm->d_state);
+}
+
+int auto_groups(const naju_dims* dm, int nck, int ntiles_f, bool tc) {
     if (g_fwd_groups > 0) return g_fwd_groups < nck ? g_fwd_groups : nck;
     const int64_t items = dm->batch * (int64_t)ntiles_f;
-    const int64_t want = 3 * kSMs;
+    // Blocks resident per SM: tensor-core blocks hold 256 (d_state 64) or 512
+    // (d_state 128) of the SM's 512 tensor-memory columns.
+    const int64_t want = tc ? (dm->d_state == 64 ? 2 : 1) * kSMs : 3 * kSMs;
     if (items >= want) return 1;
     int64_t g = cdiv(want, items);
     return (int)(g < nck ? g : nck);
@@ -64,8 +73,9 @@ Layout layout(const naju_dims* dm) {
     Layout l{};
     const int64_t Bt = dm->batch, L = dm->seqlen, d = dm->d_inner, N = dm->d_state;
     l.nck = (int)cdiv(L, kTck);
-    l.ntiles_f = (int)cdiv(d, fwd_channels_per_block(N));
-    int g = auto_groups(dm, l.nck, l.ntiles_f);
+    l.fwd_tc = use_fwd_tc(dm);
+    l.ntiles_f = (int)cdiv(d, l.fwd_tc ? fwd_tc_channels_per_block() : fwd_channels_per_block(N));
+    int g = auto_groups(dm, l.nck, l.ntiles_f, l.fwd_tc);
     l.seg_per_group = (int)cdiv(l.nck, g);
     l.ngroups = (int)cdiv(l.nck, l.seg_per_group);
     l.nsub = (int)cdiv(L, kBwdSub);
@@ -86,7 +96,9 @@ Layout layout(const naju_dims* dm) {
     }
     size_t off = sizeof(WsHeader);
     l.off_fflags = off;
-    off = up256(off + sizeof(int) * (size_t)l.ngroups * Bt * l.ntiles_f);
+    // Flags for the larger of the two forward tilings (at most nck groups), so
+    // the workspace size does not depend on which forward kernel runs.
+    off = up256(off + sizeof(int) * (size_t)l.nck * Bt * cdiv(d, 32));
     l.off_bflags = off;
     off = up256(off + sizeof(int) * (size_t)l.bgroups * Bt * l.ntiles_b);
     l.off_ckpt = off;
@@ -180,6 +192,7 @@ naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* co
     p.scale = 1.0f / std::sqrt((float)dims->d_state);
     p.wait_limit = g_wait_limit;
     p.fault_skip_publish = g_skip_publish;
+    if (l.fwd_tc) return cuda_status(launch_scan_fwd_tc(p, dims->out_dtype, s));
     return cuda_status(launch_scan_fwd(p, dims->dtype, dims->out_dtype, s));
 }
 
@@ -277,6 +290,12 @@ void naju_testing_set_wait_limit(int64_t polls) {
 void naju_testing_set_skip_publish(int32_t skip) { g_skip_publish = skip ? 1 : 0; }
 void naju_testing_set_fwd_groups(int32_t groups) { g_fwd_groups = groups > 0 ? groups : 0; }
 void naju_testing_set_bwd_groups(int32_t groups) { g_bwd_groups = groups > 0 ? groups : 0; }
+void naju_testing_set_fwd_impl(int32_t impl) { g_fwd_impl = (impl == 1) ? 1 : 0; }
+int32_t naju_testing_fwd_impl(const void* dims) {
+    const naju_dims* dm = static_cast<const naju_dims*>(dims);
+    if (check_dims(dm) != NAJU_OK) return 0;
+    return use_fwd_tc(dm) ? 2 : 1;
+}
 int32_t naju_testing_bwd_groups(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);
     if (check_dims(dm) != NAJU_OK) return 0;

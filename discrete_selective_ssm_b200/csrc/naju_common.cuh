@@ -54,6 +54,15 @@ __device__ __forceinline__ void store8(float* p, const float* v) {
 // sigmoid saturates cleanly); the accuracy of each use is covered by the
 // parity tests against the fp64 oracle.
 __device__ __forceinline__ float rcpf_(float v) { return __frcp_rn(v); }
+// Single-instruction approximate reciprocal (PTX rcp.approx.ftz.f32; about
+// one ulp), for the tensor-core path whose operands are tf32 anyway.
+__device__ __forceinline__ float rcpa_(float v) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+__device__ __forceinline__ float sigmoida_(float v) { return rcpa_(1.0f + __expf(-v)); }
+__device__ __forceinline__ float silua_(float v) { return v * sigmoida_(v); }
 __device__ __forceinline__ float sigmoidf_(float v) { return rcpf_(1.0f + __expf(-v)); }
 __device__ __forceinline__ float siluf_(float v) { return v * sigmoidf_(v); }
 // d/dv SiLU(v) = s (1 + v (1 - s)), s = sigmoid(v)

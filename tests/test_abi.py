@@ -69,7 +69,7 @@ def test_status_strings(L):
 def test_fwd_group_policy(L):
     # Few (batch x tile) items split the sequence; many do not.
     few = naju.make_dims(2, 8192, 2048, 128, naju.BF16)
-    many = naju.make_dims(16, 4096, 2048, 64, naju.BF16)
+    many = naju.make_dims(64, 4096, 2048, 64, naju.BF16)
     assert naju.testing_fwd_groups(few) > 1
     assert naju.testing_fwd_groups(many) == 1
     naju.testing_set_fwd_groups(3)

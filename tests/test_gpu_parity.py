@@ -137,6 +137,43 @@ def test_fwd_extreme_gates():
     assert_close(xf, rx, TOL_F32, name="x_final")
 
 
+@pytest.mark.parametrize("N", [64, 128])
+def test_fwd_tensor_core_exact_fallback(N):
+    """bf16 inputs with runs of vanishing forget gates: sub-chunks whose decay
+    would overflow the tensor-core factorisation take the exact path."""
+    w = wl(N, "bf16", Bt=2, L=300, d=200)
+    t = inputs(w, True, use_x0=True)
+    a = t["a"].float().clone()
+    a[:, 40:60] = -60.0
+    a[:, 100:200:2] = -25.0
+    a[:, 220:240] = 60.0
+    t["a"] = a.to(torch.bfloat16)
+    dm = naju.make_dims(2, 300, 200, N, naju.BF16)
+    assert naju.testing_fwd_impl(dm) == 2
+    y, xf, _ = run_fwd(t, True, out_dtype=naju.F32)
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_BF16, name="y")
+    assert_close(xf, rx, TOL_BF16, name="x_final")
+
+
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("impl", [1, 0])
+def test_fwd_both_implementations(N, impl):
+    """The CUDA-core and tensor-core forwards both match the oracle (bf16)."""
+    w = wl(N, "bf16", Bt=2, L=333, d=260)
+    t = inputs(w, True, use_x0=True)
+    naju.testing_set_fwd_impl(impl)
+    try:
+        y, xf, _ = run_fwd(t, True, out_dtype=naju.F32)
+        yb, _, _ = run_fwd(t, True, out_dtype=naju.BF16)
+    finally:
+        naju.testing_set_fwd_impl(0)
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_BF16, name="y")
+    assert_close(yb, ro, TOL_BF16, bf16_out=True, name="y bf16")
+    assert_close(xf, rx, TOL_BF16, name="x_final")
+
+
 def test_long_retention_overwrite_distribution():
     """Overwrite events (a ~ N(-4,1), b ~ N(3,1) on 5% of entries)."""
     w = scaled(WORKLOADS["long_retention"], batch=1, seqlen=700, d_inner=96, d_state=128)

@@ -55,15 +55,15 @@ struct Layout {
 
 bool use_fwd_tc(const naju_dims* dm) {
     if (g_fwd_impl == 1) return false;
-    return fwd_tc_supported(dm->dtype, dm->d_state);
+    return fwd_tc_supported(dm->dtype, dm->d_state, dm->d_inner);
 }
 
 int auto_groups(const naju_dims* dm, int nck, int ntiles_f, bool tc) {
     if (g_fwd_groups > 0) return g_fwd_groups < nck ? g_fwd_groups : nck;
     const int64_t items = dm->batch * (int64_t)ntiles_f;
-    // Blocks resident per SM: tensor-core blocks hold 256 (d_state 64) or 512
-    // (d_state 128) of the SM's 512 tensor-memory columns.
-    const int64_t want = tc ? (dm->d_state == 64 ? 2 : 1) * kSMs : 3 * kSMs;
+    // Blocks resident per SM: one tensor-core block (its operand stages fill
+    // most of the shared memory), three CUDA-core blocks.
+    const int64_t want = tc ? kSMs : 3 * kSMs;
     if (items >= want) return 1;
     int64_t g = cdiv(want, items);
     return (int)(g < nck ? g : nck);

@@ -80,7 +80,7 @@ int bwd_cluster_size();
 
 cudaError_t launch_scan_fwd(const FwdParams& p, int dtype, int out_dtype, cudaStream_t st);
 // Tensor-core forward (bf16 activations, d_state 64 or 128, 128 channels per block).
-bool fwd_tc_supported(int dtype, int64_t N);
+bool fwd_tc_supported(int dtype, int64_t N, int64_t d);
 int fwd_tc_channels_per_block();
 cudaError_t launch_scan_fwd_tc(const FwdParams& p, int out_dtype, cudaStream_t st);
 cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, int out_dtype, void* dB, void* dC,

@@ -6,8 +6,8 @@
 // out_n = y_n SiLU(z_n), h = SiLU(conv(u)).
 //
 // Chunked form.  A thread block owns 128 channels of one batch element (one
-// channel per thread = one tensor-memory lane) and walks its tokens in
-// sub-chunks of T = 16.  With X the state entering a sub-chunk,
+// channel = one tensor-memory lane) and walks its tokens in sub-chunks of
+// T = 16.  With X the state entering a sub-chunk,
 // E_t = prod_{k<=t} f_k (inclusive, from the sub-chunk start),
 // W_m = i_m h_m / E_m and G[t][m] = C_t.B_m (m <= t, else 0):
 //   y_t  = s E_t ( X.C_t + sum_m W_m G[t][m] ) + D h_t         (readout MMA)
@@ -25,59 +25,84 @@
 // operands give about 1e-3 relative error on the contractions; the fp32
 // activations path uses the CUDA-core kernel.
 //
-// Threads.  256 threads: channel p is TMEM lane p; the two threads of a
-// channel (warps w and w+4 share a lane quadrant) each unpack 8 of the 16
-// tokens, exchanging their decay products through shared memory, and each
-// update half of the state columns.
+// Warp roles.  Warps 0-7 produce: one thread loads raw sub-chunks with TMA
+// (two ahead, three raw buffers, an mbarrier each) and all 256 unpack each
+// sub-chunk into one of three operand stages (shared memory + tensor-memory
+// columns); channel p is handled by threads p and p + 128, each taking 8 of
+// the 16 tokens.  Warps 8-11 consume:
+// thread 256 + p owns channel p; one of them issues the MMAs of a stage, all
+// of them run the epilogue (outputs, X' = E_T X + D_state, checkpoints) and
+// release the stage.  Stages hand over through mbarriers (full: 256 producer
+// arrivals; empty: 128 consumer arrivals; one MMA-completion barrier), so
+// unpacking overlaps the tensor core and the epilogue.
 //
-// Pipeline.  While the tensor core runs sub-chunk i, the CUDA cores unpack
-// sub-chunk i+1 (double-buffered operands) and cp.async stages sub-chunk i+2.
 // Sequence groups work as in the CUDA-core kernel: an update-only pass and a
 // decoupled look-back publish each group's end state before the full pass.
+#include <string.h>
+
 #include <type_traits>
 
 #include "naju_common.cuh"
 #include "naju_kernels.h"
 #include "naju_tc.cuh"
+#include "naju_tma.h"
 
 namespace naju {
 
 namespace {
 
 constexpr int kTS = 16;                               // tokens per sub-chunk
+constexpr int kStages = 3;                            // operand stages = raw buffers
 constexpr float kTcBound = 18446744073709551616.0f;   // 2^64
+constexpr long long kMbarSpin = 1LL << 24;            // polls before giving up
 
+// Tensor-memory columns (lane = channel).  Per stage: W (readout weights,
+// or i h on the exact path), V (state weights, or f), EG (s E_t SiLU(z_t),
+// or s SiLU(z_t) on the exact path), DH (D h_t SiLU(z_t)).
 template <int N>
 struct TcCols {
-    static constexpr uint32_t X = 0;                  // state [N]
-    static constexpr uint32_t W = N;                  // 2 x kTS (parity)
-    static constexpr uint32_t V = N + 2 * kTS;        // 2 x kTS (parity)
-    static constexpr uint32_t DR = N + 4 * kTS;       // readout result [kTS]
-    static constexpr uint32_t DS = N + 5 * kTS;       // state result [N]
-    static constexpr uint32_t USED = 2 * N + 5 * kTS;
+    static constexpr uint32_t X = 0;                           // state [N]
+    static constexpr uint32_t W = N;                           // kStages x kTS each
+    static constexpr uint32_t V = W + kStages * kTS;
+    static constexpr uint32_t EG = V + kStages * kTS;
+    static constexpr uint32_t DH = EG + kStages * kTS;
+    static constexpr uint32_t DR = DH + kStages * kTS;         // readout result [kTS]
+    static constexpr uint32_t DS = DR + kTS;                   // state result [N]
+    static constexpr uint32_t USED = DS + N;
     static constexpr uint32_t ALLOC = USED <= 256 ? 256 : 512;
+    static_assert(USED <= 512, "tensor memory");
+};
+
+struct alignas(64) FwdTmaps {
+    CUtensorMap u, a, b, z, B, C;
 };
 
 template <int N>
 struct FwdTcSmem {
-    static constexpr int T = kTS, P = 128;
+    static constexpr int T = kTS, P = 128, S = kStages, NP = N + 4;
+    // TMA destinations (each 128-byte aligned; rows of 256 bytes).
     struct Raw {
-        __nv_bfloat16 u[T + 3][P];
-        __nv_bfloat16 a[T][P], b[T][P], z[T][P];
-        __nv_bfloat16 Bm[T][N], Cm[T][N];
+        alignas(128) __nv_bfloat16 u[T + 3][P];
+        alignas(128) __nv_bfloat16 a[T][P];
+        alignas(128) __nv_bfloat16 b[T][P];
+        alignas(128) __nv_bfloat16 z[T][P];
+        alignas(128) __nv_bfloat16 Bm[T][N];
+        alignas(128) __nv_bfloat16 Cm[T][N];
     };
-    alignas(128) Raw raw[2];
-    alignas(128) float bc[2][T * N];   // C: rows t, K = j      (readout B operand, part 1)
-    alignas(128) float bg[2][T * T];   // G: rows t, K = m      (readout B operand, part 2)
-    alignas(128) float bs[2][N * T];   // B^T: rows j, K = m    (state B operand)
-    alignas(16) float brow[2][T][N];   // B rows, fp32, for the Gram
-    float eg[2][T][P];                 // s E_t SiLU(z_t)  (s SiLU(z_t) on the exact path)
-    float dhg[2][T][P];                // D h_t SiLU(z_t)
-    float yacc[T][P];                  // exact path: readout of the first column half
-    float xq0[P], xe0[P], xe1[P];      // per-half decay products of a sub-chunk
-    float elast[2][P];                 // E over the whole sub-chunk
-    int slow[2];
-    uint64_t mbar;
+    // One stage of unpacked sub-chunk operands.
+    struct Stage {
+        alignas(128) float bc[T * N];   // C: rows t, K = j      (readout B operand, part 1)
+        alignas(128) float bg[T * T];   // G: rows t, K = m      (readout B operand, part 2)
+        alignas(128) float bs[N * T];   // B^T: rows j, K = m    (state B operand)
+        alignas(16) float brow[T][NP];  // B rows, fp32, padded against bank conflicts
+        alignas(16) float crow[T][NP];  // C rows, fp32, padded
+        float elast[P];                 // E over the whole sub-chunk
+        int slow;
+    };
+    Raw raw[S];
+    Stage st[S];
+    float xq0[P], xe0[P], xe1[P];       // per-half decay products of a sub-chunk
+    uint64_t loaded[S], full[S], empty[S], mma;
     uint32_t taddr;
     int item, ok;
 };
@@ -85,19 +110,24 @@ struct FwdTcSmem {
 }  // namespace
 
 template <typename Tout, int N, bool CONV>
-__global__ void __launch_bounds__(256, (N == 64 ? 2 : 1))
-scan_fwd_tc_kernel(const FwdParams p) {
+__global__ void __launch_bounds__(384, 1)
+scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
     using Tin = __nv_bfloat16;
     using Cols = TcCols<N>;
     using Sm = FwdTcSmem<N>;
-    constexpr int T = kTS, P = 128, NT = 256, H = T / 2, NH = N / 2;
-    extern __shared__ float4 smem4[];
+    constexpr int T = kTS, P = 128, H = T / 2, S = kStages;
+    constexpr int NPROD = 256, NCONS = 128;
+    extern __shared__ __align__(1024) float4 smem4[];
     Sm& sm = *reinterpret_cast<Sm*>(smem4);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
-    const int ch = tid & (P - 1);   // channel within the block = TMEM lane
-    const int half = tid >> 7;      // token half (unpacking) / column half (state)
+    const bool prod = tid < NPROD;
+    // Producers: channel pch, token half phalf.  Consumers: channel cch.
+    const int pch = tid & (P - 1);
+    const int phalf = (tid >> 7) & 1;
+    const int cch = tid - NPROD;
+    const int ch = prod ? pch : cch;
     const int64_t Bt = p.Bt, L = p.L, d = p.d;
 
     // ------------------------------------------------------------ set-up
@@ -107,7 +137,18 @@ scan_fwd_tc_kernel(const FwdParams p) {
     }
     if (tid == 0) {
         sm.item = atomicAdd(&p.hdr->fwd_ticket, 1);
-        tc::mbar_init(&sm.mbar, 1);
+        for (int s = 0; s < S; ++s) {
+            tc::mbar_init(&sm.loaded[s], 1);
+            tc::mbar_init(&sm.full[s], NPROD);
+            tc::mbar_init(&sm.empty[s], NCONS);
+        }
+        tc::mbar_init(&sm.mma, 1);
+        tma::prefetch_map(&tm.u);
+        tma::prefetch_map(&tm.a);
+        tma::prefetch_map(&tm.b);
+        if (p.z) tma::prefetch_map(&tm.z);
+        tma::prefetch_map(&tm.B);
+        tma::prefetch_map(&tm.C);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -130,14 +171,8 @@ scan_fwd_tc_kernel(const FwdParams p) {
     const bool last_group = (g == p.ngroups - 1);
 
     const int64_t boff = (int64_t)bb * L;
-    const Tin* hu = static_cast<const Tin*>(p.hu) + boff * d;
-    const Tin* ga = static_cast<const Tin*>(p.a) + boff * d;
-    const Tin* gb = static_cast<const Tin*>(p.b) + boff * d;
-    const Tin* gz = p.z ? static_cast<const Tin*>(p.z) + boff * d : nullptr;
-    const Tin* gB = static_cast<const Tin*>(p.B) + boff * N;
-    const Tin* gC = static_cast<const Tin*>(p.C) + boff * N;
+    const bool has_z = p.z != nullptr;
     Tout* gy = static_cast<Tout*>(p.y) + boff * d;
-    const bool vec = ((d * (int64_t)sizeof(Tin)) % 16) == 0;
 
     float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, wb = 0.f, Dc = 0.f;
     if (cvalid) {
@@ -154,80 +189,108 @@ scan_fwd_tc_kernel(const FwdParams p) {
     float* ck_b = p.ckpt + (int64_t)bb * (p.nck + 1) * d * N;
     bool timed_out = false;
 
-    // ---------------------------------------------------------- helpers
+    // ======================================================= producer side
+    // One thread: TMA loads of sub-chunk t0 into raw buffer `buf`.
     auto issue = [&](int64_t t0, int buf, bool full) {
         typename Sm::Raw& r = sm.raw[buf];
-        stage_rows(&r.u[0][0], hu, d, t0 - 3, T + 3, L, c0, P, vec, tid, NT);
-        stage_rows(&r.a[0][0], ga, d, t0, T, tend, c0, P, vec, tid, NT);
-        stage_rows(&r.b[0][0], gb, d, t0, T, tend, c0, P, vec, tid, NT);
-        if (full && gz) stage_rows(&r.z[0][0], gz, d, t0, T, tend, c0, P, vec, tid, NT);
-        stage_rows(&r.Bm[0][0], gB, N, t0, T, tend, 0, N, true, tid, NT);
-        if (full) stage_rows(&r.Cm[0][0], gC, N, t0, T, tend, 0, N, true, tid, NT);
-        cp_async_commit();
+        uint64_t* mb = &sm.loaded[buf];
+        const bool zz = full && has_z;
+        const uint32_t bytes = (uint32_t)sizeof(Tin) *
+                               ((T + 3) * P + 2 * T * P + (zz ? T * P : 0) + (full ? 2 : 1) * T * N);
+        tma::expect_tx(mb, bytes);
+        const int x = (int)c0, y = (int)t0, zb = bb;
+        tma::load_3d(&r.u[0][0], &tm.u, x, y - 3, zb, mb);
+        tma::load_3d(&r.a[0][0], &tm.a, x, y, zb, mb);
+        tma::load_3d(&r.b[0][0], &tm.b, x, y, zb, mb);
+        if (zz) tma::load_3d(&r.z[0][0], &tm.z, x, y, zb, mb);
+        tma::load_3d(&r.Bm[0][0], &tm.B, 0, y, zb, mb);
+        if (full) tma::load_3d(&r.Cm[0][0], &tm.C, 0, y, zb, mb);
     };
-    // Unpack sub-chunk (t0, raw buffer `buf`) into operand set `pr`.
-    auto prep = [&](int64_t t0, int buf, int pr, bool full) {
+    auto bf4 = [](const __nv_bfloat16* src) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(src);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        return make_float4(lo.x, lo.y, hi.x, hi.y);
+    };
+    // Unpack sub-chunk (t0, raw buffer `buf`) into stage `s` (producers only).
+    auto prep = [&](int64_t t0, int buf, int s, bool full) {
         const typename Sm::Raw& r = sm.raw[buf];
-        // Per-token operands: four consecutive d_state entries per step.
-        for (int e = tid; e < T * N / 4; e += NT) {
+        typename Sm::Stage& stg = sm.st[s];
+        // B and C rows to fp32 (padded rows: conflict-free reads below).
+        for (int e = tid; e < T * N / 4; e += NPROD) {
             const int tt = e / (N / 4), j = (e % (N / 4)) * 4;
-            const uint2 braw = *reinterpret_cast<const uint2*>(&r.Bm[tt][j]);
-            const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&braw.x));
-            const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&braw.y));
-            *reinterpret_cast<float4*>(&sm.brow[pr][tt][j]) = make_float4(b01.x, b01.y, b23.x, b23.y);
-            sm.bs[pr][tc::kmajor_offset(j + 0, tt, T) >> 2] = b01.x;
-            sm.bs[pr][tc::kmajor_offset(j + 1, tt, T) >> 2] = b01.y;
-            sm.bs[pr][tc::kmajor_offset(j + 2, tt, T) >> 2] = b23.x;
-            sm.bs[pr][tc::kmajor_offset(j + 3, tt, T) >> 2] = b23.y;
-            if (full) {
-                const uint2 craw = *reinterpret_cast<const uint2*>(&r.Cm[tt][j]);
-                const float2 c01 =
-                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&craw.x));
-                const float2 c23 =
-                    __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&craw.y));
-                *reinterpret_cast<float4*>(&sm.bc[pr][tc::kmajor_offset(tt, j, N) >> 2]) =
-                    make_float4(c01.x, c01.y, c23.x, c23.y);
-            }
+            *reinterpret_cast<float4*>(&stg.brow[tt][j]) = bf4(&r.Bm[tt][j]);
+            if (full) *reinterpret_cast<float4*>(&stg.crow[tt][j]) = bf4(&r.Cm[tt][j]);
         }
+        // Tokens of this thread's half inside [t0, tend) (0 for a padding channel).
+        const int nv = cvalid ? (int)max((int64_t)0, min64((int64_t)H, tend - t0 - phalf * H)) : 0;
         // Per-channel values: this thread's 8 tokens.
         float qv[H], fv[H], hv[H];
         float Qh = 1.f, Eh = 1.f;
 #pragma unroll
         for (int k = 0; k < H; ++k) {
-            const int tt = half * H + k;
-            const bool valid = cvalid && (t0 + tt < tend);
-            qv[k] = valid ? 1.f + __expf(-to_f(r.a[tt][ch])) : 1.f;
+            const int tt = phalf * H + k;
+            const bool valid = k < nv;
+            qv[k] = valid ? 1.f + __expf(-to_f(r.a[tt][pch])) : 1.f;
             fv[k] = rcpa_(qv[k]);
             Qh *= qv[k];
             Eh *= fv[k];
-            float h = 0.f;
-            if (valid) {
-                if (CONV) {
-                    h = silua_(wb + w0 * to_f(r.u[tt][ch]) + w1 * to_f(r.u[tt + 1][ch]) +
-                               w2 * to_f(r.u[tt + 2][ch]) + w3 * to_f(r.u[tt + 3][ch]));
-                } else {
-                    h = to_f(r.u[tt + 3][ch]);
-                }
+            float h;
+            if (CONV) {
+                h = silua_(wb + w0 * to_f(r.u[tt][pch]) + w1 * to_f(r.u[tt + 1][pch]) +
+                           w2 * to_f(r.u[tt + 2][pch]) + w3 * to_f(r.u[tt + 3][pch]));
+            } else {
+                h = to_f(r.u[tt + 3][pch]);
             }
-            hv[k] = h;
+            hv[k] = valid ? h : 0.f;
         }
-        if (half == 0) {
-            sm.xq0[ch] = Qh;
-            sm.xe0[ch] = Eh;
+        if (phalf == 0) {
+            sm.xq0[pch] = Qh;
+            sm.xe0[pch] = Eh;
         } else {
-            sm.xe1[ch] = Eh;
+            sm.xe1[pch] = Eh;
         }
-        __syncthreads();
-        const float Q0 = sm.xq0[ch], E0 = sm.xe0[ch], E1 = sm.xe1[ch];
-        const int slow = __syncthreads_or((half == 1 && !(Q0 * Qh <= kTcBound)) ? 1 : 0);
+        tc::named_bar(1, NPROD);
+        const float Q0 = sm.xq0[pch], E0 = sm.xe0[pch], E1 = sm.xe1[pch];
+        const bool slow = tc::named_bar_or(1, NPROD, phalf == 1 && !(Q0 * Qh <= kTcBound));
+        if (!slow) {
+            // K-major operand tiles.  bc: a quarter warp fills one 8-row core
+            // matrix; bs: one thread gathers 4 consecutive m of one row j.
+            for (int e = tid; e < T * N / 4; e += NPROD) {
+                if (full) {
+                    const int rest = e >> 3;
+                    const int tt = (rest & 1) * 8 + (e & 7), j = (rest >> 1) * 4;
+                    *reinterpret_cast<float4*>(&stg.bc[tc::kmajor_offset(tt, j, N) >> 2]) =
+                        *reinterpret_cast<const float4*>(&stg.crow[tt][j]);
+                }
+                const int jj = e % N, m0 = (e / N) * 4;
+                *reinterpret_cast<float4*>(&stg.bs[tc::kmajor_offset(jj, m0, T) >> 2]) =
+                    make_float4(stg.brow[m0][jj], stg.brow[m0 + 1][jj], stg.brow[m0 + 2][jj],
+                                stg.brow[m0 + 3][jj]);
+            }
+            if (full) {
+                // G[t][m] = C_t . B_m for m <= t (one entry per producer thread).
+                const int tt = tid / T, mm = tid % T;
+                float2 acc = make_float2(0.f, 0.f);
+                if (mm <= tt) {
+#pragma unroll 4
+                    for (int j = 0; j < N; j += 4) {
+                        const float4 cv = *reinterpret_cast<const float4*>(&stg.crow[tt][j]);
+                        const float4 bv = *reinterpret_cast<const float4*>(&stg.brow[mm][j]);
+                        acc = __ffma2_rn(make_float2(cv.x, cv.y), make_float2(bv.x, bv.y), acc);
+                        acc = __ffma2_rn(make_float2(cv.z, cv.w), make_float2(bv.z, bv.w), acc);
+                    }
+                }
+                stg.bg[tc::kmajor_offset(tt, mm, T) >> 2] = acc.x + acc.y;
+            }
+        }
         const float Elast = E0 * E1;
-        float Q = half ? Q0 : 1.f, E = half ? E0 : 1.f;
-        float Wv[H], Vv[H];
+        float Q = phalf ? Q0 : 1.f, E = phalf ? E0 : 1.f;
+        float Wv[H], Vv[H], Gv[H], Dv[H];
 #pragma unroll
         for (int k = 0; k < H; ++k) {
-            const int tt = half * H + k;
-            const bool valid = cvalid && (t0 + tt < tend);
-            const float v = valid ? sigmoida_(to_f(r.b[tt][ch])) * hv[k] : 0.f;
+            const int tt = phalf * H + k;
+            const float v = sigmoida_(to_f(r.b[tt][pch])) * hv[k];  // 0 past the end (h = 0)
             E *= fv[k];
             Q *= qv[k];
             if (slow) {
@@ -238,60 +301,52 @@ scan_fwd_tc_kernel(const FwdParams p) {
                 Vv[k] = v * Q * Elast;   // v_m E_T / E_m
             }
             if (full) {
-                const float gg = (valid && gz) ? silua_(to_f(r.z[tt][ch])) : 1.f;
-                sm.eg[pr][tt][ch] = slow ? scale * gg : scale * E * gg;
-                sm.dhg[pr][tt][ch] = Dc * hv[k] * gg;
+                const float gg = has_z ? silua_(to_f(r.z[tt][pch])) : 1.f;
+                Gv[k] = slow ? scale * gg : scale * E * gg;
+                Dv[k] = Dc * hv[k] * gg;
             }
         }
-        if (half == 0) sm.elast[pr][ch] = Elast;
-        if (tid == 0) sm.slow[pr] = slow;
-        tc::tmem_st8(tbase + lane + Cols::W + pr * T + half * H, Wv);
-        tc::tmem_st8(tbase + lane + Cols::V + pr * T + half * H, Vv);
-        tc::tmem_st_wait();
-        if (full && !slow) {
-            __syncthreads();  // bc, brow complete
-            // G[t][m] = C_t . B_m for m <= t (one entry per thread).
-            const int tt = tid / T, mm = tid % T;
-            float a = 0.f;
-            if (mm <= tt) {
-#pragma unroll 4
-                for (int j = 0; j < N; j += 4) {
-                    const float4 cv = *reinterpret_cast<const float4*>(
-                        &sm.bc[pr][tc::kmajor_offset(tt, j, N) >> 2]);
-                    const float4 bv = *reinterpret_cast<const float4*>(&sm.brow[pr][mm][j]);
-                    a = fmaf(cv.x, bv.x, fmaf(cv.y, bv.y, fmaf(cv.z, bv.z, fmaf(cv.w, bv.w, a))));
-                }
-            }
-            sm.bg[pr][tc::kmajor_offset(tt, mm, T) >> 2] = a;
-        }
-    };
-    // Issue the sub-chunk's MMAs (one thread) and commit them to the barrier.
-    auto issue_mma = [&](int pr, bool full) {
-        const uint32_t id_r = tc::idesc_tf32(128, T);
-        const uint32_t id_s = tc::idesc_tf32(128, N);
+        if (phalf == 0) stg.elast[pch] = Elast;
+        if (tid == 0) stg.slow = slow ? 1 : 0;
+        const uint32_t col = tbase + lane + s * T + phalf * H;
+        tc::tmem_st8(col + Cols::W, Wv);
+        tc::tmem_st8(col + Cols::V, Vv);
         if (full) {
-            const uint32_t sc = tc::smem_u32(&sm.bc[pr][0]);
+            tc::tmem_st8(col + Cols::EG, Gv);
+            tc::tmem_st8(col + Cols::DH, Dv);
+        }
+        tc::tmem_st_wait();
+    };
+
+    // ======================================================= consumer side
+    // Issue the sub-chunk's MMAs (one consumer thread) and commit them.
+    auto issue_mma = [&](int s, bool full) {
+        const typename Sm::Stage& stg = sm.st[s];
+        constexpr uint32_t id_r = tc::idesc_tf32(128, T);
+        constexpr uint32_t id_s = tc::idesc_tf32(128, N);
+        if (full) {
+            const uint32_t sc = tc::smem_u32(&stg.bc[0]);
 #pragma unroll
             for (int ks = 0; ks < N / 8; ++ks)
                 tc::mma_tf32_ts(tbase + Cols::DR, tbase + Cols::X + ks * 8,
                                 tc::sdesc(sc + ks * 256, 128, 32 * N), id_r, ks > 0 ? 1u : 0u);
-            const uint32_t sg = tc::smem_u32(&sm.bg[pr][0]);
+            const uint32_t sg = tc::smem_u32(&stg.bg[0]);
 #pragma unroll
             for (int ks = 0; ks < T / 8; ++ks)
-                tc::mma_tf32_ts(tbase + Cols::DR, tbase + Cols::W + pr * T + ks * 8,
+                tc::mma_tf32_ts(tbase + Cols::DR, tbase + Cols::W + s * T + ks * 8,
                                 tc::sdesc(sg + ks * 256, 128, 32 * T), id_r, 1u);
         }
-        const uint32_t ss = tc::smem_u32(&sm.bs[pr][0]);
+        const uint32_t ss = tc::smem_u32(&stg.bs[0]);
 #pragma unroll
         for (int ks = 0; ks < T / 8; ++ks)
-            tc::mma_tf32_ts(tbase + Cols::DS, tbase + Cols::V + pr * T + ks * 8,
+            tc::mma_tf32_ts(tbase + Cols::DS, tbase + Cols::V + s * T + ks * 8,
                             tc::sdesc(ss + ks * 256, 128, 32 * T), id_s, ks > 0 ? 1u : 0u);
-        tc::mma_commit(&sm.mbar);
+        tc::mma_commit(&sm.mma);
     };
-    // TMEM state row <-> global row (each thread moves its column half).
+    // TMEM state row <-> global row (consumers; full rows).
     auto state_from = [&](const float* src, bool cg) {
 #pragma unroll
-        for (int n0 = half * NH; n0 < half * NH + NH; n0 += 16) {
+        for (int n0 = 0; n0 < N; n0 += 16) {
             float v[16];
 #pragma unroll
             for (int k = 0; k < 16; k += 4) {
@@ -300,7 +355,10 @@ scan_fwd_tc_kernel(const FwdParams p) {
                     const float4* s4 = reinterpret_cast<const float4*>(src + c * N + n0 + k);
                     v4 = cg ? __ldcg(s4) : *s4;
                 }
-                v[k] = v4.x; v[k + 1] = v4.y; v[k + 2] = v4.z; v[k + 3] = v4.w;
+                v[k] = v4.x;
+                v[k + 1] = v4.y;
+                v[k + 2] = v4.z;
+                v[k + 3] = v4.w;
             }
             tc::tmem_st16(tbase + lane + Cols::X + n0, v);
         }
@@ -308,7 +366,7 @@ scan_fwd_tc_kernel(const FwdParams p) {
     };
     auto state_to = [&](float* dst) {
 #pragma unroll
-        for (int n0 = half * NH; n0 < half * NH + NH; n0 += 16) {
+        for (int n0 = 0; n0 < N; n0 += 16) {
             float v[16];
             tc::tmem_ld16(tbase + lane + Cols::X + n0, v);
             tc::tmem_ld_wait();
@@ -320,28 +378,25 @@ scan_fwd_tc_kernel(const FwdParams p) {
             }
         }
     };
-    // Sub-chunk i's results: outputs (full) and the next state.
-    float logP = 0.f;  // log of the decay product over the pass
-    auto epilogue = [&](int64_t t0, int pr, bool full) {
-        const float El = sm.elast[pr][ch];
-        if (!sm.slow[pr]) {
+    float logP = 0.f;  // log of the decay product over the pass (consumers)
+    auto epilogue = [&](int64_t t0, int s, bool full) {
+        const typename Sm::Stage& stg = sm.st[s];
+        const int ny = cvalid ? (int)min64((int64_t)T, tend - t0) : 0;  // outputs to write
+        Tout* yrow = gy + t0 * d + c;
+        if (!stg.slow) {
+            const float El = stg.elast[cch];
             if (full) {
-                float dr[H];
-                tc::tmem_ld8(tbase + lane + Cols::DR + half * H, dr);
+                float dr[16], eg[16], dh[16];
+                tc::tmem_ld16(tbase + lane + Cols::DR, dr);
+                tc::tmem_ld16(tbase + lane + Cols::EG + s * T, eg);
+                tc::tmem_ld16(tbase + lane + Cols::DH + s * T, dh);
                 tc::tmem_ld_wait();
-                if (cvalid) {
 #pragma unroll
-                    for (int k = 0; k < H; ++k) {
-                        const int tt = half * H + k;
-                        const int64_t t = t0 + tt;
-                        if (t < tend)
-                            gy[t * d + c] =
-                                from_f<Tout>(fmaf(sm.eg[pr][tt][ch], dr[k], sm.dhg[pr][tt][ch]));
-                    }
-                }
+                for (int tt = 0; tt < T; ++tt)
+                    if (tt < ny) yrow[tt * d] = from_f<Tout>(fmaf(eg[tt], dr[tt], dh[tt]));
             }
 #pragma unroll
-            for (int n0 = half * NH; n0 < half * NH + NH; n0 += 16) {
+            for (int n0 = 0; n0 < N; n0 += 16) {
                 float x[16], s2[16];
                 tc::tmem_ld16(tbase + lane + Cols::X + n0, x);
                 tc::tmem_ld16(tbase + lane + Cols::DS + n0, s2);
@@ -352,15 +407,14 @@ scan_fwd_tc_kernel(const FwdParams p) {
             }
             logP += __logf(El);
         } else {
-            // Exact path: x <- f x + (i h) B token by token, y from x . C, each
-            // thread on its column half; the halves' readouts meet in yacc.
+            // Exact path: x <- f x + (i h) B token by token, y from x . C.
             float vv[16], ff[16], yp[16];
-            tc::tmem_ld16(tbase + lane + Cols::W + pr * T, vv);
-            tc::tmem_ld16(tbase + lane + Cols::V + pr * T, ff);
+            tc::tmem_ld16(tbase + lane + Cols::W + s * T, vv);
+            tc::tmem_ld16(tbase + lane + Cols::V + s * T, ff);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int tt = 0; tt < T; ++tt) yp[tt] = 0.f;
-            for (int n0 = half * NH; n0 < half * NH + NH; n0 += 16) {
+            for (int n0 = 0; n0 < N; n0 += 16) {
                 float x[16];
                 tc::tmem_ld16(tbase + lane + Cols::X + n0, x);
                 tc::tmem_ld_wait();
@@ -369,29 +423,21 @@ scan_fwd_tc_kernel(const FwdParams p) {
                     float acc = 0.f;
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
-                        x[k] = fmaf(ff[tt], x[k], vv[tt] * sm.brow[pr][tt][n0 + k]);
-                        if (full)
-                            acc = fmaf(x[k], sm.bc[pr][tc::kmajor_offset(tt, n0 + k, N) >> 2], acc);
+                        x[k] = fmaf(ff[tt], x[k], vv[tt] * stg.brow[tt][n0 + k]);
+                        if (full) acc = fmaf(x[k], stg.crow[tt][n0 + k], acc);
                     }
                     yp[tt] += acc;
                 }
                 tc::tmem_st16(tbase + lane + Cols::X + n0, x);
             }
             if (full) {
-                if (half == 0) {
+                float eg[16], dh[16];
+                tc::tmem_ld16(tbase + lane + Cols::EG + s * T, eg);
+                tc::tmem_ld16(tbase + lane + Cols::DH + s * T, dh);
+                tc::tmem_ld_wait();
 #pragma unroll
-                    for (int tt = 0; tt < T; ++tt) sm.yacc[tt][ch] = yp[tt];
-                }
-                __syncthreads();
-                if (half == 1 && cvalid) {
-#pragma unroll
-                    for (int tt = 0; tt < T; ++tt) {
-                        const int64_t t = t0 + tt;
-                        if (t < tend)
-                            gy[t * d + c] = from_f<Tout>(fmaf(
-                                sm.eg[pr][tt][ch], yp[tt] + sm.yacc[tt][ch], sm.dhg[pr][tt][ch]));
-                    }
-                }
+                for (int tt = 0; tt < T; ++tt)
+                    if (tt < ny) yrow[tt * d] = from_f<Tout>(fmaf(eg[tt], yp[tt], dh[tt]));
             }
             float lp = 0.f;
 #pragma unroll
@@ -400,54 +446,68 @@ scan_fwd_tc_kernel(const FwdParams p) {
         }
         tc::tmem_st_wait();
     };
-    uint32_t phase = 0;
-    // One pass over the group's sub-chunks (full: readout, outputs, checkpoints).
+
+    // ============================================================ one pass
+    int gbase = 0;           // sub-chunks through the stage ring so far
+    uint32_t mma_phase = 0;  // consumers: parity of the next MMA completion
     auto run_pass = [&](bool full) {
         const int nsc = (int)((tend - tbeg + T - 1) / T);
-        issue(tbeg, 0, full);
-        if (nsc > 1) {
-            issue(tbeg + T, 1, full);
-            cp_async_wait<1>();
+        if (prod) {
+            // Raw buffer and operand stage of sub-chunk gi are both gi % S.
+            if (tid == 0) {
+                issue(tbeg, gbase % S, full);
+                if (nsc > 1) issue(tbeg + T, (gbase + 1) % S, full);
+            }
+            for (int i = 0; i < nsc; ++i) {
+                const int gi = gbase + i, s = gi % S, u = gi / S;
+                const int64_t t0 = tbeg + (int64_t)i * T;
+                // Buffer (gi + 2) % S was last read in the previous iteration.
+                if (tid == 0 && i + 2 < nsc) issue(t0 + 2 * T, (gi + 2) % S, full);
+                if (!tc::mbar_wait(&sm.loaded[s], u & 1, kMbarSpin)) timed_out = true;
+                if (u > 0 && !tc::mbar_wait(&sm.empty[s], (u - 1) & 1, kMbarSpin)) timed_out = true;
+                prep(t0, s, s, full);
+                tc::fence_proxy_async();
+                tc::fence_before_sync();
+                tc::mbar_arrive(&sm.full[s]);
+                tc::named_bar(1, NPROD);  // raw sub-chunk i consumed by every producer
+            }
         } else {
-            cp_async_wait<0>();
+            for (int i = 0; i < nsc; ++i) {
+                const int gi = gbase + i, s = gi % S;
+                const int64_t t0 = tbeg + (int64_t)i * T;
+                if (i == 0) {
+                    if (!tc::mbar_wait(&sm.full[s], (gi / S) & 1, kMbarSpin)) timed_out = true;
+                    tc::fence_after_sync();
+                    if (cch == 0 && !sm.st[s].slow) issue_mma(s, full);
+                }
+                if (!sm.st[s].slow) {
+                    if (!tc::mbar_wait(&sm.mma, mma_phase, kMbarSpin)) timed_out = true;
+                    mma_phase ^= 1u;
+                }
+                tc::fence_after_sync();
+                epilogue(t0, s, full);
+                if (full) {
+                    const int64_t tnext = t0 + T;
+                    if (tnext < tend && tnext % p.T_ck == 0)
+                        state_to(ck_b + (tnext / p.T_ck) * d * N);
+                }
+                tc::fence_before_sync();
+                tc::mbar_arrive(&sm.empty[s]);
+                if (i + 1 < nsc) {
+                    const int gn = gi + 1, sn = gn % S;
+                    if (!tc::mbar_wait(&sm.full[sn], (gn / S) & 1, kMbarSpin)) timed_out = true;
+                    tc::named_bar(2, NCONS);  // every X row updated
+                    if (cch == 0) {
+                        tc::fence_after_sync();
+                        if (!sm.st[sn].slow) issue_mma(sn, full);
+                    }
+                }
+            }
         }
-        __syncthreads();
-        prep(tbeg, 0, 0, full);
-        tc::fence_proxy_async();
+        gbase += nsc;
         tc::fence_before_sync();
         __syncthreads();
-        if (tid == 0) {
-            tc::fence_after_sync();
-            if (!sm.slow[0]) issue_mma(0, full);
-        }
-        for (int i = 0; i < nsc; ++i) {
-            const int pr = i & 1;
-            const int64_t t0 = tbeg + (int64_t)i * T;
-            const bool more = i + 1 < nsc;
-            if (more) {
-                cp_async_wait<0>();
-                __syncthreads();  // raw (i+1) visible; raw (i) free
-                if (i + 2 < nsc) issue(t0 + 2 * T, i & 1, full);
-                prep(t0 + T, (i + 1) & 1, pr ^ 1, full);
-            }
-            if (!sm.slow[pr]) {
-                if (!tc::mbar_wait(&sm.mbar, phase, 1LL << 24)) timed_out = true;
-                phase ^= 1u;
-            }
-            tc::fence_after_sync();
-            epilogue(t0, pr, full);
-            if (full) {
-                const int64_t tnext = t0 + T;
-                if (tnext < tend && tnext % p.T_ck == 0) state_to(ck_b + (tnext / p.T_ck) * d * N);
-            }
-            tc::fence_proxy_async();
-            tc::fence_before_sync();
-            __syncthreads();
-            if (more && tid == 0) {
-                tc::fence_after_sync();
-                if (!sm.slow[pr ^ 1]) issue_mma(pr ^ 1, full);
-            }
-        }
+        tc::fence_after_sync();
     };
 
     // ------------------------------------------ early pass and carry chain
@@ -458,38 +518,43 @@ scan_fwd_tc_kernel(const FwdParams p) {
     float* ck_start = ck_b + (int64_t)seg0 * d * N;
     float* ck_end = ck_b + (int64_t)seg1 * d * N;
     bool ok = true;
-    if (!last_group) {
-        state_from(g == 0 ? x0b : nullptr, false);
+    auto sync_all = [&]() {
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
-        logP = 0.f;
+    };
+    if (!last_group) {
+        if (!prod) state_from(g == 0 ? x0b : nullptr, false);
+        sync_all();
         run_pass(false);
         if (g > 0) {
-            const float Pf = __expf(logP);
             if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
             __syncthreads();
             ok = sm.ok != 0;
+            if (!prod) {
+                // X_end += (product of f over the group) X_start
+                const float Pf = __expf(logP);
 #pragma unroll
-            for (int n0 = half * NH; n0 < half * NH + NH; n0 += 16) {
-                float x[16];
-                tc::tmem_ld16(tbase + lane + Cols::X + n0, x);
-                tc::tmem_ld_wait();
+                for (int n0 = 0; n0 < N; n0 += 16) {
+                    float x[16];
+                    tc::tmem_ld16(tbase + lane + Cols::X + n0, x);
+                    tc::tmem_ld_wait();
 #pragma unroll
-                for (int k = 0; k < 16; k += 4) {
-                    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (ok && cvalid)
-                        v4 = __ldcg(reinterpret_cast<const float4*>(ck_start + c * N + n0 + k));
-                    x[k] = fmaf(Pf, v4.x, x[k]);
-                    x[k + 1] = fmaf(Pf, v4.y, x[k + 1]);
-                    x[k + 2] = fmaf(Pf, v4.z, x[k + 2]);
-                    x[k + 3] = fmaf(Pf, v4.w, x[k + 3]);
+                    for (int k = 0; k < 16; k += 4) {
+                        float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (ok && cvalid)
+                            v4 = __ldcg(reinterpret_cast<const float4*>(ck_start + c * N + n0 + k));
+                        x[k] = fmaf(Pf, v4.x, x[k]);
+                        x[k + 1] = fmaf(Pf, v4.y, x[k + 1]);
+                        x[k + 2] = fmaf(Pf, v4.z, x[k + 2]);
+                        x[k + 3] = fmaf(Pf, v4.w, x[k + 3]);
+                    }
+                    tc::tmem_st16(tbase + lane + Cols::X + n0, x);
                 }
-                tc::tmem_st16(tbase + lane + Cols::X + n0, x);
+                tc::tmem_st_wait();
             }
-            tc::tmem_st_wait();
         }
-        state_to(ck_end);
+        if (!prod) state_to(ck_end);
         __threadfence();
         __syncthreads();
         if (tid == 0 && !(g == 0 && p.fault_skip_publish)) st_release(flag_mine, 1);
@@ -498,50 +563,56 @@ scan_fwd_tc_kernel(const FwdParams p) {
         __syncthreads();
         ok = sm.ok != 0;
     }
-    if (g > 0) {
-        state_from(ok ? ck_start : nullptr, true);
-    } else {
-        state_from(x0b, false);
-        state_to(ck_b);  // checkpoint 0 = initial state
+    if (!prod) {
+        if (g > 0) {
+            state_from(ok ? ck_start : nullptr, true);
+        } else {
+            state_from(x0b, false);
+            state_to(ck_b);  // checkpoint 0 = initial state
+        }
     }
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
+    sync_all();
 
     // ------------------------------------------------------- full pass
     run_pass(true);
-    if (last_group) {
+    if (last_group && !prod) {
         state_to(ck_b + (int64_t)p.nck * d * N);
         if (p.x_final) state_to(p.x_final + (int64_t)bb * d * N);
     }
-    if (timed_out && tid == 0) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
+    if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
 
     // ---------------------------------------------------------- teardown
-    tc::fence_before_sync();
-    __syncthreads();
+    sync_all();
     if (warp == 0) tc::tmem_dealloc(tbase, Cols::ALLOC);
 }
 
 template <typename Tout, int N, bool CONV>
 static cudaError_t launch_fwd_tc_t(const FwdParams& p, cudaStream_t st) {
-    // At least enough shared memory that no more blocks share an SM than its
-    // 512 tensor-memory columns can hold.
-    const size_t need = sizeof(FwdTcSmem<N>);
-    const size_t floor_bytes = TcCols<N>::ALLOC == 512 ? (size_t)120 * 1024 : (size_t)80 * 1024;
-    const size_t smem = need > floor_bytes ? need : floor_bytes;
+    FwdTmaps tm;
+    memset(&tm, 0, sizeof(tm));
+    const int T = kTS;
+    bool ok = tma_encode_bf16_3d(&tm.u, p.hu, p.Bt, p.L, p.d, T + 3, 128) &&
+              tma_encode_bf16_3d(&tm.a, p.a, p.Bt, p.L, p.d, T, 128) &&
+              tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, T, 128) &&
+              tma_encode_bf16_3d(&tm.B, p.B, p.Bt, p.L, N, T, N) &&
+              tma_encode_bf16_3d(&tm.C, p.C, p.Bt, p.L, N, T, N);
+    if (ok && p.z) ok = tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, T, 128);
+    if (!ok) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(FwdTcSmem<N>);
     auto kern = scan_fwd_tc_kernel<Tout, N, CONV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = p.ngroups * (int)p.Bt * p.ntiles;
-    kern<<<grid, 256, smem, st>>>(p);
+    kern<<<grid, 384, smem, st>>>(p, tm);
     return cudaGetLastError();
 }
 
 int fwd_tc_channels_per_block() { return 128; }
 
-bool fwd_tc_supported(int dtype, int64_t N) {
-    return dtype == NAJU_BF16 && (N == 64 || N == 128);
+bool fwd_tc_supported(int dtype, int64_t N, int64_t d) {
+    // TMA rows must be a multiple of 16 bytes: d_inner % 8 == 0.
+    return dtype == NAJU_BF16 && (N == 64 || N == 128) && d % 8 == 0;
 }
 
 cudaError_t launch_scan_fwd_tc(const FwdParams& p, int out_dtype, cudaStream_t st) {

@@ -31,6 +31,31 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
     return d;
 }
 
+// Byte offset of element (row, k) of an R x 128 K-major tile in the 128-byte
+// swizzled layout: 8-row x 128-byte atoms (1024 bytes; rows 128 bytes apart,
+// the 16-byte chunks of row r XOR-permuted by r % 8), 8-row groups 1024 bytes
+// apart, the four 32-element K atoms R * 128 bytes apart.  The tile base must
+// be 1024-byte aligned.  A warp writing one row's 32 consecutive k (or one k
+// of 32 consecutive rows of an atom column) touches 32 distinct banks.
+__host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int k, int R) {
+    const int r = row & 7;
+    return (uint32_t)((k >> 5) * (R * 128) + (row >> 3) * 1024 + r * 128 +
+                      ((((k >> 2) & 7) ^ r) << 4) + (k & 3) * 4);
+}
+
+// Descriptor of the 128-byte swizzled K-major layout above (SBO 1024; the
+// leading offset is not used by swizzled K-major operands).  For K step ks
+// (8 tf32) the start address is base + (ks / 4) * R * 128 + (ks % 4) * 32.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
 // Instruction descriptor: D fp32, A and B tf32, both K-major, M x N.
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
     return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
@@ -130,6 +155,15 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T for one K = 8 step (tf32), issued by one thread.
+__device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 // Arrive on an mbarrier when all previously issued MMAs of this thread finish.

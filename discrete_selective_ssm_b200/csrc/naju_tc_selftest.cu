@@ -1,8 +1,9 @@
-// Self-test of the tensor-core building block used by the tensor-core scan:
-// D[128 x N] = A[128 x K] * B[N x K]^T with A staged in tensor memory, B in
-// shared memory (no-swizzle K-major core matrices) and D in tensor memory,
-// kind::tf32, K = 8 per instruction.  Exposed through naju_testing.h so the
-// test suite can check the operand conventions against a host product.
+// Self-tests of the tensor-core building blocks used by the tensor-core scan:
+// D[128 x N] = A[128 x K] * B[N x K]^T, kind::tf32, K = 8 per instruction,
+// D in tensor memory; A either in tensor memory or in shared memory, shared
+// operands either no-swizzle K-major core matrices or the 128-byte swizzled
+// K-major layout.  Exposed through naju_testing.h so the test suite can check
+// the operand conventions against a host product.
 #include "naju.h"
 #include "naju_common.cuh"
 #include "naju_tc.cuh"
@@ -71,6 +72,72 @@ tc_selftest_kernel(const float* __restrict__ A, const float* __restrict__ B,
     if (warp == 0) tc::tmem_dealloc(tbase, ncols);
 }
 
+
+// Both operands from shared memory.  A is stored as an R x K tile (R = 64 or
+// 128) while the MMA always reads 128 rows: rows past R read other bytes of
+// the A region (zeros here), which is how a 64-row operand rides an M = 128
+// MMA.  swz_a / swz_b select the 128-byte swizzled layout (K % 32 == 0).
+__global__ void __launch_bounds__(128, 1)
+tc_selftest_ss_kernel(const float* __restrict__ A, const float* __restrict__ B,
+                      float* __restrict__ D, int N, int K, int R, int swz_a, int swz_b,
+                      uint32_t ncols, int* status) {
+    extern __shared__ __align__(1024) float4 smem4[];
+    unsigned char* sa = reinterpret_cast<unsigned char*>(smem4);
+    unsigned char* sb = sa + (size_t)128 * K * 4;
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t taddr_s;
+    const int tid = threadIdx.x, warp = tid / 32;
+
+    if (warp == 0) {
+        tc::tmem_alloc(&taddr_s, ncols);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) tc::mbar_init(&mbar, 1);
+    for (int e = tid; e < 128 * K; e += 128) reinterpret_cast<float*>(sa)[e] = 0.f;
+    __syncthreads();
+    for (int e = tid; e < R * K; e += 128) {
+        const int row = e / K, k = e % K;
+        const uint32_t off = swz_a ? tc::sw128_offset(row, k, R) : tc::kmajor_offset(row, k, K);
+        *reinterpret_cast<float*>(sa + off) = A[e];
+    }
+    for (int e = tid; e < N * K; e += 128) {
+        const int row = e / K, k = e % K;
+        const uint32_t off = swz_b ? tc::sw128_offset(row, k, N) : tc::kmajor_offset(row, k, K);
+        *reinterpret_cast<float*>(sb + off) = B[e];
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = taddr_s;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    if (tid == 0) {
+        const uint32_t idesc = tc::idesc_tf32(128, N);
+        const uint32_t abase = tc::smem_u32(sa), bbase = tc::smem_u32(sb);
+        for (int ks = 0; ks < K / 8; ++ks) {
+            const uint64_t ad = swz_a ? tc::sdesc_sw128(abase + (ks >> 2) * R * 128 + (ks & 3) * 32)
+                                      : tc::sdesc(abase + ks * 256, 128, 32 * K);
+            const uint64_t bd = swz_b ? tc::sdesc_sw128(bbase + (ks >> 2) * N * 128 + (ks & 3) * 32)
+                                      : tc::sdesc(bbase + ks * 256, 128, 32 * K);
+            tc::mma_tf32_ss(tbase, ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&mbar);
+    }
+    const bool done = tc::mbar_wait(&mbar, 0, 1LL << 22);
+    if (!done && tid == 0) atomicOr(status, 1 << NAJU_ERR_TIMEOUT);
+    tc::fence_after_sync();
+    for (int n0 = 0; n0 < N; n0 += 16) {
+        float v[16];
+        tc::tmem_ld16(tbase + lane_off + n0, v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) D[tid * N + n0 + i] = done ? v[i] : __int_as_float(0x7fc00000);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, ncols);
+}
+
 }  // namespace naju
 
 extern "C" naju_status naju_testing_tc_mma(int32_t N, int32_t K, const float* A, const float* B,
@@ -86,5 +153,26 @@ extern "C" naju_status naju_testing_tc_mma(int32_t N, int32_t K, const float* A,
     if (e != cudaSuccess) return NAJU_ERR_CUDA;
     naju::tc_selftest_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(A, B, D, N, K,
                                                                                  ncols, status);
+    return cudaGetLastError() == cudaSuccess ? NAJU_OK : NAJU_ERR_CUDA;
+}
+
+extern "C" naju_status naju_testing_tc_mma_ss(int32_t N, int32_t K, int32_t rows_a,
+                                              int32_t swz_a, int32_t swz_b, const float* A,
+                                              const float* B, float* D, int* status,
+                                              void* stream) {
+    if (!A || !B || !D || !status) return NAJU_ERR_INVALID_ARG;
+    if (N < 16 || N > 128 || N % 16 != 0 || K < 16 || K > 128 || K % 16 != 0 ||
+        (rows_a != 64 && rows_a != 128))
+        return NAJU_ERR_UNSUPPORTED;
+    if ((swz_a || swz_b) && K % 32 != 0) return NAJU_ERR_UNSUPPORTED;
+    if (swz_b && N % 8 != 0) return NAJU_ERR_UNSUPPORTED;
+    uint32_t ncols = 32;
+    while (ncols < (uint32_t)N) ncols <<= 1;
+    const size_t smem = sizeof(float) * ((size_t)128 * K + (size_t)N * K);
+    cudaError_t e = cudaFuncSetAttribute(naju::tc_selftest_ss_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return NAJU_ERR_CUDA;
+    naju::tc_selftest_ss_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
+        A, B, D, N, K, rows_a, swz_a, swz_b, ncols, status);
     return cudaGetLastError() == cudaSuccess ? NAJU_OK : NAJU_ERR_CUDA;
 }

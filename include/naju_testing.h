@@ -59,6 +59,15 @@ int32_t naju_testing_fwd_impl(const void* dims);
 naju_status naju_testing_tc_mma(int32_t N, int32_t K, const float* A, const float* B, float* D,
                                 int* status, void* stream);
 
+/* Same product with both operands in shared memory.  A [rows_a x K] is staged
+ * as a rows_a-row tile (rows_a 64 or 128) and the MMA reads 128 rows; only
+ * the first rows_a rows of D are meaningful.  swz_a / swz_b select the
+ * 128-byte swizzled K-major layout for A / B (K % 32 == 0), else no-swizzle
+ * core matrices.  N in [16, 128], K in [16, 128], multiples of 16. */
+naju_status naju_testing_tc_mma_ss(int32_t N, int32_t K, int32_t rows_a, int32_t swz_a,
+                                   int32_t swz_b, const float* A, const float* B, float* D,
+                                   int* status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -81,6 +81,9 @@ def lib(build_if_missing: bool = True):
             L.naju_testing_set_fwd_impl.argtypes = [i32]
             L.naju_testing_fwd_impl.argtypes = [vp]
             L.naju_testing_fwd_impl.restype = i32
+            L.naju_testing_set_bwd_impl.argtypes = [i32]
+            L.naju_testing_bwd_impl.argtypes = [vp]
+            L.naju_testing_bwd_impl.restype = i32
             L.naju_testing_bwd_groups.argtypes = [vp]
             L.naju_testing_bwd_groups.restype = i32
             for name in ("naju_conv_silu_fwd", "naju_conv_silu_bwd", "naju_scan_fwd",
@@ -286,6 +289,14 @@ def testing_set_fwd_impl(impl: int):
 
 def testing_fwd_impl(dims: Dims) -> int:
     return int(lib().naju_testing_fwd_impl(ctypes.byref(dims)))
+
+
+def testing_set_bwd_impl(impl: int):
+    lib().naju_testing_set_bwd_impl(int(impl))
+
+
+def testing_bwd_impl(dims: Dims) -> int:
+    return int(lib().naju_testing_bwd_impl(ctypes.byref(dims)))
 
 
 def testing_set_bwd_groups(groups: int):

@@ -3,6 +3,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <cmath>
 
 #include "naju.h"
@@ -23,6 +24,7 @@ int g_skip_publish = 0;
 int g_fwd_groups = 0;
 int g_bwd_groups = 0;
 int g_fwd_impl = 0;  // 0 automatic, 1 CUDA cores, 2 tensor cores
+int g_bwd_impl = 0;  // 0 automatic, 1 CUDA cores
 
 inline bool aligned(const void* ptr, size_t a) {
     return (reinterpret_cast<uintptr_t>(ptr) % a) == 0;
@@ -47,7 +49,7 @@ naju_status check_dims(const naju_dims* dm) {
 
 // Workspace layout (every region 256-byte aligned).
 struct Layout {
-    bool fwd_tc;
+    bool fwd_tc, bwd_tc;
     int nck, ngroups, seg_per_group, ntiles_f;
     int nsub, nclus, ntiles_b, bgroups, blk_per_group;
     size_t off_fflags, off_bflags, off_ckpt, off_carry, off_dbc, off_chan, off_edge, total;
@@ -56,6 +58,40 @@ struct Layout {
 bool use_fwd_tc(const naju_dims* dm) {
     if (g_fwd_impl == 1) return false;
     return fwd_tc_supported(dm->dtype, dm->d_state, dm->d_inner);
+}
+bool use_bwd_tc(const naju_dims* dm) {
+    if (g_bwd_impl == 1) return false;
+    return bwd_tc_supported(dm->dtype, dm->d_state, dm->d_inner);
+}
+
+// Backward tiling: channel tiles, dB/dC partial sets, sequence groups.
+struct BwdTiling {
+    int ntiles, nparts, bgroups, blk_per_group;
+};
+BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
+    BwdTiling b{};
+    const int64_t d = dm->d_inner;
+    if (tc) {
+        // 128 channels per block (one per tensor-memory lane), one partial set
+        // per tile; one block per SM.
+        b.ntiles = (int)cdiv(d, 128);
+        b.nparts = b.ntiles;
+    } else {
+        // Clusters of channel tiles share one partial set; two blocks per SM.
+        const int tiles = (int)cdiv(d, bwd_channels_per_block(dm->d_state));
+        b.nparts = (int)cdiv(tiles, bwd_cluster_size());
+        b.ntiles = b.nparts * bwd_cluster_size();
+    }
+    int gb = g_bwd_groups;
+    if (gb <= 0) {
+        const int64_t ctas = dm->batch * (int64_t)b.ntiles;
+        const int64_t want = (tc ? 1 : 4) * kSMs;
+        gb = ctas >= want ? 1 : (int)cdiv(want, ctas);
+    }
+    if (gb > nsub) gb = nsub;
+    b.blk_per_group = (int)cdiv(nsub, gb);
+    b.bgroups = (int)cdiv(nsub, b.blk_per_group);
+    return b;
 }
 
 int auto_groups(const naju_dims* dm, int nck, int ntiles_f, bool tc) {
@@ -79,38 +115,37 @@ Layout layout(const naju_dims* dm) {
     l.seg_per_group = (int)cdiv(l.nck, g);
     l.ngroups = (int)cdiv(l.nck, l.seg_per_group);
     l.nsub = (int)cdiv(L, kBwdSub);
-    const int tiles_b = (int)cdiv(d, bwd_channels_per_block(N));
-    l.nclus = (int)cdiv(tiles_b, bwd_cluster_size());
-    l.ntiles_b = l.nclus * bwd_cluster_size();
-    {
-        // Backward blocks hold ~111 KB of shared memory: two per SM.
-        int gb = g_bwd_groups;
-        if (gb <= 0) {
-            const int64_t ctas = Bt * (int64_t)l.ntiles_b;
-            const int64_t want = 4 * kSMs;
-            gb = ctas >= want ? 1 : (int)cdiv(want, ctas);
-        }
-        if (gb > l.nsub) gb = l.nsub;
-        l.blk_per_group = (int)cdiv(l.nsub, gb);
-        l.bgroups = (int)cdiv(l.nsub, l.blk_per_group);
-    }
+    l.bwd_tc = use_bwd_tc(dm);
+    const BwdTiling bt = bwd_tiling(dm, l.nsub, l.bwd_tc);
+    l.ntiles_b = bt.ntiles;
+    l.nclus = bt.nparts;
+    l.bgroups = bt.bgroups;
+    l.blk_per_group = bt.blk_per_group;
+    // Regions sized for the larger of the two backward tilings, so the
+    // workspace size does not depend on which backward kernel runs.
+    const BwdTiling bo = bwd_tiling(dm, l.nsub, !l.bwd_tc);
+    const bool other_ok = l.bwd_tc || bwd_tc_supported(dm->dtype, N, d);
+    const int64_t flags_n = std::max<int64_t>((int64_t)bt.bgroups * bt.ntiles,
+                                              other_ok ? (int64_t)bo.bgroups * bo.ntiles : 0);
+    const int64_t groups_n = std::max(bt.bgroups, other_ok ? bo.bgroups : 0);
+    const int64_t parts_n = std::max(bt.nparts, other_ok ? bo.nparts : 0);
     size_t off = sizeof(WsHeader);
     l.off_fflags = off;
     // Flags for the larger of the two forward tilings (at most nck groups), so
     // the workspace size does not depend on which forward kernel runs.
     off = up256(off + sizeof(int) * (size_t)l.nck * Bt * cdiv(d, 32));
     l.off_bflags = off;
-    off = up256(off + sizeof(int) * (size_t)l.bgroups * Bt * l.ntiles_b);
+    off = up256(off + sizeof(int) * (size_t)flags_n * Bt);
     l.off_ckpt = off;
     off = up256(off + sizeof(float) * (size_t)Bt * (l.nck + 1) * d * N);
     l.off_carry = off;
-    off = up256(off + sizeof(float) * (size_t)l.bgroups * Bt * d * N);
+    off = up256(off + sizeof(float) * (size_t)groups_n * Bt * d * N);
     l.off_dbc = off;
-    off = up256(off + sizeof(float) * (size_t)l.nclus * Bt * L * 2 * N);
+    off = up256(off + sizeof(float) * (size_t)parts_n * Bt * L * 2 * N);
     l.off_chan = off;
-    off = up256(off + sizeof(float) * (size_t)Bt * l.bgroups * d * 8);
+    off = up256(off + sizeof(float) * (size_t)Bt * groups_n * d * 8);
     l.off_edge = off;
-    off = up256(off + sizeof(float) * (size_t)Bt * l.bgroups * 2 * 3 * d);
+    off = up256(off + sizeof(float) * (size_t)Bt * groups_n * 2 * 3 * d);
     l.total = off;
     return l;
 }
@@ -242,6 +277,12 @@ naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* co
     p.scale = 1.0f / std::sqrt((float)dims->d_state);
     p.wait_limit = g_wait_limit;
     p.fault_skip_publish = g_skip_publish;
+    if (l.bwd_tc) {
+        e = launch_scan_bwd_tc_main(p, dims->out_dtype, s);
+        if (e == cudaSuccess)
+            e = launch_bwd_reductions(p, dims->out_dtype, dB, dC, dD, dconv_w, dconv_b, s);
+        return cuda_status(e);
+    }
     return cuda_status(launch_scan_bwd(p, dims->dtype, dims->out_dtype, dB, dC, dD, dconv_w,
                                        dconv_b, s));
 }
@@ -291,6 +332,12 @@ void naju_testing_set_skip_publish(int32_t skip) { g_skip_publish = skip ? 1 : 0
 void naju_testing_set_fwd_groups(int32_t groups) { g_fwd_groups = groups > 0 ? groups : 0; }
 void naju_testing_set_bwd_groups(int32_t groups) { g_bwd_groups = groups > 0 ? groups : 0; }
 void naju_testing_set_fwd_impl(int32_t impl) { g_fwd_impl = (impl == 1) ? 1 : 0; }
+void naju_testing_set_bwd_impl(int32_t impl) { g_bwd_impl = (impl == 1) ? 1 : 0; }
+int32_t naju_testing_bwd_impl(const void* dims) {
+    const naju_dims* dm = static_cast<const naju_dims*>(dims);
+    if (check_dims(dm) != NAJU_OK) return 0;
+    return use_bwd_tc(dm) ? 2 : 1;
+}
 int32_t naju_testing_fwd_impl(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);
     if (check_dims(dm) != NAJU_OK) return 0;

@@ -85,6 +85,12 @@ int fwd_tc_channels_per_block();
 cudaError_t launch_scan_fwd_tc(const FwdParams& p, int out_dtype, cudaStream_t st);
 cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, int out_dtype, void* dB, void* dC,
                             float* dD, float* dconv_w, float* dconv_b, cudaStream_t st);
+// Tensor-core backward (bf16 activations, d_state 64 or 128, 128 channels per
+// block, one dB/dC partial set per channel tile), then the reductions.
+bool bwd_tc_supported(int dtype, int64_t N, int64_t d);
+cudaError_t launch_scan_bwd_tc_main(const BwdParams& p, int out_dtype, cudaStream_t st);
+cudaError_t launch_bwd_reductions(const BwdParams& p, int out_dtype, void* dB, void* dC,
+                                  float* dD, float* dw, float* dbias, cudaStream_t st);
 cudaError_t launch_conv_fwd(int64_t Bt, int64_t L, int64_t d, const void* u, const float* w,
                             const float* bias, void* h, int dtype, int out_dtype,
                             cudaStream_t st);

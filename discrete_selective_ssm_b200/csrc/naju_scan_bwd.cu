@@ -732,6 +732,31 @@ __global__ void conv_edge_kernel(const float* __restrict__ edge, const float* __
     }
 }
 
+// The follow-up kernels of a backward: dB / dC from the channel-tile partials
+// (p.nclus partial sets), the per-channel sums, the conv group-boundary fixups.
+template <typename Tout>
+static cudaError_t reductions_t(const BwdParams& p, void* dB, void* dC, float* dD, float* dw,
+                                float* dbias, cudaStream_t st) {
+    const bool conv = p.conv_w != nullptr;
+    const int64_t BtL = p.Bt * p.L;
+    reduce_dBC_kernel<Tout><<<592, 256, 0, st>>>(p.dBCp, p.nclus, BtL, p.N,
+                                                  static_cast<Tout*>(dB), static_cast<Tout*>(dC));
+    reduce_chan_kernel<<<(unsigned)((p.d + 127) / 128), 128, 0, st>>>(
+        p.chan_part, p.Bt * p.ngroups, p.d, dD, conv ? dw : nullptr, conv ? dbias : nullptr);
+    if (conv && p.ngroups > 1)
+        conv_edge_kernel<Tout><<<296, 256, 0, st>>>(p.conv_edge, p.conv_w, p.Bt, p.ngroups,
+                                                     (int64_t)p.blk_per_group * kBwdSub, p.L,
+                                                     p.d, static_cast<Tout*>(p.dhu));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_reductions(const BwdParams& p, int out_dtype, void* dB, void* dC,
+                                  float* dD, float* dw, float* dbias, cudaStream_t st) {
+    if (out_dtype == NAJU_BF16)
+        return reductions_t<__nv_bfloat16>(p, dB, dC, dD, dw, dbias, st);
+    return reductions_t<float>(p, dB, dC, dD, dw, dbias, st);
+}
+
 template <typename Tin, typename Tout, int N, bool CONV>
 static cudaError_t launch_bwd_t(const BwdParams& p, void* dB, void* dC, float* dD, float* dw,
                                 float* dbias, cudaStream_t st) {
@@ -756,16 +781,7 @@ static cudaError_t launch_bwd_t(const BwdParams& p, void* dB, void* dC, float* d
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, p);
     if (e != cudaSuccess) return e;
-    const int64_t BtL = p.Bt * p.L;
-    reduce_dBC_kernel<Tout><<<592, 256, 0, st>>>(p.dBCp, p.nclus, BtL, N,
-                                                  static_cast<Tout*>(dB), static_cast<Tout*>(dC));
-    reduce_chan_kernel<<<(unsigned)((p.d + 127) / 128), 128, 0, st>>>(
-        p.chan_part, p.Bt * p.ngroups, p.d, dD, CONV ? dw : nullptr, CONV ? dbias : nullptr);
-    if (CONV && p.ngroups > 1)
-        conv_edge_kernel<Tout><<<296, 256, 0, st>>>(p.conv_edge, p.conv_w, p.Bt, p.ngroups,
-                                                     (int64_t)p.blk_per_group * kBwdSub, p.L,
-                                                     p.d, static_cast<Tout*>(p.dhu));
-    return cudaGetLastError();
+    return reductions_t<Tout>(p, dB, dC, dD, dw, dbias, st);
 }
 
 template <typename Tin, typename Tout, bool CONV>

@@ -1,0 +1,942 @@
+// Naju backward scan with the d_state contractions on the 5th-generation
+// tensor cores (sm_100a, tcgen05, kind::tf32), for bf16 activations.
+//
+// Same gradient as naju_scan_bwd.cu (derived from the recurrence of the Naju
+// reproduction README, "Core equations"); with G_t = dLoss/dx_t,
+// s = 1/sqrt(N), f = sigmoid(a), i = sigmoid(b), v = i h:
+//   G_t = s dy_t C_t + f_{t+1} G_{t+1},  GB_t = G_t . B_t,
+//   dh_t = D dy_t + i_t GB_t,  db_t = h_t GB_t i_t (1 - i_t),
+//   da_t = (f df)_t (1 - f_t),  (f df)_t = sum_{t'>=t} dL_t' + (carry . state),
+//   dL_t = s dy_t (x_t . C_t) - v_t GB_t,
+//   dB_t = sum_ch v_t G_t,  dC_t = s sum_ch dy_t x_t.
+//
+// Chunked form.  A block owns 128 channels (tensor-memory lanes) of one batch
+// element and one sequence group; it walks the group's 64-token blocks from
+// the last to the first, each in two sweeps over 16-token sub-chunks.  With
+// E_t the decay product from the sub-chunk start (inclusive), Elast = E_15:
+//  forward sweep (from the block's forward checkpoint X):
+//   readout   R[ch][t] = X.C_t + sum_m W_m G[t][m],   W_m = v_m / E_m,
+//             x_t.C_t = E_t R (for dz and dL),
+//   state     X' = Elast X + sum_m (v_m Elast / E_m) B_m,
+//   dC        dC_t = sum_ch Y_t X + sum_{m<=t} A_C[t][m] B_m,  Y_t = s dy_t E_t,
+//             A_C[t][m] = sum_ch Y_t W_m   (contractions over channels);
+//  backward sweep (carry H = the adjoint entering the sub-chunk's end):
+//   dv        GB_t = (Elast / E_t) [H.B_t + sum_{t'>=t} U_t' (C_t'.B_t)],
+//             U_t' = s dy_t' E_t' / Elast,
+//   adjoint   H' = Elast H + sum_t' (s dy_t' E_t') C_t',
+//   dB        dB_t = sum_ch P_t H + sum_{t'>=t} A_B[t][t'] C_t',
+//             P_t = v_t Elast / E_t,  A_B[t][t'] = sum_ch P_t U_t'.
+// Readout, state, dv and adjoint run with the per-channel operand (X, H, W,
+// U, ...) in tensor memory; the channel contractions for dB and dC run with
+// both operands in shared memory, X or H written transposed into a 128-byte
+// swizzled tile (K = channels) - for d_state 64 the 64-row operand rides an
+// M = 128 MMA whose upper rows are ignored.  The small A_C / A_B products and
+// everything per (token, channel) run on the CUDA cores.
+//
+// Exactness.  A sub-chunk whose product of 1/f exceeds 2^64 in any channel of
+// the block takes an exact token-by-token path on the CUDA cores (states in
+// tensor memory, channel sums of dB / dC through warp shuffles).
+//
+// Outputs.  dB and dC partial sums over each block's 128 channels go to a
+// per-tile buffer that a small kernel sums; dD and the conv parameter
+// gradients go through per-(batch, group) channel partials; sequence groups
+// exchange the adjoint carry by a decoupled look-back backwards in time
+// (an adjoint-only early pass, bounded waits), as in the CUDA-core kernel.
+#include <string.h>
+
+#include <type_traits>
+
+#include "naju_common.cuh"
+#include "naju_kernels.h"
+#include "naju_tc.cuh"
+#include "naju_tma.h"
+
+namespace naju {
+
+namespace {
+
+constexpr int kBT = 16;                              // tokens per sub-chunk
+constexpr float kBBound = 18446744073709551616.0f;   // 2^64
+constexpr long long kBSpin = 1LL << 24;
+
+template <int N>
+struct BCols {
+    static constexpr uint32_t X = 0;            // forward state [N]
+    static constexpr uint32_t G = N;            // adjoint carry [N]
+    static constexpr uint32_t D = 2 * N;        // state / adjoint MMA result [N]
+    static constexpr uint32_t R = 3 * N;        // readout / dv MMA result [16]
+    static constexpr uint32_t BC = 3 * N + 16;  // dC / dB MMA result [16] (lanes = d_state)
+    static constexpr uint32_t WU = 3 * N + 32;  // W or U [16]
+    static constexpr uint32_t VV = 3 * N + 48;  // state weights or s dy E [16]
+    static constexpr uint32_t DL = 3 * N + 64;  // s dy_t x_t.C_t of the block [64]
+    static constexpr uint32_t USED = 3 * N + 128;
+    static constexpr uint32_t ALLOC = 512;
+    static_assert(USED <= ALLOC, "tensor memory");
+};
+
+struct alignas(64) BwdTmaps {
+    CUtensorMap u, a, b, z, dy, B, C;
+};
+
+template <int N>
+struct BwdTcSmem {
+    static constexpr int T = kBT, P = 128;
+    // Transposed state tile (X or H), 128-byte swizzled, rows = d_state,
+    // K = channels; for N = 64 the M = 128 MMA also reads 8 KB past it.
+    static constexpr int ST_FLOATS = N * 128 > 10240 ? N * 128 : 10240;
+    // B^T / C^T tile (rows = d_state, K = 16), with the same overrun for N = 64.
+    static constexpr int TS_FLOATS = N * 16 > 2048 ? N * 16 : 2048;
+    struct Raw {
+        alignas(128) __nv_bfloat16 u[T + 3][P];
+        alignas(128) __nv_bfloat16 a[T][P];
+        alignas(128) __nv_bfloat16 b[T][P];
+        alignas(128) __nv_bfloat16 z[T][P];
+        alignas(128) __nv_bfloat16 dy[T][P];
+        alignas(128) __nv_bfloat16 Bm[T][N];
+        alignas(128) __nv_bfloat16 Cm[T][N];
+    };
+    alignas(1024) float st[ST_FLOATS];
+    alignas(1024) float pk[T * P];     // Y or P, swizzled, rows t, K = channels
+    Raw raw[2];
+    alignas(128) float ta[T * N];      // C (forward) / B (backward) rows t, K = d_state
+    alignas(128) float ts[TS_FLOATS];  // B^T (forward) / C^T (backward): rows d_state, K = 16
+    alignas(128) float tg[T * T];      // G[t][m] (forward) / G^T (backward)
+    alignas(128) float ta2[T * T];     // A_C (forward) / A_B (backward)
+    alignas(16) float y1[T][P + 4];    // Y / P rows (slow path: s dy or v)
+    alignas(16) float w1[T][P + 4];    // W / U rows (slow path: exchange of half sums)
+    alignas(16) float brow[T][N + 4];
+    alignas(16) float crow[T][N + 4];
+    float dp[T + 3][P];
+    float acc[T][N];                   // slow path channel sums
+    float x0[P], x1[P], x2[P];         // per-half exchanges
+    uint64_t loaded[2], mma;
+    uint32_t taddr;
+    int item, ok;
+};
+
+enum { kSweepFwd = 0, kSweepBwd = 1, kSweepEarly = 2 };
+
+}  // namespace
+
+template <typename Tout, int N, bool CONV>
+__global__ void __launch_bounds__(256, 1)
+scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
+    using Tin = __nv_bfloat16;
+    using Cols = BCols<N>;
+    using Sm = BwdTcSmem<N>;
+    constexpr int T = kBT, P = 128, H = T / 2, NT = 256, NH = N / 2;
+    constexpr int K = kBwdSub;  // tokens per block (forward checkpoint spacing)
+    extern __shared__ __align__(1024) float4 smem4[];
+    Sm& sm = *reinterpret_cast<Sm*>(smem4);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int ch = tid & (P - 1);   // channel within the block = TMEM lane
+    const int half = tid >> 7;      // tokens [8 half, 8 half + 8) / columns [N/2 half, ...)
+    const int64_t Bt = p.Bt, L = p.L, d = p.d;
+    const float s = p.scale;
+    const bool has_z = p.z != nullptr;
+
+    // ------------------------------------------------------------ set-up
+    if (warp == 0) {
+        tc::tmem_alloc(&sm.taddr, Cols::ALLOC);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
+        tc::mbar_init(&sm.loaded[0], 1);
+        tc::mbar_init(&sm.loaded[1], 1);
+        tc::mbar_init(&sm.mma, 1);
+        tma::prefetch_map(&tm.u);
+        tma::prefetch_map(&tm.a);
+        tma::prefetch_map(&tm.b);
+        if (has_z) tma::prefetch_map(&tm.z);
+        tma::prefetch_map(&tm.dy);
+        tma::prefetch_map(&tm.B);
+        tma::prefetch_map(&tm.C);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = sm.taddr;
+    const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t trow = tbase + lane;  // this thread's TMEM row (channel)
+    const int item = sm.item;
+    const int per_g = (int)(Bt * p.ntiles);
+    const int g = p.ngroups - 1 - item / per_g;
+    const int bb = (item % per_g) / p.ntiles;
+    const int tile = item % p.ntiles;
+    const int64_t c0 = (int64_t)tile * P;
+    const int64_t c = c0 + ch;
+    const bool cvalid = c < d;
+    const int kb0 = g * p.blk_per_group;
+    const int kb1 = min(kb0 + p.blk_per_group, p.nsub);
+    const int64_t tg0 = (int64_t)kb0 * K;
+    const int64_t tg1 = min64(L, (int64_t)kb1 * K);
+    const bool lastg = (g == p.ngroups - 1);
+    const bool firstg = (g == 0);
+
+    float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, wb = 0.f, Dc = 0.f;
+    if (cvalid) {
+        if (CONV) {
+            w0 = p.conv_w[c * 4 + 0];
+            w1 = p.conv_w[c * 4 + 1];
+            w2 = p.conv_w[c * 4 + 2];
+            w3 = p.conv_w[c * 4 + 3];
+            wb = p.conv_b ? p.conv_b[c] : 0.f;
+        }
+        Dc = p.D ? p.D[c] : 0.f;
+    }
+    const int64_t boff = (int64_t)bb * L;
+    Tout* gdhu = static_cast<Tout*>(p.dhu) + boff * d + c;
+    Tout* gda = static_cast<Tout*>(p.da) + boff * d + c;
+    Tout* gdb = static_cast<Tout*>(p.db) + boff * d + c;
+    Tout* gdz = has_z ? static_cast<Tout*>(p.dz) + boff * d + c : nullptr;
+    float* part = p.dBCp + (((int64_t)tile * Bt + bb) * L) * 2 * N;  // [L][2][N]
+    float* edge = p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d;
+    bool timed_out = false;
+
+    // ------------------------------------------------ the item sequence
+    // Early pass (groups with a predecessor): the group's sub-chunks, last
+    // first.  Main: blocks last first; per block the forward sweep's
+    // sub-chunks in order, then the backward sweep's in reverse.
+    const int nE = firstg ? 0 : (int)((tg1 - tg0 + T - 1) / T);
+    const int64_t te_first = min64(L, (int64_t)kb1 * K);
+    const int nsb0 = (int)((te_first - (int64_t)(kb1 - 1) * K + T - 1) / T);
+    const int nitems = nE + 2 * nsb0 + 8 * (kb1 - 1 - kb0);
+    auto item_t0 = [&](int li) -> int64_t {
+        if (li < nE) return tg0 + (int64_t)(nE - 1 - li) * T;
+        int j = li - nE;
+        int k = kb1 - 1, nsb = nsb0;
+        if (j >= 2 * nsb0) {
+            j -= 2 * nsb0;
+            k = kb1 - 2 - j / 8;
+            j %= 8;
+            nsb = 4;
+        }
+        const int sb = j < nsb ? j : 2 * nsb - 1 - j;
+        return (int64_t)k * K + (int64_t)sb * T;
+    };
+    auto issue = [&](int li) {  // one thread
+        const int buf = li & 1;
+        typename Sm::Raw& r = sm.raw[buf];
+        uint64_t* mb = &sm.loaded[buf];
+        const uint32_t bytes =
+            (uint32_t)sizeof(Tin) * ((T + 3) * P + (has_z ? 4 : 3) * T * P + 2 * T * N);
+        tma::expect_tx(mb, bytes);
+        const int x = (int)c0, y = (int)item_t0(li), zb = bb;
+        tma::load_3d(&r.u[0][0], &tm.u, x, y - 3, zb, mb);
+        tma::load_3d(&r.a[0][0], &tm.a, x, y, zb, mb);
+        tma::load_3d(&r.b[0][0], &tm.b, x, y, zb, mb);
+        if (has_z) tma::load_3d(&r.z[0][0], &tm.z, x, y, zb, mb);
+        tma::load_3d(&r.dy[0][0], &tm.dy, x, y, zb, mb);
+        tma::load_3d(&r.Bm[0][0], &tm.B, 0, y, zb, mb);
+        tma::load_3d(&r.Cm[0][0], &tm.C, 0, y, zb, mb);
+    };
+    int li = 0;            // current item
+    uint32_t mma_phase = 0;
+    if (tid == 0 && nitems > 0) issue(0);
+
+    auto bf4 = [](const __nv_bfloat16* src) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(src);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        return make_float4(lo.x, lo.y, hi.x, hi.y);
+    };
+    auto sync = [&]() {
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+    };
+    // Transposed copy of TMEM columns [col, col + N) into the swizzled tile:
+    // element (row j, k = channel).
+    auto to_st = [&](uint32_t col) {
+#pragma unroll
+        for (int n0 = 0; n0 < NH; n0 += 16) {
+            float v[16];
+            tc::tmem_ld16(trow + col + half * NH + n0, v);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                sm.st[tc::sw128_offset(half * NH + n0 + k, ch, N) >> 2] = cvalid ? v[k] : 0.f;
+        }
+    };
+    // TMEM columns [col, col + N) of this row <-> global rows (half each).
+    auto tmem_from = [&](uint32_t col, const float* src, bool cg) {
+#pragma unroll
+        for (int n0 = 0; n0 < NH; n0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int k = 0; k < 16; k += 4) {
+                float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (src && cvalid) {
+                    const float4* s4 =
+                        reinterpret_cast<const float4*>(src + c * N + half * NH + n0 + k);
+                    v4 = cg ? __ldcg(s4) : *s4;
+                }
+                v[k] = v4.x;
+                v[k + 1] = v4.y;
+                v[k + 2] = v4.z;
+                v[k + 3] = v4.w;
+            }
+            tc::tmem_st16(trow + col + half * NH + n0, v);
+        }
+        tc::tmem_st_wait();
+    };
+    auto tmem_to = [&](uint32_t col, float* dst) {
+#pragma unroll
+        for (int n0 = 0; n0 < NH; n0 += 16) {
+            float v[16];
+            tc::tmem_ld16(trow + col + half * NH + n0, v);
+            tc::tmem_ld_wait();
+            if (cvalid) {
+#pragma unroll
+                for (int k = 0; k < 16; k += 4)
+                    *reinterpret_cast<float4*>(dst + c * N + half * NH + n0 + k) =
+                        make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+            }
+        }
+    };
+    // Dot of TMEM columns [ca, ca + N) and [cb, cb + N) of this row (both halves).
+    auto tmem_dot = [&](uint32_t ca, uint32_t cb) -> float {
+        float acc = 0.f;
+#pragma unroll
+        for (int n0 = 0; n0 < NH; n0 += 16) {
+            float va[16], vb[16];
+            tc::tmem_ld16(trow + ca + half * NH + n0, va);
+            tc::tmem_ld16(trow + cb + half * NH + n0, vb);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) acc = fmaf(va[k], vb[k], acc);
+        }
+        if (half == 1) sm.x1[ch] = acc;
+        __syncthreads();
+        acc += half == 0 ? sm.x1[ch] : 0.f;
+        if (half == 0) sm.x2[ch] = acc;
+        __syncthreads();
+        return sm.x2[ch];
+    };
+    // Scale-and-add on TMEM: col_a <- m * col_a + (col_b or a global row).
+    auto tmem_axpy = [&](uint32_t ca, float m, uint32_t cb) {
+#pragma unroll
+        for (int n0 = 0; n0 < NH; n0 += 16) {
+            float va[16], vb[16];
+            tc::tmem_ld16(trow + ca + half * NH + n0, va);
+            tc::tmem_ld16(trow + cb + half * NH + n0, vb);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) va[k] = fmaf(m, va[k], vb[k]);
+            tc::tmem_st16(trow + ca + half * NH + n0, va);
+        }
+        tc::tmem_st_wait();
+    };
+
+    // ------------------------------------------------- per-item state
+    // Per (token, channel) values of this thread's 8 tokens.
+    float fv[H], qv[H], hv[H], iv[H], dyv[H], pre[H], Ev[H], Qv[H];
+    float Elast = 1.f;
+    bool slow = false;
+    int nvh = 0;  // valid tokens of this thread's half
+
+    // Unpack item `li` (raw buffer li & 1) for a sweep; fills the registers
+    // above, the TMEM operand columns and the per-token tiles.  Returns after
+    // a block-wide barrier.
+    auto prep = [&](int64_t t0, int64_t te, int sweep) {
+        const typename Sm::Raw& r = sm.raw[li & 1];
+        const bool fwd = sweep == kSweepFwd;
+        // B and C rows to fp32.
+        for (int e = tid; e < T * N / 4; e += NT) {
+            const int tt = e / (N / 4), j = (e % (N / 4)) * 4;
+            *reinterpret_cast<float4*>(&sm.brow[tt][j]) = bf4(&r.Bm[tt][j]);
+            *reinterpret_cast<float4*>(&sm.crow[tt][j]) = bf4(&r.Cm[tt][j]);
+        }
+        nvh = cvalid ? (int)max((int64_t)0, min64((int64_t)H, te - t0 - half * H)) : 0;
+        float Qh = 1.f, Eh = 1.f;
+#pragma unroll
+        for (int k = 0; k < H; ++k) {
+            const int tt = half * H + k;
+            const bool valid = k < nvh;
+            qv[k] = valid ? 1.f + __expf(-to_f(r.a[tt][ch])) : 1.f;
+            fv[k] = rcpa_(qv[k]);
+            Qh *= qv[k];
+            Eh *= fv[k];
+            float hh, pp = 0.f;
+            if (CONV) {
+                pp = wb + w0 * to_f(r.u[tt][ch]) + w1 * to_f(r.u[tt + 1][ch]) +
+                     w2 * to_f(r.u[tt + 2][ch]) + w3 * to_f(r.u[tt + 3][ch]);
+                hh = siluf_(pp);
+            } else {
+                hh = to_f(r.u[tt + 3][ch]);
+            }
+            pre[k] = pp;
+            hv[k] = valid ? hh : 0.f;
+            iv[k] = sigmoidf_(to_f(r.b[tt][ch]));
+            const float gg = has_z ? siluf_(to_f(r.z[tt][ch])) : 1.f;
+            dyv[k] = valid ? to_f(r.dy[tt][ch]) * gg : 0.f;
+        }
+        if (half == 0) {
+            sm.x0[ch] = Qh;
+            sm.x1[ch] = Eh;
+        } else {
+            sm.x2[ch] = Eh;
+        }
+        __syncthreads();
+        const float Q0 = sm.x0[ch], E0 = sm.x1[ch], E1 = sm.x2[ch];
+        slow = __syncthreads_or(half == 1 && !(Q0 * Qh <= kBBound)) != 0;
+        Elast = E0 * E1;
+        {
+            float Q = half ? Q0 : 1.f, E = half ? E0 : 1.f;
+#pragma unroll
+            for (int k = 0; k < H; ++k) {
+                E *= fv[k];
+                Q *= qv[k];
+                Ev[k] = E;
+                Qv[k] = Q;
+            }
+        }
+        // Per-(token, channel) operands.
+        float c1[H], c2[H];
+        const float QL = rcpa_(Elast);  // product of q over the sub-chunk (fast path)
+#pragma unroll
+        for (int k = 0; k < H; ++k) {
+            const int tt = half * H + k;
+            const float v = iv[k] * hv[k];
+            if (fwd) {
+                // W (readout weights), V (state weights), Y = s dy E.
+                const float W = slow ? v : v * Qv[k];
+                c1[k] = W;
+                c2[k] = slow ? fv[k] : W * Elast;
+                const float Y = slow ? s * dyv[k] : s * dyv[k] * Ev[k];
+                sm.y1[tt][ch] = Y;
+                sm.w1[tt][ch] = W;
+                if (!slow) sm.pk[tc::sw128_offset(tt, ch, T) >> 2] = cvalid ? Y : 0.f;
+            } else {
+                // U = s dy E / Elast, s dy E (adjoint weights), P = v Elast / E.
+                const float sdy = s * dyv[k];
+                c1[k] = slow ? sdy : sdy * Ev[k] * QL;
+                c2[k] = slow ? fv[k] : sdy * Ev[k];
+                if (sweep == kSweepBwd) {
+                    const float Pv = slow ? v : v * Elast * Qv[k];
+                    sm.y1[tt][ch] = Pv;
+                    sm.w1[tt][ch] = c1[k];
+                    if (!slow) sm.pk[tc::sw128_offset(tt, ch, T) >> 2] = cvalid ? Pv : 0.f;
+                }
+            }
+        }
+        tc::tmem_st8(trow + Cols::WU + half * H, c1);
+        tc::tmem_st8(trow + Cols::VV + half * H, c2);
+        tc::tmem_st_wait();
+        __syncthreads();  // brow, crow, y1, w1 complete
+        if (!slow) {
+            // K-major per-token tiles.
+            for (int e = tid; e < T * N / 4; e += NT) {
+                const int rest = e >> 3;
+                const int tt = (rest & 1) * 8 + (e & 7), j = (rest >> 1) * 4;
+                // ta: rows t, K = d_state (C forward, B backward)
+                *reinterpret_cast<float4*>(&sm.ta[tc::kmajor_offset(tt, j, N) >> 2]) =
+                    fwd ? *reinterpret_cast<const float4*>(&sm.crow[tt][j])
+                        : *reinterpret_cast<const float4*>(&sm.brow[tt][j]);
+                // ts: rows d_state, K = 16 (B^T forward, C^T backward)
+                const int jj = e % N, m0 = (e / N) * 4;
+                const float(*src)[N + 4] = fwd ? sm.brow : sm.crow;
+                *reinterpret_cast<float4*>(&sm.ts[tc::kmajor_offset(jj, m0, T) >> 2]) =
+                    make_float4(src[m0][jj], src[m0 + 1][jj], src[m0 + 2][jj], src[m0 + 3][jj]);
+            }
+            if (sweep != kSweepEarly) {
+                // tg: forward G[t][m] = C_t . B_m (m <= t); backward G^T[t][t'] = C_t' . B_t
+                // (t' >= t).  ta2: A_C[t][m] = sum_ch Y_t W_m (m <= t) or
+                // A_B[t][t'] = sum_ch P_t U_t' (t' >= t).  One entry per thread.
+                const int tt = tid / T, mm = tid % T;
+                const bool live = fwd ? (mm <= tt) : (mm >= tt);
+                float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
+                if (live) {
+                    const float* cr = fwd ? sm.crow[tt] : sm.crow[mm];
+                    const float* br = fwd ? sm.brow[mm] : sm.brow[tt];
+#pragma unroll 4
+                    for (int j = 0; j < N; j += 4) {
+                        const float4 cv = *reinterpret_cast<const float4*>(cr + j);
+                        const float4 bv = *reinterpret_cast<const float4*>(br + j);
+                        acc = __ffma2_rn(make_float2(cv.x, cv.y), make_float2(bv.x, bv.y), acc);
+                        acc = __ffma2_rn(make_float2(cv.z, cv.w), make_float2(bv.z, bv.w), acc);
+                    }
+#pragma unroll 4
+                    for (int q = 0; q < P; q += 4) {
+                        const float4 yv = *reinterpret_cast<const float4*>(&sm.y1[tt][q]);
+                        const float4 wv = *reinterpret_cast<const float4*>(&sm.w1[mm][q]);
+                        acc2 = __ffma2_rn(make_float2(yv.x, yv.y), make_float2(wv.x, wv.y), acc2);
+                        acc2 = __ffma2_rn(make_float2(yv.z, yv.w), make_float2(wv.z, wv.w), acc2);
+                    }
+                }
+                sm.tg[tc::kmajor_offset(tt, mm, T) >> 2] = acc.x + acc.y;
+                sm.ta2[tc::kmajor_offset(tt, mm, T) >> 2] = acc2.x + acc2.y;
+            }
+        }
+        tc::fence_proxy_async();
+        sync();
+    };
+
+    // MMAs of the current item (one thread), then commit.
+    auto issue_mma = [&](int sweep) {
+        constexpr uint32_t id16 = tc::idesc_tf32(128, T);
+        constexpr uint32_t idN = tc::idesc_tf32(128, N);
+        const uint32_t a_ta = tc::smem_u32(sm.ta), a_ts = tc::smem_u32(sm.ts);
+        const uint32_t a_tg = tc::smem_u32(sm.tg), a_t2 = tc::smem_u32(sm.ta2);
+        const uint32_t a_st = tc::smem_u32(sm.st), a_pk = tc::smem_u32(sm.pk);
+        if (sweep != kSweepEarly) {
+            // readout (forward: X . C + W G) or dv (backward: H . B + U G^T)
+            const uint32_t Acol = sweep == kSweepFwd ? Cols::X : Cols::G;
+#pragma unroll
+            for (int ks = 0; ks < N / 8; ++ks)
+                tc::mma_tf32_ts(tbase + Cols::R, tbase + Acol + ks * 8,
+                                tc::sdesc(a_ta + ks * 256, 128, 32 * N), id16, ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < T / 8; ++ks)
+                tc::mma_tf32_ts(tbase + Cols::R, tbase + Cols::WU + ks * 8,
+                                tc::sdesc(a_tg + ks * 256, 128, 32 * T), id16, 1u);
+        }
+        // state (forward: V B^T) or adjoint (backward: (s dy E) C^T)
+#pragma unroll
+        for (int ks = 0; ks < T / 8; ++ks)
+            tc::mma_tf32_ts(tbase + Cols::D, tbase + Cols::VV + ks * 8,
+                            tc::sdesc(a_ts + ks * 256, 128, 32 * T), idN, ks > 0 ? 1u : 0u);
+        if (sweep != kSweepEarly) {
+            // dC or dB: (state^T)(Y or P) over channels + (B^T or C^T)(A_C or A_B)
+#pragma unroll
+            for (int ks = 0; ks < P / 8; ++ks)
+                tc::mma_tf32_ss(tbase + Cols::BC,
+                                tc::sdesc_sw128(a_st + (ks >> 2) * N * 128 + (ks & 3) * 32),
+                                tc::sdesc_sw128(a_pk + (ks >> 2) * T * 128 + (ks & 3) * 32), id16,
+                                ks > 0 ? 1u : 0u);
+#pragma unroll
+            for (int ks = 0; ks < T / 8; ++ks)
+                tc::mma_tf32_ss(tbase + Cols::BC, tc::sdesc(a_ts + ks * 256, 128, 32 * T),
+                                tc::sdesc(a_t2 + ks * 256, 128, 32 * T), id16, 1u);
+        }
+        tc::mma_commit(&sm.mma);
+    };
+
+    // Start item li: prefetch the next one, wait for this one's inputs.
+    auto begin_item = [&]() {
+        if (tid == 0 && li + 1 < nitems) issue(li + 1);
+        if (!tc::mbar_wait(&sm.loaded[li & 1], (uint32_t)((li >> 1) & 1), kBSpin))
+            timed_out = true;
+    };
+    auto run_mma = [&](int sweep) {
+        if (tid == 0) {
+            tc::fence_after_sync();
+            issue_mma(sweep);
+        }
+        if (!tc::mbar_wait(&sm.mma, mma_phase, kBSpin)) timed_out = true;
+        mma_phase ^= 1u;
+        tc::fence_after_sync();
+    };
+    // Write a [16][N] channel-sum tile (slot 0 dB, 1 dC) from TMEM BC (lanes
+    // = d_state rows, columns = tokens) to the per-tile partial buffer.
+    auto write_bc_tmem = [&](int slot, int64_t t0, int64_t te) {
+        if ((warp & 3) * 32 < N) {
+            float v[8];
+            tc::tmem_ld8(tbase + lane + Cols::BC + half * H, v);
+            tc::tmem_ld_wait();
+            const int j = ch;  // lane = d_state row
+#pragma unroll
+            for (int k = 0; k < H; ++k) {
+                const int64_t t = t0 + half * H + k;
+                if (t < te) part[t * 2 * N + slot * N + j] = v[k];
+            }
+        } else {
+            // keep the warp's tcgen05.ld count uniform per lane quadrant
+        }
+    };
+    auto write_bc_smem = [&](int slot, int64_t t0, int64_t te) {
+        for (int e = tid; e < T * N; e += NT) {
+            const int tt = e / N, j = e % N;
+            const int64_t t = t0 + tt;
+            if (t < te) part[t * 2 * N + slot * N + j] = sm.acc[tt][j];
+        }
+    };
+    auto warp_sum = [](float v) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        return v;
+    };
+
+    // ----------------------------------------------------------------
+    // Exact forward sub-chunk: token recurrence on this thread's half of
+    // the state columns; x.C partial sums exchanged between halves; dC
+    // channel sums into sm.acc.  Requires sm.acc zeroed.
+    auto fwd_exact = [&](float* ydot) {
+        float vv[16], ff[16];
+        tc::tmem_ld16(trow + Cols::WU, vv);
+        tc::tmem_ld16(trow + Cols::VV, ff);
+        tc::tmem_ld_wait();
+        float yp[16];
+#pragma unroll
+        for (int tt = 0; tt < T; ++tt) yp[tt] = 0.f;
+        for (int n0 = half * NH; n0 < half * NH + NH; n0 += 16) {
+            float x[16];
+            tc::tmem_ld16(trow + Cols::X + n0, x);
+            tc::tmem_ld_wait();
+            for (int tt = 0; tt < T; ++tt) {
+                const float sdy = cvalid ? sm.y1[tt][ch] : 0.f;
+                float a = 0.f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    x[k] = fmaf(ff[tt], x[k], vv[tt] * sm.brow[tt][n0 + k]);
+                    a = fmaf(x[k], sm.crow[tt][n0 + k], a);
+                    const float r = warp_sum(sdy * x[k]);
+                    if ((tid & 31) == 0) atomicAdd(&sm.acc[tt][n0 + k], r);
+                }
+                yp[tt] += a;
+            }
+            tc::tmem_st16(trow + Cols::X + n0, x);
+        }
+        tc::tmem_st_wait();
+        // exchange: each half needs the other half's partials for its tokens
+#pragma unroll
+        for (int tt = 0; tt < T; ++tt)
+            if ((tt >= H) != (half == 1)) sm.w1[tt][ch] = yp[tt];
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < H; ++k) ydot[k] = yp[half * H + k] + sm.w1[half * H + k][ch];
+        float lp = 0.f;
+#pragma unroll
+        for (int tt = 0; tt < T; ++tt) lp += __logf(ff[tt]);
+        return lp;
+    };
+    // Exact backward sub-chunk: adjoint recurrence over this half of the
+    // columns, G.B exchanged between halves, dB channel sums into sm.acc.
+    auto bwd_exact = [&](float* gbv, bool grads) {
+        float sd[16], ff[16];
+        tc::tmem_ld16(trow + Cols::WU, sd);
+        tc::tmem_ld16(trow + Cols::VV, ff);
+        tc::tmem_ld_wait();
+        float gp[16];
+#pragma unroll
+        for (int tt = 0; tt < T; ++tt) gp[tt] = 0.f;
+        for (int n0 = half * NH; n0 < half * NH + NH; n0 += 16) {
+            float hx[16];
+            tc::tmem_ld16(trow + Cols::G + n0, hx);
+            tc::tmem_ld_wait();
+            for (int tt = T - 1; tt >= 0; --tt) {
+                const float v = (grads && cvalid) ? sm.y1[tt][ch] : 0.f;
+                float a = 0.f;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const float gk = fmaf(sd[tt], sm.crow[tt][n0 + k], hx[k]);
+                    if (grads) {
+                        a = fmaf(gk, sm.brow[tt][n0 + k], a);
+                        const float r = warp_sum(v * gk);
+                        if ((tid & 31) == 0) atomicAdd(&sm.acc[tt][n0 + k], r);
+                    }
+                    hx[k] = ff[tt] * gk;
+                }
+                gp[tt] += a;
+            }
+            tc::tmem_st16(trow + Cols::G + n0, hx);
+        }
+        tc::tmem_st_wait();
+        if (grads) {
+#pragma unroll
+            for (int tt = 0; tt < T; ++tt)
+                if ((tt >= H) != (half == 1)) sm.w1[tt][ch] = gp[tt];
+            __syncthreads();
+#pragma unroll
+            for (int k = 0; k < H; ++k) gbv[k] = gp[half * H + k] + sm.w1[half * H + k][ch];
+        }
+        float lp = 0.f;
+#pragma unroll
+        for (int tt = 0; tt < T; ++tt) lp += __logf(ff[tt]);
+        return lp;
+    };
+
+    // ====================================================== early pass
+    // Adjoint only over the group (last sub-chunk first) to publish the
+    // carry leaving the group's start.
+    float* carry_in = p.carry + ((int64_t)g * Bt + bb) * d * N;
+    float* carry_out = g > 0 ? p.carry + ((int64_t)(g - 1) * Bt + bb) * d * N : nullptr;
+    int* flag_in = p.flags + ((int64_t)g * Bt + bb) * p.ntiles + tile;
+    int* flag_out = g > 0 ? p.flags + ((int64_t)(g - 1) * Bt + bb) * p.ntiles + tile : nullptr;
+    const float* dxf = p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr;
+    if (!firstg) {
+        tmem_from(Cols::G, lastg ? dxf : nullptr, false);
+        float logF = 0.f;
+        for (int e = 0; e < nE; ++e, ++li) {
+            const int64_t t0 = item_t0(li);
+            begin_item();
+            prep(t0, tg1, kSweepEarly);
+            if (!slow) {
+                run_mma(kSweepEarly);
+                tmem_axpy(Cols::G, Elast, Cols::D);
+                logF += __logf(Elast);
+            } else {
+                float dummy[H];
+                logF += bwd_exact(dummy, false);
+            }
+            sync();
+        }
+        if (!lastg) {
+            if (tid == 0) sm.ok = wait_flag(flag_in, &p.hdr->status, p.wait_limit) ? 1 : 0;
+            __syncthreads();
+            const bool okc = sm.ok != 0;
+            // carry out = (decay over the group) H + local contribution
+            const float Pf = __expf(logF);
+#pragma unroll
+            for (int n0 = 0; n0 < NH; n0 += 16) {
+                float hx[16];
+                tc::tmem_ld16(trow + Cols::G + half * NH + n0, hx);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int k = 0; k < 16; k += 4) {
+                    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (okc && cvalid)
+                        v4 = __ldcg(reinterpret_cast<const float4*>(carry_in + c * N + half * NH +
+                                                                    n0 + k));
+                    hx[k] = fmaf(Pf, v4.x, hx[k]);
+                    hx[k + 1] = fmaf(Pf, v4.y, hx[k + 1]);
+                    hx[k + 2] = fmaf(Pf, v4.z, hx[k + 2]);
+                    hx[k + 3] = fmaf(Pf, v4.w, hx[k + 3]);
+                }
+                tc::tmem_st16(trow + Cols::G + half * NH + n0, hx);
+            }
+            tc::tmem_st_wait();
+        }
+        tmem_to(Cols::G, carry_out);
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && !(lastg && p.fault_skip_publish)) st_release(flag_out, 1);
+    }
+    // carry entering the group's end
+    if (lastg) {
+        tmem_from(Cols::G, dxf, false);
+    } else {
+        if (tid == 0) sm.ok = wait_flag(flag_in, &p.hdr->status, p.wait_limit) ? 1 : 0;
+        __syncthreads();
+        tmem_from(Cols::G, sm.ok ? carry_in : nullptr, true);
+    }
+    for (int i = tid; i < 3 * P; i += NT) (&sm.dp[T][0])[i] = 0.f;
+    sync();
+
+    // ====================================================== main: blocks
+    float dD_acc = 0.f, dw0 = 0.f, dw1 = 0.f, dw2 = 0.f, dw3 = 0.f, dbias = 0.f;
+    for (int k = kb1 - 1; k >= kb0; --k) {
+        const int64_t tb = (int64_t)k * K;
+        const int64_t te = min64(L, tb + K);
+        const int nsb = (int)((te - tb + T - 1) / T);
+        const bool group_end_block = (k == kb1 - 1);
+        // state entering the block (forward checkpoint)
+        tmem_from(Cols::X, p.ckpt + ((int64_t)bb * (p.nck + 1) + k) * d * N, false);
+        to_st(Cols::X);
+        sync();
+
+        // --------------------------------------------- forward sweep
+        for (int sb = 0; sb < nsb; ++sb, ++li) {
+            const int64_t t0 = tb + (int64_t)sb * T;
+            begin_item();
+            prep(t0, te, kSweepFwd);
+            float yd[H];  // x_t . C_t of this thread's tokens
+            if (!slow) {
+                run_mma(kSweepFwd);
+                float r[H];
+                tc::tmem_ld8(trow + Cols::R + half * H, r);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < H; ++q) yd[q] = Ev[q] * r[q];
+                write_bc_tmem(1, t0, te);
+                tmem_axpy(Cols::X, Elast, Cols::D);
+            } else {
+                for (int e = tid; e < T * N; e += NT) (&sm.acc[0][0])[e] = 0.f;
+                __syncthreads();
+                fwd_exact(yd);
+                __syncthreads();
+                write_bc_smem(1, t0, te);
+            }
+            // dz and s dy (x.C) for the backward sweep
+            {
+                const typename Sm::Raw& r = sm.raw[li & 1];
+                float dl[H];
+#pragma unroll
+                for (int q = 0; q < H; ++q) {
+                    const int tt = half * H + q;
+                    dl[q] = s * dyv[q] * yd[q];
+                    if (has_z && q < nvh) {
+                        const float zv = to_f(r.z[tt][ch]);
+                        const float yv = fmaf(s, yd[q], Dc * hv[q]);
+                        gdz[(t0 + tt) * d] = from_f<Tout>(to_f(r.dy[tt][ch]) * yv * dsiluf_(zv));
+                    }
+                }
+                tc::tmem_st8(trow + Cols::DL + sb * T + half * H, dl);
+                tc::tmem_st_wait();
+            }
+            sync();
+            to_st(Cols::X);  // state entering the next sub-chunk
+            sync();
+        }
+        // (f df) tail of this block: carry entering the block's end . state at its end
+        const float tail = tmem_dot(Cols::G, Cols::X);
+
+        // --------------------------------------------- backward sweep
+        to_st(Cols::G);
+        sync();
+        float cum = 0.f;  // sum of dL over the later tokens of the block
+        for (int sb = nsb - 1; sb >= 0; --sb, ++li) {
+            const int64_t t0 = tb + (int64_t)sb * T;
+            begin_item();
+            prep(t0, te, kSweepBwd);
+            float gbv[H];
+            if (!slow) {
+                run_mma(kSweepBwd);
+                float r[H];
+                tc::tmem_ld8(trow + Cols::R + half * H, r);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < H; ++q) gbv[q] = Elast * Qv[q] * r[q];
+                write_bc_tmem(0, t0, te);
+                tmem_axpy(Cols::G, Elast, Cols::D);
+            } else {
+                for (int e = tid; e < T * N; e += NT) (&sm.acc[0][0])[e] = 0.f;
+                __syncthreads();
+                bwd_exact(gbv, true);
+                __syncthreads();
+                write_bc_smem(0, t0, te);
+            }
+            // per-(token, channel) gradients
+            const typename Sm::Raw& r = sm.raw[li & 1];
+            float dl[H];
+            tc::tmem_ld8(trow + Cols::DL + sb * T + half * H, dl);
+            tc::tmem_ld_wait();
+            float sfx[H];
+            float run = 0.f;
+#pragma unroll
+            for (int q = H - 1; q >= 0; --q) {
+                run += dl[q] - iv[q] * hv[q] * gbv[q];
+                sfx[q] = run;
+            }
+            if (half == 1) sm.x1[ch] = run; else sm.x2[ch] = run;
+            __syncthreads();
+            const float S1 = sm.x1[ch], S0 = sm.x2[ch];
+            const float base = cum + tail + (half == 0 ? S1 : 0.f);
+            cum += S0 + S1;
+#pragma unroll
+            for (int q = 0; q < H; ++q) {
+                const int tt = half * H + q;
+                const int64_t t = t0 + tt;
+                float dpv = 0.f;
+                if (q < nvh) {
+                    const float dh = fmaf(Dc, dyv[q], iv[q] * gbv[q]);
+                    gda[t * d] = from_f<Tout>((base + sfx[q]) * (1.f - fv[q]));
+                    gdb[t * d] = from_f<Tout>(hv[q] * gbv[q] * iv[q] * (1.f - iv[q]));
+                    dD_acc = fmaf(dyv[q], hv[q], dD_acc);
+                    if (CONV) {
+                        dpv = dh * dsiluf_(pre[q]);
+                        dw0 = fmaf(dpv, to_f(r.u[tt][ch]), dw0);
+                        dw1 = fmaf(dpv, to_f(r.u[tt + 1][ch]), dw1);
+                        dw2 = fmaf(dpv, to_f(r.u[tt + 2][ch]), dw2);
+                        dw3 = fmaf(dpv, to_f(r.u[tt + 3][ch]), dw3);
+                        dbias += dpv;
+                    } else {
+                        gdhu[t * d] = from_f<Tout>(dh);
+                    }
+                }
+                if (CONV) sm.dp[tt][ch] = dpv;
+            }
+            if (CONV) {
+                __syncthreads();
+                // du_t = w3 dp_t + w2 dp_{t+1} + w1 dp_{t+2} + w0 dp_{t+3}
+#pragma unroll
+                for (int q = 0; q < H; ++q) {
+                    const int tt = half * H + q;
+                    const int64_t t = t0 + tt;
+                    if (q < nvh) {
+                        const float duv = w3 * sm.dp[tt][ch] + w2 * sm.dp[tt + 1][ch] +
+                                          w1 * sm.dp[tt + 2][ch] + w0 * sm.dp[tt + 3][ch];
+                        if (!lastg && group_end_block && t >= te - 3) {
+                            edge[(3 + (t - (te - 3))) * d + c] = duv;  // partial, fixed up later
+                        } else {
+                            gdhu[t * d] = from_f<Tout>(duv);
+                        }
+                        if (k == kb0 && sb == 0 && tt < 3) edge[tt * d + c] = sm.dp[tt][ch];
+                    }
+                }
+                __syncthreads();
+                if (half == 0 && tid < P) {  // first three dp rows -> halo of the earlier sub-chunk
+                    sm.dp[T][ch] = sm.dp[0][ch];
+                    sm.dp[T + 1][ch] = sm.dp[1][ch];
+                    sm.dp[T + 2][ch] = sm.dp[2][ch];
+                }
+            }
+            sync();
+            to_st(Cols::G);  // carry entering the earlier sub-chunk's end
+            sync();
+        }
+    }
+
+    // ------------------------------------------------ carries and partials
+    if (firstg && p.dx0) tmem_to(Cols::G, p.dx0 + (int64_t)bb * d * N);
+    {
+        float* cpart = p.chan_part + ((int64_t)bb * p.ngroups + g) * d * 8;
+        float* red6 = &sm.acc[0][0];  // [6][P] (T * N >= 6 * P)
+        __syncthreads();
+        for (int i = tid; i < 6 * P; i += NT) red6[i] = 0.f;
+        __syncthreads();
+        if (cvalid) {
+            atomicAdd(&red6[0 * P + ch], dD_acc);
+            atomicAdd(&red6[1 * P + ch], dw0);
+            atomicAdd(&red6[2 * P + ch], dw1);
+            atomicAdd(&red6[3 * P + ch], dw2);
+            atomicAdd(&red6[4 * P + ch], dw3);
+            atomicAdd(&red6[5 * P + ch], dbias);
+        }
+        __syncthreads();
+        if (tid < P && c0 + tid < d) {
+#pragma unroll
+            for (int q = 0; q < 6; ++q) cpart[(c0 + tid) * 8 + q] = red6[q * P + tid];
+        }
+    }
+    if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
+    sync();
+    if (warp == 0) tc::tmem_dealloc(tbase, Cols::ALLOC);
+}
+
+template <typename Tout, int N, bool CONV>
+static cudaError_t launch_bwd_tc_t(const BwdParams& p, cudaStream_t st) {
+    BwdTmaps tm;
+    memset(&tm, 0, sizeof(tm));
+    const int T = kBT;
+    bool ok = tma_encode_bf16_3d(&tm.u, p.hu, p.Bt, p.L, p.d, T + 3, 128) &&
+              tma_encode_bf16_3d(&tm.a, p.a, p.Bt, p.L, p.d, T, 128) &&
+              tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, T, 128) &&
+              tma_encode_bf16_3d(&tm.dy, p.dy, p.Bt, p.L, p.d, T, 128) &&
+              tma_encode_bf16_3d(&tm.B, p.B, p.Bt, p.L, N, T, N) &&
+              tma_encode_bf16_3d(&tm.C, p.C, p.Bt, p.L, N, T, N);
+    if (ok && p.z) ok = tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, T, 128);
+    if (!ok) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(BwdTcSmem<N>);
+    auto kern = scan_bwd_tc_kernel<Tout, N, CONV>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = p.ngroups * (int)p.Bt * p.ntiles;
+    kern<<<grid, 256, smem, st>>>(p, tm);
+    return cudaGetLastError();
+}
+
+bool bwd_tc_supported(int dtype, int64_t N, int64_t d) {
+    return dtype == NAJU_BF16 && (N == 64 || N == 128) && d % 8 == 0;
+}
+
+cudaError_t launch_scan_bwd_tc_main(const BwdParams& p, int out_dtype, cudaStream_t st) {
+    const bool conv = p.conv_w != nullptr;
+#define NAJU_TC_BWD(TO, NN)                                                     \
+    return conv ? launch_bwd_tc_t<TO, NN, true>(p, st) : launch_bwd_tc_t<TO, NN, false>(p, st)
+    if (out_dtype == NAJU_BF16) {
+        if (p.N == 64) NAJU_TC_BWD(__nv_bfloat16, 64);
+        if (p.N == 128) NAJU_TC_BWD(__nv_bfloat16, 128);
+    } else {
+        if (p.N == 64) NAJU_TC_BWD(float, 64);
+        if (p.N == 128) NAJU_TC_BWD(float, 128);
+    }
+#undef NAJU_TC_BWD
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace naju

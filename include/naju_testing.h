@@ -43,12 +43,22 @@ void naju_testing_set_bwd_groups(int32_t groups);
 int32_t naju_testing_bwd_groups(const void* dims);
 
 /* Forward implementation: 0 = automatic (tensor cores for bf16 activations
- * with d_state 64 or 128, CUDA cores otherwise), 1 = always CUDA cores. */
+ * with d_state 64 or 128 and d_inner % 8 == 0, CUDA cores otherwise),
+ * 1 = always CUDA cores. */
 void naju_testing_set_fwd_impl(int32_t impl);
 
 /* The forward implementation for these dims: 1 = CUDA cores, 2 = tensor
  * cores (0 for invalid dims). */
 int32_t naju_testing_fwd_impl(const void* dims);
+
+/* Backward implementation: 0 = automatic (tensor cores for bf16 activations
+ * with d_state 64 or 128 and d_inner % 8 == 0, CUDA cores otherwise),
+ * 1 = always CUDA cores. */
+void naju_testing_set_bwd_impl(int32_t impl);
+
+/* The backward implementation for these dims: 1 = CUDA cores, 2 = tensor
+ * cores (0 for invalid dims). */
+int32_t naju_testing_bwd_impl(const void* dims);
 
 /* Self-test of the tensor-core building block of the tensor-core scans:
  * D[128 x N] = A[128 x K] * B[N x K]^T (device pointers, row-major fp32)

@@ -286,6 +286,71 @@ def test_bwd_sequence_groups(groups):
     compare_grads(g, r, True, TOL_F32)
 
 
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("impl", [1, 0])
+@pytest.mark.parametrize("conv", [True, False])
+def test_bwd_both_implementations(N, impl, conv):
+    """The CUDA-core and tensor-core backwards both match the oracle (bf16
+    inputs; 3 channel tiles, the last ragged; a ragged last block)."""
+    w = wl(N, "bf16", Bt=2, L=333, d=264)
+    t = inputs(w, conv, use_x0=True, use_dxL=True)
+    dm = naju.make_dims(2, 333, 264, N, naju.BF16)
+    naju.testing_set_bwd_impl(impl)
+    try:
+        assert naju.testing_bwd_impl(dm) == (1 if impl == 1 else 2)
+        g = run_bwd(t, conv, out_dtype=naju.F32)
+    finally:
+        naju.testing_set_bwd_impl(0)
+    r = oracle_bwd(t, conv)
+    compare_grads(g, r, conv, TOL_BF16)
+
+
+def test_bwd_tensor_core_bf16_outputs():
+    w = wl(64, "bf16", Bt=2, L=200, d=136)
+    t = inputs(w, True)
+    assert naju.testing_bwd_impl(naju.make_dims(2, 200, 136, 64, naju.BF16)) == 2
+    g = run_bwd(t, True, out_dtype=naju.BF16)
+    r = oracle_bwd(t, True)
+    compare_grads(g, r, True, TOL_BF16, bf16_out=True)
+
+
+def test_bwd_tensor_core_no_optional_inputs():
+    w = wl(128, "bf16", Bt=1, L=150, d=128)
+    t = inputs(w, False, use_z=False, use_D=False)
+    g = run_bwd(t, False, out_dtype=naju.F32)
+    r = oracle_bwd(t, False)
+    compare_grads(g, r, False, TOL_BF16, has_z=False, has_D=False)
+
+
+@pytest.mark.parametrize("N", [64, 128])
+def test_bwd_tensor_core_exact_fallback(N):
+    """Runs of vanishing forget gates: sub-chunks whose decay would overflow
+    the tensor-core factorisation take the exact path in both sweeps."""
+    w = wl(N, "bf16", Bt=1, L=300, d=136)
+    t = inputs(w, True, use_x0=True, use_dxL=True)
+    a = t["a"].float().clone()
+    a[:, 40:60] = -60.0
+    a[:, 100:200:2] = -25.0
+    a[:, 220:240] = 60.0
+    t["a"] = a.to(torch.bfloat16)
+    g = run_bwd(t, True, out_dtype=naju.F32)
+    r = oracle_bwd(t, True)
+    compare_grads(g, r, True, TOL_BF16)
+
+
+@pytest.mark.parametrize("groups", [2, 3])
+def test_bwd_tensor_core_sequence_groups(groups):
+    w = wl(64, "bf16", Bt=2, L=600, d=136)
+    t = inputs(w, True, use_x0=True, use_dxL=True)
+    r = oracle_bwd(t, True)
+    naju.testing_set_bwd_groups(groups)
+    try:
+        g = run_bwd(t, True, out_dtype=naju.F32)
+    finally:
+        naju.testing_set_bwd_groups(0)
+    compare_grads(g, r, True, TOL_BF16)
+
+
 def test_bwd_after_grouped_forward():
     """Checkpoints written by a sequence-split forward serve the backward."""
     w = wl(64, "f32", Bt=1, L=700, d=64)

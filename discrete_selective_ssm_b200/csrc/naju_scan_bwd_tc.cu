@@ -33,6 +33,11 @@
 // M = 128 MMA whose upper rows are ignored.  The small A_C / A_B products and
 // everything per (token, channel) run on the CUDA cores.
 //
+// Threads.  512 per block: channel p (TMEM lane p) is handled by threads
+// p + 128 q, q = 0..3, each taking 4 of the 16 tokens and a quarter of the
+// state columns; one thread issues the MMAs.  Raw inputs arrive by TMA one
+// sub-chunk ahead (two buffers).
+//
 // Exactness.  A sub-chunk whose product of 1/f exceeds 2^64 in any channel of
 // the block takes an exact token-by-token path on the CUDA cores (states in
 // tensor memory, channel sums of dB / dC through warp shuffles).
@@ -103,12 +108,12 @@ struct BwdTcSmem {
     alignas(128) float tg[T * T];      // G[t][m] (forward) / G^T (backward)
     alignas(128) float ta2[T * T];     // A_C (forward) / A_B (backward)
     alignas(16) float y1[T][P + 4];    // Y / P rows (slow path: s dy or v)
-    alignas(16) float w1[T][P + 4];    // W / U rows (slow path: exchange of half sums)
+    alignas(16) float w1[T][P + 4];    // W / U rows (slow path: sums over quarters)
     alignas(16) float brow[T][N + 4];
     alignas(16) float crow[T][N + 4];
     float dp[T + 3][P];
     float acc[T][N];                   // slow path channel sums
-    float x0[P], x1[P], x2[P];         // per-half exchanges
+    float xq[4][P], xe[4][P], xs[4][P];  // exchanges between a channel's four threads
     uint64_t loaded[2], mma;
     uint32_t taddr;
     int item, ok;
@@ -119,12 +124,12 @@ enum { kSweepFwd = 0, kSweepBwd = 1, kSweepEarly = 2 };
 }  // namespace
 
 template <typename Tout, int N, bool CONV>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(512, 1)
 scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     using Tin = __nv_bfloat16;
     using Cols = BCols<N>;
     using Sm = BwdTcSmem<N>;
-    constexpr int T = kBT, P = 128, H = T / 2, NT = 256, NH = N / 2;
+    constexpr int T = kBT, P = 128, NT = 512, TQ = T / 4, NC = N / 4;
     constexpr int K = kBwdSub;  // tokens per block (forward checkpoint spacing)
     extern __shared__ __align__(1024) float4 smem4[];
     Sm& sm = *reinterpret_cast<Sm*>(smem4);
@@ -132,7 +137,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int ch = tid & (P - 1);   // channel within the block = TMEM lane
-    const int half = tid >> 7;      // tokens [8 half, 8 half + 8) / columns [N/2 half, ...)
+    const int qd = tid >> 7;        // tokens [4 qd, 4 qd + 4), state columns [N/4 qd, ...)
     const int64_t Bt = p.Bt, L = p.L, d = p.d;
     const float s = p.scale;
     const bool has_z = p.z != nullptr;
@@ -252,26 +257,26 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     // element (row j, k = channel).
     auto to_st = [&](uint32_t col) {
 #pragma unroll
-        for (int n0 = 0; n0 < NH; n0 += 16) {
+        for (int n0 = 0; n0 < NC; n0 += 16) {
             float v[16];
-            tc::tmem_ld16(trow + col + half * NH + n0, v);
+            tc::tmem_ld16(trow + col + qd * NC + n0, v);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int k = 0; k < 16; ++k)
-                sm.st[tc::sw128_offset(half * NH + n0 + k, ch, N) >> 2] = cvalid ? v[k] : 0.f;
+                sm.st[tc::sw128_offset(qd * NC + n0 + k, ch, N) >> 2] = cvalid ? v[k] : 0.f;
         }
     };
-    // TMEM columns [col, col + N) of this row <-> global rows (half each).
+    // TMEM columns [col, col + N) of this row <-> global rows (a quarter each).
     auto tmem_from = [&](uint32_t col, const float* src, bool cg) {
 #pragma unroll
-        for (int n0 = 0; n0 < NH; n0 += 16) {
+        for (int n0 = 0; n0 < NC; n0 += 16) {
             float v[16];
 #pragma unroll
             for (int k = 0; k < 16; k += 4) {
                 float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (src && cvalid) {
                     const float4* s4 =
-                        reinterpret_cast<const float4*>(src + c * N + half * NH + n0 + k);
+                        reinterpret_cast<const float4*>(src + c * N + qd * NC + n0 + k);
                     v4 = cg ? __ldcg(s4) : *s4;
                 }
                 v[k] = v4.x;
@@ -279,64 +284,64 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 v[k + 2] = v4.z;
                 v[k + 3] = v4.w;
             }
-            tc::tmem_st16(trow + col + half * NH + n0, v);
+            tc::tmem_st16(trow + col + qd * NC + n0, v);
         }
         tc::tmem_st_wait();
     };
     auto tmem_to = [&](uint32_t col, float* dst) {
 #pragma unroll
-        for (int n0 = 0; n0 < NH; n0 += 16) {
+        for (int n0 = 0; n0 < NC; n0 += 16) {
             float v[16];
-            tc::tmem_ld16(trow + col + half * NH + n0, v);
+            tc::tmem_ld16(trow + col + qd * NC + n0, v);
             tc::tmem_ld_wait();
             if (cvalid) {
 #pragma unroll
                 for (int k = 0; k < 16; k += 4)
-                    *reinterpret_cast<float4*>(dst + c * N + half * NH + n0 + k) =
+                    *reinterpret_cast<float4*>(dst + c * N + qd * NC + n0 + k) =
                         make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
             }
         }
     };
-    // Dot of TMEM columns [ca, ca + N) and [cb, cb + N) of this row (both halves).
+    // Dot of TMEM columns [ca, ca + N) and [cb, cb + N) of this row (all quarters).
     auto tmem_dot = [&](uint32_t ca, uint32_t cb) -> float {
         float acc = 0.f;
 #pragma unroll
-        for (int n0 = 0; n0 < NH; n0 += 16) {
+        for (int n0 = 0; n0 < NC; n0 += 16) {
             float va[16], vb[16];
-            tc::tmem_ld16(trow + ca + half * NH + n0, va);
-            tc::tmem_ld16(trow + cb + half * NH + n0, vb);
+            tc::tmem_ld16(trow + ca + qd * NC + n0, va);
+            tc::tmem_ld16(trow + cb + qd * NC + n0, vb);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int k = 0; k < 16; ++k) acc = fmaf(va[k], vb[k], acc);
         }
-        if (half == 1) sm.x1[ch] = acc;
+        sm.xs[qd][ch] = acc;
         __syncthreads();
-        acc += half == 0 ? sm.x1[ch] : 0.f;
-        if (half == 0) sm.x2[ch] = acc;
+        acc = (sm.xs[0][ch] + sm.xs[1][ch]) + (sm.xs[2][ch] + sm.xs[3][ch]);
         __syncthreads();
-        return sm.x2[ch];
+        return acc;
     };
     // Scale-and-add on TMEM: col_a <- m * col_a + (col_b or a global row).
     auto tmem_axpy = [&](uint32_t ca, float m, uint32_t cb) {
 #pragma unroll
-        for (int n0 = 0; n0 < NH; n0 += 16) {
+        for (int n0 = 0; n0 < NC; n0 += 16) {
             float va[16], vb[16];
-            tc::tmem_ld16(trow + ca + half * NH + n0, va);
-            tc::tmem_ld16(trow + cb + half * NH + n0, vb);
+            tc::tmem_ld16(trow + ca + qd * NC + n0, va);
+            tc::tmem_ld16(trow + cb + qd * NC + n0, vb);
             tc::tmem_ld_wait();
 #pragma unroll
             for (int k = 0; k < 16; ++k) va[k] = fmaf(m, va[k], vb[k]);
-            tc::tmem_st16(trow + ca + half * NH + n0, va);
+            tc::tmem_st16(trow + ca + qd * NC + n0, va);
         }
         tc::tmem_st_wait();
     };
 
     // ------------------------------------------------- per-item state
-    // Per (token, channel) values of this thread's 8 tokens.
-    float fv[H], qv[H], hv[H], iv[H], dyv[H], pre[H], Ev[H], Qv[H];
+    // Per (token, channel) values of this thread's 4 tokens; aux is SiLU'(z)
+    // in the forward sweep and SiLU'(conv pre-activation) in the backward.
+    float fv[TQ], qv[TQ], hv[TQ], iv[TQ], dyv[TQ], aux[TQ], Ev[TQ], Qv[TQ];
     float Elast = 1.f;
     bool slow = false;
-    int nvh = 0;  // valid tokens of this thread's half
+    int nvh = 0;  // valid tokens of this thread's quarter
 
     // Unpack item `li` (raw buffer li & 1) for a sweep; fills the registers
     // above, the TMEM operand columns and the per-token tiles.  Returns after
@@ -350,44 +355,59 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             *reinterpret_cast<float4*>(&sm.brow[tt][j]) = bf4(&r.Bm[tt][j]);
             *reinterpret_cast<float4*>(&sm.crow[tt][j]) = bf4(&r.Cm[tt][j]);
         }
-        nvh = cvalid ? (int)max((int64_t)0, min64((int64_t)H, te - t0 - half * H)) : 0;
+        nvh = cvalid ? (int)max((int64_t)0, min64((int64_t)TQ, te - t0 - qd * TQ)) : 0;
         float Qh = 1.f, Eh = 1.f;
 #pragma unroll
-        for (int k = 0; k < H; ++k) {
-            const int tt = half * H + k;
+        for (int k = 0; k < TQ; ++k) {
+            const int tt = qd * TQ + k;
             const bool valid = k < nvh;
             qv[k] = valid ? 1.f + __expf(-to_f(r.a[tt][ch])) : 1.f;
             fv[k] = rcpa_(qv[k]);
             Qh *= qv[k];
             Eh *= fv[k];
-            float hh, pp = 0.f;
+            float hh, ax = 0.f;
             if (CONV) {
-                pp = wb + w0 * to_f(r.u[tt][ch]) + w1 * to_f(r.u[tt + 1][ch]) +
-                     w2 * to_f(r.u[tt + 2][ch]) + w3 * to_f(r.u[tt + 3][ch]);
-                hh = siluf_(pp);
+                const float pp = wb + w0 * to_f(r.u[tt][ch]) + w1 * to_f(r.u[tt + 1][ch]) +
+                                 w2 * to_f(r.u[tt + 2][ch]) + w3 * to_f(r.u[tt + 3][ch]);
+                const float sp = sigmoida_(pp);
+                hh = pp * sp;
+                ax = sp * fmaf(pp, 1.f - sp, 1.f);
             } else {
                 hh = to_f(r.u[tt + 3][ch]);
             }
-            pre[k] = pp;
             hv[k] = valid ? hh : 0.f;
-            iv[k] = sigmoidf_(to_f(r.b[tt][ch]));
-            const float gg = has_z ? siluf_(to_f(r.z[tt][ch])) : 1.f;
+            iv[k] = sigmoida_(to_f(r.b[tt][ch]));
+            float gg = 1.f;
+            if (has_z) {
+                const float zv = to_f(r.z[tt][ch]);
+                const float sz = sigmoida_(zv);
+                gg = zv * sz;
+                if (fwd) ax = sz * fmaf(zv, 1.f - sz, 1.f);
+            }
+            aux[k] = ax;
             dyv[k] = valid ? to_f(r.dy[tt][ch]) * gg : 0.f;
         }
-        if (half == 0) {
-            sm.x0[ch] = Qh;
-            sm.x1[ch] = Eh;
-        } else {
-            sm.x2[ch] = Eh;
-        }
+        sm.xq[qd][ch] = Qh;
+        sm.xe[qd][ch] = Eh;
         __syncthreads();
-        const float Q0 = sm.x0[ch], E0 = sm.x1[ch], E1 = sm.x2[ch];
-        slow = __syncthreads_or(half == 1 && !(Q0 * Qh <= kBBound)) != 0;
-        Elast = E0 * E1;
         {
-            float Q = half ? Q0 : 1.f, E = half ? E0 : 1.f;
+            // decay products of the earlier quarters and of the whole sub-chunk
+            float Qb = 1.f, Eb = 1.f, Qa = 1.f, Ea = 1.f;
 #pragma unroll
-            for (int k = 0; k < H; ++k) {
+            for (int q = 0; q < 4; ++q) {
+                const float xq = sm.xq[q][ch], xe = sm.xe[q][ch];
+                if (q < qd) {
+                    Qb *= xq;
+                    Eb *= xe;
+                }
+                Qa *= xq;
+                Ea *= xe;
+            }
+            slow = __syncthreads_or(qd == 0 && !(Qa <= kBBound)) != 0;
+            Elast = Ea;
+            float Q = Qb, E = Eb;
+#pragma unroll
+            for (int k = 0; k < TQ; ++k) {
                 E *= fv[k];
                 Q *= qv[k];
                 Ev[k] = E;
@@ -395,11 +415,11 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             }
         }
         // Per-(token, channel) operands.
-        float c1[H], c2[H];
+        float c1[TQ], c2[TQ];
         const float QL = rcpa_(Elast);  // product of q over the sub-chunk (fast path)
 #pragma unroll
-        for (int k = 0; k < H; ++k) {
-            const int tt = half * H + k;
+        for (int k = 0; k < TQ; ++k) {
+            const int tt = qd * TQ + k;
             const float v = iv[k] * hv[k];
             if (fwd) {
                 // W (readout weights), V (state weights), Y = s dy E.
@@ -423,8 +443,8 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 }
             }
         }
-        tc::tmem_st8(trow + Cols::WU + half * H, c1);
-        tc::tmem_st8(trow + Cols::VV + half * H, c2);
+        tc::tmem_st4(trow + Cols::WU + qd * TQ, c1);
+        tc::tmem_st4(trow + Cols::VV + qd * TQ, c2);
         tc::tmem_st_wait();
         __syncthreads();  // brow, crow, y1, w1 complete
         if (!slow) {
@@ -445,30 +465,39 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             if (sweep != kSweepEarly) {
                 // tg: forward G[t][m] = C_t . B_m (m <= t); backward G^T[t][t'] = C_t' . B_t
                 // (t' >= t).  ta2: A_C[t][m] = sum_ch Y_t W_m (m <= t) or
-                // A_B[t][t'] = sum_ch P_t U_t' (t' >= t).  One entry per thread.
-                const int tt = tid / T, mm = tid % T;
+                // A_B[t][t'] = sum_ch P_t U_t' (t' >= t).  One entry per pair of
+                // adjacent threads, each taking half of the sum.
+                const int e = tid >> 1, part = tid & 1;
+                const int tt = e / T, mm = e % T;
                 const bool live = fwd ? (mm <= tt) : (mm >= tt);
                 float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
                 if (live) {
-                    const float* cr = fwd ? sm.crow[tt] : sm.crow[mm];
-                    const float* br = fwd ? sm.brow[mm] : sm.brow[tt];
+                    const float* cr = (fwd ? sm.crow[tt] : sm.crow[mm]) + part * (N / 2);
+                    const float* br = (fwd ? sm.brow[mm] : sm.brow[tt]) + part * (N / 2);
 #pragma unroll 4
-                    for (int j = 0; j < N; j += 4) {
+                    for (int j = 0; j < N / 2; j += 4) {
                         const float4 cv = *reinterpret_cast<const float4*>(cr + j);
                         const float4 bv = *reinterpret_cast<const float4*>(br + j);
                         acc = __ffma2_rn(make_float2(cv.x, cv.y), make_float2(bv.x, bv.y), acc);
                         acc = __ffma2_rn(make_float2(cv.z, cv.w), make_float2(bv.z, bv.w), acc);
                     }
+                    const float* yr = &sm.y1[tt][part * (P / 2)];
+                    const float* wr = &sm.w1[mm][part * (P / 2)];
 #pragma unroll 4
-                    for (int q = 0; q < P; q += 4) {
-                        const float4 yv = *reinterpret_cast<const float4*>(&sm.y1[tt][q]);
-                        const float4 wv = *reinterpret_cast<const float4*>(&sm.w1[mm][q]);
+                    for (int q = 0; q < P / 2; q += 4) {
+                        const float4 yv = *reinterpret_cast<const float4*>(yr + q);
+                        const float4 wv = *reinterpret_cast<const float4*>(wr + q);
                         acc2 = __ffma2_rn(make_float2(yv.x, yv.y), make_float2(wv.x, wv.y), acc2);
                         acc2 = __ffma2_rn(make_float2(yv.z, yv.w), make_float2(wv.z, wv.w), acc2);
                     }
                 }
-                sm.tg[tc::kmajor_offset(tt, mm, T) >> 2] = acc.x + acc.y;
-                sm.ta2[tc::kmajor_offset(tt, mm, T) >> 2] = acc2.x + acc2.y;
+                float gsum = acc.x + acc.y, asum = acc2.x + acc2.y;
+                gsum += __shfl_xor_sync(0xffffffffu, gsum, 1);
+                asum += __shfl_xor_sync(0xffffffffu, asum, 1);
+                if (part == 0) {
+                    sm.tg[tc::kmajor_offset(tt, mm, T) >> 2] = gsum;
+                    sm.ta2[tc::kmajor_offset(tt, mm, T) >> 2] = asum;
+                }
             }
         }
         tc::fence_proxy_async();
@@ -534,13 +563,13 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     // = d_state rows, columns = tokens) to the per-tile partial buffer.
     auto write_bc_tmem = [&](int slot, int64_t t0, int64_t te) {
         if ((warp & 3) * 32 < N) {
-            float v[8];
-            tc::tmem_ld8(tbase + lane + Cols::BC + half * H, v);
+            float v[TQ];
+            tc::tmem_ld4(tbase + lane + Cols::BC + qd * TQ, v);
             tc::tmem_ld_wait();
             const int j = ch;  // lane = d_state row
 #pragma unroll
-            for (int k = 0; k < H; ++k) {
-                const int64_t t = t0 + half * H + k;
+            for (int k = 0; k < TQ; ++k) {
+                const int64_t t = t0 + qd * TQ + k;
                 if (t < te) part[t * 2 * N + slot * N + j] = v[k];
             }
         } else {
@@ -561,9 +590,9 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     };
 
     // ----------------------------------------------------------------
-    // Exact forward sub-chunk: token recurrence on this thread's half of
-    // the state columns; x.C partial sums exchanged between halves; dC
-    // channel sums into sm.acc.  Requires sm.acc zeroed.
+    // Exact forward sub-chunk: token recurrence on this thread's quarter of
+    // the state columns; x.C partial sums added over the quarters in sm.w1;
+    // dC channel sums into sm.acc.  Requires sm.acc and sm.w1 zeroed.
     auto fwd_exact = [&](float* ydot) {
         float vv[16], ff[16];
         tc::tmem_ld16(trow + Cols::WU, vv);
@@ -572,7 +601,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         float yp[16];
 #pragma unroll
         for (int tt = 0; tt < T; ++tt) yp[tt] = 0.f;
-        for (int n0 = half * NH; n0 < half * NH + NH; n0 += 16) {
+        for (int n0 = qd * NC; n0 < qd * NC + NC; n0 += 16) {
             float x[16];
             tc::tmem_ld16(trow + Cols::X + n0, x);
             tc::tmem_ld_wait();
@@ -591,20 +620,19 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             tc::tmem_st16(trow + Cols::X + n0, x);
         }
         tc::tmem_st_wait();
-        // exchange: each half needs the other half's partials for its tokens
 #pragma unroll
-        for (int tt = 0; tt < T; ++tt)
-            if ((tt >= H) != (half == 1)) sm.w1[tt][ch] = yp[tt];
+        for (int tt = 0; tt < T; ++tt) atomicAdd(&sm.w1[tt][ch], yp[tt]);
         __syncthreads();
 #pragma unroll
-        for (int k = 0; k < H; ++k) ydot[k] = yp[half * H + k] + sm.w1[half * H + k][ch];
+        for (int k = 0; k < TQ; ++k) ydot[k] = sm.w1[qd * TQ + k][ch];
         float lp = 0.f;
 #pragma unroll
         for (int tt = 0; tt < T; ++tt) lp += __logf(ff[tt]);
         return lp;
     };
-    // Exact backward sub-chunk: adjoint recurrence over this half of the
-    // columns, G.B exchanged between halves, dB channel sums into sm.acc.
+    // Exact backward sub-chunk: adjoint recurrence over this quarter of the
+    // columns, G.B summed over the quarters in sm.w1, dB channel sums into
+    // sm.acc.  Requires sm.acc and sm.w1 zeroed when `grads`.
     auto bwd_exact = [&](float* gbv, bool grads) {
         float sd[16], ff[16];
         tc::tmem_ld16(trow + Cols::WU, sd);
@@ -613,7 +641,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         float gp[16];
 #pragma unroll
         for (int tt = 0; tt < T; ++tt) gp[tt] = 0.f;
-        for (int n0 = half * NH; n0 < half * NH + NH; n0 += 16) {
+        for (int n0 = qd * NC; n0 < qd * NC + NC; n0 += 16) {
             float hx[16];
             tc::tmem_ld16(trow + Cols::G + n0, hx);
             tc::tmem_ld_wait();
@@ -637,11 +665,10 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         tc::tmem_st_wait();
         if (grads) {
 #pragma unroll
-            for (int tt = 0; tt < T; ++tt)
-                if ((tt >= H) != (half == 1)) sm.w1[tt][ch] = gp[tt];
+            for (int tt = 0; tt < T; ++tt) atomicAdd(&sm.w1[tt][ch], gp[tt]);
             __syncthreads();
 #pragma unroll
-            for (int k = 0; k < H; ++k) gbv[k] = gp[half * H + k] + sm.w1[half * H + k][ch];
+            for (int k = 0; k < TQ; ++k) gbv[k] = sm.w1[qd * TQ + k][ch];
         }
         float lp = 0.f;
 #pragma unroll
@@ -669,7 +696,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 tmem_axpy(Cols::G, Elast, Cols::D);
                 logF += __logf(Elast);
             } else {
-                float dummy[H];
+                float dummy[TQ];
                 logF += bwd_exact(dummy, false);
             }
             sync();
@@ -681,22 +708,22 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             // carry out = (decay over the group) H + local contribution
             const float Pf = __expf(logF);
 #pragma unroll
-            for (int n0 = 0; n0 < NH; n0 += 16) {
+            for (int n0 = 0; n0 < NC; n0 += 16) {
                 float hx[16];
-                tc::tmem_ld16(trow + Cols::G + half * NH + n0, hx);
+                tc::tmem_ld16(trow + Cols::G + qd * NC + n0, hx);
                 tc::tmem_ld_wait();
 #pragma unroll
                 for (int k = 0; k < 16; k += 4) {
                     float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
                     if (okc && cvalid)
-                        v4 = __ldcg(reinterpret_cast<const float4*>(carry_in + c * N + half * NH +
+                        v4 = __ldcg(reinterpret_cast<const float4*>(carry_in + c * N + qd * NC +
                                                                     n0 + k));
                     hx[k] = fmaf(Pf, v4.x, hx[k]);
                     hx[k + 1] = fmaf(Pf, v4.y, hx[k + 1]);
                     hx[k + 2] = fmaf(Pf, v4.z, hx[k + 2]);
                     hx[k + 3] = fmaf(Pf, v4.w, hx[k + 3]);
                 }
-                tc::tmem_st16(trow + Cols::G + half * NH + n0, hx);
+                tc::tmem_st16(trow + Cols::G + qd * NC + n0, hx);
             }
             tc::tmem_st_wait();
         }
@@ -733,18 +760,19 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             const int64_t t0 = tb + (int64_t)sb * T;
             begin_item();
             prep(t0, te, kSweepFwd);
-            float yd[H];  // x_t . C_t of this thread's tokens
+            float yd[TQ];  // x_t . C_t of this thread's tokens
             if (!slow) {
                 run_mma(kSweepFwd);
-                float r[H];
-                tc::tmem_ld8(trow + Cols::R + half * H, r);
+                float r[TQ];
+                tc::tmem_ld4(trow + Cols::R + qd * TQ, r);
                 tc::tmem_ld_wait();
 #pragma unroll
-                for (int q = 0; q < H; ++q) yd[q] = Ev[q] * r[q];
+                for (int q = 0; q < TQ; ++q) yd[q] = Ev[q] * r[q];
                 write_bc_tmem(1, t0, te);
                 tmem_axpy(Cols::X, Elast, Cols::D);
             } else {
                 for (int e = tid; e < T * N; e += NT) (&sm.acc[0][0])[e] = 0.f;
+                for (int e = tid; e < T * (P + 4); e += NT) (&sm.w1[0][0])[e] = 0.f;
                 __syncthreads();
                 fwd_exact(yd);
                 __syncthreads();
@@ -753,18 +781,17 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             // dz and s dy (x.C) for the backward sweep
             {
                 const typename Sm::Raw& r = sm.raw[li & 1];
-                float dl[H];
+                float dl[TQ];
 #pragma unroll
-                for (int q = 0; q < H; ++q) {
-                    const int tt = half * H + q;
+                for (int q = 0; q < TQ; ++q) {
+                    const int tt = qd * TQ + q;
                     dl[q] = s * dyv[q] * yd[q];
                     if (has_z && q < nvh) {
-                        const float zv = to_f(r.z[tt][ch]);
                         const float yv = fmaf(s, yd[q], Dc * hv[q]);
-                        gdz[(t0 + tt) * d] = from_f<Tout>(to_f(r.dy[tt][ch]) * yv * dsiluf_(zv));
+                        gdz[(t0 + tt) * d] = from_f<Tout>(to_f(r.dy[tt][ch]) * yv * aux[q]);
                     }
                 }
-                tc::tmem_st8(trow + Cols::DL + sb * T + half * H, dl);
+                tc::tmem_st4(trow + Cols::DL + sb * T + qd * TQ, dl);
                 tc::tmem_st_wait();
             }
             sync();
@@ -782,18 +809,19 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             const int64_t t0 = tb + (int64_t)sb * T;
             begin_item();
             prep(t0, te, kSweepBwd);
-            float gbv[H];
+            float gbv[TQ];
             if (!slow) {
                 run_mma(kSweepBwd);
-                float r[H];
-                tc::tmem_ld8(trow + Cols::R + half * H, r);
+                float r[TQ];
+                tc::tmem_ld4(trow + Cols::R + qd * TQ, r);
                 tc::tmem_ld_wait();
 #pragma unroll
-                for (int q = 0; q < H; ++q) gbv[q] = Elast * Qv[q] * r[q];
+                for (int q = 0; q < TQ; ++q) gbv[q] = Elast * Qv[q] * r[q];
                 write_bc_tmem(0, t0, te);
                 tmem_axpy(Cols::G, Elast, Cols::D);
             } else {
                 for (int e = tid; e < T * N; e += NT) (&sm.acc[0][0])[e] = 0.f;
+                for (int e = tid; e < T * (P + 4); e += NT) (&sm.w1[0][0])[e] = 0.f;
                 __syncthreads();
                 bwd_exact(gbv, true);
                 __syncthreads();
@@ -801,24 +829,30 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             }
             // per-(token, channel) gradients
             const typename Sm::Raw& r = sm.raw[li & 1];
-            float dl[H];
-            tc::tmem_ld8(trow + Cols::DL + sb * T + half * H, dl);
+            float dl[TQ];
+            tc::tmem_ld4(trow + Cols::DL + sb * T + qd * TQ, dl);
             tc::tmem_ld_wait();
-            float sfx[H];
+            float sfx[TQ];
             float run = 0.f;
 #pragma unroll
-            for (int q = H - 1; q >= 0; --q) {
+            for (int q = TQ - 1; q >= 0; --q) {
                 run += dl[q] - iv[q] * hv[q] * gbv[q];
                 sfx[q] = run;
             }
-            if (half == 1) sm.x1[ch] = run; else sm.x2[ch] = run;
+            sm.xs[qd][ch] = run;
             __syncthreads();
-            const float S1 = sm.x1[ch], S0 = sm.x2[ch];
-            const float base = cum + tail + (half == 0 ? S1 : 0.f);
-            cum += S0 + S1;
+            float later = 0.f, total = 0.f;  // sums of dL over later quarters / all
 #pragma unroll
-            for (int q = 0; q < H; ++q) {
-                const int tt = half * H + q;
+            for (int q = 0; q < 4; ++q) {
+                const float v = sm.xs[q][ch];
+                if (q > qd) later += v;
+                total += v;
+            }
+            const float base = cum + tail + later;
+            cum += total;
+#pragma unroll
+            for (int q = 0; q < TQ; ++q) {
+                const int tt = qd * TQ + q;
                 const int64_t t = t0 + tt;
                 float dpv = 0.f;
                 if (q < nvh) {
@@ -827,7 +861,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                     gdb[t * d] = from_f<Tout>(hv[q] * gbv[q] * iv[q] * (1.f - iv[q]));
                     dD_acc = fmaf(dyv[q], hv[q], dD_acc);
                     if (CONV) {
-                        dpv = dh * dsiluf_(pre[q]);
+                        dpv = dh * aux[q];
                         dw0 = fmaf(dpv, to_f(r.u[tt][ch]), dw0);
                         dw1 = fmaf(dpv, to_f(r.u[tt + 1][ch]), dw1);
                         dw2 = fmaf(dpv, to_f(r.u[tt + 2][ch]), dw2);
@@ -843,8 +877,8 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 __syncthreads();
                 // du_t = w3 dp_t + w2 dp_{t+1} + w1 dp_{t+2} + w0 dp_{t+3}
 #pragma unroll
-                for (int q = 0; q < H; ++q) {
-                    const int tt = half * H + q;
+                for (int q = 0; q < TQ; ++q) {
+                    const int tt = qd * TQ + q;
                     const int64_t t = t0 + tt;
                     if (q < nvh) {
                         const float duv = w3 * sm.dp[tt][ch] + w2 * sm.dp[tt + 1][ch] +
@@ -858,7 +892,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                     }
                 }
                 __syncthreads();
-                if (half == 0 && tid < P) {  // first three dp rows -> halo of the earlier sub-chunk
+                if (qd == 0) {  // first three dp rows -> halo of the earlier sub-chunk
                     sm.dp[T][ch] = sm.dp[0][ch];
                     sm.dp[T + 1][ch] = sm.dp[1][ch];
                     sm.dp[T + 2][ch] = sm.dp[2][ch];
@@ -916,7 +950,7 @@ static cudaError_t launch_bwd_tc_t(const BwdParams& p, cudaStream_t st) {
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = p.ngroups * (int)p.Bt * p.ntiles;
-    kern<<<grid, 256, smem, st>>>(p, tm);
+    kern<<<grid, 512, smem, st>>>(p, tm);
     return cudaGetLastError();
 }
 

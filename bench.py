@@ -229,6 +229,11 @@ def main():
     if naju.last_device_status(ws) != 0:
         raise SystemExit("device status not OK after warm-up")
 
+    # Kernels of one step: the forward kernel; the backward kernel, the dB/dC
+    # and channel reductions, and the conv group-edge fixup when the backward
+    # splits the sequence.
+    launches_per_step = 1 + 3 + (1 if naju.testing_bwd_groups(dims) > 1 else 0)
+
     # ---------------------------------------------------------- timed region
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     clk = ClockSampler(local)
@@ -336,14 +341,16 @@ def main():
                        "bwd_gbs": bwd_b / (bwd_ms / 1e3) / 1e9,
                        "fwd_frac_hbm": fwd_b / (fwd_ms / 1e3) / 1e9 / peak,
                        "bwd_frac_hbm": bwd_b / (bwd_ms / 1e3) / 1e9 / peak},
-            "roofline": {"bound": "hbm", "kernel": "scan_bwd" if dom_is_bwd else "scan_fwd",
+            "roofline": {"bound": "hbm",
+                         "kernel": ("naju_scan_bwd: scan_bwd_tc_kernel + reductions" if dom_is_bwd
+                                    else "naju_scan_fwd: scan_fwd_tc_kernel"),
                          "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "alg_bytes": dom_b, "peak_kind": pk_kind},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 5 * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }), flush=True)
     if dist is not None:

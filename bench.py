@@ -5,7 +5,9 @@
 
 One step = one forward (fused conv + scan + readout + SiLU(z) modulation) and
 one backward over one batch of the workload's synthetic inputs, all resident
-in HBM.  Prints one JSON line (rank 0).  Under torchrun each rank runs its own
+in HBM.  With the decode workload (`--workload throughput_decode`) one step is
+one decode token for the whole batch (conv state + scan state updated in
+place).  Prints one JSON line (rank 0).  Under torchrun each rank runs its own
 replica of the workload (batch elements are independent; weak scaling, no
 collective on the data path); time is the max over ranks.
 """
@@ -20,12 +22,14 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from discrete_selective_ssm_b200.workloads import WORKLOADS, make_inputs, scaled  # noqa: E402
+from discrete_selective_ssm_b200.workloads import (WORKLOADS, decode_D, decode_state0,  # noqa: E402
+                                                   decode_step_inputs, make_inputs, scaled)
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
@@ -154,6 +158,165 @@ def run_reference(args, w, rank, world):
     }), flush=True)
 
 
+def decode_bytes(w, E):
+    """Algorithmic HBM bytes of one decode token for the whole batch: inputs
+    u, a, b, z and output y (5 E d), B, C (2 E N), fp32 state read + write
+    (2 d N 4) and conv state read + write (2 d 3 4), per batch element."""
+    d, N = w.d_inner, w.d_state
+    return w.batch * (5 * E * d + 2 * E * N + 2 * d * N * 4 + 2 * d * 3 * 4)
+
+
+def decode_cpu_sample(w, n_batch=8):
+    import oracle
+    st = decode_state0(w)[:n_batch].double().numpy()
+    cs = np.zeros((n_batch, w.d_inner, 3))
+    conv = make_inputs(w, which=("conv_w", "conv_b"))
+    D = decode_D(w)
+    dt, toks, k = 0.0, 0, 0
+    while dt < 10.0 and k < w.decode_steps:
+        s_in = decode_step_inputs(w, k)
+        sl = {kk: v[:n_batch] for kk, v in s_in.items()}
+        t0 = time.perf_counter()
+        _, st, cs = oracle.block_step(st, cs, sl["h"], conv["conv_w"], conv["conv_b"], sl["a"],
+                                      sl["b"], sl["B"], sl["C"], sl["z"], D)
+        dt += time.perf_counter() - t0
+        toks += n_batch
+        k += 1
+    return toks / dt, oracle.num_threads(), f"oracle decode steps, {k} x batch {n_batch} slice of {w.name}, {dt:.1f} s"
+
+
+def run_reference_decode(args, w, rank):
+    if rank != 0:
+        return
+    val, thr, sample = decode_cpu_sample(w)
+    print(json.dumps({
+        "metric": "naju_decode_step_tokens_per_s", "value": val, "unit": "tokens/s",
+        "impl": "reference", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "d_inner": w.d_inner,
+                   "d_state": w.d_state, "conv_state": True},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def run_decode(args, w, rank, world, local):
+    """Decode-step bench: one step = one token (conv + scan step) for the batch."""
+    import discrete_selective_ssm_b200 as naju
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    # A pool of distinct per-token inputs (larger than L2 together), cycled.
+    pool = 64
+    host = [decode_step_inputs(w, k) for k in range(pool)]
+    inp = {k: torch.stack([h[k] for h in host]).to(dev) for k in host[0]}
+    state = decode_state0(w).to(dev)
+    cs = torch.zeros(w.batch, w.d_inner, 3, device=dev)
+    conv = {k: v.to(dev) for k, v in make_inputs(w, which=("conv_w", "conv_b")).items()}
+    D = decode_D(w).to(dev)
+    y = torch.empty((w.batch, w.d_inner), dtype=w.torch_dtype, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(k, src=None):
+        src = src if src is not None else {kk: v[k % pool] for kk, v in inp.items()}
+        naju.scan_step_conv(state, cs, src["h"], src["a"], src["b"], src["B"], src["C"],
+                            conv["conv_w"], conv["conv_b"], src["z"], D, y=y)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(args.steps):
+        step(args.warmup + k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = clk.stop()
+    ms_total = e0.elapsed_time(e1)
+    if dist is not None:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    value = world * w.batch / (ms_step / 1e3)
+
+    # e2e: the token's inputs H2D from pinned memory, y D2H, every step.
+    pinned = {k: v.pin_memory() for k, v in host[0].items()}
+    dev_in = {k: torch.empty_like(v[0]) for k, v in inp.items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y.numel() * y.element_size()
+
+    def e2e_step(k):
+        for kk, v in pinned.items():
+            dev_in[kk].copy_(v, non_blocking=True)
+        step(k, dev_in)
+        y_host.copy_(y, non_blocking=True)
+
+    e2e_step(0)
+    torch.cuda.synchronize()
+    s2, t2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for k in range(args.steps):
+        e2e_step(k)
+    t2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = s2.elapsed_time(t2) / args.steps
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+
+    pk, pk_kind = peaks()
+    E = 2 if w.dtype == "bf16" else 4
+    nb = decode_bytes(w, E)
+    achieved = nb / (ms_step / 1e3) / 1e9
+    peak = float(pk["hbm_gbs"])
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        val, thr, sample = decode_cpu_sample(w)
+        cpu = {"value": val, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+               "sample": sample}
+    if rank == 0:
+        print(json.dumps({
+            "metric": "naju_decode_step_tokens_per_s", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "d_inner": w.d_inner,
+                       "d_state": w.d_state, "conv_state": True, "gating": True,
+                       "parallelism": f"replicas{world}",
+                       "l2": "state (134 MB) and input pool larger than L2 (no flush)"},
+            "roofline": {"bound": "hbm", "kernel": "naju_scan_step_conv: step_kernel",
+                         "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "alg_bytes": nb,
+                         "peak_kind": pk_kind},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * w.batch / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+        }), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -171,7 +334,11 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = WORKLOADS[args.workload]
     if w.decode_steps:
-        raise SystemExit("decode workloads are parity cases; bench a training workload")
+        if args.impl == "reference":
+            run_reference_decode(args, w, rank)
+        else:
+            run_decode(args, w, rank, world, local)
+        return
 
     if args.impl == "reference":
         run_reference(args, w, rank, world)

@@ -69,6 +69,8 @@ def lib(build_if_missing: bool = True):
             L.naju_scan_fwd.argtypes = [dp] + [vp] * 13 + [sz, vp]
             L.naju_scan_bwd.argtypes = [dp] + [vp] * 23 + [sz, vp]
             L.naju_scan_step.argtypes = [i64, i64, i64, i32] + [vp] * 10
+            L.naju_conv_silu_step.argtypes = [i64, i64, i32] + [vp] * 6
+            L.naju_scan_step_conv.argtypes = [i64, i64, i64, i32] + [vp] * 13
             L.naju_last_device_status.argtypes = [vp, vp]
             L.naju_status_string.argtypes = [ctypes.c_int]
             L.naju_status_string.restype = ctypes.c_char_p
@@ -87,7 +89,8 @@ def lib(build_if_missing: bool = True):
             L.naju_testing_bwd_groups.argtypes = [vp]
             L.naju_testing_bwd_groups.restype = i32
             for name in ("naju_conv_silu_fwd", "naju_conv_silu_bwd", "naju_scan_fwd",
-                         "naju_scan_bwd", "naju_scan_step", "naju_last_device_status"):
+                         "naju_scan_bwd", "naju_scan_step", "naju_conv_silu_step",
+                         "naju_scan_step_conv", "naju_last_device_status"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -260,6 +263,39 @@ def scan_step(state, h, a, b, B, C, z=None, D=None, y=None, stream=None):
                                 _ptr(B, "B"), _ptr(C, "C"), _ptr(z, "z"),
                                 _ptr(D, "D", torch.float32), _ptr(state, "state", torch.float32),
                                 _ptr(y, "y"), _stream(stream)), "naju_scan_step")
+    return y
+
+
+def conv_silu_step(conv_state, u, conv_w, conv_b=None, h=None, stream=None):
+    """Decode step of conv + SiLU; `conv_state` [Bt, d, 3] fp32 is updated in
+    place (previous three inputs, oldest first).  Returns h."""
+    Bt, d = u.shape
+    if h is None:
+        h = torch.empty_like(u)
+    _check(lib().naju_conv_silu_step(Bt, d, _dt(u), _ptr(u, "u"),
+                                     _ptr(conv_w, "conv_w", torch.float32),
+                                     _ptr(conv_b, "conv_b", torch.float32),
+                                     _ptr(conv_state, "conv_state", torch.float32),
+                                     _ptr(h, "h"), _stream(stream)), "naju_conv_silu_step")
+    return h
+
+
+def scan_step_conv(state, conv_state, u, a, b, B, C, conv_w, conv_b=None, z=None, D=None,
+                   y=None, stream=None):
+    """One decode step from the pre-conv input u (conv + SiLU fused); `state`
+    and `conv_state` are updated in place.  Returns y."""
+    Bt, d = u.shape
+    N = B.shape[-1]
+    if y is None:
+        y = torch.empty_like(u)
+    _check(lib().naju_scan_step_conv(Bt, d, N, _dt(u), _ptr(u, "u"),
+                                     _ptr(conv_w, "conv_w", torch.float32),
+                                     _ptr(conv_b, "conv_b", torch.float32),
+                                     _ptr(conv_state, "conv_state", torch.float32),
+                                     _ptr(a, "a"), _ptr(b, "b"), _ptr(B, "B"), _ptr(C, "C"),
+                                     _ptr(z, "z"), _ptr(D, "D", torch.float32),
+                                     _ptr(state, "state", torch.float32), _ptr(y, "y"),
+                                     _stream(stream)), "naju_scan_step_conv")
     return y
 
 

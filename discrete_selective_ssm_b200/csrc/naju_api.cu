@@ -298,7 +298,35 @@ naju_status naju_scan_step(int64_t batch, int64_t d_inner, int64_t d_state, int3
     NAJU_REQUIRE(ok_act(h) && ok_act(a) && ok_act(b) && ok_act(B) && ok_act(C) && ok_act(y));
     NAJU_REQUIRE(ok_opt(z) && ok_act(state));
     return cuda_status(launch_scan_step(batch, d_inner, d_state, h, a, b, B, C, z, D, state, y,
-                                        dtype, static_cast<cudaStream_t>(stream)));
+                                        dtype, nullptr, nullptr, nullptr,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+naju_status naju_conv_silu_step(int64_t batch, int64_t d_inner, int32_t dtype, const void* u,
+                                const float* conv_w, const float* conv_b, float* conv_state,
+                                void* h, void* stream) {
+    if (batch < 1 || d_inner < 1 || batch > (1 << 20) || d_inner > (1 << 20))
+        return NAJU_ERR_INVALID_ARG;
+    if (dtype != NAJU_F32 && dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
+    NAJU_REQUIRE(ok_act(u) && ok_act(h) && conv_w && ok_act(conv_state) && ok_opt(conv_b));
+    return cuda_status(launch_conv_step(batch, d_inner, u, conv_w, conv_b, conv_state, h, dtype,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+naju_status naju_scan_step_conv(int64_t batch, int64_t d_inner, int64_t d_state, int32_t dtype,
+                                const void* u, const float* conv_w, const float* conv_b,
+                                float* conv_state, const void* a, const void* b, const void* B,
+                                const void* C, const void* z, const float* D, float* state,
+                                void* y, void* stream) {
+    if (batch < 1 || d_inner < 1 || batch > 65535) return NAJU_ERR_INVALID_ARG;
+    if (d_state != 16 && d_state != 32 && d_state != 64 && d_state != 128)
+        return NAJU_ERR_UNSUPPORTED;
+    if (dtype != NAJU_F32 && dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
+    NAJU_REQUIRE(ok_act(u) && ok_act(a) && ok_act(b) && ok_act(B) && ok_act(C) && ok_act(y));
+    NAJU_REQUIRE(ok_opt(z) && ok_act(state) && conv_w && ok_act(conv_state) && ok_opt(conv_b));
+    return cuda_status(launch_scan_step(batch, d_inner, d_state, u, a, b, B, C, z, D, state, y,
+                                        dtype, conv_w, conv_b, conv_state,
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 naju_status naju_last_device_status(void* workspace, void* stream) {

@@ -5,6 +5,8 @@
 //   p_t = bias + sum_{k<4} w[k] u_{t-3+k} (zero left padding), h_t = SiLU(p_t).
 // Decode step (README, "Core equations", one token on a carried state):
 //   x <- sigmoid(a) x + sigmoid(b) h B^T,  y = (x . C)/sqrt(N) + D h,  y *= SiLU(z).
+#include <algorithm>
+
 #include "naju_common.cuh"
 #include "naju_kernels.h"
 
@@ -136,12 +138,17 @@ cudaError_t launch_conv_bwd(int64_t Bt, int64_t L, int64_t d, const void* u, con
 // ------------------------------------------------------------ decode step
 // S = N/4 threads share a channel, each holding 4 consecutive state entries,
 // so a warp's float4 accesses cover whole contiguous state rows.
-template <typename T, int N>
+// One decode token: x <- f x + i h B^T, y = (x.C s + D h) SiLU(z).  With CONV,
+// h = SiLU(bias + w0 s0 + w1 s1 + w2 s2 + w3 u) from the conv state
+// s = (s0, s1, s2) (the previous three inputs, oldest first), which then
+// becomes (s1, s2, u).
+template <typename T, int N, bool CONV>
 __global__ void __launch_bounds__(256)
 step_kernel(int64_t d, const T* __restrict__ h, const T* __restrict__ a,
             const T* __restrict__ b, const T* __restrict__ B, const T* __restrict__ C,
             const T* __restrict__ z, const float* __restrict__ D, float* __restrict__ state,
-            T* __restrict__ y, float scale) {
+            T* __restrict__ y, float scale, const float* __restrict__ conv_w,
+            const float* __restrict__ conv_b, float* __restrict__ conv_state) {
     constexpr int S = N / 4;
     constexpr int P = 256 / S;
     __shared__ float4 sB[N / 4], sC[N / 4];
@@ -164,7 +171,23 @@ step_kernel(int64_t d, const T* __restrict__ h, const T* __restrict__ a,
     const int64_t e = bb * d + c;
     float f = 0.f, v = 0.f, hv = 0.f;
     if (valid) {
-        hv = to_f(h[e]);
+        if (CONV) {
+            const float u = to_f(h[e]);
+            const float s0 = conv_state[e * 3], s1 = conv_state[e * 3 + 1],
+                        s2 = conv_state[e * 3 + 2];
+            const float p = (conv_b ? conv_b[c] : 0.f) + conv_w[c * 4] * s0 +
+                            conv_w[c * 4 + 1] * s1 + conv_w[c * 4 + 2] * s2 +
+                            conv_w[c * 4 + 3] * u;
+            hv = siluf_(p);
+            __syncwarp(__activemask());
+            if (js == 0) {
+                conv_state[e * 3] = s1;
+                conv_state[e * 3 + 1] = s2;
+                conv_state[e * 3 + 2] = u;
+            }
+        } else {
+            hv = to_f(h[e]);
+        }
         f = sigmoidf_(to_f(a[e]));
         v = sigmoidf_(to_f(b[e])) * hv;
     }
@@ -188,18 +211,19 @@ step_kernel(int64_t d, const T* __restrict__ h, const T* __restrict__ a,
     }
 }
 
-template <typename T>
+template <typename T, bool CONV>
 static cudaError_t step_t(int64_t Bt, int64_t d, int64_t N, const void* h, const void* a,
                           const void* b, const void* B, const void* C, const void* z,
-                          const float* D, float* state, void* y, cudaStream_t st) {
+                          const float* D, float* state, void* y, const float* conv_w,
+                          const float* conv_b, float* conv_state, cudaStream_t st) {
     const float scale = 1.0f / sqrtf((float)N);
     const int P = 256 / (int)(N / 4);
     dim3 grid((unsigned)((d + P - 1) / P), (unsigned)Bt);
 #define NAJU_STEP(NN)                                                                     \
-    step_kernel<T, NN><<<grid, 256, 0, st>>>(                                            \
+    step_kernel<T, NN, CONV><<<grid, 256, 0, st>>>(                                      \
         d, static_cast<const T*>(h), static_cast<const T*>(a), static_cast<const T*>(b), \
         static_cast<const T*>(B), static_cast<const T*>(C), static_cast<const T*>(z), D,  \
-        state, static_cast<T*>(y), scale)
+        state, static_cast<T*>(y), scale, conv_w, conv_b, conv_state)
     switch (N) {
         case 16: NAJU_STEP(16); break;
         case 32: NAJU_STEP(32); break;
@@ -214,9 +238,53 @@ static cudaError_t step_t(int64_t Bt, int64_t d, int64_t N, const void* h, const
 cudaError_t launch_scan_step(int64_t Bt, int64_t d, int64_t N, const void* h, const void* a,
                              const void* b, const void* B, const void* C, const void* z,
                              const float* D, float* state, void* y, int dtype,
+                             const float* conv_w, const float* conv_b, float* conv_state,
                              cudaStream_t st) {
-    if (dtype == NAJU_F32) return step_t<float>(Bt, d, N, h, a, b, B, C, z, D, state, y, st);
-    return step_t<__nv_bfloat16>(Bt, d, N, h, a, b, B, C, z, D, state, y, st);
+    const bool conv = conv_w != nullptr;
+    if (dtype == NAJU_F32)
+        return conv ? step_t<float, true>(Bt, d, N, h, a, b, B, C, z, D, state, y, conv_w,
+                                          conv_b, conv_state, st)
+                    : step_t<float, false>(Bt, d, N, h, a, b, B, C, z, D, state, y, nullptr,
+                                           nullptr, nullptr, st);
+    return conv ? step_t<__nv_bfloat16, true>(Bt, d, N, h, a, b, B, C, z, D, state, y, conv_w,
+                                              conv_b, conv_state, st)
+                : step_t<__nv_bfloat16, false>(Bt, d, N, h, a, b, B, C, z, D, state, y, nullptr,
+                                               nullptr, nullptr, st);
+}
+
+// Standalone conv decode step: h = SiLU(bias + w . (s0, s1, s2, u)), state shift.
+template <typename T>
+__global__ void conv_step_kernel(int64_t n, int64_t d, const T* __restrict__ u,
+                                 const float* __restrict__ w, const float* __restrict__ bias,
+                                 float* __restrict__ cs, T* __restrict__ h) {
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t c = e % d;
+        const float uv = to_f(u[e]);
+        const float s0 = cs[e * 3], s1 = cs[e * 3 + 1], s2 = cs[e * 3 + 2];
+        const float p = (bias ? bias[c] : 0.f) + w[c * 4] * s0 + w[c * 4 + 1] * s1 +
+                        w[c * 4 + 2] * s2 + w[c * 4 + 3] * uv;
+        h[e] = from_f<T>(siluf_(p));
+        cs[e * 3] = s1;
+        cs[e * 3 + 1] = s2;
+        cs[e * 3 + 2] = uv;
+    }
+}
+
+cudaError_t launch_conv_step(int64_t Bt, int64_t d, const void* u, const float* w,
+                             const float* bias, float* conv_state, void* h, int dtype,
+                             cudaStream_t st) {
+    const int64_t n = Bt * d;
+    const unsigned blocks = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 16);
+    if (dtype == NAJU_F32)
+        conv_step_kernel<float><<<blocks, 256, 0, st>>>(n, d, static_cast<const float*>(u), w,
+                                                        bias, conv_state,
+                                                        static_cast<float*>(h));
+    else
+        conv_step_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+            n, d, static_cast<const __nv_bfloat16*>(u), w, bias, conv_state,
+            static_cast<__nv_bfloat16*>(h));
+    return cudaGetLastError();
 }
 
 }  // namespace naju

@@ -100,6 +100,10 @@ cudaError_t launch_conv_bwd(int64_t Bt, int64_t L, int64_t d, const void* u, con
 cudaError_t launch_scan_step(int64_t Bt, int64_t d, int64_t N, const void* h, const void* a,
                              const void* b, const void* B, const void* C, const void* z,
                              const float* D, float* state, void* y, int dtype,
+                             const float* conv_w, const float* conv_b, float* conv_state,
+                             cudaStream_t st);
+cudaError_t launch_conv_step(int64_t Bt, int64_t d, const void* u, const float* w,
+                             const float* bias, float* conv_state, void* h, int dtype,
                              cudaStream_t st);
 
 }  // namespace naju

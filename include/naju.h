@@ -149,6 +149,29 @@ naju_status naju_scan_step(int64_t batch, int64_t d_inner, int64_t d_state, int3
                            const void* C, const void* z, const float* D, float* state, void* y,
                            void* stream);
 
+/* Decode step of the causal depthwise conv + SiLU (README flowchart, "causal
+ * depthwise conv + SiLU", one token at a time).  u and h are [batch, d_inner]
+ * in `dtype`; conv_w [d_inner, 4] and conv_b [d_inner] (NULL: no bias) fp32;
+ * conv_state [batch, d_inner, 3] fp32 holds the previous three inputs of each
+ * channel, oldest first (zeros at the start of a sequence, matching the
+ * forward's left zero padding), and is updated in place to end with u.
+ *   h = SiLU(conv_b + w[0] s[0] + w[1] s[1] + w[2] s[2] + w[3] u).
+ * Uses no workspace.  Errors: INVALID_ARG for null or misaligned pointers or
+ * bad sizes, UNSUPPORTED for another dtype, CUDA for launch errors. */
+naju_status naju_conv_silu_step(int64_t batch, int64_t d_inner, int32_t dtype, const void* u,
+                                const float* conv_w, const float* conv_b, float* conv_state,
+                                void* h, void* stream);
+
+/* naju_conv_silu_step fused into naju_scan_step: one decode token of the
+ * whole path from the pre-conv input u [batch, d_inner] (same layouts and
+ * in-place updates of conv_state and state as the two calls; no h round trip
+ * through memory).  Uses no workspace. */
+naju_status naju_scan_step_conv(int64_t batch, int64_t d_inner, int64_t d_state, int32_t dtype,
+                                const void* u, const float* conv_w, const float* conv_b,
+                                float* conv_state, const void* a, const void* b, const void* B,
+                                const void* C, const void* z, const float* D, float* state,
+                                void* y, void* stream);
+
 /* Synchronises `stream`, reads the workspace's status word (NAJU_OK or
  * NAJU_ERR_TIMEOUT) and clears it.  Returns NAJU_ERR_CUDA if the stream
  * itself reports an error. */

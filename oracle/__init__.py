@@ -52,7 +52,9 @@ def _load():
             lib.naju_oracle_scan_fwd.argtypes = [i64] * 4 + [dp] * 11
             lib.naju_oracle_scan_bwd.argtypes = [i64] * 4 + [dp] * 18
             lib.naju_oracle_scan_step.argtypes = [i64] * 3 + [dp] * 9
-            for f in ("conv_silu_fwd", "conv_silu_bwd", "scan_fwd", "scan_bwd", "scan_step"):
+            lib.naju_oracle_conv_silu_step.argtypes = [i64] * 3 + [dp] * 5
+            for f in ("conv_silu_fwd", "conv_silu_bwd", "scan_fwd", "scan_bwd", "scan_step",
+                      "conv_silu_step"):
                 getattr(lib, "naju_oracle_" + f).restype = None
             _lib = lib
     return _lib
@@ -84,6 +86,27 @@ def conv_silu_fwd(u, w, bias=None, return_p: bool = False):
     p = np.empty_like(u) if return_p else None
     _load().naju_oracle_conv_silu_fwd(Bt, L, d, W, _p(u), _p(w), _p(bias), _p(p), _p(h))
     return (h, p) if return_p else h
+
+
+def conv_silu_step(conv_state, u, w, bias=None):
+    """One decode token of conv + SiLU.  conv_state [Bt,d,W-1] (previous
+    inputs, oldest first), u [Bt,d].  Returns (h, new_conv_state); the input
+    state is not modified."""
+    cs = _d(conv_state).copy()
+    u, w, bias = _d(u), _d(w), _d(bias)
+    Bt, d = u.shape
+    W = w.shape[1]
+    h = np.empty_like(u)
+    _load().naju_oracle_conv_silu_step(Bt, d, W, _p(u), _p(w), _p(bias), _p(cs), _p(h))
+    return h, cs
+
+
+def block_step(state, conv_state, u, conv_w, conv_b, a, b, B, C, z=None, D=None):
+    """One decode token of the fused path: conv + SiLU step, then the scan
+    step.  Returns (out, new_state, new_conv_state)."""
+    h, cs = conv_silu_step(conv_state, u, conv_w, conv_b)
+    out, st = scan_step(state, h, a, b, B, C, z, D)
+    return out, st, cs
 
 
 def conv_silu_bwd(u, w, bias, dh):

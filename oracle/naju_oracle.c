@@ -78,6 +78,25 @@ void naju_oracle_conv_silu_fwd(int64_t Bt, int64_t L, int64_t d, int64_t W,
             }
 }
 
+/* One decode token of the conv + SiLU above (README flowchart, "causal
+ * depthwise conv + SiLU"): cs [Bt][d][W-1] holds the previous W-1 inputs of
+ * each channel, oldest first; h = SiLU(bias + sum_{k<W-1} w[k] cs[k] +
+ * w[W-1] u), then cs shifts by one and ends with u. */
+void naju_oracle_conv_silu_step(int64_t Bt, int64_t d, int64_t W, const double* u,
+                                const double* w, const double* bias, double* cs, double* h) {
+    for (int64_t bb = 0; bb < Bt; ++bb)
+        for (int64_t c = 0; c < d; ++c) {
+            const int64_t e = bb * d + c;
+            double* s = cs + e * (W - 1);
+            double p = bias ? bias[c] : 0.0;
+            for (int64_t k = 0; k < W - 1; ++k) p += w[c * W + k] * s[k];
+            p += w[c * W + W - 1] * u[e];
+            h[e] = silu(p);
+            for (int64_t k = 0; k + 1 < W - 1; ++k) s[k] = s[k + 1];
+            s[W - 2] = u[e];
+        }
+}
+
 /* Gradient of the conv + SiLU above, given dL/dh.  dw, dbias are
  * accumulated over batch and time (overwritten, not added to). */
 void naju_oracle_conv_silu_bwd(int64_t Bt, int64_t L, int64_t d, int64_t W,

@@ -59,6 +59,11 @@ def test_rejects_bad_arguments_on_host(L):
     assert L.naju_scan_step(1, 8, 24, 0, *([null] * 10)) == 2
     assert L.naju_scan_step(1, 8, 16, 0, *([null] * 10)) == 1
     assert L.naju_last_device_status(None, None) == 1
+    # conv decode steps: null pointers / bad d_state
+    assert L.naju_conv_silu_step(1, 8, 0, *([null] * 6)) == 1
+    assert L.naju_conv_silu_step(1, 8, 7, *([null] * 6)) == 2
+    assert L.naju_scan_step_conv(1, 8, 24, 0, *([null] * 13)) == 2
+    assert L.naju_scan_step_conv(1, 8, 16, 0, *([null] * 13)) == 1
 
 
 def test_status_strings(L):

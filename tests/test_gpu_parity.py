@@ -454,3 +454,64 @@ def test_backward_wait_timeout_is_reported():
     g = run_bwd(t, True)
     r = oracle_bwd(t, True)
     compare_grads(g, r, True, TOL_F32)
+
+# ------------------------------------------------- decode step with conv state
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_conv_step_parity(dtype):
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    gen = torch.Generator().manual_seed(11)
+    Bt, d = 6, 203
+    u = torch.randn(Bt, d, generator=gen).to(tdt)
+    w = torch.randn(d, 4, generator=gen) * 0.5
+    bias = torch.randn(d, generator=gen)
+    cs = torch.randn(Bt, d, 3, generator=gen)
+    rh, rcs = oracle.conv_silu_step(cs, u, w, bias)
+    gcs = gpu(cs)
+    h = naju.conv_silu_step(gcs, gpu(u), gpu(w), gpu(bias))
+    torch.cuda.synchronize()
+    assert_close(h, rh, tol_of(dtype), bf16_out=(dtype == "bf16"), name="h")
+    assert_close(gcs, rcs, 0.0, name="conv_state")
+
+
+@pytest.mark.parametrize("N", [16, 64, 128])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_step_conv_parity(N, dtype):
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    gen = torch.Generator().manual_seed(100 + N)
+    Bt, d = 5, 77
+    state = torch.randn(Bt, d, N, generator=gen)
+    cs = torch.randn(Bt, d, 3, generator=gen)
+    u, a, b, z = (torch.randn(Bt, d, generator=gen).to(tdt) for _ in range(4))
+    a = (a.float() + 4).to(tdt)
+    B, C = (torch.randn(Bt, N, generator=gen).to(tdt) for _ in range(2))
+    D = torch.randn(d, generator=gen)
+    w = torch.randn(d, 4, generator=gen) * 0.5
+    bias = torch.randn(d, generator=gen)
+    ro, rs, rcs = oracle.block_step(state, cs, u, w, bias, a, b, B, C, z, D)
+    st, gcs = gpu(state), gpu(cs)
+    y = naju.scan_step_conv(st, gcs, gpu(u), gpu(a), gpu(b), gpu(B), gpu(C), gpu(w), gpu(bias),
+                            gpu(z), gpu(D))
+    torch.cuda.synchronize()
+    tol = tol_of(dtype)
+    assert_close(y, ro, tol, bf16_out=(dtype == "bf16"), name="y")
+    assert_close(st, rs, tol, name="state")
+    assert_close(gcs, rcs, 0.0, name="conv_state")
+
+
+def test_conv_steps_equal_fused_forward():
+    """L fused decode steps from zero conv state and x0 reproduce the fused
+    forward's outputs and final state (f32)."""
+    w = wl(64, "f32", Bt=2, L=40, d=48)
+    t = inputs(w, True, use_x0=True)
+    ro, rx, _ = oracle.block_fwd(t["u"], t["conv_w"], t["conv_b"], t["a"], t["b"], t["B"],
+                                 t["C"], t["z"], t["D"], t["x0"])
+    st = gpu(t["x0"])
+    cs = torch.zeros(2, 48, 3, device=DEV)
+    for n in range(40):
+        yn = naju.scan_step_conv(st, cs, gpu(t["u"][:, n]), gpu(t["a"][:, n]),
+                                 gpu(t["b"][:, n]), gpu(t["B"][:, n]), gpu(t["C"][:, n]),
+                                 gpu(t["conv_w"]), gpu(t["conv_b"]), gpu(t["z"][:, n]),
+                                 gpu(t["D"]))
+        assert_close(yn, ro[:, n], TOL_F32, name=f"y[{n}]")
+    torch.cuda.synchronize()
+    assert_close(st, rx, TOL_F32, name="state")

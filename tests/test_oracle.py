@@ -194,6 +194,23 @@ def test_conv_matches_torch_conv1d():
     np.testing.assert_allclose(h, torch.nn.functional.silu(pt).numpy(), rtol=1e-13, atol=1e-13)
 
 
+def test_conv_steps_match_torch_conv1d():
+    """L decode steps of the conv from a zero conv state = torch conv1d over the
+    sequence (the state holds the previous W-1 inputs, oldest first)."""
+    r = np.random.default_rng(41)
+    Bt, L, d, W = 2, 13, 5, 4
+    u, w, bias = r.normal(size=(Bt, L, d)), r.normal(size=(d, W)), r.normal(size=(d,))
+    ut = torch.tensor(u).transpose(1, 2)
+    pt = torch.nn.functional.conv1d(ut, torch.tensor(w)[:, None, :], torch.tensor(bias),
+                                    padding=W - 1, groups=d)[..., :L].transpose(1, 2)
+    ref = torch.nn.functional.silu(pt).numpy()
+    cs = np.zeros((Bt, d, W - 1))
+    for t in range(L):
+        h, cs = oracle.conv_silu_step(cs, u[:, t], w, bias)
+        np.testing.assert_allclose(h, ref[:, t], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(cs, u[:, L - (W - 1):].transpose(0, 2, 1), rtol=0, atol=0)
+
+
 # ------------------------------------------------------ finite differences
 def _loss_scan(t, dout, dxL):
     out, xL = oracle.scan_fwd(t["h"], t["a"], t["b"], t["B"], t["C"], t["z"], t["D"], t["x0"])

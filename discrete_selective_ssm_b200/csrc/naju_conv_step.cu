@@ -142,6 +142,13 @@ cudaError_t launch_conv_bwd(int64_t Bt, int64_t L, int64_t d, const void* u, con
 // h = SiLU(bias + w0 s0 + w1 s1 + w2 s2 + w3 u) from the conv state
 // s = (s0, s1, s2) (the previous three inputs, oldest first), which then
 // becomes (s1, s2, u).
+//
+// A warp owns 32 consecutive channels.  Lane l first computes the gates of
+// channel l once (coalesced per-channel loads); then the warp streams the 32
+// state rows, Q = N/4 lanes per row (one float4 each), so every load and
+// store instruction covers 128/N whole contiguous rows; the gate values
+// reach the row lanes by shuffles, the readout is a shuffle reduction over
+// the row's lanes, and y returns to lane l for one coalesced store.
 template <typename T, int N, bool CONV>
 __global__ void __launch_bounds__(256)
 step_kernel(int64_t d, const T* __restrict__ h, const T* __restrict__ a,
@@ -149,66 +156,83 @@ step_kernel(int64_t d, const T* __restrict__ h, const T* __restrict__ a,
             const T* __restrict__ z, const float* __restrict__ D, float* __restrict__ state,
             T* __restrict__ y, float scale, const float* __restrict__ conv_w,
             const float* __restrict__ conv_b, float* __restrict__ conv_state) {
-    constexpr int S = N / 4;
-    constexpr int P = 256 / S;
-    __shared__ float4 sB[N / 4], sC[N / 4];
+    constexpr int Q = N / 4;        // lanes per state row
+    constexpr int CPI = 32 / Q;     // rows per warp instruction
+    constexpr int ITER = 32 / CPI;  // instructions per 32 rows (= Q)
+    constexpr int BATCH = ITER < 8 ? ITER : 8;  // loads in flight per lane
     const int64_t bb = blockIdx.y;
-    const int tid = threadIdx.x;
-    if (tid < N / 4) {
-        float v[4], w4[4];
+    const int lane = threadIdx.x & 31;
+    const int64_t cw0 = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * 32;  // warp's first channel
+    if (cw0 >= d) return;
+    // ---- gates of channel cw0 + lane
+    const int64_t cg = cw0 + lane;
+    const bool gvalid = cg < d;
+    const int64_t eg = bb * d + cg;
+    float f = 0.f, v = 0.f, dh = 0.f, gz = 1.f;
+    if (gvalid) {
+        float hh = to_f(h[eg]);
+        if (CONV) {
+            const float s0 = conv_state[eg * 3], s1 = conv_state[eg * 3 + 1],
+                        s2 = conv_state[eg * 3 + 2];
+            const float p = (conv_b ? conv_b[cg] : 0.f) + conv_w[cg * 4] * s0 +
+                            conv_w[cg * 4 + 1] * s1 + conv_w[cg * 4 + 2] * s2 +
+                            conv_w[cg * 4 + 3] * hh;
+            conv_state[eg * 3] = s1;
+            conv_state[eg * 3 + 1] = s2;
+            conv_state[eg * 3 + 2] = hh;
+            hh = siluf_(p);
+        }
+        f = sigmoidf_(to_f(a[eg]));
+        v = sigmoidf_(to_f(b[eg])) * hh;
+        dh = D ? D[cg] * hh : 0.f;
+        if (z) gz = siluf_(to_f(z[eg]));
+    }
+    // ---- B, C slice of this lane's float4 position
+    const int q = lane % Q, grp = lane / Q;
+    float4 Bv, Cv;
+    {
+        float t4[4], u4[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            v[r] = to_f(B[bb * N + tid * 4 + r]);
-            w4[r] = to_f(C[bb * N + tid * 4 + r]);
+            t4[r] = to_f(B[bb * N + q * 4 + r]);
+            u4[r] = to_f(C[bb * N + q * 4 + r]);
         }
-        sB[tid] = make_float4(v[0], v[1], v[2], v[3]);
-        sC[tid] = make_float4(w4[0], w4[1], w4[2], w4[3]);
+        Bv = make_float4(t4[0], t4[1], t4[2], t4[3]);
+        Cv = make_float4(u4[0], u4[1], u4[2], u4[3]);
     }
-    __syncthreads();
-    const int js = tid % S;
-    const int64_t c = (int64_t)blockIdx.x * P + tid / S;
-    const bool valid = c < d;
-    const int64_t e = bb * d + c;
-    float f = 0.f, v = 0.f, hv = 0.f;
-    if (valid) {
-        if (CONV) {
-            const float u = to_f(h[e]);
-            const float s0 = conv_state[e * 3], s1 = conv_state[e * 3 + 1],
-                        s2 = conv_state[e * 3 + 2];
-            const float p = (conv_b ? conv_b[c] : 0.f) + conv_w[c * 4] * s0 +
-                            conv_w[c * 4 + 1] * s1 + conv_w[c * 4 + 2] * s2 +
-                            conv_w[c * 4 + 3] * u;
-            hv = siluf_(p);
-            __syncwarp(__activemask());
-            if (js == 0) {
-                conv_state[e * 3] = s1;
-                conv_state[e * 3 + 1] = s2;
-                conv_state[e * 3 + 2] = u;
-            }
-        } else {
-            hv = to_f(h[e]);
-        }
-        f = sigmoidf_(to_f(a[e]));
-        v = sigmoidf_(to_f(b[e])) * hv;
-    }
-    float4* st4 = reinterpret_cast<float4*>(state + e * N) + js;
-    float4 x = valid ? *st4 : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 bv = sB[js], cv = sC[js];
-    x.x = fmaf(f, x.x, v * bv.x);
-    x.y = fmaf(f, x.y, v * bv.y);
-    x.z = fmaf(f, x.z, v * bv.z);
-    x.w = fmaf(f, x.w, v * bv.w);
-    float part = (x.x * cv.x + x.y * cv.y) + (x.z * cv.z + x.w * cv.w);
+    // ---- stream the 32 rows
+    float yl = 0.f;  // y of channel cw0 + lane, gathered below
 #pragma unroll
-    for (int o = 1; o < S; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (valid) {
-        *st4 = x;
-        if (js == 0) {
-            float yv = part * scale + (D ? D[c] * hv : 0.f);
-            if (z) yv *= siluf_(to_f(z[e]));
-            y[e] = from_f<T>(yv);
+    for (int r0 = 0; r0 < ITER; r0 += BATCH) {
+        float4 x[BATCH];
+#pragma unroll
+        for (int k = 0; k < BATCH; ++k) {
+            const int64_t c = cw0 + (int64_t)(r0 + k) * CPI + grp;
+            x[k] = c < d ? reinterpret_cast<const float4*>(state + (bb * d + c) * N)[q]
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < BATCH; ++k) {
+            const int r = r0 + k;
+            const int src = r * CPI + grp;  // lane holding this row's gates
+            const int64_t c = cw0 + src;
+            const float fr = __shfl_sync(0xffffffffu, f, src);
+            const float vr = __shfl_sync(0xffffffffu, v, src);
+            float4 xk = x[k];
+            xk.x = fmaf(fr, xk.x, vr * Bv.x);
+            xk.y = fmaf(fr, xk.y, vr * Bv.y);
+            xk.z = fmaf(fr, xk.z, vr * Bv.z);
+            xk.w = fmaf(fr, xk.w, vr * Bv.w);
+            if (c < d) reinterpret_cast<float4*>(state + (bb * d + c) * N)[q] = xk;
+            float part = (xk.x * Cv.x + xk.y * Cv.y) + (xk.z * Cv.z + xk.w * Cv.w);
+#pragma unroll
+            for (int o = 1; o < Q; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            // lanes r*CPI .. r*CPI + CPI - 1 collect the sums of rows r*CPI + g
+            const float got = __shfl_sync(0xffffffffu, part, (lane - r * CPI) * Q & 31);
+            if (lane >= r * CPI && lane < r * CPI + CPI) yl = got;
         }
     }
+    if (gvalid) y[eg] = from_f<T>(fmaf(yl, scale, dh) * gz);
 }
 
 template <typename T, bool CONV>
@@ -217,8 +241,7 @@ static cudaError_t step_t(int64_t Bt, int64_t d, int64_t N, const void* h, const
                           const float* D, float* state, void* y, const float* conv_w,
                           const float* conv_b, float* conv_state, cudaStream_t st) {
     const float scale = 1.0f / sqrtf((float)N);
-    const int P = 256 / (int)(N / 4);
-    dim3 grid((unsigned)((d + P - 1) / P), (unsigned)Bt);
+    dim3 grid((unsigned)((d + 255) / 256), (unsigned)Bt);  // 8 warps x 32 channels
 #define NAJU_STEP(NN)                                                                     \
     step_kernel<T, NN, CONV><<<grid, 256, 0, st>>>(                                      \
         d, static_cast<const T*>(h), static_cast<const T*>(a), static_cast<const T*>(b), \

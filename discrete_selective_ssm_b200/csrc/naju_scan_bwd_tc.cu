@@ -448,55 +448,47 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         tc::tmem_st_wait();
         __syncthreads();  // brow, crow, y1, w1 complete
         if (!slow) {
-            // K-major per-token tiles.
-            for (int e = tid; e < T * N / 4; e += NT) {
-                const int rest = e >> 3;
-                const int tt = (rest & 1) * 8 + (e & 7), j = (rest >> 1) * 4;
-                // ta: rows t, K = d_state (C forward, B backward)
-                *reinterpret_cast<float4*>(&sm.ta[tc::kmajor_offset(tt, j, N) >> 2]) =
-                    fwd ? *reinterpret_cast<const float4*>(&sm.crow[tt][j])
-                        : *reinterpret_cast<const float4*>(&sm.brow[tt][j]);
-                // ts: rows d_state, K = 16 (B^T forward, C^T backward)
-                const int jj = e % N, m0 = (e / N) * 4;
-                const float(*src)[N + 4] = fwd ? sm.brow : sm.crow;
-                *reinterpret_cast<float4*>(&sm.ts[tc::kmajor_offset(jj, m0, T) >> 2]) =
-                    make_float4(src[m0][jj], src[m0 + 1][jj], src[m0 + 2][jj], src[m0 + 3][jj]);
-            }
-            if (sweep != kSweepEarly) {
-                // tg: forward G[t][m] = C_t . B_m (m <= t); backward G^T[t][t'] = C_t' . B_t
-                // (t' >= t).  ta2: A_C[t][m] = sum_ch Y_t W_m (m <= t) or
-                // A_B[t][t'] = sum_ch P_t U_t' (t' >= t).  One entry per pair of
-                // adjacent threads, each taking half of the sum.
-                const int e = tid >> 1, part = tid & 1;
-                const int tt = e / T, mm = e % T;
-                const bool live = fwd ? (mm <= tt) : (mm >= tt);
-                float2 acc = make_float2(0.f, 0.f), acc2 = make_float2(0.f, 0.f);
-                if (live) {
-                    const float* cr = (fwd ? sm.crow[tt] : sm.crow[mm]) + part * (N / 2);
-                    const float* br = (fwd ? sm.brow[mm] : sm.brow[tt]) + part * (N / 2);
-#pragma unroll 4
-                    for (int j = 0; j < N / 2; j += 4) {
-                        const float4 cv = *reinterpret_cast<const float4*>(cr + j);
-                        const float4 bv = *reinterpret_cast<const float4*>(br + j);
-                        acc = __ffma2_rn(make_float2(cv.x, cv.y), make_float2(bv.x, bv.y), acc);
-                        acc = __ffma2_rn(make_float2(cv.z, cv.w), make_float2(bv.z, bv.w), acc);
-                    }
-                    const float* yr = &sm.y1[tt][part * (P / 2)];
-                    const float* wr = &sm.w1[mm][part * (P / 2)];
-#pragma unroll 4
-                    for (int q = 0; q < P / 2; q += 4) {
-                        const float4 yv = *reinterpret_cast<const float4*>(yr + q);
-                        const float4 wv = *reinterpret_cast<const float4*>(wr + q);
-                        acc2 = __ffma2_rn(make_float2(yv.x, yv.y), make_float2(wv.x, wv.y), acc2);
-                        acc2 = __ffma2_rn(make_float2(yv.z, yv.w), make_float2(wv.z, wv.w), acc2);
-                    }
+            if (sweep != kSweepEarly && warp < 2) {
+                // Warp 0: A_C[t][m] = sum_ch Y_t W_m (m <= t) or A_B[t][t'] =
+                // sum_ch P_t U_t' (t' >= t) -> ta2.  Warp 1: the Gram, forward
+                // G[t][m] = C_t . B_m (m <= t), backward G^T[t][t'] = C_t' . B_t
+                // (t' >= t) -> tg.  Warp-level tf32 MMAs.
+                float dd[2][4];
+                float* dst;
+                if (warp == 0) {
+                    tc::warp_gram16<P, P + 4>(&sm.y1[0][0], &sm.w1[0][0], dd);
+                    dst = sm.ta2;
+                } else {
+                    tc::warp_gram16<N, N + 4>(fwd ? &sm.crow[0][0] : &sm.brow[0][0],
+                                              fwd ? &sm.brow[0][0] : &sm.crow[0][0], dd);
+                    dst = sm.tg;
                 }
-                float gsum = acc.x + acc.y, asum = acc2.x + acc2.y;
-                gsum += __shfl_xor_sync(0xffffffffu, gsum, 1);
-                asum += __shfl_xor_sync(0xffffffffu, asum, 1);
-                if (part == 0) {
-                    sm.tg[tc::kmajor_offset(tt, mm, T) >> 2] = gsum;
-                    sm.ta2[tc::kmajor_offset(tt, mm, T) >> 2] = asum;
+                const int lane = tid & 31, gq = lane >> 2, kq = lane & 3;
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int row = gq + (r >> 1) * 8, col = 8 * n + 2 * kq + (r & 1);
+                        const bool live = fwd ? (col <= row) : (col >= row);
+                        dst[tc::kmajor_offset(row, col, T) >> 2] = live ? dd[n][r] : 0.f;
+                    }
+            } else {
+                // K-major per-token tiles (the other warps).
+                const int t2 = sweep != kSweepEarly ? tid - 64 : tid;
+                const int n2 = sweep != kSweepEarly ? NT - 64 : NT;
+                for (int e = t2; e < T * N / 4; e += n2) {
+                    const int rest = e >> 3;
+                    const int tt = (rest & 1) * 8 + (e & 7), j = (rest >> 1) * 4;
+                    // ta: rows t, K = d_state (C forward, B backward)
+                    *reinterpret_cast<float4*>(&sm.ta[tc::kmajor_offset(tt, j, N) >> 2]) =
+                        fwd ? *reinterpret_cast<const float4*>(&sm.crow[tt][j])
+                            : *reinterpret_cast<const float4*>(&sm.brow[tt][j]);
+                    // ts: rows d_state, K = 16 (B^T forward, C^T backward)
+                    const int jj = e % N, m0 = (e / N) * 4;
+                    const float(*src)[N + 4] = fwd ? sm.brow : sm.crow;
+                    *reinterpret_cast<float4*>(&sm.ts[tc::kmajor_offset(jj, m0, T) >> 2]) =
+                        make_float4(src[m0][jj], src[m0 + 1][jj], src[m0 + 2][jj],
+                                    src[m0 + 3][jj]);
                 }
             }
         }

@@ -190,6 +190,43 @@ __device__ __forceinline__ void mma_commit(uint64_t* mbar) {
         : "memory");
 }
 
+// --------------------------------------------------- warp-level products
+// D[16 x 8] += A[16 x 8] * B[8 x 8] (tf32 operands as fp32 bits, fp32
+// accumulate), one warp.  Fragments (g = lane / 4, k = lane % 4):
+// a = {A[g][k], A[g+8][k], A[g][k+4], A[g+8][k+4]}, b = {B[k][g], B[k+4][g]},
+// d = {D[g][2k], D[g][2k+1], D[g+8][2k], D[g+8][2k+1]}.
+__device__ __forceinline__ void mma_16x8x8_tf32(float* d, const float* a, const float* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(__float_as_uint(a[0])), "r"(__float_as_uint(a[1])), "r"(__float_as_uint(a[2])),
+          "r"(__float_as_uint(a[3])), "r"(__float_as_uint(b[0])), "r"(__float_as_uint(b[1])));
+}
+
+// One warp: D[t][m] = sum_k X[t][k] Y[m][k] for t, m < 16, with X and Y
+// row-major in shared memory (row stride LD floats, LD % 32 == 4 keeps the
+// fragment loads conflict-free).  Lane (g, k) ends with
+// d[n][0..3] = D[g][8n+2k], D[g][8n+2k+1], D[g+8][8n+2k], D[g+8][8n+2k+1].
+template <int K, int LD>
+__device__ __forceinline__ void warp_gram16(const float* X, const float* Y, float (&d)[2][4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, k = lane & 3;
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) d[n][r] = 0.f;
+#pragma unroll 4
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const float a[4] = {X[g * LD + k0 + k], X[(g + 8) * LD + k0 + k], X[g * LD + k0 + k + 4],
+                            X[(g + 8) * LD + k0 + k + 4]};
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+            const float b[2] = {Y[(8 * n + g) * LD + k0 + k], Y[(8 * n + g) * LD + k0 + k + 4]};
+            mma_16x8x8_tf32(d[n], a, b);
+        }
+    }
+}
+
 // -------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* mbar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(mbar)), "r"(count)

@@ -254,34 +254,35 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
         const float Q0 = sm.xq0[pch], E0 = sm.xe0[pch], E1 = sm.xe1[pch];
         const bool slow = tc::named_bar_or(1, NPROD, phalf == 1 && !(Q0 * Qh <= kTcBound));
         if (!slow) {
-            // K-major operand tiles.  bc: a quarter warp fills one 8-row core
-            // matrix; bs: one thread gathers 4 consecutive m of one row j.
-            for (int e = tid; e < T * N / 4; e += NPROD) {
-                if (full) {
-                    const int rest = e >> 3;
-                    const int tt = (rest & 1) * 8 + (e & 7), j = (rest >> 1) * 4;
-                    *reinterpret_cast<float4*>(&stg.bc[tc::kmajor_offset(tt, j, N) >> 2]) =
-                        *reinterpret_cast<const float4*>(&stg.crow[tt][j]);
-                }
-                const int jj = e % N, m0 = (e / N) * 4;
-                *reinterpret_cast<float4*>(&stg.bs[tc::kmajor_offset(jj, m0, T) >> 2]) =
-                    make_float4(stg.brow[m0][jj], stg.brow[m0 + 1][jj], stg.brow[m0 + 2][jj],
-                                stg.brow[m0 + 3][jj]);
-            }
-            if (full) {
-                // G[t][m] = C_t . B_m for m <= t (one entry per producer thread).
-                const int tt = tid / T, mm = tid % T;
-                float2 acc = make_float2(0.f, 0.f);
-                if (mm <= tt) {
-#pragma unroll 4
-                    for (int j = 0; j < N; j += 4) {
-                        const float4 cv = *reinterpret_cast<const float4*>(&stg.crow[tt][j]);
-                        const float4 bv = *reinterpret_cast<const float4*>(&stg.brow[mm][j]);
-                        acc = __ffma2_rn(make_float2(cv.x, cv.y), make_float2(bv.x, bv.y), acc);
-                        acc = __ffma2_rn(make_float2(cv.z, cv.w), make_float2(bv.z, bv.w), acc);
+            if (full && warp == 0) {
+                // G[t][m] = C_t . B_m for m <= t: one warp, tf32 warp-level MMAs.
+                float dd[2][4];
+                tc::warp_gram16<N, N + 4>(&stg.crow[0][0], &stg.brow[0][0], dd);
+                const int lane = tid & 31, gq = lane >> 2, kq = lane & 3;
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int row = gq + (r >> 1) * 8, col = 8 * n + 2 * kq + (r & 1);
+                        stg.bg[tc::kmajor_offset(row, col, T) >> 2] = col <= row ? dd[n][r] : 0.f;
                     }
+            } else {
+                // K-major operand tiles (the other warps).  bc: a quarter warp
+                // fills one 8-row core matrix; bs: one thread gathers 4
+                // consecutive m of one row j.
+                const int t2 = full ? tid - 32 : tid, n2 = full ? NPROD - 32 : NPROD;
+                for (int e = t2; e < T * N / 4; e += n2) {
+                    if (full) {
+                        const int rest = e >> 3;
+                        const int tt = (rest & 1) * 8 + (e & 7), j = (rest >> 1) * 4;
+                        *reinterpret_cast<float4*>(&stg.bc[tc::kmajor_offset(tt, j, N) >> 2]) =
+                            *reinterpret_cast<const float4*>(&stg.crow[tt][j]);
+                    }
+                    const int jj = e % N, m0 = (e / N) * 4;
+                    *reinterpret_cast<float4*>(&stg.bs[tc::kmajor_offset(jj, m0, T) >> 2]) =
+                        make_float4(stg.brow[m0][jj], stg.brow[m0 + 1][jj], stg.brow[m0 + 2][jj],
+                                    stg.brow[m0 + 3][jj]);
                 }
-                stg.bg[tc::kmajor_offset(tt, mm, T) >> 2] = acc.x + acc.y;
             }
         }
         const float Elast = E0 * E1;

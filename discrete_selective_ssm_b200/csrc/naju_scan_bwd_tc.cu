@@ -102,7 +102,10 @@ struct BwdTcSmem {
     };
     alignas(1024) float st[ST_FLOATS];
     alignas(1024) float pk[T * P];     // Y or P, swizzled, rows t, K = channels
-    Raw raw[2];
+    // Raw-input buffers: TMA runs NRAW - 1 sub-chunks ahead.  (A third buffer
+    // for d_state 64 measured no faster.)
+    static constexpr int NRAW = 2;
+    Raw raw[NRAW];
     alignas(128) float ta[T * N];      // C (forward) / B (backward) rows t, K = d_state
     alignas(128) float ts[TS_FLOATS];  // B^T (forward) / C^T (backward): rows d_state, K = 16
     alignas(128) float tg[T * T];      // G[t][m] (forward) / G^T (backward)
@@ -114,7 +117,7 @@ struct BwdTcSmem {
     float dp[T + 3][P];
     float acc[T][N];                   // slow path channel sums
     float xq[4][P], xe[4][P], xs[4][P];  // exchanges between a channel's four threads
-    uint64_t loaded[2], mma;
+    uint64_t loaded[3], mma;
     uint32_t taddr;
     int item, ok;
 };
@@ -149,8 +152,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     }
     if (tid == 0) {
         sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
-        tc::mbar_init(&sm.loaded[0], 1);
-        tc::mbar_init(&sm.loaded[1], 1);
+        for (int q = 0; q < Sm::NRAW; ++q) tc::mbar_init(&sm.loaded[q], 1);
         tc::mbar_init(&sm.mma, 1);
         tma::prefetch_map(&tm.u);
         tma::prefetch_map(&tm.a);
@@ -223,7 +225,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         return (int64_t)k * K + (int64_t)sb * T;
     };
     auto issue = [&](int li) {  // one thread
-        const int buf = li & 1;
+        const int buf = li % Sm::NRAW;
         typename Sm::Raw& r = sm.raw[buf];
         uint64_t* mb = &sm.loaded[buf];
         const uint32_t bytes =
@@ -240,7 +242,8 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     };
     int li = 0;            // current item
     uint32_t mma_phase = 0;
-    if (tid == 0 && nitems > 0) issue(0);
+    if (tid == 0)
+        for (int q = 0; q < Sm::NRAW - 1 && q < nitems; ++q) issue(q);
 
     auto bf4 = [](const __nv_bfloat16* src) {
         const uint2 raw = *reinterpret_cast<const uint2*>(src);
@@ -343,11 +346,11 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     bool slow = false;
     int nvh = 0;  // valid tokens of this thread's quarter
 
-    // Unpack item `li` (raw buffer li & 1) for a sweep; fills the registers
+    // Unpack item `li` (raw buffer li % NRAW) for a sweep; fills the registers
     // above, the TMEM operand columns and the per-token tiles.  Returns after
     // a block-wide barrier.
     auto prep = [&](int64_t t0, int64_t te, int sweep) {
-        const typename Sm::Raw& r = sm.raw[li & 1];
+        const typename Sm::Raw& r = sm.raw[li % Sm::NRAW];
         const bool fwd = sweep == kSweepFwd;
         // B and C rows to fp32.
         for (int e = tid; e < T * N / 4; e += NT) {
@@ -503,43 +506,47 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         const uint32_t a_ta = tc::smem_u32(sm.ta), a_ts = tc::smem_u32(sm.ts);
         const uint32_t a_tg = tc::smem_u32(sm.tg), a_t2 = tc::smem_u32(sm.ta2);
         const uint32_t a_st = tc::smem_u32(sm.st), a_pk = tc::smem_u32(sm.pk);
-        if (sweep != kSweepEarly) {
-            // readout (forward: X . C + W G) or dv (backward: H . B + U G^T)
-            const uint32_t Acol = sweep == kSweepFwd ? Cols::X : Cols::G;
+        // Three independent accumulation chains, issued interleaved so the
+        // tensor core can overlap them: readout (forward: X . C + W G) or dv
+        // (backward: H . B + U G^T) into R; state (forward: V B^T) or adjoint
+        // (backward: (s dy E) C^T) into D; dC or dB ((state^T)(Y or P) over
+        // channels + (B^T or C^T)(A_C or A_B)) into BC.
+        const bool full = sweep != kSweepEarly;
+        const uint32_t Acol = sweep == kSweepFwd ? Cols::X : Cols::G;
+        constexpr int NR = N / 8 + T / 8, NBC = P / 8 + T / 8, ND = T / 8;
 #pragma unroll
-            for (int ks = 0; ks < N / 8; ++ks)
-                tc::mma_tf32_ts(tbase + Cols::R, tbase + Acol + ks * 8,
-                                tc::sdesc(a_ta + ks * 256, 128, 32 * N), id16, ks > 0 ? 1u : 0u);
-#pragma unroll
-            for (int ks = 0; ks < T / 8; ++ks)
-                tc::mma_tf32_ts(tbase + Cols::R, tbase + Cols::WU + ks * 8,
-                                tc::sdesc(a_tg + ks * 256, 128, 32 * T), id16, 1u);
-        }
-        // state (forward: V B^T) or adjoint (backward: (s dy E) C^T)
-#pragma unroll
-        for (int ks = 0; ks < T / 8; ++ks)
-            tc::mma_tf32_ts(tbase + Cols::D, tbase + Cols::VV + ks * 8,
-                            tc::sdesc(a_ts + ks * 256, 128, 32 * T), idN, ks > 0 ? 1u : 0u);
-        if (sweep != kSweepEarly) {
-            // dC or dB: (state^T)(Y or P) over channels + (B^T or C^T)(A_C or A_B)
-#pragma unroll
-            for (int ks = 0; ks < P / 8; ++ks)
-                tc::mma_tf32_ss(tbase + Cols::BC,
-                                tc::sdesc_sw128(a_st + (ks >> 2) * N * 128 + (ks & 3) * 32),
-                                tc::sdesc_sw128(a_pk + (ks >> 2) * T * 128 + (ks & 3) * 32), id16,
-                                ks > 0 ? 1u : 0u);
-#pragma unroll
-            for (int ks = 0; ks < T / 8; ++ks)
-                tc::mma_tf32_ss(tbase + Cols::BC, tc::sdesc(a_ts + ks * 256, 128, 32 * T),
-                                tc::sdesc(a_t2 + ks * 256, 128, 32 * T), id16, 1u);
+        for (int i = 0; i < NBC; ++i) {
+            if (full && i < NR) {
+                if (i < N / 8)
+                    tc::mma_tf32_ts(tbase + Cols::R, tbase + Acol + i * 8,
+                                    tc::sdesc(a_ta + i * 256, 128, 32 * N), id16, i > 0 ? 1u : 0u);
+                else
+                    tc::mma_tf32_ts(tbase + Cols::R, tbase + Cols::WU + (i - N / 8) * 8,
+                                    tc::sdesc(a_tg + (i - N / 8) * 256, 128, 32 * T), id16, 1u);
+            }
+            if (i < ND)
+                tc::mma_tf32_ts(tbase + Cols::D, tbase + Cols::VV + i * 8,
+                                tc::sdesc(a_ts + i * 256, 128, 32 * T), idN, i > 0 ? 1u : 0u);
+            if (full) {
+                if (i < P / 8)
+                    tc::mma_tf32_ss(tbase + Cols::BC,
+                                    tc::sdesc_sw128(a_st + (i >> 2) * N * 128 + (i & 3) * 32),
+                                    tc::sdesc_sw128(a_pk + (i >> 2) * T * 128 + (i & 3) * 32),
+                                    id16, i > 0 ? 1u : 0u);
+                else
+                    tc::mma_tf32_ss(tbase + Cols::BC,
+                                    tc::sdesc(a_ts + (i - P / 8) * 256, 128, 32 * T),
+                                    tc::sdesc(a_t2 + (i - P / 8) * 256, 128, 32 * T), id16, 1u);
+            }
         }
         tc::mma_commit(&sm.mma);
     };
 
     // Start item li: prefetch the next one, wait for this one's inputs.
     auto begin_item = [&]() {
-        if (tid == 0 && li + 1 < nitems) issue(li + 1);
-        if (!tc::mbar_wait(&sm.loaded[li & 1], (uint32_t)((li >> 1) & 1), kBSpin))
+        // Buffer (li + NRAW - 1) % NRAW was last read by item li - 1.
+        if (tid == 0 && li + Sm::NRAW - 1 < nitems) issue(li + Sm::NRAW - 1);
+        if (!tc::mbar_wait(&sm.loaded[li % Sm::NRAW], (uint32_t)((li / Sm::NRAW) & 1), kBSpin))
             timed_out = true;
     };
     auto run_mma = [&](int sweep) {
@@ -772,7 +779,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             }
             // dz and s dy (x.C) for the backward sweep
             {
-                const typename Sm::Raw& r = sm.raw[li & 1];
+                const typename Sm::Raw& r = sm.raw[li % Sm::NRAW];
                 float dl[TQ];
 #pragma unroll
                 for (int q = 0; q < TQ; ++q) {
@@ -820,7 +827,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 write_bc_smem(0, t0, te);
             }
             // per-(token, channel) gradients
-            const typename Sm::Raw& r = sm.raw[li & 1];
+            const typename Sm::Raw& r = sm.raw[li % Sm::NRAW];
             float dl[TQ];
             tc::tmem_ld4(trow + Cols::DL + sb * T + qd * TQ, dl);
             tc::tmem_ld_wait();

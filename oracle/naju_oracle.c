@@ -140,12 +140,19 @@ void naju_oracle_conv_silu_bwd(int64_t Bt, int64_t L, int64_t d, int64_t W,
     }
 }
 
+/* Write gate.  b == NULL selects the coupled single gate i = 1 - f
+ * (= sigma(-a)), the complementary gating analysed in the paper's abstract
+ * (|r| + w <= 1); otherwise i = sigma(b). */
+static double wgate(const double* a, const double* b, int64_t e) {
+    return b ? sigm(b[e]) : sigm(-a[e]);
+}
+
 /* Forward scan (README, Core equations):
  *   x_n = f_n (.) x_{n-1} + i_n (.) (h_n B_n^T),  f = sigma(a), i = sigma(b)
  *   y_n = x_n C_n / sqrt(N) + D (.) h_n
  *   out_n = y_n * SiLU(z_n)
  * y_pre (the readout before modulation) and xL (state after the last token)
- * are optional outputs. */
+ * are optional outputs.  b == NULL: coupled gate i = 1 - f. */
 void naju_oracle_scan_fwd(int64_t Bt, int64_t L, int64_t d, int64_t N,
                           const double* h, const double* a, const double* b,
                           const double* B, const double* C, const double* z,
@@ -160,7 +167,7 @@ void naju_oracle_scan_fwd(int64_t Bt, int64_t L, int64_t d, int64_t N,
             for (int64_t t = 0; t < L; ++t) {
                 const int64_t e = (bb * L + t) * d + c;
                 const double f = sigm(a[e]);
-                const double i = sigm(b[e]);
+                const double i = wgate(a, b, e);
                 const double* Bn = B + (bb * L + t) * N;
                 const double* Cn = C + (bb * L + t) * N;
                 double r = 0.0;
@@ -188,6 +195,8 @@ void naju_oracle_scan_fwd(int64_t Bt, int64_t L, int64_t d, int64_t N,
  *   df_n   = G_n . x_{n-1},    da_n = df_n f_n (1 - f_n)
  *   dB_n  += G_n i_n h_n,      dC_n += dy_n x_n / sqrt(N)   (summed over d)
  *   dD    += dy_n h_n,         dx0 = f_0 G_0
+ * Coupled gate (b == NULL, i = 1 - f): a reaches the loss through f and i,
+ *   da_n = (df_n - di_n) f_n (1 - f_n), and there is no db (db may be NULL).
  * All states x_n of a row are kept, so the reverse sweep reads them exactly.
  * dD is overwritten.  dz may be NULL only when z is NULL. */
 void naju_oracle_scan_bwd(int64_t Bt, int64_t L, int64_t d, int64_t N,
@@ -224,7 +233,7 @@ void naju_oracle_scan_bwd(int64_t Bt, int64_t L, int64_t d, int64_t N,
                 for (int64_t j = 0; j < N; ++j) xs[j] = x0 ? x0[(bb * d + c) * N + j] : 0.0;
                 for (int64_t t = 0; t < L; ++t) {
                     const int64_t e = (bb * L + t) * d + c;
-                    const double f = sigm(a[e]), i = sigm(b[e]);
+                    const double f = sigm(a[e]), i = wgate(a, b, e);
                     const double* Bn = B + (bb * L + t) * N;
                     for (int64_t j = 0; j < N; ++j)
                         xs[(t + 1) * N + j] = f * xs[t * N + j] + i * (h[e] * Bn[j]);
@@ -233,7 +242,7 @@ void naju_oracle_scan_bwd(int64_t Bt, int64_t L, int64_t d, int64_t N,
                 double dDc = 0.0;
                 for (int64_t t = L - 1; t >= 0; --t) {
                     const int64_t e = (bb * L + t) * d + c;
-                    const double f = sigm(a[e]), i = sigm(b[e]);
+                    const double f = sigm(a[e]), i = wgate(a, b, e);
                     const double* Bn = B + (bb * L + t) * N;
                     const double* Cn = C + (bb * L + t) * N;
                     const double* xt = xs + (t + 1) * N;
@@ -254,8 +263,14 @@ void naju_oracle_scan_bwd(int64_t Bt, int64_t L, int64_t d, int64_t N,
                         myC[t * N + j] += dy * scale * xt[j];
                     }
                     dh[e] = (D ? D[c] * dy : 0.0) + i * GB;
-                    db[e] = h[e] * GB * i * (1.0 - i);
-                    da[e] = Gx * f * (1.0 - f);
+                    const double di = h[e] * GB;
+                    if (b) {
+                        db[e] = di * i * (1.0 - i);
+                        da[e] = Gx * f * (1.0 - f);
+                    } else {
+                        if (db) db[e] = 0.0;
+                        da[e] = (Gx - di) * f * (1.0 - f);
+                    }
                     dDc += dy * h[e];
                     for (int64_t j = 0; j < N; ++j) G[j] *= f;
                 }
@@ -293,7 +308,7 @@ void naju_oracle_scan_step(int64_t Bt, int64_t d, int64_t N,
     for (int64_t bb = 0; bb < Bt; ++bb)
         for (int64_t c = 0; c < d; ++c) {
             const int64_t e = bb * d + c;
-            const double f = sigm(a[e]), i = sigm(b[e]);
+            const double f = sigm(a[e]), i = wgate(a, b, e);
             double* x = state + e * N;
             double r = 0.0;
             for (int64_t j = 0; j < N; ++j) {

@@ -281,3 +281,56 @@ def test_gradients_without_optional_inputs():
     assert g["dz"] is None and g["dD"] is None
     for key, gk in [("h", "dh"), ("a", "da"), ("b", "db"), ("B", "dB"), ("C", "dC")]:
         _fd_check(loss, t, key, g[gk])
+
+
+# ------------------------------------------- coupled single gate (i = 1 - f)
+def test_coupled_gate_equals_write_gate_minus_a():
+    """Coupled gate (b absent) = the two-gate scan with b = -a, since
+    1 - sigma(a) = sigma(-a)."""
+    t = tiny(80, Bt=2, L=7, d=3, N=4)
+    o1, x1 = oracle.scan_fwd(t["h"], t["a"], None, t["B"], t["C"], t["z"], t["D"], t["x0"])
+    o2, x2 = oracle.scan_fwd(t["h"], t["a"], -t["a"], t["B"], t["C"], t["z"], t["D"], t["x0"])
+    np.testing.assert_allclose(o1, o2, rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(x1, x2, rtol=1e-14, atol=1e-14)
+
+
+def test_coupled_gate_fixed_point_and_bound():
+    """With i = 1 - f the update is a convex combination: a state equal to
+    h B stays there for constant h and B, and |x_n| never exceeds
+    max(|x0|, max |h B|) (the abstract's |r| + w <= 1 bound)."""
+    r = np.random.default_rng(81)
+    Bt, L, d, N = 1, 30, 3, 4
+    hc, Bc = r.normal(size=(d,)), r.normal(size=(N,))
+    h = np.broadcast_to(hc, (Bt, L, d)).copy()
+    B = np.broadcast_to(Bc, (Bt, L, N)).copy()
+    a = r.normal(0, 3, size=(Bt, L, d))
+    C = r.normal(size=(Bt, L, N))
+    x0 = np.einsum("d,n->dn", hc, Bc)[None]
+    _, xL = oracle.scan_fwd(h, a, None, B, C, None, None, x0)
+    np.testing.assert_allclose(xL, x0, rtol=1e-12, atol=1e-12)
+    hr = r.normal(size=(Bt, L, d))
+    Br = r.normal(size=(Bt, L, N))
+    x0r = r.normal(size=(Bt, d, N))
+    bound = np.maximum(np.abs(x0r), np.max(np.abs(np.einsum("btd,btn->btdn", hr, Br)),
+                                           axis=1))
+    for Lk in (1, 5, 30):
+        _, xk = oracle.scan_fwd(hr[:, :Lk], a[:, :Lk], None, Br[:, :Lk], C[:, :Lk], None,
+                                None, x0r)
+        assert np.all(np.abs(xk) <= bound + 1e-12)
+
+
+def test_coupled_gate_gradients_finite_differences():
+    """Coupled gate: a enters through f and i = 1 - f; no b."""
+    t = tiny(82, Bt=2, L=6, d=3, N=4)
+    r = np.random.default_rng(83)
+    dout, dxL = r.normal(size=t["h"].shape), r.normal(size=t["x0"].shape)
+    g = oracle.scan_bwd(t["h"], t["a"], None, t["B"], t["C"], t["z"], t["D"], t["x0"], dout, dxL)
+
+    def loss(tt):
+        out, xL = oracle.scan_fwd(tt["h"], tt["a"], None, tt["B"], tt["C"], tt["z"], tt["D"],
+                                  tt["x0"])
+        return float(np.sum(out * dout) + np.sum(xL * dxL))
+
+    for key, gk in [("h", "dh"), ("a", "da"), ("B", "dB"), ("C", "dC"), ("z", "dz"),
+                    ("D", "dD"), ("x0", "dx0")]:
+        _fd_check(loss, t, key, g[gk])

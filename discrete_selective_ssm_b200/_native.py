@@ -230,7 +230,7 @@ def scan_bwd(dy, hu, a, b, B, C, workspace, *, conv_w=None, conv_b=None, z=None,
         grads = {
             "dhu": torch.empty((Bt, L, d), dtype=ot, device=dev),
             "da": torch.empty((Bt, L, d), dtype=ot, device=dev),
-            "db": torch.empty((Bt, L, d), dtype=ot, device=dev),
+            "db": torch.empty((Bt, L, d), dtype=ot, device=dev) if b is not None else None,
             "dB": torch.empty((Bt, L, N), dtype=ot, device=dev),
             "dC": torch.empty((Bt, L, N), dtype=ot, device=dev),
             "dz": torch.empty((Bt, L, d), dtype=ot, device=dev) if z is not None else None,

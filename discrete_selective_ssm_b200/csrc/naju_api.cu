@@ -201,7 +201,7 @@ naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* co
     naju_status st = check_dims(dims);
     if (st != NAJU_OK) return st;
     if (conv_w && dims->conv_width != 4) return NAJU_ERR_UNSUPPORTED;
-    NAJU_REQUIRE(ok_act(hu) && ok_act(a) && ok_act(b) && ok_act(B) && ok_act(C) && ok_act(y));
+    NAJU_REQUIRE(ok_act(hu) && ok_act(a) && ok_opt(b) && ok_act(B) && ok_act(C) && ok_act(y));
     NAJU_REQUIRE(ok_opt(z) && ok_opt(x0) && ok_opt(x_final));
     NAJU_REQUIRE(workspace && aligned(workspace, 256));
     const Layout l = layout(dims);
@@ -242,8 +242,9 @@ naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* co
     naju_status st = check_dims(dims);
     if (st != NAJU_OK) return st;
     if (conv_w && dims->conv_width != 4) return NAJU_ERR_UNSUPPORTED;
-    NAJU_REQUIRE(ok_act(hu) && ok_act(a) && ok_act(b) && ok_act(B) && ok_act(C) && ok_act(dy));
-    NAJU_REQUIRE(ok_act(dhu) && ok_act(da) && ok_act(db) && ok_act(dB) && ok_act(dC));
+    NAJU_REQUIRE(ok_act(hu) && ok_act(a) && ok_opt(b) && ok_act(B) && ok_act(C) && ok_act(dy));
+    NAJU_REQUIRE(ok_act(dhu) && ok_act(da) && ok_act(dB) && ok_act(dC));
+    NAJU_REQUIRE(b ? ok_act(db) : ok_opt(db));
     NAJU_REQUIRE(ok_opt(z) && ok_opt(dx_final) && ok_opt(dx0));
     NAJU_REQUIRE(!z || ok_act(dz));
     NAJU_REQUIRE(!conv_w || dconv_w);
@@ -295,7 +296,7 @@ naju_status naju_scan_step(int64_t batch, int64_t d_inner, int64_t d_state, int3
     if (d_state != 16 && d_state != 32 && d_state != 64 && d_state != 128)
         return NAJU_ERR_UNSUPPORTED;
     if (dtype != NAJU_F32 && dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
-    NAJU_REQUIRE(ok_act(h) && ok_act(a) && ok_act(b) && ok_act(B) && ok_act(C) && ok_act(y));
+    NAJU_REQUIRE(ok_act(h) && ok_act(a) && ok_opt(b) && ok_act(B) && ok_act(C) && ok_act(y));
     NAJU_REQUIRE(ok_opt(z) && ok_act(state));
     return cuda_status(launch_scan_step(batch, d_inner, d_state, h, a, b, B, C, z, D, state, y,
                                         dtype, nullptr, nullptr, nullptr,
@@ -322,7 +323,7 @@ naju_status naju_scan_step_conv(int64_t batch, int64_t d_inner, int64_t d_state,
     if (d_state != 16 && d_state != 32 && d_state != 64 && d_state != 128)
         return NAJU_ERR_UNSUPPORTED;
     if (dtype != NAJU_F32 && dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
-    NAJU_REQUIRE(ok_act(u) && ok_act(a) && ok_act(b) && ok_act(B) && ok_act(C) && ok_act(y));
+    NAJU_REQUIRE(ok_act(u) && ok_act(a) && ok_opt(b) && ok_act(B) && ok_act(C) && ok_act(y));
     NAJU_REQUIRE(ok_opt(z) && ok_act(state) && conv_w && ok_act(conv_state) && ok_opt(conv_b));
     return cuda_status(launch_scan_step(batch, d_inner, d_state, u, a, b, B, C, z, D, state, y,
                                         dtype, conv_w, conv_b, conv_state,

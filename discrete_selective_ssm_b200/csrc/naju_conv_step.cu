@@ -182,8 +182,10 @@ step_kernel(int64_t d, const T* __restrict__ h, const T* __restrict__ a,
             conv_state[eg * 3 + 2] = hh;
             hh = siluf_(p);
         }
-        f = sigmoidf_(to_f(a[eg]));
-        v = sigmoidf_(to_f(b[eg])) * hh;
+        const float ea = __expf(-to_f(a[eg]));
+        f = rcpf_(1.f + ea);
+        // b absent: coupled single gate i = 1 - f
+        v = (b ? sigmoidf_(to_f(b[eg])) : ea * f) * hh;
         dh = D ? D[cg] * hh : 0.f;
         if (z) gz = siluf_(to_f(z[eg]));
     }

@@ -70,7 +70,7 @@ naju_status naju_scan_fwd_noalloc(const naju_dims* dims, const void* hu, const f
     if (dims->out_dtype != NAJU_F32 && dims->out_dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
     if (dims->dtype == NAJU_F32 && dims->out_dtype != NAJU_F32) return NAJU_ERR_UNSUPPORTED;
     if (conv_w && dims->conv_width != 4) return NAJU_ERR_UNSUPPORTED;
-    if (!hu || !a || !b || !B || !C || !y) return NAJU_ERR_INVALID_ARG;
+    if (!hu || !a || !B || !C || !y) return NAJU_ERR_INVALID_ARG;  // b NULL: coupled gate
     const void* required[] = {hu, a, b, B, C, y};
     for (const void* q : required)
         if (!aligned16(q)) return NAJU_ERR_INVALID_ARG;

@@ -129,7 +129,8 @@ scan_bwd_kernel(const BwdParams p) {
     const int64_t boff = (int64_t)bb * L;
     const Tin* hu = static_cast<const Tin*>(p.hu) + boff * d;
     const Tin* ga = static_cast<const Tin*>(p.a) + boff * d;
-    const Tin* gbp = static_cast<const Tin*>(p.b) + boff * d;
+    // b absent: coupled single gate i = 1 - f (a also reaches i; no db).
+    const Tin* gbp = p.b ? static_cast<const Tin*>(p.b) + boff * d : nullptr;
     const Tin* gz = p.z ? static_cast<const Tin*>(p.z) + boff * d : nullptr;
     const Tin* gdy = static_cast<const Tin*>(p.dy) + boff * d;
     const Tin* gB = static_cast<const Tin*>(p.B) + boff * N;
@@ -150,7 +151,7 @@ scan_bwd_kernel(const BwdParams p) {
     auto issue = [&](int64_t t0, int64_t tlim) {
         stage_rows(&sm.u[0][0], hu, d, t0 - 3, T + 3, L, c0, P, vec, tid, NT);
         stage_rows(&sm.a[0][0], ga, d, t0, T, tlim, c0, P, vec, tid, NT);
-        stage_rows(&sm.b[0][0], gbp, d, t0, T, tlim, c0, P, vec, tid, NT);
+        if (gbp) stage_rows(&sm.b[0][0], gbp, d, t0, T, tlim, c0, P, vec, tid, NT);
         if (gz) stage_rows(&sm.z[0][0], gz, d, t0, T, tlim, c0, P, vec, tid, NT);
         stage_rows(&sm.dout[0][0], gdy, d, t0, T, tlim, c0, P, vec, tid, NT);
         stage_rows(&sm.Bm[0][0], gB, N, t0, T, tlim, 0, N, true, tid, NT);
@@ -176,9 +177,10 @@ scan_bwd_kernel(const BwdParams p) {
                 } else {
                     h = to_f(sm.u[tt + 3][pp]);
                 }
-                q = 1.f + __expf(-to_f(sm.a[tt][pp]));
+                const float ea = __expf(-to_f(sm.a[tt][pp]));
+                q = 1.f + ea;
                 f = rcpf_(q);
-                v = sigmoidf_(to_f(sm.b[tt][pp])) * h;
+                v = (gbp ? sigmoidf_(to_f(sm.b[tt][pp])) : ea * f) * h;
                 dyv = to_f(sm.dout[tt][pp]);
                 if (gz) dyv *= siluf_(to_f(sm.z[tt][pp]));
             }
@@ -428,7 +430,7 @@ scan_bwd_kernel(const BwdParams p) {
     float dD_acc = 0.f, dw0 = 0.f, dw1 = 0.f, dw2 = 0.f, dw3 = 0.f, dbias = 0.f;
     Tout* gdhu = static_cast<Tout*>(p.dhu) + boff * d;
     Tout* gda = static_cast<Tout*>(p.da) + boff * d;
-    Tout* gdb = static_cast<Tout*>(p.db) + boff * d;
+    Tout* gdb = p.db ? static_cast<Tout*>(p.db) + boff * d : nullptr;
     Tout* gdz = p.dz ? static_cast<Tout*>(p.dz) + boff * d : nullptr;
     float* edge = p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d;
     if (tid < P) {  // dp beyond the group: zero (the next group's terms go via the edge fixup)
@@ -589,12 +591,17 @@ scan_bwd_kernel(const BwdParams p) {
                         h = to_f(sm.u[tt + 3][pp]);
                     }
                     const float fv = sm.f[tt][pp];
-                    const float iv = sigmoidf_(to_f(sm.b[tt][pp]));
+                    const float iv = gbp ? sigmoidf_(to_f(sm.b[tt][pp]))
+                                         : __expf(-to_f(sm.a[tt][pp])) * fv;
                     const float gbv = sm.x1[tt][pp];
                     const float dyv = sm.dy[tt][pp];
                     const float dh = Dc * dyv + iv * gbv;
-                    gda[t * d + cp] = from_f<Tout>(sm.x3[tt][pp] * (1.f - fv));
-                    gdb[t * d + cp] = from_f<Tout>(h * gbv * iv * (1.f - iv));
+                    if (gbp) {
+                        gda[t * d + cp] = from_f<Tout>(sm.x3[tt][pp] * (1.f - fv));
+                        gdb[t * d + cp] = from_f<Tout>(h * gbv * iv * (1.f - iv));
+                    } else {  // da = (f df - f di)(1 - f), di = h G.B
+                        gda[t * d + cp] = from_f<Tout>((sm.x3[tt][pp] - fv * h * gbv) * iv);
+                    }
                     if (gz) {
                         const float zv = to_f(sm.z[tt][pp]);
                         const float yv = fmaf(s, sm.ys[sb * T + tt][pp], Dc * h);

@@ -144,6 +144,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     const int64_t Bt = p.Bt, L = p.L, d = p.d;
     const float s = p.scale;
     const bool has_z = p.z != nullptr;
+    const bool has_b = p.b != nullptr;  // absent: coupled single gate i = 1 - f
 
     // ------------------------------------------------------------ set-up
     if (warp == 0) {
@@ -156,7 +157,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         tc::mbar_init(&sm.mma, 1);
         tma::prefetch_map(&tm.u);
         tma::prefetch_map(&tm.a);
-        tma::prefetch_map(&tm.b);
+        if (p.b) tma::prefetch_map(&tm.b);
         if (has_z) tma::prefetch_map(&tm.z);
         tma::prefetch_map(&tm.dy);
         tma::prefetch_map(&tm.B);
@@ -197,7 +198,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     const int64_t boff = (int64_t)bb * L;
     Tout* gdhu = static_cast<Tout*>(p.dhu) + boff * d + c;
     Tout* gda = static_cast<Tout*>(p.da) + boff * d + c;
-    Tout* gdb = static_cast<Tout*>(p.db) + boff * d + c;
+    Tout* gdb = p.db ? static_cast<Tout*>(p.db) + boff * d + c : nullptr;
     Tout* gdz = has_z ? static_cast<Tout*>(p.dz) + boff * d + c : nullptr;
     float* part = p.dBCp + (((int64_t)tile * Bt + bb) * L) * 2 * N;  // [L][2][N]
     float* edge = p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d;
@@ -229,12 +230,13 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         typename Sm::Raw& r = sm.raw[buf];
         uint64_t* mb = &sm.loaded[buf];
         const uint32_t bytes =
-            (uint32_t)sizeof(Tin) * ((T + 3) * P + (has_z ? 4 : 3) * T * P + 2 * T * N);
+            (uint32_t)sizeof(Tin) *
+            ((T + 3) * P + (2 + (has_z ? 1 : 0) + (has_b ? 1 : 0)) * T * P + 2 * T * N);
         tma::expect_tx(mb, bytes);
         const int x = (int)c0, y = (int)item_t0(li), zb = bb;
         tma::load_3d(&r.u[0][0], &tm.u, x, y - 3, zb, mb);
         tma::load_3d(&r.a[0][0], &tm.a, x, y, zb, mb);
-        tma::load_3d(&r.b[0][0], &tm.b, x, y, zb, mb);
+        if (has_b) tma::load_3d(&r.b[0][0], &tm.b, x, y, zb, mb);
         if (has_z) tma::load_3d(&r.z[0][0], &tm.z, x, y, zb, mb);
         tma::load_3d(&r.dy[0][0], &tm.dy, x, y, zb, mb);
         tma::load_3d(&r.Bm[0][0], &tm.B, 0, y, zb, mb);
@@ -364,7 +366,8 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         for (int k = 0; k < TQ; ++k) {
             const int tt = qd * TQ + k;
             const bool valid = k < nvh;
-            qv[k] = valid ? 1.f + __expf(-to_f(r.a[tt][ch])) : 1.f;
+            const float ea = valid ? __expf(-to_f(r.a[tt][ch])) : 0.f;
+            qv[k] = 1.f + ea;
             fv[k] = rcpa_(qv[k]);
             Qh *= qv[k];
             Eh *= fv[k];
@@ -379,7 +382,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 hh = to_f(r.u[tt + 3][ch]);
             }
             hv[k] = valid ? hh : 0.f;
-            iv[k] = sigmoida_(to_f(r.b[tt][ch]));
+            iv[k] = has_b ? sigmoida_(to_f(r.b[tt][ch])) : ea * fv[k];
             float gg = 1.f;
             if (has_z) {
                 const float zv = to_f(r.z[tt][ch]);
@@ -856,8 +859,13 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 float dpv = 0.f;
                 if (q < nvh) {
                     const float dh = fmaf(Dc, dyv[q], iv[q] * gbv[q]);
-                    gda[t * d] = from_f<Tout>((base + sfx[q]) * (1.f - fv[q]));
-                    gdb[t * d] = from_f<Tout>(hv[q] * gbv[q] * iv[q] * (1.f - iv[q]));
+                    if (has_b) {
+                        gda[t * d] = from_f<Tout>((base + sfx[q]) * (1.f - fv[q]));
+                        gdb[t * d] = from_f<Tout>(hv[q] * gbv[q] * iv[q] * (1.f - iv[q]));
+                    } else {  // da = (f df - f di)(1 - f), di = h G.B; 1 - f = i
+                        gda[t * d] =
+                            from_f<Tout>((base + sfx[q] - fv[q] * hv[q] * gbv[q]) * iv[q]);
+                    }
                     dD_acc = fmaf(dyv[q], hv[q], dD_acc);
                     if (CONV) {
                         dpv = dh * aux[q];
@@ -937,7 +945,7 @@ static cudaError_t launch_bwd_tc_t(const BwdParams& p, cudaStream_t st) {
     const int T = kBT;
     bool ok = tma_encode_bf16_3d(&tm.u, p.hu, p.Bt, p.L, p.d, T + 3, 128) &&
               tma_encode_bf16_3d(&tm.a, p.a, p.Bt, p.L, p.d, T, 128) &&
-              tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, T, 128) &&
+              (!p.b || tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, T, 128)) &&
               tma_encode_bf16_3d(&tm.dy, p.dy, p.Bt, p.L, p.d, T, 128) &&
               tma_encode_bf16_3d(&tm.B, p.B, p.Bt, p.L, N, T, N) &&
               tma_encode_bf16_3d(&tm.C, p.C, p.Bt, p.L, N, T, N);

@@ -96,7 +96,8 @@ scan_fwd_kernel(const FwdParams p) {
     const int64_t boff = (int64_t)bb * L;
     const Tin* hu = static_cast<const Tin*>(p.hu) + boff * d;
     const Tin* ga = static_cast<const Tin*>(p.a) + boff * d;
-    const Tin* gb = static_cast<const Tin*>(p.b) + boff * d;
+    // b absent: coupled single gate i = 1 - f.
+    const Tin* gb = p.b ? static_cast<const Tin*>(p.b) + boff * d : nullptr;
     const Tin* gz = p.z ? static_cast<const Tin*>(p.z) + boff * d : nullptr;
     const Tin* gB = static_cast<const Tin*>(p.B) + boff * N;
     const Tin* gC = static_cast<const Tin*>(p.C) + boff * N;
@@ -127,7 +128,7 @@ scan_fwd_kernel(const FwdParams p) {
         FwdRaw<Tin, P, N>& r = sm.raw[buf];
         stage_rows(&r.u[0][0], hu, d, t0 - 3, T + 3, L, c0, P, vec, tid, NT);
         stage_rows(&r.a[0][0], ga, d, t0, T, tend, c0, P, vec, tid, NT);
-        stage_rows(&r.b[0][0], gb, d, t0, T, tend, c0, P, vec, tid, NT);
+        if (gb) stage_rows(&r.b[0][0], gb, d, t0, T, tend, c0, P, vec, tid, NT);
         if (full && gz) stage_rows(&r.z[0][0], gz, d, t0, T, tend, c0, P, vec, tid, NT);
         stage_rows(&r.Bm[0][0], gB, N, t0, T, tend, 0, N, true, tid, NT);
         if (full) stage_rows(&r.Cm[0][0], gC, N, t0, T, tend, 0, N, true, tid, NT);
@@ -152,9 +153,10 @@ scan_fwd_kernel(const FwdParams p) {
                 } else {
                     h = to_f(r.u[tt + 3][pp]);
                 }
-                q = 1.f + __expf(-to_f(r.a[tt][pp]));
+                const float ea = __expf(-to_f(r.a[tt][pp]));
+                q = 1.f + ea;
                 f = rcpf_(q);
-                v = sigmoidf_(to_f(r.b[tt][pp])) * h;
+                v = (gb ? sigmoidf_(to_f(r.b[tt][pp])) : ea * f) * h;
             }
             sm.sQ[tt][pp] = q;
             sm.sF[tt][pp] = f;

@@ -145,7 +145,7 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
         tc::mbar_init(&sm.mma, 1);
         tma::prefetch_map(&tm.u);
         tma::prefetch_map(&tm.a);
-        tma::prefetch_map(&tm.b);
+        if (p.b) tma::prefetch_map(&tm.b);
         if (p.z) tma::prefetch_map(&tm.z);
         tma::prefetch_map(&tm.B);
         tma::prefetch_map(&tm.C);
@@ -172,6 +172,7 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
 
     const int64_t boff = (int64_t)bb * L;
     const bool has_z = p.z != nullptr;
+    const bool has_b = p.b != nullptr;  // absent: coupled single gate i = 1 - f
     Tout* gy = static_cast<Tout*>(p.y) + boff * d;
 
     float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, wb = 0.f, Dc = 0.f;
@@ -195,13 +196,14 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
         typename Sm::Raw& r = sm.raw[buf];
         uint64_t* mb = &sm.loaded[buf];
         const bool zz = full && has_z;
-        const uint32_t bytes = (uint32_t)sizeof(Tin) *
-                               ((T + 3) * P + 2 * T * P + (zz ? T * P : 0) + (full ? 2 : 1) * T * N);
+        const uint32_t bytes =
+            (uint32_t)sizeof(Tin) * ((T + 3) * P + (has_b ? 2 : 1) * T * P + (zz ? T * P : 0) +
+                                     (full ? 2 : 1) * T * N);
         tma::expect_tx(mb, bytes);
         const int x = (int)c0, y = (int)t0, zb = bb;
         tma::load_3d(&r.u[0][0], &tm.u, x, y - 3, zb, mb);
         tma::load_3d(&r.a[0][0], &tm.a, x, y, zb, mb);
-        tma::load_3d(&r.b[0][0], &tm.b, x, y, zb, mb);
+        if (has_b) tma::load_3d(&r.b[0][0], &tm.b, x, y, zb, mb);
         if (zz) tma::load_3d(&r.z[0][0], &tm.z, x, y, zb, mb);
         tma::load_3d(&r.Bm[0][0], &tm.B, 0, y, zb, mb);
         if (full) tma::load_3d(&r.Cm[0][0], &tm.C, 0, y, zb, mb);
@@ -225,13 +227,14 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
         // Tokens of this thread's half inside [t0, tend) (0 for a padding channel).
         const int nv = cvalid ? (int)max((int64_t)0, min64((int64_t)H, tend - t0 - phalf * H)) : 0;
         // Per-channel values: this thread's 8 tokens.
-        float qv[H], fv[H], hv[H];
+        float qv[H], fv[H], hv[H], ev[H];
         float Qh = 1.f, Eh = 1.f;
 #pragma unroll
         for (int k = 0; k < H; ++k) {
             const int tt = phalf * H + k;
             const bool valid = k < nv;
-            qv[k] = valid ? 1.f + __expf(-to_f(r.a[tt][pch])) : 1.f;
+            ev[k] = valid ? __expf(-to_f(r.a[tt][pch])) : 0.f;
+            qv[k] = 1.f + ev[k];
             fv[k] = rcpa_(qv[k]);
             Qh *= qv[k];
             Eh *= fv[k];
@@ -291,7 +294,8 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
 #pragma unroll
         for (int k = 0; k < H; ++k) {
             const int tt = phalf * H + k;
-            const float v = sigmoida_(to_f(r.b[tt][pch])) * hv[k];  // 0 past the end (h = 0)
+            const float iw = has_b ? sigmoida_(to_f(r.b[tt][pch])) : ev[k] * fv[k];
+            const float v = iw * hv[k];  // 0 past the end (h = 0)
             E *= fv[k];
             Q *= qv[k];
             if (slow) {
@@ -594,7 +598,7 @@ static cudaError_t launch_fwd_tc_t(const FwdParams& p, cudaStream_t st) {
     const int T = kTS;
     bool ok = tma_encode_bf16_3d(&tm.u, p.hu, p.Bt, p.L, p.d, T + 3, 128) &&
               tma_encode_bf16_3d(&tm.a, p.a, p.Bt, p.L, p.d, T, 128) &&
-              tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, T, 128) &&
+              (!p.b || tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, T, 128)) &&
               tma_encode_bf16_3d(&tm.B, p.B, p.Bt, p.L, N, T, N) &&
               tma_encode_bf16_3d(&tm.C, p.C, p.Bt, p.L, N, T, N);
     if (ok && p.z) ok = tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, T, 128);

@@ -96,9 +96,11 @@ naju_status naju_conv_silu_bwd(const naju_dims* dims, const void* u, const float
 /* Forward scan (README, "Core equations"), fused with the conv + SiLU that
  * produces h when conv_w != NULL (then `hu` is u; otherwise `hu` is h) and
  * with the SiLU(z) output modulation when z != NULL.  D == NULL means no
- * feedthrough; x0 == NULL means a zero initial state.  Writes y (out_dtype),
- * optionally x_final, and the state checkpoints the backward needs into the
- * workspace. */
+ * feedthrough; x0 == NULL means a zero initial state.  b == NULL selects the
+ * coupled single gate i = 1 - sigmoid(a) (the complementary gating analysed in
+ * the paper's abstract) instead of i = sigmoid(b); the same holds for every
+ * entry point below that takes b.  Writes y (out_dtype), optionally x_final,
+ * and the state checkpoints the backward needs into the workspace. */
 naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* conv_w,
                           const float* conv_b, const void* a, const void* b, const void* B,
                           const void* C, const void* z, const float* D, const float* x0,
@@ -131,7 +133,8 @@ naju_status naju_scan_fwd_noalloc(const naju_dims* dims, const void* hu, const f
  * workspace must hold that forward's checkpoints.  Writes dhu (du in fused
  * mode, dh otherwise), da, db, dB, dC and dz (when z != NULL) in out_dtype,
  * and overwrites dD (when D != NULL), dconv_w and dconv_b (fused mode) and
- * dx0 (when not NULL) in fp32. */
+ * dx0 (when not NULL) in fp32.  With b == NULL (coupled gate) da includes the
+ * write-gate path, db is not written and may be NULL. */
 naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* conv_w,
                           const float* conv_b, const void* a, const void* b, const void* B,
                           const void* C, const void* z, const float* D, const float* x0,

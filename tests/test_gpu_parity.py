@@ -515,3 +515,64 @@ def test_conv_steps_equal_fused_forward():
         assert_close(yn, ro[:, n], TOL_F32, name=f"y[{n}]")
     torch.cuda.synchronize()
     assert_close(st, rx, TOL_F32, name="state")
+
+
+# ------------------------------------------- coupled single gate (i = 1 - f)
+@pytest.mark.parametrize("N", [16, 64, 128])
+@pytest.mark.parametrize("impl", [1, 0])
+def test_coupled_gate_fwd_bwd(N, impl):
+    """b absent: i = 1 - f in the forward and the backward (both
+    implementations; bf16, fused conv, ragged sizes)."""
+    w = wl(N, "bf16", Bt=2, L=333, d=264)
+    t = inputs(w, True, use_x0=True, use_dxL=True)
+    t["b"] = None
+    naju.testing_set_fwd_impl(impl)
+    naju.testing_set_bwd_impl(impl)
+    try:
+        g = run_bwd(t, True, out_dtype=naju.F32)
+        y, xf, _ = run_fwd(t, True, out_dtype=naju.F32)
+    finally:
+        naju.testing_set_fwd_impl(0)
+        naju.testing_set_bwd_impl(0)
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_BF16, name="y")
+    assert_close(xf, rx, TOL_BF16, name="x_final")
+    r = oracle_bwd(t, True)
+    assert g["db"] is None
+    assert_close(g["dhu"], r["du"], TOL_BF16, name="du")
+    for k in ("da", "dB", "dC", "dz"):
+        assert_close(g[k], r[k], TOL_BF16, name=k)
+    assert_close(g["dx0"], r["dx0"], TOL_BF16, name="dx0")
+    assert_close(g["dconv_w"], r["dconv_w"], TOL_BF16, name="dconv_w")
+
+
+def test_coupled_gate_fp32_unfused():
+    w = wl(32, "f32", Bt=2, L=200, d=70)
+    t = inputs(w, False, use_x0=True, use_dxL=True)
+    t["b"] = None
+    g = run_bwd(t, False)
+    r = oracle_bwd(t, False)
+    assert_close(g["dhu"], r["dh"], TOL_F32, name="dh")
+    for k in ("da", "dB", "dC", "dz", "dx0"):
+        assert_close(g[k], r[k], TOL_F32, name=k)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_coupled_gate_step(dtype):
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    gen = torch.Generator().manual_seed(7)
+    Bt, d, N = 3, 50, 64
+    state = torch.randn(Bt, d, N, generator=gen)
+    cs = torch.randn(Bt, d, 3, generator=gen)
+    u, a, z = (torch.randn(Bt, d, generator=gen).to(tdt) for _ in range(3))
+    B, C = (torch.randn(Bt, N, generator=gen).to(tdt) for _ in range(2))
+    D = torch.randn(d, generator=gen)
+    w = torch.randn(d, 4, generator=gen) * 0.5
+    ro, rs, rcs = oracle.block_step(state, cs, u, w, None, a, None, B, C, z, D)
+    st, gcs = gpu(state), gpu(cs)
+    y = naju.scan_step_conv(st, gcs, gpu(u), gpu(a), None, gpu(B), gpu(C), gpu(w), None,
+                            gpu(z), gpu(D))
+    torch.cuda.synchronize()
+    tol = tol_of(dtype)
+    assert_close(y, ro, tol, bf16_out=(dtype == "bf16"), name="y")
+    assert_close(st, rs, tol, name="state")

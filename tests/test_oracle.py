@@ -334,3 +334,30 @@ def test_coupled_gate_gradients_finite_differences():
     for key, gk in [("h", "dh"), ("a", "da"), ("B", "dB"), ("C", "dC"), ("z", "dz"),
                     ("D", "dD"), ("x0", "dx0")]:
         _fd_check(loss, t, key, g[gk])
+
+
+# ------------------------------------------------------ the full block
+@pytest.mark.parametrize("coupled", [False, True])
+def test_block_oracle_finite_differences(coupled):
+    """Full block (norm, projections, conv, scan, modulation, residual): every
+    gradient against central finite differences."""
+    from oracle import block as ob
+    r = np.random.default_rng(90)
+    Bt, L, dm, di, N = 1, 5, 4, 3, 4
+    p = {k: v.astype(np.float64) for k, v in ob.init_params(dm, di, N, seed=91).items()}
+    x = r.normal(size=(Bt, L, dm))
+    dout = r.normal(size=(Bt, L, dm))
+    out, cache = ob.block_fwd(x, p, coupled)
+    dx, g = ob.block_bwd(cache, dout, coupled)
+    t = dict(p, x=x)
+
+    def loss(tt):
+        pp = {k: tt[k] for k in ob.PARAMS}
+        o, _ = ob.block_fwd(tt["x"], pp, coupled)
+        return float(np.sum(o * dout))
+
+    _fd_check(loss, t, "x", dx, rtol=1e-5)
+    for k in ob.PARAMS:
+        if coupled and k in ("W_b", "b_b"):
+            continue
+        _fd_check(loss, t, k, g[k], rtol=1e-5)

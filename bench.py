@@ -317,6 +317,71 @@ def run_decode(args, w, rank, world, local):
         dist.destroy_process_group()
 
 
+def run_block(args, w, rank, world, local):
+    """Full-block bench: one step = block forward + backward over the batch."""
+    from discrete_selective_ssm_b200.block import NajuBlock
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dm = w.d_inner // 2
+    blk = NajuBlock(dm, w.d_inner, w.d_state, dev, dtype=w.torch_dtype, seed=1,
+                    coupled=args.coupled)
+    gen = torch.Generator().manual_seed(2)
+    x = torch.randn(w.batch, w.seqlen, dm, generator=gen).to(dev, w.torch_dtype)
+    dout = torch.randn(w.batch, w.seqlen, dm, generator=gen).to(dev, w.torch_dtype)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        out, ctx = blk.forward(x)
+        blk.backward(ctx, dout)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = clk.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if dist is not None:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    di, N = w.d_inner, w.d_state
+    gemm_flop = 2 * w.batch * w.seqlen * (dm * 2 * di + 2 * di * di + 2 * di * N + di * dm) * 3
+    if rank == 0:
+        print(json.dumps({
+            "metric": "naju_block_fwd_bwd_tokens_per_s", "value": world * w.batch * w.seqlen /
+            (ms / 1e3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name + "_block", "batch": w.batch, "seqlen": w.seqlen,
+                       "d_model": dm, "d_inner": di, "d_state": N, "coupled": args.coupled,
+                       "gemm_tflop_per_step": gemm_flop / 1e12,
+                       "parallelism": f"replicas{world}"},
+            "roofline": None, "cpu_baseline": None, "e2e": None,
+            "gpu_launches": None, "clocks": clocks,
+        }), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -326,6 +391,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--block", action="store_true",
+                    help="time the full Naju block (norm, projections, conv, scan, residual) "
+                         "with d_model = d_inner / 2 instead of the scan alone")
+    ap.add_argument("--coupled", action="store_true",
+                    help="coupled single gate i = 1 - f (no b input)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -342,6 +412,9 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, w, rank, world)
+        return
+    if args.block:
+        run_block(args, w, rank, world, local)
         return
 
     import discrete_selective_ssm_b200 as naju
@@ -379,12 +452,14 @@ def main():
     def step(inp, ev=None):
         if ev is not None:
             ev[0].record(stream)
-        naju.scan_fwd(inp["u"], inp["a"], inp["b"], inp["B"], inp["C"], conv_w=inp["conv_w"],
+        naju.scan_fwd(inp["u"], inp["a"], None if args.coupled else inp["b"], inp["B"], inp["C"],
+                      conv_w=inp["conv_w"],
                       conv_b=inp["conv_b"], z=inp["z"], D=inp["D"], out_dtype=out_dt,
                       workspace=ws, want_final=False, y=y)
         if ev is not None:
             ev[1].record(stream)
-        naju.scan_bwd(inp["dout"], inp["u"], inp["a"], inp["b"], inp["B"], inp["C"], ws,
+        naju.scan_bwd(inp["dout"], inp["u"], inp["a"], None if args.coupled else inp["b"],
+                      inp["B"], inp["C"], ws,
                       conv_w=inp["conv_w"], conv_b=inp["conv_b"], z=inp["z"], D=inp["D"],
                       out_dtype=out_dt, grads=grads)
         if ev is not None:
@@ -501,7 +576,8 @@ def main():
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
                        "d_inner": w.d_inner, "d_state": w.d_state, "conv_width": 4,
-                       "fused_conv": True, "gating": True, "parallelism": f"replicas{world}",
+                       "fused_conv": True, "gating": True, "coupled_gate": args.coupled,
+                       "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (no flush)",
                        "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
                        "fwd_gbs": fwd_b / (fwd_ms / 1e3) / 1e9,

@@ -36,7 +36,7 @@
 // Threads.  512 per block: channel p (TMEM lane p) is handled by threads
 // p + 128 q, q = 0..3, each taking 4 of the 16 tokens and a quarter of the
 // state columns; one thread issues the MMAs.  Raw inputs arrive by TMA one
-// sub-chunk ahead (two buffers).
+// or two sub-chunks ahead (two or three buffers), issued while the MMAs run.
 //
 // Exactness.  A sub-chunk whose product of 1/f exceeds 2^64 in any channel of
 // the block takes an exact token-by-token path on the CUDA cores (states in
@@ -102,9 +102,9 @@ struct BwdTcSmem {
     };
     alignas(1024) float st[ST_FLOATS];
     alignas(1024) float pk[T * P];     // Y or P, swizzled, rows t, K = channels
-    // Raw-input buffers: TMA runs NRAW - 1 sub-chunks ahead.  (A third buffer
-    // for d_state 64 measured no faster.)
-    static constexpr int NRAW = 2;
+    // Raw-input buffers: TMA runs up to NRAW - 1 sub-chunks ahead (three for
+    // d_state 64; shared memory allows two for 128).
+    static constexpr int NRAW = N <= 64 ? 3 : 2;
     Raw raw[NRAW];
     alignas(128) float ta[T * N];      // C (forward) / B (backward) rows t, K = d_state
     alignas(128) float ts[TS_FLOATS];  // B^T (forward) / C^T (backward): rows d_state, K = 16
@@ -500,6 +500,10 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         }
         tc::fence_proxy_async();
         sync();
+        // Prefetch: buffer (li + NRAW - 1) % NRAW was last read by item li - 1.
+        // Issued here, by a thread other than the MMA issuer, so it overlaps
+        // the MMA wait instead of delaying the item's first barrier.
+        if (tid == 32 && li + Sm::NRAW - 1 < nitems) issue(li + Sm::NRAW - 1);
     };
 
     // MMAs of the current item (one thread), then commit.
@@ -547,8 +551,6 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
 
     // Start item li: prefetch the next one, wait for this one's inputs.
     auto begin_item = [&]() {
-        // Buffer (li + NRAW - 1) % NRAW was last read by item li - 1.
-        if (tid == 0 && li + Sm::NRAW - 1 < nitems) issue(li + Sm::NRAW - 1);
         if (!tc::mbar_wait(&sm.loaded[li % Sm::NRAW], (uint32_t)((li / Sm::NRAW) & 1), kBSpin))
             timed_out = true;
     };

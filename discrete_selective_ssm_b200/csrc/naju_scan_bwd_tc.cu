@@ -154,7 +154,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     if (tid == 0) {
         sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
         for (int q = 0; q < Sm::NRAW; ++q) tc::mbar_init(&sm.loaded[q], 1);
-        tc::mbar_init(&sm.mma, 1);
+        tc::mbar_init(&sm.mma, 3);  // one arrival per MMA chain
         tma::prefetch_map(&tm.u);
         tma::prefetch_map(&tm.a);
         if (p.b) tma::prefetch_map(&tm.b);
@@ -507,44 +507,51 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     };
 
     // MMAs of the current item (one thread), then commit.
-    auto issue_mma = [&](int sweep) {
+    // MMAs of the current item: three independent accumulation chains, each
+    // issued (and committed to the 3-arrival barrier sm.mma) by lane 0 of its
+    // own warp so their issue overlaps: chain 0, readout (forward: X . C + W G)
+    // or dv (backward: H . B + U G^T) into R; chain 1, state (forward: V B^T)
+    // or adjoint (backward: (s dy E) C^T) into D; chain 2, dC or dB
+    // ((state^T)(Y or P) over channels + (B^T or C^T)(A_C or A_B)) into BC.
+    // The early sweep runs chain 1 only; the other two lanes just arrive.
+    auto issue_chain = [&](int chain, int sweep) {
         constexpr uint32_t id16 = tc::idesc_tf32(128, T);
         constexpr uint32_t idN = tc::idesc_tf32(128, N);
-        const uint32_t a_ta = tc::smem_u32(sm.ta), a_ts = tc::smem_u32(sm.ts);
-        const uint32_t a_tg = tc::smem_u32(sm.tg), a_t2 = tc::smem_u32(sm.ta2);
-        const uint32_t a_st = tc::smem_u32(sm.st), a_pk = tc::smem_u32(sm.pk);
-        // Three independent accumulation chains, issued interleaved so the
-        // tensor core can overlap them: readout (forward: X . C + W G) or dv
-        // (backward: H . B + U G^T) into R; state (forward: V B^T) or adjoint
-        // (backward: (s dy E) C^T) into D; dC or dB ((state^T)(Y or P) over
-        // channels + (B^T or C^T)(A_C or A_B)) into BC.
         const bool full = sweep != kSweepEarly;
-        const uint32_t Acol = sweep == kSweepFwd ? Cols::X : Cols::G;
-        constexpr int NR = N / 8 + T / 8, NBC = P / 8 + T / 8, ND = T / 8;
+        if (chain != 1 && !full) {
+            tc::mbar_arrive(&sm.mma);
+            return;
+        }
+        if (chain == 0) {
+            const uint32_t a_ta = tc::smem_u32(sm.ta), a_tg = tc::smem_u32(sm.tg);
+            const uint32_t Acol = sweep == kSweepFwd ? Cols::X : Cols::G;
 #pragma unroll
-        for (int i = 0; i < NBC; ++i) {
-            if (full && i < NR) {
-                if (i < N / 8)
-                    tc::mma_tf32_ts(tbase + Cols::R, tbase + Acol + i * 8,
-                                    tc::sdesc(a_ta + i * 256, 128, 32 * N), id16, i > 0 ? 1u : 0u);
-                else
-                    tc::mma_tf32_ts(tbase + Cols::R, tbase + Cols::WU + (i - N / 8) * 8,
-                                    tc::sdesc(a_tg + (i - N / 8) * 256, 128, 32 * T), id16, 1u);
-            }
-            if (i < ND)
+            for (int i = 0; i < N / 8; ++i)
+                tc::mma_tf32_ts(tbase + Cols::R, tbase + Acol + i * 8,
+                                tc::sdesc(a_ta + i * 256, 128, 32 * N), id16, i > 0 ? 1u : 0u);
+#pragma unroll
+            for (int i = 0; i < T / 8; ++i)
+                tc::mma_tf32_ts(tbase + Cols::R, tbase + Cols::WU + i * 8,
+                                tc::sdesc(a_tg + i * 256, 128, 32 * T), id16, 1u);
+        } else if (chain == 1) {
+            const uint32_t a_ts = tc::smem_u32(sm.ts);
+#pragma unroll
+            for (int i = 0; i < T / 8; ++i)
                 tc::mma_tf32_ts(tbase + Cols::D, tbase + Cols::VV + i * 8,
                                 tc::sdesc(a_ts + i * 256, 128, 32 * T), idN, i > 0 ? 1u : 0u);
-            if (full) {
-                if (i < P / 8)
-                    tc::mma_tf32_ss(tbase + Cols::BC,
-                                    tc::sdesc_sw128(a_st + (i >> 2) * N * 128 + (i & 3) * 32),
-                                    tc::sdesc_sw128(a_pk + (i >> 2) * T * 128 + (i & 3) * 32),
-                                    id16, i > 0 ? 1u : 0u);
-                else
-                    tc::mma_tf32_ss(tbase + Cols::BC,
-                                    tc::sdesc(a_ts + (i - P / 8) * 256, 128, 32 * T),
-                                    tc::sdesc(a_t2 + (i - P / 8) * 256, 128, 32 * T), id16, 1u);
-            }
+        } else {
+            const uint32_t a_ts = tc::smem_u32(sm.ts), a_t2 = tc::smem_u32(sm.ta2);
+            const uint32_t a_st = tc::smem_u32(sm.st), a_pk = tc::smem_u32(sm.pk);
+#pragma unroll
+            for (int i = 0; i < P / 8; ++i)
+                tc::mma_tf32_ss(tbase + Cols::BC,
+                                tc::sdesc_sw128(a_st + (i >> 2) * N * 128 + (i & 3) * 32),
+                                tc::sdesc_sw128(a_pk + (i >> 2) * T * 128 + (i & 3) * 32), id16,
+                                i > 0 ? 1u : 0u);
+#pragma unroll
+            for (int i = 0; i < T / 8; ++i)
+                tc::mma_tf32_ss(tbase + Cols::BC, tc::sdesc(a_ts + i * 256, 128, 32 * T),
+                                tc::sdesc(a_t2 + i * 256, 128, 32 * T), id16, 1u);
         }
         tc::mma_commit(&sm.mma);
     };
@@ -555,9 +562,9 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             timed_out = true;
     };
     auto run_mma = [&](int sweep) {
-        if (tid == 0) {
+        if ((tid & 31) == 0 && warp < 3) {
             tc::fence_after_sync();
-            issue_mma(sweep);
+            issue_chain(warp, sweep);
         }
         if (!tc::mbar_wait(&sm.mma, mma_phase, kBSpin)) timed_out = true;
         mma_phase ^= 1u;

@@ -74,7 +74,11 @@ struct BCols {
     static constexpr uint32_t WU = 3 * N + 32;  // W or U [16]
     static constexpr uint32_t VV = 3 * N + 48;  // state weights or s dy E [16]
     static constexpr uint32_t DL = 3 * N + 64;  // s dy_t x_t.C_t of the block [64]
-    static constexpr uint32_t USED = 3 * N + 128;
+    // d_state 64 has room to split the dC / dB chain over two accumulators
+    // (second half of the channel sum), shortening the longest MMA chain.
+    static constexpr bool SPLIT = 3 * N + 144 <= 512;
+    static constexpr uint32_t BC2 = 3 * N + 128;
+    static constexpr uint32_t USED = SPLIT ? 3 * N + 144 : 3 * N + 128;
     static constexpr uint32_t ALLOC = 512;
     static_assert(USED <= ALLOC, "tensor memory");
 };
@@ -154,7 +158,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     if (tid == 0) {
         sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
         for (int q = 0; q < Sm::NRAW; ++q) tc::mbar_init(&sm.loaded[q], 1);
-        tc::mbar_init(&sm.mma, 3);  // one arrival per MMA chain
+        tc::mbar_init(&sm.mma, Cols::SPLIT ? 4 : 3);  // one arrival per MMA chain
         tma::prefetch_map(&tm.u);
         tma::prefetch_map(&tm.a);
         if (p.b) tma::prefetch_map(&tm.b);
@@ -522,6 +526,17 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             tc::mbar_arrive(&sm.mma);
             return;
         }
+        if (chain == 3) {  // second half of the dC / dB channel sum into BC2
+            const uint32_t a_st = tc::smem_u32(sm.st), a_pk = tc::smem_u32(sm.pk);
+#pragma unroll
+            for (int i = P / 16; i < P / 8; ++i)
+                tc::mma_tf32_ss(tbase + Cols::BC2,
+                                tc::sdesc_sw128(a_st + (i >> 2) * N * 128 + (i & 3) * 32),
+                                tc::sdesc_sw128(a_pk + (i >> 2) * T * 128 + (i & 3) * 32), id16,
+                                i > P / 16 ? 1u : 0u);
+            tc::mma_commit(&sm.mma);
+            return;
+        }
         if (chain == 0) {
             const uint32_t a_ta = tc::smem_u32(sm.ta), a_tg = tc::smem_u32(sm.tg);
             const uint32_t Acol = sweep == kSweepFwd ? Cols::X : Cols::G;
@@ -542,8 +557,9 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         } else {
             const uint32_t a_ts = tc::smem_u32(sm.ts), a_t2 = tc::smem_u32(sm.ta2);
             const uint32_t a_st = tc::smem_u32(sm.st), a_pk = tc::smem_u32(sm.pk);
+            constexpr int KE = Cols::SPLIT ? P / 16 : P / 8;  // K steps of this chain
 #pragma unroll
-            for (int i = 0; i < P / 8; ++i)
+            for (int i = 0; i < KE; ++i)
                 tc::mma_tf32_ss(tbase + Cols::BC,
                                 tc::sdesc_sw128(a_st + (i >> 2) * N * 128 + (i & 3) * 32),
                                 tc::sdesc_sw128(a_pk + (i >> 2) * T * 128 + (i & 3) * 32), id16,
@@ -562,7 +578,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             timed_out = true;
     };
     auto run_mma = [&](int sweep) {
-        if ((tid & 31) == 0 && warp < 3) {
+        if ((tid & 31) == 0 && warp < (Cols::SPLIT ? 4 : 3)) {
             tc::fence_after_sync();
             issue_chain(warp, sweep);
         }
@@ -576,6 +592,13 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         if ((warp & 3) * 32 < N) {
             float v[TQ];
             tc::tmem_ld4(tbase + lane + Cols::BC + qd * TQ, v);
+            if (Cols::SPLIT) {
+                float v2[TQ];
+                tc::tmem_ld4(tbase + lane + Cols::BC2 + qd * TQ, v2);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int k = 0; k < TQ; ++k) v[k] += v2[k];
+            }
             tc::tmem_ld_wait();
             const int j = ch;  // lane = d_state row
 #pragma unroll

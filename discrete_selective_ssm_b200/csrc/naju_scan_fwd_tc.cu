@@ -25,16 +25,16 @@
 // operands give about 1e-3 relative error on the contractions; the fp32
 // activations path uses the CUDA-core kernel.
 //
-// Warp roles.  Warps 0-7 produce: one thread loads raw sub-chunks with TMA
-// (two ahead, three raw buffers, an mbarrier each) and all 256 unpack each
+// Warp roles.  Warps 0-15 produce: one thread loads raw sub-chunks with TMA
+// (two ahead, three raw buffers, an mbarrier each) and all 512 unpack each
 // sub-chunk into one of three operand stages (shared memory + tensor-memory
-// columns); channel p is handled by threads p and p + 128, each taking 8 of
-// the 16 tokens.  Warps 8-11 consume:
-// thread 256 + p owns channel p; one of them issues the MMAs of a stage, all
-// of them run the epilogue (outputs, X' = E_T X + D_state, checkpoints) and
-// release the stage.  Stages hand over through mbarriers (full: 256 producer
-// arrivals; empty: 128 consumer arrivals; one MMA-completion barrier), so
-// unpacking overlaps the tensor core and the epilogue.
+// columns); channel p is handled by threads p + 128 q, q = 0..3, each taking
+// 4 of the 16 tokens.  Warps 16-19 consume: thread 512 + p owns channel p;
+// one of them issues the MMAs of a stage, all of them run the epilogue
+// (outputs, X' = E_T X + D_state, checkpoints) and release the stage.  Stages
+// hand over through mbarriers (full: 512 producer arrivals; empty: 128
+// consumer arrivals; one MMA-completion barrier), so unpacking overlaps the
+// tensor core and the epilogue.
 //
 // Sequence groups work as in the CUDA-core kernel: an update-only pass and a
 // decoupled look-back publish each group's end state before the full pass.
@@ -101,7 +101,7 @@ struct FwdTcSmem {
     };
     Raw raw[S];
     Stage st[S];
-    float xq0[P], xe0[P], xe1[P];       // per-half decay products of a sub-chunk
+    float xq[4][P], xe[4][P];           // per-quarter decay products of a sub-chunk
     uint64_t loaded[S], full[S], empty[S], mma;
     uint32_t taddr;
     int item, ok;
@@ -110,22 +110,22 @@ struct FwdTcSmem {
 }  // namespace
 
 template <typename Tout, int N, bool CONV>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(640, 1)
 scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
     using Tin = __nv_bfloat16;
     using Cols = TcCols<N>;
     using Sm = FwdTcSmem<N>;
-    constexpr int T = kTS, P = 128, H = T / 2, S = kStages;
-    constexpr int NPROD = 256, NCONS = 128;
+    constexpr int T = kTS, P = 128, TQ = T / 4, S = kStages;
+    constexpr int NPROD = 512, NCONS = 128;
     extern __shared__ __align__(1024) float4 smem4[];
     Sm& sm = *reinterpret_cast<Sm*>(smem4);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const bool prod = tid < NPROD;
-    // Producers: channel pch, token half phalf.  Consumers: channel cch.
+    // Producers: channel pch, token quarter pq.  Consumers: channel cch.
     const int pch = tid & (P - 1);
-    const int phalf = (tid >> 7) & 1;
+    const int pq = (tid >> 7) & 3;
     const int cch = tid - NPROD;
     const int ch = prod ? pch : cch;
     const int64_t Bt = p.Bt, L = p.L, d = p.d;
@@ -224,14 +224,14 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
             *reinterpret_cast<float4*>(&stg.brow[tt][j]) = bf4(&r.Bm[tt][j]);
             if (full) *reinterpret_cast<float4*>(&stg.crow[tt][j]) = bf4(&r.Cm[tt][j]);
         }
-        // Tokens of this thread's half inside [t0, tend) (0 for a padding channel).
-        const int nv = cvalid ? (int)max((int64_t)0, min64((int64_t)H, tend - t0 - phalf * H)) : 0;
-        // Per-channel values: this thread's 8 tokens.
-        float qv[H], fv[H], hv[H], ev[H];
+        // Tokens of this thread's quarter inside [t0, tend) (0 for a padding channel).
+        const int nv = cvalid ? (int)max((int64_t)0, min64((int64_t)TQ, tend - t0 - pq * TQ)) : 0;
+        // Per-channel values: this thread's 4 tokens.
+        float qv[TQ], fv[TQ], hv[TQ], ev[TQ];
         float Qh = 1.f, Eh = 1.f;
 #pragma unroll
-        for (int k = 0; k < H; ++k) {
-            const int tt = phalf * H + k;
+        for (int k = 0; k < TQ; ++k) {
+            const int tt = pq * TQ + k;
             const bool valid = k < nv;
             ev[k] = valid ? __expf(-to_f(r.a[tt][pch])) : 0.f;
             qv[k] = 1.f + ev[k];
@@ -247,15 +247,22 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
             }
             hv[k] = valid ? h : 0.f;
         }
-        if (phalf == 0) {
-            sm.xq0[pch] = Qh;
-            sm.xe0[pch] = Eh;
-        } else {
-            sm.xe1[pch] = Eh;
-        }
+        sm.xq[pq][pch] = Qh;
+        sm.xe[pq][pch] = Eh;
         tc::named_bar(1, NPROD);
-        const float Q0 = sm.xq0[pch], E0 = sm.xe0[pch], E1 = sm.xe1[pch];
-        const bool slow = tc::named_bar_or(1, NPROD, phalf == 1 && !(Q0 * Qh <= kTcBound));
+        // decay products of the earlier quarters and of the whole sub-chunk
+        float Qb = 1.f, Eb = 1.f, Qa = 1.f, Ea = 1.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float xq = sm.xq[q][pch], xe = sm.xe[q][pch];
+            if (q < pq) {
+                Qb *= xq;
+                Eb *= xe;
+            }
+            Qa *= xq;
+            Ea *= xe;
+        }
+        const bool slow = tc::named_bar_or(1, NPROD, pq == 0 && !(Qa <= kTcBound));
         if (!slow) {
             if (full && warp == 0) {
                 // G[t][m] = C_t . B_m for m <= t: one warp, tf32 warp-level MMAs.
@@ -288,12 +295,12 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
                 }
             }
         }
-        const float Elast = E0 * E1;
-        float Q = phalf ? Q0 : 1.f, E = phalf ? E0 : 1.f;
-        float Wv[H], Vv[H], Gv[H], Dv[H];
+        const float Elast = Ea;
+        float Q = Qb, E = Eb;
+        float Wv[TQ], Vv[TQ], Gv[TQ], Dv[TQ];
 #pragma unroll
-        for (int k = 0; k < H; ++k) {
-            const int tt = phalf * H + k;
+        for (int k = 0; k < TQ; ++k) {
+            const int tt = pq * TQ + k;
             const float iw = has_b ? sigmoida_(to_f(r.b[tt][pch])) : ev[k] * fv[k];
             const float v = iw * hv[k];  // 0 past the end (h = 0)
             E *= fv[k];
@@ -311,14 +318,14 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
                 Dv[k] = Dc * hv[k] * gg;
             }
         }
-        if (phalf == 0) stg.elast[pch] = Elast;
+        if (pq == 0) stg.elast[pch] = Elast;
         if (tid == 0) stg.slow = slow ? 1 : 0;
-        const uint32_t col = tbase + lane + s * T + phalf * H;
-        tc::tmem_st8(col + Cols::W, Wv);
-        tc::tmem_st8(col + Cols::V, Vv);
+        const uint32_t col = tbase + lane + s * T + pq * TQ;
+        tc::tmem_st4(col + Cols::W, Wv);
+        tc::tmem_st4(col + Cols::V, Vv);
         if (full) {
-            tc::tmem_st8(col + Cols::EG, Gv);
-            tc::tmem_st8(col + Cols::DH, Dv);
+            tc::tmem_st4(col + Cols::EG, Gv);
+            tc::tmem_st4(col + Cols::DH, Dv);
         }
         tc::tmem_st_wait();
     };
@@ -609,7 +616,7 @@ static cudaError_t launch_fwd_tc_t(const FwdParams& p, cudaStream_t st) {
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = p.ngroups * (int)p.Bt * p.ntiles;
-    kern<<<grid, 384, smem, st>>>(p, tm);
+    kern<<<grid, 640, smem, st>>>(p, tm);
     return cudaGetLastError();
 }
 

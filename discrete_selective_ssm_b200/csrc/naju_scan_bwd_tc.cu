@@ -118,7 +118,7 @@ struct BwdTcSmem {
     alignas(16) float w1[T][P + 4];    // W / U rows (slow path: sums over quarters)
     alignas(16) float brow[T][N + 4];
     alignas(16) float crow[T][N + 4];
-    float dp[T + 3][P];
+    float dp[2][T][P];                 // conv dp of the last two backward sub-chunks
     float acc[T][N];                   // slow path channel sums
     float xq[4][P], xe[4][P], xs[4][P];  // exchanges between a channel's four threads
     uint64_t loaded[3], mma;
@@ -774,7 +774,9 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         __syncthreads();
         tmem_from(Cols::G, sm.ok ? carry_in : nullptr, true);
     }
-    for (int i = tid; i < 3 * P; i += NT) (&sm.dp[T][0])[i] = 0.f;
+    // dp beyond the group: zero (the next group's terms go via the edge fixup)
+    for (int i = tid; i < 3 * P; i += NT) (&sm.dp[1][0][0])[i] = 0.f;
+    int bi = 0;  // backward-sweep items so far (dp buffer bi & 1; the later sub-chunk's in the other)
     sync();
 
     // ====================================================== main: blocks
@@ -828,9 +830,10 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 tc::tmem_st4(trow + Cols::DL + sb * T + qd * TQ, dl);
                 tc::tmem_st_wait();
             }
-            sync();
-            to_st(Cols::X);  // state entering the next sub-chunk
-            sync();
+            // State entering the next sub-chunk: each thread copies its own TMEM
+            // columns (no barrier needed; the next item's MMAs follow its
+            // unpacking barriers).
+            to_st(Cols::X);
         }
         // (f df) tail of this block: carry entering the block's end . state at its end
         const float tail = tmem_dot(Cols::G, Cols::X);
@@ -873,8 +876,29 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 run += dl[q] - iv[q] * hv[q] * gbv[q];
                 sfx[q] = run;
             }
+            // conv dp (needs no suffix sums) into this item's buffer
+            float(*dpc)[P] = sm.dp[bi & 1];
+            const float(*dpl)[P] = sm.dp[(bi & 1) ^ 1];  // the later sub-chunk's (halo)
+            float dhv[TQ];
+#pragma unroll
+            for (int q = 0; q < TQ; ++q) {
+                const int tt = qd * TQ + q;
+                dhv[q] = fmaf(Dc, dyv[q], iv[q] * gbv[q]);
+                if (CONV) {
+                    float dpv = 0.f;
+                    if (q < nvh) {
+                        dpv = dhv[q] * aux[q];
+                        dw0 = fmaf(dpv, to_f(r.u[tt][ch]), dw0);
+                        dw1 = fmaf(dpv, to_f(r.u[tt + 1][ch]), dw1);
+                        dw2 = fmaf(dpv, to_f(r.u[tt + 2][ch]), dw2);
+                        dw3 = fmaf(dpv, to_f(r.u[tt + 3][ch]), dw3);
+                        dbias += dpv;
+                    }
+                    dpc[tt][ch] = dpv;
+                }
+            }
             sm.xs[qd][ch] = run;
-            __syncthreads();
+            __syncthreads();  // suffix partials and dp complete
             float later = 0.f, total = 0.f;  // sums of dL over later quarters / all
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -888,9 +912,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             for (int q = 0; q < TQ; ++q) {
                 const int tt = qd * TQ + q;
                 const int64_t t = t0 + tt;
-                float dpv = 0.f;
                 if (q < nvh) {
-                    const float dh = fmaf(Dc, dyv[q], iv[q] * gbv[q]);
                     if (has_b) {
                         gda[t * d] = from_f<Tout>((base + sfx[q]) * (1.f - fv[q]));
                         gdb[t * d] = from_f<Tout>(hv[q] * gbv[q] * iv[q] * (1.f - iv[q]));
@@ -900,46 +922,27 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                     }
                     dD_acc = fmaf(dyv[q], hv[q], dD_acc);
                     if (CONV) {
-                        dpv = dh * aux[q];
-                        dw0 = fmaf(dpv, to_f(r.u[tt][ch]), dw0);
-                        dw1 = fmaf(dpv, to_f(r.u[tt + 1][ch]), dw1);
-                        dw2 = fmaf(dpv, to_f(r.u[tt + 2][ch]), dw2);
-                        dw3 = fmaf(dpv, to_f(r.u[tt + 3][ch]), dw3);
-                        dbias += dpv;
-                    } else {
-                        gdhu[t * d] = from_f<Tout>(dh);
-                    }
-                }
-                if (CONV) sm.dp[tt][ch] = dpv;
-            }
-            if (CONV) {
-                __syncthreads();
-                // du_t = w3 dp_t + w2 dp_{t+1} + w1 dp_{t+2} + w0 dp_{t+3}
-#pragma unroll
-                for (int q = 0; q < TQ; ++q) {
-                    const int tt = qd * TQ + q;
-                    const int64_t t = t0 + tt;
-                    if (q < nvh) {
-                        const float duv = w3 * sm.dp[tt][ch] + w2 * sm.dp[tt + 1][ch] +
-                                          w1 * sm.dp[tt + 2][ch] + w0 * sm.dp[tt + 3][ch];
+                        // du_t = w3 dp_t + w2 dp_{t+1} + w1 dp_{t+2} + w0 dp_{t+3}
+                        auto dpat = [&](int row) {
+                            return row < T ? dpc[row][ch] : dpl[row - T][ch];
+                        };
+                        const float duv = w3 * dpc[tt][ch] + w2 * dpat(tt + 1) +
+                                          w1 * dpat(tt + 2) + w0 * dpat(tt + 3);
                         if (!lastg && group_end_block && t >= te - 3) {
                             edge[(3 + (t - (te - 3))) * d + c] = duv;  // partial, fixed up later
                         } else {
                             gdhu[t * d] = from_f<Tout>(duv);
                         }
-                        if (k == kb0 && sb == 0 && tt < 3) edge[tt * d + c] = sm.dp[tt][ch];
+                        if (k == kb0 && sb == 0 && tt < 3) edge[tt * d + c] = dpc[tt][ch];
+                    } else {
+                        gdhu[t * d] = from_f<Tout>(dhv[q]);
                     }
                 }
-                __syncthreads();
-                if (qd == 0) {  // first three dp rows -> halo of the earlier sub-chunk
-                    sm.dp[T][ch] = sm.dp[0][ch];
-                    sm.dp[T + 1][ch] = sm.dp[1][ch];
-                    sm.dp[T + 2][ch] = sm.dp[2][ch];
-                }
             }
-            sync();
-            to_st(Cols::G);  // carry entering the earlier sub-chunk's end
-            sync();
+            ++bi;
+            // Carry entering the earlier sub-chunk's end: own TMEM columns, no
+            // barrier needed (see the forward sweep).
+            to_st(Cols::G);
         }
     }
 

@@ -390,7 +390,7 @@ def main():
     ap.add_argument("--workload", default="throughput_train", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--block", action="store_true",
                     help="time the full Naju block (norm, projections, conv, scan, residual) "
                          "with d_model = d_inner / 2 instead of the scan alone")
@@ -449,19 +449,21 @@ def main():
              "dx0": None}
     stream = torch.cuda.current_stream()
 
-    def step(inp, ev=None):
+    def step(inp, ev=None, y_out=None, g_out=None):
+        y_out = y if y_out is None else y_out
+        g_out = grads if g_out is None else g_out
         if ev is not None:
             ev[0].record(stream)
         naju.scan_fwd(inp["u"], inp["a"], None if args.coupled else inp["b"], inp["B"], inp["C"],
                       conv_w=inp["conv_w"],
                       conv_b=inp["conv_b"], z=inp["z"], D=inp["D"], out_dtype=out_dt,
-                      workspace=ws, want_final=False, y=y)
+                      workspace=ws, want_final=False, y=y_out)
         if ev is not None:
             ev[1].record(stream)
         naju.scan_bwd(inp["dout"], inp["u"], inp["a"], None if args.coupled else inp["b"],
                       inp["B"], inp["C"], ws,
                       conv_w=inp["conv_w"], conv_b=inp["conv_b"], z=inp["z"], D=inp["D"],
-                      out_dtype=out_dt, grads=grads)
+                      out_dtype=out_dt, grads=g_out)
         if ev is not None:
             ev[2].record(stream)
 
@@ -507,31 +509,56 @@ def main():
     value = world * tokens / (ms_step / 1e3)
 
     # -------------------------------------------------------------- e2e leg
+    # Every step copies its inputs host -> device (pinned) and all its outputs
+    # device -> host inside the timed region.  Copies run on their own streams
+    # with double-buffered device inputs and outputs, so step i's compute
+    # overlaps step i+1's upload and step i-1's download (separate copy
+    # engines); the timed region spans the first upload to the last download.
     pinned = {k: v.pin_memory() for k, v in t_host.items()}
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-    outs = [y] + [v for v in grads.values() if v is not None]
-    host_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-    d2h = sum(o.numel() * o.element_size() for o in outs)
-    dev_in = {k: torch.empty_like(v) for k, v in t.items()}
+    dev_in = [{k: torch.empty_like(v) for k, v in t.items()} for _ in range(2)]
+    y2 = [y, torch.empty_like(y)]
+    g2 = [grads, {k: (torch.empty_like(v) if v is not None else None) for k, v in grads.items()}]
+    outs2 = [[y2[i]] + [v for v in g2[i].values() if v is not None] for i in range(2)]
+    host_outs = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs2[i]]
+                 for i in range(2)]
+    d2h = sum(o.numel() * o.element_size() for o in outs2[0])
+    s_up, s_down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    n_e2e = max(args.e2e_steps, 1)
 
-    def e2e_step():
-        for k, v in pinned.items():
-            dev_in[k].copy_(v, non_blocking=True)
-        step(dev_in)
-        for ho, o in zip(host_outs, outs):
-            ho.copy_(o, non_blocking=True)
+    def e2e_run(n):
+        up_done = [torch.cuda.Event() for _ in range(n)]
+        comp_done = [torch.cuda.Event() for _ in range(n)]
+        down_done = [torch.cuda.Event() for _ in range(n)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s_up)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_up):
+                if i >= 2:
+                    s_up.wait_event(comp_done[i - 2])  # inputs buffer b free again
+                for k, v in pinned.items():
+                    dev_in[b][k].copy_(v, non_blocking=True)
+                up_done[i].record(s_up)
+            stream.wait_event(up_done[i])
+            if i >= 2:
+                stream.wait_event(down_done[i - 2])  # outputs buffer b copied out
+            step(dev_in[b], y_out=y2[b], g_out=g2[b])
+            comp_done[i].record(stream)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(comp_done[i])
+                for ho, o in zip(host_outs[b], outs2[b]):
+                    ho.copy_(o, non_blocking=True)
+                down_done[i].record(s_down)
+        stream.wait_event(down_done[n - 1])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / n
 
-    e2e_step()
-    torch.cuda.synchronize()
+    e2e_run(2)
     if dist is not None:
         dist.barrier()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e2.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = s2.elapsed_time(e2) / args.e2e_steps
+    e2e_ms = e2e_run(n_e2e)
     if dist is not None:
         tt = torch.tensor([e2e_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)

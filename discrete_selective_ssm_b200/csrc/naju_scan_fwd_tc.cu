@@ -25,11 +25,12 @@
 // operands give about 1e-3 relative error on the contractions; the fp32
 // activations path uses the CUDA-core kernel.
 //
-// Warp roles.  Warps 0-15 produce: one thread loads raw sub-chunks with TMA
-// (two ahead, three raw buffers, an mbarrier each) and all 512 unpack each
-// sub-chunk into one of three operand stages (shared memory + tensor-memory
-// columns); channel p is handled by threads p + 128 q, q = 0..3, each taking
-// 4 of the 16 tokens.  Warps 16-19 consume: thread 512 + p owns channel p;
+// Warp roles.  Warps 0-15 produce: one thread issues TMA loads of raw
+// sub-chunks two ahead into three buffers (an mbarrier each), refilling a
+// buffer once every producer has unpacked it (its stage's full barrier), and
+// all 512 unpack each sub-chunk into one of three operand stages (shared
+// memory + tensor-memory columns); channel p is handled by threads p + 128 q,
+// q = 0..3, each taking 4 of the 16 tokens.  Warps 16-19 consume: thread 512 + p owns channel p;
 // one of them issues the MMAs of a stage, all of them run the epilogue
 // (outputs, X' = E_T X + D_state, checkpoints) and release the stage.  Stages
 // hand over through mbarriers (full: 512 producer arrivals; empty: 128
@@ -123,6 +124,7 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const bool prod = tid < NPROD;
+    const bool cons = !prod;
     // Producers: channel pch, token quarter pq.  Consumers: channel cch.
     const int pch = tid & (P - 1);
     const int pq = (tid >> 7) & 3;
@@ -473,15 +475,20 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
             for (int i = 0; i < nsc; ++i) {
                 const int gi = gbase + i, s = gi % S, u = gi / S;
                 const int64_t t0 = tbeg + (int64_t)i * T;
-                // Buffer (gi + 2) % S was last read in the previous iteration.
-                if (tid == 0 && i + 2 < nsc) issue(t0 + 2 * T, (gi + 2) % S, full);
+                if (tid == 0 && i + 2 < nsc) {
+                    // Buffer (gi + 2) % S held sub-chunk gi - 1: refill it once
+                    // every producer has unpacked that one (its full barrier).
+                    if (i > 0 && !tc::mbar_wait(&sm.full[(gi - 1) % S], ((gi - 1) / S) & 1,
+                                                kMbarSpin))
+                        timed_out = true;
+                    issue(t0 + 2 * T, (gi + 2) % S, full);
+                }
                 if (!tc::mbar_wait(&sm.loaded[s], u & 1, kMbarSpin)) timed_out = true;
                 if (u > 0 && !tc::mbar_wait(&sm.empty[s], (u - 1) & 1, kMbarSpin)) timed_out = true;
                 prep(t0, s, s, full);
                 tc::fence_proxy_async();
                 tc::fence_before_sync();
                 tc::mbar_arrive(&sm.full[s]);
-                tc::named_bar(1, NPROD);  // raw sub-chunk i consumed by every producer
             }
         } else {
             for (int i = 0; i < nsc; ++i) {
@@ -536,14 +543,14 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
         tc::fence_after_sync();
     };
     if (!last_group) {
-        if (!prod) state_from(g == 0 ? x0b : nullptr, false);
+        if (cons) state_from(g == 0 ? x0b : nullptr, false);
         sync_all();
         run_pass(false);
         if (g > 0) {
             if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
             __syncthreads();
             ok = sm.ok != 0;
-            if (!prod) {
+            if (cons) {
                 // X_end += (product of f over the group) X_start
                 const float Pf = __expf(logP);
 #pragma unroll
@@ -566,7 +573,7 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
                 tc::tmem_st_wait();
             }
         }
-        if (!prod) state_to(ck_end);
+        if (cons) state_to(ck_end);
         __threadfence();
         __syncthreads();
         if (tid == 0 && !(g == 0 && p.fault_skip_publish)) st_release(flag_mine, 1);
@@ -575,7 +582,7 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
         __syncthreads();
         ok = sm.ok != 0;
     }
-    if (!prod) {
+    if (cons) {
         if (g > 0) {
             state_from(ok ? ck_start : nullptr, true);
         } else {
@@ -587,7 +594,7 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
 
     // ------------------------------------------------------- full pass
     run_pass(true);
-    if (last_group && !prod) {
+    if (last_group && cons) {
         state_to(ck_b + (int64_t)p.nck * d * N);
         if (p.x_final) state_to(p.x_final + (int64_t)bb * d * N);
     }

@@ -28,6 +28,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from discrete_selective_ssm_b200.parallel import max_over_ranks  # noqa: E402
 from discrete_selective_ssm_b200.workloads import (WORKLOADS, decode_D, decode_state0,  # noqa: E402
                                                    decode_step_inputs, make_inputs, scaled)
 
@@ -249,9 +250,7 @@ def run_decode(args, w, rank, world, local):
     clocks = clk.stop()
     ms_total = e0.elapsed_time(e1)
     if dist is not None:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+        ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
     value = world * w.batch / (ms_step / 1e3)
 
@@ -278,9 +277,7 @@ def run_decode(args, w, rank, world, local):
     torch.cuda.synchronize()
     e2e_ms = s2.elapsed_time(t2) / args.steps
     if dist is not None:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e2e_ms, dev)
 
     pk, pk_kind = peaks()
     E = 2 if w.dtype == "bf16" else 4
@@ -359,9 +356,7 @@ def run_block(args, w, rank, world, local):
     clocks = clk.stop()
     ms = e0.elapsed_time(e1) / args.steps
     if dist is not None:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, dev)
     di, N = w.d_inner, w.d_state
     gemm_flop = 2 * w.batch * w.seqlen * (dm * 2 * di + 2 * di * di + 2 * di * N + di * dm) * 3
     if rank == 0:
@@ -501,9 +496,7 @@ def main():
     if naju.last_device_status(ws) != 0:
         raise SystemExit("device status not OK after the timed region")
     if dist is not None:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+        ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
     tokens = w.batch * w.seqlen
     value = world * tokens / (ms_step / 1e3)
@@ -560,9 +553,7 @@ def main():
         dist.barrier()
     e2e_ms = e2e_run(n_e2e)
     if dist is not None:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(e2e_ms, dev)
     e2e_val = world * tokens / (e2e_ms / 1e3)
 
     # ---------------------------------------------------------------- roofline

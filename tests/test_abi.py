@@ -88,3 +88,32 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         _native._ptr(torch.zeros(4), "x")
+
+
+def test_empty_and_oversized_dims_are_rejected(L):
+    """Empty inputs (batch, length or width 0) and sizes past the documented
+    limits are rejected on the host before any launch."""
+    null = None
+    for dims in (naju.make_dims(0, 8, 8, 16, naju.F32), naju.make_dims(1, 0, 8, 16, naju.F32),
+                 naju.make_dims(1, 8, 0, 16, naju.F32),
+                 naju.make_dims(1 << 21, 8, 8, 16, naju.F32),
+                 naju.make_dims(1, 1 << 27, 8, 16, naju.F32),
+                 naju.make_dims(1 << 20, 1 << 12, 1 << 10, 16, naju.F32)):
+        assert naju.workspace_bytes(dims) == 0
+        assert L.naju_scan_fwd(ctypes.byref(dims), *([null] * 13), 0, null) == 1
+        assert L.naju_scan_bwd(ctypes.byref(dims), *([null] * 23), 0, null) == 1
+    assert L.naju_scan_step(0, 8, 16, 0, *([null] * 10)) == 1
+    assert L.naju_scan_step_conv(0, 8, 16, 0, *([null] * 13)) == 1
+    assert L.naju_conv_silu_step(0, 8, 0, *([null] * 6)) == 1
+
+
+def test_tensor_core_dispatch_rules(L):
+    """Tensor-core kernels for bf16 with d_state 64/128 and d_inner % 8 == 0;
+    CUDA-core kernels otherwise (fp32, d_state 16/32, other widths)."""
+    assert naju.testing_fwd_impl(naju.make_dims(2, 64, 256, 64, naju.BF16)) == 2
+    assert naju.testing_bwd_impl(naju.make_dims(2, 64, 256, 128, naju.BF16)) == 2
+    assert naju.testing_fwd_impl(naju.make_dims(2, 64, 264, 64, naju.BF16)) == 2
+    assert naju.testing_fwd_impl(naju.make_dims(2, 64, 258, 64, naju.BF16)) == 1
+    assert naju.testing_bwd_impl(naju.make_dims(2, 64, 258, 64, naju.BF16)) == 1
+    assert naju.testing_fwd_impl(naju.make_dims(2, 64, 256, 32, naju.BF16)) == 1
+    assert naju.testing_bwd_impl(naju.make_dims(2, 64, 256, 64, naju.F32)) == 1

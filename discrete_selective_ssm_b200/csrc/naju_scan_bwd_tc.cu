@@ -78,7 +78,12 @@ struct BCols {
     // (second half of the channel sum), shortening the longest MMA chain.
     static constexpr bool SPLIT = 3 * N + 144 <= 512;
     static constexpr uint32_t BC2 = 3 * N + 128;
-    static constexpr uint32_t USED = SPLIT ? 3 * N + 144 : 3 * N + 128;
+    // d_state 64 also has room to keep h and SiLU'(conv pre-activation) of the
+    // block's 64 tokens from the forward sweep for the backward sweep.
+    static constexpr bool GCACHE = 3 * N + 272 <= 512;
+    static constexpr uint32_t GH = 3 * N + 144;   // h [64]
+    static constexpr uint32_t GA = 3 * N + 208;   // SiLU'(pre) [64]
+    static constexpr uint32_t USED = GCACHE ? 3 * N + 272 : SPLIT ? 3 * N + 144 : 3 * N + 128;
     static constexpr uint32_t ALLOC = 512;
     static_assert(USED <= ALLOC, "tensor memory");
 };
@@ -124,6 +129,7 @@ struct BwdTcSmem {
     uint64_t loaded[3], mma;
     uint32_t taddr;
     int item, ok;
+    int slowf[4];                      // exact-path decision of the block's sub-chunks
 };
 
 enum { kSweepFwd = 0, kSweepBwd = 1, kSweepEarly = 2 };
@@ -355,9 +361,19 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     // Unpack item `li` (raw buffer li % NRAW) for a sweep; fills the registers
     // above, the TMEM operand columns and the per-token tiles.  Returns after
     // a block-wide barrier.
-    auto prep = [&](int64_t t0, int64_t te, int sweep) {
+    // sb: the sub-chunk's index in its 64-token block (main phase).  The
+    // backward sweep reuses the forward sweep's decision and, with GCACHE and
+    // the fused conv, its h and SiLU'(pre).
+    auto prep = [&](int64_t t0, int64_t te, int sweep, int sb) {
         const typename Sm::Raw& r = sm.raw[li % Sm::NRAW];
         const bool fwd = sweep == kSweepFwd;
+        constexpr bool CACHE = CONV && Cols::GCACHE;
+        float hc[TQ], ac[TQ];
+        if (CACHE && sweep == kSweepBwd) {
+            tc::tmem_ld4(trow + Cols::GH + sb * T + qd * TQ, hc);
+            tc::tmem_ld4(trow + Cols::GA + sb * T + qd * TQ, ac);
+            tc::tmem_ld_wait();
+        }
         // B and C rows to fp32.
         for (int e = tid; e < T * N / 4; e += NT) {
             const int tt = e / (N / 4), j = (e % (N / 4)) * 4;
@@ -376,12 +392,19 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             Qh *= qv[k];
             Eh *= fv[k];
             float hh, ax = 0.f;
-            if (CONV) {
+            if (CACHE && sweep == kSweepBwd) {
+                hh = hc[k];
+                ax = ac[k];
+            } else if (CONV) {
                 const float pp = wb + w0 * to_f(r.u[tt][ch]) + w1 * to_f(r.u[tt + 1][ch]) +
                                  w2 * to_f(r.u[tt + 2][ch]) + w3 * to_f(r.u[tt + 3][ch]);
                 const float sp = sigmoida_(pp);
                 hh = pp * sp;
                 ax = sp * fmaf(pp, 1.f - sp, 1.f);
+                if (CACHE && fwd) {
+                    hc[k] = valid ? hh : 0.f;
+                    ac[k] = ax;
+                }
             } else {
                 hh = to_f(r.u[tt + 3][ch]);
             }
@@ -396,6 +419,10 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             }
             aux[k] = ax;
             dyv[k] = valid ? to_f(r.dy[tt][ch]) * gg : 0.f;
+        }
+        if (CACHE && fwd) {
+            tc::tmem_st4(trow + Cols::GH + sb * T + qd * TQ, hc);
+            tc::tmem_st4(trow + Cols::GA + sb * T + qd * TQ, ac);
         }
         sm.xq[qd][ch] = Qh;
         sm.xe[qd][ch] = Eh;
@@ -413,7 +440,12 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 Qa *= xq;
                 Ea *= xe;
             }
-            slow = __syncthreads_or(qd == 0 && !(Qa <= kBBound)) != 0;
+            if (sweep == kSweepBwd) {
+                slow = sm.slowf[sb] != 0;  // same sub-chunk as the forward sweep's
+            } else {
+                slow = __syncthreads_or(qd == 0 && !(Qa <= kBBound)) != 0;
+                if (fwd && tid == 0) sm.slowf[sb] = slow ? 1 : 0;
+            }
             Elast = Ea;
             float Q = Qb, E = Eb;
 #pragma unroll
@@ -724,7 +756,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         for (int e = 0; e < nE; ++e, ++li) {
             const int64_t t0 = item_t0(li);
             begin_item();
-            prep(t0, tg1, kSweepEarly);
+            prep(t0, tg1, kSweepEarly, 0);
             if (!slow) {
                 run_mma(kSweepEarly);
                 tmem_axpy(Cols::G, Elast, Cols::D);
@@ -795,7 +827,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         for (int sb = 0; sb < nsb; ++sb, ++li) {
             const int64_t t0 = tb + (int64_t)sb * T;
             begin_item();
-            prep(t0, te, kSweepFwd);
+            prep(t0, te, kSweepFwd, sb);
             float yd[TQ];  // x_t . C_t of this thread's tokens
             if (!slow) {
                 run_mma(kSweepFwd);
@@ -845,7 +877,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         for (int sb = nsb - 1; sb >= 0; --sb, ++li) {
             const int64_t t0 = tb + (int64_t)sb * T;
             begin_item();
-            prep(t0, te, kSweepBwd);
+            prep(t0, te, kSweepBwd, sb);
             float gbv[TQ];
             if (!slow) {
                 run_mma(kSweepBwd);

@@ -88,6 +88,9 @@ def lib(build_if_missing: bool = True):
             L.naju_testing_bwd_impl.restype = i32
             L.naju_testing_bwd_groups.argtypes = [vp]
             L.naju_testing_bwd_groups.restype = i32
+            L.naju_testing_set_bwd_pieces.argtypes = [i32]
+            L.naju_testing_bwd_pieces.argtypes = [vp]
+            L.naju_testing_bwd_pieces.restype = i32
             for name in ("naju_conv_silu_fwd", "naju_conv_silu_bwd", "naju_scan_fwd",
                          "naju_scan_bwd", "naju_scan_step", "naju_conv_silu_step",
                          "naju_scan_step_conv", "naju_last_device_status"):
@@ -341,3 +344,11 @@ def testing_set_bwd_groups(groups: int):
 
 def testing_bwd_groups(dims: Dims) -> int:
     return int(lib().naju_testing_bwd_groups(ctypes.byref(dims)))
+
+
+def testing_set_bwd_pieces(pieces: int):
+    lib().naju_testing_set_bwd_pieces(int(pieces))
+
+
+def testing_bwd_pieces(dims: Dims) -> int:
+    return int(lib().naju_testing_bwd_pieces(ctypes.byref(dims)))

@@ -23,6 +23,7 @@ long long g_wait_limit = kDefaultWait;
 int g_skip_publish = 0;
 int g_fwd_groups = 0;
 int g_bwd_groups = 0;
+int g_bwd_pieces = 0;  // 0 automatic, < 0 never, > 0 that many ranges
 int g_fwd_impl = 0;  // 0 automatic, 1 CUDA cores, 2 tensor cores
 int g_bwd_impl = 0;  // 0 automatic, 1 CUDA cores
 
@@ -51,7 +52,7 @@ naju_status check_dims(const naju_dims* dm) {
 struct Layout {
     bool fwd_tc, bwd_tc;
     int nck, ngroups, seg_per_group, ntiles_f;
-    int nsub, nclus, ntiles_b, bgroups, blk_per_group;
+    int nsub, nclus, ntiles_b, bgroups, blk_per_group, npieces;
     size_t off_fflags, off_bflags, off_ckpt, off_carry, off_dbc, off_chan, off_edge, total;
 };
 
@@ -66,7 +67,7 @@ bool use_bwd_tc(const naju_dims* dm) {
 
 // Backward tiling: channel tiles, dB/dC partial sets, sequence groups.
 struct BwdTiling {
-    int ntiles, nparts, bgroups, blk_per_group;
+    int ntiles, nparts, bgroups, blk_per_group, npieces;
 };
 BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
     BwdTiling b{};
@@ -81,6 +82,25 @@ BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
         const int tiles = (int)cdiv(d, bwd_channels_per_block(dm->d_state));
         b.nparts = (int)cdiv(tiles, bwd_cluster_size());
         b.ntiles = b.nparts * bwd_cluster_size();
+    }
+    // Tensor-core piece mode: with at least one unit (128 channels of one
+    // batch element) per SM but not a whole number of waves, cut the units'
+    // blocks into one equal range per SM instead of leaving the last wave
+    // part-empty.  Sequence groups are not used then (two carry slots).
+    if (tc && g_bwd_groups <= 0 && g_bwd_pieces >= 0 && nsub >= 2) {
+        const int64_t units = dm->batch * (int64_t)b.ntiles;
+        int np = 0;
+        if (g_bwd_pieces > 0) {
+            np = units >= g_bwd_pieces ? g_bwd_pieces : 0;
+        } else if (units >= kSMs && units % kSMs != 0) {
+            np = kSMs;
+        }
+        if (np > 0) {
+            b.npieces = np;
+            b.bgroups = 2;
+            b.blk_per_group = nsub;
+            return b;
+        }
     }
     int gb = g_bwd_groups;
     if (gb <= 0) {
@@ -121,6 +141,7 @@ Layout layout(const naju_dims* dm) {
     l.nclus = bt.nparts;
     l.bgroups = bt.bgroups;
     l.blk_per_group = bt.blk_per_group;
+    l.npieces = bt.npieces;
     // Regions sized for the larger of the two backward tilings, so the
     // workspace size does not depend on which backward kernel runs.
     const BwdTiling bo = bwd_tiling(dm, l.nsub, !l.bwd_tc);
@@ -274,7 +295,7 @@ naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* co
     p.hdr = hdr;
     p.Bt = dims->batch; p.L = dims->seqlen; p.d = dims->d_inner; p.N = dims->d_state;
     p.T_ck = kTck; p.nck = l.nck; p.nsub = l.nsub; p.ntiles = l.ntiles_b; p.nclus = l.nclus;
-    p.blk_per_group = l.blk_per_group; p.ngroups = l.bgroups;
+    p.blk_per_group = l.blk_per_group; p.ngroups = l.bgroups; p.npieces = l.npieces;
     p.scale = 1.0f / std::sqrt((float)dims->d_state);
     p.wait_limit = g_wait_limit;
     p.fault_skip_publish = g_skip_publish;
@@ -360,6 +381,12 @@ void naju_testing_set_wait_limit(int64_t polls) {
 void naju_testing_set_skip_publish(int32_t skip) { g_skip_publish = skip ? 1 : 0; }
 void naju_testing_set_fwd_groups(int32_t groups) { g_fwd_groups = groups > 0 ? groups : 0; }
 void naju_testing_set_bwd_groups(int32_t groups) { g_bwd_groups = groups > 0 ? groups : 0; }
+void naju_testing_set_bwd_pieces(int32_t pieces) { g_bwd_pieces = pieces; }
+int32_t naju_testing_bwd_pieces(const void* dims) {
+    const naju_dims* dm = static_cast<const naju_dims*>(dims);
+    if (check_dims(dm) != NAJU_OK) return 0;
+    return layout(dm).npieces;
+}
 void naju_testing_set_fwd_impl(int32_t impl) { g_fwd_impl = (impl == 1) ? 1 : 0; }
 void naju_testing_set_bwd_impl(int32_t impl) { g_bwd_impl = (impl == 1) ? 1 : 0; }
 int32_t naju_testing_bwd_impl(const void* dims) {

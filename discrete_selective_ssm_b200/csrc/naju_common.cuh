@@ -9,6 +9,7 @@
 namespace naju {
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 
 // ----------------------------------------------------------------- dtypes
 __device__ __forceinline__ float to_f(float v) { return v; }

@@ -69,6 +69,7 @@ struct BwdParams {
     int ngroups;
     int ntiles;
     int nclus;             // ceil(ntiles / cluster size)
+    int npieces;           // tensor-core kernel: > 0 for piece mode (ngroups == 2)
     float scale;
     long long wait_limit;
     int fault_skip_publish;

@@ -712,6 +712,42 @@ __global__ void reduce_chan_kernel(const float* __restrict__ part, int64_t rows,
     if (dbias) dbias[c] = acc[5];
 }
 
+// Piece mode of the tensor-core backward: the same fixup at the cut of each
+// cut unit (128 channels of one batch element).  The units' blocks, laid end
+// to end (Wb in all), are cut at k Wb / npieces; unit u holds blocks
+// [u nsub, (u + 1) nsub) and at most one cut.  Head edges are group slot 0,
+// tail edges slot 1.
+template <typename Tout>
+__global__ void conv_edge_pieces_kernel(const float* __restrict__ edge,
+                                        const float* __restrict__ w, int64_t Bt, int ntiles,
+                                        int nsub, int npieces, int64_t L, int64_t d,
+                                        Tout* __restrict__ du) {
+    const int64_t n = Bt * 3 * d;
+    const int64_t Wb = Bt * ntiles * (int64_t)nsub;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t c = i % d;
+        const int r = (int)((i / d) % 3);
+        const int64_t bb = i / (3 * d);
+        const int64_t x = (bb * ntiles + c / 128) * nsub;  // the unit's first block
+        // first cut after x: smallest k with k Wb / npieces > x
+        const int64_t k = ((x + 1) * npieces + Wb - 1) / Wb;
+        if (k >= npieces) continue;
+        const int64_t cut = k * Wb / npieces;
+        if (cut >= x + nsub) continue;  // uncut unit
+        const int64_t tend = (cut - x) * kBwdSub;
+        const int64_t t = tend - 3 + r;
+        const float* mine = edge + ((bb * 2 + 0) * 2 + 1) * 3 * d;
+        const float* next = edge + ((bb * 2 + 1) * 2 + 0) * 3 * d;
+        float v = mine[r * d + c];
+        for (int kk = 0; kk < 4; ++kk) {
+            const int64_t ts = t + 3 - kk - tend;
+            if (ts >= 0 && ts < 3) v += w[c * 4 + kk] * next[ts * d + c];
+        }
+        du[(bb * L + t) * d + c] = from_f<Tout>(v);
+    }
+}
+
 // du of the last three tokens of each non-final sequence group: the group's
 // own partial plus the terms from the first three dp of the next group.
 template <typename Tout>
@@ -750,7 +786,11 @@ static cudaError_t reductions_t(const BwdParams& p, void* dB, void* dC, float* d
                                                   static_cast<Tout*>(dB), static_cast<Tout*>(dC));
     reduce_chan_kernel<<<(unsigned)((p.d + 127) / 128), 128, 0, st>>>(
         p.chan_part, p.Bt * p.ngroups, p.d, dD, conv ? dw : nullptr, conv ? dbias : nullptr);
-    if (conv && p.ngroups > 1)
+    if (conv && p.npieces > 0)
+        conv_edge_pieces_kernel<Tout><<<296, 256, 0, st>>>(p.conv_edge, p.conv_w, p.Bt, p.ntiles,
+                                                            p.nsub, p.npieces, p.L, p.d,
+                                                            static_cast<Tout*>(p.dhu));
+    else if (conv && p.ngroups > 1)
         conv_edge_kernel<Tout><<<296, 256, 0, st>>>(p.conv_edge, p.conv_w, p.Bt, p.ngroups,
                                                      (int64_t)p.blk_per_group * kBwdSub, p.L,
                                                      p.d, static_cast<Tout*>(p.dhu));

@@ -117,8 +117,11 @@ struct BwdTcSmem {
     Raw raw[NRAW];
     alignas(128) float ta[T * N];      // C (forward) / B (backward) rows t, K = d_state
     alignas(128) float ts[TS_FLOATS];  // B^T (forward) / C^T (backward): rows d_state, K = 16
-    alignas(128) float tg[T * T];      // G[t][m] (forward) / G^T (backward)
-    alignas(128) float ta2[T * T];     // A_C (forward) / A_B (backward)
+    // G[t][m] (forward) / G^T (backward) and A_C (forward) / A_B (backward),
+    // each as two partial sums over halves of the contraction (two warps each;
+    // the MMAs accumulate both halves).
+    alignas(128) float tg[2][T * T];
+    alignas(128) float ta2[2][T * T];
     alignas(16) float y1[T][P + 4];    // Y / P rows (slow path: s dy or v)
     alignas(16) float w1[T][P + 4];    // W / U rows (slow path: sums over quarters)
     alignas(16) float brow[T][N + 4];
@@ -136,7 +139,7 @@ enum { kSweepFwd = 0, kSweepBwd = 1, kSweepEarly = 2 };
 
 }  // namespace
 
-template <typename Tout, int N, bool CONV>
+template <typename Tout, int N, bool CONV, bool PIECES>
 __global__ void __launch_bounds__(512, 1)
 scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     using Tin = __nv_bfloat16;
@@ -164,7 +167,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     if (tid == 0) {
         sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
         for (int q = 0; q < Sm::NRAW; ++q) tc::mbar_init(&sm.loaded[q], 1);
-        tc::mbar_init(&sm.mma, Cols::SPLIT ? 4 : 3);  // one arrival per MMA chain
+        tc::mbar_init(&sm.mma, 3);  // three committing (or arriving) lanes per item
         tma::prefetch_map(&tm.u);
         tma::prefetch_map(&tm.a);
         if (p.b) tma::prefetch_map(&tm.b);
@@ -180,60 +183,122 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t trow = tbase + lane;  // this thread's TMEM row (channel)
     const int item = sm.item;
-    const int per_g = (int)(Bt * p.ntiles);
-    const int g = p.ngroups - 1 - item / per_g;
-    const int bb = (item % per_g) / p.ntiles;
-    const int tile = item % p.ntiles;
-    const int64_t c0 = (int64_t)tile * P;
-    const int64_t c = c0 + ch;
-    const bool cvalid = c < d;
-    const int kb0 = g * p.blk_per_group;
-    const int kb1 = min(kb0 + p.blk_per_group, p.nsub);
-    const int64_t tg0 = (int64_t)kb0 * K;
-    const int64_t tg1 = min64(L, (int64_t)kb1 * K);
-    const bool lastg = (g == p.ngroups - 1);
-    const bool firstg = (g == 0);
-
+    // Work unit u = bb * ntiles + tile: 128 channels of one batch element.
+    // Group mode: one (sequence group, unit) per block.  Piece mode: the
+    // units' 64-token blocks, laid end to end, are cut into npieces equal
+    // ranges; a block walks its range in order, so a unit cut in two has its
+    // later part (tail) at the start of one range and its earlier part (head)
+    // at the end of the previous range, and the tail's adjoint carry reaches
+    // the head through the workspace (slot g = 0; head g = 0, tail g = 1).
+    // Group mode is its own instantiation (no per-unit state to carry: it
+    // keeps the register budget); the piece instantiation still reads the
+    // mode at run time, which measured faster than folding it.
+    const bool pieces = PIECES ? p.npieces > 0 : false;
+    int g = 0, bb = 0, tile = 0, kb0 = 0, kb1 = 0;
+    int64_t c0 = 0, c = 0, tg0 = 0, tg1 = 0;
+    bool cvalid = false, lastg = true, firstg = true;
     float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, wb = 0.f, Dc = 0.f;
-    if (cvalid) {
-        if (CONV) {
-            w0 = p.conv_w[c * 4 + 0];
-            w1 = p.conv_w[c * 4 + 1];
-            w2 = p.conv_w[c * 4 + 2];
-            w3 = p.conv_w[c * 4 + 3];
-            wb = p.conv_b ? p.conv_b[c] : 0.f;
+    int64_t goff = 0;  // (bb L) d + c: this thread's channel in the [Bt][L][d] outputs
+    auto set_unit = [&](int u, int g_, int k0, int k1) {
+        g = g_;
+        bb = u / p.ntiles;
+        tile = u % p.ntiles;
+        c0 = (int64_t)tile * P;
+        c = c0 + ch;
+        cvalid = c < d;
+        kb0 = k0;
+        kb1 = k1;
+        tg0 = (int64_t)kb0 * K;
+        tg1 = min64(L, (int64_t)kb1 * K);
+        lastg = kb1 == p.nsub;
+        firstg = kb0 == 0;
+        w0 = w1 = w2 = w3 = wb = Dc = 0.f;
+        if (cvalid) {
+            if (CONV) {
+                w0 = p.conv_w[c * 4 + 0];
+                w1 = p.conv_w[c * 4 + 1];
+                w2 = p.conv_w[c * 4 + 2];
+                w3 = p.conv_w[c * 4 + 3];
+                wb = p.conv_b ? p.conv_b[c] : 0.f;
+            }
+            Dc = p.D ? p.D[c] : 0.f;
         }
-        Dc = p.D ? p.D[c] : 0.f;
-    }
-    const int64_t boff = (int64_t)bb * L;
-    Tout* gdhu = static_cast<Tout*>(p.dhu) + boff * d + c;
-    Tout* gda = static_cast<Tout*>(p.da) + boff * d + c;
-    Tout* gdb = p.db ? static_cast<Tout*>(p.db) + boff * d + c : nullptr;
-    Tout* gdz = has_z ? static_cast<Tout*>(p.dz) + boff * d + c : nullptr;
-    float* part = p.dBCp + (((int64_t)tile * Bt + bb) * L) * 2 * N;  // [L][2][N]
-    float* edge = p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d;
+        goff = (int64_t)bb * L * d + c;
+    };
+    // Per-unit output rows, formed where used (fewer live registers).
+    auto gout = [&](void* base) { return static_cast<Tout*>(base) + goff; };
+    auto part_row = [&]() {  // [L][2][N] dB / dC partials of this tile
+        return p.dBCp + (((int64_t)tile * Bt + bb) * L) * 2 * N;
+    };
+    auto edge_row = [&]() { return p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d; };
     bool timed_out = false;
 
     // ------------------------------------------------ the item sequence
-    // Early pass (groups with a predecessor): the group's sub-chunks, last
-    // first.  Main: blocks last first; per block the forward sweep's
-    // sub-chunks in order, then the backward sweep's in reverse.
-    const int nE = firstg ? 0 : (int)((tg1 - tg0 + T - 1) / T);
-    const int64_t te_first = min64(L, (int64_t)kb1 * K);
-    const int nsb0 = (int)((te_first - (int64_t)(kb1 - 1) * K + T - 1) / T);
-    const int nitems = nE + 2 * nsb0 + 8 * (kb1 - 1 - kb0);
-    auto item_t0 = [&](int li) -> int64_t {
-        if (li < nE) return tg0 + (int64_t)(nE - 1 - li) * T;
-        int j = li - nE;
-        int k = kb1 - 1, nsb = nsb0;
-        if (j >= 2 * nsb0) {
-            j -= 2 * nsb0;
-            k = kb1 - 2 - j / 8;
+    // Per unit segment [k0, k1) of blocks: blocks last first; per block the
+    // forward sweep's sub-chunks in order, then the backward sweep's in
+    // reverse.  Group mode puts an early pass (the group's sub-chunks, last
+    // first) in front when the group has a predecessor.
+    const int nsbL = (int)((L - (int64_t)(p.nsub - 1) * K + T - 1) / T);  // last block's
+    auto seg_items = [&](int k0, int k1) {
+        return 2 * (4 * (k1 - k0) - (k1 == p.nsub ? 4 - nsbL : 0));
+    };
+    auto seg_t0 = [&](int j, int k0, int k1) -> int64_t {
+        int k = k1 - 1, nsb = k1 == p.nsub ? nsbL : 4;
+        if (j >= 2 * nsb) {
+            j -= 2 * nsb;
+            k = k1 - 2 - j / 8;
             j %= 8;
             nsb = 4;
         }
         const int sb = j < nsb ? j : 2 * nsb - 1 - j;
         return (int64_t)k * K + (int64_t)sb * T;
+    };
+    // Piece mode: this block's range [F0, F1) of the units' blocks.  Ranges
+    // are taken in reverse ticket order, so the range holding a cut unit's
+    // tail started before the one waiting for it.
+    const int64_t Wb = Bt * p.ntiles * (int64_t)p.nsub;
+    const int piece = pieces ? p.npieces - 1 - item : 0;
+    const int64_t F0 = pieces ? (int64_t)piece * Wb / p.npieces : 0;
+    const int64_t F1 = pieces ? (int64_t)(piece + 1) * Wb / p.npieces : 0;
+    // Segment holding item li of the range: unit u, blocks [k0, k1); returns
+    // the item's index inside the segment.
+    auto piece_seg = [&](int li, int& u, int& k0, int& k1) -> int {
+        u = (int)(F0 / p.nsub);
+        for (;;) {
+            const int64_t ub = (int64_t)u * p.nsub;
+            k0 = (int)(max64(F0, ub) - ub);
+            k1 = (int)(min64(F1, ub + p.nsub) - ub);
+            const int n = seg_items(k0, k1);
+            if (li < n || ub + p.nsub >= F1) return li;
+            li -= n;
+            ++u;
+        }
+    };
+    int nE = 0, nitems = 0;
+    if (pieces) {
+        for (int64_t ub = (F0 / p.nsub) * p.nsub; ub < F1; ub += p.nsub)
+            nitems += seg_items((int)(max64(F0, ub) - ub), (int)(min64(F1, ub + p.nsub) - ub));
+    } else {
+        const int per_g = (int)(Bt * p.ntiles);
+        const int gg = p.ngroups - 1 - item / per_g;
+        const int k0 = gg * p.blk_per_group;
+        set_unit(item % per_g, gg, k0, min(k0 + p.blk_per_group, p.nsub));
+        nE = firstg ? 0 : (int)((tg1 - tg0 + T - 1) / T);
+        nitems = nE + seg_items(kb0, kb1);
+    }
+    // Input coordinates of item li: batch element, first channel, first token.
+    auto item_at = [&](int li, int& zb, int& x) -> int64_t {
+        if (pieces) {
+            int u, k0, k1;
+            const int j = piece_seg(li, u, k0, k1);
+            zb = u / p.ntiles;
+            x = (u % p.ntiles) * P;
+            return seg_t0(j, k0, k1);
+        }
+        zb = bb;
+        x = (int)c0;
+        if (li < nE) return tg0 + (int64_t)(nE - 1 - li) * T;
+        return seg_t0(li - nE, kb0, kb1);
     };
     auto issue = [&](int li) {  // one thread
         const int buf = li % Sm::NRAW;
@@ -243,7 +308,8 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             (uint32_t)sizeof(Tin) *
             ((T + 3) * P + (2 + (has_z ? 1 : 0) + (has_b ? 1 : 0)) * T * P + 2 * T * N);
         tma::expect_tx(mb, bytes);
-        const int x = (int)c0, y = (int)item_t0(li), zb = bb;
+        int zb, x;
+        const int y = (int)item_at(li, zb, x);
         tma::load_3d(&r.u[0][0], &tm.u, x, y - 3, zb, mb);
         tma::load_3d(&r.a[0][0], &tm.a, x, y, zb, mb);
         if (has_b) tma::load_3d(&r.b[0][0], &tm.b, x, y, zb, mb);
@@ -488,76 +554,70 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         tc::tmem_st4(trow + Cols::WU + qd * TQ, c1);
         tc::tmem_st4(trow + Cols::VV + qd * TQ, c2);
         tc::tmem_st_wait();
-        __syncthreads();  // brow, crow, y1, w1 complete
         if (!slow) {
-            if (sweep != kSweepEarly && warp < 2) {
-                // Warp 0: A_C[t][m] = sum_ch Y_t W_m (m <= t) or A_B[t][t'] =
-                // sum_ch P_t U_t' (t' >= t) -> ta2.  Warp 1: the Gram, forward
-                // G[t][m] = C_t . B_m (m <= t), backward G^T[t][t'] = C_t' . B_t
-                // (t' >= t) -> tg.  Warp-level tf32 MMAs.
-                float dd[2][4];
-                float* dst;
-                if (warp == 0) {
-                    tc::warp_gram16<P, P + 4>(&sm.y1[0][0], &sm.w1[0][0], dd);
-                    dst = sm.ta2;
-                } else {
-                    tc::warp_gram16<N, N + 4>(fwd ? &sm.crow[0][0] : &sm.brow[0][0],
-                                              fwd ? &sm.brow[0][0] : &sm.crow[0][0], dd);
-                    dst = sm.tg;
-                }
-                const int lane = tid & 31, gq = lane >> 2, kq = lane & 3;
-#pragma unroll
-                for (int n = 0; n < 2; ++n)
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int row = gq + (r >> 1) * 8, col = 8 * n + 2 * kq + (r & 1);
-                        const bool live = fwd ? (col <= row) : (col >= row);
-                        dst[tc::kmajor_offset(row, col, T) >> 2] = live ? dd[n][r] : 0.f;
-                    }
-            } else {
-                // K-major per-token tiles (the other warps).
-                const int t2 = sweep != kSweepEarly ? tid - 64 : tid;
-                const int n2 = sweep != kSweepEarly ? NT - 64 : NT;
-                for (int e = t2; e < T * N / 4; e += n2) {
-                    const int rest = e >> 3;
-                    const int tt = (rest & 1) * 8 + (e & 7), j = (rest >> 1) * 4;
-                    // ta: rows t, K = d_state (C forward, B backward)
-                    *reinterpret_cast<float4*>(&sm.ta[tc::kmajor_offset(tt, j, N) >> 2]) =
-                        fwd ? *reinterpret_cast<const float4*>(&sm.crow[tt][j])
-                            : *reinterpret_cast<const float4*>(&sm.brow[tt][j]);
-                    // ts: rows d_state, K = 16 (B^T forward, C^T backward)
-                    const int jj = e % N, m0 = (e / N) * 4;
-                    const float(*src)[N + 4] = fwd ? sm.brow : sm.crow;
-                    *reinterpret_cast<float4*>(&sm.ts[tc::kmajor_offset(jj, m0, T) >> 2]) =
-                        make_float4(src[m0][jj], src[m0 + 1][jj], src[m0 + 2][jj],
-                                    src[m0 + 3][jj]);
-                }
+            // K-major per-token tiles (all threads; brow / crow are complete
+            // since the exchange barrier).
+            for (int e = tid; e < T * N / 4; e += NT) {
+                const int rest = e >> 3;
+                const int tt = (rest & 1) * 8 + (e & 7), j = (rest >> 1) * 4;
+                // ta: rows t, K = d_state (C forward, B backward)
+                *reinterpret_cast<float4*>(&sm.ta[tc::kmajor_offset(tt, j, N) >> 2]) =
+                    fwd ? *reinterpret_cast<const float4*>(&sm.crow[tt][j])
+                        : *reinterpret_cast<const float4*>(&sm.brow[tt][j]);
+                // ts: rows d_state, K = 16 (B^T forward, C^T backward)
+                const int jj = e % N, m0 = (e / N) * 4;
+                const float(*src)[N + 4] = fwd ? sm.brow : sm.crow;
+                *reinterpret_cast<float4*>(&sm.ts[tc::kmajor_offset(jj, m0, T) >> 2]) =
+                    make_float4(src[m0][jj], src[m0 + 1][jj], src[m0 + 2][jj], src[m0 + 3][jj]);
             }
         }
         tc::fence_proxy_async();
-        sync();
+        sync();  // y1, w1, pk, tiles and the TMEM operand columns complete
         // Prefetch: buffer (li + NRAW - 1) % NRAW was last read by item li - 1.
-        // Issued here, by a thread other than the MMA issuer, so it overlaps
-        // the MMA wait instead of delaying the item's first barrier.
-        if (tid == 32 && li + Sm::NRAW - 1 < nitems) issue(li + Sm::NRAW - 1);
+        // Issued here, by a thread that neither computes the small products nor
+        // issues MMAs, so it overlaps the MMA wait.
+        if (tid == 160 && li + Sm::NRAW - 1 < nitems) issue(li + Sm::NRAW - 1);
     };
 
-    // MMAs of the current item (one thread), then commit.
-    // MMAs of the current item: three independent accumulation chains, each
-    // issued (and committed to the 3-arrival barrier sm.mma) by lane 0 of its
-    // own warp so their issue overlaps: chain 0, readout (forward: X . C + W G)
-    // or dv (backward: H . B + U G^T) into R; chain 1, state (forward: V B^T)
-    // or adjoint (backward: (s dy E) C^T) into D; chain 2, dC or dB
-    // ((state^T)(Y or P) over channels + (B^T or C^T)(A_C or A_B)) into BC.
-    // The early sweep runs chain 1 only; the other two lanes just arrive.
+    // The small per-sub-chunk products on warps 0-3 (warp-level tf32 MMAs):
+    // warps 0, 1 take halves (64 channels each) of A_C[t][m] = sum_ch Y_t W_m
+    // (m <= t) or A_B[t][t'] = sum_ch P_t U_t' (t' >= t) -> ta2; warps 2, 3
+    // halves (d_state / 2 each) of the Gram, forward G[t][m] = C_t . B_m
+    // (m <= t), backward G^T[t][t'] = C_t' . B_t (t' >= t) -> tg.  The MMAs
+    // accumulate both halves.
+    auto small_products = [&](bool fwd) {
+        float dd[2][4];
+        float* dst;
+        const int h = warp & 1;
+        if (warp < 2) {
+            tc::warp_gram16<P / 2, P + 4>(&sm.y1[0][h * (P / 2)], &sm.w1[0][h * (P / 2)], dd);
+            dst = sm.ta2[h];
+        } else {
+            const int k0 = h * (N / 2);
+            tc::warp_gram16<N / 2, N + 4>(fwd ? &sm.crow[0][k0] : &sm.brow[0][k0],
+                                          fwd ? &sm.brow[0][k0] : &sm.crow[0][k0], dd);
+            dst = sm.tg[h];
+        }
+        const int lane = tid & 31, gq = lane >> 2, kq = lane & 3;
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int row = gq + (r >> 1) * 8, col = 8 * n + 2 * kq + (r & 1);
+                const bool live = fwd ? (col <= row) : (col >= row);
+                dst[tc::kmajor_offset(row, col, T) >> 2] = live ? dd[n][r] : 0.f;
+            }
+    };
+
+    // MMAs of the current item, in independent accumulation chains: chain 0,
+    // readout (forward: X . C + W G) or dv (backward: H . B + U G^T) into R;
+    // chain 1, state (forward: V B^T) or adjoint (backward: (s dy E) C^T)
+    // into D; chain 2, dC or dB ((state^T)(Y or P) over channels + (B^T or
+    // C^T)(A_C or A_B)) into BC; chain 3 (d_state 64), the second half of
+    // the channel sum into BC2.
     auto issue_chain = [&](int chain, int sweep) {
         constexpr uint32_t id16 = tc::idesc_tf32(128, T);
         constexpr uint32_t idN = tc::idesc_tf32(128, N);
-        const bool full = sweep != kSweepEarly;
-        if (chain != 1 && !full) {
-            tc::mbar_arrive(&sm.mma);
-            return;
-        }
         if (chain == 3) {  // second half of the dC / dB channel sum into BC2
             const uint32_t a_st = tc::smem_u32(sm.st), a_pk = tc::smem_u32(sm.pk);
 #pragma unroll
@@ -566,20 +626,21 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                                 tc::sdesc_sw128(a_st + (i >> 2) * N * 128 + (i & 3) * 32),
                                 tc::sdesc_sw128(a_pk + (i >> 2) * T * 128 + (i & 3) * 32), id16,
                                 i > P / 16 ? 1u : 0u);
-            tc::mma_commit(&sm.mma);
             return;
         }
         if (chain == 0) {
-            const uint32_t a_ta = tc::smem_u32(sm.ta), a_tg = tc::smem_u32(sm.tg);
+            const uint32_t a_ta = tc::smem_u32(sm.ta), a_tg = tc::smem_u32(&sm.tg[0][0]);
             const uint32_t Acol = sweep == kSweepFwd ? Cols::X : Cols::G;
 #pragma unroll
             for (int i = 0; i < N / 8; ++i)
                 tc::mma_tf32_ts(tbase + Cols::R, tbase + Acol + i * 8,
                                 tc::sdesc(a_ta + i * 256, 128, 32 * N), id16, i > 0 ? 1u : 0u);
 #pragma unroll
-            for (int i = 0; i < T / 8; ++i)
-                tc::mma_tf32_ts(tbase + Cols::R, tbase + Cols::WU + i * 8,
-                                tc::sdesc(a_tg + i * 256, 128, 32 * T), id16, 1u);
+            for (int i = 0; i < 2 * (T / 8); ++i)  // both partial Gram tiles
+                tc::mma_tf32_ts(tbase + Cols::R, tbase + Cols::WU + (i % (T / 8)) * 8,
+                                tc::sdesc(a_tg + (i / (T / 8)) * T * T * 4 + (i % (T / 8)) * 256,
+                                          128, 32 * T),
+                                id16, 1u);
         } else if (chain == 1) {
             const uint32_t a_ts = tc::smem_u32(sm.ts);
 #pragma unroll
@@ -587,7 +648,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 tc::mma_tf32_ts(tbase + Cols::D, tbase + Cols::VV + i * 8,
                                 tc::sdesc(a_ts + i * 256, 128, 32 * T), idN, i > 0 ? 1u : 0u);
         } else {
-            const uint32_t a_ts = tc::smem_u32(sm.ts), a_t2 = tc::smem_u32(sm.ta2);
+            const uint32_t a_ts = tc::smem_u32(sm.ts), a_t2 = tc::smem_u32(&sm.ta2[0][0]);
             const uint32_t a_st = tc::smem_u32(sm.st), a_pk = tc::smem_u32(sm.pk);
             constexpr int KE = Cols::SPLIT ? P / 16 : P / 8;  // K steps of this chain
 #pragma unroll
@@ -597,11 +658,13 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                                 tc::sdesc_sw128(a_pk + (i >> 2) * T * 128 + (i & 3) * 32), id16,
                                 i > 0 ? 1u : 0u);
 #pragma unroll
-            for (int i = 0; i < T / 8; ++i)
-                tc::mma_tf32_ss(tbase + Cols::BC, tc::sdesc(a_ts + i * 256, 128, 32 * T),
-                                tc::sdesc(a_t2 + i * 256, 128, 32 * T), id16, 1u);
+            for (int i = 0; i < 2 * (T / 8); ++i) {  // both partial A_C / A_B tiles
+                const int kk = i % (T / 8), hh = i / (T / 8);
+                tc::mma_tf32_ss(tbase + Cols::BC, tc::sdesc(a_ts + kk * 256, 128, 32 * T),
+                                tc::sdesc(a_t2 + hh * T * T * 4 + kk * 256, 128, 32 * T), id16,
+                                1u);
+            }
         }
-        tc::mma_commit(&sm.mma);
     };
 
     // Start item li: prefetch the next one, wait for this one's inputs.
@@ -609,10 +672,32 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         if (!tc::mbar_wait(&sm.loaded[li % Sm::NRAW], (uint32_t)((li / Sm::NRAW) & 1), kBSpin))
             timed_out = true;
     };
+    // Three arrivals on sm.mma per item.  Warp 4 issues the chains that need
+    // no small product (1, and 3 for d_state 64) at once; warps 0-3 compute
+    // the small products meanwhile, meet on named barrier 1, and lanes 0 of
+    // warps 0 and 1 issue chains 0 and 2.  The early sweep runs chain 1 only.
     auto run_mma = [&](int sweep) {
-        if ((tid & 31) == 0 && warp < (Cols::SPLIT ? 4 : 3)) {
-            tc::fence_after_sync();
-            issue_chain(warp, sweep);
+        const bool full = sweep != kSweepEarly;
+        if (full && warp < 4) {
+            small_products(sweep == kSweepFwd);
+            tc::fence_proxy_async();
+            tc::named_bar(1, 128);
+        }
+        if ((tid & 31) == 0) {
+            if (warp == 4) {
+                tc::fence_after_sync();
+                issue_chain(1, sweep);
+                if (Cols::SPLIT && full) issue_chain(3, sweep);
+                tc::mma_commit(&sm.mma);
+            } else if (warp < 2) {
+                if (full) {
+                    tc::fence_after_sync();
+                    issue_chain(warp == 0 ? 0 : 2, sweep);
+                    tc::mma_commit(&sm.mma);
+                } else {
+                    tc::mbar_arrive(&sm.mma);
+                }
+            }
         }
         if (!tc::mbar_wait(&sm.mma, mma_phase, kBSpin)) timed_out = true;
         mma_phase ^= 1u;
@@ -636,7 +721,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
 #pragma unroll
             for (int k = 0; k < TQ; ++k) {
                 const int64_t t = t0 + qd * TQ + k;
-                if (t < te) part[t * 2 * N + slot * N + j] = v[k];
+                if (t < te) part_row()[t * 2 * N + slot * N + j] = v[k];
             }
         } else {
             // keep the warp's tcgen05.ld count uniform per lane quadrant
@@ -646,7 +731,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         for (int e = tid; e < T * N; e += NT) {
             const int tt = e / N, j = e % N;
             const int64_t t = t0 + tt;
-            if (t < te) part[t * 2 * N + slot * N + j] = sm.acc[tt][j];
+            if (t < te) part_row()[t * 2 * N + slot * N + j] = sm.acc[tt][j];
         }
     };
     auto warp_sum = [](float v) {
@@ -745,16 +830,18 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     // ====================================================== early pass
     // Adjoint only over the group (last sub-chunk first) to publish the
     // carry leaving the group's start.
-    float* carry_in = p.carry + ((int64_t)g * Bt + bb) * d * N;
-    float* carry_out = g > 0 ? p.carry + ((int64_t)(g - 1) * Bt + bb) * d * N : nullptr;
-    int* flag_in = p.flags + ((int64_t)g * Bt + bb) * p.ntiles + tile;
-    int* flag_out = g > 0 ? p.flags + ((int64_t)(g - 1) * Bt + bb) * p.ntiles + tile : nullptr;
-    const float* dxf = p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr;
-    if (!firstg) {
+    // (Group mode.)  Carry slots: group mode, the carry entering group g's
+    // end in slot g; piece mode, a cut unit's carry in slot 0.
+    auto carry_slot = [&](int slot) { return p.carry + ((int64_t)slot * Bt + bb) * d * N; };
+    auto flag_slot = [&](int slot) { return p.flags + ((int64_t)slot * Bt + bb) * p.ntiles + tile; };
+    if (!pieces && !firstg) {
+        float* carry_in = carry_slot(g);
+        const float* dxf = p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr;
         tmem_from(Cols::G, lastg ? dxf : nullptr, false);
         float logF = 0.f;
         for (int e = 0; e < nE; ++e, ++li) {
-            const int64_t t0 = item_t0(li);
+            int zb_, x_;
+            const int64_t t0 = item_at(li, zb_, x_);
             begin_item();
             prep(t0, tg1, kSweepEarly, 0);
             if (!slow) {
@@ -768,7 +855,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             sync();
         }
         if (!lastg) {
-            if (tid == 0) sm.ok = wait_flag(flag_in, &p.hdr->status, p.wait_limit) ? 1 : 0;
+            if (tid == 0) sm.ok = wait_flag(flag_slot(g), &p.hdr->status, p.wait_limit) ? 1 : 0;
             __syncthreads();
             const bool okc = sm.ok != 0;
             // carry out = (decay over the group) H + local contribution
@@ -793,18 +880,29 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             }
             tc::tmem_st_wait();
         }
-        tmem_to(Cols::G, carry_out);
+        tmem_to(Cols::G, carry_slot(g - 1));
         __threadfence();
         __syncthreads();
-        if (tid == 0 && !(lastg && p.fault_skip_publish)) st_release(flag_out, 1);
+        if (tid == 0 && !(lastg && p.fault_skip_publish)) st_release(flag_slot(g - 1), 1);
     }
-    // carry entering the group's end
+
+    // ====================================================== main phase
+    // Per unit segment [kb0, kb1) (group mode: the one set above), from the
+    // carry entering its end.
+    const int64_t ub_first = pieces ? (F0 / p.nsub) * p.nsub : 0;
+    const int64_t ub_end = pieces ? F1 : 1;
+    for (int64_t ub = ub_first; ub < ub_end; ub += pieces ? p.nsub : 1) {
+    if (pieces) {
+        const int k0 = (int)(max64(F0, ub) - ub), k1 = (int)(min64(F1, ub + p.nsub) - ub);
+        set_unit((int)(ub / p.nsub), k0 > 0 ? 1 : 0, k0, k1);
+    }
     if (lastg) {
-        tmem_from(Cols::G, dxf, false);
+        tmem_from(Cols::G, p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr, false);
     } else {
-        if (tid == 0) sm.ok = wait_flag(flag_in, &p.hdr->status, p.wait_limit) ? 1 : 0;
+        const int slot = pieces ? 0 : g;
+        if (tid == 0) sm.ok = wait_flag(flag_slot(slot), &p.hdr->status, p.wait_limit) ? 1 : 0;
         __syncthreads();
-        tmem_from(Cols::G, sm.ok ? carry_in : nullptr, true);
+        tmem_from(Cols::G, sm.ok ? carry_slot(slot) : nullptr, true);
     }
     // dp beyond the group: zero (the next group's terms go via the edge fixup)
     for (int i = tid; i < 3 * P; i += NT) (&sm.dp[1][0][0])[i] = 0.f;
@@ -856,7 +954,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                     dl[q] = s * dyv[q] * yd[q];
                     if (has_z && q < nvh) {
                         const float yv = fmaf(s, yd[q], Dc * hv[q]);
-                        gdz[(t0 + tt) * d] = from_f<Tout>(to_f(r.dy[tt][ch]) * yv * aux[q]);
+                        gout(p.dz)[(t0 + tt) * d] = from_f<Tout>(to_f(r.dy[tt][ch]) * yv * aux[q]);
                     }
                 }
                 tc::tmem_st4(trow + Cols::DL + sb * T + qd * TQ, dl);
@@ -946,10 +1044,10 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 const int64_t t = t0 + tt;
                 if (q < nvh) {
                     if (has_b) {
-                        gda[t * d] = from_f<Tout>((base + sfx[q]) * (1.f - fv[q]));
-                        gdb[t * d] = from_f<Tout>(hv[q] * gbv[q] * iv[q] * (1.f - iv[q]));
+                        gout(p.da)[t * d] = from_f<Tout>((base + sfx[q]) * (1.f - fv[q]));
+                        gout(p.db)[t * d] = from_f<Tout>(hv[q] * gbv[q] * iv[q] * (1.f - iv[q]));
                     } else {  // da = (f df - f di)(1 - f), di = h G.B; 1 - f = i
-                        gda[t * d] =
+                        gout(p.da)[t * d] =
                             from_f<Tout>((base + sfx[q] - fv[q] * hv[q] * gbv[q]) * iv[q]);
                     }
                     dD_acc = fmaf(dyv[q], hv[q], dD_acc);
@@ -961,13 +1059,13 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                         const float duv = w3 * dpc[tt][ch] + w2 * dpat(tt + 1) +
                                           w1 * dpat(tt + 2) + w0 * dpat(tt + 3);
                         if (!lastg && group_end_block && t >= te - 3) {
-                            edge[(3 + (t - (te - 3))) * d + c] = duv;  // partial, fixed up later
+                            edge_row()[(3 + (t - (te - 3))) * d + c] = duv;  // partial, fixed up later
                         } else {
-                            gdhu[t * d] = from_f<Tout>(duv);
+                            gout(p.dhu)[t * d] = from_f<Tout>(duv);
                         }
-                        if (k == kb0 && sb == 0 && tt < 3) edge[tt * d + c] = dpc[tt][ch];
+                        if (k == kb0 && sb == 0 && tt < 3) edge_row()[tt * d + c] = dpc[tt][ch];
                     } else {
-                        gdhu[t * d] = from_f<Tout>(dhv[q]);
+                        gout(p.dhu)[t * d] = from_f<Tout>(dhv[q]);
                     }
                 }
             }
@@ -979,7 +1077,15 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
     }
 
     // ------------------------------------------------ carries and partials
-    if (firstg && p.dx0) tmem_to(Cols::G, p.dx0 + (int64_t)bb * d * N);
+    if (firstg) {
+        if (p.dx0) tmem_to(Cols::G, p.dx0 + (int64_t)bb * d * N);
+    } else if (pieces) {
+        // the tail of a cut unit: publish the carry leaving its start
+        tmem_to(Cols::G, carry_slot(0));
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && !p.fault_skip_publish) st_release(flag_slot(0), 1);
+    }
     {
         float* cpart = p.chan_part + ((int64_t)bb * p.ngroups + g) * d * 8;
         float* red6 = &sm.acc[0][0];  // [6][P] (T * N >= 6 * P)
@@ -998,14 +1104,21 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         if (tid < P && c0 + tid < d) {
 #pragma unroll
             for (int q = 0; q < 6; ++q) cpart[(c0 + tid) * 8 + q] = red6[q * P + tid];
+            if (pieces && firstg && lastg) {  // uncut unit: its tail slot stays empty
+                float* cp1 = p.chan_part + ((int64_t)bb * p.ngroups + 1) * d * 8;
+#pragma unroll
+                for (int q = 0; q < 6; ++q) cp1[(c0 + tid) * 8 + q] = 0.f;
+            }
         }
     }
+    }  // unit segments
+
     if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
     sync();
     if (warp == 0) tc::tmem_dealloc(tbase, Cols::ALLOC);
 }
 
-template <typename Tout, int N, bool CONV>
+template <typename Tout, int N, bool CONV, bool PIECES>
 static cudaError_t launch_bwd_tc_t(const BwdParams& p, cudaStream_t st) {
     BwdTmaps tm;
     memset(&tm, 0, sizeof(tm));
@@ -1019,11 +1132,11 @@ static cudaError_t launch_bwd_tc_t(const BwdParams& p, cudaStream_t st) {
     if (ok && p.z) ok = tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, T, 128);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(BwdTcSmem<N>);
-    auto kern = scan_bwd_tc_kernel<Tout, N, CONV>;
+    auto kern = scan_bwd_tc_kernel<Tout, N, CONV, PIECES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = p.ngroups * (int)p.Bt * p.ntiles;
+    const int grid = p.npieces > 0 ? p.npieces : p.ngroups * (int)p.Bt * p.ntiles;
     kern<<<grid, 512, smem, st>>>(p, tm);
     return cudaGetLastError();
 }
@@ -1034,8 +1147,12 @@ bool bwd_tc_supported(int dtype, int64_t N, int64_t d) {
 
 cudaError_t launch_scan_bwd_tc_main(const BwdParams& p, int out_dtype, cudaStream_t st) {
     const bool conv = p.conv_w != nullptr;
-#define NAJU_TC_BWD(TO, NN)                                                     \
-    return conv ? launch_bwd_tc_t<TO, NN, true>(p, st) : launch_bwd_tc_t<TO, NN, false>(p, st)
+    const bool pc = p.npieces > 0;
+#define NAJU_TC_BWD(TO, NN)                                                          \
+    return conv ? (pc ? launch_bwd_tc_t<TO, NN, true, true>(p, st)                   \
+                      : launch_bwd_tc_t<TO, NN, true, false>(p, st))                 \
+                : (pc ? launch_bwd_tc_t<TO, NN, false, true>(p, st)                  \
+                      : launch_bwd_tc_t<TO, NN, false, false>(p, st))
     if (out_dtype == NAJU_BF16) {
         if (p.N == 64) NAJU_TC_BWD(__nv_bfloat16, 64);
         if (p.N == 128) NAJU_TC_BWD(__nv_bfloat16, 128);

@@ -42,6 +42,15 @@ void naju_testing_set_bwd_groups(int32_t groups);
 /* The backward's number of sequence groups for these dims. */
 int32_t naju_testing_bwd_groups(const void* dims);
 
+/* Piece mode of the tensor-core backward: 0 = automatic (one range per SM
+ * when there are at least as many 128-channel units as SMs but not a whole
+ * number of waves), < 0 = never, > 0 = that many ranges (used when there
+ * are at least that many units and no forced group count). */
+void naju_testing_set_bwd_pieces(int32_t pieces);
+
+/* The backward's number of piece-mode ranges for these dims (0: group mode). */
+int32_t naju_testing_bwd_pieces(const void* dims);
+
 /* Forward implementation: 0 = automatic (tensor cores for bf16 activations
  * with d_state 64 or 128 and d_inner % 8 == 0, CUDA cores otherwise),
  * 1 = always CUDA cores. */

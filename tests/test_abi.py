@@ -117,3 +117,27 @@ def test_tensor_core_dispatch_rules(L):
     assert naju.testing_bwd_impl(naju.make_dims(2, 64, 258, 64, naju.BF16)) == 1
     assert naju.testing_fwd_impl(naju.make_dims(2, 64, 256, 32, naju.BF16)) == 1
     assert naju.testing_bwd_impl(naju.make_dims(2, 64, 256, 64, naju.F32)) == 1
+
+
+def test_backward_piece_mode_rules(L):
+    """The tensor-core backward cuts the units' blocks into one range per SM
+    (148) when there are at least that many 128-channel units but not a whole
+    number of waves; otherwise it keeps sequence groups."""
+    dm = naju.make_dims(16, 4096, 2048, 64, naju.BF16)  # 256 units
+    assert naju.testing_bwd_pieces(dm) == 148
+    assert naju.testing_bwd_groups(dm) == 2  # the two carry slots
+    assert naju.testing_bwd_pieces(naju.make_dims(8, 2048, 1536, 64, naju.BF16)) == 0  # 96
+    assert naju.testing_bwd_pieces(naju.make_dims(37, 512, 1024, 64, naju.BF16)) == 0  # 296
+    assert naju.testing_bwd_pieces(naju.make_dims(16, 4096, 2048, 64, naju.F32)) == 0
+    assert naju.testing_bwd_pieces(naju.make_dims(160, 64, 128, 64, naju.BF16)) == 0  # 1 block
+    naju.testing_set_bwd_pieces(-1)
+    try:
+        assert naju.testing_bwd_pieces(dm) == 0
+    finally:
+        naju.testing_set_bwd_pieces(0)
+    naju.testing_set_bwd_pieces(5)
+    try:
+        assert naju.testing_bwd_pieces(naju.make_dims(1, 512, 512, 64, naju.BF16)) == 0  # 4 units
+        assert naju.testing_bwd_pieces(naju.make_dims(2, 512, 512, 64, naju.BF16)) == 5
+    finally:
+        naju.testing_set_bwd_pieces(0)

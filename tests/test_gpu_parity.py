@@ -351,6 +351,50 @@ def test_bwd_tensor_core_sequence_groups(groups):
     compare_grads(g, r, True, TOL_BF16)
 
 
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("conv", [True, False])
+@pytest.mark.parametrize("pieces", [2, 4, 7])
+def test_bwd_tensor_core_pieces(pieces, conv, N):
+    """Piece mode: the units' 64-token blocks cut into equal ranges, one per
+    block, with cuts inside units (adjoint carry handed from a unit's tail to
+    its head, conv terms fixed up across the cut).  9 units (3 batch x 3
+    channel tiles, the last ragged), 6 blocks each (the last ragged)."""
+    w = wl(N, "bf16", Bt=3, L=333, d=264)
+    t = inputs(w, conv, use_x0=True, use_dxL=True)
+    r = oracle_bwd(t, conv)
+    naju.testing_set_bwd_pieces(pieces)
+    try:
+        assert naju.testing_bwd_pieces(naju.make_dims(3, 333, 264, N, naju.BF16)) == pieces
+        g = run_bwd(t, conv, out_dtype=naju.F32)
+    finally:
+        naju.testing_set_bwd_pieces(0)
+    compare_grads(g, r, conv, TOL_BF16)
+
+
+def test_bwd_tensor_core_pieces_timeout_is_reported():
+    """A head whose tail never publishes gives up after the wait limit and
+    reports a timeout; the next call is correct."""
+    w = wl(64, "bf16", Bt=2, L=320, d=256)
+    t = inputs(w, True)
+    naju.testing_set_bwd_pieces(3)
+    try:
+        y, xf, ws = run_fwd(t, True)
+        naju.testing_set_wait_limit(2000)
+        naju.testing_set_skip_publish(True)
+        try:
+            naju.scan_bwd(gpu(t["dout"]), gpu(t["u"]), gpu(t["a"]), gpu(t["b"]), gpu(t["B"]),
+                          gpu(t["C"]), ws, conv_w=gpu(t["conv_w"]), conv_b=gpu(t["conv_b"]),
+                          z=gpu(t["z"]), D=gpu(t["D"]))
+            assert naju.last_device_status(ws) == 4
+        finally:
+            naju.testing_set_skip_publish(False)
+            naju.testing_set_wait_limit(0)
+        g = run_bwd(t, True, out_dtype=naju.F32)
+    finally:
+        naju.testing_set_bwd_pieces(0)
+    compare_grads(g, oracle_bwd(t, True), True, TOL_BF16)
+
+
 def test_bwd_after_grouped_forward():
     """Checkpoints written by a sequence-split forward serve the backward."""
     w = wl(64, "f32", Bt=1, L=700, d=64)

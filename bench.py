@@ -469,8 +469,8 @@ def main():
         raise SystemExit("device status not OK after warm-up")
 
     # Kernels of one step: the forward kernel; the backward kernel, the dB/dC
-    # and channel reductions, and the conv group-edge fixup when the backward
-    # splits the sequence.
+    # and channel reductions, and the conv fixup across sequence-group edges or
+    # piece-mode cuts when the backward splits the sequence.
     launches_per_step = 1 + 3 + (1 if naju.testing_bwd_groups(dims) > 1 else 0)
 
     # ---------------------------------------------------------- timed region

@@ -11,7 +11,7 @@ from ._native import (BF16, F32, Dims, NajuError, alloc_workspace, conv_silu_bwd
                       conv_silu_fwd, conv_silu_step, declared_symbols, last_device_status, lib,
                       library_path, make_dims, scan_bwd, scan_fwd, scan_step, scan_step_conv,
                       testing_bwd_groups, testing_bwd_impl, testing_bwd_pieces,
-                      testing_fwd_groups, testing_fwd_impl, testing_set_bwd_groups,
-                      testing_set_bwd_impl, testing_set_bwd_pieces, testing_set_fwd_groups,
-                      testing_set_fwd_impl, testing_set_skip_publish, testing_set_wait_limit,
-                      workspace_bytes)
+                      testing_fwd_groups, testing_fwd_impl, testing_fwd_pieces,
+                      testing_set_bwd_groups, testing_set_bwd_impl, testing_set_bwd_pieces,
+                      testing_set_fwd_groups, testing_set_fwd_impl, testing_set_fwd_pieces,
+                      testing_set_skip_publish, testing_set_wait_limit, workspace_bytes)

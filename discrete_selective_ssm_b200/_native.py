@@ -89,6 +89,9 @@ def lib(build_if_missing: bool = True):
             L.naju_testing_bwd_groups.argtypes = [vp]
             L.naju_testing_bwd_groups.restype = i32
             L.naju_testing_set_bwd_pieces.argtypes = [i32]
+            L.naju_testing_set_fwd_pieces.argtypes = [i32]
+            L.naju_testing_fwd_pieces.argtypes = [vp]
+            L.naju_testing_fwd_pieces.restype = i32
             L.naju_testing_bwd_pieces.argtypes = [vp]
             L.naju_testing_bwd_pieces.restype = i32
             for name in ("naju_conv_silu_fwd", "naju_conv_silu_bwd", "naju_scan_fwd",
@@ -352,3 +355,11 @@ def testing_set_bwd_pieces(pieces: int):
 
 def testing_bwd_pieces(dims: Dims) -> int:
     return int(lib().naju_testing_bwd_pieces(ctypes.byref(dims)))
+
+
+def testing_set_fwd_pieces(pieces: int):
+    lib().naju_testing_set_fwd_pieces(int(pieces))
+
+
+def testing_fwd_pieces(dims: Dims) -> int:
+    return int(lib().naju_testing_fwd_pieces(ctypes.byref(dims)))

@@ -24,6 +24,7 @@ int g_skip_publish = 0;
 int g_fwd_groups = 0;
 int g_bwd_groups = 0;
 int g_bwd_pieces = 0;  // 0 automatic, < 0 never, > 0 that many ranges
+int g_fwd_pieces = 0;  // the same for the tensor-core forward
 int g_fwd_impl = 0;  // 0 automatic, 1 CUDA cores, 2 tensor cores
 int g_bwd_impl = 0;  // 0 automatic, 1 CUDA cores
 
@@ -51,7 +52,7 @@ naju_status check_dims(const naju_dims* dm) {
 // Workspace layout (every region 256-byte aligned).
 struct Layout {
     bool fwd_tc, bwd_tc;
-    int nck, ngroups, seg_per_group, ntiles_f;
+    int nck, ngroups, seg_per_group, ntiles_f, npieces_f;
     int nsub, nclus, ntiles_b, bgroups, blk_per_group, npieces;
     size_t off_fflags, off_bflags, off_ckpt, off_carry, off_dbc, off_chan, off_edge, total;
 };
@@ -125,13 +126,24 @@ int auto_groups(const naju_dims* dm, int nck, int ntiles_f, bool tc) {
     return (int)(g < nck ? g : nck);
 }
 
+// Tensor-core forward piece mode: the rule of the backward's (one range of
+// checkpoint segments per SM when the 128-channel units fill at least one
+// wave but not a whole number of them); one flag slot per unit.
+int fwd_pieces(const naju_dims* dm, int nck, int ntiles_f, bool tc) {
+    if (!tc || g_fwd_groups > 0 || g_fwd_pieces < 0 || nck < 2) return 0;
+    const int64_t units = dm->batch * (int64_t)ntiles_f;
+    if (g_fwd_pieces > 0) return units >= g_fwd_pieces ? g_fwd_pieces : 0;
+    return (units >= kSMs && units % kSMs != 0) ? kSMs : 0;
+}
+
 Layout layout(const naju_dims* dm) {
     Layout l{};
     const int64_t Bt = dm->batch, L = dm->seqlen, d = dm->d_inner, N = dm->d_state;
     l.nck = (int)cdiv(L, kTck);
     l.fwd_tc = use_fwd_tc(dm);
     l.ntiles_f = (int)cdiv(d, l.fwd_tc ? fwd_tc_channels_per_block() : fwd_channels_per_block(N));
-    int g = auto_groups(dm, l.nck, l.ntiles_f, l.fwd_tc);
+    l.npieces_f = fwd_pieces(dm, l.nck, l.ntiles_f, l.fwd_tc);
+    int g = l.npieces_f > 0 ? 1 : auto_groups(dm, l.nck, l.ntiles_f, l.fwd_tc);
     l.seg_per_group = (int)cdiv(l.nck, g);
     l.ngroups = (int)cdiv(l.nck, l.seg_per_group);
     l.nsub = (int)cdiv(L, kBwdSub);
@@ -245,6 +257,7 @@ naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* co
     p.Bt = dims->batch; p.L = dims->seqlen; p.d = dims->d_inner; p.N = dims->d_state;
     p.T_ck = kTck; p.nck = l.nck; p.seg_per_group = l.seg_per_group; p.ngroups = l.ngroups;
     p.ntiles = l.ntiles_f;
+    p.npieces = l.npieces_f;
     p.scale = 1.0f / std::sqrt((float)dims->d_state);
     p.wait_limit = g_wait_limit;
     p.fault_skip_publish = g_skip_publish;
@@ -382,6 +395,12 @@ void naju_testing_set_skip_publish(int32_t skip) { g_skip_publish = skip ? 1 : 0
 void naju_testing_set_fwd_groups(int32_t groups) { g_fwd_groups = groups > 0 ? groups : 0; }
 void naju_testing_set_bwd_groups(int32_t groups) { g_bwd_groups = groups > 0 ? groups : 0; }
 void naju_testing_set_bwd_pieces(int32_t pieces) { g_bwd_pieces = pieces; }
+void naju_testing_set_fwd_pieces(int32_t pieces) { g_fwd_pieces = pieces; }
+int32_t naju_testing_fwd_pieces(const void* dims) {
+    const naju_dims* dm = static_cast<const naju_dims*>(dims);
+    if (check_dims(dm) != NAJU_OK) return 0;
+    return layout(dm).npieces_f;
+}
 int32_t naju_testing_bwd_pieces(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);
     if (check_dims(dm) != NAJU_OK) return 0;

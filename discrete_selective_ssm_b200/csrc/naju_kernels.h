@@ -36,6 +36,7 @@ struct FwdParams {
     float scale;        // 1 / sqrt(N)
     long long wait_limit;
     int fault_skip_publish;
+    int npieces;        // tensor-core kernel: > 0 for piece mode (ngroups == 1)
 };
 
 struct BwdParams {

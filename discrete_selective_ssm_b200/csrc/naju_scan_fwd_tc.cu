@@ -110,7 +110,7 @@ struct FwdTcSmem {
 
 }  // namespace
 
-template <typename Tout, int N, bool CONV>
+template <typename Tout, int N, bool CONV, bool PIECES>
 __global__ void __launch_bounds__(640, 1)
 scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
     using Tin = __nv_bfloat16;
@@ -158,38 +158,55 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
     const uint32_t tbase = sm.taddr;
     const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;  // this warp's TMEM lanes
     const int item = sm.item;
-    const int per_g = (int)(Bt * p.ntiles);
-    const int g = item / per_g;
-    const int bb = (item % per_g) / p.ntiles;
-    const int tile = item % p.ntiles;
-    const int64_t c0 = (int64_t)tile * P;
-    const int64_t c = c0 + ch;
-    const bool cvalid = c < d;
-
-    const int seg0 = g * p.seg_per_group;
-    const int seg1 = min(seg0 + p.seg_per_group, p.nck);
-    const int64_t tbeg = (int64_t)seg0 * p.T_ck;
-    const int64_t tend = min64(L, (int64_t)seg1 * p.T_ck);
-    const bool last_group = (g == p.ngroups - 1);
-
-    const int64_t boff = (int64_t)bb * L;
     const bool has_z = p.z != nullptr;
     const bool has_b = p.b != nullptr;  // absent: coupled single gate i = 1 - f
-    Tout* gy = static_cast<Tout*>(p.y) + boff * d;
-
+    // Work unit u = bb * ntiles + tile: 128 channels of one batch element,
+    // over checkpoint segments [seg0, seg1).  Group mode: one (sequence group,
+    // unit) per block.  Piece mode (PIECES): the units' segments, laid end to
+    // end, are cut into npieces equal ranges, one per block; a block takes its
+    // range's unit segments last first, so the head of a unit cut in two (the
+    // last segment of the earlier range) runs first and publishes the state at
+    // the cut for the tail (the first segment of the later range), which runs
+    // last in a block that started after it.
+    int g = 0, bb = 0, tile = 0, seg0 = 0, seg1 = 0;
+    int64_t c0 = 0, c = 0, tbeg = 0, tend = 0;
+    bool cvalid = false, last_group = true;
+    Tout* gy = nullptr;
+    float* ck_b = nullptr;
     float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, wb = 0.f, Dc = 0.f;
-    if (cvalid) {
-        if (CONV) {
-            w0 = p.conv_w[c * 4 + 0];
-            w1 = p.conv_w[c * 4 + 1];
-            w2 = p.conv_w[c * 4 + 2];
-            w3 = p.conv_w[c * 4 + 3];
-            wb = p.conv_b ? p.conv_b[c] : 0.f;
+    auto set_unit = [&](int u, int g_, int s0, int s1) {
+        g = g_;
+        bb = u / p.ntiles;
+        tile = u % p.ntiles;
+        c0 = (int64_t)tile * P;
+        c = c0 + ch;
+        cvalid = c < d;
+        seg0 = s0;
+        seg1 = s1;
+        tbeg = (int64_t)seg0 * p.T_ck;
+        tend = min64(L, (int64_t)seg1 * p.T_ck);
+        last_group = seg1 == p.nck;
+        gy = static_cast<Tout*>(p.y) + (int64_t)bb * L * d;
+        ck_b = p.ckpt + (int64_t)bb * (p.nck + 1) * d * N;
+        w0 = w1 = w2 = w3 = wb = Dc = 0.f;
+        if (cvalid) {
+            if (CONV) {
+                w0 = p.conv_w[c * 4 + 0];
+                w1 = p.conv_w[c * 4 + 1];
+                w2 = p.conv_w[c * 4 + 2];
+                w3 = p.conv_w[c * 4 + 3];
+                wb = p.conv_b ? p.conv_b[c] : 0.f;
+            }
+            Dc = p.D ? p.D[c] : 0.f;
         }
-        Dc = p.D ? p.D[c] : 0.f;
+    };
+    if (!PIECES) {
+        const int per_g = (int)(Bt * p.ntiles);
+        const int gg = item / per_g;
+        const int s0 = gg * p.seg_per_group;
+        set_unit(item % per_g, gg, s0, min(s0 + p.seg_per_group, p.nck));
     }
     const float scale = p.scale;
-    float* ck_b = p.ckpt + (int64_t)bb * (p.nck + 1) * d * N;
     bool timed_out = false;
 
     // ======================================================= producer side
@@ -529,74 +546,111 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
         tc::fence_after_sync();
     };
 
-    // ------------------------------------------ early pass and carry chain
-    const float* x0b = p.x0 ? p.x0 + (int64_t)bb * d * N : nullptr;
-    const int* flag_prev = (g > 0) ? p.flags + ((int64_t)(g - 1) * Bt + bb) * p.ntiles + tile
-                                   : nullptr;
-    int* flag_mine = p.flags + ((int64_t)g * Bt + bb) * p.ntiles + tile;
-    float* ck_start = ck_b + (int64_t)seg0 * d * N;
-    float* ck_end = ck_b + (int64_t)seg1 * d * N;
-    bool ok = true;
     auto sync_all = [&]() {
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
     };
-    if (!last_group) {
-        if (cons) state_from(g == 0 ? x0b : nullptr, false);
-        sync_all();
-        run_pass(false);
-        if (g > 0) {
+    if (PIECES) {
+        // ----------------------------------------------- piece mode
+        const int64_t Wb = Bt * p.ntiles * (int64_t)p.nck;
+        const int64_t F0 = (int64_t)item * Wb / p.npieces;
+        const int64_t F1 = (int64_t)(item + 1) * Wb / p.npieces;
+        const int64_t ub_lo = (F0 / p.nck) * p.nck;
+        for (int64_t ub = ((F1 - 1) / p.nck) * p.nck; ub >= ub_lo; ub -= p.nck) {
+            const int s0 = (int)(max64(F0, ub) - ub), s1 = (int)(min64(F1, ub + p.nck) - ub);
+            set_unit((int)(ub / p.nck), 0, s0, s1);
+            int* flag_cut = p.flags + (int64_t)bb * p.ntiles + tile;
+            if (s0 == 0) {
+                if (cons) {
+                    state_from(p.x0 ? p.x0 + (int64_t)bb * d * N : nullptr, false);
+                    state_to(ck_b);  // checkpoint 0 = initial state
+                }
+            } else {
+                // tail of a cut unit: the state at the cut from its head
+                if (tid == 0) sm.ok = wait_flag(flag_cut, &p.hdr->status, p.wait_limit) ? 1 : 0;
+                __syncthreads();
+                if (cons) state_from(sm.ok ? ck_b + (int64_t)s0 * d * N : nullptr, true);
+            }
+            sync_all();
+            run_pass(true);
+            if (cons) {
+                state_to(ck_b + (int64_t)s1 * d * N);
+                if (s1 == p.nck && p.x_final) state_to(p.x_final + (int64_t)bb * d * N);
+            }
+            if (s1 < p.nck) {  // head of a cut unit: publish the state at the cut
+                __threadfence();
+                __syncthreads();
+                if (tid == 0 && !p.fault_skip_publish) st_release(flag_cut, 1);
+            }
+            sync_all();
+        }
+    } else {
+        // ------------------------------------------ early pass and carry chain
+        const float* x0b = p.x0 ? p.x0 + (int64_t)bb * d * N : nullptr;
+        const int* flag_prev = (g > 0) ? p.flags + ((int64_t)(g - 1) * Bt + bb) * p.ntiles + tile
+                                       : nullptr;
+        int* flag_mine = p.flags + ((int64_t)g * Bt + bb) * p.ntiles + tile;
+        float* ck_start = ck_b + (int64_t)seg0 * d * N;
+        float* ck_end = ck_b + (int64_t)seg1 * d * N;
+        bool ok = true;
+        if (!last_group) {
+            if (cons) state_from(g == 0 ? x0b : nullptr, false);
+            sync_all();
+            run_pass(false);
+            if (g > 0) {
+                if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
+                __syncthreads();
+                ok = sm.ok != 0;
+                if (cons) {
+                    // X_end += (product of f over the group) X_start
+                    const float Pf = __expf(logP);
+#pragma unroll
+                    for (int n0 = 0; n0 < N; n0 += 16) {
+                        float x[16];
+                        tc::tmem_ld16(tbase + lane + Cols::X + n0, x);
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int k = 0; k < 16; k += 4) {
+                            float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (ok && cvalid)
+                                v4 = __ldcg(reinterpret_cast<const float4*>(ck_start + c * N +
+                                                                            n0 + k));
+                            x[k] = fmaf(Pf, v4.x, x[k]);
+                            x[k + 1] = fmaf(Pf, v4.y, x[k + 1]);
+                            x[k + 2] = fmaf(Pf, v4.z, x[k + 2]);
+                            x[k + 3] = fmaf(Pf, v4.w, x[k + 3]);
+                        }
+                        tc::tmem_st16(tbase + lane + Cols::X + n0, x);
+                    }
+                    tc::tmem_st_wait();
+                }
+            }
+            if (cons) state_to(ck_end);
+            __threadfence();
+            __syncthreads();
+            if (tid == 0 && !(g == 0 && p.fault_skip_publish)) st_release(flag_mine, 1);
+        } else if (g > 0) {
             if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
             __syncthreads();
             ok = sm.ok != 0;
-            if (cons) {
-                // X_end += (product of f over the group) X_start
-                const float Pf = __expf(logP);
-#pragma unroll
-                for (int n0 = 0; n0 < N; n0 += 16) {
-                    float x[16];
-                    tc::tmem_ld16(tbase + lane + Cols::X + n0, x);
-                    tc::tmem_ld_wait();
-#pragma unroll
-                    for (int k = 0; k < 16; k += 4) {
-                        float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (ok && cvalid)
-                            v4 = __ldcg(reinterpret_cast<const float4*>(ck_start + c * N + n0 + k));
-                        x[k] = fmaf(Pf, v4.x, x[k]);
-                        x[k + 1] = fmaf(Pf, v4.y, x[k + 1]);
-                        x[k + 2] = fmaf(Pf, v4.z, x[k + 2]);
-                        x[k + 3] = fmaf(Pf, v4.w, x[k + 3]);
-                    }
-                    tc::tmem_st16(tbase + lane + Cols::X + n0, x);
-                }
-                tc::tmem_st_wait();
+        }
+        if (cons) {
+            if (g > 0) {
+                state_from(ok ? ck_start : nullptr, true);
+            } else {
+                state_from(x0b, false);
+                state_to(ck_b);  // checkpoint 0 = initial state
             }
         }
-        if (cons) state_to(ck_end);
-        __threadfence();
-        __syncthreads();
-        if (tid == 0 && !(g == 0 && p.fault_skip_publish)) st_release(flag_mine, 1);
-    } else if (g > 0) {
-        if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
-        __syncthreads();
-        ok = sm.ok != 0;
-    }
-    if (cons) {
-        if (g > 0) {
-            state_from(ok ? ck_start : nullptr, true);
-        } else {
-            state_from(x0b, false);
-            state_to(ck_b);  // checkpoint 0 = initial state
-        }
-    }
-    sync_all();
+        sync_all();
 
-    // ------------------------------------------------------- full pass
-    run_pass(true);
-    if (last_group && cons) {
-        state_to(ck_b + (int64_t)p.nck * d * N);
-        if (p.x_final) state_to(p.x_final + (int64_t)bb * d * N);
+        // ------------------------------------------------------- full pass
+        run_pass(true);
+        if (last_group && cons) {
+            state_to(ck_b + (int64_t)p.nck * d * N);
+            if (p.x_final) state_to(p.x_final + (int64_t)bb * d * N);
+        }
     }
     if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
 
@@ -605,7 +659,7 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
     if (warp == 0) tc::tmem_dealloc(tbase, Cols::ALLOC);
 }
 
-template <typename Tout, int N, bool CONV>
+template <typename Tout, int N, bool CONV, bool PIECES>
 static cudaError_t launch_fwd_tc_t(const FwdParams& p, cudaStream_t st) {
     FwdTmaps tm;
     memset(&tm, 0, sizeof(tm));
@@ -618,11 +672,11 @@ static cudaError_t launch_fwd_tc_t(const FwdParams& p, cudaStream_t st) {
     if (ok && p.z) ok = tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, T, 128);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(FwdTcSmem<N>);
-    auto kern = scan_fwd_tc_kernel<Tout, N, CONV>;
+    auto kern = scan_fwd_tc_kernel<Tout, N, CONV, PIECES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int grid = p.ngroups * (int)p.Bt * p.ntiles;
+    const int grid = PIECES ? p.npieces : p.ngroups * (int)p.Bt * p.ntiles;
     kern<<<grid, 640, smem, st>>>(p, tm);
     return cudaGetLastError();
 }
@@ -636,8 +690,12 @@ bool fwd_tc_supported(int dtype, int64_t N, int64_t d) {
 
 cudaError_t launch_scan_fwd_tc(const FwdParams& p, int out_dtype, cudaStream_t st) {
     const bool conv = p.conv_w != nullptr;
-#define NAJU_TC_FWD(TO, NN)                                                     \
-    return conv ? launch_fwd_tc_t<TO, NN, true>(p, st) : launch_fwd_tc_t<TO, NN, false>(p, st)
+    const bool pc = p.npieces > 0;
+#define NAJU_TC_FWD(TO, NN)                                                          \
+    return conv ? (pc ? launch_fwd_tc_t<TO, NN, true, true>(p, st)                   \
+                      : launch_fwd_tc_t<TO, NN, true, false>(p, st))                 \
+                : (pc ? launch_fwd_tc_t<TO, NN, false, true>(p, st)                  \
+                      : launch_fwd_tc_t<TO, NN, false, false>(p, st))
     if (out_dtype == NAJU_BF16) {
         if (p.N == 64) NAJU_TC_FWD(__nv_bfloat16, 64);
         if (p.N == 128) NAJU_TC_FWD(__nv_bfloat16, 128);

@@ -51,6 +51,13 @@ void naju_testing_set_bwd_pieces(int32_t pieces);
 /* The backward's number of piece-mode ranges for these dims (0: group mode). */
 int32_t naju_testing_bwd_pieces(const void* dims);
 
+/* Piece mode of the tensor-core forward, with the same values and rule as
+ * the backward's (ranges of 64-token checkpoint segments). */
+void naju_testing_set_fwd_pieces(int32_t pieces);
+
+/* The forward's number of piece-mode ranges for these dims (0: group mode). */
+int32_t naju_testing_fwd_pieces(const void* dims);
+
 /* Forward implementation: 0 = automatic (tensor cores for bf16 activations
  * with d_state 64 or 128 and d_inner % 8 == 0, CUDA cores otherwise),
  * 1 = always CUDA cores. */

@@ -141,3 +141,17 @@ def test_backward_piece_mode_rules(L):
         assert naju.testing_bwd_pieces(naju.make_dims(2, 512, 512, 64, naju.BF16)) == 5
     finally:
         naju.testing_set_bwd_pieces(0)
+
+
+def test_forward_piece_mode_rules(L):
+    """The tensor-core forward takes piece mode under the backward's rule."""
+    dm = naju.make_dims(16, 4096, 2048, 64, naju.BF16)
+    assert naju.testing_fwd_pieces(dm) == 148
+    assert naju.testing_fwd_groups(dm) == 1
+    assert naju.testing_fwd_pieces(naju.make_dims(8, 2048, 1536, 64, naju.BF16)) == 0
+    assert naju.testing_fwd_pieces(naju.make_dims(16, 4096, 2048, 64, naju.F32)) == 0
+    naju.testing_set_fwd_pieces(-1)
+    try:
+        assert naju.testing_fwd_pieces(dm) == 0
+    finally:
+        naju.testing_set_fwd_pieces(0)

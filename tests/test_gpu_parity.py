@@ -395,6 +395,54 @@ def test_bwd_tensor_core_pieces_timeout_is_reported():
     compare_grads(g, oracle_bwd(t, True), True, TOL_BF16)
 
 
+@pytest.mark.parametrize("N", [64, 128])
+@pytest.mark.parametrize("conv", [True, False])
+@pytest.mark.parametrize("pieces", [2, 4, 7])
+def test_fwd_tensor_core_pieces(pieces, conv, N):
+    """Forward piece mode: ranges of the units' checkpoint segments with cuts
+    inside units (the state at a cut handed from the head to the tail); the
+    checkpoints it writes serve the backward (both in piece mode)."""
+    w = wl(N, "bf16", Bt=3, L=333, d=264)
+    t = inputs(w, conv, use_x0=True, use_dxL=True)
+    naju.testing_set_fwd_pieces(pieces)
+    naju.testing_set_bwd_pieces(pieces)
+    try:
+        assert naju.testing_fwd_pieces(naju.make_dims(3, 333, 264, N, naju.BF16)) == pieces
+        y, xf, _ = run_fwd(t, conv, out_dtype=naju.F32)
+        g = run_bwd(t, conv, out_dtype=naju.F32)
+    finally:
+        naju.testing_set_fwd_pieces(0)
+        naju.testing_set_bwd_pieces(0)
+    ro, rx = oracle_fwd(t, conv)
+    assert_close(y, ro, TOL_BF16, name="y")
+    assert_close(xf, rx, TOL_BF16, name="x_final")
+    compare_grads(g, oracle_bwd(t, conv), conv, TOL_BF16)
+
+
+def test_fwd_tensor_core_pieces_timeout_is_reported():
+    """A tail whose head never publishes gives up after the wait limit and
+    reports a timeout; the next call is correct."""
+    w = wl(64, "bf16", Bt=2, L=320, d=256)
+    t = inputs(w, True)
+    naju.testing_set_fwd_pieces(3)
+    try:
+        naju.testing_set_wait_limit(2000)
+        naju.testing_set_skip_publish(True)
+        try:
+            y, xf, ws = naju.scan_fwd(gpu(t["u"]), gpu(t["a"]), gpu(t["b"]), gpu(t["B"]),
+                                      gpu(t["C"]), conv_w=gpu(t["conv_w"]),
+                                      conv_b=gpu(t["conv_b"]), z=gpu(t["z"]), D=gpu(t["D"]))
+            assert naju.last_device_status(ws) == 4
+        finally:
+            naju.testing_set_skip_publish(False)
+            naju.testing_set_wait_limit(0)
+        y, xf, _ = run_fwd(t, True, out_dtype=naju.F32)
+    finally:
+        naju.testing_set_fwd_pieces(0)
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_BF16, name="y after timeout")
+
+
 def test_bwd_after_grouped_forward():
     """Checkpoints written by a sequence-split forward serve the backward."""
     w = wl(64, "f32", Bt=1, L=700, d=64)

@@ -391,6 +391,11 @@ def main():
                          "with d_model = d_inner / 2 instead of the scan alone")
     ap.add_argument("--coupled", action="store_true",
                     help="coupled single gate i = 1 - f (no b input)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (a smaller case of the same kernels, "
+                         "for profiling; the JSON line's config shows the sizes)")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="override the workload's sequence length (as --batch)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -398,6 +403,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     w = WORKLOADS[args.workload]
+    if args.batch or args.seqlen:
+        w = scaled(w, batch=args.batch or w.batch, seqlen=args.seqlen or w.seqlen)
     if w.decode_steps:
         if args.impl == "reference":
             run_reference_decode(args, w, rank)
@@ -564,9 +571,9 @@ def main():
     dom_b = bwd_b if dom_is_bwd else fwd_b
     achieved = dom_b / (dom_ms / 1e3) / 1e9
     peak = float(pk["hbm_gbs"])
-    traffic = None
+    traffic = None  # measured for the named workload as benched by default only
     prof = os.path.join(ROOT, "profiles", f"traffic_{w.name}.json")
-    if os.path.exists(prof):
+    if not (args.batch or args.seqlen or args.coupled) and os.path.exists(prof):
         with open(prof) as fh:
             tr = json.load(fh)
         traffic = tr.get("bwd" if dom_is_bwd else "fwd")

@@ -62,6 +62,8 @@ namespace {
 
 constexpr int kBT = 16;                              // tokens per sub-chunk
 constexpr float kBBound = 18446744073709551616.0f;   // 2^64
+// No quarter (4 tokens) above 2^16 means no channel's sub-chunk above 2^64.
+constexpr float kBQuarter = 65536.0f;
 constexpr long long kBSpin = 1LL << 24;
 
 template <int N>
@@ -492,7 +494,10 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
         }
         sm.xq[qd][ch] = Qh;
         sm.xe[qd][ch] = Eh;
-        __syncthreads();
+        // The exchange barrier also ORs a conservative per-quarter test (not
+        // needed by the backward sweep, which reuses the forward sweep's
+        // decision); only when it fires does the exact test take a barrier.
+        const bool maybe_slow = __syncthreads_or(sweep != kSweepBwd && !(Qh <= kBQuarter)) != 0;
         {
             // decay products of the earlier quarters and of the whole sub-chunk
             float Qb = 1.f, Eb = 1.f, Qa = 1.f, Ea = 1.f;
@@ -509,7 +514,7 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
             if (sweep == kSweepBwd) {
                 slow = sm.slowf[sb] != 0;  // same sub-chunk as the forward sweep's
             } else {
-                slow = __syncthreads_or(qd == 0 && !(Qa <= kBBound)) != 0;
+                slow = maybe_slow && __syncthreads_or(qd == 0 && !(Qa <= kBBound)) != 0;
                 if (fwd && tid == 0) sm.slowf[sb] = slow ? 1 : 0;
             }
             Elast = Ea;

@@ -55,6 +55,8 @@ namespace {
 constexpr int kTS = 16;                               // tokens per sub-chunk
 constexpr int kStages = 3;                            // operand stages = raw buffers
 constexpr float kTcBound = 18446744073709551616.0f;   // 2^64
+// No quarter (4 tokens) above 2^16 means no channel's sub-chunk above 2^64.
+constexpr float kTcQuarter = 65536.0f;
 constexpr long long kMbarSpin = 1LL << 24;            // polls before giving up
 
 // Tensor-memory columns (lane = channel).  Per stage: W (readout weights,
@@ -268,7 +270,9 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
         }
         sm.xq[pq][pch] = Qh;
         sm.xe[pq][pch] = Eh;
-        tc::named_bar(1, NPROD);
+        // The exchange barrier also ORs a conservative per-quarter test; only
+        // when it fires does the exact per-sub-chunk test below take a barrier.
+        const bool maybe_slow = tc::named_bar_or(1, NPROD, !(Qh <= kTcQuarter));
         // decay products of the earlier quarters and of the whole sub-chunk
         float Qb = 1.f, Eb = 1.f, Qa = 1.f, Ea = 1.f;
 #pragma unroll
@@ -281,7 +285,8 @@ scan_fwd_tc_kernel(const FwdParams p, const __grid_constant__ FwdTmaps tm) {
             Qa *= xq;
             Ea *= xe;
         }
-        const bool slow = tc::named_bar_or(1, NPROD, pq == 0 && !(Qa <= kTcBound));
+        const bool slow =
+            maybe_slow && tc::named_bar_or(1, NPROD, pq == 0 && !(Qa <= kTcBound));
         if (!slow) {
             if (full && warp == 0) {
                 // G[t][m] = C_t . B_m for m <= t: one warp, tf32 warp-level MMAs.

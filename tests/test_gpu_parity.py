@@ -338,6 +338,25 @@ def test_bwd_tensor_core_exact_fallback(N):
     compare_grads(g, r, True, TOL_BF16)
 
 
+@pytest.mark.parametrize("N", [64, 128])
+def test_tensor_core_moderate_decay_runs(N):
+    """Runs of small forget gates whose 4-token products exceed 2^16 while no
+    16-token product exceeds 2^64: the conservative test on the exchange
+    barrier fires, the exact one keeps the tensor-core path."""
+    w = wl(N, "bf16", Bt=2, L=300, d=136)
+    t = inputs(w, True, use_x0=True, use_dxL=True)
+    a = t["a"].float().clone()
+    a[:, 36:44] = -3.0      # 1/f = 21 per token: 2^17.6 per 4 tokens, 2^35 per 8
+    a[0, 130:134] = -2.9
+    a[1, 201:205] = -3.2
+    t["a"] = a.to(torch.bfloat16)
+    y, xf, _ = run_fwd(t, True, out_dtype=naju.F32)
+    ro, rx = oracle_fwd(t, True)
+    assert_close(y, ro, TOL_BF16, name="y")
+    assert_close(xf, rx, TOL_BF16, name="x_final")
+    compare_grads(run_bwd(t, True, out_dtype=naju.F32), oracle_bwd(t, True), True, TOL_BF16)
+
+
 @pytest.mark.parametrize("groups", [2, 3])
 def test_bwd_tensor_core_sequence_groups(groups):
     w = wl(64, "bf16", Bt=2, L=600, d=136)

@@ -66,6 +66,28 @@ bool use_bwd_tc(const naju_dims* dm) {
     return bwd_tc_supported(dm->dtype, dm->d_state, dm->d_inner);
 }
 
+// Tensor-core kernels run one block per SM, so the launch's last wave
+// decides the time.  Sequence-group count for `units` blocks' worth of work
+// per group over `nseg` 64-token segments: the g (at most 16) with the least
+// modelled time: waves of units * G blocks, G the groups after rounding to
+// whole segments, each over ceil(nseg / g) segments, plus 17 % for the early
+// (backward) or update-only (forward) pass that all but the last group run.
+int tc_groups(int64_t units, int nseg) {
+    int best = 1;
+    double best_cost = 1e30;
+    for (int g = 1; g <= nseg && g <= 16; ++g) {
+        const int64_t per = cdiv(nseg, g), groups = cdiv(nseg, per);
+        const double waves = (double)cdiv(units * groups, kSMs);
+        const double cost =
+            waves * (double)per / nseg * (1.0 + 0.17 * (double)(groups - 1) / groups);
+        if (cost < best_cost - 1e-12) {
+            best_cost = cost;
+            best = g;
+        }
+    }
+    return best;
+}
+
 // Backward tiling: channel tiles, dB/dC partial sets, sequence groups.
 struct BwdTiling {
     int ntiles, nparts, bgroups, blk_per_group, npieces;
@@ -106,8 +128,12 @@ BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
     int gb = g_bwd_groups;
     if (gb <= 0) {
         const int64_t ctas = dm->batch * (int64_t)b.ntiles;
-        const int64_t want = (tc ? 1 : 4) * kSMs;
-        gb = ctas >= want ? 1 : (int)cdiv(want, ctas);
+        if (tc) {
+            gb = tc_groups(ctas, nsub);
+        } else {
+            const int64_t want = 4 * kSMs;
+            gb = ctas >= want ? 1 : (int)cdiv(want, ctas);
+        }
     }
     if (gb > nsub) gb = nsub;
     b.blk_per_group = (int)cdiv(nsub, gb);
@@ -118,9 +144,10 @@ BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
 int auto_groups(const naju_dims* dm, int nck, int ntiles_f, bool tc) {
     if (g_fwd_groups > 0) return g_fwd_groups < nck ? g_fwd_groups : nck;
     const int64_t items = dm->batch * (int64_t)ntiles_f;
-    // Blocks resident per SM: one tensor-core block (its operand stages fill
-    // most of the shared memory), three CUDA-core blocks.
-    const int64_t want = tc ? kSMs : 3 * kSMs;
+    // One tensor-core block per SM (its operand stages fill most of the
+    // shared memory): the wave model; three CUDA-core blocks per SM.
+    if (tc) return tc_groups(items, nck);
+    const int64_t want = 3 * kSMs;
     if (items >= want) return 1;
     int64_t g = cdiv(want, items);
     return (int)(g < nck ? g : nck);

@@ -103,8 +103,9 @@ BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
     } else {
         // Clusters of channel tiles share one partial set; two blocks per SM.
         const int tiles = (int)cdiv(d, bwd_channels_per_block(dm->d_state));
-        b.nparts = (int)cdiv(tiles, bwd_cluster_size());
-        b.ntiles = b.nparts * bwd_cluster_size();
+        const int cl = bwd_cluster_size(tiles);
+        b.nparts = (int)cdiv(tiles, cl);
+        b.ntiles = b.nparts * cl;
     }
     // Tensor-core piece mode: with at least one unit (128 channels of one
     // batch element) per SM but not a whole number of waves, cut the units'

@@ -78,7 +78,7 @@ struct BwdParams {
 
 int fwd_channels_per_block(int64_t N);
 int bwd_channels_per_block(int64_t N);
-int bwd_cluster_size();
+int bwd_cluster_size(int tiles);
 
 cudaError_t launch_scan_fwd(const FwdParams& p, int dtype, int out_dtype, cudaStream_t st);
 // Tensor-core forward (bf16 activations, d_state 64 or 128, 128 channels per block).

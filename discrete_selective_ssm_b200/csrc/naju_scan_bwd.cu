@@ -62,7 +62,9 @@ template <> struct BwdShape<64> { static constexpr int NS = 32, S = 2; };
 template <> struct BwdShape<128> { static constexpr int NS = 32, S = 4; };
 
 int bwd_channels_per_block(int64_t N) { return N <= 32 ? 128 : (N == 64 ? 64 : 32); }
-int bwd_cluster_size() { return kCluster; }
+// Cluster of channel tiles sharing one dB/dC partial set: 2 when the tiles
+// fit (no padding blocks for narrow d_inner), else 8.
+int bwd_cluster_size(int tiles) { return tiles <= 2 ? 2 : kCluster; }
 
 template <typename Tin, int N, int P>
 struct BwdSmem {
@@ -86,7 +88,7 @@ struct BwdSmem {
     int item, ok;
 };
 
-template <typename Tin, typename Tout, int N, bool CONV>
+template <typename Tin, typename Tout, int N, bool CONV, int CL>
 __global__ void __launch_bounds__(128, 2)
 scan_bwd_kernel(const BwdParams p) {
     constexpr int NS = BwdShape<N>::NS, S = BwdShape<N>::S;
@@ -113,7 +115,7 @@ scan_bwd_kernel(const BwdParams p) {
     const int g = p.ngroups - 1 - item / per_g;
     const int bb = (item % per_g) / p.nclus;
     const int cgi = item % p.nclus;
-    const int tile = cgi * kCluster + crank;
+    const int tile = cgi * CL + crank;
     const int64_t c0 = (int64_t)tile * P;
     const int64_t c = c0 + pl;
     const bool cvalid = c < d;
@@ -352,7 +354,7 @@ scan_bwd_kernel(const BwdParams p) {
     // Cluster sum of acc[K][N] into the dB (slot 0) or dC (slot 1) partials.
     auto cluster_reduce = [&](int slot, int64_t tb, int64_t te) {
         cluster.sync();
-        constexpr int ROWS = K / kCluster;
+        constexpr int ROWS = K / CL;
         const int r0 = crank * ROWS;
         float* out = p.dBCp + (((int64_t)cgi * Bt + bb) * L) * 2 * N + slot * N;
         for (int e = tid; e < ROWS * N; e += NT) {
@@ -360,7 +362,7 @@ scan_bwd_kernel(const BwdParams p) {
             const int j = e % N;
             float a = 0.f;
 #pragma unroll
-            for (int qr = 0; qr < kCluster; ++qr)
+            for (int qr = 0; qr < CL; ++qr)
                 a += cluster.map_shared_rank(&sm.acc[0][0], qr)[tt * N + j];
             const int64_t t = tb + tt;
             if (t < te) out[t * 2 * N + j] = a;
@@ -804,24 +806,24 @@ cudaError_t launch_bwd_reductions(const BwdParams& p, int out_dtype, void* dB, v
     return reductions_t<float>(p, dB, dC, dD, dw, dbias, st);
 }
 
-template <typename Tin, typename Tout, int N, bool CONV>
+template <typename Tin, typename Tout, int N, bool CONV, int CL>
 static cudaError_t launch_bwd_t(const BwdParams& p, void* dB, void* dC, float* dD, float* dw,
                                 float* dbias, cudaStream_t st) {
     constexpr int S = BwdShape<N>::S;
     constexpr int P = 128 / S;
     const size_t smem = sizeof(BwdSmem<Tin, N, P>);
-    auto kern = scan_bwd_kernel<Tin, Tout, N, CONV>;
+    auto kern = scan_bwd_kernel<Tin, Tout, N, CONV, CL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.nclus * kCluster), (unsigned)p.Bt, (unsigned)p.ngroups);
+    cfg.gridDim = dim3((unsigned)(p.nclus * CL), (unsigned)p.Bt, (unsigned)p.ngroups);
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kCluster;
+    attr[0].val.clusterDim.x = CL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -834,13 +836,19 @@ static cudaError_t launch_bwd_t(const BwdParams& p, void* dB, void* dC, float* d
 template <typename Tin, typename Tout, bool CONV>
 static cudaError_t launch_bwd_n(const BwdParams& p, void* dB, void* dC, float* dD, float* dw,
                                 float* dbias, cudaStream_t st) {
+    const int cl = p.ntiles / p.nclus;  // blocks per cluster (bwd_cluster_size)
+#define NAJU_BWD_N(NN)                                                                     \
+    return cl == 2 ? launch_bwd_t<Tin, Tout, NN, CONV, 2>(p, dB, dC, dD, dw, dbias, st)  \
+                   : launch_bwd_t<Tin, Tout, NN, CONV, kCluster>(p, dB, dC, dD, dw, dbias, st)
+    if (cl != 2 && cl != kCluster) return cudaErrorInvalidValue;
     switch (p.N) {
-        case 16: return launch_bwd_t<Tin, Tout, 16, CONV>(p, dB, dC, dD, dw, dbias, st);
-        case 32: return launch_bwd_t<Tin, Tout, 32, CONV>(p, dB, dC, dD, dw, dbias, st);
-        case 64: return launch_bwd_t<Tin, Tout, 64, CONV>(p, dB, dC, dD, dw, dbias, st);
-        case 128: return launch_bwd_t<Tin, Tout, 128, CONV>(p, dB, dC, dD, dw, dbias, st);
+        case 16: NAJU_BWD_N(16);
+        case 32: NAJU_BWD_N(32);
+        case 64: NAJU_BWD_N(64);
+        case 128: NAJU_BWD_N(128);
         default: return cudaErrorInvalidValue;
     }
+#undef NAJU_BWD_N
 }
 
 cudaError_t launch_scan_bwd(const BwdParams& p, int dtype, int out_dtype, void* dB, void* dC,

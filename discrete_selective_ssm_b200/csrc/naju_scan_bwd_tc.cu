@@ -704,7 +704,10 @@ scan_bwd_tc_kernel(const BwdParams p, const __grid_constant__ BwdTmaps tm) {
                 }
             }
         }
-        if (!tc::mbar_wait(&sm.mma, mma_phase, kBSpin)) timed_out = true;
+        // One warp (it issues nothing) polls the completion barrier; the rest
+        // wait on the block barrier instead of spinning.
+        if (warp == NT / 32 - 1 && !tc::mbar_wait(&sm.mma, mma_phase, kBSpin)) timed_out = true;
+        __syncthreads();
         mma_phase ^= 1u;
         tc::fence_after_sync();
     };

@@ -47,6 +47,9 @@
 // gradients go through per-(batch, group) channel partials; sequence groups
 // exchange the adjoint carry by a decoupled look-back backwards in time
 // (an adjoint-only early pass, bounded waits), as in the CUDA-core kernel.
+// Piece mode (at least one wave of 128-channel units, not a whole number
+// of waves) instead gives each block one equal range of all units' 64-token
+// blocks; a unit cut in two hands its carry from its tail to its head.
 #include <string.h>
 
 #include <type_traits>

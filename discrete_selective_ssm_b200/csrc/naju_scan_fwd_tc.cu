@@ -39,6 +39,10 @@
 //
 // Sequence groups work as in the CUDA-core kernel: an update-only pass and a
 // decoupled look-back publish each group's end state before the full pass.
+// Piece mode (at least one wave of 128-channel units, not a whole number of
+// waves) instead gives each block one equal range of all units' 64-token
+// checkpoint segments; a unit cut in two hands the state at the cut from its
+// head to its tail.
 #include <string.h>
 
 #include <type_traits>

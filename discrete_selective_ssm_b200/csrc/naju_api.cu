@@ -73,6 +73,7 @@ bool use_bwd_tc(const naju_dims* dm) {
 // whole segments, each over ceil(nseg / g) segments, plus 17 % for the early
 // (backward) or update-only (forward) pass that all but the last group run.
 int tc_groups(int64_t units, int nseg) {
+    if (units >= kSMs) return 1;  // a wave or more: piece mode, or whole waves already
     int best = 1;
     double best_cost = 1e30;
     for (int g = 1; g <= nseg && g <= 16; ++g) {

@@ -168,3 +168,11 @@ def test_tensor_core_group_counts_follow_the_wave_model(L):
     one = naju.make_dims(148, 1024, 128, 64, naju.BF16)  # exactly one wave
     assert naju.testing_fwd_groups(one) == 1 and naju.testing_bwd_groups(one) == 1
     assert naju.testing_bwd_pieces(one) == 0
+    big = naju.make_dims(16, 4096, 2048, 64, naju.BF16)  # 256 units, piece mode off
+    naju.testing_set_fwd_pieces(-1)
+    naju.testing_set_bwd_pieces(-1)
+    try:
+        assert naju.testing_fwd_groups(big) == 1 and naju.testing_bwd_groups(big) == 1
+    finally:
+        naju.testing_set_fwd_pieces(0)
+        naju.testing_set_bwd_pieces(0)

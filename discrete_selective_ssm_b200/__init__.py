@@ -14,4 +14,5 @@ from ._native import (BF16, F32, Dims, NajuError, alloc_workspace, conv_silu_bwd
                       testing_fwd_groups, testing_fwd_impl, testing_fwd_pieces,
                       testing_set_bwd_groups, testing_set_bwd_impl, testing_set_bwd_pieces,
                       testing_set_fwd_groups, testing_set_fwd_impl, testing_set_fwd_pieces,
-                      testing_set_skip_publish, testing_set_wait_limit, workspace_bytes)
+                      testing_set_skip_publish, testing_set_sm_count, testing_set_wait_limit,
+                      testing_sm_count, workspace_bytes)

@@ -363,3 +363,11 @@ def testing_set_fwd_pieces(pieces: int):
 
 def testing_fwd_pieces(dims: Dims) -> int:
     return int(lib().naju_testing_fwd_pieces(ctypes.byref(dims)))
+
+
+def testing_set_sm_count(sms: int):
+    lib().naju_testing_set_sm_count(int(sms))
+
+
+def testing_sm_count() -> int:
+    return int(lib().naju_testing_sm_count())

@@ -4,6 +4,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 
 #include "naju.h"
@@ -15,7 +16,6 @@ using namespace naju;
 
 namespace {
 
-constexpr int kSMs = 148;
 constexpr int kTck = kBwdSub;      // tokens per forward checkpoint segment (= backward block)
 constexpr long long kDefaultWait = 1LL << 21;
 
@@ -27,27 +27,39 @@ int g_bwd_pieces = 0;  // 0 automatic, < 0 never, > 0 that many ranges
 int g_fwd_pieces = 0;  // the same for the tensor-core forward
 int g_fwd_impl = 0;  // 0 automatic, 1 CUDA cores, 2 tensor cores
 int g_bwd_impl = 0;  // 0 automatic, 1 CUDA cores
+int g_sm_override = 0;  // > 0: SM count used by the tiling (tests)
+
+// Streaming multiprocessors of the current device, queried once per device
+// ordinal (the tensor-core kernels run one block per SM, so the tiling below
+// depends on it).  148 (B200) when no device can be queried.
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_cache[kMaxDevices];
+
+int sm_count() {
+    if (g_sm_override > 0) return g_sm_override;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    if (dev < kMaxDevices) {
+        const int c = g_sm_cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        return 148;
+    }
+    if (dev < kMaxDevices) g_sm_cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
 
 inline bool aligned(const void* ptr, size_t a) {
     return (reinterpret_cast<uintptr_t>(ptr) % a) == 0;
 }
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
-
-naju_status check_dims(const naju_dims* dm) {
-    if (!dm) return NAJU_ERR_INVALID_ARG;
-    if (dm->batch < 1 || dm->seqlen < 1 || dm->d_inner < 1 || dm->reserved != 0)
-        return NAJU_ERR_INVALID_ARG;
-    if (dm->batch > (1 << 20) || dm->seqlen > (1LL << 26) || dm->d_inner > (1 << 20))
-        return NAJU_ERR_INVALID_ARG;
-    if (dm->batch * dm->seqlen * dm->d_inner > (1LL << 40)) return NAJU_ERR_INVALID_ARG;
-    if (dm->d_state != 16 && dm->d_state != 32 && dm->d_state != 64 && dm->d_state != 128)
-        return NAJU_ERR_UNSUPPORTED;
-    if (dm->dtype != NAJU_F32 && dm->dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
-    if (dm->out_dtype != NAJU_F32 && dm->out_dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
-    if (dm->dtype == NAJU_F32 && dm->out_dtype != NAJU_F32) return NAJU_ERR_UNSUPPORTED;
-    return NAJU_OK;
-}
 
 // Workspace layout (every region 256-byte aligned).
 struct Layout {
@@ -72,13 +84,13 @@ bool use_bwd_tc(const naju_dims* dm) {
 // modelled time: waves of units * G blocks, G the groups after rounding to
 // whole segments, each over ceil(nseg / g) segments, plus 17 % for the early
 // (backward) or update-only (forward) pass that all but the last group run.
-int tc_groups(int64_t units, int nseg) {
-    if (units >= kSMs) return 1;  // a wave or more: piece mode, or whole waves already
+int tc_groups(int64_t units, int nseg, int sms) {
+    if (units >= sms) return 1;  // a wave or more: piece mode, or whole waves already
     int best = 1;
     double best_cost = 1e30;
     for (int g = 1; g <= nseg && g <= 16; ++g) {
         const int64_t per = cdiv(nseg, g), groups = cdiv(nseg, per);
-        const double waves = (double)cdiv(units * groups, kSMs);
+        const double waves = (double)cdiv(units * groups, sms);
         const double cost =
             waves * (double)per / nseg * (1.0 + 0.17 * (double)(groups - 1) / groups);
         if (cost < best_cost - 1e-12) {
@@ -93,7 +105,7 @@ int tc_groups(int64_t units, int nseg) {
 struct BwdTiling {
     int ntiles, nparts, bgroups, blk_per_group, npieces;
 };
-BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
+BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc, int sms) {
     BwdTiling b{};
     const int64_t d = dm->d_inner;
     if (tc) {
@@ -117,8 +129,8 @@ BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
         int np = 0;
         if (g_bwd_pieces > 0) {
             np = units >= g_bwd_pieces ? g_bwd_pieces : 0;
-        } else if (units >= kSMs && units % kSMs != 0) {
-            np = kSMs;
+        } else if (units >= sms && units % sms != 0) {
+            np = sms;
         }
         if (np > 0) {
             b.npieces = np;
@@ -131,9 +143,9 @@ BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
     if (gb <= 0) {
         const int64_t ctas = dm->batch * (int64_t)b.ntiles;
         if (tc) {
-            gb = tc_groups(ctas, nsub);
+            gb = tc_groups(ctas, nsub, sms);
         } else {
-            const int64_t want = 4 * kSMs;
+            const int64_t want = 4 * (int64_t)sms;
             gb = ctas >= want ? 1 : (int)cdiv(want, ctas);
         }
     }
@@ -143,13 +155,13 @@ BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc) {
     return b;
 }
 
-int auto_groups(const naju_dims* dm, int nck, int ntiles_f, bool tc) {
+int auto_groups(const naju_dims* dm, int nck, int ntiles_f, bool tc, int sms) {
     if (g_fwd_groups > 0) return g_fwd_groups < nck ? g_fwd_groups : nck;
     const int64_t items = dm->batch * (int64_t)ntiles_f;
     // One tensor-core block per SM (its operand stages fill most of the
     // shared memory): the wave model; three CUDA-core blocks per SM.
-    if (tc) return tc_groups(items, nck);
-    const int64_t want = 3 * kSMs;
+    if (tc) return tc_groups(items, nck, sms);
+    const int64_t want = 3 * (int64_t)sms;
     if (items >= want) return 1;
     int64_t g = cdiv(want, items);
     return (int)(g < nck ? g : nck);
@@ -158,26 +170,27 @@ int auto_groups(const naju_dims* dm, int nck, int ntiles_f, bool tc) {
 // Tensor-core forward piece mode: the rule of the backward's (one range of
 // checkpoint segments per SM when the 128-channel units fill at least one
 // wave but not a whole number of them); one flag slot per unit.
-int fwd_pieces(const naju_dims* dm, int nck, int ntiles_f, bool tc) {
+int fwd_pieces(const naju_dims* dm, int nck, int ntiles_f, bool tc, int sms) {
     if (!tc || g_fwd_groups > 0 || g_fwd_pieces < 0 || nck < 2) return 0;
     const int64_t units = dm->batch * (int64_t)ntiles_f;
     if (g_fwd_pieces > 0) return units >= g_fwd_pieces ? g_fwd_pieces : 0;
-    return (units >= kSMs && units % kSMs != 0) ? kSMs : 0;
+    return (units >= sms && units % sms != 0) ? sms : 0;
 }
 
 Layout layout(const naju_dims* dm) {
     Layout l{};
+    const int sms = sm_count();
     const int64_t Bt = dm->batch, L = dm->seqlen, d = dm->d_inner, N = dm->d_state;
     l.nck = (int)cdiv(L, kTck);
     l.fwd_tc = use_fwd_tc(dm);
     l.ntiles_f = (int)cdiv(d, l.fwd_tc ? fwd_tc_channels_per_block() : fwd_channels_per_block(N));
-    l.npieces_f = fwd_pieces(dm, l.nck, l.ntiles_f, l.fwd_tc);
-    int g = l.npieces_f > 0 ? 1 : auto_groups(dm, l.nck, l.ntiles_f, l.fwd_tc);
+    l.npieces_f = fwd_pieces(dm, l.nck, l.ntiles_f, l.fwd_tc, sms);
+    int g = l.npieces_f > 0 ? 1 : auto_groups(dm, l.nck, l.ntiles_f, l.fwd_tc, sms);
     l.seg_per_group = (int)cdiv(l.nck, g);
     l.ngroups = (int)cdiv(l.nck, l.seg_per_group);
     l.nsub = (int)cdiv(L, kBwdSub);
     l.bwd_tc = use_bwd_tc(dm);
-    const BwdTiling bt = bwd_tiling(dm, l.nsub, l.bwd_tc);
+    const BwdTiling bt = bwd_tiling(dm, l.nsub, l.bwd_tc, sms);
     l.ntiles_b = bt.ntiles;
     l.nclus = bt.nparts;
     l.bgroups = bt.bgroups;
@@ -185,7 +198,7 @@ Layout layout(const naju_dims* dm) {
     l.npieces = bt.npieces;
     // Regions sized for the larger of the two backward tilings, so the
     // workspace size does not depend on which backward kernel runs.
-    const BwdTiling bo = bwd_tiling(dm, l.nsub, !l.bwd_tc);
+    const BwdTiling bo = bwd_tiling(dm, l.nsub, !l.bwd_tc, sms);
     const bool other_ok = l.bwd_tc || bwd_tc_supported(dm->dtype, N, d);
     const int64_t flags_n = std::max<int64_t>((int64_t)bt.bgroups * bt.ntiles,
                                               other_ok ? (int64_t)bo.bgroups * bo.ntiles : 0);
@@ -223,6 +236,25 @@ inline bool ok_act(const void* p) { return p && aligned(p, 16); }
 inline bool ok_opt(const void* p) { return !p || aligned(p, 16); }
 
 }  // namespace
+
+namespace naju {
+
+naju_status check_dims(const naju_dims* dm) {
+    if (!dm) return NAJU_ERR_INVALID_ARG;
+    if (dm->batch < 1 || dm->seqlen < 1 || dm->d_inner < 1 || dm->reserved != 0)
+        return NAJU_ERR_INVALID_ARG;
+    if (dm->batch > (1 << 20) || dm->seqlen > (1LL << 26) || dm->d_inner > (1 << 20))
+        return NAJU_ERR_INVALID_ARG;
+    if (dm->batch * dm->seqlen * dm->d_inner > (1LL << 40)) return NAJU_ERR_INVALID_ARG;
+    if (dm->d_state != 16 && dm->d_state != 32 && dm->d_state != 64 && dm->d_state != 128)
+        return NAJU_ERR_UNSUPPORTED;
+    if (dm->dtype != NAJU_F32 && dm->dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
+    if (dm->out_dtype != NAJU_F32 && dm->out_dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
+    if (dm->dtype == NAJU_F32 && dm->out_dtype != NAJU_F32) return NAJU_ERR_UNSUPPORTED;
+    return NAJU_OK;
+}
+
+}  // namespace naju
 
 extern "C" {
 
@@ -435,6 +467,8 @@ int32_t naju_testing_bwd_pieces(const void* dims) {
     if (check_dims(dm) != NAJU_OK) return 0;
     return layout(dm).npieces;
 }
+void naju_testing_set_sm_count(int32_t sms) { g_sm_override = sms > 0 ? sms : 0; }
+int32_t naju_testing_sm_count(void) { return sm_count(); }
 void naju_testing_set_fwd_impl(int32_t impl) { g_fwd_impl = (impl == 1) ? 1 : 0; }
 void naju_testing_set_bwd_impl(int32_t impl) { g_bwd_impl = (impl == 1) ? 1 : 0; }
 int32_t naju_testing_bwd_impl(const void* dims) {

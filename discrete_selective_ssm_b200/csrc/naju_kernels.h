@@ -3,9 +3,15 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "naju.h"
+
 namespace naju {
 
 struct WsHeader;
+
+// Host-side validation of the dims shared by every sequence entry point:
+// NAJU_OK, NAJU_ERR_INVALID_ARG (sizes out of range) or NAJU_ERR_UNSUPPORTED.
+naju_status check_dims(const naju_dims* dm);
 
 constexpr int kFwdChunk = 16;   // tokens staged per forward chunk
 constexpr int kBwdSub = 64;     // tokens per backward work item
@@ -24,7 +30,8 @@ struct FwdParams {
     const float* x0;
     void* y;
     float* x_final;
-    float* ckpt;        // [Bt][nck+1][d][N] fp32 state at segment starts (+ final)
+    float* ckpt;        // [Bt][nck+1][d][N] fp32 state at segment starts (+ final);
+                        // CUDA-core kernel, one group: may be null (no checkpoints)
     int* flags;         // [ngroups][Bt][ntiles]
     WsHeader* hdr;
     int64_t Bt, L, d, N;

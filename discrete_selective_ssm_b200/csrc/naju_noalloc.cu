@@ -8,10 +8,11 @@
 // fixed array in this file, reserved on every GPU when the library's module
 // is loaded and kept until the process exits.
 //
-// The forward's scratch is a work ticket, one ready-flag per (batch, channel
-// tile) and the state at the start and end of each batch element.  With the
-// whole sequence in one group (no sequence split, so no waits between thread
-// blocks) that is kScratchBytes at most; larger problems are rejected.
+// The whole sequence runs as one group on the CUDA-core forward kernel (no
+// sequence split, so no waits between thread blocks), and without
+// checkpoints (nothing can follow with a backward).  The scratch then holds
+// only the work ticket and one ready-flag per (batch, channel tile): problems
+// with more flags than fit in kScratchBytes are rejected.
 #include <mutex>
 
 #include "naju.h"
@@ -31,7 +32,8 @@ std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
 
 // Device address of g_scratch on the current device (looked up once per
-// device, with that device current).
+// device, with that device current, and kept for the life of the process: a
+// cudaDeviceReset invalidates it).
 cudaError_t scratch_address(void** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
@@ -60,15 +62,9 @@ naju_status naju_scan_fwd_noalloc(const naju_dims* dims, const void* hu, const f
                                   const void* B, const void* C, const void* z, const float* D,
                                   const float* x0, void* y, float* x_final, void* stream) {
     using namespace naju;
-    if (!dims || dims->batch < 1 || dims->seqlen < 1 || dims->d_inner < 1 ||
-        dims->reserved != 0 || dims->seqlen > (1LL << 26) || dims->batch > (1 << 20) ||
-        dims->d_inner > (1 << 20))
-        return NAJU_ERR_INVALID_ARG;
+    const naju_status chk = check_dims(dims);  // the workspace forward's own checks
+    if (chk != NAJU_OK) return chk;
     const int64_t N = dims->d_state;
-    if (N != 16 && N != 32 && N != 64 && N != 128) return NAJU_ERR_UNSUPPORTED;
-    if (dims->dtype != NAJU_F32 && dims->dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
-    if (dims->out_dtype != NAJU_F32 && dims->out_dtype != NAJU_BF16) return NAJU_ERR_UNSUPPORTED;
-    if (dims->dtype == NAJU_F32 && dims->out_dtype != NAJU_F32) return NAJU_ERR_UNSUPPORTED;
     if (conv_w && dims->conv_width != 4) return NAJU_ERR_UNSUPPORTED;
     if (!hu || !a || !B || !C || !y) return NAJU_ERR_INVALID_ARG;  // b NULL: coupled gate
     const void* required[] = {hu, a, b, B, C, y};
@@ -80,12 +76,10 @@ naju_status naju_scan_fwd_noalloc(const naju_dims* dims, const void* hu, const f
 
     const int64_t Bt = dims->batch, L = dims->seqlen, d = dims->d_inner;
     const int ntiles = (int)((d + fwd_channels_per_block(N) - 1) / fwd_channels_per_block(N));
-    // One sequence group covering the whole sequence: a single checkpoint
-    // segment of L rounded up to the chunk, so only the start and end
-    // states are stored.
+    // One sequence group covering the whole sequence (a single segment of L
+    // rounded up to the chunk), no checkpoints: the header and the flags.
     const size_t off_flags = sizeof(WsHeader);
-    const size_t off_ck = up256(off_flags + sizeof(int) * (size_t)Bt * ntiles);
-    const size_t need = up256(off_ck + sizeof(float) * (size_t)Bt * 2 * d * N);
+    const size_t need = up256(off_flags + sizeof(int) * (size_t)Bt * ntiles);
     if (need > kScratchBytes) return NAJU_ERR_UNSUPPORTED;  // beyond the fixed scratch
 
     void* base = nullptr;
@@ -102,7 +96,7 @@ naju_status naju_scan_fwd_noalloc(const naju_dims* dims, const void* hu, const f
     FwdParams p{};
     p.hu = hu; p.conv_w = conv_w; p.conv_b = conv_b; p.a = a; p.b = b; p.B = B; p.C = C;
     p.z = z; p.D = D; p.x0 = x0; p.y = y; p.x_final = x_final;
-    p.ckpt = reinterpret_cast<float*>(ws + off_ck);
+    p.ckpt = nullptr;  // no checkpoints
     p.flags = reinterpret_cast<int*>(ws + off_flags);
     p.hdr = hdr;
     p.Bt = Bt; p.L = L; p.d = d; p.N = N;

@@ -110,19 +110,25 @@ naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* co
 /* Allocation-free forward for callers that cannot allocate device memory
  * (for example code running where no allocator is available, or a plugin
  * that is handed only its input and output buffers).  The Naju pages have no
- * counterpart: this is a library convenience.  Same arguments and results as
- * naju_scan_fwd (y, optional x_final), but no workspace: the scratch is a
- * fixed 32 MiB device array inside the library, reserved on every GPU that
- * loads the library until the process exits.  The whole sequence runs as one
- * group, so the scratch holds only a work ticket, per-tile flags and the
- * start and end states: problems needing more than 32 MiB (about
- * batch * d_inner * d_state * 8 bytes) return NAJU_ERR_UNSUPPORTED before any
- * launch.  It writes no checkpoints, so naju_scan_bwd cannot follow it.
+ * counterpart: this is a library convenience.  Same arguments, checks and
+ * results (y, optional x_final) as naju_scan_fwd, but no workspace: the
+ * scratch is a fixed 32 MiB device array inside the library, reserved on
+ * every GPU that loads the library until the process exits.
+ * It always runs the CUDA-core forward kernel with the whole sequence as one
+ * sequence group, whatever the dtype and d_state: bf16 calls with d_state 64
+ * or 128 do not get the tensor-core kernel of naju_scan_fwd, and a small
+ * batch leaves most of the GPU idle, so it is slower than naju_scan_fwd.  It
+ * writes no checkpoints, so naju_scan_bwd cannot follow it.  The scratch
+ * holds a work ticket and one flag per (batch element, channel tile):
+ * batch * ceil(d_inner / P) <= about 8.4 million (P = 128, 64, 64, 32
+ * channels for d_state 16, 32, 64, 128); larger problems return
+ * NAJU_ERR_UNSUPPORTED before any launch.
  * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
- * Every call shares the one array, and each call clears what must start at
- * zero; calls that may overlap on the GPU (other streams, other threads) race
- * on it and must be serialised by the caller. */
+ * that device current) and keeps it until the process exits; make that first
+ * call before any stream capture, and do not call it after a
+ * cudaDeviceReset.  Every call shares the one array, and each call clears
+ * what must start at zero; calls that may overlap on the GPU (other streams,
+ * other threads) race on it and must be serialised by the caller. */
 naju_status naju_scan_fwd_noalloc(const naju_dims* dims, const void* hu, const float* conv_w,
                                   const float* conv_b, const void* a, const void* b,
                                   const void* B, const void* C, const void* z, const float* D,

@@ -58,6 +58,15 @@ void naju_testing_set_fwd_pieces(int32_t pieces);
 /* The forward's number of piece-mode ranges for these dims (0: group mode). */
 int32_t naju_testing_fwd_pieces(const void* dims);
 
+/* Forces the streaming-multiprocessor count that the automatic tiling
+ * (piece mode, the wave model of the sequence-group count) is computed for;
+ * sms <= 0 restores the current device's own count, queried once per device
+ * (148 when no device can be queried). */
+void naju_testing_set_sm_count(int32_t sms);
+
+/* The SM count the tiling currently uses. */
+int32_t naju_testing_sm_count(void);
+
 /* Forward implementation: 0 = automatic (tensor cores for bf16 activations
  * with d_state 64 or 128 and d_inner % 8 == 0, CUDA cores otherwise),
  * 1 = always CUDA cores. */

@@ -13,6 +13,14 @@ def L():
     return naju.lib()
 
 
+@pytest.fixture
+def b200_sms(L):
+    """Tiling rules below are stated for a B200's 148 SMs."""
+    naju.testing_set_sm_count(148)
+    yield
+    naju.testing_set_sm_count(0)
+
+
 def test_exports_every_declared_symbol(L):
     names = naju.declared_symbols()
     assert "naju_scan_fwd" in names and "naju_scan_bwd" in names and "naju_scan_step" in names
@@ -71,7 +79,7 @@ def test_status_strings(L):
         assert L.naju_status_string(code)
 
 
-def test_fwd_group_policy(L):
+def test_fwd_group_policy(L, b200_sms):
     # Few (batch x tile) items split the sequence; many do not.
     few = naju.make_dims(2, 8192, 2048, 128, naju.BF16)
     many = naju.make_dims(64, 4096, 2048, 64, naju.BF16)
@@ -119,7 +127,7 @@ def test_tensor_core_dispatch_rules(L):
     assert naju.testing_bwd_impl(naju.make_dims(2, 64, 256, 64, naju.F32)) == 1
 
 
-def test_backward_piece_mode_rules(L):
+def test_backward_piece_mode_rules(L, b200_sms):
     """The tensor-core backward cuts the units' blocks into one range per SM
     (148) when there are at least that many 128-channel units but not a whole
     number of waves; otherwise it keeps sequence groups."""
@@ -143,7 +151,7 @@ def test_backward_piece_mode_rules(L):
         naju.testing_set_bwd_pieces(0)
 
 
-def test_forward_piece_mode_rules(L):
+def test_forward_piece_mode_rules(L, b200_sms):
     """The tensor-core forward takes piece mode under the backward's rule."""
     dm = naju.make_dims(16, 4096, 2048, 64, naju.BF16)
     assert naju.testing_fwd_pieces(dm) == 148
@@ -157,7 +165,7 @@ def test_forward_piece_mode_rules(L):
         naju.testing_set_fwd_pieces(0)
 
 
-def test_tensor_core_group_counts_follow_the_wave_model(L):
+def test_tensor_core_group_counts_follow_the_wave_model(L, b200_sms):
     """Fewer 128-channel units than SMs: the sequence-group count that packs
     the launch's waves best (mid_lm: 96 units -> 3 groups, 288 blocks, two
     full waves; long_retention: 32 units -> 9 groups, 288 blocks)."""
@@ -176,3 +184,27 @@ def test_tensor_core_group_counts_follow_the_wave_model(L):
     finally:
         naju.testing_set_fwd_pieces(0)
         naju.testing_set_bwd_pieces(0)
+
+
+def test_tiling_follows_the_sm_count(L):
+    """Piece mode and the wave model use the SM count of the device (queried
+    once per device; forced here): 256 units of the bench workload are cut
+    into one range per SM unless they fill whole waves."""
+    dm = naju.make_dims(16, 4096, 2048, 64, naju.BF16)  # 256 units of 128 channels
+    mid = naju.make_dims(8, 2048, 1536, 64, naju.BF16)  # 96 units
+    try:
+        naju.testing_set_sm_count(132)
+        assert naju.testing_sm_count() == 132
+        assert naju.testing_fwd_pieces(dm) == 132 and naju.testing_bwd_pieces(dm) == 132
+        naju.testing_set_sm_count(128)  # two whole waves: no cut
+        assert naju.testing_fwd_pieces(dm) == 0 and naju.testing_bwd_pieces(dm) == 0
+        assert naju.testing_fwd_groups(dm) == 1
+        naju.testing_set_sm_count(96)   # mid_lm fills exactly one wave
+        assert naju.testing_fwd_groups(mid) == 1 and naju.testing_bwd_groups(mid) == 1
+        naju.testing_set_sm_count(1000)  # 96 units on 1000 SMs: more sequence groups
+        assert naju.testing_fwd_groups(mid) > 3 and naju.testing_bwd_groups(mid) > 3
+        # the workspace is sized for the tiling in force
+        assert naju.workspace_bytes(mid) > 0
+    finally:
+        naju.testing_set_sm_count(0)
+    assert naju.testing_sm_count() > 0

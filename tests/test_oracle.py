@@ -361,3 +361,40 @@ def test_block_oracle_finite_differences(coupled):
         if coupled and k in ("W_b", "b_b"):
             continue
         _fd_check(loss, t, k, g[k], rtol=1e-5)
+
+
+@pytest.mark.parametrize("coupled", [False, True])
+def test_block_oracle_forward_independent_composition(coupled):
+    """The block oracle's forward (README block flowchart: normalized token ->
+    input projection -> conv + SiLU -> projections of h -> scan -> SiLU(z)
+    modulation -> output projection -> residual) equals a composition of
+    library routines written independently of it, in fp64: torch rms_norm,
+    linear maps, a depthwise conv1d with left zero padding, torch silu, and
+    the affine-prefix evaluation of the scan (coupled gate: b = -a, since
+    sigma(-a) = 1 - sigma(a)).  Pins the norm (RMS with eps 1e-6 and a
+    learned scale), the order of the u / z split, the bias placement and the
+    residual."""
+    import torch.nn.functional as F
+    from oracle import block as ob
+    r = np.random.default_rng(95)
+    Bt, L, dm, di, N = 2, 9, 6, 5, 4
+    p = {k: v.astype(np.float64) for k, v in ob.init_params(dm, di, N, seed=96).items()}
+    x = r.normal(size=(Bt, L, dm))
+    out, _ = ob.block_fwd(x, p, coupled)
+
+    T = {k: torch.from_numpy(v) for k, v in p.items()}
+    xt = torch.from_numpy(x)
+    xn = F.rms_norm(xt, (dm,), weight=T["norm_w"], eps=1e-6)
+    uz = F.linear(xn, T["W_in"].T)
+    u, z = uz[..., :di], uz[..., di:]
+    pre = F.conv1d(u.transpose(1, 2), T["conv_w"][:, None, :], bias=T["conv_b"],
+                   padding=3, groups=di)[..., :L].transpose(1, 2)
+    h = F.silu(pre)
+    a = F.linear(h, T["W_a"].T, T["b_a"])
+    b = -a if coupled else F.linear(h, T["W_b"].T, T["b_b"])
+    B = F.linear(h, T["W_B"].T)
+    C = F.linear(h, T["W_C"].T)
+    y, _ = scan_fwd_prefix(h.numpy(), a.numpy(), b.numpy(), B.numpy(), C.numpy(),
+                           z.numpy(), p["D"])
+    ref = xt + F.linear(torch.from_numpy(y), T["W_out"].T)
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)

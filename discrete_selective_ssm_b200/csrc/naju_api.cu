@@ -25,8 +25,8 @@ int g_fwd_groups = 0;
 int g_bwd_groups = 0;
 int g_bwd_pieces = 0;  // 0 automatic, < 0 never, > 0 that many ranges
 int g_fwd_pieces = 0;  // the same for the tensor-core forward
-int g_fwd_impl = 0;  // 0 automatic, 1 CUDA cores, 2 tensor cores
-int g_bwd_impl = 0;  // 0 automatic, 1 CUDA cores
+int g_fwd_impl = 0;  // 0 automatic, 1 CUDA cores, 2 tensor-core sub-chunk, 3 block form
+int g_bwd_impl = 0;  // 0 automatic, 1 CUDA cores, 2 tensor-core sub-chunk, 3 block form
 int g_sm_override = 0;  // > 0: SM count used by the tiling (tests)
 
 // Streaming multiprocessors of the current device, queried once per device
@@ -322,6 +322,9 @@ naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* co
     p.scale = 1.0f / std::sqrt((float)dims->d_state);
     p.wait_limit = g_wait_limit;
     p.fault_skip_publish = g_skip_publish;
+    if (l.fwd_tc && g_fwd_impl == 3 &&
+        fwd_blk_supported(dims->dtype, dims->d_state, dims->d_inner, p.T_ck))
+        return cuda_status(launch_scan_fwd_blk(p, dims->out_dtype, s));
     if (l.fwd_tc) return cuda_status(launch_scan_fwd_tc(p, dims->out_dtype, s));
     return cuda_status(launch_scan_fwd(p, dims->dtype, dims->out_dtype, s));
 }
@@ -373,6 +376,13 @@ naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* co
     p.scale = 1.0f / std::sqrt((float)dims->d_state);
     p.wait_limit = g_wait_limit;
     p.fault_skip_publish = g_skip_publish;
+    if (l.bwd_tc && g_bwd_impl == 3 &&
+        bwd_blk_supported(dims->dtype, dims->d_state, dims->d_inner)) {
+        e = launch_scan_bwd_blk(p, dims->out_dtype, s);
+        if (e == cudaSuccess)
+            e = launch_bwd_reductions_acc(p, dims->out_dtype, dB, dC, dD, dconv_w, dconv_b, s);
+        return cuda_status(e);
+    }
     if (l.bwd_tc) {
         e = launch_scan_bwd_tc_main(p, dims->out_dtype, s);
         if (e == cudaSuccess)
@@ -469,17 +479,24 @@ int32_t naju_testing_bwd_pieces(const void* dims) {
 }
 void naju_testing_set_sm_count(int32_t sms) { g_sm_override = sms > 0 ? sms : 0; }
 int32_t naju_testing_sm_count(void) { return sm_count(); }
-void naju_testing_set_fwd_impl(int32_t impl) { g_fwd_impl = (impl == 1) ? 1 : 0; }
-void naju_testing_set_bwd_impl(int32_t impl) { g_bwd_impl = (impl == 1) ? 1 : 0; }
+void naju_testing_set_fwd_impl(int32_t impl) {
+    g_fwd_impl = (impl >= 1 && impl <= 3) ? impl : 0;
+}
+void naju_testing_set_bwd_impl(int32_t impl) {
+    g_bwd_impl = (impl >= 1 && impl <= 3) ? impl : 0;
+}
 int32_t naju_testing_bwd_impl(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);
     if (check_dims(dm) != NAJU_OK) return 0;
-    return use_bwd_tc(dm) ? 2 : 1;
+    if (!use_bwd_tc(dm)) return 1;
+    return (g_bwd_impl == 3 && bwd_blk_supported(dm->dtype, dm->d_state, dm->d_inner)) ? 3 : 2;
 }
 int32_t naju_testing_fwd_impl(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);
     if (check_dims(dm) != NAJU_OK) return 0;
-    return use_fwd_tc(dm) ? 2 : 1;
+    if (!use_fwd_tc(dm)) return 1;
+    return (g_fwd_impl == 3 && fwd_blk_supported(dm->dtype, dm->d_state, dm->d_inner, kTck)) ? 3
+                                                                                           : 2;
 }
 int32_t naju_testing_bwd_groups(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);

@@ -1,0 +1,1081 @@
+// Naju backward scan in block form on the 5th-generation tensor cores
+// (sm_100a, tcgen05, kind::tf32), for bf16 activations with d_state 64.
+//
+// Gradient of the Naju recurrence (Naju reproduction README, "Core
+// equations"): x_n = f_n x_{n-1} + i_n h_n B_n^T, y_n = x_n.C_n/sqrt(N) + D h_n,
+// out = y SiLU(z), h = SiLU(conv(u)); s = 1/sqrt(N), v = i h, dy = dout SiLU(z).
+//
+// A thread block owns 128 channels of one batch element (one channel per
+// tensor-memory lane) and walks its 64-token blocks from the last to the
+// first.  A block needs only the state X entering it (the forward pass's
+// checkpoint) and the adjoint carry H entering its end (H = f_next lambda_next,
+// from the later block).  Relative to the block start, per channel, with
+// E_t = prod_{k<=t} f_k, Q_t = 1/E_t, W_t = v_t Q_t, U_t = s dy_t E_t,
+// H' = E_63 H and G[t][m] = C_t.B_m kept for m <= t:
+//   x_t . C_t       = E_t R_t,   R  = X C^T + W G^T
+//   lambda_t . B_t  = Q_t GB_t,  GB = H' B^T + U G      (G read transposed)
+//   carry out       = U C + H'   (the adjoint carry entering the earlier block)
+//   dC_t = sum_ch U_t X + sum_{m<=t} P[t][m] B_m,     P = U^T W (over channels)
+//   dB_t = sum_ch W_t H' + sum_{t'>=t} P[t'][t] C_t'
+//   dL_t = U_t R_t - W_t GB_t,  (f df)_t = sum_{t'>=t} dL_t' + H . x_63,
+//   da = (f df)(1 - f), dz = dout y SiLU'(z), dh = D dy + i lambda.B,
+//   db = h (lambda.B) i (1 - i), and the conv backward from dp = dh SiLU'(p).
+// Every product runs on the tensor core.  The operands are fp32 tiles in
+// shared memory in one 128-byte swizzled row layout (rows = channels or
+// tokens), which serves as the K-major operand (contraction over its columns)
+// and as the MN-major operand (contraction over its rows: over channels for
+// P, dC, dB, over tokens for the carry and for GB), so no thread ever
+// transposes an operand.  X arrives by TMA from the checkpoint (the copy
+// writes the swizzled layout), everything else is written by the threads.
+// The 64 x 64 products G and P (M = 64) share tensor-memory columns at lane
+// offsets 0 and 16, and later dC^T and dB^T do the same.
+//
+// Threads.  512: warp w handles tensor-memory lanes 32 (w % 4) .. + 31, i.e.
+// channels 32 (w % 4) + lane, and the 16 tokens [16 q, 16 q + 16) of the
+// block, q = w / 4 (and the state columns [16 q, 16 q + 16) where a channel's
+// state row is split).  Per-token inputs are read straight from global
+// memory (prefetched into L2 one block ahead by TMA prefetches); the
+// per-token coefficients the gradients need after the MMAs wait in tensor
+// memory and registers.
+//
+// Exactness.  A block in which some channel's decay product over the block
+// falls below 2^-90 (the factorisation's range) runs an exact token-by-token
+// recurrence instead, on the CUDA cores, and hands its results to the same
+// epilogue through tensor memory.
+//
+// dB and dC: each block adds its channels' partial sums into an fp32
+// accumulator with red.global.add (a small kernel converts it to the output
+// dtype), so no per-tile partial sets go through HBM.  Sequence groups
+// (below one wave of 128-channel units) and piece mode (at least one wave)
+// split the work exactly as in the sub-chunk tensor-core backward.
+#include <stddef.h>
+#include <string.h>
+
+#include "naju_common.cuh"
+#include "naju_kernels.h"
+#include "naju_tc.cuh"
+#include "naju_tma.h"
+
+namespace naju {
+
+namespace {
+
+constexpr int kK = 64;    // tokens per block (the forward's checkpoint spacing)
+constexpr int kP = 128;   // channels per unit
+constexpr int kNT = 512;  // threads
+constexpr float kBound = 1.2379400392853803e27f;  // 2^90
+constexpr float kQuarter = 4194304.f;             // 2^22: four quarters below it stay below 2^88
+constexpr long long kSpin = 1LL << 24;
+
+// Tensor-memory columns (lane = channel unless stated).
+template <int N>
+struct BkCols {
+    static constexpr uint32_t R = 0;        // R[ch][t]           (64)
+    static constexpr uint32_t GB = 64;      // GB[ch][t]          (64)
+    static constexpr uint32_t H = 128;      // carry [ch][j]      (N)
+    static constexpr uint32_t BC = 128 + N; // G / P, then dC^T / dB^T (M = 64 at lanes +0 / +16)
+    static constexpr uint32_t SV = 192 + N; // four per-token coefficients [ch][t] (4 x 64)
+    static constexpr uint32_t USED = SV + 256;
+    static_assert(USED <= 512, "tensor memory");
+};
+
+struct alignas(64) BkTmaps {
+    CUtensorMap u, a, b, z, dy, B, C;  // bf16, for L2 prefetches
+    CUtensorMap X;                     // fp32 checkpoints, 128-byte swizzled box loads
+};
+
+template <int N>
+struct BkSmem {
+    alignas(1024) float X[kP * N];    // checkpoint: rows ch, cols j
+    alignas(1024) float H[kP * N];    // H' = E_63 H: rows ch, cols j
+    alignas(1024) float W[kP * kK];   // rows ch, cols t
+    alignas(1024) float U[kP * kK];   // rows ch, cols t
+    alignas(1024) float Bf[kK * N];   // rows t, cols j
+    alignas(1024) float Cf[kK * N];   // rows t, cols j
+    alignas(1024) float G[kK * kK];   // rows t, cols m (m <= t)
+    alignas(1024) float Pm[kK * kK];  // rows t, cols m (m <= t)
+    float xq[4][kP], xe[4][kP];       // per-quarter decay products
+    float xs[4][kP];                  // per-quarter sums of dL
+    float tailp[2][4][kP];            // partial H . x_63 of the next block to run
+    float dph[4][3][kP];              // first three dp of each quarter
+    float dnext[2][3][kP];            // first three dp of the later block
+    float red6[6][kP];                // per-channel parameter sums
+    uint64_t mb_x, mb0, mb2;
+    uint32_t taddr;
+    int item, ok;
+};
+
+__device__ __forceinline__ float ldbf(const __nv_bfloat16* p) {
+    return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16);
+}
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ void red_add(float* p, float v) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+}  // namespace
+
+template <typename Tout, bool CONV, bool PIECES>
+__global__ void __launch_bounds__(512, 1)
+scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
+    constexpr int N = 64;
+    using Cols = BkCols<N>;
+    using Sm = BkSmem<N>;
+    using Tin = __nv_bfloat16;
+    extern __shared__ __align__(1024) float4 smem4[];
+    Sm& sm = *reinterpret_cast<Sm*>(smem4);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lid = tid & 31;
+    const int s4 = warp & 3;       // tensor-memory sub-partition
+    const int q = warp >> 2;       // token quarter / state-column quarter
+    const int ch = s4 * 32 + lid;  // channel within the unit = TMEM lane
+    const int64_t Bt = p.Bt, L = p.L, d = p.d;
+    const float sc = p.scale;
+    const bool has_z = p.z != nullptr;
+    const bool has_b = p.b != nullptr;
+
+    // ------------------------------------------------------------ set-up
+    if (warp == 0) {
+        tc::tmem_alloc(&sm.taddr, 512);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) {
+        sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
+        tc::mbar_init(&sm.mb_x, 1);
+        tc::mbar_init(&sm.mb0, 1);
+        tc::mbar_init(&sm.mb2, 1);
+        tma::prefetch_map(&tm.X);
+        tma::prefetch_map(&tm.u);
+        tma::prefetch_map(&tm.a);
+        if (has_b) tma::prefetch_map(&tm.b);
+        if (has_z) tma::prefetch_map(&tm.z);
+        tma::prefetch_map(&tm.dy);
+        tma::prefetch_map(&tm.B);
+        tma::prefetch_map(&tm.C);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = sm.taddr;
+    const uint32_t trow = tbase + ((uint32_t)(s4 * 32) << 16);  // this warp's lanes
+    const int item = sm.item;
+    const uint32_t sbase = tc::smem_u32(&sm);
+    const uint32_t aX = sbase + (uint32_t)offsetof(Sm, X), aH = sbase + (uint32_t)offsetof(Sm, H),
+                   aW = sbase + (uint32_t)offsetof(Sm, W), aU = sbase + (uint32_t)offsetof(Sm, U),
+                   aB = sbase + (uint32_t)offsetof(Sm, Bf), aC = sbase + (uint32_t)offsetof(Sm, Cf),
+                   aG = sbase + (uint32_t)offsetof(Sm, G), aP = sbase + (uint32_t)offsetof(Sm, Pm);
+    uint32_t ph_x = 0, ph0 = 0, ph2 = 0;  // mbarrier parities
+    bool timed_out = false;
+
+    // ------------------------------------------------------------ work units
+    constexpr bool pieces = PIECES;  // the launch picks the instantiation by p.npieces
+    int g = 0, bb = 0, tile = 0, kb0 = 0, kb1 = 0;
+    int64_t c0 = 0, c = 0;
+    bool cvalid = false, lastg = true, firstg = true;
+    float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, wb = 0.f, Dc = 0.f;
+    auto set_unit = [&](int u, int g_, int k0, int k1) {
+        g = g_;
+        bb = u / p.ntiles;
+        tile = u % p.ntiles;
+        c0 = (int64_t)tile * kP;
+        c = c0 + ch;
+        cvalid = c < d;
+        kb0 = k0;
+        kb1 = k1;
+        lastg = kb1 == p.nsub;
+        firstg = kb0 == 0;
+        w0 = w1 = w2 = w3 = wb = Dc = 0.f;
+        if (cvalid) {
+            if (CONV) {
+                w0 = p.conv_w[c * 4 + 0];
+                w1 = p.conv_w[c * 4 + 1];
+                w2 = p.conv_w[c * 4 + 2];
+                w3 = p.conv_w[c * 4 + 3];
+                wb = p.conv_b ? p.conv_b[c] : 0.f;
+            }
+            Dc = p.D ? p.D[c] : 0.f;
+        }
+    };
+    const int64_t Wb = Bt * p.ntiles * (int64_t)p.nsub;
+    const int piece = pieces ? p.npieces - 1 - item : 0;
+    const int64_t F0 = pieces ? (int64_t)piece * Wb / p.npieces : 0;
+    const int64_t F1 = pieces ? (int64_t)(piece + 1) * Wb / p.npieces : 0;
+    if (!pieces) {
+        const int per_g = (int)(Bt * p.ntiles);
+        const int gg = p.ngroups - 1 - item / per_g;
+        const int k0 = gg * p.blk_per_group;
+        set_unit(item % per_g, gg, k0, min(k0 + p.blk_per_group, p.nsub));
+    }
+    auto carry_slot = [&](int slot) { return p.carry + ((int64_t)slot * Bt + bb) * d * N; };
+    auto flag_slot = [&](int slot) {
+        return p.flags + ((int64_t)slot * Bt + bb) * p.ntiles + tile;
+    };
+    auto edge_row = [&]() { return p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d; };
+
+    // Global rows of this batch element.
+    auto gin = [&](const void* base) {
+        return static_cast<const Tin*>(base) + (int64_t)bb * L * d + c;
+    };
+    auto gout = [&](void* base) { return static_cast<Tout*>(base) + (int64_t)bb * L * d + c; };
+
+    auto sync = [&]() {
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+    };
+    // TMEM carry columns of this thread (state columns [16 q, 16 q + 16)) <->
+    // a global [d][N] state row.
+    auto carry_from = [&](const float* src, bool cg) {
+        float v[16];
+#pragma unroll
+        for (int k = 0; k < 16; k += 4) {
+            float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (src && cvalid) {
+                const float4* s4p = reinterpret_cast<const float4*>(src + c * N + 16 * q + k);
+                v4 = cg ? __ldcg(s4p) : *s4p;
+            }
+            v[k] = v4.x; v[k + 1] = v4.y; v[k + 2] = v4.z; v[k + 3] = v4.w;
+        }
+        tc::tmem_st16(trow + Cols::H + 16 * q, v);
+        tc::tmem_st_wait();
+    };
+    auto carry_to = [&](float* dst) {
+        float v[16];
+        tc::tmem_ld16(trow + Cols::H + 16 * q, v);
+        tc::tmem_ld_wait();
+        if (cvalid) {
+#pragma unroll
+            for (int k = 0; k < 16; k += 4)
+                *reinterpret_cast<float4*>(dst + c * N + 16 * q + k) =
+                    make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+        }
+    };
+    // X tile of block k by TMA (one thread).
+    auto load_x = [&](int k) {
+        tma::expect_tx(&sm.mb_x, (uint32_t)(sizeof(float) * kP * N));
+        const int z = (int)((int64_t)bb * (p.nck + 1) + k);
+#pragma unroll
+        for (int jb = 0; jb < N / 32; ++jb)
+            tma::load_3d(sm.X + jb * kP * 32, &tm.X, jb * 32, (int)c0, z, &sm.mb_x);
+    };
+    // L2 prefetch of block k's per-token inputs (one thread).
+    auto prefetch_block = [&](int k) {
+        const int x = (int)c0, y = k * kK, zb = bb;
+        tma::prefetch_l2_3d(&tm.u, x, y > 3 ? y - 3 : 0, zb);
+        tma::prefetch_l2_3d(&tm.a, x, y, zb);
+        if (has_b) tma::prefetch_l2_3d(&tm.b, x, y, zb);
+        if (has_z) tma::prefetch_l2_3d(&tm.z, x, y, zb);
+        tma::prefetch_l2_3d(&tm.dy, x, y, zb);
+        tma::prefetch_l2_3d(&tm.B, 0, y, zb);
+        tma::prefetch_l2_3d(&tm.C, 0, y, zb);
+    };
+    // Swizzled row-tile element offsets (floats).
+    auto sw = [](int row, int col, int R) { return tc::sw128_offset(row, col, R) >> 2; };
+
+    // ---------------------------------------------------- loop 1: decays
+    // Per thread: f, q = 1/f of its 16 tokens; exchange of the quarter
+    // products; returns the block's exact-path decision.
+    float fv[16], qv[16];
+    float Eb = 1.f, Qb = 1.f, E63 = 1.f;
+    auto decays = [&](int64_t tb, int nv) -> bool {
+        const Tin* ga = gin(p.a);
+        float Qh = 1.f, Eh = 1.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const int tt = 16 * q + k;
+            const bool valid = cvalid && tt < nv;
+            const float av = valid ? ldbf(ga + (tb + tt) * d) : 0.f;
+            const float ea = __expf(-av);
+            qv[k] = valid ? 1.f + ea : 1.f;
+            fv[k] = valid ? rcpa_(qv[k]) : 1.f;
+            Qh *= qv[k];
+            Eh *= fv[k];
+        }
+        // f and 1/f of these tokens wait in the W / U tiles until the unpack
+        // overwrites them with W and U (same thread, same positions)
+#pragma unroll
+        for (int k = 0; k < 16; k += 4) {
+            *reinterpret_cast<float4*>(&sm.W[sw(ch, 16 * q + k, kP)]) =
+                make_float4(fv[k], fv[k + 1], fv[k + 2], fv[k + 3]);
+            *reinterpret_cast<float4*>(&sm.U[sw(ch, 16 * q + k, kP)]) =
+                make_float4(qv[k], qv[k + 1], qv[k + 2], qv[k + 3]);
+        }
+        sm.xq[q][ch] = Qh;
+        sm.xe[q][ch] = Eh;
+        const bool maybe = __syncthreads_or(!(Qh <= kQuarter)) != 0;
+        float Qa = 1.f, Ea = 1.f;
+        Qb = 1.f;
+        Eb = 1.f;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+            const float xq = sm.xq[qq][ch], xe = sm.xe[qq][ch];
+            if (qq < q) {
+                Qb *= xq;
+                Eb *= xe;
+            }
+            Qa *= xq;
+            Ea *= xe;
+        }
+        E63 = Ea;
+        return maybe && __syncthreads_or(!(Qa <= kBound)) != 0;
+    };
+
+    // ------------------------------------------------ full unpack (loop 2)
+    // Writes W, U (shared), four coefficients per token (tensor memory) and
+    // keeps c0v, c1v (dp = c0 + c1 GB) and the u window in registers.
+    float c0v[16], c1v[16];
+    uint32_t upk[10] = {};  // u at tokens 16q-3 .. 16q+15 (bf16 pairs)
+    float dD_acc = 0.f;  // this block's sum of dy h (added to red6 in phase C)
+    // u of window entry m (token 16q - 3 + m of the block)
+    auto uwin = [&](int m) { return (m & 1) ? bf_hi(upk[m >> 1]) : bf_lo(upk[m >> 1]); };
+    auto unpack = [&](int64_t tb, int nv, bool slow) {
+        const Tin* gu = gin(p.hu);
+        const Tin* gbp = has_b ? gin(p.b) : nullptr;
+        const Tin* gz = has_z ? gin(p.z) : nullptr;
+        const Tin* gdy = gin(p.dy);
+        // u window (bf16 pairs): tokens tb + 16q - 3 + i, i < 19
+        auto ubits = [&](int i) -> uint32_t {
+            const int tt = 16 * q - 3 + i;
+            const int64_t t = tb + tt;
+            const bool ok = cvalid && tt < nv && t >= 0 && (CONV || i >= 3);
+            return ok ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(gu + t * d)) : 0u;
+        };
+#pragma unroll
+        for (int i = 0; i < 10; ++i) upk[i] = ubits(2 * i) | (i < 9 ? ubits(2 * i + 1) << 16 : 0u);
+        float E = slow ? 1.f : Eb, Q = slow ? 1.f : Qb;
+        dD_acc = 0.f;
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+            float Wv[4], Uv[4], s0[4], s1[4], s2[4], s3[4];
+            const int col = 16 * q + 4 * g4;
+            const float4 f4 = *reinterpret_cast<const float4*>(&sm.W[sw(ch, col, kP)]);
+            const float4 q4 = *reinterpret_cast<const float4*>(&sm.U[sw(ch, col, kP)]);
+            const float fa[4] = {f4.x, f4.y, f4.z, f4.w}, qa[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int k = 4 * g4 + k4;
+                const int tt = 16 * q + k;
+                const int64_t t = tb + tt;
+                const bool valid = cvalid && tt < nv;
+                float h, spd = 1.f;
+                if (CONV) {
+                    const float pp = fmaf(w3, uwin(k + 3), fmaf(w2, uwin(k + 2),
+                                         fmaf(w1, uwin(k + 1), fmaf(w0, uwin(k), wb))));
+                    const float sp = sigmoida_(pp);
+                    h = pp * sp;
+                    spd = sp * fmaf(pp, 1.f - sp, 1.f);
+                } else {
+                    h = uwin(k + 3);
+                }
+                if (!valid) h = 0.f;
+                const float f = fa[k4], qq = qa[k4];
+                // 1 - f = (1/f - 1) f, exact for f near 1; 1 where exp(-a) overflowed
+                const float omf = qq < 3.0e38f ? (qq - 1.f) * f : 1.f;
+                const float iw = has_b ? (valid ? sigmoida_(ldbf(gbp + t * d)) : 0.f) : omf;
+                float gg = 1.f, gd = 0.f;
+                if (has_z) {
+                    const float zv = valid ? ldbf(gz + t * d) : 0.f;
+                    const float sz = sigmoida_(zv);
+                    gg = zv * sz;
+                    gd = sz * fmaf(zv, 1.f - sz, 1.f);
+                }
+                const float dout = valid ? ldbf(gdy + t * d) : 0.f;
+                const float dyv = dout * gg;
+                const float dzc = dout * gd;
+                if (!slow) {
+                    E *= f;
+                    Q *= qq;
+                }
+                const float v = iw * h;
+                Wv[k4] = v * Q;
+                Uv[k4] = sc * dyv * E;
+                s0[k4] = sc * dzc * E;                               // dz = s0 R + s1
+                s1[k4] = dzc * Dc * h;
+                s2[k4] = has_b ? h * (1.f - iw) * iw * Q : f * h * Q;  // db = s2 GB
+                s3[k4] = omf;
+                const float c1 = valid ? iw * Q * spd : 0.f;         // dp = c0 + c1 GB
+                const float cc0 = valid ? Dc * dyv * spd : 0.f;
+                c1v[k] = c1;
+                c0v[k] = cc0;
+                dD_acc = fmaf(dyv, h, dD_acc);
+            }
+            *reinterpret_cast<float4*>(&sm.W[sw(ch, col, kP)]) = make_float4(Wv[0], Wv[1], Wv[2], Wv[3]);
+            *reinterpret_cast<float4*>(&sm.U[sw(ch, col, kP)]) = make_float4(Uv[0], Uv[1], Uv[2], Uv[3]);
+            tc::tmem_st4(trow + Cols::SV + 0 * 64 + col, s0);
+            tc::tmem_st4(trow + Cols::SV + 1 * 64 + col, s1);
+            tc::tmem_st4(trow + Cols::SV + 2 * 64 + col, s2);
+            tc::tmem_st4(trow + Cols::SV + 3 * 64 + col, s3);
+        }
+    };
+    // B, C rows of block [tb, tb + nv) to the fp32 tiles (rows t, cols j).
+    auto load_bc = [&](int64_t tb, int nv, bool want_b) {
+        const int e0 = tid * 8;
+        const int tt = e0 / N, j = e0 % N;
+        float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo, clo = lo, chi = lo;
+        if (tt < nv) {
+            const int64_t off = ((int64_t)bb * L + tb + tt) * N + j;
+            const uint4 cr = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.C) + off));
+            clo = make_float4(bf_lo(cr.x), bf_hi(cr.x), bf_lo(cr.y), bf_hi(cr.y));
+            chi = make_float4(bf_lo(cr.z), bf_hi(cr.z), bf_lo(cr.w), bf_hi(cr.w));
+            if (want_b) {
+                const uint4 br = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.B) + off));
+                lo = make_float4(bf_lo(br.x), bf_hi(br.x), bf_lo(br.y), bf_hi(br.y));
+                hi = make_float4(bf_lo(br.z), bf_hi(br.z), bf_lo(br.w), bf_hi(br.w));
+            }
+        }
+        *reinterpret_cast<float4*>(&sm.Cf[sw(tt, j, kK)]) = clo;
+        *reinterpret_cast<float4*>(&sm.Cf[sw(tt, j + 4, kK)]) = chi;
+        if (want_b) {
+            *reinterpret_cast<float4*>(&sm.Bf[sw(tt, j, kK)]) = lo;
+            *reinterpret_cast<float4*>(&sm.Bf[sw(tt, j + 4, kK)]) = hi;
+        }
+    };
+    // H' = E_63 H into the H tile and into the carry accumulator (its
+    // initial value: carry out = U C + H').
+    auto scale_carry = [&]() {
+        float hv[16];
+        tc::tmem_ld16(trow + Cols::H + 16 * q, hv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) hv[j] *= E63;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(&sm.H[sw(ch, 16 * q + j, kP)]) =
+                make_float4(hv[j], hv[j + 1], hv[j + 2], hv[j + 3]);
+        tc::tmem_st16(trow + Cols::H + 16 * q, hv);
+    };
+
+    // --------------------------------------------------------- the MMAs
+    // Descriptors of a row tile with `rows` rows: K-major operand, K step ks
+    // (8 columns); MN-major operand (tile rows = K), K step ks (8 rows).
+    auto kd = [](uint32_t base, int rows, int ks) {
+        return tc::sdesc_sw128(base + (ks >> 2) * rows * 128 + (ks & 3) * 32);
+    };
+    auto md = [](uint32_t base, int rows, int ks) {
+        return tc::sdesc_sw128_mn(base + ks * 1024, rows * 128);
+    };
+    const uint32_t lane16 = 16u << 16;
+    // Batch 0: G = C B^T (lanes +0), P = U^T W (lanes +16), both M = 64.
+    // Batch 1: R = X C^T, GB = H' B^T, carry += U C.
+    auto issue_b01 = [&]() {
+        constexpr uint32_t id64 = tc::idesc_tf32(64, 64);
+        constexpr uint32_t id64mm = tc::idesc_tf32(64, 64, true, true);
+        constexpr uint32_t idR = tc::idesc_tf32(128, 64);
+        constexpr uint32_t idH = tc::idesc_tf32(128, N, false, true);
+#pragma unroll
+        for (int ks = 0; ks < N / 8; ++ks)
+            tc::mma_tf32_ss(tbase + Cols::BC, kd(aC, kK, ks), kd(aB, kK, ks), id64, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < kP / 8; ++ks)
+            tc::mma_tf32_ss(tbase + lane16 + Cols::BC, md(aU, kP, ks), md(aW, kP, ks), id64mm,
+                            ks > 0);
+        tc::mma_commit(&sm.mb0);
+#pragma unroll
+        for (int ks = 0; ks < N / 8; ++ks) {
+            tc::mma_tf32_ss(tbase + Cols::R, kd(aX, kP, ks), kd(aC, kK, ks), idR, ks > 0);
+            tc::mma_tf32_ss(tbase + Cols::GB, kd(aH, kP, ks), kd(aB, kK, ks), idR, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kK / 8; ++ks)
+            tc::mma_tf32_ss(tbase + Cols::H, kd(aU, kP, ks), md(aC, kK, ks), idH, 1u);
+    };
+    // Batch 2: R += W G^T, GB += U G (G transposed), dC^T = X^T U + B^T Pm^T
+    // (lanes +0), dB^T = H'^T W + C^T Pm (lanes +16), all over the masked tiles.
+    auto issue_b2 = [&]() {
+        constexpr uint32_t idR = tc::idesc_tf32(128, 64);
+        constexpr uint32_t idGB = tc::idesc_tf32(128, 64, false, true);
+        constexpr uint32_t idMM = tc::idesc_tf32(64, 64, true, true);
+        constexpr uint32_t idMK = tc::idesc_tf32(64, 64, true, false);
+#pragma unroll
+        for (int ks = 0; ks < kK / 8; ++ks) {
+            tc::mma_tf32_ss(tbase + Cols::R, kd(aW, kP, ks), kd(aG, kK, ks), idR, 1u);
+            tc::mma_tf32_ss(tbase + Cols::GB, kd(aU, kP, ks), md(aG, kK, ks), idGB, 1u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kP / 8; ++ks) {
+            tc::mma_tf32_ss(tbase + Cols::BC, md(aX, kP, ks), md(aU, kP, ks), idMM, ks > 0);
+            tc::mma_tf32_ss(tbase + lane16 + Cols::BC, md(aH, kP, ks), md(aW, kP, ks), idMM,
+                            ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kK / 8; ++ks) {
+            tc::mma_tf32_ss(tbase + Cols::BC, md(aB, kK, ks), kd(aP, kK, ks), idMK, 1u);
+            tc::mma_tf32_ss(tbase + lane16 + Cols::BC, md(aC, kK, ks), md(aP, kK, ks), idMM, 1u);
+        }
+        tc::mma_commit(&sm.mb2);
+    };
+    // G (lanes +0) and P (lanes +16) from tensor memory to their tiles, lower
+    // triangle kept: this warp's lanes, columns [16 q, 16 q + 16).
+    auto copy_gp = [&]() {
+        float v[16];
+        tc::tmem_ld16(trow + Cols::BC + 16 * q, v);
+        tc::tmem_ld_wait();
+        const int row = 16 * s4 + (lid & 15);
+        float* dst = lid < 16 ? sm.G : sm.Pm;
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+            const int col = 16 * q + j;
+            float4 o;
+            o.x = col + 0 <= row ? v[j] : 0.f;
+            o.y = col + 1 <= row ? v[j + 1] : 0.f;
+            o.z = col + 2 <= row ? v[j + 2] : 0.f;
+            o.w = col + 3 <= row ? v[j + 3] : 0.f;
+            *reinterpret_cast<float4*>(&dst[sw(row, col, kK)]) = o;
+        }
+    };
+    auto wait_mb = [&](uint64_t* mb, uint32_t& ph) {
+        // one warp polls; the others wait at the block barrier
+        if (warp == kNT / 32 - 1 && !tc::mbar_wait(mb, ph, kSpin)) timed_out = true;
+        __syncthreads();
+        ph ^= 1u;
+        tc::fence_after_sync();
+    };
+
+    // ---------------------------------------------------- exact path
+    // Token-by-token recurrences for a block outside the factorisation's
+    // range.  W holds v, U holds s dy (E = Q = 1), f = 1 - (saved 1 - f).
+    // Results go where the MMAs would have put them: R <- x.C, GB <- lambda.B,
+    // carry <- f_0 lambda_0; dB and dC are added to the accumulator directly.
+    auto exact_block = [&](int64_t tb, int nv) {
+        float* rsum = sm.G;  // [64 t][128 ch] (G and Pm are adjacent)
+        float* gsum = sm.H;  // [64 t][128 ch]
+        for (int e = tid; e < kK * kP; e += kNT) {
+            rsum[e] = 0.f;
+            gsum[e] = 0.f;
+        }
+        // f of token tt: 1 - (the saved 1 - f), one tensor-memory column each
+        auto f_at = [&](int tt) {
+            const float om = tc::tmem_ld1(trow + Cols::SV + 3 * 64 + tt);
+            return 1.f - om;
+        };
+        float hx[16];
+        tc::tmem_ld16(trow + Cols::H + 16 * q, hx);  // carry entering the block end
+        tc::tmem_ld_wait();
+        float x[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) x[j] = sm.X[sw(ch, 16 * q + j, kP)];
+        __syncthreads();
+        float* acc = p.dBCp + (int64_t)bb * L * 2 * N;
+        for (int tt = 0; tt < nv; ++tt) {
+            const float f = f_at(tt), v = sm.W[sw(ch, tt, kP)], sdy = sm.U[sw(ch, tt, kP)];
+            float rp = 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                x[j] = fmaf(f, x[j], v * sm.Bf[sw(tt, 16 * q + j, kK)]);
+                rp = fmaf(x[j], sm.Cf[sw(tt, 16 * q + j, kK)], rp);
+            }
+            atomicAdd(&rsum[tt * kP + ch], rp);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float r = warp_sum(sdy * x[j]);
+                if (lid == 0) red_add(acc + (tb + tt) * 2 * N + N + 16 * q + j, r);
+            }
+        }
+        for (int tt = nv - 1; tt >= 0; --tt) {
+            const float f = f_at(tt), v = sm.W[sw(ch, tt, kP)], sdy = sm.U[sw(ch, tt, kP)];
+            float gp = 0.f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                hx[j] = fmaf(sdy, sm.Cf[sw(tt, 16 * q + j, kK)], hx[j]);
+                gp = fmaf(hx[j], sm.Bf[sw(tt, 16 * q + j, kK)], gp);
+            }
+            atomicAdd(&gsum[tt * kP + ch], gp);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float r = warp_sum(v * hx[j]);
+                if (lid == 0) red_add(acc + (tb + tt) * 2 * N + 16 * q + j, r);
+                hx[j] *= f;
+            }
+        }
+        tc::tmem_st16(trow + Cols::H + 16 * q, hx);
+        __syncthreads();
+        float rv[16], gv[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            rv[k] = rsum[(16 * q + k) * kP + ch];
+            gv[k] = gsum[(16 * q + k) * kP + ch];
+        }
+        tc::tmem_st16(trow + Cols::R + 16 * q, rv);
+        tc::tmem_st16(trow + Cols::GB + 16 * q, gv);
+        tc::tmem_st_wait();
+        sync();
+    };
+    // Adjoint-only exact block (early pass): W holds f, U holds s dy.
+    auto exact_carry = [&](int nv) {
+        float hx[16];
+        tc::tmem_ld16(trow + Cols::H + 16 * q, hx);
+        tc::tmem_ld_wait();
+        for (int tt = nv - 1; tt >= 0; --tt) {
+            const float f = sm.W[sw(ch, tt, kP)], sdy = sm.U[sw(ch, tt, kP)];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                hx[j] = f * fmaf(sdy, sm.Cf[sw(tt, 16 * q + j, kK)], hx[j]);
+        }
+        tc::tmem_st16(trow + Cols::H + 16 * q, hx);
+        tc::tmem_st_wait();
+        sync();
+    };
+
+    // ============================================================ early pass
+    // Group mode, every group but the first: the adjoint alone over the
+    // group (last block first) from a zero carry (the sequence's dx_final for
+    // the last group), then the carry leaving the group's start is published
+    // after adding the decayed carry of the later group (bounded wait).
+    if (!pieces && !firstg) {
+        const float* dxf = p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr;
+        carry_from(lastg ? dxf : nullptr, false);
+        float logF = 0.f;
+        for (int k = kb1 - 1; k >= kb0; --k) {
+            const int64_t tb = (int64_t)k * kK;
+            const int nv = (int)min64((int64_t)kK, L - tb);
+            if (tid == 0 && k > kb0) prefetch_block(k - 1);
+            const bool slow = decays(tb, nv);
+            // U = s dy E (slow: s dy, and f in W)
+            {
+                const Tin* gz = has_z ? gin(p.z) : nullptr;
+                const Tin* gdy = gin(p.dy);
+                float E = slow ? 1.f : Eb;
+#pragma unroll
+                for (int g4 = 0; g4 < 4; ++g4) {
+                    float Uv[4];
+                    const int col = 16 * q + 4 * g4;
+                    const float4 f4 = *reinterpret_cast<const float4*>(&sm.W[sw(ch, col, kP)]);
+                    const float fa[4] = {f4.x, f4.y, f4.z, f4.w};
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int kk = 4 * g4 + k4, tt = 16 * q + kk;
+                        const bool valid = cvalid && tt < nv;
+                        float gg = 1.f;
+                        if (has_z) {
+                            const float zv = valid ? ldbf(gz + (tb + tt) * d) : 0.f;
+                            gg = zv * sigmoida_(zv);
+                        }
+                        const float dout = valid ? ldbf(gdy + (tb + tt) * d) : 0.f;
+                        if (!slow) E *= fa[k4];
+                        Uv[k4] = sc * dout * gg * E;
+                    }
+                    *reinterpret_cast<float4*>(&sm.U[sw(ch, col, kP)]) =
+                        make_float4(Uv[0], Uv[1], Uv[2], Uv[3]);
+                }
+            }
+            load_bc(tb, nv, false);
+            logF += __logf(E63);
+            if (!slow) {
+                scale_carry();
+                tc::tmem_st_wait();
+                tc::fence_proxy_async();
+                sync();
+                if (tid == 0) {
+                    constexpr uint32_t idH = tc::idesc_tf32(128, N, false, true);
+#pragma unroll
+                    for (int ks = 0; ks < kK / 8; ++ks)
+                        tc::mma_tf32_ss(tbase + Cols::H, kd(aU, kP, ks), md(aC, kK, ks), idH, 1u);
+                    tc::mma_commit(&sm.mb2);
+                }
+                wait_mb(&sm.mb2, ph2);
+            } else {
+                sync();
+                exact_carry(nv);
+            }
+        }
+        if (!lastg) {
+            if (tid == 0) sm.ok = wait_flag(flag_slot(g), &p.hdr->status, p.wait_limit) ? 1 : 0;
+            __syncthreads();
+            const bool okc = sm.ok != 0;
+            const float Pf = __expf(logF);  // decay over the whole group
+            const float* cin = carry_slot(g);
+            float hx[16];
+            tc::tmem_ld16(trow + Cols::H + 16 * q, hx);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 16; k += 4) {
+                float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (okc && cvalid)
+                    v4 = __ldcg(reinterpret_cast<const float4*>(cin + c * N + 16 * q + k));
+                hx[k] = fmaf(Pf, v4.x, hx[k]);
+                hx[k + 1] = fmaf(Pf, v4.y, hx[k + 1]);
+                hx[k + 2] = fmaf(Pf, v4.z, hx[k + 2]);
+                hx[k + 3] = fmaf(Pf, v4.w, hx[k + 3]);
+            }
+            tc::tmem_st16(trow + Cols::H + 16 * q, hx);
+            tc::tmem_st_wait();
+        }
+        carry_to(carry_slot(g - 1));
+        __threadfence();
+        __syncthreads();
+        if (tid == 0 && !(lastg && p.fault_skip_publish)) st_release(flag_slot(g - 1), 1);
+        sync();
+    }
+
+    // ============================================================ main phase
+    const int64_t ub_first = pieces ? (F0 / p.nsub) * p.nsub : 0;
+    const int64_t ub_end = pieces ? F1 : 1;
+    for (int64_t ub = ub_first; ub < ub_end; ub += pieces ? p.nsub : 1) {
+        if (pieces) {
+            const int k0 = (int)(max64(F0, ub) - ub), k1 = (int)(min64(F1, ub + p.nsub) - ub);
+            set_unit((int)(ub / p.nsub), k0 > 0 ? 1 : 0, k0, k1);
+        }
+        // carry entering the segment's end, and the tail H . x at that end
+        if (lastg) {
+            carry_from(p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr, false);
+        } else {
+            const int slot = pieces ? 0 : g;
+            if (tid == 0) sm.ok = wait_flag(flag_slot(slot), &p.hdr->status, p.wait_limit) ? 1 : 0;
+            __syncthreads();
+            carry_from(sm.ok ? carry_slot(slot) : nullptr, true);
+        }
+        int par = 0;  // parity of the block within the segment (double buffers)
+        {
+            // tail of the segment's last block: H . (state at the segment end)
+            float hx[16];
+            tc::tmem_ld16(trow + Cols::H + 16 * q, hx);
+            tc::tmem_ld_wait();
+            const float* xe = p.ckpt + ((int64_t)bb * (p.nck + 1) + kb1) * d * N;
+            float tp = 0.f;
+            if (cvalid) {
+#pragma unroll
+                for (int k = 0; k < 16; k += 4) {
+                    const float4 x4 = __ldcg(reinterpret_cast<const float4*>(xe + c * N + 16 * q + k));
+                    tp = fmaf(hx[k], x4.x, tp);
+                    tp = fmaf(hx[k + 1], x4.y, tp);
+                    tp = fmaf(hx[k + 2], x4.z, tp);
+                    tp = fmaf(hx[k + 3], x4.w, tp);
+                }
+            }
+            sm.tailp[par][q][ch] = tp;
+            if (q == 0) {
+#pragma unroll
+                for (int i = 0; i < 3; ++i) sm.dnext[par][i][ch] = 0.f;
+            }
+        }
+        if (q == 0) {
+#pragma unroll
+            for (int v = 0; v < 6; ++v) sm.red6[v][ch] = 0.f;
+        }
+        if (tid == 0) {
+            load_x(kb1 - 1);
+            prefetch_block(kb1 - 1);
+        }
+        sync();
+
+        for (int k = kb1 - 1; k >= kb0; --k, par ^= 1) {
+            const int64_t tb = (int64_t)k * kK;
+            const int nv = (int)min64((int64_t)kK, L - tb);
+            if (tid == 0 && k > kb0) prefetch_block(k - 1);
+            // ------------------------------------------------ phase A
+            const bool slow = decays(tb, nv);
+            unpack(tb, nv, slow);
+            load_bc(tb, nv, true);
+            if (!slow) scale_carry();
+            tc::tmem_st_wait();
+            tc::fence_proxy_async();
+            sync();
+            // ------------------------------------------------ phase B
+            if (!slow) {
+                if (tid == 0) {
+                    if (!tc::mbar_wait(&sm.mb_x, ph_x, kSpin)) timed_out = true;
+                    issue_b01();
+                }
+                ph_x ^= 1u;
+                wait_mb(&sm.mb0, ph0);
+                copy_gp();
+                tc::fence_proxy_async();
+                sync();
+                if (tid == 0) issue_b2();
+                wait_mb(&sm.mb2, ph2);
+            } else {
+                if (tid == 0 && !tc::mbar_wait(&sm.mb_x, ph_x, kSpin)) timed_out = true;
+                ph_x ^= 1u;
+                sync();
+                exact_block(tb, nv);
+            }
+            // ------------------------------------------------ phase C
+            // Pass 1 (tokens in order): dL, dz, db; the quarter's sum of dL and
+            // its first three dp for the neighbouring quarter.
+            float dL[16];
+            float qsum = 0.f, dpf0 = 0.f, dpf1 = 0.f, dpf2 = 0.f;
+#pragma unroll
+            for (int g4 = 0; g4 < 4; ++g4) {
+                const int col = 16 * q + 4 * g4;
+                float R4[4], G4[4], z1[4], z0[4], b2[4];
+                tc::tmem_ld4(trow + Cols::R + col, R4);
+                tc::tmem_ld4(trow + Cols::GB + col, G4);
+                tc::tmem_ld4(trow + Cols::SV + 0 * 64 + col, z1);
+                tc::tmem_ld4(trow + Cols::SV + 1 * 64 + col, z0);
+                tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
+                tc::tmem_ld_wait();
+                const float4 U4 = *reinterpret_cast<const float4*>(&sm.U[sw(ch, col, kP)]);
+                const float4 W4 = *reinterpret_cast<const float4*>(&sm.W[sw(ch, col, kP)]);
+                const float Ua[4] = {U4.x, U4.y, U4.z, U4.w};
+                const float Wa[4] = {W4.x, W4.y, W4.z, W4.w};
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int kk = 4 * g4 + k4, tt = col + k4;
+                    const int64_t t = tb + tt;
+                    const bool valid = cvalid && tt < nv;
+                    float dl = Ua[k4] * R4[k4] - Wa[k4] * G4[k4];
+                    // coupled gate: (f df) loses f h lambda.B, carried in dL
+                    if (!has_b) dl = fmaf(-b2[k4], G4[k4], dl);
+                    dL[kk] = dl;
+                    qsum += dl;
+                    if (kk == 0) dpf0 = fmaf(c1v[0], G4[k4], c0v[0]);
+                    if (kk == 1) dpf1 = fmaf(c1v[1], G4[k4], c0v[1]);
+                    if (kk == 2) dpf2 = fmaf(c1v[2], G4[k4], c0v[2]);
+                    if (valid) {
+                        if (has_z) gout(p.dz)[t * d] = from_f<Tout>(fmaf(z1[k4], R4[k4], z0[k4]));
+                        if (has_b) gout(p.db)[t * d] = from_f<Tout>(b2[k4] * G4[k4]);
+                    }
+                }
+            }
+            // the coupled term entered qsum: take it out again (it belongs to
+            // this token's da only, not to the sums over later tokens)
+            if (!has_b) {
+                qsum = 0.f;
+#pragma unroll
+                for (int g4 = 0; g4 < 4; ++g4) {
+                    const int col = 16 * q + 4 * g4;
+                    float G4[4], b2[4];
+                    tc::tmem_ld4(trow + Cols::GB + col, G4);
+                    tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) qsum += fmaf(b2[k4], G4[k4], dL[4 * g4 + k4]);
+                }
+            }
+            sm.xs[q][ch] = qsum;
+            sm.dph[q][0][ch] = dpf0;
+            sm.dph[q][1][ch] = dpf1;
+            sm.dph[q][2][ch] = dpf2;
+            __syncthreads();
+            // sums over the later quarters, the tail, the halo of dp
+            float base = 0.f;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                if (qq > q) base += sm.xs[qq][ch];
+                base += sm.tailp[par][qq][ch];
+            }
+            float n1, n2, n3;  // dp of the three tokens after the current one
+            if (q < 3) {
+                n1 = sm.dph[q + 1][0][ch];
+                n2 = sm.dph[q + 1][1][ch];
+                n3 = sm.dph[q + 1][2][ch];
+            } else {
+                n1 = sm.dnext[par][0][ch];
+                n2 = sm.dnext[par][1][ch];
+                n3 = sm.dnext[par][2][ch];
+            }
+            // Pass 2 (tokens in reverse): da from the suffix sums of dL; dp,
+            // the conv backward (du, dw, dbias) from a window of later dp.
+            {
+                float dw0 = 0.f, dw1 = 0.f, dw2 = 0.f, dw3 = 0.f, dbias = 0.f;
+                float run = base;
+                const bool seg_end = !lastg && k == kb1 - 1;
+#pragma unroll
+                for (int g4 = 3; g4 >= 0; --g4) {
+                    const int col = 16 * q + 4 * g4;
+                    float G4[4], om[4], b2[4];
+                    tc::tmem_ld4(trow + Cols::GB + col, G4);
+                    tc::tmem_ld4(trow + Cols::SV + 3 * 64 + col, om);
+                    tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
+                    tc::tmem_ld_wait();
+#pragma unroll
+                    for (int k4 = 3; k4 >= 0; --k4) {
+                        const int kk = 4 * g4 + k4, tt = col + k4;
+                        const int64_t t = tb + tt;
+                        const bool valid = cvalid && tt < nv;
+                        float fdf;
+                        if (has_b) {
+                            run += dL[kk];
+                            fdf = run;
+                        } else {  // dL[kk] holds dL - f h lambda.B
+                            const float cpl = b2[k4] * G4[k4];
+                            fdf = run + dL[kk];
+                            run += dL[kk] + cpl;
+                        }
+                        const float dpv = fmaf(c1v[kk], G4[k4], c0v[kk]);
+                        if (valid) gout(p.da)[t * d] = from_f<Tout>(fdf * om[k4]);
+                        if (CONV) {
+                            const float duv = fmaf(w3, dpv, fmaf(w2, n1, fmaf(w1, n2, w0 * n3)));
+                            if (valid) {
+                                dw0 = fmaf(dpv, uwin(kk), dw0);
+                                dw1 = fmaf(dpv, uwin(kk + 1), dw1);
+                                dw2 = fmaf(dpv, uwin(kk + 2), dw2);
+                                dw3 = fmaf(dpv, uwin(kk + 3), dw3);
+                                dbias += dpv;
+                                if (seg_end && tt >= nv - 3) {
+                                    edge_row()[(3 + (tt - (nv - 3))) * d + c] = duv;  // fixed up later
+                                } else {
+                                    gout(p.dhu)[t * d] = from_f<Tout>(duv);
+                                }
+                                if (k == kb0 && tt < 3) edge_row()[tt * d + c] = dpv;
+                            }
+                            n3 = n2;
+                            n2 = n1;
+                            n1 = dpv;
+                        } else if (valid) {
+                            gout(p.dhu)[t * d] = from_f<Tout>(dpv);
+                        }
+                    }
+                }
+                if (cvalid) {
+                    atomicAdd(&sm.red6[0][ch], dD_acc);
+                    if (CONV) {
+                        atomicAdd(&sm.red6[1][ch], dw0);
+                        atomicAdd(&sm.red6[2][ch], dw1);
+                        atomicAdd(&sm.red6[3][ch], dw2);
+                        atomicAdd(&sm.red6[4][ch], dw3);
+                        atomicAdd(&sm.red6[5][ch], dbias);
+                    }
+                }
+            }
+            // dC^T (lanes +0) and dB^T (lanes +16): this warp's lanes, columns
+            // [16 q, 16 q + 16), added into the accumulator
+            if (!slow) {
+                float v[16];
+                tc::tmem_ld16(trow + Cols::BC + 16 * q, v);
+                tc::tmem_ld_wait();
+                const int j = 16 * s4 + (lid & 15);
+                const int slot = lid < 16 ? 1 : 0;  // slot 0 dB, 1 dC
+                float* acc = p.dBCp + (int64_t)bb * L * 2 * N + slot * N + j;
+#pragma unroll
+                for (int k2 = 0; k2 < 16; ++k2) {
+                    const int tt = 16 * q + k2;
+                    if (tt < nv) red_add(acc + (tb + tt) * 2 * N, v[k2]);
+                }
+            }
+            // tail of the earlier block: (carry entering it) . (this block's X)
+            {
+                float hx[16];
+                tc::tmem_ld16(trow + Cols::H + 16 * q, hx);
+                tc::tmem_ld_wait();
+                float tp = 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) {
+                    const float4 x4 = *reinterpret_cast<const float4*>(&sm.X[sw(ch, 16 * q + j, kP)]);
+                    tp = fmaf(hx[j], x4.x, tp);
+                    tp = fmaf(hx[j + 1], x4.y, tp);
+                    tp = fmaf(hx[j + 2], x4.z, tp);
+                    tp = fmaf(hx[j + 3], x4.w, tp);
+                }
+                sm.tailp[par ^ 1][q][ch] = tp;
+                if (q == 0) {
+                    sm.dnext[par ^ 1][0][ch] = dpf0;
+                    sm.dnext[par ^ 1][1][ch] = dpf1;
+                    sm.dnext[par ^ 1][2][ch] = dpf2;
+                }
+            }
+            sync();  // X, W, U, H tiles and tensor memory free for the next block
+            if (tid == 0 && k > kb0) load_x(k - 1);
+        }
+
+        // ------------------------------------------- carries and partials
+        if (firstg) {
+            if (p.dx0) carry_to(p.dx0 + (int64_t)bb * d * N);
+        } else if (pieces) {
+            carry_to(carry_slot(0));
+            __threadfence();
+            __syncthreads();
+            if (tid == 0 && !p.fault_skip_publish) st_release(flag_slot(0), 1);
+        }
+        {
+            float* cpart = p.chan_part + ((int64_t)bb * p.ngroups + g) * d * 8;
+            __syncthreads();
+            if (tid < kP && c0 + tid < d) {
+#pragma unroll
+                for (int v = 0; v < 6; ++v) cpart[(c0 + tid) * 8 + v] = sm.red6[v][tid];
+                if (pieces && firstg && lastg) {  // uncut unit: its tail slot stays empty
+                    float* cp1 = p.chan_part + ((int64_t)bb * p.ngroups + 1) * d * 8;
+#pragma unroll
+                    for (int v = 0; v < 6; ++v) cp1[(c0 + tid) * 8 + v] = 0.f;
+                }
+            }
+            sync();
+        }
+    }
+
+    if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
+    sync();
+    if (warp == 0) tc::tmem_dealloc(tbase, 512);
+}
+
+// dB, dC from the fp32 accumulator [Bt][L][2][N] (slot 0 dB, 1 dC).
+template <typename Tout>
+__global__ void finish_dBC_kernel(const float* __restrict__ acc, int64_t BtL, int64_t N,
+                                  Tout* __restrict__ dB, Tout* __restrict__ dC) {
+    const int64_t n4 = BtL * N / 4;
+    for (int64_t i4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4;
+         i4 += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = i4 * 4, row = i / N, j = i % N;
+        const float4 b4 = *reinterpret_cast<const float4*>(acc + row * 2 * N + j);
+        const float4 c4 = *reinterpret_cast<const float4*>(acc + row * 2 * N + N + j);
+        dB[i] = from_f<Tout>(b4.x); dB[i + 1] = from_f<Tout>(b4.y);
+        dB[i + 2] = from_f<Tout>(b4.z); dB[i + 3] = from_f<Tout>(b4.w);
+        dC[i] = from_f<Tout>(c4.x); dC[i + 1] = from_f<Tout>(c4.y);
+        dC[i + 2] = from_f<Tout>(c4.z); dC[i + 3] = from_f<Tout>(c4.w);
+    }
+}
+
+template <typename Tout, bool CONV, bool PIECES>
+static cudaError_t launch_blk_t(const BwdParams& p, cudaStream_t st) {
+    constexpr int N = 64;
+    BkTmaps tm;
+    memset(&tm, 0, sizeof(tm));
+    bool ok = tma_encode_bf16_3d(&tm.u, p.hu, p.Bt, p.L, p.d, kK + 3, kP) &&
+              tma_encode_bf16_3d(&tm.a, p.a, p.Bt, p.L, p.d, kK, kP) &&
+              (!p.b || tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, kK, kP)) &&
+              (!p.z || tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, kK, kP)) &&
+              tma_encode_bf16_3d(&tm.dy, p.dy, p.Bt, p.L, p.d, kK, kP) &&
+              tma_encode_bf16_3d(&tm.B, p.B, p.Bt, p.L, N, kK, N) &&
+              tma_encode_bf16_3d(&tm.C, p.C, p.Bt, p.L, N, kK, N) &&
+              tma_encode_f32_3d_sw128(&tm.X, p.ckpt, p.Bt * (int64_t)(p.nck + 1), p.d, N, kP);
+    if (!ok) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(BkSmem<N>);
+    auto kern = scan_bwd_blk_kernel<Tout, CONV, PIECES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = p.npieces > 0 ? p.npieces : p.ngroups * (int)p.Bt * p.ntiles;
+    kern<<<grid, kNT, smem, st>>>(p, tm);
+    return cudaGetLastError();
+}
+
+bool bwd_blk_supported(int dtype, int64_t N, int64_t d) {
+    return dtype == NAJU_BF16 && N == 64 && d % 8 == 0;
+}
+
+cudaError_t launch_scan_bwd_blk(const BwdParams& p, int out_dtype, cudaStream_t st) {
+    // the dB / dC accumulator starts at zero
+    cudaError_t e = cudaMemsetAsync(p.dBCp, 0, sizeof(float) * (size_t)p.Bt * p.L * 2 * p.N, st);
+    if (e != cudaSuccess) return e;
+    const bool conv = p.conv_w != nullptr, pc = p.npieces > 0;
+    if (out_dtype == NAJU_BF16) {
+        using T = __nv_bfloat16;
+        return conv ? (pc ? launch_blk_t<T, true, true>(p, st) : launch_blk_t<T, true, false>(p, st))
+                    : (pc ? launch_blk_t<T, false, true>(p, st) : launch_blk_t<T, false, false>(p, st));
+    }
+    return conv ? (pc ? launch_blk_t<float, true, true>(p, st)
+                      : launch_blk_t<float, true, false>(p, st))
+                : (pc ? launch_blk_t<float, false, true>(p, st)
+                      : launch_blk_t<float, false, false>(p, st));
+}
+
+cudaError_t launch_finish_dBC(const BwdParams& p, int out_dtype, void* dB, void* dC,
+                              cudaStream_t st) {
+    const int64_t BtL = p.Bt * p.L;
+    if (out_dtype == NAJU_BF16)
+        finish_dBC_kernel<__nv_bfloat16><<<592, 256, 0, st>>>(
+            p.dBCp, BtL, p.N, static_cast<__nv_bfloat16*>(dB), static_cast<__nv_bfloat16*>(dC));
+    else
+        finish_dBC_kernel<float><<<592, 256, 0, st>>>(p.dBCp, BtL, p.N, static_cast<float*>(dB),
+                                                       static_cast<float*>(dC));
+    return cudaGetLastError();
+}
+
+}  // namespace naju

@@ -100,6 +100,19 @@ bool bwd_tc_supported(int dtype, int64_t N, int64_t d);
 cudaError_t launch_scan_bwd_tc_main(const BwdParams& p, int out_dtype, cudaStream_t st);
 cudaError_t launch_bwd_reductions(const BwdParams& p, int out_dtype, void* dB, void* dC,
                                   float* dD, float* dw, float* dbias, cudaStream_t st);
+// Block-form tensor-core forward (bf16 activations, d_state 64 or 128,
+// checkpoints every 64 tokens).
+bool fwd_blk_supported(int dtype, int64_t N, int64_t d, int T_ck);
+cudaError_t launch_scan_fwd_blk(const FwdParams& p, int out_dtype, cudaStream_t st);
+// Block-form tensor-core backward (bf16 activations, d_state 64): dB / dC go
+// into an fp32 accumulator [Bt][L][2][N] at p.dBCp (zeroed by the launch);
+// launch_bwd_reductions_acc then finishes dB, dC and the per-channel sums.
+bool bwd_blk_supported(int dtype, int64_t N, int64_t d);
+cudaError_t launch_scan_bwd_blk(const BwdParams& p, int out_dtype, cudaStream_t st);
+cudaError_t launch_finish_dBC(const BwdParams& p, int out_dtype, void* dB, void* dC,
+                              cudaStream_t st);
+cudaError_t launch_bwd_reductions_acc(const BwdParams& p, int out_dtype, void* dB, void* dC,
+                                      float* dD, float* dw, float* dbias, cudaStream_t st);
 cudaError_t launch_conv_fwd(int64_t Bt, int64_t L, int64_t d, const void* u, const float* w,
                             const float* bias, void* h, int dtype, int out_dtype,
                             cudaStream_t st);

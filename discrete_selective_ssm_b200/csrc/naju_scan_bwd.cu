@@ -786,13 +786,21 @@ __global__ void conv_edge_kernel(const float* __restrict__ edge, const float* __
 
 // The follow-up kernels of a backward: dB / dC from the channel-tile partials
 // (p.nclus partial sets), the per-channel sums, the conv group-boundary fixups.
+// acc: dB / dC are already summed in an fp32 accumulator (one set).
 template <typename Tout>
 static cudaError_t reductions_t(const BwdParams& p, void* dB, void* dC, float* dD, float* dw,
-                                float* dbias, cudaStream_t st) {
+                                float* dbias, cudaStream_t st, bool acc = false) {
     const bool conv = p.conv_w != nullptr;
     const int64_t BtL = p.Bt * p.L;
-    reduce_dBC_kernel<Tout><<<592, 256, 0, st>>>(p.dBCp, p.nclus, BtL, p.N,
-                                                  static_cast<Tout*>(dB), static_cast<Tout*>(dC));
+    if (acc) {
+        cudaError_t e = launch_finish_dBC(p, std::is_same<Tout, float>::value ? NAJU_F32 : NAJU_BF16,
+                                          dB, dC, st);
+        if (e != cudaSuccess) return e;
+    } else {
+        reduce_dBC_kernel<Tout><<<592, 256, 0, st>>>(p.dBCp, p.nclus, BtL, p.N,
+                                                      static_cast<Tout*>(dB),
+                                                      static_cast<Tout*>(dC));
+    }
     reduce_chan_kernel<<<(unsigned)((p.d + 127) / 128), 128, 0, st>>>(
         p.chan_part, p.Bt * p.ngroups, p.d, dD, conv ? dw : nullptr, conv ? dbias : nullptr);
     if (conv && p.npieces > 0)
@@ -804,6 +812,13 @@ static cudaError_t reductions_t(const BwdParams& p, void* dB, void* dC, float* d
                                                      (int64_t)p.blk_per_group * kBwdSub, p.L,
                                                      p.d, static_cast<Tout*>(p.dhu));
     return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_reductions_acc(const BwdParams& p, int out_dtype, void* dB, void* dC,
+                                      float* dD, float* dw, float* dbias, cudaStream_t st) {
+    if (out_dtype == NAJU_BF16)
+        return reductions_t<__nv_bfloat16>(p, dB, dC, dD, dw, dbias, st, true);
+    return reductions_t<float>(p, dB, dC, dD, dw, dbias, st, true);
 }
 
 cudaError_t launch_bwd_reductions(const BwdParams& p, int out_dtype, void* dB, void* dC,

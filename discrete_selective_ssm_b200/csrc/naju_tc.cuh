@@ -56,10 +56,28 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: D fp32, A and B tf32, both K-major, M x N.
-__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
-    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+// Descriptor of a 128-byte swizzled operand with explicit leading and
+// stride byte offsets.  Used for the MN-major form of a row tile (see
+// sw128_offset): the tile's rows are the operand's K index and its columns
+// the M (or N) index, so one MMA K step (8 tf32) is one 8-row group at
+// base + ks * 1024, the 32-element M / N blocks are LBO = rows * 128 bytes
+// apart and successive 8-row groups SBO = 1024 bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor: D fp32, A and B tf32, M x N; a_mn / b_mn select the
+// MN-major form of the shared-memory A / B operand (K-major otherwise).
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn = false,
+                                                  bool b_mn = false) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -126,6 +144,16 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float* v) {
                  "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
                  "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
                  : "memory");
+}
+// One 32-bit column of this warp's 32 lanes (waits for the load).
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r)
+                 : "r"(taddr)
+                 : "memory");
+    return __uint_as_float(r);
 }
 // 4 consecutive 32-bit columns of this warp's 32 lanes <-> 4 registers.
 __device__ __forceinline__ void tmem_ld4(uint32_t taddr, float* v) {

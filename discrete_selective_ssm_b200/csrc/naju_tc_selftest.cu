@@ -138,7 +138,104 @@ tc_selftest_ss_kernel(const float* __restrict__ A, const float* __restrict__ B,
     if (warp == 0) tc::tmem_dealloc(tbase, ncols);
 }
 
+// General form: D = A[M x K] * B[N x K]^T with both operands in shared
+// memory as 128-byte swizzled row tiles (sw128_offset).  a_mn = 0: A is
+// stored as the tile A[m][k] (K-major); a_mn = 1: as the tile A^T[k][m]
+// (MN-major).  Likewise b_mn for B.  M = 64 or 128; d_lane (0 or 16) is the
+// lane offset of D in tensor memory.  Every lane of the D columns is copied
+// out raw (D_out[128][N]), so the test can check the accumulator layout.
+__global__ void __launch_bounds__(128, 1)
+tc_selftest_gen_kernel(const float* __restrict__ A, const float* __restrict__ B,
+                       float* __restrict__ D, int M, int N, int K, int a_mn, int b_mn,
+                       int d_lane, uint32_t ncols, int* status) {
+    extern __shared__ __align__(1024) float4 smem4[];
+    unsigned char* sa = reinterpret_cast<unsigned char*>(smem4);
+    unsigned char* sb = sa + (size_t)M * K * 4;
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t taddr_s;
+    const int tid = threadIdx.x, warp = tid / 32;
+
+    if (warp == 0) {
+        tc::tmem_alloc(&taddr_s, ncols);
+        tc::tmem_relinquish();
+    }
+    if (tid == 0) tc::mbar_init(&mbar, 1);
+    for (int e = tid; e < M * K; e += 128) {
+        const int m = e / K, k = e % K;
+        const uint32_t off = a_mn ? tc::sw128_offset(k, m, K) : tc::sw128_offset(m, k, M);
+        *reinterpret_cast<float*>(sa + off) = A[e];
+    }
+    for (int e = tid; e < N * K; e += 128) {
+        const int n = e / K, k = e % K;
+        const uint32_t off = b_mn ? tc::sw128_offset(k, n, K) : tc::sw128_offset(n, k, N);
+        *reinterpret_cast<float*>(sb + off) = B[e];
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tbase = taddr_s;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    // zero the D columns of every lane (the MMA overwrites only its own lanes)
+    for (int n0 = 0; n0 < N; n0 += 16) {
+        float z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0.f;
+        tc::tmem_st16(tbase + lane_off + n0, z);
+    }
+    tc::tmem_st_wait();
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0) {
+        const uint32_t idesc = tc::idesc_tf32(M, N, a_mn != 0, b_mn != 0);
+        const uint32_t abase = tc::smem_u32(sa), bbase = tc::smem_u32(sb);
+        for (int ks = 0; ks < K / 8; ++ks) {
+            const uint64_t ad = a_mn ? tc::sdesc_sw128_mn(abase + ks * 1024, K * 128)
+                                     : tc::sdesc_sw128(abase + (ks >> 2) * M * 128 + (ks & 3) * 32);
+            const uint64_t bd = b_mn ? tc::sdesc_sw128_mn(bbase + ks * 1024, K * 128)
+                                     : tc::sdesc_sw128(bbase + (ks >> 2) * N * 128 + (ks & 3) * 32);
+            tc::mma_tf32_ss(tbase + ((uint32_t)d_lane << 16), ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&mbar);
+    }
+    const bool done = tc::mbar_wait(&mbar, 0, 1LL << 22);
+    if (!done && tid == 0) atomicOr(status, 1 << NAJU_ERR_TIMEOUT);
+    tc::fence_after_sync();
+    for (int n0 = 0; n0 < N; n0 += 16) {
+        float v[16];
+        tc::tmem_ld16(tbase + lane_off + n0, v);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) D[tid * N + n0 + i] = done ? v[i] : __int_as_float(0x7fc00000);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tbase, ncols);
+}
+
 }  // namespace naju
+
+extern "C" naju_status naju_testing_tc_mma_gen(int32_t M, int32_t N, int32_t K, int32_t a_mn,
+                                               int32_t b_mn, int32_t d_lane, const float* A,
+                                               const float* B, float* D, int* status,
+                                               void* stream) {
+    if (!A || !B || !D || !status) return NAJU_ERR_INVALID_ARG;
+    if ((M != 64 && M != 128) || N < 16 || N > 128 || N % 16 != 0 || K < 32 || K > 128 ||
+        K % 32 != 0)
+        return NAJU_ERR_UNSUPPORTED;
+    if (b_mn && N % 32 != 0) return NAJU_ERR_UNSUPPORTED;  // MN-major: 32-element blocks
+    if (d_lane != 0 && !(d_lane == 16 && M == 64)) return NAJU_ERR_UNSUPPORTED;
+    uint32_t ncols = 32;
+    while (ncols < (uint32_t)N) ncols <<= 1;
+    const size_t smem = sizeof(float) * ((size_t)M * K + (size_t)N * K);
+    cudaError_t e = cudaFuncSetAttribute(naju::tc_selftest_gen_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return NAJU_ERR_CUDA;
+    naju::tc_selftest_gen_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
+        A, B, D, M, N, K, a_mn, b_mn, d_lane, ncols, status);
+    return cudaGetLastError() == cudaSuccess ? NAJU_OK : NAJU_ERR_CUDA;
+}
 
 extern "C" naju_status naju_testing_tc_mma(int32_t N, int32_t K, const float* A, const float* B,
                                            float* D, int* status, void* stream) {

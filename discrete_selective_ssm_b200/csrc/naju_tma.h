@@ -20,6 +20,14 @@ namespace naju {
 bool tma_encode_bf16_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows,
                         int64_t cols, int box_rows, int box_cols);
 
+// Encode a 3-D fp32 tensor map [outer][rows][cols] whose box is box_rows rows
+// of 32 columns (128 bytes), written to shared memory in the 128-byte swizzled
+// layout: box row r lands at byte 128 r with its 16-byte chunks XOR-permuted
+// by r % 8 (the destination must be 1024-byte aligned).  Requirements
+// (checked): base 16-byte aligned, cols * 4 a multiple of 16, box_rows <= 256.
+bool tma_encode_f32_3d_sw128(CUtensorMap* map, const void* base, int64_t outer, int64_t rows,
+                             int64_t cols, int box_rows);
+
 #ifdef __CUDACC__
 namespace tma {
 
@@ -45,6 +53,16 @@ __device__ __forceinline__ void load_3d(void* dst, const CUtensorMap* map, int x
             static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z),
         "r"(static_cast<uint32_t>(__cvta_generic_to_shared(mbar)))
+        : "memory");
+}
+
+// Hint: bring the box at (x, y, z) into L2 (no shared memory, no completion
+// signal).  Coordinates outside the tensor are ignored.
+__device__ __forceinline__ void prefetch_l2_3d(const CUtensorMap* map, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(z)
         : "memory");
 }
 

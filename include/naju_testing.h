@@ -69,20 +69,23 @@ int32_t naju_testing_sm_count(void);
 
 /* Forward implementation: 0 = automatic (tensor cores for bf16 activations
  * with d_state 64 or 128 and d_inner % 8 == 0, CUDA cores otherwise),
- * 1 = always CUDA cores. */
+ * 1 = always CUDA cores, 2 = the tensor-core sub-chunk kernel, 3 = the
+ * tensor-core block-form kernel, where tensor cores apply. */
 void naju_testing_set_fwd_impl(int32_t impl);
 
-/* The forward implementation for these dims: 1 = CUDA cores, 2 = tensor
- * cores (0 for invalid dims). */
+/* The forward implementation for these dims: 1 = CUDA cores, 2 = tensor-core
+ * sub-chunk kernel, 3 = tensor-core block-form kernel (0 for invalid dims). */
 int32_t naju_testing_fwd_impl(const void* dims);
 
 /* Backward implementation: 0 = automatic (tensor cores for bf16 activations
- * with d_state 64 or 128 and d_inner % 8 == 0, CUDA cores otherwise),
- * 1 = always CUDA cores. */
+ * with d_state 64 or 128 and d_inner % 8 == 0: the block-form kernel for
+ * d_state 64, the sub-chunk kernel for 128; CUDA cores otherwise),
+ * 1 = always CUDA cores, 2 = the tensor-core sub-chunk kernel where tensor
+ * cores apply. */
 void naju_testing_set_bwd_impl(int32_t impl);
 
-/* The backward implementation for these dims: 1 = CUDA cores, 2 = tensor
- * cores (0 for invalid dims). */
+/* The backward implementation for these dims: 1 = CUDA cores, 2 = tensor-core
+ * sub-chunk kernel, 3 = tensor-core block-form kernel (0 for invalid dims). */
 int32_t naju_testing_bwd_impl(const void* dims);
 
 /* Self-test of the tensor-core building block of the tensor-core scans:
@@ -102,6 +105,18 @@ naju_status naju_testing_tc_mma(int32_t N, int32_t K, const float* A, const floa
 naju_status naju_testing_tc_mma_ss(int32_t N, int32_t K, int32_t rows_a, int32_t swz_a,
                                    int32_t swz_b, const float* A, const float* B, float* D,
                                    int* status, void* stream);
+
+/* General form of the same product, both operands in shared memory as
+ * 128-byte swizzled tiles: a_mn = 0 stores A as its [M x K] tile (K-major
+ * operand), a_mn = 1 as the transposed [K x M] tile (MN-major operand);
+ * likewise b_mn for B.  M is 64 or 128; d_lane (0, or 16 with M = 64) is the
+ * tensor-memory lane offset of D.  D receives all 128 tensor-memory lanes of
+ * the N result columns, row-major [128 x N], so the caller can check where
+ * an M = 64 result lands.  K in {32, 64, 96, 128}; N a multiple of 16 up to
+ * 128 (of 32 when b_mn). */
+naju_status naju_testing_tc_mma_gen(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn,
+                                    int32_t d_lane, const float* A, const float* B, float* D,
+                                    int* status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -62,3 +62,47 @@ def test_tc_mma_tf32_shared_operands(N, K, rows_a, swz_a, swz_b):
     got = dD.cpu().double().numpy()[:rows_a]
     err = np.max(np.abs(got - ref)) / np.max(np.abs(ref))
     assert err < 4e-3, err
+
+
+def _tmem_rows(M, d_lane):
+    """TMEM lane of each result row: M = 128 fills lanes 0-127 in order; M = 64
+    fills 16 lanes of each 32-lane sub-partition (rows 16 s + i -> lane
+    32 s + i + d_lane)."""
+    if M == 128:
+        return list(range(128))
+    return [32 * (r // 16) + (r % 16) + d_lane for r in range(64)]
+
+
+@pytest.mark.parametrize("M,N,K,a_mn,b_mn,d_lane", [
+    (128, 64, 64, 0, 0, 0), (128, 64, 64, 1, 0, 0), (128, 64, 64, 0, 1, 0),
+    (128, 64, 128, 1, 1, 0), (128, 128, 64, 1, 1, 0), (128, 32, 96, 1, 0, 0),
+    (64, 64, 64, 0, 0, 0), (64, 64, 64, 1, 1, 0), (64, 64, 128, 1, 0, 16),
+    (64, 64, 64, 0, 1, 16), (64, 32, 32, 1, 1, 16), (64, 128, 64, 1, 1, 0)])
+def test_tc_mma_tf32_mn_major_and_m64(M, N, K, a_mn, b_mn, d_lane):
+    """MN-major (transposed) shared operands, M = 64 accumulators and their
+    placement at lane offset 16, against a host product."""
+    L = naju.lib()
+    f = L.naju_testing_tc_mma_gen
+    f.argtypes = [ctypes.c_int32] * 6 + [ctypes.c_void_p] * 5
+    f.restype = ctypes.c_int
+    g = torch.Generator().manual_seed(M * 7 + N * 1000 + K * 10 + a_mn * 2 + b_mn + d_lane)
+    A = torch.randn(M, K, generator=g)
+    B = torch.randn(N, K, generator=g)
+    dA, dB = A.cuda(), B.cuda()
+    dD = torch.full((128, N), float("nan"), device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rc = f(M, N, K, a_mn, b_mn, d_lane, ctypes.c_void_p(dA.data_ptr()),
+           ctypes.c_void_p(dB.data_ptr()), ctypes.c_void_p(dD.data_ptr()),
+           ctypes.c_void_p(st.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref = A.double().numpy() @ B.double().numpy().T
+    raw = dD.cpu().double().numpy()
+    lanes = _tmem_rows(M, d_lane)
+    got = raw[lanes]
+    err = np.max(np.abs(got - ref)) / np.max(np.abs(ref))
+    assert err < 4e-3, err
+    others = sorted(set(range(128)) - set(lanes))
+    if others:  # lanes outside the result keep the zeros written before the MMA
+        assert np.all(raw[others] == 0.0)

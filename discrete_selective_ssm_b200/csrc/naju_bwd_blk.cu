@@ -20,22 +20,24 @@
 //   dL_t = U_t R_t - W_t GB_t,  (f df)_t = sum_{t'>=t} dL_t' + H . x_63,
 //   da = (f df)(1 - f), dz = dout y SiLU'(z), dh = D dy + i lambda.B,
 //   db = h (lambda.B) i (1 - i), and the conv backward from dp = dh SiLU'(p).
-// Every product runs on the tensor core.  The operands are fp32 tiles in
-// shared memory in one 128-byte swizzled row layout (rows = channels or
-// tokens), which serves as the K-major operand (contraction over its columns)
-// and as the MN-major operand (contraction over its rows: over channels for
-// P, dC, dB, over tokens for the carry and for GB), so no thread ever
-// transposes an operand.  X arrives by TMA from the checkpoint (the copy
-// writes the swizzled layout), everything else is written by the threads.
-// The 64 x 64 products G and P (M = 64) share tensor-memory columns at lane
-// offsets 0 and 16, and later dC^T and dB^T do the same.
+// Every product runs on the tensor core (kind::f16, fp32 accumulation).  Each
+// fp32 operand is held as a pair of bf16 tiles, hi = bf16(v) and
+// lo = bf16(v - hi), and a product takes the three terms hi.hi + hi.lo + lo.hi
+// (about 2^-16 relative error, finer than tf32); B and C are bf16 inputs and
+// exact in one tile.  The tiles are 128-byte swizzled row tiles (rows =
+// channels or tokens); for 16-bit elements the same bytes serve as the K-major
+// operand (contraction over the columns) and as the MN-major operand
+// (contraction over the rows: over channels for P, dC, dB, over tokens for
+// the carry and for GB), so no thread ever transposes an operand.  The 64 x 64
+// products G and P (M = 64) share tensor-memory columns at lane offsets 0 and
+// 16, and later dC^T and dB^T do the same.
 //
 // Threads.  512: warp w handles tensor-memory lanes 32 (w % 4) .. + 31, i.e.
 // channels 32 (w % 4) + lane, and the 16 tokens [16 q, 16 q + 16) of the
 // block, q = w / 4 (and the state columns [16 q, 16 q + 16) where a channel's
-// state row is split).  Per-token inputs are read straight from global
-// memory (prefetched into L2 one block ahead by TMA prefetches); the
-// per-token coefficients the gradients need after the MMAs wait in tensor
+// state row is split).  Per-token inputs and the checkpoint are read straight
+// from global memory (prefetched into L2 one block ahead by TMA prefetches);
+// the per-token coefficients the gradients need after the MMAs wait in tensor
 // memory and registers.
 //
 // Exactness.  A block in which some channel's decay product over the block
@@ -55,52 +57,50 @@
 #include "naju_kernels.h"
 #include "naju_tc.cuh"
 #include "naju_tma.h"
-
 namespace naju {
 
 namespace {
 
 constexpr int kK = 64;    // tokens per block (the forward's checkpoint spacing)
 constexpr int kP = 128;   // channels per unit
+constexpr int kN = 64;    // d_state
 constexpr int kNT = 512;  // threads
 constexpr float kBound = 1.2379400392853803e27f;  // 2^90
 constexpr float kQuarter = 4194304.f;             // 2^22: four quarters below it stay below 2^88
 constexpr long long kSpin = 1LL << 24;
 
 // Tensor-memory columns (lane = channel unless stated).
-template <int N>
 struct BkCols {
-    static constexpr uint32_t R = 0;        // R[ch][t]           (64)
-    static constexpr uint32_t GB = 64;      // GB[ch][t]          (64)
-    static constexpr uint32_t H = 128;      // carry [ch][j]      (N)
-    static constexpr uint32_t BC = 128 + N; // G / P, then dC^T / dB^T (M = 64 at lanes +0 / +16)
-    static constexpr uint32_t SV = 192 + N; // four per-token coefficients [ch][t] (4 x 64)
-    static constexpr uint32_t USED = SV + 256;
-    static_assert(USED <= 512, "tensor memory");
+    static constexpr uint32_t R = 0;     // R[ch][t]           (64)
+    static constexpr uint32_t GB = 64;   // GB[ch][t]          (64)
+    static constexpr uint32_t H = 128;   // carry [ch][j]      (64)
+    static constexpr uint32_t BC = 192;  // G / P, then dC^T / dB^T (M = 64 at lanes +0 / +16)
+    // four per-token coefficients [ch][t]: s dzc E, dzc D h, the db (coupled:
+    // da) coefficient, 1 - f; slots 2 and 3 first hold f and 1/f
+    static constexpr uint32_t SV = 256;
 };
 
 struct alignas(64) BkTmaps {
     CUtensorMap u, a, b, z, dy, B, C;  // bf16, for L2 prefetches
-    CUtensorMap X;                     // fp32 checkpoints, 128-byte swizzled box loads
+    CUtensorMap X;                     // fp32 checkpoints, for L2 prefetches
 };
 
-template <int N>
+// bf16 operand tiles (hi / lo pairs of the fp32 operands), 1024-byte aligned.
 struct BkSmem {
-    alignas(1024) float X[kP * N];    // checkpoint: rows ch, cols j
-    alignas(1024) float H[kP * N];    // H' = E_63 H: rows ch, cols j
-    alignas(1024) float W[kP * kK];   // rows ch, cols t
-    alignas(1024) float U[kP * kK];   // rows ch, cols t
-    alignas(1024) float Bf[kK * N];   // rows t, cols j
-    alignas(1024) float Cf[kK * N];   // rows t, cols j
-    alignas(1024) float G[kK * kK];   // rows t, cols m (m <= t)
-    alignas(1024) float Pm[kK * kK];  // rows t, cols m (m <= t)
-    float xq[4][kP], xe[4][kP];       // per-quarter decay products
-    float xs[4][kP];                  // per-quarter sums of dL
-    float tailp[2][4][kP];            // partial H . x_63 of the next block to run
-    float dph[4][3][kP];              // first three dp of each quarter
-    float dnext[2][3][kP];            // first three dp of the later block
-    float red6[6][kP];                // per-channel parameter sums
-    uint64_t mb_x, mb0, mb2;
+    alignas(1024) __nv_bfloat16 Xh[kP * kN], Xl[kP * kN];  // checkpoint: rows ch, cols j
+    alignas(1024) __nv_bfloat16 Hh[kP * kN], Hl[kP * kN];  // H' = E_63 H: rows ch, cols j
+    alignas(1024) __nv_bfloat16 Wh[kP * kK], Wl[kP * kK];  // rows ch, cols t
+    alignas(1024) __nv_bfloat16 Uh[kP * kK], Ul[kP * kK];  // rows ch, cols t
+    alignas(1024) __nv_bfloat16 Bs[kK * kN], Cs[kK * kN];  // rows t, cols j (exact)
+    alignas(1024) __nv_bfloat16 Gh[kK * kK], Gl[kK * kK];  // rows t, cols m (m <= t)
+    alignas(1024) __nv_bfloat16 Ph[kK * kK], Pl[kK * kK];  // rows t, cols m (m <= t)
+    float xq[4][kP], xe[4][kP];   // per-quarter decay products
+    float xs[4][kP];              // per-quarter sums of dL
+    float tailp[2][4][kP];        // partial H . x_63 of the next block to run
+    float dph[4][3][kP];          // first three dp of each quarter
+    float dnext[2][3][kP];        // first three dp of the later block
+    float red6[6][kP];            // per-channel parameter sums
+    uint64_t mb0, mb2;
     uint32_t taddr;
     int item, ok;
 };
@@ -118,15 +118,53 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ void red_add(float* p, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
+// hi = bf16(a, b) (round to nearest), lo = bf16 of the remainders.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+// Four consecutive values (row, col .. col + 3; col % 4 == 0) into a tile pair.
+__device__ __forceinline__ void st4(__nv_bfloat16* th, __nv_bfloat16* tl, int row, int col,
+                                    float v0, float v1, float v2, float v3) {
+    uint32_t h0, l0, h1, l1;
+    split2(v0, v1, h0, l0);
+    split2(v2, v3, h1, l1);
+    const uint32_t o = tc::bf_offset(row, col);
+    *reinterpret_cast<uint2*>(reinterpret_cast<char*>(th) + o) = make_uint2(h0, h1);
+    *reinterpret_cast<uint2*>(reinterpret_cast<char*>(tl) + o) = make_uint2(l0, l1);
+}
+// Four consecutive values (hi + lo) back from a tile pair.
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16* th, const __nv_bfloat16* tl, int row,
+                                      int col) {
+    const uint32_t o = tc::bf_offset(row, col);
+    const uint2 h = *reinterpret_cast<const uint2*>(reinterpret_cast<const char*>(th) + o);
+    const uint2 l = *reinterpret_cast<const uint2*>(reinterpret_cast<const char*>(tl) + o);
+    return make_float4(bf_lo(h.x) + bf_lo(l.x), bf_hi(h.x) + bf_hi(l.x), bf_lo(h.y) + bf_lo(l.y),
+                       bf_hi(h.y) + bf_hi(l.y));
+}
+// One value (hi + lo) back from a tile pair, and one value of an exact tile.
+__device__ __forceinline__ float ld1(const __nv_bfloat16* th, const __nv_bfloat16* tl, int row,
+                                     int col) {
+    const uint32_t o = tc::bf_offset(row, col);
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(th) + o)) +
+           __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(tl) + o));
+}
+__device__ __forceinline__ float ld1(const __nv_bfloat16* t, int row, int col) {
+    return __bfloat162float(
+        *reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(t) + tc::bf_offset(row, col)));
+}
 
 }  // namespace
 
 template <typename Tout, bool CONV, bool PIECES>
 __global__ void __launch_bounds__(512, 1)
 scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
-    constexpr int N = 64;
-    using Cols = BkCols<N>;
-    using Sm = BkSmem<N>;
+    constexpr int N = kN;
+    using Cols = BkCols;
+    using Sm = BkSmem;
     using Tin = __nv_bfloat16;
     extern __shared__ __align__(1024) float4 smem4[];
     Sm& sm = *reinterpret_cast<Sm*>(smem4);
@@ -148,7 +186,6 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     }
     if (tid == 0) {
         sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
-        tc::mbar_init(&sm.mb_x, 1);
         tc::mbar_init(&sm.mb0, 1);
         tc::mbar_init(&sm.mb2, 1);
         tma::prefetch_map(&tm.X);
@@ -167,11 +204,8 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     const uint32_t trow = tbase + ((uint32_t)(s4 * 32) << 16);  // this warp's lanes
     const int item = sm.item;
     const uint32_t sbase = tc::smem_u32(&sm);
-    const uint32_t aX = sbase + (uint32_t)offsetof(Sm, X), aH = sbase + (uint32_t)offsetof(Sm, H),
-                   aW = sbase + (uint32_t)offsetof(Sm, W), aU = sbase + (uint32_t)offsetof(Sm, U),
-                   aB = sbase + (uint32_t)offsetof(Sm, Bf), aC = sbase + (uint32_t)offsetof(Sm, Cf),
-                   aG = sbase + (uint32_t)offsetof(Sm, G), aP = sbase + (uint32_t)offsetof(Sm, Pm);
-    uint32_t ph_x = 0, ph0 = 0, ph2 = 0;  // mbarrier parities
+#define NAJU_SA(f) (sbase + (uint32_t)offsetof(Sm, f))
+    uint32_t ph0 = 0, ph2 = 0;  // mbarrier parities
     bool timed_out = false;
 
     // ------------------------------------------------------------ work units
@@ -218,12 +252,11 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         return p.flags + ((int64_t)slot * Bt + bb) * p.ntiles + tile;
     };
     auto edge_row = [&]() { return p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d; };
-
-    // Global rows of this batch element.
     auto gin = [&](const void* base) {
         return static_cast<const Tin*>(base) + (int64_t)bb * L * d + c;
     };
     auto gout = [&](void* base) { return static_cast<Tout*>(base) + (int64_t)bb * L * d + c; };
+    auto ck_at = [&](int k) { return p.ckpt + ((int64_t)bb * (p.nck + 1) + k) * d * N; };
 
     auto sync = [&]() {
         tc::fence_before_sync();
@@ -257,15 +290,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
         }
     };
-    // X tile of block k by TMA (one thread).
-    auto load_x = [&](int k) {
-        tma::expect_tx(&sm.mb_x, (uint32_t)(sizeof(float) * kP * N));
-        const int z = (int)((int64_t)bb * (p.nck + 1) + k);
-#pragma unroll
-        for (int jb = 0; jb < N / 32; ++jb)
-            tma::load_3d(sm.X + jb * kP * 32, &tm.X, jb * 32, (int)c0, z, &sm.mb_x);
-    };
-    // L2 prefetch of block k's per-token inputs (one thread).
+    // L2 prefetch of block k's inputs (one thread).
     auto prefetch_block = [&](int k) {
         const int x = (int)c0, y = k * kK, zb = bb;
         tma::prefetch_l2_3d(&tm.u, x, y > 3 ? y - 3 : 0, zb);
@@ -275,17 +300,17 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tma::prefetch_l2_3d(&tm.dy, x, y, zb);
         tma::prefetch_l2_3d(&tm.B, 0, y, zb);
         tma::prefetch_l2_3d(&tm.C, 0, y, zb);
+        tma::prefetch_l2_3d(&tm.X, 0, x, (int)((int64_t)bb * (p.nck + 1) + k));
+        tma::prefetch_l2_3d(&tm.X, 32, x, (int)((int64_t)bb * (p.nck + 1) + k));
     };
-    // Swizzled row-tile element offsets (floats).
-    auto sw = [](int row, int col, int R) { return tc::sw128_offset(row, col, R) >> 2; };
 
     // ---------------------------------------------------- loop 1: decays
-    // Per thread: f, q = 1/f of its 16 tokens; exchange of the quarter
-    // products; returns the block's exact-path decision.
-    float fv[16], qv[16];
+    // f and 1/f of this thread's 16 tokens, parked in tensor memory (slots 2
+    // and 3); exchange of the quarter products; the exact-path decision.
     float Eb = 1.f, Qb = 1.f, E63 = 1.f;
     auto decays = [&](int64_t tb, int nv) -> bool {
         const Tin* ga = gin(p.a);
+        float fv[16], qv[16];
         float Qh = 1.f, Eh = 1.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -298,15 +323,8 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             Qh *= qv[k];
             Eh *= fv[k];
         }
-        // f and 1/f of these tokens wait in the W / U tiles until the unpack
-        // overwrites them with W and U (same thread, same positions)
-#pragma unroll
-        for (int k = 0; k < 16; k += 4) {
-            *reinterpret_cast<float4*>(&sm.W[sw(ch, 16 * q + k, kP)]) =
-                make_float4(fv[k], fv[k + 1], fv[k + 2], fv[k + 3]);
-            *reinterpret_cast<float4*>(&sm.U[sw(ch, 16 * q + k, kP)]) =
-                make_float4(qv[k], qv[k + 1], qv[k + 2], qv[k + 3]);
-        }
+        tc::tmem_st16(trow + Cols::SV + 2 * 64 + 16 * q, fv);
+        tc::tmem_st16(trow + Cols::SV + 3 * 64 + 16 * q, qv);
         sm.xq[q][ch] = Qh;
         sm.xe[q][ch] = Eh;
         const bool maybe = __syncthreads_or(!(Qh <= kQuarter)) != 0;
@@ -324,15 +342,16 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             Ea *= xe;
         }
         E63 = Ea;
+        tc::tmem_st_wait();
         return maybe && __syncthreads_or(!(Qa <= kBound)) != 0;
     };
 
     // ------------------------------------------------ full unpack (loop 2)
-    // Writes W, U (shared), four coefficients per token (tensor memory) and
-    // keeps c0v, c1v (dp = c0 + c1 GB) and the u window in registers.
+    // Writes the W, U tile pairs, four coefficients per token (tensor memory)
+    // and keeps c0v, c1v (dp = c0 + c1 GB) and the u window in registers.
     float c0v[16], c1v[16];
     uint32_t upk[10] = {};  // u at tokens 16q-3 .. 16q+15 (bf16 pairs)
-    float dD_acc = 0.f;  // this block's sum of dy h (added to red6 in phase C)
+    float dD_acc = 0.f;     // this block's sum of dy h (added to red6 in phase C)
     // u of window entry m (token 16q - 3 + m of the block)
     auto uwin = [&](int m) { return (m & 1) ? bf_hi(upk[m >> 1]) : bf_lo(upk[m >> 1]); };
     auto unpack = [&](int64_t tb, int nv, bool slow) {
@@ -340,7 +359,6 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         const Tin* gbp = has_b ? gin(p.b) : nullptr;
         const Tin* gz = has_z ? gin(p.z) : nullptr;
         const Tin* gdy = gin(p.dy);
-        // u window (bf16 pairs): tokens tb + 16q - 3 + i, i < 19
         auto ubits = [&](int i) -> uint32_t {
             const int tt = 16 * q - 3 + i;
             const int64_t t = tb + tt;
@@ -353,11 +371,11 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         dD_acc = 0.f;
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
-            float Wv[4], Uv[4], s0[4], s1[4], s2[4], s3[4];
+            float Wv[4], Uv[4], s0[4], s1[4], s2[4], s3[4], fa[4], qa[4];
             const int col = 16 * q + 4 * g4;
-            const float4 f4 = *reinterpret_cast<const float4*>(&sm.W[sw(ch, col, kP)]);
-            const float4 q4 = *reinterpret_cast<const float4*>(&sm.U[sw(ch, col, kP)]);
-            const float fa[4] = {f4.x, f4.y, f4.z, f4.w}, qa[4] = {q4.x, q4.y, q4.z, q4.w};
+            tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, fa);
+            tc::tmem_ld4(trow + Cols::SV + 3 * 64 + col, qa);
+            tc::tmem_ld_wait();
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
                 const int k = 4 * g4 + k4;
@@ -396,48 +414,49 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 const float v = iw * h;
                 Wv[k4] = v * Q;
                 Uv[k4] = sc * dyv * E;
-                s0[k4] = sc * dzc * E;                               // dz = s0 R + s1
+                s0[k4] = sc * dzc * E;                                // dz = s0 R + s1
                 s1[k4] = dzc * Dc * h;
                 s2[k4] = has_b ? h * (1.f - iw) * iw * Q : f * h * Q;  // db = s2 GB
                 s3[k4] = omf;
-                const float c1 = valid ? iw * Q * spd : 0.f;         // dp = c0 + c1 GB
-                const float cc0 = valid ? Dc * dyv * spd : 0.f;
-                c1v[k] = c1;
-                c0v[k] = cc0;
+                c1v[k] = valid ? iw * Q * spd : 0.f;                  // dp = c0 + c1 GB
+                c0v[k] = valid ? Dc * dyv * spd : 0.f;
                 dD_acc = fmaf(dyv, h, dD_acc);
             }
-            *reinterpret_cast<float4*>(&sm.W[sw(ch, col, kP)]) = make_float4(Wv[0], Wv[1], Wv[2], Wv[3]);
-            *reinterpret_cast<float4*>(&sm.U[sw(ch, col, kP)]) = make_float4(Uv[0], Uv[1], Uv[2], Uv[3]);
+            st4(sm.Wh, sm.Wl, ch, col, Wv[0], Wv[1], Wv[2], Wv[3]);
+            st4(sm.Uh, sm.Ul, ch, col, Uv[0], Uv[1], Uv[2], Uv[3]);
             tc::tmem_st4(trow + Cols::SV + 0 * 64 + col, s0);
             tc::tmem_st4(trow + Cols::SV + 1 * 64 + col, s1);
             tc::tmem_st4(trow + Cols::SV + 2 * 64 + col, s2);
             tc::tmem_st4(trow + Cols::SV + 3 * 64 + col, s3);
         }
     };
-    // B, C rows of block [tb, tb + nv) to the fp32 tiles (rows t, cols j).
+    // B (when want_b) and C rows of the block to their exact bf16 tiles: one
+    // 16-byte chunk (8 state columns of one token) per thread and tile.
     auto load_bc = [&](int64_t tb, int nv, bool want_b) {
-        const int e0 = tid * 8;
-        const int tt = e0 / N, j = e0 % N;
-        float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo, clo = lo, chi = lo;
+        const int tt = tid >> 3, j = (tid & 7) * 8;
+        uint4 br = make_uint4(0u, 0u, 0u, 0u), cr = br;
         if (tt < nv) {
             const int64_t off = ((int64_t)bb * L + tb + tt) * N + j;
-            const uint4 cr = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.C) + off));
-            clo = make_float4(bf_lo(cr.x), bf_hi(cr.x), bf_lo(cr.y), bf_hi(cr.y));
-            chi = make_float4(bf_lo(cr.z), bf_hi(cr.z), bf_lo(cr.w), bf_hi(cr.w));
-            if (want_b) {
-                const uint4 br = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.B) + off));
-                lo = make_float4(bf_lo(br.x), bf_hi(br.x), bf_lo(br.y), bf_hi(br.y));
-                hi = make_float4(bf_lo(br.z), bf_hi(br.z), bf_lo(br.w), bf_hi(br.w));
-            }
+            cr = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.C) + off));
+            if (want_b) br = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.B) + off));
         }
-        *reinterpret_cast<float4*>(&sm.Cf[sw(tt, j, kK)]) = clo;
-        *reinterpret_cast<float4*>(&sm.Cf[sw(tt, j + 4, kK)]) = chi;
-        if (want_b) {
-            *reinterpret_cast<float4*>(&sm.Bf[sw(tt, j, kK)]) = lo;
-            *reinterpret_cast<float4*>(&sm.Bf[sw(tt, j + 4, kK)]) = hi;
-        }
+        const uint32_t o = tc::bf_offset(tt, j);
+        *reinterpret_cast<uint4*>(reinterpret_cast<char*>(sm.Cs) + o) = cr;
+        if (want_b) *reinterpret_cast<uint4*>(reinterpret_cast<char*>(sm.Bs) + o) = br;
     };
-    // H' = E_63 H into the H tile and into the carry accumulator (its
+    // This block's checkpoint (the state entering it) to the X tile pair:
+    // this thread's 16 state columns of its channel.
+    auto load_x = [&](int k) {
+        const float* xs = ck_at(k) + c * N + 16 * q;
+        float4 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            v[i] = cvalid ? __ldcg(reinterpret_cast<const float4*>(xs) + i)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) st4(sm.Xh, sm.Xl, ch, 16 * q + 4 * i, v[i].x, v[i].y, v[i].z, v[i].w);
+    };
+    // H' = E_63 H into the H tile pair and into the carry accumulator (its
     // initial value: carry out = U C + H').
     auto scale_carry = [&]() {
         float hv[16];
@@ -446,88 +465,92 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) hv[j] *= E63;
 #pragma unroll
-        for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(&sm.H[sw(ch, 16 * q + j, kP)]) =
-                make_float4(hv[j], hv[j + 1], hv[j + 2], hv[j + 3]);
+        for (int j = 0; j < 16; j += 4) st4(sm.Hh, sm.Hl, ch, 16 * q + j, hv[j], hv[j + 1], hv[j + 2], hv[j + 3]);
         tc::tmem_st16(trow + Cols::H + 16 * q, hv);
     };
 
     // --------------------------------------------------------- the MMAs
-    // Descriptors of a row tile with `rows` rows: K-major operand, K step ks
-    // (8 columns); MN-major operand (tile rows = K), K step ks (8 rows).
-    auto kd = [](uint32_t base, int rows, int ks) {
-        return tc::sdesc_sw128(base + (ks >> 2) * rows * 128 + (ks & 3) * 32);
-    };
-    auto md = [](uint32_t base, int rows, int ks) {
-        return tc::sdesc_sw128_mn(base + ks * 1024, rows * 128);
-    };
     const uint32_t lane16 = 16u << 16;
-    // Batch 0: G = C B^T (lanes +0), P = U^T W (lanes +16), both M = 64.
+    // one product A.B over K steps ks < nks, into d (accumulating unless first)
+    auto prod = [&](uint32_t dcol, uint32_t a, bool a_mn, uint32_t b, bool b_mn, int nks,
+                    uint32_t idesc, bool& first) {
+        for (int ks = 0; ks < nks; ++ks) {
+            const uint64_t ad = a_mn ? tc::sdesc_bf_mn(a, ks) : tc::sdesc_bf_k(a, ks);
+            const uint64_t bd = b_mn ? tc::sdesc_bf_mn(b, ks) : tc::sdesc_bf_k(b, ks);
+            tc::mma_bf16_ss(dcol, ad, bd, idesc, first ? 0u : 1u);
+            first = false;
+        }
+    };
+    // the three terms of a split product (hi.hi + hi.lo + lo.hi)
+    auto prod3 = [&](uint32_t dcol, uint32_t ah, uint32_t al, bool a_mn, uint32_t bh, uint32_t bl,
+                     bool b_mn, int nks, uint32_t idesc, bool& first) {
+        prod(dcol, ah, a_mn, bh, b_mn, nks, idesc, first);
+        prod(dcol, ah, a_mn, bl, b_mn, nks, idesc, first);
+        prod(dcol, al, a_mn, bh, b_mn, nks, idesc, first);
+    };
+    // and of a product with an exact operand B (hi.B + lo.B)
+    auto prod2 = [&](uint32_t dcol, uint32_t ah, uint32_t al, bool a_mn, uint32_t b, bool b_mn,
+                     int nks, uint32_t idesc, bool& first) {
+        prod(dcol, ah, a_mn, b, b_mn, nks, idesc, first);
+        prod(dcol, al, a_mn, b, b_mn, nks, idesc, first);
+    };
+    // Batch 0: G = C B^T (lanes +0), P = U^T W (lanes +16), M = 64.
     // Batch 1: R = X C^T, GB = H' B^T, carry += U C.
     auto issue_b01 = [&]() {
-        constexpr uint32_t id64 = tc::idesc_tf32(64, 64);
-        constexpr uint32_t id64mm = tc::idesc_tf32(64, 64, true, true);
-        constexpr uint32_t idR = tc::idesc_tf32(128, 64);
-        constexpr uint32_t idH = tc::idesc_tf32(128, N, false, true);
-#pragma unroll
-        for (int ks = 0; ks < N / 8; ++ks)
-            tc::mma_tf32_ss(tbase + Cols::BC, kd(aC, kK, ks), kd(aB, kK, ks), id64, ks > 0);
-#pragma unroll
-        for (int ks = 0; ks < kP / 8; ++ks)
-            tc::mma_tf32_ss(tbase + lane16 + Cols::BC, md(aU, kP, ks), md(aW, kP, ks), id64mm,
-                            ks > 0);
+        bool f0 = true, f1 = true, f2 = true, f3 = true, fh = false;
+        prod(tbase + Cols::BC, NAJU_SA(Cs), false, NAJU_SA(Bs), false, kN / 16,
+             tc::idesc_bf16(64, 64), f0);
+        prod3(tbase + lane16 + Cols::BC, NAJU_SA(Uh), NAJU_SA(Ul), true, NAJU_SA(Wh), NAJU_SA(Wl),
+              true, kP / 16, tc::idesc_bf16(64, 64, true, true), f1);
         tc::mma_commit(&sm.mb0);
-#pragma unroll
-        for (int ks = 0; ks < N / 8; ++ks) {
-            tc::mma_tf32_ss(tbase + Cols::R, kd(aX, kP, ks), kd(aC, kK, ks), idR, ks > 0);
-            tc::mma_tf32_ss(tbase + Cols::GB, kd(aH, kP, ks), kd(aB, kK, ks), idR, ks > 0);
-        }
-#pragma unroll
-        for (int ks = 0; ks < kK / 8; ++ks)
-            tc::mma_tf32_ss(tbase + Cols::H, kd(aU, kP, ks), md(aC, kK, ks), idH, 1u);
+        prod2(tbase + Cols::R, NAJU_SA(Xh), NAJU_SA(Xl), false, NAJU_SA(Cs), false, kN / 16,
+              tc::idesc_bf16(128, 64), f2);
+        prod2(tbase + Cols::GB, NAJU_SA(Hh), NAJU_SA(Hl), false, NAJU_SA(Bs), false, kN / 16,
+              tc::idesc_bf16(128, 64), f3);
+        prod2(tbase + Cols::H, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Cs), true, kK / 16,
+              tc::idesc_bf16(128, kN, false, true), fh);
     };
     // Batch 2: R += W G^T, GB += U G (G transposed), dC^T = X^T U + B^T Pm^T
     // (lanes +0), dB^T = H'^T W + C^T Pm (lanes +16), all over the masked tiles.
     auto issue_b2 = [&]() {
-        constexpr uint32_t idR = tc::idesc_tf32(128, 64);
-        constexpr uint32_t idGB = tc::idesc_tf32(128, 64, false, true);
-        constexpr uint32_t idMM = tc::idesc_tf32(64, 64, true, true);
-        constexpr uint32_t idMK = tc::idesc_tf32(64, 64, true, false);
-#pragma unroll
-        for (int ks = 0; ks < kK / 8; ++ks) {
-            tc::mma_tf32_ss(tbase + Cols::R, kd(aW, kP, ks), kd(aG, kK, ks), idR, 1u);
-            tc::mma_tf32_ss(tbase + Cols::GB, kd(aU, kP, ks), md(aG, kK, ks), idGB, 1u);
+        bool fr = false, fg = false, fc = true, fb = true;
+        prod3(tbase + Cols::R, NAJU_SA(Wh), NAJU_SA(Wl), false, NAJU_SA(Gh), NAJU_SA(Gl), false,
+              kK / 16, tc::idesc_bf16(128, 64), fr);
+        prod3(tbase + Cols::GB, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Gh), NAJU_SA(Gl), true,
+              kK / 16, tc::idesc_bf16(128, 64, false, true), fg);
+        prod3(tbase + Cols::BC, NAJU_SA(Xh), NAJU_SA(Xl), true, NAJU_SA(Uh), NAJU_SA(Ul), true,
+              kP / 16, tc::idesc_bf16(64, 64, true, true), fc);
+        {
+            // B^T Pm^T: B (rows m = K) against Pm (rows t, K = m): hi and lo of Pm
+            prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Ph), false, kK / 16,
+                 tc::idesc_bf16(64, 64, true, false), fc);
+            prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Pl), false, kK / 16,
+                 tc::idesc_bf16(64, 64, true, false), fc);
         }
-#pragma unroll
-        for (int ks = 0; ks < kP / 8; ++ks) {
-            tc::mma_tf32_ss(tbase + Cols::BC, md(aX, kP, ks), md(aU, kP, ks), idMM, ks > 0);
-            tc::mma_tf32_ss(tbase + lane16 + Cols::BC, md(aH, kP, ks), md(aW, kP, ks), idMM,
-                            ks > 0);
-        }
-#pragma unroll
-        for (int ks = 0; ks < kK / 8; ++ks) {
-            tc::mma_tf32_ss(tbase + Cols::BC, md(aB, kK, ks), kd(aP, kK, ks), idMK, 1u);
-            tc::mma_tf32_ss(tbase + lane16 + Cols::BC, md(aC, kK, ks), md(aP, kK, ks), idMM, 1u);
+        prod3(tbase + lane16 + Cols::BC, NAJU_SA(Hh), NAJU_SA(Hl), true, NAJU_SA(Wh), NAJU_SA(Wl),
+              true, kP / 16, tc::idesc_bf16(64, 64, true, true), fb);
+        {
+            prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Ph), true, kK / 16,
+                 tc::idesc_bf16(64, 64, true, true), fb);
+            prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Pl), true, kK / 16,
+                 tc::idesc_bf16(64, 64, true, true), fb);
         }
         tc::mma_commit(&sm.mb2);
     };
-    // G (lanes +0) and P (lanes +16) from tensor memory to their tiles, lower
-    // triangle kept: this warp's lanes, columns [16 q, 16 q + 16).
+    // G (lanes +0) and P (lanes +16) from tensor memory to their tile pairs,
+    // lower triangle kept: this warp's lanes, columns [16 q, 16 q + 16).
     auto copy_gp = [&]() {
         float v[16];
         tc::tmem_ld16(trow + Cols::BC + 16 * q, v);
         tc::tmem_ld_wait();
         const int row = 16 * s4 + (lid & 15);
-        float* dst = lid < 16 ? sm.G : sm.Pm;
+        __nv_bfloat16* dh = lid < 16 ? sm.Gh : sm.Ph;
+        __nv_bfloat16* dl = lid < 16 ? sm.Gl : sm.Pl;
 #pragma unroll
         for (int j = 0; j < 16; j += 4) {
             const int col = 16 * q + j;
-            float4 o;
-            o.x = col + 0 <= row ? v[j] : 0.f;
-            o.y = col + 1 <= row ? v[j + 1] : 0.f;
-            o.z = col + 2 <= row ? v[j + 2] : 0.f;
-            o.w = col + 3 <= row ? v[j + 3] : 0.f;
-            *reinterpret_cast<float4*>(&dst[sw(row, col, kK)]) = o;
+            st4(dh, dl, row, col, col + 0 <= row ? v[j] : 0.f, col + 1 <= row ? v[j + 1] : 0.f,
+                col + 2 <= row ? v[j + 2] : 0.f, col + 3 <= row ? v[j + 3] : 0.f);
         }
     };
     auto wait_mb = [&](uint64_t* mb, uint32_t& ph) {
@@ -544,13 +567,12 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     // Results go where the MMAs would have put them: R <- x.C, GB <- lambda.B,
     // carry <- f_0 lambda_0; dB and dC are added to the accumulator directly.
     auto exact_block = [&](int64_t tb, int nv) {
-        float* rsum = sm.G;  // [64 t][128 ch] (G and Pm are adjacent)
-        float* gsum = sm.H;  // [64 t][128 ch]
+        float* rsum = reinterpret_cast<float*>(sm.Gh);  // [64 t][128 ch] over G and P
+        float* gsum = reinterpret_cast<float*>(sm.Hh);  // [64 t][128 ch] over the H pair
         for (int e = tid; e < kK * kP; e += kNT) {
             rsum[e] = 0.f;
             gsum[e] = 0.f;
         }
-        // f of token tt: 1 - (the saved 1 - f), one tensor-memory column each
         auto f_at = [&](int tt) {
             const float om = tc::tmem_ld1(trow + Cols::SV + 3 * 64 + tt);
             return 1.f - om;
@@ -560,16 +582,19 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tc::tmem_ld_wait();
         float x[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) x[j] = sm.X[sw(ch, 16 * q + j, kP)];
+        for (int j = 0; j < 16; j += 4) {
+            const float4 x4 = ld4(sm.Xh, sm.Xl, ch, 16 * q + j);
+            x[j] = x4.x; x[j + 1] = x4.y; x[j + 2] = x4.z; x[j + 3] = x4.w;
+        }
         __syncthreads();
         float* acc = p.dBCp + (int64_t)bb * L * 2 * N;
         for (int tt = 0; tt < nv; ++tt) {
-            const float f = f_at(tt), v = sm.W[sw(ch, tt, kP)], sdy = sm.U[sw(ch, tt, kP)];
+            const float f = f_at(tt), v = ld1(sm.Wh, sm.Wl, ch, tt), sdy = ld1(sm.Uh, sm.Ul, ch, tt);
             float rp = 0.f;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                x[j] = fmaf(f, x[j], v * sm.Bf[sw(tt, 16 * q + j, kK)]);
-                rp = fmaf(x[j], sm.Cf[sw(tt, 16 * q + j, kK)], rp);
+                x[j] = fmaf(f, x[j], v * ld1(sm.Bs, tt, 16 * q + j));
+                rp = fmaf(x[j], ld1(sm.Cs, tt, 16 * q + j), rp);
             }
             atomicAdd(&rsum[tt * kP + ch], rp);
 #pragma unroll
@@ -579,12 +604,12 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             }
         }
         for (int tt = nv - 1; tt >= 0; --tt) {
-            const float f = f_at(tt), v = sm.W[sw(ch, tt, kP)], sdy = sm.U[sw(ch, tt, kP)];
+            const float f = f_at(tt), v = ld1(sm.Wh, sm.Wl, ch, tt), sdy = ld1(sm.Uh, sm.Ul, ch, tt);
             float gp = 0.f;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                hx[j] = fmaf(sdy, sm.Cf[sw(tt, 16 * q + j, kK)], hx[j]);
-                gp = fmaf(hx[j], sm.Bf[sw(tt, 16 * q + j, kK)], gp);
+                hx[j] = fmaf(sdy, ld1(sm.Cs, tt, 16 * q + j), hx[j]);
+                gp = fmaf(hx[j], ld1(sm.Bs, tt, 16 * q + j), gp);
             }
             atomicAdd(&gsum[tt * kP + ch], gp);
 #pragma unroll
@@ -607,16 +632,18 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tc::tmem_st_wait();
         sync();
     };
-    // Adjoint-only exact block (early pass): W holds f, U holds s dy.
+    // Adjoint-only exact block (early pass): f from tensor memory (slot 2),
+    // U holds s dy.
     auto exact_carry = [&](int nv) {
         float hx[16];
         tc::tmem_ld16(trow + Cols::H + 16 * q, hx);
         tc::tmem_ld_wait();
         for (int tt = nv - 1; tt >= 0; --tt) {
-            const float f = sm.W[sw(ch, tt, kP)], sdy = sm.U[sw(ch, tt, kP)];
+            const float f = tc::tmem_ld1(trow + Cols::SV + 2 * 64 + tt);
+            const float sdy = ld1(sm.Uh, sm.Ul, ch, tt);
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-                hx[j] = f * fmaf(sdy, sm.Cf[sw(tt, 16 * q + j, kK)], hx[j]);
+                hx[j] = f * fmaf(sdy, ld1(sm.Cs, tt, 16 * q + j), hx[j]);
         }
         tc::tmem_st16(trow + Cols::H + 16 * q, hx);
         tc::tmem_st_wait();
@@ -637,17 +664,17 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             const int nv = (int)min64((int64_t)kK, L - tb);
             if (tid == 0 && k > kb0) prefetch_block(k - 1);
             const bool slow = decays(tb, nv);
-            // U = s dy E (slow: s dy, and f in W)
+            // U = s dy E (slow: s dy)
             {
                 const Tin* gz = has_z ? gin(p.z) : nullptr;
                 const Tin* gdy = gin(p.dy);
                 float E = slow ? 1.f : Eb;
 #pragma unroll
                 for (int g4 = 0; g4 < 4; ++g4) {
-                    float Uv[4];
+                    float Uv[4], fa[4];
                     const int col = 16 * q + 4 * g4;
-                    const float4 f4 = *reinterpret_cast<const float4*>(&sm.W[sw(ch, col, kP)]);
-                    const float fa[4] = {f4.x, f4.y, f4.z, f4.w};
+                    tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, fa);
+                    tc::tmem_ld_wait();
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         const int kk = 4 * g4 + k4, tt = 16 * q + kk;
@@ -661,8 +688,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                         if (!slow) E *= fa[k4];
                         Uv[k4] = sc * dout * gg * E;
                     }
-                    *reinterpret_cast<float4*>(&sm.U[sw(ch, col, kP)]) =
-                        make_float4(Uv[0], Uv[1], Uv[2], Uv[3]);
+                    st4(sm.Uh, sm.Ul, ch, col, Uv[0], Uv[1], Uv[2], Uv[3]);
                 }
             }
             load_bc(tb, nv, false);
@@ -673,10 +699,9 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 tc::fence_proxy_async();
                 sync();
                 if (tid == 0) {
-                    constexpr uint32_t idH = tc::idesc_tf32(128, N, false, true);
-#pragma unroll
-                    for (int ks = 0; ks < kK / 8; ++ks)
-                        tc::mma_tf32_ss(tbase + Cols::H, kd(aU, kP, ks), md(aC, kK, ks), idH, 1u);
+                    bool fh = false;
+                    prod2(tbase + Cols::H, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Cs), true, kK / 16,
+                          tc::idesc_bf16(128, kN, false, true), fh);
                     tc::mma_commit(&sm.mb2);
                 }
                 wait_mb(&sm.mb2, ph2);
@@ -733,11 +758,10 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         }
         int par = 0;  // parity of the block within the segment (double buffers)
         {
-            // tail of the segment's last block: H . (state at the segment end)
             float hx[16];
             tc::tmem_ld16(trow + Cols::H + 16 * q, hx);
             tc::tmem_ld_wait();
-            const float* xe = p.ckpt + ((int64_t)bb * (p.nck + 1) + kb1) * d * N;
+            const float* xe = ck_at(kb1);
             float tp = 0.f;
             if (cvalid) {
 #pragma unroll
@@ -753,16 +777,11 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             if (q == 0) {
 #pragma unroll
                 for (int i = 0; i < 3; ++i) sm.dnext[par][i][ch] = 0.f;
+#pragma unroll
+                for (int v = 0; v < 6; ++v) sm.red6[v][ch] = 0.f;
             }
         }
-        if (q == 0) {
-#pragma unroll
-            for (int v = 0; v < 6; ++v) sm.red6[v][ch] = 0.f;
-        }
-        if (tid == 0) {
-            load_x(kb1 - 1);
-            prefetch_block(kb1 - 1);
-        }
+        if (tid == 0) prefetch_block(kb1 - 1);
         sync();
 
         for (int k = kb1 - 1; k >= kb0; --k, par ^= 1) {
@@ -773,17 +792,14 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             const bool slow = decays(tb, nv);
             unpack(tb, nv, slow);
             load_bc(tb, nv, true);
+            load_x(k);
             if (!slow) scale_carry();
             tc::tmem_st_wait();
             tc::fence_proxy_async();
             sync();
             // ------------------------------------------------ phase B
             if (!slow) {
-                if (tid == 0) {
-                    if (!tc::mbar_wait(&sm.mb_x, ph_x, kSpin)) timed_out = true;
-                    issue_b01();
-                }
-                ph_x ^= 1u;
+                if (tid == 0) issue_b01();
                 wait_mb(&sm.mb0, ph0);
                 copy_gp();
                 tc::fence_proxy_async();
@@ -791,9 +807,6 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 if (tid == 0) issue_b2();
                 wait_mb(&sm.mb2, ph2);
             } else {
-                if (tid == 0 && !tc::mbar_wait(&sm.mb_x, ph_x, kSpin)) timed_out = true;
-                ph_x ^= 1u;
-                sync();
                 exact_block(tb, nv);
             }
             // ------------------------------------------------ phase C
@@ -811,8 +824,8 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 tc::tmem_ld4(trow + Cols::SV + 1 * 64 + col, z0);
                 tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
                 tc::tmem_ld_wait();
-                const float4 U4 = *reinterpret_cast<const float4*>(&sm.U[sw(ch, col, kP)]);
-                const float4 W4 = *reinterpret_cast<const float4*>(&sm.W[sw(ch, col, kP)]);
+                const float4 U4 = ld4(sm.Uh, sm.Ul, ch, col);
+                const float4 W4 = ld4(sm.Wh, sm.Wl, ch, col);
                 const float Ua[4] = {U4.x, U4.y, U4.z, U4.w};
                 const float Wa[4] = {W4.x, W4.y, W4.z, W4.w};
 #pragma unroll
@@ -821,7 +834,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     const int64_t t = tb + tt;
                     const bool valid = cvalid && tt < nv;
                     float dl = Ua[k4] * R4[k4] - Wa[k4] * G4[k4];
-                    // coupled gate: (f df) loses f h lambda.B, carried in dL
+                    // coupled gate: this token's da loses f h lambda.B (kept in dL[kk])
                     if (!has_b) dl = fmaf(-b2[k4], G4[k4], dl);
                     dL[kk] = dl;
                     qsum += dl;
@@ -834,9 +847,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     }
                 }
             }
-            // the coupled term entered qsum: take it out again (it belongs to
-            // this token's da only, not to the sums over later tokens)
-            if (!has_b) {
+            if (!has_b) {  // the sums over later tokens keep the plain dL
                 qsum = 0.f;
 #pragma unroll
                 for (int g4 = 0; g4 < 4; ++g4) {
@@ -854,8 +865,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             sm.dph[q][1][ch] = dpf1;
             sm.dph[q][2][ch] = dpf2;
             __syncthreads();
-            // sums over the later quarters, the tail, the halo of dp
-            float base = 0.f;
+            float base = 0.f;  // dL over the later quarters, plus the tail
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
                 if (qq > q) base += sm.xs[qq][ch];
@@ -895,9 +905,8 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                             run += dL[kk];
                             fdf = run;
                         } else {  // dL[kk] holds dL - f h lambda.B
-                            const float cpl = b2[k4] * G4[k4];
                             fdf = run + dL[kk];
-                            run += dL[kk] + cpl;
+                            run += fmaf(b2[k4], G4[k4], dL[kk]);
                         }
                         const float dpv = fmaf(c1v[kk], G4[k4], c0v[kk]);
                         if (valid) gout(p.da)[t * d] = from_f<Tout>(fdf * om[k4]);
@@ -958,7 +967,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 float tp = 0.f;
 #pragma unroll
                 for (int j = 0; j < 16; j += 4) {
-                    const float4 x4 = *reinterpret_cast<const float4*>(&sm.X[sw(ch, 16 * q + j, kP)]);
+                    const float4 x4 = ld4(sm.Xh, sm.Xl, ch, 16 * q + j);
                     tp = fmaf(hx[j], x4.x, tp);
                     tp = fmaf(hx[j + 1], x4.y, tp);
                     tp = fmaf(hx[j + 2], x4.z, tp);
@@ -971,8 +980,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     sm.dnext[par ^ 1][2][ch] = dpf2;
                 }
             }
-            sync();  // X, W, U, H tiles and tensor memory free for the next block
-            if (tid == 0 && k > kb0) load_x(k - 1);
+            sync();  // tiles and tensor memory free for the next block
         }
 
         // ------------------------------------------- carries and partials
@@ -999,6 +1007,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             sync();
         }
     }
+#undef NAJU_SA
 
     if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
     sync();
@@ -1024,7 +1033,6 @@ __global__ void finish_dBC_kernel(const float* __restrict__ acc, int64_t BtL, in
 
 template <typename Tout, bool CONV, bool PIECES>
 static cudaError_t launch_blk_t(const BwdParams& p, cudaStream_t st) {
-    constexpr int N = 64;
     BkTmaps tm;
     memset(&tm, 0, sizeof(tm));
     bool ok = tma_encode_bf16_3d(&tm.u, p.hu, p.Bt, p.L, p.d, kK + 3, kP) &&
@@ -1032,11 +1040,11 @@ static cudaError_t launch_blk_t(const BwdParams& p, cudaStream_t st) {
               (!p.b || tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, kK, kP)) &&
               (!p.z || tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, kK, kP)) &&
               tma_encode_bf16_3d(&tm.dy, p.dy, p.Bt, p.L, p.d, kK, kP) &&
-              tma_encode_bf16_3d(&tm.B, p.B, p.Bt, p.L, N, kK, N) &&
-              tma_encode_bf16_3d(&tm.C, p.C, p.Bt, p.L, N, kK, N) &&
-              tma_encode_f32_3d_sw128(&tm.X, p.ckpt, p.Bt * (int64_t)(p.nck + 1), p.d, N, kP);
+              tma_encode_bf16_3d(&tm.B, p.B, p.Bt, p.L, kN, kK, kN) &&
+              tma_encode_bf16_3d(&tm.C, p.C, p.Bt, p.L, kN, kK, kN) &&
+              tma_encode_f32_3d_sw128(&tm.X, p.ckpt, p.Bt * (int64_t)(p.nck + 1), p.d, kN, kP);
     if (!ok) return cudaErrorInvalidValue;
-    const size_t smem = sizeof(BkSmem<N>);
+    const size_t smem = sizeof(BkSmem);
     auto kern = scan_bwd_blk_kernel<Tout, CONV, PIECES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -1047,7 +1055,7 @@ static cudaError_t launch_blk_t(const BwdParams& p, cudaStream_t st) {
 }
 
 bool bwd_blk_supported(int dtype, int64_t N, int64_t d) {
-    return dtype == NAJU_BF16 && N == 64 && d % 8 == 0;
+    return dtype == NAJU_BF16 && N == kN && d % 8 == 0;
 }
 
 cudaError_t launch_scan_bwd_blk(const BwdParams& p, int out_dtype, cudaStream_t st) {

@@ -15,7 +15,8 @@
 //   X'   = E_63 (X + S),                            S = W B
 // G = C B^T (M = 64) goes from tensor memory to a masked shared tile; R and S
 // run with X from tensor memory and the other operands from shared memory
-// (fp32 tiles in the 128-byte swizzled row layout; B read MN-major for S).
+// (tf32: fp32 tiles in the 128-byte swizzled row layout; S reads B MN-major,
+// which for tf32 needs a second copy of B with 32-byte swizzle atoms).
 // The state chain from one block to the next is the per-channel update X';
 // everything per (token, channel) runs on the CUDA cores, 512 threads: warp w
 // handles channels 32 (w % 4) + lane and tokens [16 q, 16 q + 16) of the
@@ -69,6 +70,7 @@ struct FkSmem {
     alignas(1024) float Bf[kK * N];   // rows t, cols j
     alignas(1024) float Cf[kK * N];   // rows t, cols j
     alignas(1024) float G[kK * kK];   // rows t, cols m (m <= t)
+    alignas(1024) float Bm[kK * N];   // B again, MN-major layout for S = W B
     alignas(1024) float F[kP * kK];   // f of the block (exact path), rows ch, cols t
     alignas(1024) float rsum[kK * kP];// exact path: x_t . C_t [t][ch]
     float xq[4][kP], xe[4][kP];
@@ -127,7 +129,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     const int item = sm.item;
     const uint32_t sbase = tc::smem_u32(&sm);
     const uint32_t aW = sbase + (uint32_t)offsetof(Sm, W), aB = sbase + (uint32_t)offsetof(Sm, Bf),
-                   aC = sbase + (uint32_t)offsetof(Sm, Cf), aG = sbase + (uint32_t)offsetof(Sm, G);
+                   aC = sbase + (uint32_t)offsetof(Sm, Cf), aG = sbase + (uint32_t)offsetof(Sm, G),
+                   aBm = sbase + (uint32_t)offsetof(Sm, Bm);
     uint32_t ph0 = 0, ph2 = 0;
     bool timed_out = false;
 
@@ -324,6 +327,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             }
             *reinterpret_cast<float4*>(&sm.Bf[sw(tt, j, kK)]) = lo;
             *reinterpret_cast<float4*>(&sm.Bf[sw(tt, j + 4, kK)]) = hi;
+            *reinterpret_cast<float4*>(&sm.Bm[tc::mn32_offset(tt, j, kK) >> 2]) = lo;
+            *reinterpret_cast<float4*>(&sm.Bm[tc::mn32_offset(tt, j + 4, kK) >> 2]) = hi;
             if (want_c) {
                 *reinterpret_cast<float4*>(&sm.Cf[sw(tt, j, kK)]) = clo;
                 *reinterpret_cast<float4*>(&sm.Cf[sw(tt, j + 4, kK)]) = chi;
@@ -332,9 +337,6 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     };
     auto kd = [](uint32_t base, int rows, int ks) {
         return tc::sdesc_sw128(base + (ks >> 2) * rows * 128 + (ks & 3) * 32);
-    };
-    auto md = [](uint32_t base, int rows, int ks) {
-        return tc::sdesc_sw128_mn(base + ks * 1024, rows * 128);
     };
     auto wait_mb = [&](uint64_t* mb, uint32_t& ph) {
         if (warp == kNT / 32 - 1 && !tc::mbar_wait(mb, ph, kSpin)) timed_out = true;
@@ -347,7 +349,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         constexpr uint32_t idS = tc::idesc_tf32(128, N, false, true);
 #pragma unroll
         for (int ks = 0; ks < kK / 8; ++ks)
-            tc::mma_tf32_ss(tbase + Cols::S, kd(aW, kP, ks), md(aB, kK, ks), idS, ks > 0);
+            tc::mma_tf32_ss(tbase + Cols::S, kd(aW, kP, ks), tc::sdesc_mn32(aBm, kK, ks), idS, ks > 0);
     };
     // Exact path: plain recurrence over the block on this thread's state
     // columns; full: x . C summed over the quarters into rsum, then R.

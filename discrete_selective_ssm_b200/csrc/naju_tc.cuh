@@ -72,6 +72,26 @@ __device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t lbo)
     return d;
 }
 
+// MN-major tf32 operands need the 128-byte swizzle with 32-byte atoms: a tile
+// with rows = the operand's K index (R rows) and columns = its M or N index,
+// 32-column blocks R * 128 bytes apart, 4-row groups 512 bytes apart, each
+// 128-byte row's 32-byte chunks (8 elements) XOR-permuted by row % 4.
+__host__ __device__ __forceinline__ uint32_t mn32_offset(int row, int col, int R) {
+    return (uint32_t)((col >> 5) * (R * 128) + (row >> 2) * 512 + (row & 3) * 128 +
+                      ((((col >> 3) & 3) ^ (row & 3)) << 5) + (col & 7) * 4);
+}
+// Its descriptor for K step ks (8 rows = two 4-row groups).
+__device__ __forceinline__ uint64_t sdesc_mn32(uint32_t base, int R, int ks) {
+    const uint32_t saddr = base + (uint32_t)ks * 1024;
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)(((uint32_t)R * 128 >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(512 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)1 << 61;
+    return d;
+}
+
 // Instruction descriptor: D fp32, A and B tf32, M x N; a_mn / b_mn select the
 // MN-major form of the shared-memory A / B operand (K-major otherwise).
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn = false,
@@ -82,6 +102,33 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, bool a_mn = fals
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ------------------------------------------------------- bf16 operand tiles
+// A bf16 row tile of R rows and at most 64 columns in the 128-byte swizzled
+// layout: one 128-byte line per row, its 16-byte chunks (8 elements)
+// XOR-permuted by row % 8, 8-row groups 1024 bytes apart (base 1024-byte
+// aligned).  For 16-bit operands the same bytes are the K-major operand with
+// rows = M or N (K = columns) and the MN-major operand with rows = K
+// (M or N = columns): one tile serves both contractions.
+__host__ __device__ __forceinline__ uint32_t bf_offset(int row, int col) {
+    return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((((col >> 3) & 7) ^ (row & 7)) << 4) +
+                      (col & 7) * 2);
+}
+// Descriptors of such a tile for one kind::f16 K step (16 elements):
+// K-major, step ks < 4 (32 bytes of each line); MN-major, step ks (16 rows =
+// two 8-row groups).
+__device__ __forceinline__ uint64_t sdesc_bf_k(uint32_t base, int ks) {
+    return sdesc_sw128(base + (uint32_t)ks * 32);
+}
+__device__ __forceinline__ uint64_t sdesc_bf_mn(uint32_t base, int ks) {
+    return sdesc_sw128_mn(base + (uint32_t)ks * 2048, 1024);
+}
+// Instruction descriptor: D fp32, A and B bf16 (kind::f16), M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn = false,
+                                                  bool b_mn = false) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // ------------------------------------------------------------------ TMEM
@@ -207,6 +254,16 @@ __device__ __forceinline__ void mma_tf32_ss(uint32_t d_tmem, uint64_t a_desc, ui
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T for one K = 16 step, bf16 operands
+// (kind::f16, fp32 accumulate), issued by one thread.
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }

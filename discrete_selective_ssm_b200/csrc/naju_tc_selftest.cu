@@ -4,6 +4,8 @@
 // operands either no-swizzle K-major core matrices or the 128-byte swizzled
 // K-major layout.  Exposed through naju_testing.h so the test suite can check
 // the operand conventions against a host product.
+#include <cuda_bf16.h>
+
 #include "naju.h"
 #include "naju_common.cuh"
 #include "naju_tc.cuh"
@@ -139,18 +141,22 @@ tc_selftest_ss_kernel(const float* __restrict__ A, const float* __restrict__ B,
 }
 
 // General form: D = A[M x K] * B[N x K]^T with both operands in shared
-// memory as 128-byte swizzled row tiles (sw128_offset).  a_mn = 0: A is
-// stored as the tile A[m][k] (K-major); a_mn = 1: as the tile A^T[k][m]
-// (MN-major).  Likewise b_mn for B.  M = 64 or 128; d_lane (0 or 16) is the
-// lane offset of D in tensor memory.  Every lane of the D columns is copied
-// out raw (D_out[128][N]), so the test can check the accumulator layout.
+// memory, in the layouts the block-form kernels use.
+//  kind 0 (tf32): a_mn = 0 stores A as its [M x K] tile in the 128-byte
+//    swizzled layout (K-major operand); a_mn = 1 as the transposed [K x M]
+//    tile with 32-byte swizzle atoms (MN-major operand).  Likewise B.
+//  kind 1 (bf16, kind::f16): A and B are split into bf16 hi + lo tiles (one
+//    128-byte swizzled row tile serves both majors: a_mn selects whether the
+//    tile holds [M x K] or [K x M]) and D = hi.hi + hi.lo + lo.hi.
+// M = 64 or 128; d_lane (0 or 16) is the lane offset of D in tensor memory.
+// Every lane of the D columns is copied out raw (D_out[128][N]).
 __global__ void __launch_bounds__(128, 1)
 tc_selftest_gen_kernel(const float* __restrict__ A, const float* __restrict__ B,
                        float* __restrict__ D, int M, int N, int K, int a_mn, int b_mn,
-                       int d_lane, uint32_t ncols, int* status) {
+                       int d_lane, int kind, uint32_t ncols, int* status) {
     extern __shared__ __align__(1024) float4 smem4[];
     unsigned char* sa = reinterpret_cast<unsigned char*>(smem4);
-    unsigned char* sb = sa + (size_t)M * K * 4;
+    unsigned char* sb = sa + (size_t)M * K * 4;  // tf32 A, or bf16 A hi + lo
     __shared__ uint64_t mbar;
     __shared__ uint32_t taddr_s;
     const int tid = threadIdx.x, warp = tid / 32;
@@ -160,15 +166,36 @@ tc_selftest_gen_kernel(const float* __restrict__ A, const float* __restrict__ B,
         tc::tmem_relinquish();
     }
     if (tid == 0) tc::mbar_init(&mbar, 1);
-    for (int e = tid; e < M * K; e += 128) {
-        const int m = e / K, k = e % K;
-        const uint32_t off = a_mn ? tc::sw128_offset(k, m, K) : tc::sw128_offset(m, k, M);
-        *reinterpret_cast<float*>(sa + off) = A[e];
-    }
-    for (int e = tid; e < N * K; e += 128) {
-        const int n = e / K, k = e % K;
-        const uint32_t off = b_mn ? tc::sw128_offset(k, n, K) : tc::sw128_offset(n, k, N);
-        *reinterpret_cast<float*>(sb + off) = B[e];
+    if (kind == 0) {
+        for (int e = tid; e < M * K; e += 128) {
+            const int m = e / K, k = e % K;
+            const uint32_t off = a_mn ? tc::mn32_offset(k, m, K) : tc::sw128_offset(m, k, M);
+            *reinterpret_cast<float*>(sa + off) = A[e];
+        }
+        for (int e = tid; e < N * K; e += 128) {
+            const int n = e / K, k = e % K;
+            const uint32_t off = b_mn ? tc::mn32_offset(k, n, K) : tc::sw128_offset(n, k, N);
+            *reinterpret_cast<float*>(sb + off) = B[e];
+        }
+    } else {
+        // bf16 tiles hold at most 64 columns: the stored tile is [rows][64]
+        const size_t ha = (size_t)M * K * 2, hb = (size_t)N * K * 2;
+        for (int e = tid; e < M * K; e += 128) {
+            const int m = e / K, k = e % K;
+            const uint32_t off = a_mn ? tc::bf_offset(k, m) : tc::bf_offset(m, k);
+            const __nv_bfloat16 h = __float2bfloat16_rn(A[e]);
+            *reinterpret_cast<__nv_bfloat16*>(sa + off) = h;
+            *reinterpret_cast<__nv_bfloat16*>(sa + ha + off) =
+                __float2bfloat16_rn(A[e] - __bfloat162float(h));
+        }
+        for (int e = tid; e < N * K; e += 128) {
+            const int n = e / K, k = e % K;
+            const uint32_t off = b_mn ? tc::bf_offset(k, n) : tc::bf_offset(n, k);
+            const __nv_bfloat16 h = __float2bfloat16_rn(B[e]);
+            *reinterpret_cast<__nv_bfloat16*>(sb + off) = h;
+            *reinterpret_cast<__nv_bfloat16*>(sb + hb + off) =
+                __float2bfloat16_rn(B[e] - __bfloat162float(h));
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -188,14 +215,31 @@ tc_selftest_gen_kernel(const float* __restrict__ A, const float* __restrict__ B,
     __syncthreads();
     tc::fence_after_sync();
     if (tid == 0) {
-        const uint32_t idesc = tc::idesc_tf32(M, N, a_mn != 0, b_mn != 0);
         const uint32_t abase = tc::smem_u32(sa), bbase = tc::smem_u32(sb);
-        for (int ks = 0; ks < K / 8; ++ks) {
-            const uint64_t ad = a_mn ? tc::sdesc_sw128_mn(abase + ks * 1024, K * 128)
-                                     : tc::sdesc_sw128(abase + (ks >> 2) * M * 128 + (ks & 3) * 32);
-            const uint64_t bd = b_mn ? tc::sdesc_sw128_mn(bbase + ks * 1024, K * 128)
-                                     : tc::sdesc_sw128(bbase + (ks >> 2) * N * 128 + (ks & 3) * 32);
-            tc::mma_tf32_ss(tbase + ((uint32_t)d_lane << 16), ad, bd, idesc, ks > 0 ? 1u : 0u);
+        const uint32_t dcol = tbase + ((uint32_t)d_lane << 16);
+        if (kind == 0) {
+            const uint32_t idesc = tc::idesc_tf32(M, N, a_mn != 0, b_mn != 0);
+            for (int ks = 0; ks < K / 8; ++ks) {
+                const uint64_t ad = a_mn ? tc::sdesc_mn32(abase, K, ks)
+                                         : tc::sdesc_sw128(abase + (ks >> 2) * M * 128 + (ks & 3) * 32);
+                const uint64_t bd = b_mn ? tc::sdesc_mn32(bbase, K, ks)
+                                         : tc::sdesc_sw128(bbase + (ks >> 2) * N * 128 + (ks & 3) * 32);
+                tc::mma_tf32_ss(dcol, ad, bd, idesc, ks > 0 ? 1u : 0u);
+            }
+        } else {
+            const uint32_t idesc = tc::idesc_bf16(M, N, a_mn != 0, b_mn != 0);
+            const uint32_t ha = (uint32_t)M * K * 2, hb = (uint32_t)N * K * 2;
+            const uint32_t pa[3] = {0, 0, ha}, pb[3] = {0, hb, 0};
+            bool first = true;
+            for (int pr = 0; pr < 3; ++pr)
+                for (int ks = 0; ks < K / 16; ++ks) {
+                    const uint64_t ad = a_mn ? tc::sdesc_bf_mn(abase + pa[pr], ks)
+                                             : tc::sdesc_bf_k(abase + pa[pr], ks);
+                    const uint64_t bd = b_mn ? tc::sdesc_bf_mn(bbase + pb[pr], ks)
+                                             : tc::sdesc_bf_k(bbase + pb[pr], ks);
+                    tc::mma_bf16_ss(dcol, ad, bd, idesc, first ? 0u : 1u);
+                    first = false;
+                }
         }
         tc::mma_commit(&mbar);
     }
@@ -217,14 +261,16 @@ tc_selftest_gen_kernel(const float* __restrict__ A, const float* __restrict__ B,
 }  // namespace naju
 
 extern "C" naju_status naju_testing_tc_mma_gen(int32_t M, int32_t N, int32_t K, int32_t a_mn,
-                                               int32_t b_mn, int32_t d_lane, const float* A,
-                                               const float* B, float* D, int* status,
-                                               void* stream) {
+                                               int32_t b_mn, int32_t d_lane, int32_t kind,
+                                               const float* A, const float* B, float* D,
+                                               int* status, void* stream) {
     if (!A || !B || !D || !status) return NAJU_ERR_INVALID_ARG;
     if ((M != 64 && M != 128) || N < 16 || N > 128 || N % 16 != 0 || K < 32 || K > 128 ||
-        K % 32 != 0)
+        K % 32 != 0 || (kind != 0 && kind != 1))
         return NAJU_ERR_UNSUPPORTED;
-    if (b_mn && N % 32 != 0) return NAJU_ERR_UNSUPPORTED;  // MN-major: 32-element blocks
+    if (kind == 0 && b_mn && N % 32 != 0) return NAJU_ERR_UNSUPPORTED;  // 32-column blocks
+    // bf16 tiles: exactly 64 columns (one 128-byte line per row)
+    if (kind == 1 && ((a_mn ? M : K) != 64 || (b_mn ? N : K) != 64)) return NAJU_ERR_UNSUPPORTED;
     if (d_lane != 0 && !(d_lane == 16 && M == 64)) return NAJU_ERR_UNSUPPORTED;
     uint32_t ncols = 32;
     while (ncols < (uint32_t)N) ncols <<= 1;
@@ -233,7 +279,7 @@ extern "C" naju_status naju_testing_tc_mma_gen(int32_t M, int32_t N, int32_t K, 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return NAJU_ERR_CUDA;
     naju::tc_selftest_gen_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
-        A, B, D, M, N, K, a_mn, b_mn, d_lane, ncols, status);
+        A, B, D, M, N, K, a_mn, b_mn, d_lane, kind, ncols, status);
     return cudaGetLastError() == cudaSuccess ? NAJU_OK : NAJU_ERR_CUDA;
 }
 

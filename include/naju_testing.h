@@ -106,17 +106,22 @@ naju_status naju_testing_tc_mma_ss(int32_t N, int32_t K, int32_t rows_a, int32_t
                                    int32_t swz_b, const float* A, const float* B, float* D,
                                    int* status, void* stream);
 
-/* General form of the same product, both operands in shared memory as
- * 128-byte swizzled tiles: a_mn = 0 stores A as its [M x K] tile (K-major
- * operand), a_mn = 1 as the transposed [K x M] tile (MN-major operand);
- * likewise b_mn for B.  M is 64 or 128; d_lane (0, or 16 with M = 64) is the
- * tensor-memory lane offset of D.  D receives all 128 tensor-memory lanes of
- * the N result columns, row-major [128 x N], so the caller can check where
- * an M = 64 result lands.  K in {32, 64, 96, 128}; N a multiple of 16 up to
- * 128 (of 32 when b_mn). */
+/* General form of the same product, both operands in shared memory, in the
+ * forms the block-form kernels use.  kind 0 (tf32): a_mn = 0 stores A as its
+ * [M x K] tile, 128-byte swizzled (K-major operand); a_mn = 1 as the
+ * transposed [K x M] tile with 32-byte swizzle atoms (MN-major operand, the
+ * only layout tf32 accepts for it); likewise b_mn for B.  kind 1 (bf16): A and
+ * B are split into bf16 hi + lo tiles in the 128-byte swizzled layout (one
+ * tile serves both majors for 16-bit data) and D = hi.hi + hi.lo + lo.hi
+ * (kind::f16 MMAs); the stored tiles are exactly 64 columns wide.  M is 64 or
+ * 128; d_lane (0, or 16 with M = 64) is the tensor-memory lane offset of D.
+ * D receives all 128 tensor-memory lanes of the N result columns, row-major
+ * [128 x N], so the caller can check where an M = 64 result lands.  K in
+ * {32, 64, 96, 128}; N a multiple of 16 up to 128 (of 32 for a tf32 MN-major
+ * B). */
 naju_status naju_testing_tc_mma_gen(int32_t M, int32_t N, int32_t K, int32_t a_mn, int32_t b_mn,
-                                    int32_t d_lane, const float* A, const float* B, float* D,
-                                    int* status, void* stream);
+                                    int32_t d_lane, int32_t kind, const float* A, const float* B,
+                                    float* D, int* status, void* stream);
 
 #ifdef __cplusplus
 }

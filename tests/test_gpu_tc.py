@@ -73,25 +73,30 @@ def _tmem_rows(M, d_lane):
     return [32 * (r // 16) + (r % 16) + d_lane for r in range(64)]
 
 
-@pytest.mark.parametrize("M,N,K,a_mn,b_mn,d_lane", [
-    (128, 64, 64, 0, 0, 0), (128, 64, 64, 1, 0, 0), (128, 64, 64, 0, 1, 0),
-    (128, 64, 128, 1, 1, 0), (128, 128, 64, 1, 1, 0), (128, 32, 96, 1, 0, 0),
-    (64, 64, 64, 0, 0, 0), (64, 64, 64, 1, 1, 0), (64, 64, 128, 1, 0, 16),
-    (64, 64, 64, 0, 1, 16), (64, 32, 32, 1, 1, 16), (64, 128, 64, 1, 1, 0)])
-def test_tc_mma_tf32_mn_major_and_m64(M, N, K, a_mn, b_mn, d_lane):
+@pytest.mark.parametrize("M,N,K,a_mn,b_mn,d_lane,kind", [
+    # tf32: K-major 128-byte swizzle, MN-major 32-byte swizzle atoms
+    (128, 64, 64, 0, 0, 0, 0), (128, 64, 64, 1, 0, 0, 0), (128, 64, 64, 0, 1, 0, 0),
+    (128, 64, 128, 1, 1, 0, 0), (128, 128, 64, 0, 1, 0, 0), (128, 32, 96, 1, 0, 0, 0),
+    (64, 64, 64, 0, 0, 0, 0), (64, 64, 64, 1, 1, 0, 0), (64, 64, 128, 1, 0, 16, 0),
+    (64, 64, 64, 0, 1, 16, 0), (64, 32, 32, 1, 1, 16, 0), (64, 128, 64, 1, 1, 0, 0),
+    # bf16 hi/lo split (kind::f16), the block-form backward's products
+    (128, 64, 64, 0, 0, 0, 1), (128, 64, 64, 0, 1, 0, 1), (64, 64, 128, 1, 1, 0, 1),
+    (64, 64, 128, 1, 1, 16, 1), (64, 64, 64, 1, 0, 0, 1), (64, 64, 64, 1, 1, 16, 1)])
+def test_tc_mma_mn_major_m64_and_split(M, N, K, a_mn, b_mn, d_lane, kind):
     """MN-major (transposed) shared operands, M = 64 accumulators and their
-    placement at lane offset 16, against a host product."""
+    placement at lane offset 16, tf32 and bf16 hi/lo split products, against a
+    host product."""
     L = naju.lib()
     f = L.naju_testing_tc_mma_gen
-    f.argtypes = [ctypes.c_int32] * 6 + [ctypes.c_void_p] * 5
+    f.argtypes = [ctypes.c_int32] * 7 + [ctypes.c_void_p] * 5
     f.restype = ctypes.c_int
-    g = torch.Generator().manual_seed(M * 7 + N * 1000 + K * 10 + a_mn * 2 + b_mn + d_lane)
+    g = torch.Generator().manual_seed(M * 7 + N * 1000 + K * 10 + a_mn * 2 + b_mn + d_lane + kind)
     A = torch.randn(M, K, generator=g)
     B = torch.randn(N, K, generator=g)
     dA, dB = A.cuda(), B.cuda()
     dD = torch.full((128, N), float("nan"), device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    rc = f(M, N, K, a_mn, b_mn, d_lane, ctypes.c_void_p(dA.data_ptr()),
+    rc = f(M, N, K, a_mn, b_mn, d_lane, kind, ctypes.c_void_p(dA.data_ptr()),
            ctypes.c_void_p(dB.data_ptr()), ctypes.c_void_p(dD.data_ptr()),
            ctypes.c_void_p(st.data_ptr()), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert rc == 0
@@ -102,7 +107,8 @@ def test_tc_mma_tf32_mn_major_and_m64(M, N, K, a_mn, b_mn, d_lane):
     lanes = _tmem_rows(M, d_lane)
     got = raw[lanes]
     err = np.max(np.abs(got - ref)) / np.max(np.abs(ref))
-    assert err < 4e-3, err
+    # tf32 operands: ~2^-11 per element; bf16 hi/lo split: ~2^-16
+    assert err < (4e-3 if kind == 0 else 5e-5), err
     others = sorted(set(range(128)) - set(lanes))
     if others:  # lanes outside the result keep the zeros written before the MMA
         assert np.all(raw[others] == 0.0)

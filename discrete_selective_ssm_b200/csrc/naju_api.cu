@@ -77,6 +77,16 @@ bool use_bwd_tc(const naju_dims* dm) {
     if (g_bwd_impl == 1) return false;
     return bwd_tc_supported(dm->dtype, dm->d_state, dm->d_inner);
 }
+// The block-form kernels are the automatic choice wherever they apply; the
+// sub-chunk kernels stay reachable for testing (impl 2).
+bool use_fwd_blk(const naju_dims* dm) {
+    return use_fwd_tc(dm) && g_fwd_impl != 2 &&
+           fwd_blk_supported(dm->dtype, dm->d_state, dm->d_inner, kTck);
+}
+bool use_bwd_blk(const naju_dims* dm) {
+    return use_bwd_tc(dm) && g_bwd_impl != 2 &&
+           bwd_blk_supported(dm->dtype, dm->d_state, dm->d_inner);
+}
 
 // Tensor-core kernels run one block per SM, so the launch's last wave
 // decides the time.  Sequence-group count for `units` blocks' worth of work
@@ -322,8 +332,7 @@ naju_status naju_scan_fwd(const naju_dims* dims, const void* hu, const float* co
     p.scale = 1.0f / std::sqrt((float)dims->d_state);
     p.wait_limit = g_wait_limit;
     p.fault_skip_publish = g_skip_publish;
-    if (l.fwd_tc && g_fwd_impl == 3 &&
-        fwd_blk_supported(dims->dtype, dims->d_state, dims->d_inner, p.T_ck))
+    if (use_fwd_blk(dims))
         return cuda_status(launch_scan_fwd_blk(p, dims->out_dtype, s));
     if (l.fwd_tc) return cuda_status(launch_scan_fwd_tc(p, dims->out_dtype, s));
     return cuda_status(launch_scan_fwd(p, dims->dtype, dims->out_dtype, s));
@@ -376,8 +385,7 @@ naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* co
     p.scale = 1.0f / std::sqrt((float)dims->d_state);
     p.wait_limit = g_wait_limit;
     p.fault_skip_publish = g_skip_publish;
-    if (l.bwd_tc && g_bwd_impl == 3 &&
-        bwd_blk_supported(dims->dtype, dims->d_state, dims->d_inner)) {
+    if (use_bwd_blk(dims)) {
         e = launch_scan_bwd_blk(p, dims->out_dtype, s);
         if (e == cudaSuccess)
             e = launch_bwd_reductions_acc(p, dims->out_dtype, dB, dC, dD, dconv_w, dconv_b, s);
@@ -489,14 +497,13 @@ int32_t naju_testing_bwd_impl(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);
     if (check_dims(dm) != NAJU_OK) return 0;
     if (!use_bwd_tc(dm)) return 1;
-    return (g_bwd_impl == 3 && bwd_blk_supported(dm->dtype, dm->d_state, dm->d_inner)) ? 3 : 2;
+    return use_bwd_blk(dm) ? 3 : 2;
 }
 int32_t naju_testing_fwd_impl(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);
     if (check_dims(dm) != NAJU_OK) return 0;
     if (!use_fwd_tc(dm)) return 1;
-    return (g_fwd_impl == 3 && fwd_blk_supported(dm->dtype, dm->d_state, dm->d_inner, kTck)) ? 3
-                                                                                           : 2;
+    return use_fwd_blk(dm) ? 3 : 2;
 }
 int32_t naju_testing_bwd_groups(const void* dims) {
     const naju_dims* dm = static_cast<const naju_dims*>(dims);

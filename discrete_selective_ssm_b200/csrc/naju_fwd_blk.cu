@@ -1,5 +1,6 @@
 // Naju forward scan in block form on the 5th-generation tensor cores
-// (sm_100a, tcgen05, kind::tf32), for bf16 activations with d_state 64 or 128.
+// (sm_100a, tcgen05, kind::f16 with fp32 accumulation), for bf16 activations
+// with d_state 64 or 128.
 //
 // Same computation as the CUDA-core forward (Naju reproduction README, "Core
 // equations"): x_n = f_n x_{n-1} + i_n h_n B_n^T, y_n = x_n.C_n/sqrt(N) + D h_n,
@@ -8,19 +9,26 @@
 // A thread block owns 128 channels of one batch element (one channel per
 // tensor-memory lane) and walks its tokens in blocks of 64, the spacing of
 // the checkpoints it writes for the backward.  With X the state entering a
-// block (resident in tensor memory for the whole pass), per channel
+// block (kept in tensor memory for the whole pass), per channel
 // E_t = prod_{k<=t} f_k from the block start, Q_t = 1/E_t, W_t = i_t h_t Q_t and
 // G[t][m] = C_t.B_m kept for m <= t:
 //   y_t  = s E_t R_t SiLU(z_t) + D h_t SiLU(z_t),   R = X C^T + W G^T
 //   X'   = E_63 (X + S),                            S = W B
-// G = C B^T (M = 64) goes from tensor memory to a masked shared tile; R and S
-// run with X from tensor memory and the other operands from shared memory
-// (tf32: fp32 tiles in the 128-byte swizzled row layout; S reads B MN-major,
-// which for tf32 needs a second copy of B with 32-byte swizzle atoms).
-// The state chain from one block to the next is the per-channel update X';
-// everything per (token, channel) runs on the CUDA cores, 512 threads: warp w
-// handles channels 32 (w % 4) + lane and tokens [16 q, 16 q + 16) of the
-// block, q = w / 4, and the state columns [q N / 4, (q + 1) N / 4).
+// All three products run on the tensor core.  Each fp32 operand (X, W, G) is
+// a pair of bf16 tiles hi = bf16(v), lo = bf16(v - hi) and a product takes
+// hi.hi + hi.lo + lo.hi (about 2^-16 relative error; B and C are bf16 inputs,
+// exact in one tile), so the state handed from block to block - and the
+// checkpoints the backward starts from - keep nearly fp32 accuracy.  The
+// tiles are 128-byte swizzled row tiles; for 16-bit data the same bytes serve
+// as the K-major operand and as the MN-major one (B in S = W B).
+//
+// The raw inputs of a block (u with its 3-token conv halo, a, b, z) arrive by
+// TMA into one shared buffer as soon as the previous block has read its own;
+// B and C arrive by TMA straight into their swizzled tiles once the previous
+// block's products are done.  Everything per (token, channel) runs on the
+// CUDA cores, 512 threads: warp w handles channels 32 (w % 4) + lane and
+// tokens [16 q, 16 q + 16) of the block, q = w / 4, and the state columns
+// [q N / 4, (q + 1) N / 4).
 //
 // Exactness.  A block where some channel's decay product over the block
 // falls below 2^-90 runs the plain recurrence token by token instead.
@@ -50,40 +58,63 @@ constexpr long long kSpin = 1LL << 24;
 
 template <int N>
 struct FkCols {
-    static constexpr uint32_t X = 0;            // state [ch][j]
-    static constexpr uint32_t S = N;            // W B   [ch][j]
-    static constexpr uint32_t R = 2 * N;        // R     [ch][t]
-    static constexpr uint32_t G = 2 * N + 64;   // G (M = 64)
-    static constexpr uint32_t SV = 2 * N + 128; // s E SiLU(z), D h SiLU(z)  [ch][t] x 2
+    static constexpr uint32_t X = 0;             // state [ch][j]
+    static constexpr uint32_t S = N;             // W B   [ch][j]
+    static constexpr uint32_t R = 2 * N;         // R     [ch][t]
+    static constexpr uint32_t G = 2 * N + 64;    // G (M = 64)
+    static constexpr uint32_t SV = 2 * N + 128;  // s E SiLU(z), D h SiLU(z)  [ch][t] x 2
     static constexpr uint32_t USED = 2 * N + 256;
     static constexpr uint32_t ALLOC = USED <= 256 ? 256 : 512;
     static_assert(USED <= 512, "tensor memory");
 };
 
 struct alignas(64) FkTmaps {
-    CUtensorMap u, a, b, z, B, C;  // bf16, for L2 prefetches
+    CUtensorMap u, a, b, z;  // bf16 [Bt][L][d], plain boxes of 128 channels
+    CUtensorMap B, C;        // bf16 [Bt][L][N], swizzled boxes of 64 columns
 };
 
 template <int N>
 struct FkSmem {
-    alignas(1024) float W[kP * kK];   // rows ch, cols t
-    alignas(1024) float Bf[kK * N];   // rows t, cols j
-    alignas(1024) float Cf[kK * N];   // rows t, cols j
-    alignas(1024) float G[kK * kK];   // rows t, cols m (m <= t)
-    alignas(1024) float Bm[kK * N];   // B again, MN-major layout for S = W B
-    alignas(1024) float F[kP * kK];   // f of the block (exact path), rows ch, cols t
-    alignas(1024) float rsum[kK * kP];// exact path: x_t . C_t [t][ch]
+    alignas(1024) __nv_bfloat16 Wh[kP * kK], Wl[kP * kK];  // rows ch, cols t
+    alignas(1024) __nv_bfloat16 Xh[kP * N], Xl[kP * N];    // rows ch, cols j
+    alignas(1024) __nv_bfloat16 Bs[kK * N], Cs[kK * N];    // rows t, cols j
+    alignas(1024) __nv_bfloat16 Gh[kK * kK], Gl[kK * kK];  // rows t, cols m (m <= t)
+    alignas(1024) __nv_bfloat16 ru[(kK + 3) * kP];         // u of tokens tb - 3 ..
+    alignas(128) __nv_bfloat16 ra[kK * kP], rb[kK * kP], rz[kK * kP];
     float xq[4][kP], xe[4][kP];
-    uint64_t mb0, mb2;
+    uint64_t mb_raw, mb_bc, mb0, mb2;
     uint32_t taddr;
     int item, ok;
 };
 
-__device__ __forceinline__ float ldbf(const __nv_bfloat16* p) {
-    return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16);
+__device__ __forceinline__ float bf2f(__nv_bfloat16 v) {
+    return __uint_as_float((uint32_t)__bfloat16_as_ushort(v) << 16);
 }
-__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+// hi = bf16(v), lo = bf16(v - hi) for two values, packed.
+__device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+// Eight consecutive values (row, col .. col + 7; col % 8 == 0) into a tile
+// pair of R rows: one 16-byte chunk in each.
+__device__ __forceinline__ void st8(__nv_bfloat16* th, __nv_bfloat16* tl, int row, int col, int R,
+                                    const float* v) {
+    uint4 h, l;
+    split2(v[0], v[1], h.x, l.x);
+    split2(v[2], v[3], h.y, l.y);
+    split2(v[4], v[5], h.z, l.z);
+    split2(v[6], v[7], h.w, l.w);
+    const uint32_t o = tc::bf_offset_w(row, col, R);
+    *reinterpret_cast<uint4*>(reinterpret_cast<char*>(th) + o) = h;
+    *reinterpret_cast<uint4*>(reinterpret_cast<char*>(tl) + o) = l;
+}
+__device__ __forceinline__ float ld1(const __nv_bfloat16* t, int row, int col, int R) {
+    return bf2f(*reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(t) +
+                                                          tc::bf_offset_w(row, col, R)));
+}
 
 }  // namespace
 
@@ -92,8 +123,9 @@ __global__ void __launch_bounds__(512, 1)
 scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     using Cols = FkCols<N>;
     using Sm = FkSmem<N>;
-    using Tin = __nv_bfloat16;
     constexpr int NQ = N / 4;  // state columns per thread
+    static_assert(sizeof(Sm::Xh) + sizeof(Sm::Xl) >= kK * kP * sizeof(float),
+                  "the exact path's row sums live over the X tiles");
     extern __shared__ __align__(1024) float4 smem4[];
     Sm& sm = *reinterpret_cast<Sm*>(smem4);
 
@@ -112,8 +144,11 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     }
     if (tid == 0) {
         sm.item = atomicAdd(&p.hdr->fwd_ticket, 1);
+        tc::mbar_init(&sm.mb_raw, 1);
+        tc::mbar_init(&sm.mb_bc, 1);
         tc::mbar_init(&sm.mb0, 1);
         tc::mbar_init(&sm.mb2, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         tma::prefetch_map(&tm.u);
         tma::prefetch_map(&tm.a);
         if (has_b) tma::prefetch_map(&tm.b);
@@ -128,10 +163,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     const uint32_t trow = tbase + ((uint32_t)(s4 * 32) << 16);
     const int item = sm.item;
     const uint32_t sbase = tc::smem_u32(&sm);
-    const uint32_t aW = sbase + (uint32_t)offsetof(Sm, W), aB = sbase + (uint32_t)offsetof(Sm, Bf),
-                   aC = sbase + (uint32_t)offsetof(Sm, Cf), aG = sbase + (uint32_t)offsetof(Sm, G),
-                   aBm = sbase + (uint32_t)offsetof(Sm, Bm);
-    uint32_t ph0 = 0, ph2 = 0;
+#define NAJU_SA(f) (sbase + (uint32_t)offsetof(Sm, f))
+    uint32_t ph_raw = 0, ph_bc = 0, ph0 = 0, ph2 = 0;
     bool timed_out = false;
 
     int bb = 0, tile = 0, seg0 = 0, seg1 = 0;
@@ -158,18 +191,44 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             Dc = p.D ? p.D[c] : 0.f;
         }
     };
-    auto gin = [&](const void* base) {
-        return static_cast<const Tin*>(base) + (int64_t)bb * L * d + c;
-    };
     auto ck_at = [&](int k) { return p.ckpt + ((int64_t)bb * (p.nck + 1) + k) * d * N; };
     auto sync = [&]() {
         tc::fence_before_sync();
         __syncthreads();
         tc::fence_after_sync();
     };
-    auto sw = [](int row, int col, int R) { return tc::sw128_offset(row, col, R) >> 2; };
+    auto wait_mb = [&](uint64_t* mb, uint32_t& ph) {
+        // one warp polls (until a first time-out); the others wait at the barrier
+        if (warp == kNT / 32 - 1 && !timed_out && !tc::mbar_wait(mb, ph, kSpin)) timed_out = true;
+        __syncthreads();
+        ph ^= 1u;
+        tc::fence_after_sync();
+    };
 
-    // This thread's state columns of the TMEM state <-> a global [d][N] row.
+    // ------------------------------------------------------- TMA issue
+    // Raw per-token inputs of block k (thread 0; z only when full).
+    auto load_raw = [&](int k, bool full) {
+        const bool zz = full && has_z;
+        const uint32_t rows = (kK + 3) + kK * (1 + (has_b ? 1 : 0) + (zz ? 1 : 0));
+        tma::expect_tx(&sm.mb_raw, rows * kP * 2u);
+        const int x = (int)c0, y = k * kK, zb = bb;
+        tma::load_3d(sm.ru, &tm.u, x, y - 3, zb, &sm.mb_raw);
+        tma::load_3d(sm.ra, &tm.a, x, y, zb, &sm.mb_raw);
+        if (has_b) tma::load_3d(sm.rb, &tm.b, x, y, zb, &sm.mb_raw);
+        if (zz) tma::load_3d(sm.rz, &tm.z, x, y, zb, &sm.mb_raw);
+    };
+    // B (and C when full) of block k into their tiles (thread 0).
+    auto load_bc = [&](int k, bool full) {
+        tma::expect_tx(&sm.mb_bc, (uint32_t)(2 * kK * N * (full ? 2 : 1)));
+        const int y = k * kK, zb = bb;
+#pragma unroll
+        for (int jb = 0; jb < N / 64; ++jb) {
+            tma::load_3d(sm.Bs + jb * kK * 64, &tm.B, jb * 64, y, zb, &sm.mb_bc);
+            if (full) tma::load_3d(sm.Cs + jb * kK * 64, &tm.C, jb * 64, y, zb, &sm.mb_bc);
+        }
+    };
+
+    // This thread's state columns: global [d][N] row -> tensor memory.
     auto state_from = [&](const float* src, bool cg) {
         float v[NQ];
 #pragma unroll
@@ -185,49 +244,41 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         for (int k = 0; k < NQ; k += 16) tc::tmem_st16(trow + Cols::X + NQ * q + k, &v[k]);
         tc::tmem_st_wait();
     };
-    auto state_to = [&](float* dst) {
-        float v[NQ];
+    // This thread's state columns from tensor memory to a global [d][N] row
+    // (dst != null) and to the X tile pair (tiles).
+    auto state_out = [&](float* dst, bool tiles) {
 #pragma unroll
-        for (int k = 0; k < NQ; k += 16) tc::tmem_ld16(trow + Cols::X + NQ * q + k, &v[k]);
-        tc::tmem_ld_wait();
-        if (cvalid) {
+        for (int k = 0; k < NQ; k += 16) {
+            float v[16];
+            tc::tmem_ld16(trow + Cols::X + NQ * q + k, v);
+            tc::tmem_ld_wait();
+            if (dst && cvalid) {
 #pragma unroll
-            for (int k = 0; k < NQ; k += 4)
-                *reinterpret_cast<float4*>(dst + c * N + NQ * q + k) =
-                    make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+                for (int j = 0; j < 16; j += 4)
+                    *reinterpret_cast<float4*>(dst + c * N + NQ * q + k + j) =
+                        make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
+            if (tiles) {
+                st8(sm.Xh, sm.Xl, ch, NQ * q + k, kP, v);
+                st8(sm.Xh, sm.Xl, ch, NQ * q + k + 8, kP, v + 8);
+            }
         }
-    };
-    auto prefetch_block = [&](int k) {
-        const int x = (int)c0, y = k * kK, zb = bb;
-        tma::prefetch_l2_3d(&tm.u, x, y > 3 ? y - 3 : 0, zb);
-        tma::prefetch_l2_3d(&tm.a, x, y, zb);
-        if (has_b) tma::prefetch_l2_3d(&tm.b, x, y, zb);
-        if (has_z) tma::prefetch_l2_3d(&tm.z, x, y, zb);
-        tma::prefetch_l2_3d(&tm.B, 0, y, zb);
-        tma::prefetch_l2_3d(&tm.C, 0, y, zb);
     };
 
     // ------------------------------------------------- decays (loop 1)
     float fv[16], qv[16];
     float Eb = 1.f, Qb = 1.f, E63 = 1.f;
-    auto decays = [&](int64_t tb, int nv) -> bool {
-        const Tin* ga = gin(p.a);
+    auto decays = [&](int nv) -> bool {
+        const __nv_bfloat16* rap = sm.ra + 16 * q * kP + ch;
         float Qh = 1.f, Eh = 1.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const int tt = 16 * q + k;
-            const bool valid = cvalid && tt < nv;
-            const float av = valid ? ldbf(ga + (tb + tt) * d) : 0.f;
-            const float ea = __expf(-av);
-            qv[k] = valid ? 1.f + ea : 1.f;
+            const bool valid = cvalid && 16 * q + k < nv;
+            qv[k] = valid ? 1.f + __expf(-bf2f(rap[k * kP])) : 1.f;
             fv[k] = valid ? rcpa_(qv[k]) : 1.f;
             Qh *= qv[k];
             Eh *= fv[k];
         }
-#pragma unroll
-        for (int k = 0; k < 16; k += 4)
-            *reinterpret_cast<float4*>(&sm.F[sw(ch, 16 * q + k, kP)]) =
-                make_float4(fv[k], fv[k + 1], fv[k + 2], fv[k + 3]);
         sm.xq[q][ch] = Qh;
         sm.xe[q][ch] = Eh;
         const bool maybe = __syncthreads_or(!(Qh <= kQuarter)) != 0;
@@ -248,114 +299,97 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         return maybe && __syncthreads_or(!(Qa <= kBound)) != 0;
     };
     // ------------------------------------------------- unpack (loop 2)
-    // W (shared tile); full: s E SiLU(z) and D h SiLU(z) (tensor memory).
-    auto unpack = [&](int64_t tb, int nv, bool slow, bool full) {
-        const Tin* gu = gin(p.hu);
-        const Tin* gbp = has_b ? gin(p.b) : nullptr;
-        const Tin* gz = has_z ? gin(p.z) : nullptr;
-        auto ubits = [&](int i) -> uint32_t {
-            const int tt = 16 * q - 3 + i;
-            const int64_t t = tb + tt;
-            const bool ok = cvalid && tt < nv && t >= 0 && (CONV || i >= 3);
-            return ok ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(gu + t * d)) : 0u;
-        };
-        uint32_t upk[10];
-#pragma unroll
-        for (int i = 0; i < 10; ++i) upk[i] = ubits(2 * i) | (i < 9 ? ubits(2 * i + 1) << 16 : 0u);
-        auto uwin = [&](int m) { return (m & 1) ? bf_hi(upk[m >> 1]) : bf_lo(upk[m >> 1]); };
+    // W to its tile pair; full: s E SiLU(z) and D h SiLU(z) to tensor memory.
+    // slow (exact path): E = Q = 1, so W = i h.
+    auto unpack = [&](int nv, bool slow, bool full) {
+        const __nv_bfloat16* rup = sm.ru + 16 * q * kP + ch;  // row i: token 16 q - 3 + i
+        const __nv_bfloat16* rbp = sm.rb + 16 * q * kP + ch;
+        const __nv_bfloat16* rzp = sm.rz + 16 * q * kP + ch;
         float E = slow ? 1.f : Eb, Q = slow ? 1.f : Qb;
+        float u0 = 0.f, u1 = 0.f, u2 = 0.f;
+        if (CONV) {
+            u0 = bf2f(rup[0]);
+            u1 = bf2f(rup[kP]);
+            u2 = bf2f(rup[2 * kP]);
+        }
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-            float Wv[4], s0[4], s1[4];
+        for (int g8 = 0; g8 < 2; ++g8) {
+            float Wv[8], s0[8], s1[8];
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) {
-                const int k = 4 * g4 + k4;
-                const int tt = 16 * q + k;
-                const int64_t t = tb + tt;
-                const bool valid = cvalid && tt < nv;
+            for (int k8 = 0; k8 < 8; ++k8) {
+                const int k = 8 * g8 + k8;
+                const bool valid = cvalid && 16 * q + k < nv;
+                const float u3 = bf2f(rup[(k + 3) * kP]);
                 float h;
                 if (CONV) {
-                    const float pp = fmaf(w3, uwin(k + 3), fmaf(w2, uwin(k + 2),
-                                         fmaf(w1, uwin(k + 1), fmaf(w0, uwin(k), wb))));
+                    const float pp = fmaf(w3, u3, fmaf(w2, u2, fmaf(w1, u1, fmaf(w0, u0, wb))));
                     h = pp * sigmoida_(pp);
+                    u0 = u1;
+                    u1 = u2;
+                    u2 = u3;
                 } else {
-                    h = uwin(k + 3);
+                    h = u3;
                 }
                 if (!valid) h = 0.f;
                 const float f = fv[k], qq = qv[k];
                 // coupled: i = 1 - f = (1/f - 1) f (1 where exp(-a) overflowed)
-                const float iw = has_b ? (valid ? sigmoida_(ldbf(gbp + t * d)) : 0.f)
+                const float iw = has_b ? sigmoida_(bf2f(rbp[k * kP]))
                                        : (qq < 3.0e38f ? (qq - 1.f) * f : 1.f);
                 if (!slow) {
                     E *= f;
                     Q *= qq;
                 }
-                Wv[k4] = iw * h * Q;
+                Wv[k8] = iw * h * Q;
                 if (full) {
                     float gg = 1.f;
                     if (has_z) {
-                        const float zv = valid ? ldbf(gz + t * d) : 0.f;
+                        const float zv = bf2f(rzp[k * kP]);
                         gg = zv * sigmoida_(zv);
                     }
-                    s0[k4] = sc * E * gg;
-                    s1[k4] = Dc * h * gg;
+                    s0[k8] = sc * E * gg;
+                    s1[k8] = Dc * h * gg;
                 }
             }
-            const int col = 16 * q + 4 * g4;
-            *reinterpret_cast<float4*>(&sm.W[sw(ch, col, kP)]) = make_float4(Wv[0], Wv[1], Wv[2], Wv[3]);
+            const int col = 16 * q + 8 * g8;
+            st8(sm.Wh, sm.Wl, ch, col, kP, Wv);
             if (full) {
-                tc::tmem_st4(trow + Cols::SV + col, s0);
-                tc::tmem_st4(trow + Cols::SV + 64 + col, s1);
+                tc::tmem_st8(trow + Cols::SV + col, s0);
+                tc::tmem_st8(trow + Cols::SV + 64 + col, s1);
             }
         }
     };
-    auto load_bc = [&](int64_t tb, int nv, bool want_c) {
-#pragma unroll
-        for (int e0 = tid * 8; e0 < kK * N; e0 += kNT * 8) {
-            const int tt = e0 / N, j = e0 % N;
-            float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo, clo = lo, chi = lo;
-            if (tt < nv) {
-                const int64_t off = ((int64_t)bb * L + tb + tt) * N + j;
-                const uint4 br = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.B) + off));
-                lo = make_float4(bf_lo(br.x), bf_hi(br.x), bf_lo(br.y), bf_hi(br.y));
-                hi = make_float4(bf_lo(br.z), bf_hi(br.z), bf_lo(br.w), bf_hi(br.w));
-                if (want_c) {
-                    const uint4 cr = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.C) + off));
-                    clo = make_float4(bf_lo(cr.x), bf_hi(cr.x), bf_lo(cr.y), bf_hi(cr.y));
-                    chi = make_float4(bf_lo(cr.z), bf_hi(cr.z), bf_lo(cr.w), bf_hi(cr.w));
-                }
-            }
-            *reinterpret_cast<float4*>(&sm.Bf[sw(tt, j, kK)]) = lo;
-            *reinterpret_cast<float4*>(&sm.Bf[sw(tt, j + 4, kK)]) = hi;
-            *reinterpret_cast<float4*>(&sm.Bm[tc::mn32_offset(tt, j, kK) >> 2]) = lo;
-            *reinterpret_cast<float4*>(&sm.Bm[tc::mn32_offset(tt, j + 4, kK) >> 2]) = hi;
-            if (want_c) {
-                *reinterpret_cast<float4*>(&sm.Cf[sw(tt, j, kK)]) = clo;
-                *reinterpret_cast<float4*>(&sm.Cf[sw(tt, j + 4, kK)]) = chi;
-            }
+
+    // --------------------------------------------------------- the MMAs
+    // D (+)= A B over nks K steps of 16, A and B bf16 tiles in the layout of
+    // tc::bf_offset_w (a_rows, b_rows: their row counts).
+    auto prod = [&](uint32_t dcol, uint32_t a, int a_rows, uint32_t b, int b_rows, bool b_mn,
+                    int nks, uint32_t idesc, bool& first) {
+        for (int ks = 0; ks < nks; ++ks) {
+            const uint64_t bd = b_mn ? tc::sdesc_bfw_mn(b, b_rows, ks) : tc::sdesc_bfw_k(b, b_rows, ks);
+            tc::mma_bf16_ss(dcol, tc::sdesc_bfw_k(a, a_rows, ks), bd, idesc, first ? 0u : 1u);
+            first = false;
         }
     };
-    auto kd = [](uint32_t base, int rows, int ks) {
-        return tc::sdesc_sw128(base + (ks >> 2) * rows * 128 + (ks & 3) * 32);
-    };
-    auto wait_mb = [&](uint64_t* mb, uint32_t& ph) {
-        if (warp == kNT / 32 - 1 && !tc::mbar_wait(mb, ph, kSpin)) timed_out = true;
-        __syncthreads();
-        ph ^= 1u;
-        tc::fence_after_sync();
-    };
-    // S = W B (the state update's product), on its own (update-only pass).
-    auto mma_S = [&]() {
-        constexpr uint32_t idS = tc::idesc_tf32(128, N, false, true);
+    // S = W B: W (rows ch, K = t) against B (rows t = K, columns j = N),
+    // one 64-column block of j per product.
+    auto issue_S = [&]() {
+        constexpr uint32_t id = tc::idesc_bf16(128, 64, false, true);
 #pragma unroll
-        for (int ks = 0; ks < kK / 8; ++ks)
-            tc::mma_tf32_ss(tbase + Cols::S, kd(aW, kP, ks), tc::sdesc_mn32(aBm, kK, ks), idS, ks > 0);
+        for (int jb = 0; jb < N / 64; ++jb) {
+            const uint32_t bsrc = NAJU_SA(Bs) + (uint32_t)(jb * kK * 128);
+            bool f = true;
+            prod(tbase + Cols::S + 64 * jb, NAJU_SA(Wh), kP, bsrc, kK, true, kK / 16, id, f);
+            prod(tbase + Cols::S + 64 * jb, NAJU_SA(Wl), kP, bsrc, kK, true, kK / 16, id, f);
+        }
     };
-    // Exact path: plain recurrence over the block on this thread's state
-    // columns; full: x . C summed over the quarters into rsum, then R.
+
+    // Exact path: the plain recurrence over the block on this thread's state
+    // columns (f recomputed from the raw a); full: x . C summed over the
+    // quarters (in the X tiles' bytes, rewritten after the block), then R.
     auto exact_block = [&](int nv, bool full) {
+        float* rsum = reinterpret_cast<float*>(sm.Xh);  // [64 t][128 ch]
         if (full) {
-            for (int e = tid; e < kK * kP; e += kNT) sm.rsum[e] = 0.f;
+            for (int e = tid; e < kK * kP; e += kNT) rsum[e] = 0.f;
             __syncthreads();
         }
         float x[NQ];
@@ -363,14 +397,15 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         for (int k = 0; k < NQ; k += 16) tc::tmem_ld16(trow + Cols::X + NQ * q + k, &x[k]);
         tc::tmem_ld_wait();
         for (int tt = 0; tt < nv; ++tt) {
-            const float f = sm.F[sw(ch, tt, kP)], v = sm.W[sw(ch, tt, kP)];
+            const float f = sigmoidf_(bf2f(sm.ra[tt * kP + ch]));
+            const float v = ld1(sm.Wh, ch, tt, kP) + ld1(sm.Wl, ch, tt, kP);
             float rp = 0.f;
 #pragma unroll
             for (int j = 0; j < NQ; ++j) {
-                x[j] = fmaf(f, x[j], v * sm.Bf[sw(tt, NQ * q + j, kK)]);
-                if (full) rp = fmaf(x[j], sm.Cf[sw(tt, NQ * q + j, kK)], rp);
+                x[j] = fmaf(f, x[j], v * ld1(sm.Bs, tt, NQ * q + j, kK));
+                if (full) rp = fmaf(x[j], ld1(sm.Cs, tt, NQ * q + j, kK), rp);
             }
-            if (full) atomicAdd(&sm.rsum[tt * kP + ch], rp);
+            if (full) atomicAdd(&rsum[tt * kP + ch], rp);
         }
 #pragma unroll
         for (int k = 0; k < NQ; k += 16) tc::tmem_st16(trow + Cols::X + NQ * q + k, &x[k]);
@@ -378,7 +413,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             __syncthreads();
             float rv[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) rv[k] = sm.rsum[(16 * q + k) * kP + ch];
+            for (int k = 0; k < 16; ++k) rv[k] = rsum[(16 * q + k) * kP + ch];
             tc::tmem_st16(trow + Cols::R + 16 * q, rv);
         }
         tc::tmem_st_wait();
@@ -399,88 +434,115 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         tc::tmem_st_wait();
     };
 
-    // One block: full (outputs) or update-only.  The state X in tensor
-    // memory enters the block and leaves it updated.
+    // One block: full (outputs) or update-only.  On entry the block's raw
+    // inputs and B (and C) are on their way and, when full, the X tile pair
+    // holds the state entering it; on exit the state in tensor memory is
+    // updated and, for next >= 0, block next's loads are issued.
     float logP = 0.f;  // log of the decay product over an update-only pass
-    auto run_block = [&](int k, bool full) {
+    auto run_block = [&](int k, bool full, int next) {
         const int64_t tb = (int64_t)k * kK;
         const int nv = (int)min64((int64_t)kK, L - tb);
-        const bool slow = decays(tb, nv);
-        unpack(tb, nv, slow, full);
-        load_bc(tb, nv, full);
+        wait_mb(&sm.mb_raw, ph_raw);
+        const bool slow = decays(nv);
+        unpack(nv, slow, full);
+        tc::tmem_st_wait();
         tc::fence_proxy_async();
         sync();
+        // the raw buffer is read (the exact path still needs a)
+        if (tid == 0 && next >= 0 && !slow) load_raw(next, full);
+        wait_mb(&sm.mb_bc, ph_bc);
         if (!slow) {
-            if (full) {
-                if (tid == 0) {
-                    constexpr uint32_t id64 = tc::idesc_tf32(64, 64);
-                    constexpr uint32_t idR = tc::idesc_tf32(128, 64);
-#pragma unroll
-                    for (int ks = 0; ks < N / 8; ++ks)
-                        tc::mma_tf32_ss(tbase + Cols::G, kd(aC, kK, ks), kd(aB, kK, ks), id64, ks > 0);
+            constexpr uint32_t idR = tc::idesc_bf16(128, 64);
+            if (tid == 0) {
+                if (full) {
+                    // G = C B^T (M = 64; B and C exact)
+                    bool fg = true;
+                    prod(tbase + Cols::G, NAJU_SA(Cs), kK, NAJU_SA(Bs), kK, false, N / 16,
+                         tc::idesc_bf16(64, 64), fg);
                     tc::mma_commit(&sm.mb0);
-                    mma_S();
-#pragma unroll
-                    for (int ks = 0; ks < N / 8; ++ks)
-                        tc::mma_tf32_ts(tbase + Cols::R, tbase + Cols::X + ks * 8, kd(aC, kK, ks), idR,
-                                        ks > 0);
                 }
+                issue_S();
+                if (full) {
+                    // R = X C^T
+                    bool fr = true;
+                    prod(tbase + Cols::R, NAJU_SA(Xh), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
+                    prod(tbase + Cols::R, NAJU_SA(Xl), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
+                } else {
+                    tc::mma_commit(&sm.mb2);
+                }
+            }
+            if (full) {
                 wait_mb(&sm.mb0, ph0);
-                {   // masked G to its tile: lanes +0 of each sub-partition hold rows
+                {   // masked G to its tile pair: lanes 0-15 of each sub-partition hold rows
                     float v[16];
                     tc::tmem_ld16(trow + Cols::G + 16 * q, v);
                     tc::tmem_ld_wait();
                     if (lid < 16) {
                         const int row = 16 * s4 + lid;
 #pragma unroll
-                        for (int j = 0; j < 16; j += 4) {
-                            const int col = 16 * q + j;
-                            float4 o;
-                            o.x = col + 0 <= row ? v[j] : 0.f;
-                            o.y = col + 1 <= row ? v[j + 1] : 0.f;
-                            o.z = col + 2 <= row ? v[j + 2] : 0.f;
-                            o.w = col + 3 <= row ? v[j + 3] : 0.f;
-                            *reinterpret_cast<float4*>(&sm.G[sw(row, col, kK)]) = o;
-                        }
+                        for (int j = 0; j < 16; ++j)
+                            if (16 * q + j > row) v[j] = 0.f;
+                        st8(sm.Gh, sm.Gl, row, 16 * q, kK, v);
+                        st8(sm.Gh, sm.Gl, row, 16 * q + 8, kK, v + 8);
                     }
                 }
                 tc::fence_proxy_async();
                 sync();
                 if (tid == 0) {
-                    constexpr uint32_t idR = tc::idesc_tf32(128, 64);
-#pragma unroll
-                    for (int ks = 0; ks < kK / 8; ++ks)
-                        tc::mma_tf32_ss(tbase + Cols::R, kd(aW, kP, ks), kd(aG, kK, ks), idR, 1u);
+                    // R += W G^T (three terms)
+                    bool fr = false;
+                    prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
+                    prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gl), kK, false, kK / 16, idR, fr);
+                    prod(tbase + Cols::R, NAJU_SA(Wl), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
                     tc::mma_commit(&sm.mb2);
                 }
-            } else if (tid == 0) {
-                mma_S();
-                tc::mma_commit(&sm.mb2);
             }
             wait_mb(&sm.mb2, ph2);
         } else {
             exact_block(nv, full);
+            if (tid == 0 && next >= 0) load_raw(next, full);
         }
+        // the B and C tiles are free
+        if (tid == 0 && next >= 0) load_bc(next, full);
         if (full) {
-            Tout* gy = static_cast<Tout*>(p.y) + (int64_t)bb * L * d + c;
+            Tout* gy = static_cast<Tout*>(p.y) + ((int64_t)bb * L + tb + 16 * q) * d + c;
             float r[16], e[16], dh[16];
             tc::tmem_ld16(trow + Cols::R + 16 * q, r);
             tc::tmem_ld16(trow + Cols::SV + 16 * q, e);
             tc::tmem_ld16(trow + Cols::SV + 64 + 16 * q, dh);
             tc::tmem_ld_wait();
+            const int nk = cvalid ? min(16, nv - 16 * q) : 0;
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-                const int tt = 16 * q + kk;
-                if (cvalid && tt < nv) gy[(tb + tt) * d] = from_f<Tout>(fmaf(e[kk], r[kk], dh[kk]));
-            }
+            for (int kk = 0; kk < 16; ++kk)
+                if (kk < nk) gy[(int64_t)kk * d] = from_f<Tout>(fmaf(e[kk], r[kk], dh[kk]));
         }
         if (!slow) update_state();
         logP += __logf(E63);  // decay over the block (for the look-back)
-        sync();
     };
 
     // ============================================================ passes
-    if (PIECES) {
+    // Blocks [s0, s1) of the current unit from the state in tensor memory:
+    // full passes write the checkpoint after every block but the last (and
+    // after the last when end_ckpt) and the outputs.
+    auto run_segment = [&](int s0, int s1, bool full, bool end_ckpt) {
+        if (tid == 0) {
+            load_raw(s0, full);
+            load_bc(s0, full);
+        }
+        if (full) state_out(nullptr, true);
+        tc::fence_proxy_async();
+        sync();
+        for (int k = s0; k < s1; ++k) {
+            const bool last = k + 1 == s1;
+            run_block(k, full, last ? -1 : k + 1);
+            state_out(full && (!last || end_ckpt) ? ck_at(k + 1) : nullptr, full && !last);
+            tc::fence_proxy_async();
+            sync();
+        }
+    };
+    if (sbase & 1023u) {  // the swizzled tiles need 1024-byte alignment
+        if (tid == 0) atomicOr(&p.hdr->status, 1 << NAJU_ERR_INVALID_ARG);
+    } else if (PIECES) {
         const int64_t Wb = Bt * p.ntiles * (int64_t)p.nck;
         const int64_t F0 = (int64_t)item * Wb / p.npieces;
         const int64_t F1 = (int64_t)(item + 1) * Wb / p.npieces;
@@ -491,20 +553,14 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             int* flag_cut = p.flags + (int64_t)bb * p.ntiles + tile;
             if (s0 == 0) {
                 state_from(p.x0 ? p.x0 + (int64_t)bb * d * N : nullptr, false);
-                state_to(ck_at(0));
+                state_out(ck_at(0), false);
             } else {
                 if (tid == 0) sm.ok = wait_flag(flag_cut, &p.hdr->status, p.wait_limit) ? 1 : 0;
                 __syncthreads();
                 state_from(sm.ok ? ck_at(s0) : nullptr, true);
             }
-            if (tid == 0) prefetch_block(s0);
-            sync();
-            for (int k = s0; k < s1; ++k) {
-                if (tid == 0 && k + 1 < s1) prefetch_block(k + 1);
-                run_block(k, true);
-                state_to(ck_at(k + 1));
-            }
-            if (s1 == p.nck && p.x_final) state_to(p.x_final + (int64_t)bb * d * N);
+            run_segment(s0, s1, true, true);
+            if (s1 == p.nck && p.x_final) state_out(p.x_final + (int64_t)bb * d * N, false);
             if (s1 < p.nck) {  // head of a cut unit: the state at the cut is published
                 __threadfence();
                 __syncthreads();
@@ -526,12 +582,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         if (!last_group) {
             // update-only pass from x0 (first group) or zero, then the look-back
             state_from(g == 0 ? x0b : nullptr, false);
-            sync();
             logP = 0.f;
-            for (int k = seg0; k < seg1; ++k) {
-                if (tid == 0 && k + 1 < seg1) prefetch_block(k + 1);
-                run_block(k, false);
-            }
+            run_segment(seg0, seg1, false, false);
             if (g > 0) {
                 if (tid == 0) sm.ok = wait_flag(flag_prev, &p.hdr->status, p.wait_limit) ? 1 : 0;
                 __syncthreads();
@@ -557,7 +609,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                 }
                 tc::tmem_st_wait();
             }
-            state_to(ck_at(seg1));
+            state_out(ck_at(seg1), false);
             __threadfence();
             __syncthreads();
             if (tid == 0 && !(g == 0 && p.fault_skip_publish)) st_release(flag_mine, 1);
@@ -570,17 +622,12 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             state_from(ok ? ck_at(seg0) : nullptr, true);
         } else {
             state_from(x0b, false);
-            state_to(ck_at(0));
+            state_out(ck_at(0), false);
         }
-        if (tid == 0) prefetch_block(seg0);
-        sync();
-        for (int k = seg0; k < seg1; ++k) {
-            if (tid == 0 && k + 1 < seg1) prefetch_block(k + 1);
-            run_block(k, true);
-            if (k + 1 < seg1 || last_group) state_to(ck_at(k + 1));
-        }
-        if (last_group && p.x_final) state_to(p.x_final + (int64_t)bb * d * N);
+        run_segment(seg0, seg1, true, last_group);
+        if (last_group && p.x_final) state_out(p.x_final + (int64_t)bb * d * N, false);
     }
+#undef NAJU_SA
     if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
     sync();
     if (warp == 0) tc::tmem_dealloc(tbase, Cols::ALLOC);
@@ -594,8 +641,8 @@ static cudaError_t launch_fwd_blk_t(const FwdParams& p, cudaStream_t st) {
               tma_encode_bf16_3d(&tm.a, p.a, p.Bt, p.L, p.d, kK, kP) &&
               (!p.b || tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, kK, kP)) &&
               (!p.z || tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, kK, kP)) &&
-              tma_encode_bf16_3d(&tm.B, p.B, p.Bt, p.L, N, kK, N) &&
-              tma_encode_bf16_3d(&tm.C, p.C, p.Bt, p.L, N, kK, N);
+              tma_encode_bf16_3d_sw128(&tm.B, p.B, p.Bt, p.L, N, kK) &&
+              tma_encode_bf16_3d_sw128(&tm.C, p.C, p.Bt, p.L, N, kK);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(FkSmem<N>);
     auto kern = scan_fwd_blk_kernel<Tout, N, CONV, PIECES>;

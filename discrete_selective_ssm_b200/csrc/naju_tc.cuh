@@ -124,6 +124,17 @@ __device__ __forceinline__ uint64_t sdesc_bf_k(uint32_t base, int ks) {
 __device__ __forceinline__ uint64_t sdesc_bf_mn(uint32_t base, int ks) {
     return sdesc_sw128_mn(base + (uint32_t)ks * 2048, 1024);
 }
+// Wider bf16 tiles (R rows, up to 128 columns): 64-column blocks R * 128
+// bytes apart, each in the layout above.
+__host__ __device__ __forceinline__ uint32_t bf_offset_w(int row, int col, int R) {
+    return (uint32_t)((col >> 6) * (R * 128)) + bf_offset(row, col & 63);
+}
+__device__ __forceinline__ uint64_t sdesc_bfw_k(uint32_t base, int R, int ks) {
+    return sdesc_sw128(base + (uint32_t)((ks >> 2) * R * 128 + (ks & 3) * 32));
+}
+__device__ __forceinline__ uint64_t sdesc_bfw_mn(uint32_t base, int R, int ks) {
+    return sdesc_sw128_mn(base + (uint32_t)ks * 2048, (uint32_t)R * 128);
+}
 // Instruction descriptor: D fp32, A and B bf16 (kind::f16), M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn = false,
                                                   bool b_mn = false) {

@@ -44,6 +44,23 @@ bool tma_encode_bf16_3d(CUtensorMap* map, const void* base, int64_t outer, int64
     return r == CUDA_SUCCESS;
 }
 
+bool tma_encode_bf16_3d_sw128(CUtensorMap* map, const void* base, int64_t outer, int64_t rows,
+                              int64_t cols, int box_rows) {
+    if (!map || !base || outer < 1 || rows < 1 || cols < 64) return false;
+    if (reinterpret_cast<uintptr_t>(base) % 16 != 0 || (cols * 2) % 16 != 0) return false;
+    if (box_rows < 1 || box_rows > 256) return false;
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)outer};
+    const cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)(rows * cols) * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool tma_encode_f32_3d_sw128(CUtensorMap* map, const void* base, int64_t outer, int64_t rows,
                              int64_t cols, int box_rows) {
     if (!map || !base || outer < 1 || rows < 1 || cols < 32) return false;

@@ -20,6 +20,13 @@ namespace naju {
 bool tma_encode_bf16_3d(CUtensorMap* map, const void* base, int64_t outer, int64_t rows,
                         int64_t cols, int box_rows, int box_cols);
 
+// Encode a 3-D bf16 tensor map whose box is box_rows rows of 64 columns (128
+// bytes), written to shared memory in the 128-byte swizzled layout (box row r
+// at byte 128 r, its 16-byte chunks XOR-permuted by r % 8; destination
+// 1024-byte aligned).  Same checks as tma_encode_bf16_3d.
+bool tma_encode_bf16_3d_sw128(CUtensorMap* map, const void* base, int64_t outer, int64_t rows,
+                              int64_t cols, int box_rows);
+
 // Encode a 3-D fp32 tensor map [outer][rows][cols] whose box is box_rows rows
 // of 32 columns (128 bytes), written to shared memory in the 128-byte swizzled
 // layout: box row r lands at byte 128 r with its 16-byte chunks XOR-permuted

@@ -67,10 +67,10 @@ void naju_testing_set_sm_count(int32_t sms);
 /* The SM count the tiling currently uses. */
 int32_t naju_testing_sm_count(void);
 
-/* Forward implementation: 0 = automatic (tensor cores for bf16 activations
- * with d_state 64 or 128 and d_inner % 8 == 0, CUDA cores otherwise),
- * 1 = always CUDA cores, 2 = the tensor-core sub-chunk kernel, 3 = the
- * tensor-core block-form kernel, where tensor cores apply. */
+/* Forward implementation: 0 = automatic (the tensor-core block-form kernel
+ * for bf16 activations with d_state 64 or 128 and d_inner % 8 == 0, CUDA
+ * cores otherwise), 1 = always CUDA cores, 2 = the tensor-core sub-chunk
+ * kernel, 3 = the tensor-core block-form kernel, where tensor cores apply. */
 void naju_testing_set_fwd_impl(int32_t impl);
 
 /* The forward implementation for these dims: 1 = CUDA cores, 2 = tensor-core
@@ -80,8 +80,8 @@ int32_t naju_testing_fwd_impl(const void* dims);
 /* Backward implementation: 0 = automatic (tensor cores for bf16 activations
  * with d_state 64 or 128 and d_inner % 8 == 0: the block-form kernel for
  * d_state 64, the sub-chunk kernel for 128; CUDA cores otherwise),
- * 1 = always CUDA cores, 2 = the tensor-core sub-chunk kernel where tensor
- * cores apply. */
+ * 1 = always CUDA cores, 2 = the tensor-core sub-chunk kernel, 3 = the
+ * block-form kernel (as automatic), where tensor cores apply. */
 void naju_testing_set_bwd_impl(int32_t impl);
 
 /* The backward implementation for these dims: 1 = CUDA cores, 2 = tensor-core

@@ -149,7 +149,7 @@ def test_fwd_tensor_core_exact_fallback(N):
     a[:, 220:240] = 60.0
     t["a"] = a.to(torch.bfloat16)
     dm = naju.make_dims(2, 300, 200, N, naju.BF16)
-    assert naju.testing_fwd_impl(dm) == 2
+    assert naju.testing_fwd_impl(dm) == 3
     y, xf, _ = run_fwd(t, True, out_dtype=naju.F32)
     ro, rx = oracle_fwd(t, True)
     assert_close(y, ro, TOL_BF16, name="y")
@@ -157,9 +157,10 @@ def test_fwd_tensor_core_exact_fallback(N):
 
 
 @pytest.mark.parametrize("N", [64, 128])
-@pytest.mark.parametrize("impl", [1, 0])
+@pytest.mark.parametrize("impl", [1, 2, 0])
 def test_fwd_both_implementations(N, impl):
-    """The CUDA-core and tensor-core forwards both match the oracle (bf16)."""
+    """The CUDA-core, sub-chunk and block-form tensor-core forwards all match
+    the oracle (bf16)."""
     w = wl(N, "bf16", Bt=2, L=333, d=260)
     t = inputs(w, True, use_x0=True)
     naju.testing_set_fwd_impl(impl)
@@ -287,17 +288,17 @@ def test_bwd_sequence_groups(groups):
 
 
 @pytest.mark.parametrize("N", [64, 128])
-@pytest.mark.parametrize("impl", [1, 0])
+@pytest.mark.parametrize("impl", [1, 2, 0])
 @pytest.mark.parametrize("conv", [True, False])
 def test_bwd_both_implementations(N, impl, conv):
-    """The CUDA-core and tensor-core backwards both match the oracle (bf16
+    """The CUDA-core and both tensor-core backwards match the oracle (bf16
     inputs; 3 channel tiles, the last ragged; a ragged last block)."""
     w = wl(N, "bf16", Bt=2, L=333, d=264)
     t = inputs(w, conv, use_x0=True, use_dxL=True)
     dm = naju.make_dims(2, 333, 264, N, naju.BF16)
     naju.testing_set_bwd_impl(impl)
     try:
-        assert naju.testing_bwd_impl(dm) == (1 if impl == 1 else 2)
+        assert naju.testing_bwd_impl(dm) == (impl if impl else (3 if N == 64 else 2))
         g = run_bwd(t, conv, out_dtype=naju.F32)
     finally:
         naju.testing_set_bwd_impl(0)
@@ -308,7 +309,7 @@ def test_bwd_both_implementations(N, impl, conv):
 def test_bwd_tensor_core_bf16_outputs():
     w = wl(64, "bf16", Bt=2, L=200, d=136)
     t = inputs(w, True)
-    assert naju.testing_bwd_impl(naju.make_dims(2, 200, 136, 64, naju.BF16)) == 2
+    assert naju.testing_bwd_impl(naju.make_dims(2, 200, 136, 64, naju.BF16)) == 3
     g = run_bwd(t, True, out_dtype=naju.BF16)
     r = oracle_bwd(t, True)
     compare_grads(g, r, True, TOL_BF16, bf16_out=True)

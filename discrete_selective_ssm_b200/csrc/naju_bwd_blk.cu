@@ -1,5 +1,6 @@
 // Naju backward scan in block form on the 5th-generation tensor cores
-// (sm_100a, tcgen05, kind::tf32), for bf16 activations with d_state 64.
+// (sm_100a, tcgen05, kind::f16 with fp32 accumulation), for bf16 activations
+// with d_state 64.
 //
 // Gradient of the Naju recurrence (Naju reproduction README, "Core
 // equations"): x_n = f_n x_{n-1} + i_n h_n B_n^T, y_n = x_n.C_n/sqrt(N) + D h_n,
@@ -32,13 +33,20 @@
 // products G and P (M = 64) share tensor-memory columns at lane offsets 0 and
 // 16, and later dC^T and dB^T do the same.
 //
+// Data movement.  Every input of a block arrives by TMA while the block
+// before it (the later one) finishes: the per-token inputs u (with its 3-token
+// conv halo), a, b, z and dout into shared memory that the carry, G and P tiles
+// occupy only between the two phases that need them; B and C straight into
+// their swizzled tiles; the fp32 checkpoint into the X tiles' bytes, which the
+// block turns into its hi / lo pair.  bf16 gradients dz, db, da and dh (du)
+// are written to shared memory in the W and U tiles' bytes once the block no
+// longer reads them and leave by TMA stores, which clip the ragged edges.
+//
 // Threads.  512: warp w handles tensor-memory lanes 32 (w % 4) .. + 31, i.e.
 // channels 32 (w % 4) + lane, and the 16 tokens [16 q, 16 q + 16) of the
 // block, q = w / 4 (and the state columns [16 q, 16 q + 16) where a channel's
-// state row is split).  Per-token inputs and the checkpoint are read straight
-// from global memory (prefetched into L2 one block ahead by TMA prefetches);
-// the per-token coefficients the gradients need after the MMAs wait in tensor
-// memory and registers.
+// state row is split); the per-token coefficients the gradients need after
+// the MMAs wait in tensor memory and registers.
 //
 // Exactness.  A block in which some channel's decay product over the block
 // falls below 2^-90 (the factorisation's range) runs an exact token-by-token
@@ -52,6 +60,8 @@
 // split the work exactly as in the sub-chunk tensor-core backward.
 #include <stddef.h>
 #include <string.h>
+
+#include <type_traits>
 
 #include "naju_common.cuh"
 #include "naju_kernels.h"
@@ -81,32 +91,45 @@ struct BkCols {
 };
 
 struct alignas(64) BkTmaps {
-    CUtensorMap u, a, b, z, dy, B, C;  // bf16, for L2 prefetches
-    CUtensorMap X;                     // fp32 checkpoints, for L2 prefetches
+    CUtensorMap u, a, b, z, dy;  // bf16 [Bt][L][d]: 64 tokens (u: 67) x 128 channels
+    CUtensorMap B, C;            // bf16 [Bt][L][N]: 64 tokens x 64 columns, swizzled
+    CUtensorMap X;               // fp32 checkpoints [Bt (nck+1)][d][N]: 128 x 32, swizzled
+    CUtensorMap oz, ob, oa, ou;  // bf16 outputs dz, db, da, dh (du): 64 tokens x 128 channels
 };
 
-// bf16 operand tiles (hi / lo pairs of the fp32 operands), 1024-byte aligned.
+// Shared memory, 1024-byte aligned tiles.  Region A (the carry, G and P tile
+// pairs) is dead from the end of one block's products to the next block's
+// carry scaling and takes that block's per-token inputs in between; the W and
+// U pairs take the staged bf16 outputs once the second-to-last pass is done;
+// the X pair takes the next fp32 checkpoint once the block's tail sum has
+// read it.
 struct BkSmem {
     alignas(1024) __nv_bfloat16 Xh[kP * kN], Xl[kP * kN];  // checkpoint: rows ch, cols j
-    alignas(1024) __nv_bfloat16 Hh[kP * kN], Hl[kP * kN];  // H' = E_63 H: rows ch, cols j
     alignas(1024) __nv_bfloat16 Wh[kP * kK], Wl[kP * kK];  // rows ch, cols t
     alignas(1024) __nv_bfloat16 Uh[kP * kK], Ul[kP * kK];  // rows ch, cols t
     alignas(1024) __nv_bfloat16 Bs[kK * kN], Cs[kK * kN];  // rows t, cols j (exact)
-    alignas(1024) __nv_bfloat16 Gh[kK * kK], Gl[kK * kK];  // rows t, cols m (m <= t)
-    alignas(1024) __nv_bfloat16 Ph[kK * kK], Pl[kK * kK];  // rows t, cols m (m <= t)
+    // region A
+    alignas(1024) __nv_bfloat16 Hh[kP * kN], Hl[kP * kN];  // H' = E_63 H: rows ch, cols j
+    __nv_bfloat16 Gh[kK * kK], Gl[kK * kK];                // rows t, cols m (m <= t)
+    __nv_bfloat16 Ph[kK * kK], Pl[kK * kK];                // rows t, cols m (m <= t)
+    alignas(1024) __nv_bfloat16 ru[(kK + 3) * kP];         // u of tokens tb - 3 .. tb + 63
     float xq[4][kP], xe[4][kP];   // per-quarter decay products
     float xs[4][kP];              // per-quarter sums of dL
     float tailp[2][4][kP];        // partial H . x_63 of the next block to run
     float dph[4][3][kP];          // first three dp of each quarter
     float dnext[2][3][kP];        // first three dp of the later block
     float red6[6][kP];            // per-channel parameter sums
-    uint64_t mb0, mb2;
+    uint64_t mb_in, mb_bc, mb_x, mb0, mb2;
     uint32_t taddr;
     int item, ok;
 };
+static_assert(offsetof(BkSmem, Pl) + sizeof(BkSmem::Pl) - offsetof(BkSmem, Hh) == 4 * kK * kP * 2,
+              "region A holds the four raw per-token inputs");
+static_assert(sizeof(BkSmem::Xh) + sizeof(BkSmem::Xl) == kP * kN * 4, "fp32 checkpoint");
+static_assert(sizeof(BkSmem) <= 232448, "shared memory");
 
-__device__ __forceinline__ float ldbf(const __nv_bfloat16* p) {
-    return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p)) << 16);
+__device__ __forceinline__ float bf2f(__nv_bfloat16 v) {
+    return __uint_as_float((uint32_t)__bfloat16_as_ushort(v) << 16);
 }
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
@@ -126,35 +149,38 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t&
     hi = *reinterpret_cast<const uint32_t*>(&h);
     lo = *reinterpret_cast<const uint32_t*>(&l);
 }
-// Four consecutive values (row, col .. col + 3; col % 4 == 0) into a tile pair.
-__device__ __forceinline__ void st4(__nv_bfloat16* th, __nv_bfloat16* tl, int row, int col,
-                                    float v0, float v1, float v2, float v3) {
-    uint32_t h0, l0, h1, l1;
-    split2(v0, v1, h0, l0);
-    split2(v2, v3, h1, l1);
-    const uint32_t o = tc::bf_offset(row, col);
-    *reinterpret_cast<uint2*>(reinterpret_cast<char*>(th) + o) = make_uint2(h0, h1);
-    *reinterpret_cast<uint2*>(reinterpret_cast<char*>(tl) + o) = make_uint2(l0, l1);
+// Eight consecutive values into a tile pair at byte offset o (one 16-byte
+// chunk of each).
+__device__ __forceinline__ void st8o(__nv_bfloat16* th, __nv_bfloat16* tl, uint32_t o,
+                                     const float* v) {
+    uint4 h, l;
+    split2(v[0], v[1], h.x, l.x);
+    split2(v[2], v[3], h.y, l.y);
+    split2(v[4], v[5], h.z, l.z);
+    split2(v[6], v[7], h.w, l.w);
+    *reinterpret_cast<uint4*>(reinterpret_cast<char*>(th) + o) = h;
+    *reinterpret_cast<uint4*>(reinterpret_cast<char*>(tl) + o) = l;
 }
-// Four consecutive values (hi + lo) back from a tile pair.
-__device__ __forceinline__ float4 ld4(const __nv_bfloat16* th, const __nv_bfloat16* tl, int row,
-                                      int col) {
-    const uint32_t o = tc::bf_offset(row, col);
+// Four consecutive values (hi + lo) from a tile pair at byte offset o.
+__device__ __forceinline__ void ld4o(const __nv_bfloat16* th, const __nv_bfloat16* tl, uint32_t o,
+                                     float* v) {
     const uint2 h = *reinterpret_cast<const uint2*>(reinterpret_cast<const char*>(th) + o);
     const uint2 l = *reinterpret_cast<const uint2*>(reinterpret_cast<const char*>(tl) + o);
-    return make_float4(bf_lo(h.x) + bf_lo(l.x), bf_hi(h.x) + bf_hi(l.x), bf_lo(h.y) + bf_lo(l.y),
-                       bf_hi(h.y) + bf_hi(l.y));
+    v[0] = bf_lo(h.x) + bf_lo(l.x);
+    v[1] = bf_hi(h.x) + bf_hi(l.x);
+    v[2] = bf_lo(h.y) + bf_lo(l.y);
+    v[3] = bf_hi(h.y) + bf_hi(l.y);
 }
-// One value (hi + lo) back from a tile pair, and one value of an exact tile.
+// One value (hi + lo) of a tile pair, and one value of an exact tile.
 __device__ __forceinline__ float ld1(const __nv_bfloat16* th, const __nv_bfloat16* tl, int row,
                                      int col) {
     const uint32_t o = tc::bf_offset(row, col);
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(th) + o)) +
-           __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(tl) + o));
+    return bf2f(*reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(th) + o)) +
+           bf2f(*reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(tl) + o));
 }
 __device__ __forceinline__ float ld1(const __nv_bfloat16* t, int row, int col) {
-    return __bfloat162float(
-        *reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(t) + tc::bf_offset(row, col)));
+    return bf2f(*reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(t) +
+                                                          tc::bf_offset(row, col)));
 }
 
 }  // namespace
@@ -163,9 +189,11 @@ template <typename Tout, bool CONV, bool PIECES>
 __global__ void __launch_bounds__(512, 1)
 scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     constexpr int N = kN;
+    // bf16 gradients leave through shared memory and TMA stores; fp32 ones
+    // are stored directly
+    constexpr bool kStage = std::is_same<Tout, __nv_bfloat16>::value;
     using Cols = BkCols;
     using Sm = BkSmem;
-    using Tin = __nv_bfloat16;
     extern __shared__ __align__(1024) float4 smem4[];
     Sm& sm = *reinterpret_cast<Sm*>(smem4);
 
@@ -186,6 +214,9 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     }
     if (tid == 0) {
         sm.item = atomicAdd(&p.hdr->bwd_ticket, 1);
+        tc::mbar_init(&sm.mb_in, 1);
+        tc::mbar_init(&sm.mb_bc, 1);
+        tc::mbar_init(&sm.mb_x, 1);
         tc::mbar_init(&sm.mb0, 1);
         tc::mbar_init(&sm.mb2, 1);
         tma::prefetch_map(&tm.X);
@@ -196,6 +227,12 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tma::prefetch_map(&tm.dy);
         tma::prefetch_map(&tm.B);
         tma::prefetch_map(&tm.C);
+        if (kStage) {
+            tma::prefetch_map(&tm.oa);
+            tma::prefetch_map(&tm.ou);
+            if (has_z) tma::prefetch_map(&tm.oz);
+            if (has_b) tma::prefetch_map(&tm.ob);
+        }
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -205,8 +242,24 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     const int item = sm.item;
     const uint32_t sbase = tc::smem_u32(&sm);
 #define NAJU_SA(f) (sbase + (uint32_t)offsetof(Sm, f))
-    uint32_t ph0 = 0, ph2 = 0;  // mbarrier parities
+    uint32_t ph_in = 0, ph_bc = 0, ph_x = 0, ph0 = 0, ph2 = 0;  // mbarrier parities
     bool timed_out = false;
+
+    // This thread's two 16-byte chunks (columns [16 q, 16 q + 8) and
+    // [16 q + 8, 16 q + 16) of row ch) in every row tile with rows = channels.
+    const uint32_t oc0 = tc::bf_offset(ch, 16 * q), oc1 = tc::bf_offset(ch, 16 * q + 8);
+    // Element offset of (token 16 q, channel ch) in a [64][128] per-token
+    // buffer (raw inputs, staged outputs).
+    const int ro = 16 * q * kP + ch;
+    // the raw per-token inputs in region A
+    auto region_a = [&](int i) {
+        return reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<char*>(&sm) + offsetof(Sm, Hh) +
+                                                (size_t)i * kK * kP * 2);
+    };
+    __nv_bfloat16* const ra = region_a(0);
+    __nv_bfloat16* const rb = region_a(1);
+    __nv_bfloat16* const rz = region_a(2);
+    __nv_bfloat16* const rdy = region_a(3);
 
     // ------------------------------------------------------------ work units
     constexpr bool pieces = PIECES;  // the launch picks the instantiation by p.npieces
@@ -252,15 +305,28 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         return p.flags + ((int64_t)slot * Bt + bb) * p.ntiles + tile;
     };
     auto edge_row = [&]() { return p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d; };
-    auto gin = [&](const void* base) {
-        return static_cast<const Tin*>(base) + (int64_t)bb * L * d + c;
-    };
-    auto gout = [&](void* base) { return static_cast<Tout*>(base) + (int64_t)bb * L * d + c; };
     auto ck_at = [&](int k) { return p.ckpt + ((int64_t)bb * (p.nck + 1) + k) * d * N; };
 
     auto sync = [&]() {
         tc::fence_before_sync();
         __syncthreads();
+        tc::fence_after_sync();
+    };
+    // Bounded mbarrier waits: one warp polls (until a first time-out), the
+    // others wait at the block barrier.
+    auto wait_mb = [&](uint64_t* mb, uint32_t& ph) {
+        if (warp == kNT / 32 - 1 && !timed_out && !tc::mbar_wait(mb, ph, kSpin)) timed_out = true;
+        __syncthreads();
+        ph ^= 1u;
+        tc::fence_after_sync();
+    };
+    auto wait_mb2 = [&](uint64_t* ma, uint32_t& pa, uint64_t* mb, uint32_t& pb) {
+        if (warp == kNT / 32 - 1 && !timed_out &&
+            !(tc::mbar_wait(ma, pa, kSpin) && tc::mbar_wait(mb, pb, kSpin)))
+            timed_out = true;
+        __syncthreads();
+        pa ^= 1u;
+        pb ^= 1u;
         tc::fence_after_sync();
     };
     // TMEM carry columns of this thread (state columns [16 q, 16 q + 16)) <->
@@ -290,35 +356,62 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
         }
     };
-    // L2 prefetch of block k's inputs (one thread).
-    auto prefetch_block = [&](int k) {
+
+    // ------------------------------------------------------- TMA loads
+    // Per-token inputs of block k (thread 0): full: u, a, b, z, dout;
+    // adjoint only: a, z, dout.
+    auto load_raw = [&](int k, bool full) {
         const int x = (int)c0, y = k * kK, zb = bb;
-        tma::prefetch_l2_3d(&tm.u, x, y > 3 ? y - 3 : 0, zb);
-        tma::prefetch_l2_3d(&tm.a, x, y, zb);
-        if (has_b) tma::prefetch_l2_3d(&tm.b, x, y, zb);
-        if (has_z) tma::prefetch_l2_3d(&tm.z, x, y, zb);
-        tma::prefetch_l2_3d(&tm.dy, x, y, zb);
-        tma::prefetch_l2_3d(&tm.B, 0, y, zb);
-        tma::prefetch_l2_3d(&tm.C, 0, y, zb);
-        tma::prefetch_l2_3d(&tm.X, 0, x, (int)((int64_t)bb * (p.nck + 1) + k));
-        tma::prefetch_l2_3d(&tm.X, 32, x, (int)((int64_t)bb * (p.nck + 1) + k));
+        uint32_t rows = kK * (2 + (has_z ? 1 : 0));
+        if (full) rows += (kK + 3) + (has_b ? kK : 0);
+        tma::expect_tx(&sm.mb_in, rows * kP * 2u);
+        tma::load_3d(ra, &tm.a, x, y, zb, &sm.mb_in);
+        tma::load_3d(rdy, &tm.dy, x, y, zb, &sm.mb_in);
+        if (has_z) tma::load_3d(rz, &tm.z, x, y, zb, &sm.mb_in);
+        if (full) {
+            tma::load_3d(sm.ru, &tm.u, x, y - 3, zb, &sm.mb_in);
+            if (has_b) tma::load_3d(rb, &tm.b, x, y, zb, &sm.mb_in);
+        }
+    };
+    // C (and B when full) of block k into their tiles (thread 0).
+    auto load_bc = [&](int k, bool full) {
+        tma::expect_tx(&sm.mb_bc, (uint32_t)(2 * kK * kN * (full ? 2 : 1)));
+        tma::load_3d(sm.Cs, &tm.C, 0, k * kK, bb, &sm.mb_bc);
+        if (full) tma::load_3d(sm.Bs, &tm.B, 0, k * kK, bb, &sm.mb_bc);
+    };
+    // The fp32 checkpoint entering block k into the X tiles' bytes (thread 0):
+    // two swizzled boxes of 32 state columns.
+    auto load_x = [&](int k) {
+        tma::expect_tx(&sm.mb_x, (uint32_t)(kP * kN * 4));
+        const int zz = (int)((int64_t)bb * (p.nck + 1) + k);
+        tma::load_3d(sm.Xh, &tm.X, 0, (int)c0, zz, &sm.mb_x);
+        tma::load_3d(sm.Xl, &tm.X, 32, (int)c0, zz, &sm.mb_x);
+    };
+    // This thread's 16 checkpoint values from the fp32 landing layout (box
+    // q / 2, chunks 4 (q % 2) .. + 3 of row ch, XOR-permuted by ch % 8).
+    auto read_x = [&](float* xr) {
+        const char* base = reinterpret_cast<const char*>(sm.Xh) + (q >> 1) * 16384 + ch * 128;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 v =
+                *reinterpret_cast<const float4*>(base + ((((q & 1) * 4 + i) ^ (ch & 7)) << 4));
+            xr[4 * i] = v.x; xr[4 * i + 1] = v.y; xr[4 * i + 2] = v.z; xr[4 * i + 3] = v.w;
+        }
     };
 
     // ---------------------------------------------------- loop 1: decays
     // f and 1/f of this thread's 16 tokens, parked in tensor memory (slots 2
     // and 3); exchange of the quarter products; the exact-path decision.
     float Eb = 1.f, Qb = 1.f, E63 = 1.f;
-    auto decays = [&](int64_t tb, int nv) -> bool {
-        const Tin* ga = gin(p.a);
+    auto decays = [&](int nv) -> bool {
+        const __nv_bfloat16* rap = ra + ro;
+        const int nq = cvalid ? nv - 16 * q : 0;  // valid tokens of this thread
         float fv[16], qv[16];
         float Qh = 1.f, Eh = 1.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const int tt = 16 * q + k;
-            const bool valid = cvalid && tt < nv;
-            const float av = valid ? ldbf(ga + (tb + tt) * d) : 0.f;
-            const float ea = __expf(-av);
-            qv[k] = valid ? 1.f + ea : 1.f;
+            const bool valid = k < nq;
+            qv[k] = valid ? 1.f + __expf(-bf2f(rap[k * kP])) : 1.f;
             fv[k] = valid ? rcpa_(qv[k]) : 1.f;
             Qh *= qv[k];
             Eh *= fv[k];
@@ -354,19 +447,16 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     float dD_acc = 0.f;     // this block's sum of dy h (added to red6 in phase C)
     // u of window entry m (token 16q - 3 + m of the block)
     auto uwin = [&](int m) { return (m & 1) ? bf_hi(upk[m >> 1]) : bf_lo(upk[m >> 1]); };
-    auto unpack = [&](int64_t tb, int nv, bool slow) {
-        const Tin* gu = gin(p.hu);
-        const Tin* gbp = has_b ? gin(p.b) : nullptr;
-        const Tin* gz = has_z ? gin(p.z) : nullptr;
-        const Tin* gdy = gin(p.dy);
-        auto ubits = [&](int i) -> uint32_t {
-            const int tt = 16 * q - 3 + i;
-            const int64_t t = tb + tt;
-            const bool ok = cvalid && tt < nv && t >= 0 && (CONV || i >= 3);
-            return ok ? (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(gu + t * d)) : 0u;
-        };
+    auto unpack = [&](int nv, bool slow) {
+        const unsigned short* rup = reinterpret_cast<const unsigned short*>(sm.ru) + ro;
+        const __nv_bfloat16* rbp = rb + ro;
+        const __nv_bfloat16* rzp = rz + ro;
+        const __nv_bfloat16* rdp = rdy + ro;
+        const int nq = cvalid ? nv - 16 * q : 0;
 #pragma unroll
-        for (int i = 0; i < 10; ++i) upk[i] = ubits(2 * i) | (i < 9 ? ubits(2 * i + 1) << 16 : 0u);
+        for (int i = 0; i < 10; ++i)
+            upk[i] = (uint32_t)rup[(2 * i) * kP] |
+                     (i < 9 ? (uint32_t)rup[(2 * i + 1) * kP] << 16 : 0u);
         float E = slow ? 1.f : Eb, Q = slow ? 1.f : Qb;
         dD_acc = 0.f;
 #pragma unroll
@@ -379,9 +469,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
                 const int k = 4 * g4 + k4;
-                const int tt = 16 * q + k;
-                const int64_t t = tb + tt;
-                const bool valid = cvalid && tt < nv;
+                const bool valid = k < nq;
                 float h, spd = 1.f;
                 if (CONV) {
                     const float pp = fmaf(w3, uwin(k + 3), fmaf(w2, uwin(k + 2),
@@ -396,15 +484,15 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 const float f = fa[k4], qq = qa[k4];
                 // 1 - f = (1/f - 1) f, exact for f near 1; 1 where exp(-a) overflowed
                 const float omf = qq < 3.0e38f ? (qq - 1.f) * f : 1.f;
-                const float iw = has_b ? (valid ? sigmoida_(ldbf(gbp + t * d)) : 0.f) : omf;
+                const float iw = has_b ? sigmoida_(bf2f(rbp[k * kP])) : omf;
                 float gg = 1.f, gd = 0.f;
                 if (has_z) {
-                    const float zv = valid ? ldbf(gz + t * d) : 0.f;
+                    const float zv = bf2f(rzp[k * kP]);
                     const float sz = sigmoida_(zv);
                     gg = zv * sz;
                     gd = sz * fmaf(zv, 1.f - sz, 1.f);
                 }
-                const float dout = valid ? ldbf(gdy + t * d) : 0.f;
+                const float dout = bf2f(rdp[k * kP]);  // zero outside the tensor
                 const float dyv = dout * gg;
                 const float dzc = dout * gd;
                 if (!slow) {
@@ -422,50 +510,36 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 c0v[k] = valid ? Dc * dyv * spd : 0.f;
                 dD_acc = fmaf(dyv, h, dD_acc);
             }
-            st4(sm.Wh, sm.Wl, ch, col, Wv[0], Wv[1], Wv[2], Wv[3]);
-            st4(sm.Uh, sm.Ul, ch, col, Uv[0], Uv[1], Uv[2], Uv[3]);
+            const uint32_t o = (g4 < 2 ? oc0 : oc1) + (g4 & 1) * 8;
+            {
+                uint32_t h0, l0, h1, l1;
+                split2(Wv[0], Wv[1], h0, l0);
+                split2(Wv[2], Wv[3], h1, l1);
+                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Wh) + o) = make_uint2(h0, h1);
+                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Wl) + o) = make_uint2(l0, l1);
+                split2(Uv[0], Uv[1], h0, l0);
+                split2(Uv[2], Uv[3], h1, l1);
+                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Uh) + o) = make_uint2(h0, h1);
+                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Ul) + o) = make_uint2(l0, l1);
+            }
             tc::tmem_st4(trow + Cols::SV + 0 * 64 + col, s0);
             tc::tmem_st4(trow + Cols::SV + 1 * 64 + col, s1);
             tc::tmem_st4(trow + Cols::SV + 2 * 64 + col, s2);
             tc::tmem_st4(trow + Cols::SV + 3 * 64 + col, s3);
         }
     };
-    // B (when want_b) and C rows of the block to their exact bf16 tiles: one
-    // 16-byte chunk (8 state columns of one token) per thread and tile.
-    auto load_bc = [&](int64_t tb, int nv, bool want_b) {
-        const int tt = tid >> 3, j = (tid & 7) * 8;
-        uint4 br = make_uint4(0u, 0u, 0u, 0u), cr = br;
-        if (tt < nv) {
-            const int64_t off = ((int64_t)bb * L + tb + tt) * N + j;
-            cr = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.C) + off));
-            if (want_b) br = __ldg(reinterpret_cast<const uint4*>(static_cast<const Tin*>(p.B) + off));
-        }
-        const uint32_t o = tc::bf_offset(tt, j);
-        *reinterpret_cast<uint4*>(reinterpret_cast<char*>(sm.Cs) + o) = cr;
-        if (want_b) *reinterpret_cast<uint4*>(reinterpret_cast<char*>(sm.Bs) + o) = br;
-    };
-    // This block's checkpoint (the state entering it) to the X tile pair:
-    // this thread's 16 state columns of its channel.
-    auto load_x = [&](int k) {
-        const float* xs = ck_at(k) + c * N + 16 * q;
-        float4 v[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            v[i] = cvalid ? __ldcg(reinterpret_cast<const float4*>(xs) + i)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) st4(sm.Xh, sm.Xl, ch, 16 * q + 4 * i, v[i].x, v[i].y, v[i].z, v[i].w);
-    };
-    // H' = E_63 H into the H tile pair and into the carry accumulator (its
+    // H' = E_63 H into tensor memory and (tiles) into the H tile pair (its
     // initial value: carry out = U C + H').
-    auto scale_carry = [&]() {
+    auto scale_carry = [&](bool tiles) {
         float hv[16];
         tc::tmem_ld16(trow + Cols::H + 16 * q, hv);
         tc::tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 16; ++j) hv[j] *= E63;
-#pragma unroll
-        for (int j = 0; j < 16; j += 4) st4(sm.Hh, sm.Hl, ch, 16 * q + j, hv[j], hv[j + 1], hv[j + 2], hv[j + 3]);
+        if (tiles) {
+            st8o(sm.Hh, sm.Hl, oc0, hv);
+            st8o(sm.Hh, sm.Hl, oc1, hv + 8);
+        }
         tc::tmem_st16(trow + Cols::H + 16 * q, hv);
     };
 
@@ -520,21 +594,17 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
               kK / 16, tc::idesc_bf16(128, 64, false, true), fg);
         prod3(tbase + Cols::BC, NAJU_SA(Xh), NAJU_SA(Xl), true, NAJU_SA(Uh), NAJU_SA(Ul), true,
               kP / 16, tc::idesc_bf16(64, 64, true, true), fc);
-        {
-            // B^T Pm^T: B (rows m = K) against Pm (rows t, K = m): hi and lo of Pm
-            prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Ph), false, kK / 16,
-                 tc::idesc_bf16(64, 64, true, false), fc);
-            prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Pl), false, kK / 16,
-                 tc::idesc_bf16(64, 64, true, false), fc);
-        }
+        // B^T Pm^T: B (rows m = K) against Pm (rows t, K = m): hi and lo of Pm
+        prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Ph), false, kK / 16,
+             tc::idesc_bf16(64, 64, true, false), fc);
+        prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Pl), false, kK / 16,
+             tc::idesc_bf16(64, 64, true, false), fc);
         prod3(tbase + lane16 + Cols::BC, NAJU_SA(Hh), NAJU_SA(Hl), true, NAJU_SA(Wh), NAJU_SA(Wl),
               true, kP / 16, tc::idesc_bf16(64, 64, true, true), fb);
-        {
-            prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Ph), true, kK / 16,
-                 tc::idesc_bf16(64, 64, true, true), fb);
-            prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Pl), true, kK / 16,
-                 tc::idesc_bf16(64, 64, true, true), fb);
-        }
+        prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Ph), true, kK / 16,
+             tc::idesc_bf16(64, 64, true, true), fb);
+        prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Pl), true, kK / 16,
+             tc::idesc_bf16(64, 64, true, true), fb);
         tc::mma_commit(&sm.mb2);
     };
     // G (lanes +0) and P (lanes +16) from tensor memory to their tile pairs,
@@ -544,21 +614,13 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tc::tmem_ld16(trow + Cols::BC + 16 * q, v);
         tc::tmem_ld_wait();
         const int row = 16 * s4 + (lid & 15);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (16 * q + j > row) v[j] = 0.f;
         __nv_bfloat16* dh = lid < 16 ? sm.Gh : sm.Ph;
         __nv_bfloat16* dl = lid < 16 ? sm.Gl : sm.Pl;
-#pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-            const int col = 16 * q + j;
-            st4(dh, dl, row, col, col + 0 <= row ? v[j] : 0.f, col + 1 <= row ? v[j + 1] : 0.f,
-                col + 2 <= row ? v[j + 2] : 0.f, col + 3 <= row ? v[j + 3] : 0.f);
-        }
-    };
-    auto wait_mb = [&](uint64_t* mb, uint32_t& ph) {
-        // one warp polls; the others wait at the block barrier
-        if (warp == kNT / 32 - 1 && !tc::mbar_wait(mb, ph, kSpin)) timed_out = true;
-        __syncthreads();
-        ph ^= 1u;
-        tc::fence_after_sync();
+        st8o(dh, dl, tc::bf_offset(row, 16 * q), v);
+        st8o(dh, dl, tc::bf_offset(row, 16 * q + 8), v + 8);
     };
 
     // ---------------------------------------------------- exact path
@@ -566,6 +628,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     // range.  W holds v, U holds s dy (E = Q = 1), f = 1 - (saved 1 - f).
     // Results go where the MMAs would have put them: R <- x.C, GB <- lambda.B,
     // carry <- f_0 lambda_0; dB and dC are added to the accumulator directly.
+    // Its row sums live in region A (the per-token inputs are read by now).
     auto exact_block = [&](int64_t tb, int nv) {
         float* rsum = reinterpret_cast<float*>(sm.Gh);  // [64 t][128 ch] over G and P
         float* gsum = reinterpret_cast<float*>(sm.Hh);  // [64 t][128 ch] over the H pair
@@ -582,10 +645,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tc::tmem_ld_wait();
         float x[16];
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-            const float4 x4 = ld4(sm.Xh, sm.Xl, ch, 16 * q + j);
-            x[j] = x4.x; x[j + 1] = x4.y; x[j + 2] = x4.z; x[j + 3] = x4.w;
-        }
+        for (int j = 0; j < 16; j += 4) ld4o(sm.Xh, sm.Xl, (j < 8 ? oc0 : oc1) + (j & 4) * 2, x + j);
         __syncthreads();
         float* acc = p.dBCp + (int64_t)bb * L * 2 * N;
         for (int tt = 0; tt < nv; ++tt) {
@@ -658,16 +718,20 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     if (!pieces && !firstg) {
         const float* dxf = p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr;
         carry_from(lastg ? dxf : nullptr, false);
+        if (tid == 0) {
+            load_raw(kb1 - 1, false);
+            load_bc(kb1 - 1, false);
+        }
         float logF = 0.f;
         for (int k = kb1 - 1; k >= kb0; --k) {
             const int64_t tb = (int64_t)k * kK;
             const int nv = (int)min64((int64_t)kK, L - tb);
-            if (tid == 0 && k > kb0) prefetch_block(k - 1);
-            const bool slow = decays(tb, nv);
+            wait_mb(&sm.mb_in, ph_in);
+            const bool slow = decays(nv);
             // U = s dy E (slow: s dy)
             {
-                const Tin* gz = has_z ? gin(p.z) : nullptr;
-                const Tin* gdy = gin(p.dy);
+                const __nv_bfloat16* rzp = rz + ro;
+                const __nv_bfloat16* rdp = rdy + ro;
                 float E = slow ? 1.f : Eb;
 #pragma unroll
                 for (int g4 = 0; g4 < 4; ++g4) {
@@ -677,26 +741,33 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
-                        const int kk = 4 * g4 + k4, tt = 16 * q + kk;
-                        const bool valid = cvalid && tt < nv;
+                        const int kk = 4 * g4 + k4;
                         float gg = 1.f;
                         if (has_z) {
-                            const float zv = valid ? ldbf(gz + (tb + tt) * d) : 0.f;
+                            const float zv = bf2f(rzp[kk * kP]);
                             gg = zv * sigmoida_(zv);
                         }
-                        const float dout = valid ? ldbf(gdy + (tb + tt) * d) : 0.f;
+                        const float dout = bf2f(rdp[kk * kP]);  // zero outside the tensor
                         if (!slow) E *= fa[k4];
                         Uv[k4] = sc * dout * gg * E;
                     }
-                    st4(sm.Uh, sm.Ul, ch, col, Uv[0], Uv[1], Uv[2], Uv[3]);
+                    uint32_t h0, l0, h1, l1;
+                    split2(Uv[0], Uv[1], h0, l0);
+                    split2(Uv[2], Uv[3], h1, l1);
+                    const uint32_t o = (g4 < 2 ? oc0 : oc1) + (g4 & 1) * 8;
+                    *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Uh) + o) = make_uint2(h0, h1);
+                    *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Ul) + o) = make_uint2(l0, l1);
                 }
             }
-            load_bc(tb, nv, false);
+            tc::tmem_st_wait();
+            tc::fence_proxy_async();
+            sync();  // the per-token inputs are read
+            if (tid == 0 && k > kb0) load_raw(k - 1, false);
+            wait_mb(&sm.mb_bc, ph_bc);
             logF += __logf(E63);
             if (!slow) {
-                scale_carry();
+                scale_carry(false);
                 tc::tmem_st_wait();
-                tc::fence_proxy_async();
                 sync();
                 if (tid == 0) {
                     bool fh = false;
@@ -706,9 +777,9 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 }
                 wait_mb(&sm.mb2, ph2);
             } else {
-                sync();
                 exact_carry(nv);
             }
+            if (tid == 0 && k > kb0) load_bc(k - 1, false);  // the C tile is free
         }
         if (!lastg) {
             if (tid == 0) sm.ok = wait_flag(flag_slot(g), &p.hdr->status, p.wait_limit) ? 1 : 0;
@@ -781,19 +852,30 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 for (int v = 0; v < 6; ++v) sm.red6[v][ch] = 0.f;
             }
         }
-        if (tid == 0) prefetch_block(kb1 - 1);
+        if (tid == 0) {
+            load_raw(kb1 - 1, true);
+            load_bc(kb1 - 1, true);
+            load_x(kb1 - 1);
+        }
         sync();
 
         for (int k = kb1 - 1; k >= kb0; --k, par ^= 1) {
             const int64_t tb = (int64_t)k * kK;
             const int nv = (int)min64((int64_t)kK, L - tb);
-            if (tid == 0 && k > kb0) prefetch_block(k - 1);
+            const int nq = cvalid ? nv - 16 * q : 0;  // valid tokens of this thread
             // ------------------------------------------------ phase A
-            const bool slow = decays(tb, nv);
-            unpack(tb, nv, slow);
-            load_bc(tb, nv, true);
-            load_x(k);
-            if (!slow) scale_carry();
+            // (the previous block's staged outputs must have left the W / U bytes)
+            if (kStage && tid == 0) tma::store_wait_read();
+            wait_mb2(&sm.mb_in, ph_in, &sm.mb_x, ph_x);
+            float xr[16];
+            read_x(xr);
+            const bool slow = decays(nv);  // (its barriers end the reads of the fp32 checkpoint)
+            st8o(sm.Xh, sm.Xl, oc0, xr);
+            st8o(sm.Xh, sm.Xl, oc1, xr + 8);
+            unpack(nv, slow);
+            tc::tmem_st_wait();
+            wait_mb(&sm.mb_bc, ph_bc);  // and region A's per-token inputs are read
+            if (!slow) scale_carry(true);
             tc::tmem_st_wait();
             tc::fence_proxy_async();
             sync();
@@ -810,54 +892,56 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 exact_block(tb, nv);
             }
             // ------------------------------------------------ phase C
-            // Pass 1 (tokens in order): dL, dz, db; the quarter's sum of dL and
-            // its first three dp for the neighbouring quarter.
+            // Region A, the u buffer and the B, C tiles are free: the earlier
+            // block's inputs are requested.
+            if (tid == 0 && k > kb0) {
+                load_raw(k - 1, true);
+                load_bc(k - 1, true);
+            }
+            // tail of the earlier block: (carry entering it) . (this block's X)
+            {
+                float hx[16], xv[16];
+                tc::tmem_ld16(trow + Cols::H + 16 * q, hx);
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                    ld4o(sm.Xh, sm.Xl, (j < 8 ? oc0 : oc1) + (j & 4) * 2, xv + j);
+                tc::tmem_ld_wait();
+                float tp = 0.f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) tp = fmaf(hx[j], xv[j], tp);
+                sm.tailp[par ^ 1][q][ch] = tp;
+            }
+            // Pass 1 (tokens in order): dL; the quarter's sum of dL and its
+            // first three dp for the neighbouring quarter.
             float dL[16];
             float qsum = 0.f, dpf0 = 0.f, dpf1 = 0.f, dpf2 = 0.f;
 #pragma unroll
             for (int g4 = 0; g4 < 4; ++g4) {
                 const int col = 16 * q + 4 * g4;
-                float R4[4], G4[4], z1[4], z0[4], b2[4];
+                float R4[4], G4[4], b2[4], Ua[4], Wa[4];
                 tc::tmem_ld4(trow + Cols::R + col, R4);
                 tc::tmem_ld4(trow + Cols::GB + col, G4);
-                tc::tmem_ld4(trow + Cols::SV + 0 * 64 + col, z1);
-                tc::tmem_ld4(trow + Cols::SV + 1 * 64 + col, z0);
-                tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
+                if (!has_b) tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
+                const uint32_t o = (g4 < 2 ? oc0 : oc1) + (g4 & 1) * 8;
+                ld4o(sm.Uh, sm.Ul, o, Ua);
+                ld4o(sm.Wh, sm.Wl, o, Wa);
                 tc::tmem_ld_wait();
-                const float4 U4 = ld4(sm.Uh, sm.Ul, ch, col);
-                const float4 W4 = ld4(sm.Wh, sm.Wl, ch, col);
-                const float Ua[4] = {U4.x, U4.y, U4.z, U4.w};
-                const float Wa[4] = {W4.x, W4.y, W4.z, W4.w};
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
-                    const int kk = 4 * g4 + k4, tt = col + k4;
-                    const int64_t t = tb + tt;
-                    const bool valid = cvalid && tt < nv;
+                    const int kk = 4 * g4 + k4;
                     float dl = Ua[k4] * R4[k4] - Wa[k4] * G4[k4];
-                    // coupled gate: this token's da loses f h lambda.B (kept in dL[kk])
-                    if (!has_b) dl = fmaf(-b2[k4], G4[k4], dl);
+                    if (has_b) {
+                        qsum += dl;
+                    } else {
+                        // coupled gate: the sums over later tokens keep the plain dL,
+                        // this token's da loses f h lambda.B (kept in dL[kk])
+                        qsum += dl;
+                        dl = fmaf(-b2[k4], G4[k4], dl);
+                    }
                     dL[kk] = dl;
-                    qsum += dl;
                     if (kk == 0) dpf0 = fmaf(c1v[0], G4[k4], c0v[0]);
                     if (kk == 1) dpf1 = fmaf(c1v[1], G4[k4], c0v[1]);
                     if (kk == 2) dpf2 = fmaf(c1v[2], G4[k4], c0v[2]);
-                    if (valid) {
-                        if (has_z) gout(p.dz)[t * d] = from_f<Tout>(fmaf(z1[k4], R4[k4], z0[k4]));
-                        if (has_b) gout(p.db)[t * d] = from_f<Tout>(b2[k4] * G4[k4]);
-                    }
-                }
-            }
-            if (!has_b) {  // the sums over later tokens keep the plain dL
-                qsum = 0.f;
-#pragma unroll
-                for (int g4 = 0; g4 < 4; ++g4) {
-                    const int col = 16 * q + 4 * g4;
-                    float G4[4], b2[4];
-                    tc::tmem_ld4(trow + Cols::GB + col, G4);
-                    tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
-                    tc::tmem_ld_wait();
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) qsum += fmaf(b2[k4], G4[k4], dL[4 * g4 + k4]);
                 }
             }
             sm.xs[q][ch] = qsum;
@@ -865,6 +949,8 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             sm.dph[q][1][ch] = dpf1;
             sm.dph[q][2][ch] = dpf2;
             __syncthreads();
+            // the X tiles and the W, U tiles are read: the next checkpoint may land
+            if (tid == 0 && k > kb0) load_x(k - 1);
             float base = 0.f;  // dL over the later quarters, plus the tail
 #pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
@@ -881,25 +967,38 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 n2 = sm.dnext[par][1][ch];
                 n3 = sm.dnext[par][2][ch];
             }
-            // Pass 2 (tokens in reverse): da from the suffix sums of dL; dp,
-            // the conv backward (du, dw, dbias) from a window of later dp.
+            // Pass 2 (tokens in reverse): da from the suffix sums of dL, dz, db;
+            // dp, the conv backward (du, dw, dbias) from a window of later dp.
+            // bf16 gradients go to the staging buffers over the W and U tiles
+            // (dz, db, da, dh or du), fp32 ones straight to global memory.
             {
+                const int64_t gofs = ((int64_t)bb * L + tb + 16 * q) * d + c;
+                auto put = [&](__nv_bfloat16* stage, void* gbase, int kk, float v) {
+                    if constexpr (kStage) {
+                        stage[ro + kk * kP] = __float2bfloat16_rn(v);
+                    } else {
+                        if (kk < nq) static_cast<float*>(gbase)[gofs + (int64_t)kk * d] = v;
+                    }
+                };
                 float dw0 = 0.f, dw1 = 0.f, dw2 = 0.f, dw3 = 0.f, dbias = 0.f;
                 float run = base;
-                const bool seg_end = !lastg && k == kb1 - 1;
+                const bool seg_end = !lastg && k == kb1 - 1;  // a full block
 #pragma unroll
                 for (int g4 = 3; g4 >= 0; --g4) {
                     const int col = 16 * q + 4 * g4;
-                    float G4[4], om[4], b2[4];
+                    float G4[4], om[4], b2[4], R4[4], z1[4], z0[4];
                     tc::tmem_ld4(trow + Cols::GB + col, G4);
                     tc::tmem_ld4(trow + Cols::SV + 3 * 64 + col, om);
                     tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
+                    if (has_z) {
+                        tc::tmem_ld4(trow + Cols::R + col, R4);
+                        tc::tmem_ld4(trow + Cols::SV + 0 * 64 + col, z1);
+                        tc::tmem_ld4(trow + Cols::SV + 1 * 64 + col, z0);
+                    }
                     tc::tmem_ld_wait();
 #pragma unroll
                     for (int k4 = 3; k4 >= 0; --k4) {
-                        const int kk = 4 * g4 + k4, tt = col + k4;
-                        const int64_t t = tb + tt;
-                        const bool valid = cvalid && tt < nv;
+                        const int kk = 4 * g4 + k4;
                         float fdf;
                         if (has_b) {
                             run += dL[kk];
@@ -908,28 +1007,28 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                             fdf = run + dL[kk];
                             run += fmaf(b2[k4], G4[k4], dL[kk]);
                         }
-                        const float dpv = fmaf(c1v[kk], G4[k4], c0v[kk]);
-                        if (valid) gout(p.da)[t * d] = from_f<Tout>(fdf * om[k4]);
+                        put(sm.Uh, p.da, kk, fdf * om[k4]);
+                        if (has_z) put(sm.Wh, p.dz, kk, fmaf(z1[k4], R4[k4], z0[k4]));
+                        if (has_b) put(sm.Wl, p.db, kk, b2[k4] * G4[k4]);
+                        const float dpv = fmaf(c1v[kk], G4[k4], c0v[kk]);  // 0 outside
                         if (CONV) {
                             const float duv = fmaf(w3, dpv, fmaf(w2, n1, fmaf(w1, n2, w0 * n3)));
-                            if (valid) {
-                                dw0 = fmaf(dpv, uwin(kk), dw0);
-                                dw1 = fmaf(dpv, uwin(kk + 1), dw1);
-                                dw2 = fmaf(dpv, uwin(kk + 2), dw2);
-                                dw3 = fmaf(dpv, uwin(kk + 3), dw3);
-                                dbias += dpv;
-                                if (seg_end && tt >= nv - 3) {
-                                    edge_row()[(3 + (tt - (nv - 3))) * d + c] = duv;  // fixed up later
-                                } else {
-                                    gout(p.dhu)[t * d] = from_f<Tout>(duv);
-                                }
-                                if (k == kb0 && tt < 3) edge_row()[tt * d + c] = dpv;
-                            }
+                            // u and dp vanish outside the tensor: no masks
+                            dw0 = fmaf(dpv, uwin(kk), dw0);
+                            dw1 = fmaf(dpv, uwin(kk + 1), dw1);
+                            dw2 = fmaf(dpv, uwin(kk + 2), dw2);
+                            dw3 = fmaf(dpv, uwin(kk + 3), dw3);
+                            dbias += dpv;
+                            put(sm.Ul, p.dhu, kk, duv);
+                            // the segment's last three du are partial (fixed up later)
+                            if (kk >= 13 && q == 3 && seg_end && cvalid)
+                                edge_row()[(3 + (kk - 13)) * d + c] = duv;
+                            if (kk < 3 && q == 0 && k == kb0 && kk < nq) edge_row()[kk * d + c] = dpv;
                             n3 = n2;
                             n2 = n1;
                             n1 = dpv;
-                        } else if (valid) {
-                            gout(p.dhu)[t * d] = from_f<Tout>(dpv);
+                        } else {
+                            put(sm.Ul, p.dhu, kk, dpv);
                         }
                     }
                 }
@@ -952,35 +1051,27 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 tc::tmem_ld_wait();
                 const int j = 16 * s4 + (lid & 15);
                 const int slot = lid < 16 ? 1 : 0;  // slot 0 dB, 1 dC
-                float* acc = p.dBCp + (int64_t)bb * L * 2 * N + slot * N + j;
+                float* acc = p.dBCp + ((int64_t)bb * L + tb + 16 * q) * 2 * N + slot * N + j;
+                const int nvq = nv - 16 * q;
 #pragma unroll
-                for (int k2 = 0; k2 < 16; ++k2) {
-                    const int tt = 16 * q + k2;
-                    if (tt < nv) red_add(acc + (tb + tt) * 2 * N, v[k2]);
-                }
+                for (int k2 = 0; k2 < 16; ++k2)
+                    if (k2 < nvq) red_add(acc + k2 * 2 * N, v[k2]);
             }
-            // tail of the earlier block: (carry entering it) . (this block's X)
-            {
-                float hx[16];
-                tc::tmem_ld16(trow + Cols::H + 16 * q, hx);
-                tc::tmem_ld_wait();
-                float tp = 0.f;
-#pragma unroll
-                for (int j = 0; j < 16; j += 4) {
-                    const float4 x4 = ld4(sm.Xh, sm.Xl, ch, 16 * q + j);
-                    tp = fmaf(hx[j], x4.x, tp);
-                    tp = fmaf(hx[j + 1], x4.y, tp);
-                    tp = fmaf(hx[j + 2], x4.z, tp);
-                    tp = fmaf(hx[j + 3], x4.w, tp);
-                }
-                sm.tailp[par ^ 1][q][ch] = tp;
-                if (q == 0) {
-                    sm.dnext[par ^ 1][0][ch] = dpf0;
-                    sm.dnext[par ^ 1][1][ch] = dpf1;
-                    sm.dnext[par ^ 1][2][ch] = dpf2;
-                }
+            if (q == 0) {
+                sm.dnext[par ^ 1][0][ch] = dpf0;
+                sm.dnext[par ^ 1][1][ch] = dpf1;
+                sm.dnext[par ^ 1][2][ch] = dpf2;
             }
+            if (kStage) tc::fence_proxy_async();  // staged outputs -> TMA
             sync();  // tiles and tensor memory free for the next block
+            if (kStage && tid == 0) {
+                const int x = (int)c0, y = (int)tb;
+                if (has_z) tma::store_3d(&tm.oz, x, y, bb, sm.Wh);
+                if (has_b) tma::store_3d(&tm.ob, x, y, bb, sm.Wl);
+                tma::store_3d(&tm.oa, x, y, bb, sm.Uh);
+                tma::store_3d(&tm.ou, x, y, bb, sm.Ul);
+                tma::store_commit();
+            }
         }
 
         // ------------------------------------------- carries and partials
@@ -1009,6 +1100,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     }
 #undef NAJU_SA
 
+    if (kStage && tid == 0) tma::store_wait_all();
     if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
     sync();
     if (warp == 0) tc::tmem_dealloc(tbase, 512);
@@ -1040,9 +1132,15 @@ static cudaError_t launch_blk_t(const BwdParams& p, cudaStream_t st) {
               (!p.b || tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, kK, kP)) &&
               (!p.z || tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, kK, kP)) &&
               tma_encode_bf16_3d(&tm.dy, p.dy, p.Bt, p.L, p.d, kK, kP) &&
-              tma_encode_bf16_3d(&tm.B, p.B, p.Bt, p.L, kN, kK, kN) &&
-              tma_encode_bf16_3d(&tm.C, p.C, p.Bt, p.L, kN, kK, kN) &&
+              tma_encode_bf16_3d_sw128(&tm.B, p.B, p.Bt, p.L, kN, kK) &&
+              tma_encode_bf16_3d_sw128(&tm.C, p.C, p.Bt, p.L, kN, kK) &&
               tma_encode_f32_3d_sw128(&tm.X, p.ckpt, p.Bt * (int64_t)(p.nck + 1), p.d, kN, kP);
+    if (ok && std::is_same<Tout, __nv_bfloat16>::value) {
+        ok = tma_encode_bf16_3d(&tm.oa, p.da, p.Bt, p.L, p.d, kK, kP) &&
+             tma_encode_bf16_3d(&tm.ou, p.dhu, p.Bt, p.L, p.d, kK, kP) &&
+             (!p.z || tma_encode_bf16_3d(&tm.oz, p.dz, p.Bt, p.L, p.d, kK, kP)) &&
+             (!p.b || tma_encode_bf16_3d(&tm.ob, p.db, p.Bt, p.L, p.d, kK, kP));
+    }
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(BkSmem);
     auto kern = scan_bwd_blk_kernel<Tout, CONV, PIECES>;

@@ -1,6 +1,7 @@
 // Tensor Memory Accelerator (TMA) support: host-side tensor-map encoding and
 // the device-side bulk tensor load into shared memory with an mbarrier
-// transaction count.  Loads only, never with cluster multicast.
+// transaction count, and the bulk tensor store back.  Never with cluster
+// multicast.
 //
 // A tensor map describes a row-major bf16 tensor [outer][rows][cols] and a
 // box [box_rows][box_cols]; a load copies the box at (col, row, outer) into
@@ -61,6 +62,31 @@ __device__ __forceinline__ void load_3d(void* dst, const CUtensorMap* map, int x
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z),
         "r"(static_cast<uint32_t>(__cvta_generic_to_shared(mbar)))
         : "memory");
+}
+
+// Box store from shared memory (the layout a load of the same map writes) to
+// (x, y, z); elements outside the tensor are not written.  x * 2 bytes must
+// be a multiple of 16 and no coordinate may be negative.  Generic writes to
+// the source must be fenced (fence.proxy.async) and synchronised first; the
+// store joins the issuing thread's current bulk group.
+__device__ __forceinline__ void store_3d(const CUtensorMap* map, int x, int y, int z,
+                                         const void* src) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(z), "r"(static_cast<uint32_t>(__cvta_generic_to_shared(src)))
+        : "memory");
+}
+__device__ __forceinline__ void store_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until the issuing thread's committed stores have read their shared
+// memory (the source may be rewritten), or have completed entirely.
+__device__ __forceinline__ void store_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void store_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Hint: bring the box at (x, y, z) into L2 (no shared memory, no completion

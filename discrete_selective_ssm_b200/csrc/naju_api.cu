@@ -66,7 +66,8 @@ struct Layout {
     bool fwd_tc, bwd_tc;
     int nck, ngroups, seg_per_group, ntiles_f, npieces_f;
     int nsub, nclus, ntiles_b, bgroups, blk_per_group, npieces;
-    size_t off_fflags, off_bflags, off_ckpt, off_carry, off_dbc, off_chan, off_edge, total;
+    size_t off_fflags, off_bflags, off_ckpt, off_carry, off_dbc, off_chan, off_edge, off_rgb,
+        off_tail, total;
 };
 
 bool use_fwd_tc(const naju_dims* dm) {
@@ -231,6 +232,12 @@ Layout layout(const naju_dims* dm) {
     off = up256(off + sizeof(float) * (size_t)Bt * groups_n * d * 8);
     l.off_edge = off;
     off = up256(off + sizeof(float) * (size_t)Bt * groups_n * 2 * 3 * d);
+    // d_state 128 block backward: the first pass's partial R, GB and tails
+    const bool halves = N == 128 && bwd_blk_supported(dm->dtype, N, d);
+    l.off_rgb = off;
+    off = up256(off + (halves ? sizeof(float) * (size_t)2 * Bt * L * d : 0));
+    l.off_tail = off;
+    off = up256(off + (halves ? sizeof(float) * (size_t)Bt * l.nsub * d : 0));
     l.total = off;
     return l;
 }
@@ -378,6 +385,8 @@ naju_status naju_scan_bwd(const naju_dims* dims, const void* hu, const float* co
     p.dBCp = reinterpret_cast<float*>(ws + l.off_dbc);
     p.chan_part = reinterpret_cast<float*>(ws + l.off_chan);
     p.conv_edge = reinterpret_cast<float*>(ws + l.off_edge);
+    p.rgb_part = reinterpret_cast<float*>(ws + l.off_rgb);
+    p.tail_part = reinterpret_cast<float*>(ws + l.off_tail);
     p.hdr = hdr;
     p.Bt = dims->batch; p.L = dims->seqlen; p.d = dims->d_inner; p.N = dims->d_state;
     p.T_ck = kTck; p.nck = l.nck; p.nsub = l.nsub; p.ntiles = l.ntiles_b; p.nclus = l.nclus;

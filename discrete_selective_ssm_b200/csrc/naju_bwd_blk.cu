@@ -1,6 +1,6 @@
 // Naju backward scan in block form on the 5th-generation tensor cores
 // (sm_100a, tcgen05, kind::f16 with fp32 accumulation), for bf16 activations
-// with d_state 64.
+// with d_state 64 (d_state 128 as two passes over 64-column state halves).
 //
 // Gradient of the Naju recurrence (Naju reproduction README, "Core
 // equations"): x_n = f_n x_{n-1} + i_n h_n B_n^T, y_n = x_n.C_n/sqrt(N) + D h_n,
@@ -95,6 +95,7 @@ struct alignas(64) BkTmaps {
     CUtensorMap B, C;            // bf16 [Bt][L][N]: 64 tokens x 64 columns, swizzled
     CUtensorMap X;               // fp32 checkpoints [Bt (nck+1)][d][N]: 128 x 32, swizzled
     CUtensorMap oz, ob, oa, ou;  // bf16 outputs dz, db, da, dh (du): 64 tokens x 128 channels
+    CUtensorMap pr, pg;          // second d_state-128 pass: partial R, GB [Bt][L][d] fp32 (L2 prefetch)
 };
 
 // Shared memory, 1024-byte aligned tiles.  Region A (the carry, G and P tile
@@ -185,13 +186,22 @@ __device__ __forceinline__ float ld1(const __nv_bfloat16* t, int row, int col) {
 
 }  // namespace
 
-template <typename Tout, bool CONV, bool PIECES>
+// MODE 0: d_state 64.  d_state 128 runs twice over 64-column halves of the
+// state (the columns evolve independently; only R, GB and the tail sums
+// couple them, and linearly): MODE 1 takes columns 0..63 and writes its
+// partial R, GB and tails to p.rgb_part / p.tail_part (no gradients of the
+// per-token inputs), MODE 2 takes columns 64..127, adds them and finishes.
+// The carry, dB, dC and the initial-state gradient split by columns.
+template <typename Tout, bool CONV, bool PIECES, int MODE>
 __global__ void __launch_bounds__(512, 1)
 scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
-    constexpr int N = kN;
+    constexpr int NS = MODE == 0 ? kN : 2 * kN;  // d_state (row stride of states)
+    constexpr int JH = MODE == 2 ? kN : 0;    // this pass's first state column
+    constexpr bool kExport = MODE == 1;
+    constexpr bool kImport = MODE == 2;
     // bf16 gradients leave through shared memory and TMA stores; fp32 ones
     // are stored directly
-    constexpr bool kStage = std::is_same<Tout, __nv_bfloat16>::value;
+    constexpr bool kStage = !kExport && std::is_same<Tout, __nv_bfloat16>::value;
     using Cols = BkCols;
     using Sm = BkSmem;
     extern __shared__ __align__(1024) float4 smem4[];
@@ -227,7 +237,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tma::prefetch_map(&tm.dy);
         tma::prefetch_map(&tm.B);
         tma::prefetch_map(&tm.C);
-        if (kStage) {
+        if constexpr (kStage) {
             tma::prefetch_map(&tm.oa);
             tma::prefetch_map(&tm.ou);
             if (has_z) tma::prefetch_map(&tm.oz);
@@ -300,12 +310,12 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         const int k0 = gg * p.blk_per_group;
         set_unit(item % per_g, gg, k0, min(k0 + p.blk_per_group, p.nsub));
     }
-    auto carry_slot = [&](int slot) { return p.carry + ((int64_t)slot * Bt + bb) * d * N; };
+    auto carry_slot = [&](int slot) { return p.carry + ((int64_t)slot * Bt + bb) * d * NS; };
     auto flag_slot = [&](int slot) {
         return p.flags + ((int64_t)slot * Bt + bb) * p.ntiles + tile;
     };
     auto edge_row = [&]() { return p.conv_edge + ((int64_t)bb * p.ngroups + g) * 2 * 3 * d; };
-    auto ck_at = [&](int k) { return p.ckpt + ((int64_t)bb * (p.nck + 1) + k) * d * N; };
+    auto ck_at = [&](int k) { return p.ckpt + ((int64_t)bb * (p.nck + 1) + k) * d * NS; };
 
     auto sync = [&]() {
         tc::fence_before_sync();
@@ -337,7 +347,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         for (int k = 0; k < 16; k += 4) {
             float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
             if (src && cvalid) {
-                const float4* s4p = reinterpret_cast<const float4*>(src + c * N + 16 * q + k);
+                const float4* s4p = reinterpret_cast<const float4*>(src + c * NS + JH + 16 * q + k);
                 v4 = cg ? __ldcg(s4p) : *s4p;
             }
             v[k] = v4.x; v[k + 1] = v4.y; v[k + 2] = v4.z; v[k + 3] = v4.w;
@@ -352,7 +362,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         if (cvalid) {
 #pragma unroll
             for (int k = 0; k < 16; k += 4)
-                *reinterpret_cast<float4*>(dst + c * N + 16 * q + k) =
+                *reinterpret_cast<float4*>(dst + c * NS + JH + 16 * q + k) =
                     make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
         }
     };
@@ -376,16 +386,16 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     // C (and B when full) of block k into their tiles (thread 0).
     auto load_bc = [&](int k, bool full) {
         tma::expect_tx(&sm.mb_bc, (uint32_t)(2 * kK * kN * (full ? 2 : 1)));
-        tma::load_3d(sm.Cs, &tm.C, 0, k * kK, bb, &sm.mb_bc);
-        if (full) tma::load_3d(sm.Bs, &tm.B, 0, k * kK, bb, &sm.mb_bc);
+        tma::load_3d(sm.Cs, &tm.C, JH, k * kK, bb, &sm.mb_bc);
+        if (full) tma::load_3d(sm.Bs, &tm.B, JH, k * kK, bb, &sm.mb_bc);
     };
     // The fp32 checkpoint entering block k into the X tiles' bytes (thread 0):
     // two swizzled boxes of 32 state columns.
     auto load_x = [&](int k) {
         tma::expect_tx(&sm.mb_x, (uint32_t)(kP * kN * 4));
         const int zz = (int)((int64_t)bb * (p.nck + 1) + k);
-        tma::load_3d(sm.Xh, &tm.X, 0, (int)c0, zz, &sm.mb_x);
-        tma::load_3d(sm.Xl, &tm.X, 32, (int)c0, zz, &sm.mb_x);
+        tma::load_3d(sm.Xh, &tm.X, JH, (int)c0, zz, &sm.mb_x);
+        tma::load_3d(sm.Xl, &tm.X, JH + 32, (int)c0, zz, &sm.mb_x);
     };
     // This thread's 16 checkpoint values from the fp32 landing layout (box
     // q / 2, chunks 4 (q % 2) .. + 3 of row ch, XOR-permuted by ch % 8).
@@ -522,9 +532,11 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Uh) + o) = make_uint2(h0, h1);
                 *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Ul) + o) = make_uint2(l0, l1);
             }
-            tc::tmem_st4(trow + Cols::SV + 0 * 64 + col, s0);
-            tc::tmem_st4(trow + Cols::SV + 1 * 64 + col, s1);
-            tc::tmem_st4(trow + Cols::SV + 2 * 64 + col, s2);
+            if constexpr (!kExport) {
+                tc::tmem_st4(trow + Cols::SV + 0 * 64 + col, s0);
+                tc::tmem_st4(trow + Cols::SV + 1 * 64 + col, s1);
+                tc::tmem_st4(trow + Cols::SV + 2 * 64 + col, s2);
+            }
             tc::tmem_st4(trow + Cols::SV + 3 * 64 + col, s3);
         }
     };
@@ -647,7 +659,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 #pragma unroll
         for (int j = 0; j < 16; j += 4) ld4o(sm.Xh, sm.Xl, (j < 8 ? oc0 : oc1) + (j & 4) * 2, x + j);
         __syncthreads();
-        float* acc = p.dBCp + (int64_t)bb * L * 2 * N;
+        float* acc = p.dBCp + (int64_t)bb * L * 2 * NS + JH;
         for (int tt = 0; tt < nv; ++tt) {
             const float f = f_at(tt), v = ld1(sm.Wh, sm.Wl, ch, tt), sdy = ld1(sm.Uh, sm.Ul, ch, tt);
             float rp = 0.f;
@@ -660,7 +672,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const float r = warp_sum(sdy * x[j]);
-                if (lid == 0) red_add(acc + (tb + tt) * 2 * N + N + 16 * q + j, r);
+                if (lid == 0) red_add(acc + (tb + tt) * 2 * NS + NS + 16 * q + j, r);
             }
         }
         for (int tt = nv - 1; tt >= 0; --tt) {
@@ -675,7 +687,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const float r = warp_sum(v * hx[j]);
-                if (lid == 0) red_add(acc + (tb + tt) * 2 * N + 16 * q + j, r);
+                if (lid == 0) red_add(acc + (tb + tt) * 2 * NS + 16 * q + j, r);
                 hx[j] *= f;
             }
         }
@@ -716,7 +728,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     // the last group), then the carry leaving the group's start is published
     // after adding the decayed carry of the later group (bounded wait).
     if (!pieces && !firstg) {
-        const float* dxf = p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr;
+        const float* dxf = p.dx_final ? p.dx_final + (int64_t)bb * d * NS : nullptr;
         carry_from(lastg ? dxf : nullptr, false);
         if (tid == 0) {
             load_raw(kb1 - 1, false);
@@ -794,7 +806,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             for (int k = 0; k < 16; k += 4) {
                 float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (okc && cvalid)
-                    v4 = __ldcg(reinterpret_cast<const float4*>(cin + c * N + 16 * q + k));
+                    v4 = __ldcg(reinterpret_cast<const float4*>(cin + c * NS + JH + 16 * q + k));
                 hx[k] = fmaf(Pf, v4.x, hx[k]);
                 hx[k + 1] = fmaf(Pf, v4.y, hx[k + 1]);
                 hx[k + 2] = fmaf(Pf, v4.z, hx[k + 2]);
@@ -820,7 +832,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         }
         // carry entering the segment's end, and the tail H . x at that end
         if (lastg) {
-            carry_from(p.dx_final ? p.dx_final + (int64_t)bb * d * N : nullptr, false);
+            carry_from(p.dx_final ? p.dx_final + (int64_t)bb * d * NS : nullptr, false);
         } else {
             const int slot = pieces ? 0 : g;
             if (tid == 0) sm.ok = wait_flag(flag_slot(slot), &p.hdr->status, p.wait_limit) ? 1 : 0;
@@ -837,7 +849,8 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             if (cvalid) {
 #pragma unroll
                 for (int k = 0; k < 16; k += 4) {
-                    const float4 x4 = __ldcg(reinterpret_cast<const float4*>(xe + c * N + 16 * q + k));
+                    const float4 x4 =
+                        __ldcg(reinterpret_cast<const float4*>(xe + c * NS + JH + 16 * q + k));
                     tp = fmaf(hx[k], x4.x, tp);
                     tp = fmaf(hx[k + 1], x4.y, tp);
                     tp = fmaf(hx[k + 2], x4.z, tp);
@@ -866,6 +879,13 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             // ------------------------------------------------ phase A
             // (the previous block's staged outputs must have left the W / U bytes)
             if (kStage && tid == 0) tma::store_wait_read();
+            if (kImport && tid == 0) {
+#pragma unroll
+                for (int i = 0; i < kP; i += 32) {
+                    tma::prefetch_l2_3d(&tm.pr, (int)c0 + i, (int)tb, bb);
+                    tma::prefetch_l2_3d(&tm.pg, (int)c0 + i, (int)tb, bb);
+                }
+            }
             wait_mb2(&sm.mb_in, ph_in, &sm.mb_x, ph_x);
             float xr[16];
             read_x(xr);
@@ -898,6 +918,25 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 load_raw(k - 1, true);
                 load_bc(k - 1, true);
             }
+            if constexpr (kImport) {
+                // the first pass's R and GB of this block (state columns 0..63)
+                const float* rp = p.rgb_part + ((int64_t)bb * L + tb + 16 * q) * d + c;
+                const float* gp = rp + Bt * L * d;
+                float r[16], gv[16];
+                tc::tmem_ld16(trow + Cols::R + 16 * q, r);
+                tc::tmem_ld16(trow + Cols::GB + 16 * q, gv);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    if (kk < nq) {
+                        r[kk] += __ldcg(rp + (int64_t)kk * d);
+                        gv[kk] += __ldcg(gp + (int64_t)kk * d);
+                    }
+                }
+                tc::tmem_st16(trow + Cols::R + 16 * q, r);
+                tc::tmem_st16(trow + Cols::GB + 16 * q, gv);
+                tc::tmem_st_wait();
+            }
             // tail of the earlier block: (carry entering it) . (this block's X)
             {
                 float hx[16], xv[16];
@@ -911,6 +950,30 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 for (int j = 0; j < 16; ++j) tp = fmaf(hx[j], xv[j], tp);
                 sm.tailp[par ^ 1][q][ch] = tp;
             }
+            if constexpr (kExport) {
+                // partial R, GB and this block's tail go to the second pass
+                float* rp = p.rgb_part + ((int64_t)bb * L + tb + 16 * q) * d + c;
+                float* gp = rp + Bt * L * d;
+                float r[16], gv[16];
+                tc::tmem_ld16(trow + Cols::R + 16 * q, r);
+                tc::tmem_ld16(trow + Cols::GB + 16 * q, gv);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    if (kk < nq) {
+                        rp[(int64_t)kk * d] = r[kk];
+                        gp[(int64_t)kk * d] = gv[kk];
+                    }
+                }
+                if (q == 0 && cvalid) {
+                    float ts = 0.f;
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) ts += sm.tailp[par][qq][ch];
+                    p.tail_part[((int64_t)bb * p.nsub + k) * d + c] = ts;
+                }
+                __syncthreads();
+                if (tid == 0 && k > kb0) load_x(k - 1);
+            } else {
             // Pass 1 (tokens in order): dL; the quarter's sum of dL and its
             // first three dp for the neighbouring quarter.
             float dL[16];
@@ -957,6 +1020,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 if (qq > q) base += sm.xs[qq][ch];
                 base += sm.tailp[par][qq][ch];
             }
+            if (kImport && cvalid) base += __ldcg(p.tail_part + ((int64_t)bb * p.nsub + k) * d + c);
             float n1, n2, n3;  // dp of the three tokens after the current one
             if (q < 3) {
                 n1 = sm.dph[q + 1][0][ch];
@@ -1032,6 +1096,11 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                         }
                     }
                 }
+                if (q == 0) {
+                    sm.dnext[par ^ 1][0][ch] = dpf0;
+                    sm.dnext[par ^ 1][1][ch] = dpf1;
+                    sm.dnext[par ^ 1][2][ch] = dpf2;
+                }
                 if (cvalid) {
                     atomicAdd(&sm.red6[0][ch], dD_acc);
                     if (CONV) {
@@ -1043,6 +1112,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     }
                 }
             }
+            }  // (gradients of the per-token inputs)
             // dC^T (lanes +0) and dB^T (lanes +16): this warp's lanes, columns
             // [16 q, 16 q + 16), added into the accumulator
             if (!slow) {
@@ -1051,16 +1121,11 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 tc::tmem_ld_wait();
                 const int j = 16 * s4 + (lid & 15);
                 const int slot = lid < 16 ? 1 : 0;  // slot 0 dB, 1 dC
-                float* acc = p.dBCp + ((int64_t)bb * L + tb + 16 * q) * 2 * N + slot * N + j;
+                float* acc = p.dBCp + ((int64_t)bb * L + tb + 16 * q) * 2 * NS + slot * NS + JH + j;
                 const int nvq = nv - 16 * q;
 #pragma unroll
                 for (int k2 = 0; k2 < 16; ++k2)
-                    if (k2 < nvq) red_add(acc + k2 * 2 * N, v[k2]);
-            }
-            if (q == 0) {
-                sm.dnext[par ^ 1][0][ch] = dpf0;
-                sm.dnext[par ^ 1][1][ch] = dpf1;
-                sm.dnext[par ^ 1][2][ch] = dpf2;
+                    if (k2 < nvq) red_add(acc + k2 * 2 * NS, v[k2]);
             }
             if (kStage) tc::fence_proxy_async();  // staged outputs -> TMA
             sync();  // tiles and tensor memory free for the next block
@@ -1076,14 +1141,14 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 
         // ------------------------------------------- carries and partials
         if (firstg) {
-            if (p.dx0) carry_to(p.dx0 + (int64_t)bb * d * N);
+            if (p.dx0) carry_to(p.dx0 + (int64_t)bb * d * NS);
         } else if (pieces) {
             carry_to(carry_slot(0));
             __threadfence();
             __syncthreads();
             if (tid == 0 && !p.fault_skip_publish) st_release(flag_slot(0), 1);
         }
-        {
+        if constexpr (!kExport) {
             float* cpart = p.chan_part + ((int64_t)bb * p.ngroups + g) * d * 8;
             __syncthreads();
             if (tid < kP && c0 + tid < d) {
@@ -1123,8 +1188,9 @@ __global__ void finish_dBC_kernel(const float* __restrict__ acc, int64_t BtL, in
     }
 }
 
-template <typename Tout, bool CONV, bool PIECES>
+template <typename Tout, bool CONV, bool PIECES, int MODE>
 static cudaError_t launch_blk_t(const BwdParams& p, cudaStream_t st) {
+    constexpr int NS = MODE == 0 ? kN : 2 * kN;
     BkTmaps tm;
     memset(&tm, 0, sizeof(tm));
     bool ok = tma_encode_bf16_3d(&tm.u, p.hu, p.Bt, p.L, p.d, kK + 3, kP) &&
@@ -1132,10 +1198,13 @@ static cudaError_t launch_blk_t(const BwdParams& p, cudaStream_t st) {
               (!p.b || tma_encode_bf16_3d(&tm.b, p.b, p.Bt, p.L, p.d, kK, kP)) &&
               (!p.z || tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, kK, kP)) &&
               tma_encode_bf16_3d(&tm.dy, p.dy, p.Bt, p.L, p.d, kK, kP) &&
-              tma_encode_bf16_3d_sw128(&tm.B, p.B, p.Bt, p.L, kN, kK) &&
-              tma_encode_bf16_3d_sw128(&tm.C, p.C, p.Bt, p.L, kN, kK) &&
-              tma_encode_f32_3d_sw128(&tm.X, p.ckpt, p.Bt * (int64_t)(p.nck + 1), p.d, kN, kP);
-    if (ok && std::is_same<Tout, __nv_bfloat16>::value) {
+              tma_encode_bf16_3d_sw128(&tm.B, p.B, p.Bt, p.L, NS, kK) &&
+              tma_encode_bf16_3d_sw128(&tm.C, p.C, p.Bt, p.L, NS, kK) &&
+              tma_encode_f32_3d_sw128(&tm.X, p.ckpt, p.Bt * (int64_t)(p.nck + 1), p.d, NS, kP);
+    if (ok && MODE == 2)
+        ok = tma_encode_f32_3d_sw128(&tm.pr, p.rgb_part, p.Bt, p.L, p.d, kK) &&
+             tma_encode_f32_3d_sw128(&tm.pg, p.rgb_part + p.Bt * p.L * p.d, p.Bt, p.L, p.d, kK);
+    if (ok && MODE != 1 && std::is_same<Tout, __nv_bfloat16>::value) {
         ok = tma_encode_bf16_3d(&tm.oa, p.da, p.Bt, p.L, p.d, kK, kP) &&
              tma_encode_bf16_3d(&tm.ou, p.dhu, p.Bt, p.L, p.d, kK, kP) &&
              (!p.z || tma_encode_bf16_3d(&tm.oz, p.dz, p.Bt, p.L, p.d, kK, kP)) &&
@@ -1143,7 +1212,7 @@ static cudaError_t launch_blk_t(const BwdParams& p, cudaStream_t st) {
     }
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(BkSmem);
-    auto kern = scan_bwd_blk_kernel<Tout, CONV, PIECES>;
+    auto kern = scan_bwd_blk_kernel<Tout, CONV, PIECES, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
@@ -1153,23 +1222,37 @@ static cudaError_t launch_blk_t(const BwdParams& p, cudaStream_t st) {
 }
 
 bool bwd_blk_supported(int dtype, int64_t N, int64_t d) {
-    return dtype == NAJU_BF16 && N == kN && d % 8 == 0;
+    return dtype == NAJU_BF16 && (N == kN || N == 2 * kN) && d % 8 == 0;
+}
+
+template <int MODE>
+static cudaError_t launch_blk_mode(const BwdParams& p, int out_dtype, cudaStream_t st) {
+    const bool conv = p.conv_w != nullptr, pc = p.npieces > 0;
+    if (out_dtype == NAJU_BF16) {
+        using T = __nv_bfloat16;
+        return conv ? (pc ? launch_blk_t<T, true, true, MODE>(p, st)
+                          : launch_blk_t<T, true, false, MODE>(p, st))
+                    : (pc ? launch_blk_t<T, false, true, MODE>(p, st)
+                          : launch_blk_t<T, false, false, MODE>(p, st));
+    }
+    return conv ? (pc ? launch_blk_t<float, true, true, MODE>(p, st)
+                      : launch_blk_t<float, true, false, MODE>(p, st))
+                : (pc ? launch_blk_t<float, false, true, MODE>(p, st)
+                      : launch_blk_t<float, false, false, MODE>(p, st));
 }
 
 cudaError_t launch_scan_bwd_blk(const BwdParams& p, int out_dtype, cudaStream_t st) {
     // the dB / dC accumulator starts at zero
     cudaError_t e = cudaMemsetAsync(p.dBCp, 0, sizeof(float) * (size_t)p.Bt * p.L * 2 * p.N, st);
     if (e != cudaSuccess) return e;
-    const bool conv = p.conv_w != nullptr, pc = p.npieces > 0;
-    if (out_dtype == NAJU_BF16) {
-        using T = __nv_bfloat16;
-        return conv ? (pc ? launch_blk_t<T, true, true>(p, st) : launch_blk_t<T, true, false>(p, st))
-                    : (pc ? launch_blk_t<T, false, true>(p, st) : launch_blk_t<T, false, false>(p, st));
-    }
-    return conv ? (pc ? launch_blk_t<float, true, true>(p, st)
-                      : launch_blk_t<float, true, false>(p, st))
-                : (pc ? launch_blk_t<float, false, true>(p, st)
-                      : launch_blk_t<float, false, false>(p, st));
+    if (p.N == kN) return launch_blk_mode<0>(p, out_dtype, st);
+    // d_state 128: state columns 0..63, then 64..127 with fresh tickets and flags
+    e = launch_blk_mode<1>(p, out_dtype, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(&p.hdr->bwd_ticket, 0, sizeof(int), st);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(p.flags, 0, sizeof(int) * (size_t)p.ngroups * p.Bt * p.ntiles, st);
+    if (e == cudaSuccess) e = launch_blk_mode<2>(p, out_dtype, st);
+    return e;
 }
 
 cudaError_t launch_finish_dBC(const BwdParams& p, int out_dtype, void* dB, void* dC,

@@ -69,6 +69,9 @@ struct BwdParams {
     float* dBCp;           // [nclus][Bt][L][2][N] partial dB, dC over channel clusters
     float* chan_part;      // [Bt*ngroups][d][8] partial dD, dconv_w[4], dconv_b
     float* conv_edge;      // [Bt][ngroups][2][3][d]: first 3 dp / last 3 partial du
+    float* rgb_part;       // block backward, d_state 128: [2][Bt][L][d] partial R, GB of
+                           // state columns 0..63 (first pass), read by the second
+    float* tail_part;      // same: [Bt][nsub][d] partial H . x_63 of each block
     WsHeader* hdr;
     int64_t Bt, L, d, N;
     int T_ck, nck;         // forward checkpoint spacing (== kBwdSub) and count
@@ -104,9 +107,11 @@ cudaError_t launch_bwd_reductions(const BwdParams& p, int out_dtype, void* dB, v
 // checkpoints every 64 tokens).
 bool fwd_blk_supported(int dtype, int64_t N, int64_t d, int T_ck);
 cudaError_t launch_scan_fwd_blk(const FwdParams& p, int out_dtype, cudaStream_t st);
-// Block-form tensor-core backward (bf16 activations, d_state 64): dB / dC go
-// into an fp32 accumulator [Bt][L][2][N] at p.dBCp (zeroed by the launch);
-// launch_bwd_reductions_acc then finishes dB, dC and the per-channel sums.
+// Block-form tensor-core backward (bf16 activations, d_state 64 or 128; 128 as
+// two passes over 64-column state halves through p.rgb_part / p.tail_part):
+// dB / dC go into an fp32 accumulator [Bt][L][2][N] at p.dBCp (zeroed by the
+// launch); launch_bwd_reductions_acc then finishes dB, dC and the per-channel
+// sums.
 bool bwd_blk_supported(int dtype, int64_t N, int64_t d);
 cudaError_t launch_scan_bwd_blk(const BwdParams& p, int out_dtype, cudaStream_t st);
 cudaError_t launch_finish_dBC(const BwdParams& p, int out_dtype, void* dB, void* dC,

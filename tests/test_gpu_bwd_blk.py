@@ -1,9 +1,9 @@
 """The block-form tensor-core backward (64-token blocks, bf16 activations,
-d_state 64) against the fp64 oracle, forced through the testing hook so it
-runs whatever the automatic choice is: every optional input, the coupled
-gate, both output dtypes, sequence groups, piece mode with cuts inside units,
-the exact path for blocks outside the factorisation's range, and ragged
-lengths and widths."""
+d_state 64, and 128 as two passes over state halves) against the fp64
+oracle, forced through the testing hook so it runs whatever the automatic
+choice is: every optional input, the coupled gate, both output dtypes,
+sequence groups, piece mode with cuts inside units, the exact path for
+blocks outside the factorisation's range, and ragged lengths and widths."""
 import pytest
 import torch
 
@@ -28,28 +28,32 @@ def _check(t, conv, out_dtype=naju.F32, **kw):
     compare_grads(g, oracle_bwd(t, conv), conv, TOL_BF16, bf16_out=out_dtype == naju.BF16, **kw)
 
 
+@pytest.mark.parametrize("N", [64, 128])
 @pytest.mark.parametrize("conv", [True, False])
-def test_blk_basic(conv):
-    w = wl(64, "bf16", Bt=2, L=333, d=264)
+def test_blk_basic(conv, N):
+    w = wl(N, "bf16", Bt=2, L=333, d=264)
     t = inputs(w, conv, use_x0=True, use_dxL=True)
-    assert naju.testing_bwd_impl(naju.make_dims(2, 333, 264, 64, naju.BF16)) == 3
+    assert naju.testing_bwd_impl(naju.make_dims(2, 333, 264, N, naju.BF16)) == 3
     _check(t, conv)
 
 
-def test_blk_bf16_outputs():
-    w = wl(64, "bf16", Bt=2, L=200, d=136)
+@pytest.mark.parametrize("N", [64, 128])
+def test_blk_bf16_outputs(N):
+    w = wl(N, "bf16", Bt=2, L=200, d=136)
     _check(inputs(w, True), True, out_dtype=naju.BF16)
 
 
-def test_blk_no_optional_inputs():
-    w = wl(64, "bf16", Bt=1, L=150, d=128)
+@pytest.mark.parametrize("N", [64, 128])
+def test_blk_no_optional_inputs(N):
+    w = wl(N, "bf16", Bt=1, L=150, d=128)
     t = inputs(w, False, use_z=False, use_D=False)
     _check(t, False, has_z=False, has_D=False)
 
 
+@pytest.mark.parametrize("N", [64, 128])
 @pytest.mark.parametrize("conv", [True, False])
-def test_blk_coupled_gate(conv):
-    w = wl(64, "bf16", Bt=2, L=260, d=136)
+def test_blk_coupled_gate(conv, N):
+    w = wl(N, "bf16", Bt=2, L=260, d=136)
     t = inputs(w, conv, use_x0=True, use_dxL=True)
     t["b"] = None
     g = run_bwd(t, conv, out_dtype=naju.F32)
@@ -60,35 +64,39 @@ def test_blk_coupled_gate(conv):
         assert_close(g[k], r[k], TOL_BF16, name=k)
 
 
+@pytest.mark.parametrize("N", [64, 128])
 @pytest.mark.parametrize("L", [1, 5, 63, 64, 65, 130])
-def test_blk_lengths(L):
-    w = wl(64, "bf16", Bt=2, L=L, d=136)
+def test_blk_lengths(L, N):
+    w = wl(N, "bf16", Bt=2, L=L, d=136)
     _check(inputs(w, True, use_x0=True, use_dxL=True), True)
 
 
+@pytest.mark.parametrize("N", [64, 128])
 @pytest.mark.parametrize("groups", [2, 3, 5])
-def test_blk_sequence_groups(groups):
-    w = wl(64, "bf16", Bt=2, L=600, d=136)
+def test_blk_sequence_groups(groups, N):
+    w = wl(N, "bf16", Bt=2, L=600, d=136)
     t = inputs(w, True, use_x0=True, use_dxL=True)
     naju.testing_set_bwd_groups(groups)
     _check(t, True)
 
 
+@pytest.mark.parametrize("N", [64, 128])
 @pytest.mark.parametrize("conv", [True, False])
 @pytest.mark.parametrize("pieces", [2, 4, 7])
-def test_blk_pieces(pieces, conv):
-    w = wl(64, "bf16", Bt=3, L=333, d=264)
+def test_blk_pieces(pieces, conv, N):
+    w = wl(N, "bf16", Bt=3, L=333, d=264)
     t = inputs(w, conv, use_x0=True, use_dxL=True)
     naju.testing_set_bwd_pieces(pieces)
-    assert naju.testing_bwd_pieces(naju.make_dims(3, 333, 264, 64, naju.BF16)) == pieces
+    assert naju.testing_bwd_pieces(naju.make_dims(3, 333, 264, N, naju.BF16)) == pieces
     _check(t, conv)
 
 
-def test_blk_exact_path():
+@pytest.mark.parametrize("N", [64, 128])
+def test_blk_exact_path(N):
     """Runs of vanishing forget gates push blocks outside the factorisation's
     range (decay below 2^-90 over 64 tokens): those blocks take the exact
     token-by-token path; f = 0 exactly and f = 1 exactly included."""
-    w = wl(64, "bf16", Bt=1, L=300, d=136)
+    w = wl(N, "bf16", Bt=1, L=300, d=136)
     t = inputs(w, True, use_x0=True, use_dxL=True)
     a = t["a"].float().clone()
     a[:, 40:60] = -60.0
@@ -99,9 +107,10 @@ def test_blk_exact_path():
     _check(t, True)
 
 
-def test_blk_exact_path_in_groups():
+@pytest.mark.parametrize("N", [64, 128])
+def test_blk_exact_path_in_groups(N):
     """The exact path inside the early (adjoint-only) pass of sequence groups."""
-    w = wl(64, "bf16", Bt=2, L=600, d=136)
+    w = wl(N, "bf16", Bt=2, L=600, d=136)
     t = inputs(w, True, use_x0=True, use_dxL=True)
     a = t["a"].float().clone()
     a[:, 330:350] = -60.0
@@ -122,14 +131,16 @@ def test_blk_moderate_decay_runs():
     _check(t, True)
 
 
-def test_blk_overwrite_events():
-    """The long-horizon distribution (5 % overwrite events) at d_state 64."""
-    w = wl(64, "bf16", Bt=2, L=700, d=136, base="long_retention")
+@pytest.mark.parametrize("N", [64, 128])
+def test_blk_overwrite_events(N):
+    """The long-horizon distribution (5 % overwrite events)."""
+    w = wl(N, "bf16", Bt=2, L=700, d=136, base="long_retention")
     _check(inputs(w, True, use_x0=True, use_dxL=True), True)
 
 
-def test_blk_pieces_timeout_is_reported():
-    w = wl(64, "bf16", Bt=2, L=320, d=256)
+@pytest.mark.parametrize("N", [64, 128])
+def test_blk_pieces_timeout_is_reported(N):
+    w = wl(N, "bf16", Bt=2, L=320, d=256)
     t = inputs(w, True)
     naju.testing_set_bwd_pieces(3)
     y, xf, ws = run_fwd(t, True)

@@ -298,7 +298,7 @@ def test_bwd_both_implementations(N, impl, conv):
     dm = naju.make_dims(2, 333, 264, N, naju.BF16)
     naju.testing_set_bwd_impl(impl)
     try:
-        assert naju.testing_bwd_impl(dm) == (impl if impl else (3 if N == 64 else 2))
+        assert naju.testing_bwd_impl(dm) == (impl if impl else 3)
         g = run_bwd(t, conv, out_dtype=naju.F32)
     finally:
         naju.testing_set_bwd_impl(0)

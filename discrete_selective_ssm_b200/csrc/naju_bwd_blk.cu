@@ -413,18 +413,29 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     // f and 1/f of this thread's 16 tokens, parked in tensor memory (slots 2
     // and 3); exchange of the quarter products; the exact-path decision.
     float Eb = 1.f, Qb = 1.f, E63 = 1.f;
+    // Tokens past the end (last block only) decay by 1; channels past d
+    // read zeros (finite values that are never stored).
     auto decays = [&](int nv) -> bool {
         const __nv_bfloat16* rap = ra + ro;
-        const int nq = cvalid ? nv - 16 * q : 0;  // valid tokens of this thread
         float fv[16], qv[16];
         float Qh = 1.f, Eh = 1.f;
+        if (nv == kK) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const bool valid = k < nq;
-            qv[k] = valid ? 1.f + __expf(-bf2f(rap[k * kP])) : 1.f;
-            fv[k] = valid ? rcpa_(qv[k]) : 1.f;
-            Qh *= qv[k];
-            Eh *= fv[k];
+            for (int k = 0; k < 16; ++k) {
+                qv[k] = 1.f + __expf(-bf2f(rap[k * kP]));
+                fv[k] = rcpa_(qv[k]);
+                Qh *= qv[k];
+                Eh *= fv[k];
+            }
+        } else {
+            const int nq = nv - 16 * q;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                qv[k] = k < nq ? 1.f + __expf(-bf2f(rap[k * kP])) : 1.f;
+                fv[k] = k < nq ? rcpa_(qv[k]) : 1.f;
+                Qh *= qv[k];
+                Eh *= fv[k];
+            }
         }
         tc::tmem_st16(trow + Cols::SV + 2 * 64 + 16 * q, fv);
         tc::tmem_st16(trow + Cols::SV + 3 * 64 + 16 * q, qv);
@@ -457,67 +468,82 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     float dD_acc = 0.f;     // this block's sum of dy h (added to red6 in phase C)
     // u of window entry m (token 16q - 3 + m of the block)
     auto uwin = [&](int m) { return (m & 1) ? bf_hi(upk[m >> 1]) : bf_lo(upk[m >> 1]); };
-    auto unpack = [&](int nv, bool slow) {
+    // No token masks: past the end, dout, B and C read zero, so U, GB and
+    // dp = c0 + c1 GB vanish and W meets only zero rows; the decays mask.
+    auto unpack = [&](bool slow) {
         const unsigned short* rup = reinterpret_cast<const unsigned short*>(sm.ru) + ro;
         const __nv_bfloat16* rbp = rb + ro;
         const __nv_bfloat16* rzp = rz + ro;
         const __nv_bfloat16* rdp = rdy + ro;
-        const int nq = cvalid ? nv - 16 * q : 0;
 #pragma unroll
         for (int i = 0; i < 10; ++i)
             upk[i] = (uint32_t)rup[(2 * i) * kP] |
                      (i < 9 ? (uint32_t)rup[(2 * i + 1) * kP] << 16 : 0u);
-        float E = slow ? 1.f : Eb, Q = slow ? 1.f : Qb;
+        float E = slow ? sc : sc * Eb, Q = slow ? 1.f : Qb;  // E carries the scale s
         dD_acc = 0.f;
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
             float Wv[4], Uv[4], s0[4], s1[4], s2[4], s3[4], fa[4], qa[4];
+            float hv[4], spd[4], iw[4], gg[4], gd[4], dout[4];
             const int col = 16 * q + 4 * g4;
             tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, fa);
             tc::tmem_ld4(trow + Cols::SV + 3 * 64 + col, qa);
-            tc::tmem_ld_wait();
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
                 const int k = 4 * g4 + k4;
-                const bool valid = k < nq;
-                float h, spd = 1.f;
                 if (CONV) {
                     const float pp = fmaf(w3, uwin(k + 3), fmaf(w2, uwin(k + 2),
                                          fmaf(w1, uwin(k + 1), fmaf(w0, uwin(k), wb))));
                     const float sp = sigmoida_(pp);
-                    h = pp * sp;
-                    spd = sp * fmaf(pp, 1.f - sp, 1.f);
+                    hv[k4] = pp * sp;
+                    spd[k4] = sp * fmaf(pp, 1.f - sp, 1.f);
                 } else {
-                    h = uwin(k + 3);
+                    hv[k4] = uwin(k + 3);
+                    spd[k4] = 1.f;
                 }
-                if (!valid) h = 0.f;
-                const float f = fa[k4], qq = qa[k4];
+                dout[k4] = bf2f(rdp[k * kP]);
+            }
+            if (has_b) {
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) iw[k4] = sigmoida_(bf2f(rbp[(4 * g4 + k4) * kP]));
+            }
+            if (has_z) {
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float zv = bf2f(rzp[(4 * g4 + k4) * kP]);
+                    const float sz = sigmoida_(zv);
+                    gg[k4] = zv * sz;
+                    gd[k4] = sz * fmaf(zv, 1.f - sz, 1.f);
+                }
+            } else {
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    gg[k4] = 1.f;
+                    gd[k4] = 0.f;
+                }
+            }
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int k = 4 * g4 + k4;
+                const float f = fa[k4], qq = qa[k4], h = hv[k4];
                 // 1 - f = (1/f - 1) f, exact for f near 1; 1 where exp(-a) overflowed
                 const float omf = qq < 3.0e38f ? (qq - 1.f) * f : 1.f;
-                const float iw = has_b ? sigmoida_(bf2f(rbp[k * kP])) : omf;
-                float gg = 1.f, gd = 0.f;
-                if (has_z) {
-                    const float zv = bf2f(rzp[k * kP]);
-                    const float sz = sigmoida_(zv);
-                    gg = zv * sz;
-                    gd = sz * fmaf(zv, 1.f - sz, 1.f);
-                }
-                const float dout = bf2f(rdp[k * kP]);  // zero outside the tensor
-                const float dyv = dout * gg;
-                const float dzc = dout * gd;
+                const float i = has_b ? iw[k4] : omf;
+                const float dyv = dout[k4] * gg[k4];
+                const float dzc = dout[k4] * gd[k4];
                 if (!slow) {
                     E *= f;
                     Q *= qq;
                 }
-                const float v = iw * h;
-                Wv[k4] = v * Q;
-                Uv[k4] = sc * dyv * E;
-                s0[k4] = sc * dzc * E;                                // dz = s0 R + s1
+                Wv[k4] = i * h * Q;
+                Uv[k4] = dyv * E;
+                s0[k4] = dzc * E;                                    // dz = s0 R + s1
                 s1[k4] = dzc * Dc * h;
-                s2[k4] = has_b ? h * (1.f - iw) * iw * Q : f * h * Q;  // db = s2 GB
+                s2[k4] = has_b ? h * (1.f - i) * i * Q : f * h * Q;  // db = s2 GB
                 s3[k4] = omf;
-                c1v[k] = valid ? iw * Q * spd : 0.f;                  // dp = c0 + c1 GB
-                c0v[k] = valid ? Dc * dyv * spd : 0.f;
+                c1v[k] = i * Q * spd[k4];                            // dp = c0 + c1 GB
+                c0v[k] = Dc * dyv * spd[k4];
                 dD_acc = fmaf(dyv, h, dD_acc);
             }
             const uint32_t o = (g4 < 2 ? oc0 : oc1) + (g4 & 1) * 8;
@@ -892,7 +918,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             const bool slow = decays(nv);  // (its barriers end the reads of the fp32 checkpoint)
             st8o(sm.Xh, sm.Xl, oc0, xr);
             st8o(sm.Xh, sm.Xl, oc1, xr + 8);
-            unpack(nv, slow);
+            unpack(slow);
             tc::tmem_st_wait();
             wait_mb(&sm.mb_bc, ph_bc);  // and region A's per-token inputs are read
             if (!slow) scale_carry(true);

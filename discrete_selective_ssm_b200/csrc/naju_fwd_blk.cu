@@ -40,6 +40,8 @@
 #include <stddef.h>
 #include <string.h>
 
+#include <type_traits>
+
 #include "naju_common.cuh"
 #include "naju_kernels.h"
 #include "naju_tc.cuh"
@@ -71,6 +73,7 @@ struct FkCols {
 struct alignas(64) FkTmaps {
     CUtensorMap u, a, b, z;  // bf16 [Bt][L][d], plain boxes of 128 channels
     CUtensorMap B, C;        // bf16 [Bt][L][N], swizzled boxes of 64 columns
+    CUtensorMap y;           // bf16 output [Bt][L][d] (bf16 outputs only), store boxes
 };
 
 template <int N>
@@ -124,6 +127,9 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     using Cols = FkCols<N>;
     using Sm = FkSmem<N>;
     constexpr int NQ = N / 4;  // state columns per thread
+    // bf16 outputs are staged in the G tiles' bytes (free once R is complete)
+    // and leave by one TMA store per block; fp32 outputs are stored directly
+    constexpr bool kStageY = std::is_same<Tout, __nv_bfloat16>::value;
     static_assert(sizeof(Sm::Xh) + sizeof(Sm::Xl) >= kK * kP * sizeof(float),
                   "the exact path's row sums live over the X tiles");
     extern __shared__ __align__(1024) float4 smem4[];
@@ -155,6 +161,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         if (has_z) tma::prefetch_map(&tm.z);
         tma::prefetch_map(&tm.B);
         tma::prefetch_map(&tm.C);
+        if (kStageY) tma::prefetch_map(&tm.y);
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -268,16 +275,28 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     // ------------------------------------------------- decays (loop 1)
     float fv[16], qv[16];
     float Eb = 1.f, Qb = 1.f, E63 = 1.f;
+    // Tokens past the end (last block only) decay by 1; channels past d
+    // read zeros (their values are finite and never stored).
     auto decays = [&](int nv) -> bool {
         const __nv_bfloat16* rap = sm.ra + 16 * q * kP + ch;
         float Qh = 1.f, Eh = 1.f;
+        if (nv == kK) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const bool valid = cvalid && 16 * q + k < nv;
-            qv[k] = valid ? 1.f + __expf(-bf2f(rap[k * kP])) : 1.f;
-            fv[k] = valid ? rcpa_(qv[k]) : 1.f;
-            Qh *= qv[k];
-            Eh *= fv[k];
+            for (int k = 0; k < 16; ++k) {
+                qv[k] = 1.f + __expf(-bf2f(rap[k * kP]));
+                fv[k] = rcpa_(qv[k]);
+                Qh *= qv[k];
+                Eh *= fv[k];
+            }
+        } else {
+            const int nq = nv - 16 * q;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                qv[k] = k < nq ? 1.f + __expf(-bf2f(rap[k * kP])) : 1.f;
+                fv[k] = k < nq ? rcpa_(qv[k]) : 1.f;
+                Qh *= qv[k];
+                Eh *= fv[k];
+            }
         }
         sm.xq[q][ch] = Qh;
         sm.xe[q][ch] = Eh;
@@ -300,12 +319,13 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     };
     // ------------------------------------------------- unpack (loop 2)
     // W to its tile pair; full: s E SiLU(z) and D h SiLU(z) to tensor memory.
-    // slow (exact path): E = Q = 1, so W = i h.
-    auto unpack = [&](int nv, bool slow, bool full) {
+    // slow (exact path): E = Q = 1, so W = i h.  W of a token past the end
+    // meets only zero rows of B (and of G), so no token mask is needed here.
+    auto unpack = [&](bool slow, bool full) {
         const __nv_bfloat16* rup = sm.ru + 16 * q * kP + ch;  // row i: token 16 q - 3 + i
         const __nv_bfloat16* rbp = sm.rb + 16 * q * kP + ch;
         const __nv_bfloat16* rzp = sm.rz + 16 * q * kP + ch;
-        float E = slow ? 1.f : Eb, Q = slow ? 1.f : Qb;
+        float E = slow ? sc : sc * Eb, Q = slow ? 1.f : Qb;  // E carries the scale s
         float u0 = 0.f, u1 = 0.f, u2 = 0.f;
         if (CONV) {
             u0 = bf2f(rup[0]);
@@ -316,38 +336,53 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         for (int g8 = 0; g8 < 2; ++g8) {
             float Wv[8], s0[8], s1[8];
 #pragma unroll
-            for (int k8 = 0; k8 < 8; ++k8) {
-                const int k = 8 * g8 + k8;
-                const bool valid = cvalid && 16 * q + k < nv;
-                const float u3 = bf2f(rup[(k + 3) * kP]);
-                float h;
-                if (CONV) {
-                    const float pp = fmaf(w3, u3, fmaf(w2, u2, fmaf(w1, u1, fmaf(w0, u0, wb))));
-                    h = pp * sigmoida_(pp);
-                    u0 = u1;
-                    u1 = u2;
-                    u2 = u3;
-                } else {
-                    h = u3;
-                }
-                if (!valid) h = 0.f;
-                const float f = fv[k], qq = qv[k];
-                // coupled: i = 1 - f = (1/f - 1) f (1 where exp(-a) overflowed)
-                const float iw = has_b ? sigmoida_(bf2f(rbp[k * kP]))
-                                       : (qq < 3.0e38f ? (qq - 1.f) * f : 1.f);
-                if (!slow) {
-                    E *= f;
-                    Q *= qq;
-                }
-                Wv[k8] = iw * h * Q;
-                if (full) {
-                    float gg = 1.f;
-                    if (has_z) {
-                        const float zv = bf2f(rzp[k * kP]);
-                        gg = zv * sigmoida_(zv);
+            for (int h4 = 0; h4 < 2; ++h4) {
+                const int kb = 8 * g8 + 4 * h4;  // first of four tokens
+                float hv[4], iw[4], gg[4];
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float u3 = bf2f(rup[(kb + k4 + 3) * kP]);
+                    if (CONV) {
+                        const float pp = fmaf(w3, u3, fmaf(w2, u2, fmaf(w1, u1, fmaf(w0, u0, wb))));
+                        hv[k4] = pp * sigmoida_(pp);
+                        u0 = u1;
+                        u1 = u2;
+                        u2 = u3;
+                    } else {
+                        hv[k4] = u3;
                     }
-                    s0[k8] = sc * E * gg;
-                    s1[k8] = Dc * h * gg;
+                }
+                if (has_b) {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) iw[k4] = sigmoida_(bf2f(rbp[(kb + k4) * kP]));
+                } else {
+                    // coupled: i = 1 - f = (1/f - 1) f (1 where exp(-a) overflowed)
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float qq = qv[kb + k4];
+                        iw[k4] = qq < 3.0e38f ? (qq - 1.f) * fv[kb + k4] : 1.f;
+                    }
+                }
+                if (full && has_z) {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float zv = bf2f(rzp[(kb + k4) * kP]);
+                        gg[k4] = zv * sigmoida_(zv);
+                    }
+                } else {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) gg[k4] = 1.f;
+                }
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int k = kb + k4;
+                    if (!slow) {
+                        E *= fv[k];
+                        Q *= qv[k];
+                    }
+                    Wv[4 * h4 + k4] = iw[k4] * hv[k4] * Q;
+                    s0[4 * h4 + k4] = E * gg[k4];
+                    s1[4 * h4 + k4] = Dc * hv[k4] * gg[k4];
                 }
             }
             const int col = 16 * q + 8 * g8;
@@ -444,12 +479,13 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         const int nv = (int)min64((int64_t)kK, L - tb);
         wait_mb(&sm.mb_raw, ph_raw);
         const bool slow = decays(nv);
-        unpack(nv, slow, full);
+        unpack(slow, full);
         tc::tmem_st_wait();
         tc::fence_proxy_async();
         sync();
         // the raw buffer is read (the exact path still needs a)
         if (tid == 0 && next >= 0 && !slow) load_raw(next, full);
+        if (kStageY && tid == 0) tma::store_wait_read();  // the previous y has left G
         wait_mb(&sm.mb_bc, ph_bc);
         if (!slow) {
             constexpr uint32_t idR = tc::idesc_bf16(128, 64);
@@ -505,16 +541,23 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         // the B and C tiles are free
         if (tid == 0 && next >= 0) load_bc(next, full);
         if (full) {
-            Tout* gy = static_cast<Tout*>(p.y) + ((int64_t)bb * L + tb + 16 * q) * d + c;
             float r[16], e[16], dh[16];
             tc::tmem_ld16(trow + Cols::R + 16 * q, r);
             tc::tmem_ld16(trow + Cols::SV + 16 * q, e);
             tc::tmem_ld16(trow + Cols::SV + 64 + 16 * q, dh);
             tc::tmem_ld_wait();
-            const int nk = cvalid ? min(16, nv - 16 * q) : 0;
+            if constexpr (kStageY) {
+                __nv_bfloat16* ys = sm.Gh + 16 * q * kP + ch;  // [64 t][128 ch]
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk)
-                if (kk < nk) gy[(int64_t)kk * d] = from_f<Tout>(fmaf(e[kk], r[kk], dh[kk]));
+                for (int kk = 0; kk < 16; ++kk)
+                    ys[kk * kP] = __float2bfloat16_rn(fmaf(e[kk], r[kk], dh[kk]));
+            } else {
+                Tout* gy = static_cast<Tout*>(p.y) + ((int64_t)bb * L + tb + 16 * q) * d + c;
+                const int nk = cvalid ? min(16, nv - 16 * q) : 0;
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk)
+                    if (kk < nk) gy[(int64_t)kk * d] = from_f<Tout>(fmaf(e[kk], r[kk], dh[kk]));
+            }
         }
         if (!slow) update_state();
         logP += __logf(E63);  // decay over the block (for the look-back)
@@ -536,8 +579,12 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             const bool last = k + 1 == s1;
             run_block(k, full, last ? -1 : k + 1);
             state_out(full && (!last || end_ckpt) ? ck_at(k + 1) : nullptr, full && !last);
-            tc::fence_proxy_async();
+            tc::fence_proxy_async();  // (X tiles and the staged y -> async proxy)
             sync();
+            if (kStageY && full && tid == 0) {
+                tma::store_3d(&tm.y, (int)c0, k * kK, bb, sm.Gh);
+                tma::store_commit();
+            }
         }
     };
     if (sbase & 1023u) {  // the swizzled tiles need 1024-byte alignment
@@ -628,6 +675,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         if (last_group && p.x_final) state_out(p.x_final + (int64_t)bb * d * N, false);
     }
 #undef NAJU_SA
+    if (kStageY && tid == 0) tma::store_wait_all();
     if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
     sync();
     if (warp == 0) tc::tmem_dealloc(tbase, Cols::ALLOC);
@@ -643,6 +691,8 @@ static cudaError_t launch_fwd_blk_t(const FwdParams& p, cudaStream_t st) {
               (!p.z || tma_encode_bf16_3d(&tm.z, p.z, p.Bt, p.L, p.d, kK, kP)) &&
               tma_encode_bf16_3d_sw128(&tm.B, p.B, p.Bt, p.L, N, kK) &&
               tma_encode_bf16_3d_sw128(&tm.C, p.C, p.Bt, p.L, N, kK);
+    if (ok && std::is_same<Tout, __nv_bfloat16>::value)
+        ok = tma_encode_bf16_3d(&tm.y, p.y, p.Bt, p.L, p.d, kK, kP);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(FkSmem<N>);
     auto kern = scan_fwd_blk_kernel<Tout, N, CONV, PIECES>;

@@ -610,8 +610,8 @@ def main():
                        "fwd_frac_hbm": fwd_b / (fwd_ms / 1e3) / 1e9 / peak,
                        "bwd_frac_hbm": bwd_b / (bwd_ms / 1e3) / 1e9 / peak},
             "roofline": {"bound": "hbm",
-                         "kernel": ("naju_scan_bwd: scan_bwd_tc_kernel + reductions" if dom_is_bwd
-                                    else "naju_scan_fwd: scan_fwd_tc_kernel"),
+                         "kernel": ("naju_scan_bwd: scan_bwd_blk_kernel + finish_dBC + reductions"
+                                    if dom_is_bwd else "naju_scan_fwd: scan_fwd_blk_kernel"),
                          "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "alg_bytes": dom_b, "peak_kind": pk_kind},

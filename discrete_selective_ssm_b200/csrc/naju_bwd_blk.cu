@@ -422,7 +422,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         if (nv == kK) {
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                qv[k] = 1.f + __expf(-bf2f(rap[k * kP]));
+                qv[k] = 1.f + expa_(-bf2f(rap[k * kP]));
                 fv[k] = rcpa_(qv[k]);
                 Qh *= qv[k];
                 Eh *= fv[k];
@@ -431,7 +431,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             const int nq = nv - 16 * q;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                qv[k] = k < nq ? 1.f + __expf(-bf2f(rap[k * kP])) : 1.f;
+                qv[k] = k < nq ? 1.f + expa_(-bf2f(rap[k * kP])) : 1.f;
                 fv[k] = k < nq ? rcpa_(qv[k]) : 1.f;
                 Qh *= qv[k];
                 Eh *= fv[k];
@@ -494,7 +494,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 if (CONV) {
                     const float pp = fmaf(w3, uwin(k + 3), fmaf(w2, uwin(k + 2),
                                          fmaf(w1, uwin(k + 1), fmaf(w0, uwin(k), wb))));
-                    const float sp = sigmoida_(pp);
+                    const float sp = sigmoidx_(pp);
                     hv[k4] = pp * sp;
                     spd[k4] = sp * fmaf(pp, 1.f - sp, 1.f);
                 } else {
@@ -505,13 +505,13 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             }
             if (has_b) {
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) iw[k4] = sigmoida_(bf2f(rbp[(4 * g4 + k4) * kP]));
+                for (int k4 = 0; k4 < 4; ++k4) iw[k4] = sigmoidx_(bf2f(rbp[(4 * g4 + k4) * kP]));
             }
             if (has_z) {
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
                     const float zv = bf2f(rzp[(4 * g4 + k4) * kP]);
-                    const float sz = sigmoida_(zv);
+                    const float sz = sigmoidx_(zv);
                     gg[k4] = zv * sz;
                     gd[k4] = sz * fmaf(zv, 1.f - sz, 1.f);
                 }
@@ -783,7 +783,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                         float gg = 1.f;
                         if (has_z) {
                             const float zv = bf2f(rzp[kk * kP]);
-                            gg = zv * sigmoida_(zv);
+                            gg = zv * sigmoidx_(zv);
                         }
                         const float dout = bf2f(rdp[kk * kP]);  // zero outside the tensor
                         if (!slow) E *= fa[k4];

@@ -63,6 +63,17 @@ __device__ __forceinline__ float rcpa_(float v) {
     return r;
 }
 __device__ __forceinline__ float sigmoida_(float v) { return rcpa_(1.0f + __expf(-v)); }
+// e^v as 2^(v log2 e) on the MUFU unit (PTX ex2.approx.ftz.f32: a few ulp,
+// results below the normal range flushed to zero), and the sigmoid on it.
+// The block-form tensor-core kernels use these; the parity tests against the
+// fp64 oracle bound their effect.
+__device__ __forceinline__ float exp2a_(float v) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+__device__ __forceinline__ float expa_(float v) { return exp2a_(v * 1.4426950408889634f); }
+__device__ __forceinline__ float sigmoidx_(float v) { return rcpa_(1.0f + expa_(-v)); }
 __device__ __forceinline__ float silua_(float v) { return v * sigmoida_(v); }
 __device__ __forceinline__ float sigmoidf_(float v) { return rcpf_(1.0f + __expf(-v)); }
 __device__ __forceinline__ float siluf_(float v) { return v * sigmoidf_(v); }

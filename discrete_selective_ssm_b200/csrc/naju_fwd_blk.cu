@@ -283,7 +283,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         if (nv == kK) {
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                qv[k] = 1.f + __expf(-bf2f(rap[k * kP]));
+                qv[k] = 1.f + expa_(-bf2f(rap[k * kP]));
                 fv[k] = rcpa_(qv[k]);
                 Qh *= qv[k];
                 Eh *= fv[k];
@@ -292,7 +292,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             const int nq = nv - 16 * q;
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                qv[k] = k < nq ? 1.f + __expf(-bf2f(rap[k * kP])) : 1.f;
+                qv[k] = k < nq ? 1.f + expa_(-bf2f(rap[k * kP])) : 1.f;
                 fv[k] = k < nq ? rcpa_(qv[k]) : 1.f;
                 Qh *= qv[k];
                 Eh *= fv[k];
@@ -344,7 +344,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                     const float u3 = bf2f(rup[(kb + k4 + 3) * kP]);
                     if (CONV) {
                         const float pp = fmaf(w3, u3, fmaf(w2, u2, fmaf(w1, u1, fmaf(w0, u0, wb))));
-                        hv[k4] = pp * sigmoida_(pp);
+                        hv[k4] = pp * sigmoidx_(pp);
                         u0 = u1;
                         u1 = u2;
                         u2 = u3;
@@ -354,7 +354,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                 }
                 if (has_b) {
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) iw[k4] = sigmoida_(bf2f(rbp[(kb + k4) * kP]));
+                    for (int k4 = 0; k4 < 4; ++k4) iw[k4] = sigmoidx_(bf2f(rbp[(kb + k4) * kP]));
                 } else {
                     // coupled: i = 1 - f = (1/f - 1) f (1 where exp(-a) overflowed)
 #pragma unroll
@@ -367,7 +367,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         const float zv = bf2f(rzp[(kb + k4) * kP]);
-                        gg[k4] = zv * sigmoida_(zv);
+                        gg[k4] = zv * sigmoidx_(zv);
                     }
                 } else {
 #pragma unroll
@@ -477,38 +477,35 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     auto run_block = [&](int k, bool full, int next) {
         const int64_t tb = (int64_t)k * kK;
         const int nv = (int)min64((int64_t)kK, L - tb);
+        constexpr uint32_t idR = tc::idesc_bf16(128, 64);
+        // G = C B^T (M = 64; B and C exact) goes to the tensor core as soon as
+        // this block's B and C have landed (thread 0 waits for them) and
+        // overlaps the CUDA-core work below.
+        if (tid == 0) {
+            if (!timed_out && !tc::mbar_wait(&sm.mb_bc, ph_bc, kSpin)) timed_out = true;
+            if (full) {
+                bool fg = true;
+                prod(tbase + Cols::G, NAJU_SA(Cs), kK, NAJU_SA(Bs), kK, false, N / 16,
+                     tc::idesc_bf16(64, 64), fg);
+                tc::mma_commit(&sm.mb0);
+            }
+        }
+        ph_bc ^= 1u;
         wait_mb(&sm.mb_raw, ph_raw);
         const bool slow = decays(nv);
         unpack(slow, full);
         tc::tmem_st_wait();
         tc::fence_proxy_async();
-        sync();
+        if (kStageY && tid == 0) tma::store_wait_read();  // the previous y has left G
+        if (full) {
+            wait_mb(&sm.mb0, ph0);
+        } else {
+            sync();
+        }
         // the raw buffer is read (the exact path still needs a)
         if (tid == 0 && next >= 0 && !slow) load_raw(next, full);
-        if (kStageY && tid == 0) tma::store_wait_read();  // the previous y has left G
-        wait_mb(&sm.mb_bc, ph_bc);
         if (!slow) {
-            constexpr uint32_t idR = tc::idesc_bf16(128, 64);
-            if (tid == 0) {
-                if (full) {
-                    // G = C B^T (M = 64; B and C exact)
-                    bool fg = true;
-                    prod(tbase + Cols::G, NAJU_SA(Cs), kK, NAJU_SA(Bs), kK, false, N / 16,
-                         tc::idesc_bf16(64, 64), fg);
-                    tc::mma_commit(&sm.mb0);
-                }
-                issue_S();
-                if (full) {
-                    // R = X C^T
-                    bool fr = true;
-                    prod(tbase + Cols::R, NAJU_SA(Xh), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
-                    prod(tbase + Cols::R, NAJU_SA(Xl), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
-                } else {
-                    tc::mma_commit(&sm.mb2);
-                }
-            }
             if (full) {
-                wait_mb(&sm.mb0, ph0);
                 {   // masked G to its tile pair: lanes 0-15 of each sub-partition hold rows
                     float v[16];
                     tc::tmem_ld16(trow + Cols::G + 16 * q, v);
@@ -524,14 +521,19 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                 }
                 tc::fence_proxy_async();
                 sync();
-                if (tid == 0) {
-                    // R += W G^T (three terms)
-                    bool fr = false;
+            }
+            if (tid == 0) {
+                issue_S();
+                if (full) {
+                    // R = X C^T + W G^T (three terms)
+                    bool fr = true;
+                    prod(tbase + Cols::R, NAJU_SA(Xh), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
+                    prod(tbase + Cols::R, NAJU_SA(Xl), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
                     prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
                     prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gl), kK, false, kK / 16, idR, fr);
                     prod(tbase + Cols::R, NAJU_SA(Wl), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
-                    tc::mma_commit(&sm.mb2);
                 }
+                tc::mma_commit(&sm.mb2);
             }
             wait_mb(&sm.mb2, ph2);
         } else {

@@ -481,6 +481,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                      (i < 9 ? (uint32_t)rup[(2 * i + 1) * kP] << 16 : 0u);
         float E = slow ? sc : sc * Eb, Q = slow ? 1.f : Qb;  // E carries the scale s
         dD_acc = 0.f;
+        uint32_t pk[8];  // packed W, U hi / lo of the previous group of four
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
             float Wv[4], Uv[4], s0[4], s1[4], s2[4], s3[4], fa[4], qa[4];
@@ -536,27 +537,36 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     E *= f;
                     Q *= qq;
                 }
-                Wv[k4] = i * h * Q;
+                const float iQ = i * Q;
+                Wv[k4] = iQ * h;
                 Uv[k4] = dyv * E;
-                s0[k4] = dzc * E;                                    // dz = s0 R + s1
+                s0[k4] = dzc * E;                                        // dz = s0 R + s1
                 s1[k4] = dzc * Dc * h;
-                s2[k4] = has_b ? h * (1.f - i) * i * Q : f * h * Q;  // db = s2 GB
+                s2[k4] = has_b ? Wv[k4] * (1.f - i) : f * h * Q;         // db = s2 GB
                 s3[k4] = omf;
-                c1v[k] = i * Q * spd[k4];                            // dp = c0 + c1 GB
+                c1v[k] = iQ * spd[k4];                                   // dp = c0 + c1 GB
                 c0v[k] = Dc * dyv * spd[k4];
                 dD_acc = fmaf(dyv, h, dD_acc);
             }
-            const uint32_t o = (g4 < 2 ? oc0 : oc1) + (g4 & 1) * 8;
-            {
-                uint32_t h0, l0, h1, l1;
-                split2(Wv[0], Wv[1], h0, l0);
-                split2(Wv[2], Wv[3], h1, l1);
-                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Wh) + o) = make_uint2(h0, h1);
-                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Wl) + o) = make_uint2(l0, l1);
-                split2(Uv[0], Uv[1], h0, l0);
-                split2(Uv[2], Uv[3], h1, l1);
-                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Uh) + o) = make_uint2(h0, h1);
-                *reinterpret_cast<uint2*>(reinterpret_cast<char*>(sm.Ul) + o) = make_uint2(l0, l1);
+            {   // W and U hi / lo: one 16-byte chunk per tile every second group
+                uint32_t wh0, wl0, wh1, wl1, uh0, ul0, uh1, ul1;
+                split2(Wv[0], Wv[1], wh0, wl0);
+                split2(Wv[2], Wv[3], wh1, wl1);
+                split2(Uv[0], Uv[1], uh0, ul0);
+                split2(Uv[2], Uv[3], uh1, ul1);
+                if ((g4 & 1) == 0) {
+                    pk[0] = wh0; pk[1] = wh1; pk[2] = wl0; pk[3] = wl1;
+                    pk[4] = uh0; pk[5] = uh1; pk[6] = ul0; pk[7] = ul1;
+                } else {
+                    const uint32_t o = g4 < 2 ? oc0 : oc1;
+                    auto st = [&](__nv_bfloat16* t, uint4 v) {
+                        *reinterpret_cast<uint4*>(reinterpret_cast<char*>(t) + o) = v;
+                    };
+                    st(sm.Wh, make_uint4(pk[0], pk[1], wh0, wh1));
+                    st(sm.Wl, make_uint4(pk[2], pk[3], wl0, wl1));
+                    st(sm.Uh, make_uint4(pk[4], pk[5], uh0, uh1));
+                    st(sm.Ul, make_uint4(pk[6], pk[7], ul0, ul1));
+                }
             }
             if constexpr (!kExport) {
                 tc::tmem_st4(trow + Cols::SV + 0 * 64 + col, s0);
@@ -866,6 +876,20 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             carry_from(sm.ok ? carry_slot(slot) : nullptr, true);
         }
         int par = 0;  // parity of the block within the segment (double buffers)
+        // The staged gradients of a block leave after the next block's first
+        // barrier (no barrier of their own): that block's first token, or -1.
+        int out_pending = -1;
+        auto store_out = [&]() {
+            if (kStage && tid == 0 && out_pending >= 0) {
+                const int x = (int)c0, y = out_pending;
+                if (has_z) tma::store_3d(&tm.oz, x, y, bb, sm.Wh);
+                if (has_b) tma::store_3d(&tm.ob, x, y, bb, sm.Wl);
+                tma::store_3d(&tm.oa, x, y, bb, sm.Uh);
+                tma::store_3d(&tm.ou, x, y, bb, sm.Ul);
+                tma::store_commit();
+            }
+            out_pending = -1;
+        };
         {
             float hx[16];
             tc::tmem_ld16(trow + Cols::H + 16 * q, hx);
@@ -903,8 +927,6 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             const int nv = (int)min64((int64_t)kK, L - tb);
             const int nq = cvalid ? nv - 16 * q : 0;  // valid tokens of this thread
             // ------------------------------------------------ phase A
-            // (the previous block's staged outputs must have left the W / U bytes)
-            if (kStage && tid == 0) tma::store_wait_read();
             if (kImport && tid == 0) {
 #pragma unroll
                 for (int i = 0; i < kP; i += 32) {
@@ -913,8 +935,11 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 }
             }
             wait_mb2(&sm.mb_in, ph_in, &sm.mb_x, ph_x);
+            store_out();  // the previous block's staged gradients (after that barrier)
             float xr[16];
             read_x(xr);
+            // the staged gradients must have left the W / U bytes before unpack
+            if (kStage && tid == 0) tma::store_wait_read();
             const bool slow = decays(nv);  // (its barriers end the reads of the fp32 checkpoint)
             st8o(sm.Xh, sm.Xl, oc0, xr);
             st8o(sm.Xh, sm.Xl, oc1, xr + 8);
@@ -1004,6 +1029,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             // first three dp for the neighbouring quarter.
             float dL[16];
             float qsum = 0.f, dpf0 = 0.f, dpf1 = 0.f, dpf2 = 0.f;
+            uint4 uh4, ul4, wh4, wl4;  // 8 tokens of U and W hi / lo
 #pragma unroll
             for (int g4 = 0; g4 < 4; ++g4) {
                 const int col = 16 * q + 4 * g4;
@@ -1011,9 +1037,27 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 tc::tmem_ld4(trow + Cols::R + col, R4);
                 tc::tmem_ld4(trow + Cols::GB + col, G4);
                 if (!has_b) tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
-                const uint32_t o = (g4 < 2 ? oc0 : oc1) + (g4 & 1) * 8;
-                ld4o(sm.Uh, sm.Ul, o, Ua);
-                ld4o(sm.Wh, sm.Wl, o, Wa);
+                if ((g4 & 1) == 0) {
+                    const uint32_t o = g4 < 2 ? oc0 : oc1;
+                    auto ld = [&](const __nv_bfloat16* t) {
+                        return *reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(t) + o);
+                    };
+                    uh4 = ld(sm.Uh);
+                    ul4 = ld(sm.Ul);
+                    wh4 = ld(sm.Wh);
+                    wl4 = ld(sm.Wl);
+                }
+                {
+                    const bool hi = (g4 & 1) != 0;
+                    const uint32_t a0 = hi ? uh4.z : uh4.x, a1 = hi ? uh4.w : uh4.y;
+                    const uint32_t b0 = hi ? ul4.z : ul4.x, b1 = hi ? ul4.w : ul4.y;
+                    const uint32_t c0_ = hi ? wh4.z : wh4.x, c1_ = hi ? wh4.w : wh4.y;
+                    const uint32_t d0 = hi ? wl4.z : wl4.x, d1 = hi ? wl4.w : wl4.y;
+                    Ua[0] = bf_lo(a0) + bf_lo(b0); Ua[1] = bf_hi(a0) + bf_hi(b0);
+                    Ua[2] = bf_lo(a1) + bf_lo(b1); Ua[3] = bf_hi(a1) + bf_hi(b1);
+                    Wa[0] = bf_lo(c0_) + bf_lo(d0); Wa[1] = bf_hi(c0_) + bf_hi(d0);
+                    Wa[2] = bf_lo(c1_) + bf_lo(d1); Wa[3] = bf_hi(c1_) + bf_hi(d1);
+                }
                 tc::tmem_ld_wait();
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
@@ -1153,17 +1197,14 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 for (int k2 = 0; k2 < 16; ++k2)
                     if (k2 < nvq) red_add(acc + k2 * 2 * NS, v[k2]);
             }
-            if (kStage) tc::fence_proxy_async();  // staged outputs -> TMA
-            sync();  // tiles and tensor memory free for the next block
-            if (kStage && tid == 0) {
-                const int x = (int)c0, y = (int)tb;
-                if (has_z) tma::store_3d(&tm.oz, x, y, bb, sm.Wh);
-                if (has_b) tma::store_3d(&tm.ob, x, y, bb, sm.Wl);
-                tma::store_3d(&tm.oa, x, y, bb, sm.Uh);
-                tma::store_3d(&tm.ou, x, y, bb, sm.Ul);
-                tma::store_commit();
-            }
+            // staged outputs -> async proxy; the next block's first barrier
+            // orders them (and this block's reads of tiles and tensor memory)
+            // before its stores and writes
+            if (kStage) tc::fence_proxy_async();
+            out_pending = (int)tb;
         }
+        sync();
+        store_out();
 
         // ------------------------------------------- carries and partials
         if (firstg) {

@@ -57,6 +57,7 @@ constexpr int kNT = 512;
 constexpr float kBound = 1.2379400392853803e27f;  // 2^90
 constexpr float kQuarter = 4194304.f;             // 2^22
 constexpr long long kSpin = 1LL << 24;
+constexpr float kLog2e = 1.4426950408889634f;
 
 template <int N>
 struct FkCols {
@@ -338,40 +339,61 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
 #pragma unroll
             for (int h4 = 0; h4 < 2; ++h4) {
                 const int kb = 8 * g8 + 4 * h4;  // first of four tokens
-                float hv[4], iw[4], gg[4];
+                // SiLU(conv), sigma(b) and SiLU(z) share one reciprocal:
+                // q = 1 + e^{-v} with e^{-v} capped at 2^36 (the product stays
+                // finite; a sigmoid below 1.5e-11 moves by at most that much),
+                // r = 1 / (qp qb qz), sigma_p = r qb qz and so on.
+                float pv[4], qp[4], qb[4], qz[4], zv[4];
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
                     const float u3 = bf2f(rup[(kb + k4 + 3) * kP]);
                     if (CONV) {
-                        const float pp = fmaf(w3, u3, fmaf(w2, u2, fmaf(w1, u1, fmaf(w0, u0, wb))));
-                        hv[k4] = pp * sigmoidx_(pp);
+                        pv[k4] = fmaf(w3, u3, fmaf(w2, u2, fmaf(w1, u1, fmaf(w0, u0, wb))));
+                        qp[k4] = 1.f + exp2a_(fminf(-kLog2e * pv[k4], 36.f));
                         u0 = u1;
                         u1 = u2;
                         u2 = u3;
                     } else {
-                        hv[k4] = u3;
+                        pv[k4] = u3;
+                        qp[k4] = 1.f;
                     }
                 }
                 if (has_b) {
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) iw[k4] = sigmoidx_(bf2f(rbp[(kb + k4) * kP]));
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        qb[k4] = 1.f + exp2a_(fminf(-kLog2e * bf2f(rbp[(kb + k4) * kP]), 36.f));
                 } else {
-                    // coupled: i = 1 - f = (1/f - 1) f (1 where exp(-a) overflowed)
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const float qq = qv[kb + k4];
-                        iw[k4] = qq < 3.0e38f ? (qq - 1.f) * fv[kb + k4] : 1.f;
-                    }
+                    for (int k4 = 0; k4 < 4; ++k4) qb[k4] = 1.f;
                 }
                 if (full && has_z) {
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
-                        const float zv = bf2f(rzp[(kb + k4) * kP]);
-                        gg[k4] = zv * sigmoidx_(zv);
+                        zv[k4] = bf2f(rzp[(kb + k4) * kP]);
+                        qz[k4] = 1.f + exp2a_(fminf(-kLog2e * zv[k4], 36.f));
                     }
                 } else {
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) gg[k4] = 1.f;
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        zv[k4] = 1.f;
+                        qz[k4] = 1.f;
+                    }
+                }
+                float hv[4], iw[4], gg[4];
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float qbz = qb[k4] * qz[k4];
+                    const float r = rcpa_(qp[k4] * qbz);
+                    hv[k4] = CONV ? pv[k4] * (r * qbz) : pv[k4];
+                    const float rp = r * qp[k4];
+                    if (has_b) {
+                        iw[k4] = rp * qz[k4];
+                    } else {
+                        // coupled: i = 1 - f = (1/f - 1) f (1 where exp(-a) overflowed)
+                        const float qq = qv[kb + k4];
+                        iw[k4] = qq < 3.0e38f ? (qq - 1.f) * fv[kb + k4] : 1.f;
+                    }
+                    gg[k4] = (full && has_z) ? zv[k4] * (rp * qb[k4]) : 1.f;
                 }
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
@@ -474,6 +496,16 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     // holds the state entering it; on exit the state in tensor memory is
     // updated and, for next >= 0, block next's loads are issued.
     float logP = 0.f;  // log of the decay product over an update-only pass
+    // The staged y of a block leaves after the next block's first barrier
+    // (no barrier of its own): the block whose y is pending, or -1.
+    int y_pending = -1;
+    auto store_y = [&]() {
+        if (kStageY && tid == 0 && y_pending >= 0) {
+            tma::store_3d(&tm.y, (int)c0, y_pending * kK, bb, sm.Gh);
+            tma::store_commit();
+        }
+        y_pending = -1;
+    };
     auto run_block = [&](int k, bool full, int next) {
         const int64_t tb = (int64_t)k * kK;
         const int nv = (int)min64((int64_t)kK, L - tb);
@@ -492,6 +524,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         }
         ph_bc ^= 1u;
         wait_mb(&sm.mb_raw, ph_raw);
+        store_y();
         const bool slow = decays(nv);
         unpack(slow, full);
         tc::tmem_st_wait();
@@ -581,13 +614,13 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             const bool last = k + 1 == s1;
             run_block(k, full, last ? -1 : k + 1);
             state_out(full && (!last || end_ckpt) ? ck_at(k + 1) : nullptr, full && !last);
-            tc::fence_proxy_async();  // (X tiles and the staged y -> async proxy)
-            sync();
-            if (kStageY && full && tid == 0) {
-                tma::store_3d(&tm.y, (int)c0, k * kK, bb, sm.Gh);
-                tma::store_commit();
-            }
+            // X tiles and the staged y -> async proxy; the next block's first
+            // barrier orders them before its MMAs and y's store
+            tc::fence_proxy_async();
+            if (full) y_pending = k;
         }
+        sync();
+        store_y();
     };
     if (sbase & 1023u) {  // the swizzled tiles need 1024-byte alignment
         if (tid == 0) atomicOr(&p.hdr->status, 1 << NAJU_ERR_INVALID_ARG);

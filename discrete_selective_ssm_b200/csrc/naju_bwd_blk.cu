@@ -78,6 +78,11 @@ constexpr int kNT = 512;  // threads
 constexpr float kBound = 1.2379400392853803e27f;  // 2^90
 constexpr float kQuarter = 4194304.f;             // 2^22: four quarters below it stay below 2^88
 constexpr long long kSpin = 1LL << 24;
+// The tensor-core chains of a block are issued by lanes 0 of warps 0..5 (one
+// accumulator per thread, so each chain keeps its order): committing
+// threads per completion barrier.
+constexpr int kIss0 = 2;  // G (warp 0), P (warp 5)
+constexpr int kIss2 = 5;  // dB (0), R (1), GB (2), carry (3), dC (4)
 
 // Tensor-memory columns (lane = channel unless stated).
 struct BkCols {
@@ -120,7 +125,7 @@ struct BkSmem {
     float dph[4][3][kP];          // first three dp of each quarter
     float dnext[2][3][kP];        // first three dp of the later block
     float red6[6][kP];            // per-channel parameter sums
-    uint64_t mb_in, mb_bc, mb_x, mb0, mb2;
+    uint64_t mb_in, mb_bc, mb_x, mb0, mb2, mb_e;
     uint32_t taddr;
     int item, ok;
 };
@@ -227,8 +232,9 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tc::mbar_init(&sm.mb_in, 1);
         tc::mbar_init(&sm.mb_bc, 1);
         tc::mbar_init(&sm.mb_x, 1);
-        tc::mbar_init(&sm.mb0, 1);
-        tc::mbar_init(&sm.mb2, 1);
+        tc::mbar_init(&sm.mb0, kIss0);  // G and P
+        tc::mbar_init(&sm.mb2, kIss2);  // every chain of the block
+        tc::mbar_init(&sm.mb_e, 1);     // the early pass's carry
         tma::prefetch_map(&tm.X);
         tma::prefetch_map(&tm.u);
         tma::prefetch_map(&tm.a);
@@ -251,8 +257,12 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     const uint32_t trow = tbase + ((uint32_t)(s4 * 32) << 16);  // this warp's lanes
     const int item = sm.item;
     const uint32_t sbase = tc::smem_u32(&sm);
-#define NAJU_SA(f) (sbase + (uint32_t)offsetof(Sm, f))
-    uint32_t ph_in = 0, ph_bc = 0, ph_x = 0, ph0 = 0, ph2 = 0;  // mbarrier parities
+// tile start addresses / 16 (the base is 1024-byte aligned: checked below)
+#define NAJU_SA(f) (sb4 + (uint32_t)(offsetof(Sm, f) >> 4))
+    const uint32_t sb4 = sbase >> 4;
+    const bool aligned1k = (sbase & 1023u) == 0;  // the swizzled tiles need it
+    if (!aligned1k && tid == 0) atomicOr(&p.hdr->status, 1 << NAJU_ERR_INVALID_ARG);
+    uint32_t ph_in = 0, ph_bc = 0, ph_x = 0, ph0 = 0, ph2 = 0, ph_e = 0;  // mbarrier parities
     bool timed_out = false;
 
     // This thread's two 16-byte chunks (columns [16 q, 16 q + 8) and
@@ -594,11 +604,16 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     // --------------------------------------------------------- the MMAs
     const uint32_t lane16 = 16u << 16;
     // one product A.B over K steps ks < nks, into d (accumulating unless first)
+    // (a, b: tile start addresses / 16; a K step of 16 elements is 32 bytes
+    // along a K-major row, 16 rows = 2048 bytes of an MN-major tile)
     auto prod = [&](uint32_t dcol, uint32_t a, bool a_mn, uint32_t b, bool b_mn, int nks,
                     uint32_t idesc, bool& first) {
+#pragma unroll
         for (int ks = 0; ks < nks; ++ks) {
-            const uint64_t ad = a_mn ? tc::sdesc_bf_mn(a, ks) : tc::sdesc_bf_k(a, ks);
-            const uint64_t bd = b_mn ? tc::sdesc_bf_mn(b, ks) : tc::sdesc_bf_k(b, ks);
+            const uint64_t ad = a_mn ? tc::sdesc_sw128_mn_a4(a + ks * 128u, 1024)
+                                     : tc::sdesc_sw128_a4(a + ks * 2u);
+            const uint64_t bd = b_mn ? tc::sdesc_sw128_mn_a4(b + ks * 128u, 1024)
+                                     : tc::sdesc_sw128_a4(b + ks * 2u);
             tc::mma_bf16_ss(dcol, ad, bd, idesc, first ? 0u : 1u);
             first = false;
         }
@@ -618,42 +633,68 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     };
     // Batch 0: G = C B^T (lanes +0), P = U^T W (lanes +16), M = 64.
     // Batch 1: R = X C^T, GB = H' B^T, carry += U C.
+    // Each accumulator's chain is issued by one thread (lane 0 of warp
+    // `issuer`), so the chains run side by side and keep their own order.
+    const int issuer = lid == 0 ? warp : -1;
     auto issue_b01 = [&]() {
-        bool f0 = true, f1 = true, f2 = true, f3 = true, fh = false;
-        prod(tbase + Cols::BC, NAJU_SA(Cs), false, NAJU_SA(Bs), false, kN / 16,
-             tc::idesc_bf16(64, 64), f0);
-        prod3(tbase + lane16 + Cols::BC, NAJU_SA(Uh), NAJU_SA(Ul), true, NAJU_SA(Wh), NAJU_SA(Wl),
-              true, kP / 16, tc::idesc_bf16(64, 64, true, true), f1);
-        tc::mma_commit(&sm.mb0);
-        prod2(tbase + Cols::R, NAJU_SA(Xh), NAJU_SA(Xl), false, NAJU_SA(Cs), false, kN / 16,
-              tc::idesc_bf16(128, 64), f2);
-        prod2(tbase + Cols::GB, NAJU_SA(Hh), NAJU_SA(Hl), false, NAJU_SA(Bs), false, kN / 16,
-              tc::idesc_bf16(128, 64), f3);
-        prod2(tbase + Cols::H, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Cs), true, kK / 16,
-              tc::idesc_bf16(128, kN, false, true), fh);
+        if (issuer == 0) {
+            bool f = true;
+            prod(tbase + Cols::BC, NAJU_SA(Cs), false, NAJU_SA(Bs), false, kN / 16,
+                 tc::idesc_bf16(64, 64), f);
+            tc::mma_commit(&sm.mb0);
+        } else if (issuer == 5) {
+            bool f = true;
+            prod3(tbase + lane16 + Cols::BC, NAJU_SA(Uh), NAJU_SA(Ul), true, NAJU_SA(Wh),
+                  NAJU_SA(Wl), true, kP / 16, tc::idesc_bf16(64, 64, true, true), f);
+            tc::mma_commit(&sm.mb0);
+        } else if (issuer == 1) {
+            bool f = true;
+            prod2(tbase + Cols::R, NAJU_SA(Xh), NAJU_SA(Xl), false, NAJU_SA(Cs), false, kN / 16,
+                  tc::idesc_bf16(128, 64), f);
+        } else if (issuer == 2) {
+            bool f = true;
+            prod2(tbase + Cols::GB, NAJU_SA(Hh), NAJU_SA(Hl), false, NAJU_SA(Bs), false, kN / 16,
+                  tc::idesc_bf16(128, 64), f);
+        } else if (issuer == 3) {
+            bool f = false;
+            prod2(tbase + Cols::H, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Cs), true, kK / 16,
+                  tc::idesc_bf16(128, kN, false, true), f);
+            tc::mma_commit(&sm.mb2);
+        }
     };
     // Batch 2: R += W G^T, GB += U G (G transposed), dC^T = X^T U + B^T Pm^T
     // (lanes +0), dB^T = H'^T W + C^T Pm (lanes +16), all over the masked tiles.
     auto issue_b2 = [&]() {
-        bool fr = false, fg = false, fc = true, fb = true;
-        prod3(tbase + Cols::R, NAJU_SA(Wh), NAJU_SA(Wl), false, NAJU_SA(Gh), NAJU_SA(Gl), false,
-              kK / 16, tc::idesc_bf16(128, 64), fr);
-        prod3(tbase + Cols::GB, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Gh), NAJU_SA(Gl), true,
-              kK / 16, tc::idesc_bf16(128, 64, false, true), fg);
-        prod3(tbase + Cols::BC, NAJU_SA(Xh), NAJU_SA(Xl), true, NAJU_SA(Uh), NAJU_SA(Ul), true,
-              kP / 16, tc::idesc_bf16(64, 64, true, true), fc);
-        // B^T Pm^T: B (rows m = K) against Pm (rows t, K = m): hi and lo of Pm
-        prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Ph), false, kK / 16,
-             tc::idesc_bf16(64, 64, true, false), fc);
-        prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Pl), false, kK / 16,
-             tc::idesc_bf16(64, 64, true, false), fc);
-        prod3(tbase + lane16 + Cols::BC, NAJU_SA(Hh), NAJU_SA(Hl), true, NAJU_SA(Wh), NAJU_SA(Wl),
-              true, kP / 16, tc::idesc_bf16(64, 64, true, true), fb);
-        prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Ph), true, kK / 16,
-             tc::idesc_bf16(64, 64, true, true), fb);
-        prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Pl), true, kK / 16,
-             tc::idesc_bf16(64, 64, true, true), fb);
-        tc::mma_commit(&sm.mb2);
+        if (issuer == 1) {
+            bool f = false;
+            prod3(tbase + Cols::R, NAJU_SA(Wh), NAJU_SA(Wl), false, NAJU_SA(Gh), NAJU_SA(Gl), false,
+                  kK / 16, tc::idesc_bf16(128, 64), f);
+            tc::mma_commit(&sm.mb2);
+        } else if (issuer == 2) {
+            bool f = false;
+            prod3(tbase + Cols::GB, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Gh), NAJU_SA(Gl), true,
+                  kK / 16, tc::idesc_bf16(128, 64, false, true), f);
+            tc::mma_commit(&sm.mb2);
+        } else if (issuer == 4) {
+            bool f = true;
+            prod3(tbase + Cols::BC, NAJU_SA(Xh), NAJU_SA(Xl), true, NAJU_SA(Uh), NAJU_SA(Ul), true,
+                  kP / 16, tc::idesc_bf16(64, 64, true, true), f);
+            // B^T Pm^T: B (rows m = K) against Pm (rows t, K = m): hi and lo of Pm
+            prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Ph), false, kK / 16,
+                 tc::idesc_bf16(64, 64, true, false), f);
+            prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Pl), false, kK / 16,
+                 tc::idesc_bf16(64, 64, true, false), f);
+            tc::mma_commit(&sm.mb2);
+        } else if (issuer == 0) {
+            bool f = true;
+            prod3(tbase + lane16 + Cols::BC, NAJU_SA(Hh), NAJU_SA(Hl), true, NAJU_SA(Wh),
+                  NAJU_SA(Wl), true, kP / 16, tc::idesc_bf16(64, 64, true, true), f);
+            prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Ph), true, kK / 16,
+                 tc::idesc_bf16(64, 64, true, true), f);
+            prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Pl), true, kK / 16,
+                 tc::idesc_bf16(64, 64, true, true), f);
+            tc::mma_commit(&sm.mb2);
+        }
     };
     // G (lanes +0) and P (lanes +16) from tensor memory to their tile pairs,
     // lower triangle kept: this warp's lanes, columns [16 q, 16 q + 16).
@@ -763,7 +804,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     // group (last block first) from a zero carry (the sequence's dx_final for
     // the last group), then the carry leaving the group's start is published
     // after adding the decayed carry of the later group (bounded wait).
-    if (!pieces && !firstg) {
+    if (aligned1k && !pieces && !firstg) {
         const float* dxf = p.dx_final ? p.dx_final + (int64_t)bb * d * NS : nullptr;
         carry_from(lastg ? dxf : nullptr, false);
         if (tid == 0) {
@@ -821,9 +862,9 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     bool fh = false;
                     prod2(tbase + Cols::H, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Cs), true, kK / 16,
                           tc::idesc_bf16(128, kN, false, true), fh);
-                    tc::mma_commit(&sm.mb2);
+                    tc::mma_commit(&sm.mb_e);
                 }
-                wait_mb(&sm.mb2, ph2);
+                wait_mb(&sm.mb_e, ph_e);
             } else {
                 exact_carry(nv);
             }
@@ -860,7 +901,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 
     // ============================================================ main phase
     const int64_t ub_first = pieces ? (F0 / p.nsub) * p.nsub : 0;
-    const int64_t ub_end = pieces ? F1 : 1;
+    const int64_t ub_end = !aligned1k ? ub_first : pieces ? F1 : 1;
     for (int64_t ub = ub_first; ub < ub_end; ub += pieces ? p.nsub : 1) {
         if (pieces) {
             const int k0 = (int)(max64(F0, ub) - ub), k1 = (int)(min64(F1, ub + p.nsub) - ub);
@@ -952,12 +993,12 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             sync();
             // ------------------------------------------------ phase B
             if (!slow) {
-                if (tid == 0) issue_b01();
+                issue_b01();
                 wait_mb(&sm.mb0, ph0);
                 copy_gp();
                 tc::fence_proxy_async();
                 sync();
-                if (tid == 0) issue_b2();
+                issue_b2();
                 wait_mb(&sm.mb2, ph2);
             } else {
                 exact_block(tb, nv);

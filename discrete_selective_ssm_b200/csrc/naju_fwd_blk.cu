@@ -154,7 +154,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         tc::mbar_init(&sm.mb_raw, 1);
         tc::mbar_init(&sm.mb_bc, 1);
         tc::mbar_init(&sm.mb0, 1);
-        tc::mbar_init(&sm.mb2, 1);
+        tc::mbar_init(&sm.mb2, 1 + N / 64);  // R (warp 0), S by 64 columns (warps 1, 2)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         tma::prefetch_map(&tm.u);
         tma::prefetch_map(&tm.a);
@@ -171,7 +171,9 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     const uint32_t trow = tbase + ((uint32_t)(s4 * 32) << 16);
     const int item = sm.item;
     const uint32_t sbase = tc::smem_u32(&sm);
-#define NAJU_SA(f) (sbase + (uint32_t)offsetof(Sm, f))
+// tile start addresses / 16 (the base is 1024-byte aligned: checked below)
+#define NAJU_SA(f) (sb4 + (uint32_t)(offsetof(Sm, f) >> 4))
+    const uint32_t sb4 = sbase >> 4;
     uint32_t ph_raw = 0, ph_bc = 0, ph0 = 0, ph2 = 0;
     bool timed_out = false;
 
@@ -419,25 +421,31 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     // --------------------------------------------------------- the MMAs
     // D (+)= A B over nks K steps of 16, A and B bf16 tiles in the layout of
     // tc::bf_offset_w (a_rows, b_rows: their row counts).
+    // (a, b: tile start addresses / 16; K-major steps walk 32 bytes along a
+    // 128-byte row, then the next 64-column block R * 128 bytes on; MN-major
+    // steps walk 16 rows = 2048 bytes)
+    auto kstep = [](int rows, int ks) { return (uint32_t)((ks >> 2) * rows * 8 + (ks & 3) * 2); };
     auto prod = [&](uint32_t dcol, uint32_t a, int a_rows, uint32_t b, int b_rows, bool b_mn,
                     int nks, uint32_t idesc, bool& first) {
+#pragma unroll
         for (int ks = 0; ks < nks; ++ks) {
-            const uint64_t bd = b_mn ? tc::sdesc_bfw_mn(b, b_rows, ks) : tc::sdesc_bfw_k(b, b_rows, ks);
-            tc::mma_bf16_ss(dcol, tc::sdesc_bfw_k(a, a_rows, ks), bd, idesc, first ? 0u : 1u);
+            const uint64_t bd = b_mn ? tc::sdesc_sw128_mn_a4(b + ks * 128u, (uint32_t)b_rows * 128)
+                                     : tc::sdesc_sw128_a4(b + kstep(b_rows, ks));
+            tc::mma_bf16_ss(dcol, tc::sdesc_sw128_a4(a + kstep(a_rows, ks)), bd, idesc,
+                            first ? 0u : 1u);
             first = false;
         }
     };
     // S = W B: W (rows ch, K = t) against B (rows t = K, columns j = N),
     // one 64-column block of j per product.
-    auto issue_S = [&]() {
+    // (one 64-column block of S per issuing thread: lane 0 of warp 1 + jb)
+    auto issue_S = [&](int jb) {
         constexpr uint32_t id = tc::idesc_bf16(128, 64, false, true);
-#pragma unroll
-        for (int jb = 0; jb < N / 64; ++jb) {
-            const uint32_t bsrc = NAJU_SA(Bs) + (uint32_t)(jb * kK * 128);
-            bool f = true;
-            prod(tbase + Cols::S + 64 * jb, NAJU_SA(Wh), kP, bsrc, kK, true, kK / 16, id, f);
-            prod(tbase + Cols::S + 64 * jb, NAJU_SA(Wl), kP, bsrc, kK, true, kK / 16, id, f);
-        }
+        const uint32_t bsrc = NAJU_SA(Bs) + (uint32_t)(jb * kK * 8);
+        bool f = true;
+        prod(tbase + Cols::S + 64 * jb, NAJU_SA(Wh), kP, bsrc, kK, true, kK / 16, id, f);
+        prod(tbase + Cols::S + 64 * jb, NAJU_SA(Wl), kP, bsrc, kK, true, kK / 16, id, f);
+        tc::mma_commit(&sm.mb2);
     };
 
     // Exact path: the plain recurrence over the block on this thread's state
@@ -555,8 +563,9 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                 tc::fence_proxy_async();
                 sync();
             }
+            // three independent chains, one issuing thread each
+            if (lid == 0 && warp >= 1 && warp <= N / 64) issue_S(warp - 1);
             if (tid == 0) {
-                issue_S();
                 if (full) {
                     // R = X C^T + W G^T (three terms)
                     bool fr = true;
@@ -565,8 +574,10 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                     prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
                     prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gl), kK, false, kK / 16, idR, fr);
                     prod(tbase + Cols::R, NAJU_SA(Wl), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
+                    tc::mma_commit(&sm.mb2);
+                } else {
+                    tc::mbar_arrive(&sm.mb2);  // no R in an update-only pass
                 }
-                tc::mma_commit(&sm.mb2);
             }
             wait_mb(&sm.mb2, ph2);
         } else {

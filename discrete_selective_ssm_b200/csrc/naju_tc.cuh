@@ -135,6 +135,17 @@ __device__ __forceinline__ uint64_t sdesc_bfw_k(uint32_t base, int R, int ks) {
 __device__ __forceinline__ uint64_t sdesc_bfw_mn(uint32_t base, int R, int ks) {
     return sdesc_sw128_mn(base + (uint32_t)ks * 2048, (uint32_t)R * 128);
 }
+// The same two descriptors from the start address already divided by 16
+// (shared-memory addresses below 256 KB fit the 14-bit field): with the
+// tile base 1024-byte aligned, (base + offset) / 16 = base / 16 + offset / 16,
+// so a descriptor for a compile-time offset costs one add.
+__device__ __forceinline__ uint64_t sdesc_sw128_a4(uint32_t a4) {
+    return ((uint64_t)((1024u >> 4) | (1u << 14) | (2u << 29)) << 32) | (uint64_t)(a4 | (1u << 16));
+}
+__device__ __forceinline__ uint64_t sdesc_sw128_mn_a4(uint32_t a4, uint32_t lbo) {
+    return ((uint64_t)((1024u >> 4) | (1u << 14) | (2u << 29)) << 32) |
+           (uint64_t)(a4 | ((lbo >> 4) << 16));
+}
 // Instruction descriptor: D fp32, A and B bf16 (kind::f16), M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn = false,
                                                   bool b_mn = false) {

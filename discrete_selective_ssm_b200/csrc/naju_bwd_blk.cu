@@ -81,7 +81,7 @@ constexpr long long kSpin = 1LL << 24;
 // The tensor-core chains of a block are issued by lanes 0 of warps 0..5 (one
 // accumulator per thread, so each chain keeps its order): committing
 // threads per completion barrier.
-constexpr int kIss0 = 2;  // G (warp 0), P (warp 5)
+constexpr int kIss0 = 2;  // G (warp 0), P (warp 5); the exact path arrives for P
 constexpr int kIss2 = 5;  // dB (0), R (1), GB (2), carry (3), dC (4)
 
 // Tensor-memory columns (lane = channel unless stated).
@@ -636,13 +636,20 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     // Each accumulator's chain is issued by one thread (lane 0 of warp
     // `issuer`), so the chains run side by side and keep their own order.
     const int issuer = lid == 0 ? warp : -1;
-    auto issue_b01 = [&]() {
+    // G as soon as B and C have landed (thread 0 waits for them), at the start
+    // of phase A; P and R once W, U and X are in their tiles; GB and the
+    // carry once H' is.
+    auto issue_g = [&]() {
         if (issuer == 0) {
+            if (!timed_out && !tc::mbar_wait(&sm.mb_bc, ph_bc, kSpin)) timed_out = true;
             bool f = true;
             prod(tbase + Cols::BC, NAJU_SA(Cs), false, NAJU_SA(Bs), false, kN / 16,
                  tc::idesc_bf16(64, 64), f);
             tc::mma_commit(&sm.mb0);
-        } else if (issuer == 5) {
+        }
+    };
+    auto issue_pr = [&]() {
+        if (issuer == 5) {
             bool f = true;
             prod3(tbase + lane16 + Cols::BC, NAJU_SA(Uh), NAJU_SA(Ul), true, NAJU_SA(Wh),
                   NAJU_SA(Wl), true, kP / 16, tc::idesc_bf16(64, 64, true, true), f);
@@ -651,7 +658,10 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             bool f = true;
             prod2(tbase + Cols::R, NAJU_SA(Xh), NAJU_SA(Xl), false, NAJU_SA(Cs), false, kN / 16,
                   tc::idesc_bf16(128, 64), f);
-        } else if (issuer == 2) {
+        }
+    };
+    auto issue_gbh = [&]() {
+        if (issuer == 2) {
             bool f = true;
             prod2(tbase + Cols::GB, NAJU_SA(Hh), NAJU_SA(Hl), false, NAJU_SA(Bs), false, kN / 16,
                   tc::idesc_bf16(128, 64), f);
@@ -977,6 +987,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             }
             wait_mb2(&sm.mb_in, ph_in, &sm.mb_x, ph_x);
             store_out();  // the previous block's staged gradients (after that barrier)
+            issue_g();    // (the exact path waits for it too, to keep the barrier phases)
             float xr[16];
             read_x(xr);
             // the staged gradients must have left the W / U bytes before unpack
@@ -986,14 +997,20 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             st8o(sm.Xh, sm.Xl, oc1, xr + 8);
             unpack(slow);
             tc::tmem_st_wait();
+            tc::fence_proxy_async();
             wait_mb(&sm.mb_bc, ph_bc);  // and region A's per-token inputs are read
-            if (!slow) scale_carry(true);
+            if (!slow) {
+                issue_pr();
+                scale_carry(true);
+            } else if (issuer == 5) {
+                tc::mbar_arrive(&sm.mb0);  // no P on the exact path
+            }
             tc::tmem_st_wait();
             tc::fence_proxy_async();
             sync();
             // ------------------------------------------------ phase B
             if (!slow) {
-                issue_b01();
+                issue_gbh();
                 wait_mb(&sm.mb0, ph0);
                 copy_gp();
                 tc::fence_proxy_async();
@@ -1001,6 +1018,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 issue_b2();
                 wait_mb(&sm.mb2, ph2);
             } else {
+                wait_mb(&sm.mb0, ph0);  // G (unused here)
                 exact_block(tb, nv);
             }
             // ------------------------------------------------ phase C

@@ -480,7 +480,9 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     auto uwin = [&](int m) { return (m & 1) ? bf_hi(upk[m >> 1]) : bf_lo(upk[m >> 1]); };
     // No token masks: past the end, dout, B and C read zero, so U, GB and
     // dp = c0 + c1 GB vanish and W meets only zero rows; the decays mask.
-    auto unpack = [&](bool slow) {
+    auto unpack_v = [&](bool slow, auto hb_c, auto hz_c) {
+        constexpr bool has_b = decltype(hb_c)::value;
+        constexpr bool has_z = decltype(hz_c)::value;
         const unsigned short* rup = reinterpret_cast<const unsigned short*>(sm.ru) + ro;
         const __nv_bfloat16* rbp = rb + ro;
         const __nv_bfloat16* rzp = rz + ro;
@@ -586,6 +588,17 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             tc::tmem_st4(trow + Cols::SV + 3 * 64 + col, s3);
         }
     };
+    // (four variants: b and z present or not)
+    auto unpack = [&](bool slow) {
+        if (p.b != nullptr) {
+            if (p.z != nullptr) unpack_v(slow, std::true_type{}, std::true_type{});
+            else unpack_v(slow, std::true_type{}, std::false_type{});
+        } else {
+            if (p.z != nullptr) unpack_v(slow, std::false_type{}, std::true_type{});
+            else unpack_v(slow, std::false_type{}, std::false_type{});
+        }
+    };
+
     // H' = E_63 H into tensor memory and (tiles) into the H tile pair (its
     // initial value: carry out = U C + H').
     auto scale_carry = [&](bool tiles) {
@@ -1084,162 +1097,175 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 __syncthreads();
                 if (tid == 0 && k > kb0) load_x(k - 1);
             } else {
-            // Pass 1 (tokens in order): dL; the quarter's sum of dL and its
-            // first three dp for the neighbouring quarter.
-            float dL[16];
-            float qsum = 0.f, dpf0 = 0.f, dpf1 = 0.f, dpf2 = 0.f;
-            uint4 uh4, ul4, wh4, wl4;  // 8 tokens of U and W hi / lo
+            // The epilogue in four variants (b and z present or not), so no
+            // per-token branch tests them.
+            auto epilogue = [&](auto hb_c, auto hz_c) {
+                constexpr bool hb = decltype(hb_c)::value;
+                constexpr bool hz = decltype(hz_c)::value;
+                // Pass 1 (tokens in order): dL; the quarter's sum of dL and its
+                // first three dp for the neighbouring quarter.
+                float dL[16];
+                float qsum = 0.f, dpf0 = 0.f, dpf1 = 0.f, dpf2 = 0.f;
+                uint4 uh4, ul4, wh4, wl4;  // 8 tokens of U and W hi / lo
 #pragma unroll
-            for (int g4 = 0; g4 < 4; ++g4) {
-                const int col = 16 * q + 4 * g4;
-                float R4[4], G4[4], b2[4], Ua[4], Wa[4];
-                tc::tmem_ld4(trow + Cols::R + col, R4);
-                tc::tmem_ld4(trow + Cols::GB + col, G4);
-                if (!has_b) tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
-                if ((g4 & 1) == 0) {
-                    const uint32_t o = g4 < 2 ? oc0 : oc1;
-                    auto ld = [&](const __nv_bfloat16* t) {
-                        return *reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(t) + o);
-                    };
-                    uh4 = ld(sm.Uh);
-                    ul4 = ld(sm.Ul);
-                    wh4 = ld(sm.Wh);
-                    wl4 = ld(sm.Wl);
-                }
-                {
-                    const bool hi = (g4 & 1) != 0;
-                    const uint32_t a0 = hi ? uh4.z : uh4.x, a1 = hi ? uh4.w : uh4.y;
-                    const uint32_t b0 = hi ? ul4.z : ul4.x, b1 = hi ? ul4.w : ul4.y;
-                    const uint32_t c0_ = hi ? wh4.z : wh4.x, c1_ = hi ? wh4.w : wh4.y;
-                    const uint32_t d0 = hi ? wl4.z : wl4.x, d1 = hi ? wl4.w : wl4.y;
-                    Ua[0] = bf_lo(a0) + bf_lo(b0); Ua[1] = bf_hi(a0) + bf_hi(b0);
-                    Ua[2] = bf_lo(a1) + bf_lo(b1); Ua[3] = bf_hi(a1) + bf_hi(b1);
-                    Wa[0] = bf_lo(c0_) + bf_lo(d0); Wa[1] = bf_hi(c0_) + bf_hi(d0);
-                    Wa[2] = bf_lo(c1_) + bf_lo(d1); Wa[3] = bf_hi(c1_) + bf_hi(d1);
-                }
-                tc::tmem_ld_wait();
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const int kk = 4 * g4 + k4;
-                    float dl = Ua[k4] * R4[k4] - Wa[k4] * G4[k4];
-                    if (has_b) {
-                        qsum += dl;
-                    } else {
-                        // coupled gate: the sums over later tokens keep the plain dL,
-                        // this token's da loses f h lambda.B (kept in dL[kk])
-                        qsum += dl;
-                        dl = fmaf(-b2[k4], G4[k4], dl);
-                    }
-                    dL[kk] = dl;
-                    if (kk == 0) dpf0 = fmaf(c1v[0], G4[k4], c0v[0]);
-                    if (kk == 1) dpf1 = fmaf(c1v[1], G4[k4], c0v[1]);
-                    if (kk == 2) dpf2 = fmaf(c1v[2], G4[k4], c0v[2]);
-                }
-            }
-            sm.xs[q][ch] = qsum;
-            sm.dph[q][0][ch] = dpf0;
-            sm.dph[q][1][ch] = dpf1;
-            sm.dph[q][2][ch] = dpf2;
-            __syncthreads();
-            // the X tiles and the W, U tiles are read: the next checkpoint may land
-            if (tid == 0 && k > kb0) load_x(k - 1);
-            float base = 0.f;  // dL over the later quarters, plus the tail
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                if (qq > q) base += sm.xs[qq][ch];
-                base += sm.tailp[par][qq][ch];
-            }
-            if (kImport && cvalid) base += __ldcg(p.tail_part + ((int64_t)bb * p.nsub + k) * d + c);
-            float n1, n2, n3;  // dp of the three tokens after the current one
-            if (q < 3) {
-                n1 = sm.dph[q + 1][0][ch];
-                n2 = sm.dph[q + 1][1][ch];
-                n3 = sm.dph[q + 1][2][ch];
-            } else {
-                n1 = sm.dnext[par][0][ch];
-                n2 = sm.dnext[par][1][ch];
-                n3 = sm.dnext[par][2][ch];
-            }
-            // Pass 2 (tokens in reverse): da from the suffix sums of dL, dz, db;
-            // dp, the conv backward (du, dw, dbias) from a window of later dp.
-            // bf16 gradients go to the staging buffers over the W and U tiles
-            // (dz, db, da, dh or du), fp32 ones straight to global memory.
-            {
-                const int64_t gofs = ((int64_t)bb * L + tb + 16 * q) * d + c;
-                auto put = [&](__nv_bfloat16* stage, void* gbase, int kk, float v) {
-                    if constexpr (kStage) {
-                        stage[ro + kk * kP] = __float2bfloat16_rn(v);
-                    } else {
-                        if (kk < nq) static_cast<float*>(gbase)[gofs + (int64_t)kk * d] = v;
-                    }
-                };
-                float dw0 = 0.f, dw1 = 0.f, dw2 = 0.f, dw3 = 0.f, dbias = 0.f;
-                float run = base;
-                const bool seg_end = !lastg && k == kb1 - 1;  // a full block
-#pragma unroll
-                for (int g4 = 3; g4 >= 0; --g4) {
+                for (int g4 = 0; g4 < 4; ++g4) {
                     const int col = 16 * q + 4 * g4;
-                    float G4[4], om[4], b2[4], R4[4], z1[4], z0[4];
+                    float R4[4], G4[4], b2[4], Ua[4], Wa[4];
+                    tc::tmem_ld4(trow + Cols::R + col, R4);
                     tc::tmem_ld4(trow + Cols::GB + col, G4);
-                    tc::tmem_ld4(trow + Cols::SV + 3 * 64 + col, om);
-                    tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
-                    if (has_z) {
-                        tc::tmem_ld4(trow + Cols::R + col, R4);
-                        tc::tmem_ld4(trow + Cols::SV + 0 * 64 + col, z1);
-                        tc::tmem_ld4(trow + Cols::SV + 1 * 64 + col, z0);
+                    if (!hb) tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
+                    if ((g4 & 1) == 0) {
+                        const uint32_t o = g4 < 2 ? oc0 : oc1;
+                        auto ld = [&](const __nv_bfloat16* t) {
+                            return *reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(t) + o);
+                        };
+                        uh4 = ld(sm.Uh);
+                        ul4 = ld(sm.Ul);
+                        wh4 = ld(sm.Wh);
+                        wl4 = ld(sm.Wl);
+                    }
+                    {
+                        const bool hi = (g4 & 1) != 0;
+                        const uint32_t a0 = hi ? uh4.z : uh4.x, a1 = hi ? uh4.w : uh4.y;
+                        const uint32_t b0 = hi ? ul4.z : ul4.x, b1 = hi ? ul4.w : ul4.y;
+                        const uint32_t c0_ = hi ? wh4.z : wh4.x, c1_ = hi ? wh4.w : wh4.y;
+                        const uint32_t d0 = hi ? wl4.z : wl4.x, d1 = hi ? wl4.w : wl4.y;
+                        Ua[0] = bf_lo(a0) + bf_lo(b0); Ua[1] = bf_hi(a0) + bf_hi(b0);
+                        Ua[2] = bf_lo(a1) + bf_lo(b1); Ua[3] = bf_hi(a1) + bf_hi(b1);
+                        Wa[0] = bf_lo(c0_) + bf_lo(d0); Wa[1] = bf_hi(c0_) + bf_hi(d0);
+                        Wa[2] = bf_lo(c1_) + bf_lo(d1); Wa[3] = bf_hi(c1_) + bf_hi(d1);
                     }
                     tc::tmem_ld_wait();
 #pragma unroll
-                    for (int k4 = 3; k4 >= 0; --k4) {
+                    for (int k4 = 0; k4 < 4; ++k4) {
                         const int kk = 4 * g4 + k4;
-                        float fdf;
-                        if (has_b) {
-                            run += dL[kk];
-                            fdf = run;
-                        } else {  // dL[kk] holds dL - f h lambda.B
-                            fdf = run + dL[kk];
-                            run += fmaf(b2[k4], G4[k4], dL[kk]);
-                        }
-                        put(sm.Uh, p.da, kk, fdf * om[k4]);
-                        if (has_z) put(sm.Wh, p.dz, kk, fmaf(z1[k4], R4[k4], z0[k4]));
-                        if (has_b) put(sm.Wl, p.db, kk, b2[k4] * G4[k4]);
-                        const float dpv = fmaf(c1v[kk], G4[k4], c0v[kk]);  // 0 outside
-                        if (CONV) {
-                            const float duv = fmaf(w3, dpv, fmaf(w2, n1, fmaf(w1, n2, w0 * n3)));
-                            // u and dp vanish outside the tensor: no masks
-                            dw0 = fmaf(dpv, uwin(kk), dw0);
-                            dw1 = fmaf(dpv, uwin(kk + 1), dw1);
-                            dw2 = fmaf(dpv, uwin(kk + 2), dw2);
-                            dw3 = fmaf(dpv, uwin(kk + 3), dw3);
-                            dbias += dpv;
-                            put(sm.Ul, p.dhu, kk, duv);
-                            // the segment's last three du are partial (fixed up later)
-                            if (kk >= 13 && q == 3 && seg_end && cvalid)
-                                edge_row()[(3 + (kk - 13)) * d + c] = duv;
-                            if (kk < 3 && q == 0 && k == kb0 && kk < nq) edge_row()[kk * d + c] = dpv;
-                            n3 = n2;
-                            n2 = n1;
-                            n1 = dpv;
+                        float dl = Ua[k4] * R4[k4] - Wa[k4] * G4[k4];
+                        if (hb) {
+                            qsum += dl;
                         } else {
-                            put(sm.Ul, p.dhu, kk, dpv);
+                            // coupled gate: the sums over later tokens keep the plain dL,
+                            // this token's da loses f h lambda.B (kept in dL[kk])
+                            qsum += dl;
+                            dl = fmaf(-b2[k4], G4[k4], dl);
+                        }
+                        dL[kk] = dl;
+                        if (kk == 0) dpf0 = fmaf(c1v[0], G4[k4], c0v[0]);
+                        if (kk == 1) dpf1 = fmaf(c1v[1], G4[k4], c0v[1]);
+                        if (kk == 2) dpf2 = fmaf(c1v[2], G4[k4], c0v[2]);
+                    }
+                }
+                sm.xs[q][ch] = qsum;
+                sm.dph[q][0][ch] = dpf0;
+                sm.dph[q][1][ch] = dpf1;
+                sm.dph[q][2][ch] = dpf2;
+                __syncthreads();
+                // the X tiles and the W, U tiles are read: the next checkpoint may land
+                if (tid == 0 && k > kb0) load_x(k - 1);
+                float base = 0.f;  // dL over the later quarters, plus the tail
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    if (qq > q) base += sm.xs[qq][ch];
+                    base += sm.tailp[par][qq][ch];
+                }
+                if (kImport && cvalid) base += __ldcg(p.tail_part + ((int64_t)bb * p.nsub + k) * d + c);
+                float n1, n2, n3;  // dp of the three tokens after the current one
+                if (q < 3) {
+                    n1 = sm.dph[q + 1][0][ch];
+                    n2 = sm.dph[q + 1][1][ch];
+                    n3 = sm.dph[q + 1][2][ch];
+                } else {
+                    n1 = sm.dnext[par][0][ch];
+                    n2 = sm.dnext[par][1][ch];
+                    n3 = sm.dnext[par][2][ch];
+                }
+                // Pass 2 (tokens in reverse): da from the suffix sums of dL, dz, db;
+                // dp, the conv backward (du, dw, dbias) from a window of later dp.
+                // bf16 gradients go to the staging buffers over the W and U tiles
+                // (dz, db, da, dh or du), fp32 ones straight to global memory.
+                {
+                    [[maybe_unused]] const int64_t gofs = ((int64_t)bb * L + tb + 16 * q) * d + c;
+                    auto put = [&](__nv_bfloat16* stage, void* gbase, int kk, float v) {
+                        if constexpr (kStage) {
+                            stage[ro + kk * kP] = __float2bfloat16_rn(v);
+                        } else {
+                            if (kk < nq) static_cast<float*>(gbase)[gofs + (int64_t)kk * d] = v;
+                        }
+                    };
+                    float dw0 = 0.f, dw1 = 0.f, dw2 = 0.f, dw3 = 0.f, dbias = 0.f;
+                    float run = base;
+                    const bool seg_end = !lastg && k == kb1 - 1;  // a full block
+#pragma unroll
+                    for (int g4 = 3; g4 >= 0; --g4) {
+                        const int col = 16 * q + 4 * g4;
+                        float G4[4], om[4], b2[4], R4[4], z1[4], z0[4];
+                        tc::tmem_ld4(trow + Cols::GB + col, G4);
+                        tc::tmem_ld4(trow + Cols::SV + 3 * 64 + col, om);
+                        tc::tmem_ld4(trow + Cols::SV + 2 * 64 + col, b2);
+                        if (hz) {
+                            tc::tmem_ld4(trow + Cols::R + col, R4);
+                            tc::tmem_ld4(trow + Cols::SV + 0 * 64 + col, z1);
+                            tc::tmem_ld4(trow + Cols::SV + 1 * 64 + col, z0);
+                        }
+                        tc::tmem_ld_wait();
+#pragma unroll
+                        for (int k4 = 3; k4 >= 0; --k4) {
+                            const int kk = 4 * g4 + k4;
+                            float fdf;
+                            if (hb) {
+                                run += dL[kk];
+                                fdf = run;
+                            } else {  // dL[kk] holds dL - f h lambda.B
+                                fdf = run + dL[kk];
+                                run += fmaf(b2[k4], G4[k4], dL[kk]);
+                            }
+                            put(sm.Uh, p.da, kk, fdf * om[k4]);
+                            if (hz) put(sm.Wh, p.dz, kk, fmaf(z1[k4], R4[k4], z0[k4]));
+                            if (hb) put(sm.Wl, p.db, kk, b2[k4] * G4[k4]);
+                            const float dpv = fmaf(c1v[kk], G4[k4], c0v[kk]);  // 0 outside
+                            if (CONV) {
+                                const float duv = fmaf(w3, dpv, fmaf(w2, n1, fmaf(w1, n2, w0 * n3)));
+                                // u and dp vanish outside the tensor: no masks
+                                dw0 = fmaf(dpv, uwin(kk), dw0);
+                                dw1 = fmaf(dpv, uwin(kk + 1), dw1);
+                                dw2 = fmaf(dpv, uwin(kk + 2), dw2);
+                                dw3 = fmaf(dpv, uwin(kk + 3), dw3);
+                                dbias += dpv;
+                                put(sm.Ul, p.dhu, kk, duv);
+                                // the segment's last three du are partial (fixed up later)
+                                if (kk >= 13 && q == 3 && seg_end && cvalid)
+                                    edge_row()[(3 + (kk - 13)) * d + c] = duv;
+                                if (kk < 3 && q == 0 && k == kb0 && kk < nq) edge_row()[kk * d + c] = dpv;
+                                n3 = n2;
+                                n2 = n1;
+                                n1 = dpv;
+                            } else {
+                                put(sm.Ul, p.dhu, kk, dpv);
+                            }
+                        }
+                    }
+                    if (q == 0) {
+                        sm.dnext[par ^ 1][0][ch] = dpf0;
+                        sm.dnext[par ^ 1][1][ch] = dpf1;
+                        sm.dnext[par ^ 1][2][ch] = dpf2;
+                    }
+                    if (cvalid) {
+                        atomicAdd(&sm.red6[0][ch], dD_acc);
+                        if (CONV) {
+                            atomicAdd(&sm.red6[1][ch], dw0);
+                            atomicAdd(&sm.red6[2][ch], dw1);
+                            atomicAdd(&sm.red6[3][ch], dw2);
+                            atomicAdd(&sm.red6[4][ch], dw3);
+                            atomicAdd(&sm.red6[5][ch], dbias);
                         }
                     }
                 }
-                if (q == 0) {
-                    sm.dnext[par ^ 1][0][ch] = dpf0;
-                    sm.dnext[par ^ 1][1][ch] = dpf1;
-                    sm.dnext[par ^ 1][2][ch] = dpf2;
-                }
-                if (cvalid) {
-                    atomicAdd(&sm.red6[0][ch], dD_acc);
-                    if (CONV) {
-                        atomicAdd(&sm.red6[1][ch], dw0);
-                        atomicAdd(&sm.red6[2][ch], dw1);
-                        atomicAdd(&sm.red6[3][ch], dw2);
-                        atomicAdd(&sm.red6[4][ch], dw3);
-                        atomicAdd(&sm.red6[5][ch], dbias);
-                    }
-                }
+            };
+            if (has_b) {
+                if (has_z) epilogue(std::true_type{}, std::true_type{});
+                else epilogue(std::true_type{}, std::false_type{});
+            } else {
+                if (has_z) epilogue(std::false_type{}, std::true_type{});
+                else epilogue(std::false_type{}, std::false_type{});
             }
             }  // (gradients of the per-token inputs)
             // dC^T (lanes +0) and dB^T (lanes +16): this warp's lanes, columns

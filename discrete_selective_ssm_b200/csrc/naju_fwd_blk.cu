@@ -324,7 +324,9 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     // W to its tile pair; full: s E SiLU(z) and D h SiLU(z) to tensor memory.
     // slow (exact path): E = Q = 1, so W = i h.  W of a token past the end
     // meets only zero rows of B (and of G), so no token mask is needed here.
-    auto unpack = [&](bool slow, bool full) {
+    auto unpack_v = [&](bool slow, bool full, auto hb_c, auto hz_c) {
+        constexpr bool has_b = decltype(hb_c)::value;
+        constexpr bool has_z = decltype(hz_c)::value;  // (z read only in a full pass)
         const __nv_bfloat16* rup = sm.ru + 16 * q * kP + ch;  // row i: token 16 q - 3 + i
         const __nv_bfloat16* rbp = sm.rb + 16 * q * kP + ch;
         const __nv_bfloat16* rzp = sm.rz + 16 * q * kP + ch;
@@ -415,6 +417,17 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                 tc::tmem_st8(trow + Cols::SV + col, s0);
                 tc::tmem_st8(trow + Cols::SV + 64 + col, s1);
             }
+        }
+    };
+    // (four variants: b present or not, z used or not)
+    auto unpack = [&](bool slow, bool full) {
+        const bool uz = full && p.z != nullptr;
+        if (p.b != nullptr) {
+            if (uz) unpack_v(slow, full, std::true_type{}, std::true_type{});
+            else unpack_v(slow, full, std::true_type{}, std::false_type{});
+        } else {
+            if (uz) unpack_v(slow, full, std::false_type{}, std::true_type{});
+            else unpack_v(slow, full, std::false_type{}, std::false_type{});
         }
     };
 

@@ -123,6 +123,15 @@ naju_status naju_testing_tc_mma_gen(int32_t M, int32_t N, int32_t K, int32_t a_m
                                     int32_t d_lane, int32_t kind, const float* A, const float* B,
                                     float* D, int* status, void* stream);
 
+/* The block-form kernels' fast exponential and sigmoids, for n device fp32
+ * inputs x: ex = e^x computed as 2^(x log2 e) with the MUFU base-2 unit (PTX
+ * ex2.approx.ftz; results below the normal range flush to zero), sig =
+ * 1 / (1 + e^{-x}) with the approximate reciprocal, and sig3 = the forward's
+ * shared-reciprocal form of sigma(x) taken together with sigma(x / 2) and
+ * sigma(-x) (each e^{-v} capped at 2^36).  Device pointers, n >= 0. */
+naju_status naju_testing_fast_math(const float* x, float* ex, float* sig, float* sig3, int64_t n,
+                                   void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -112,3 +112,53 @@ def test_tc_mma_mn_major_m64_and_split(M, N, K, a_mn, b_mn, d_lane, kind):
     others = sorted(set(range(128)) - set(lanes))
     if others:  # lanes outside the result keep the zeros written before the MMA
         assert np.all(raw[others] == 0.0)
+
+
+def test_fast_math_against_fp64_and_cuda_expf():
+    """The block-form kernels compute e^x as 2^(x log2 e) on the MUFU base-2
+    unit (PTX ex2.approx.ftz) and sigma(x) = 1 / (1 + e^{-x}) with the
+    approximate reciprocal; the forward shares one reciprocal among three
+    sigmoids with each e^{-v} capped at 2^36.  Bounds, derived: rounding
+    x log2 e costs |x| log2(e) 2^-24 in the exponent, i.e. a relative error
+    of at most 88 * 1.4427 * 2^-24 * ln 2 < 5.3e-6 in e^x for |x| <= 88, plus
+    the base-2 unit's few ulp; results below the normal range (x < -87.33)
+    may flush to zero.  sigma(x) then errs by < 2e-6 absolute; the capped
+    form also moves sigma(x) for x < -24.95 to 1 / (1 + 2^36) < 1.46e-11."""
+    L = naju.lib()
+    f = L.naju_testing_fast_math
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    g = torch.Generator().manual_seed(7)
+    x = torch.cat([torch.linspace(-100.0, 100.0, 200001), 5.0 * torch.randn(100000, generator=g),
+                   torch.tensor([0.0, 1e-30, -1e-30, 88.0, -87.3, -87.4, 40.0, -40.0, 24.9, -24.9,
+                                 -25.0, 25.0])])
+    dx = x.cuda()
+    ex = torch.empty_like(dx)
+    sig = torch.empty_like(dx)
+    sig3 = torch.empty_like(dx)
+    rc = f(ctypes.c_void_p(dx.data_ptr()), ctypes.c_void_p(ex.data_ptr()),
+           ctypes.c_void_p(sig.data_ptr()), ctypes.c_void_p(sig3.data_ptr()), x.numel(),
+           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    cuda_exp = torch.exp(dx).cpu().double().numpy()  # CUDA's expf
+    torch.cuda.synchronize()
+    xd = x.double().numpy()
+    e64 = np.exp(xd)
+    got = ex.cpu().double().numpy()
+    normal = (xd > -87.3) & (xd < 88.5)
+    rel = np.abs(got[normal] - e64[normal]) / e64[normal]
+    assert rel.max() < 6e-6, rel.max()
+    rel_cuda = np.abs(got[normal] - cuda_exp[normal]) / cuda_exp[normal]
+    assert rel_cuda.max() < 6e-6, rel_cuda.max()
+    assert np.all(got[xd <= -87.3] <= 1.22e-38)  # e^-87.3 = 1.2193e-38
+    s64 = 1.0 / (1.0 + np.exp(-xd))
+    s = sig.cpu().double().numpy()
+    assert np.max(np.abs(s - s64)) < 2e-6
+    big = s64 > 1e-30
+    assert np.max(np.abs(s[big] - s64[big]) / s64[big]) < 1e-5
+    s3 = sig3.cpu().double().numpy()
+    assert np.all(np.isfinite(s3))
+    assert np.max(np.abs(s3 - s64)) < 2e-6
+    unc = xd > -24.9
+    assert np.max(np.abs(s3[unc] - s64[unc]) / s64[unc]) < 2e-5
+    assert np.max(np.abs(s3[~unc] - s64[~unc])) < 1.46e-11

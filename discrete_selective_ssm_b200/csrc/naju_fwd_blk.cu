@@ -451,7 +451,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     };
     // S = W B: W (rows ch, K = t) against B (rows t = K, columns j = N),
     // one 64-column block of j per product.
-    // (one 64-column block of S per issuing thread: lane 0 of warp 1 + jb)
+    // (one 64-column block of S per issuing thread: lane 0 of warp 1 + jb;
+    // on the exact path those threads arrive instead)
     auto issue_S = [&](int jb) {
         constexpr uint32_t id = tc::idesc_bf16(128, 64, false, true);
         const uint32_t bsrc = NAJU_SA(Bs) + (uint32_t)(jb * kK * 8);
@@ -546,6 +547,13 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         ph_bc ^= 1u;
         wait_mb(&sm.mb_raw, ph_raw);
         store_y();
+        // R = X C^T: the X tiles (state entering the block) are in place since
+        // that barrier and C has landed; R += W G^T follows on the same thread
+        if (full && tid == 0) {
+            bool fr = true;
+            prod(tbase + Cols::R, NAJU_SA(Xh), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
+            prod(tbase + Cols::R, NAJU_SA(Xl), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
+        }
         const bool slow = decays(nv);
         unpack(slow, full);
         tc::tmem_st_wait();
@@ -558,6 +566,11 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         }
         // the raw buffer is read (the exact path still needs a)
         if (tid == 0 && next >= 0 && !slow) load_raw(next, full);
+        // S = W B, one 64-column block per issuing thread, runs during the G copy
+        if (lid == 0 && warp >= 1 && warp <= N / 64) {
+            if (!slow) issue_S(warp - 1);
+            else tc::mbar_arrive(&sm.mb2);
+        }
         if (!slow) {
             if (full) {
                 {   // masked G to its tile pair: lanes 0-15 of each sub-partition hold rows
@@ -576,14 +589,10 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                 tc::fence_proxy_async();
                 sync();
             }
-            // three independent chains, one issuing thread each
-            if (lid == 0 && warp >= 1 && warp <= N / 64) issue_S(warp - 1);
             if (tid == 0) {
                 if (full) {
-                    // R = X C^T + W G^T (three terms)
-                    bool fr = true;
-                    prod(tbase + Cols::R, NAJU_SA(Xh), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
-                    prod(tbase + Cols::R, NAJU_SA(Xl), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
+                    // R += W G^T (three terms)
+                    bool fr = false;
                     prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
                     prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gl), kK, false, kK / 16, idR, fr);
                     prod(tbase + Cols::R, NAJU_SA(Wl), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
@@ -594,6 +603,12 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             }
             wait_mb(&sm.mb2, ph2);
         } else {
+            // R = X C^T may still read the X tiles, whose bytes the exact path reuses
+            if (tid == 0) {
+                if (full) tc::mma_commit(&sm.mb2);
+                else tc::mbar_arrive(&sm.mb2);
+            }
+            wait_mb(&sm.mb2, ph2);
             exact_block(nv, full);
             if (tid == 0 && next >= 0) load_raw(next, full);
         }

@@ -499,16 +499,31 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         sync();
     };
     // X <- E_63 (X + S) on this thread's columns.
-    auto update_state = [&]() {
+    // After a block: X <- E_63 (X + S) on this thread's columns (the exact
+    // path has updated X already), then the new state to a global [d][N] row
+    // (dst != null) and to the X tile pair (tiles), from the same registers.
+    auto advance = [&](bool slow, float* dst, bool tiles) {
 #pragma unroll
         for (int k = 0; k < NQ; k += 16) {
-            float xv[16], sv[16];
-            tc::tmem_ld16(trow + Cols::X + NQ * q + k, xv);
-            tc::tmem_ld16(trow + Cols::S + NQ * q + k, sv);
+            float v[16], sv[16];
+            tc::tmem_ld16(trow + Cols::X + NQ * q + k, v);
+            if (!slow) tc::tmem_ld16(trow + Cols::S + NQ * q + k, sv);
             tc::tmem_ld_wait();
+            if (!slow) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xv[j] = E63 * (xv[j] + sv[j]);
-            tc::tmem_st16(trow + Cols::X + NQ * q + k, xv);
+                for (int j = 0; j < 16; ++j) v[j] = E63 * (v[j] + sv[j]);
+                tc::tmem_st16(trow + Cols::X + NQ * q + k, v);
+            }
+            if (dst && cvalid) {
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                    *reinterpret_cast<float4*>(dst + c * N + NQ * q + k + j) =
+                        make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
+            if (tiles) {
+                st8(sm.Xh, sm.Xl, ch, NQ * q + k, kP, v);
+                st8(sm.Xh, sm.Xl, ch, NQ * q + k + 8, kP, v + 8);
+            }
         }
         tc::tmem_st_wait();
     };
@@ -633,8 +648,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                     if (kk < nk) gy[(int64_t)kk * d] = from_f<Tout>(fmaf(e[kk], r[kk], dh[kk]));
             }
         }
-        if (!slow) update_state();
         logP += __logf(E63);  // decay over the block (for the look-back)
+        return slow;
     };
 
     // ============================================================ passes
@@ -651,8 +666,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         sync();
         for (int k = s0; k < s1; ++k) {
             const bool last = k + 1 == s1;
-            run_block(k, full, last ? -1 : k + 1);
-            state_out(full && (!last || end_ckpt) ? ck_at(k + 1) : nullptr, full && !last);
+            const bool slow = run_block(k, full, last ? -1 : k + 1);
+            advance(slow, full && (!last || end_ckpt) ? ck_at(k + 1) : nullptr, full && !last);
             // X tiles and the staged y -> async proxy; the next block's first
             // barrier orders them before its MMAs and y's store
             tc::fence_proxy_async();

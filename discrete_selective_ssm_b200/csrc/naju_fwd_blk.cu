@@ -81,8 +81,10 @@ template <int N>
 struct FkSmem {
     alignas(1024) __nv_bfloat16 Wh[kP * kK], Wl[kP * kK];  // rows ch, cols t
     alignas(1024) __nv_bfloat16 Xh[kP * N], Xl[kP * N];    // rows ch, cols j
-    alignas(1024) __nv_bfloat16 Bs[kK * N], Cs[kK * N];    // rows t, cols j
-    alignas(1024) __nv_bfloat16 Gh[kK * kK], Gl[kK * kK];  // rows t, cols m (m <= t)
+    // B (rows t, cols j) and the hi tile of G^T (rows m, cols t', m <= t') side by
+    // side: one MN-major operand [B | G^T] of N + 64 columns for S and R together
+    alignas(1024) __nv_bfloat16 Bs[kK * N], GTh[kK * kK];
+    alignas(1024) __nv_bfloat16 Cs[kK * N], GTl[kK * kK];  // C: rows t, cols j
     alignas(1024) __nv_bfloat16 ru[(kK + 3) * kP];         // u of tokens tb - 3 ..
     alignas(128) __nv_bfloat16 ra[kK * kP], rb[kK * kP], rz[kK * kP];
     float xq[4][kP], xe[4][kP];
@@ -131,6 +133,11 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     // bf16 outputs are staged in the G tiles' bytes (free once R is complete)
     // and leave by one TMA store per block; fp32 outputs are stored directly
     constexpr bool kStageY = std::is_same<Tout, __nv_bfloat16>::value;
+    static_assert(offsetof(Sm, GTh) == offsetof(Sm, Bs) + sizeof(Sm::Bs) &&
+                      sizeof(Sm::Bs) == (size_t)(N / 64) * kK * 128,
+                  "B and G^T are one MN-major operand: 64-column blocks kK * 128 bytes apart");
+    static_assert(Cols::R == Cols::S + N, "S and R are one accumulator [S | R]");
+    const float kZero16[16] = {};
     static_assert(sizeof(Sm::Xh) + sizeof(Sm::Xl) >= kK * kP * sizeof(float),
                   "the exact path's row sums live over the X tiles");
     extern __shared__ __align__(1024) float4 smem4[];
@@ -513,6 +520,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = E63 * (v[j] + sv[j]);
                 tc::tmem_st16(trow + Cols::X + NQ * q + k, v);
+                tc::tmem_st16(trow + Cols::S + NQ * q + k, kZero16);  // S accumulates from zero
             }
             if (dst && cvalid) {
 #pragma unroll
@@ -538,7 +546,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     int y_pending = -1;
     auto store_y = [&]() {
         if (kStageY && tid == 0 && y_pending >= 0) {
-            tma::store_3d(&tm.y, (int)c0, y_pending * kK, bb, sm.Gh);
+            tma::store_3d(&tm.y, (int)c0, y_pending * kK, bb, sm.Wh);
             tma::store_commit();
         }
         y_pending = -1;
@@ -553,8 +561,9 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         if (tid == 0) {
             if (!timed_out && !tc::mbar_wait(&sm.mb_bc, ph_bc, kSpin)) timed_out = true;
             if (full) {
+                // G^T = B C^T (M = 64: rows m, columns t')
                 bool fg = true;
-                prod(tbase + Cols::G, NAJU_SA(Cs), kK, NAJU_SA(Bs), kK, false, N / 16,
+                prod(tbase + Cols::G, NAJU_SA(Bs), kK, NAJU_SA(Cs), kK, false, N / 16,
                      tc::idesc_bf16(64, 64), fg);
                 tc::mma_commit(&sm.mb0);
             }
@@ -569,11 +578,13 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             prod(tbase + Cols::R, NAJU_SA(Xh), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
             prod(tbase + Cols::R, NAJU_SA(Xl), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
         }
+        // the previous block's y (staged over W) must have left before unpack
+        // rewrites W (the decays' barrier orders this wait)
+        if (kStageY && tid == 0) tma::store_wait_read();
         const bool slow = decays(nv);
         unpack(slow, full);
         tc::tmem_st_wait();
         tc::fence_proxy_async();
-        if (kStageY && tid == 0) tma::store_wait_read();  // the previous y has left G
         if (full) {
             wait_mb(&sm.mb0, ph0);
         } else {
@@ -581,14 +592,16 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         }
         // the raw buffer is read (the exact path still needs a)
         if (tid == 0 && next >= 0 && !slow) load_raw(next, full);
-        // S = W B, one 64-column block per issuing thread, runs during the G copy
+        // update-only pass: S = W B, one 64-column block per issuing thread
+        // (a full pass has S in the chain below; those threads arrive)
         if (lid == 0 && warp >= 1 && warp <= N / 64) {
-            if (!slow) issue_S(warp - 1);
+            if (!slow && !full) issue_S(warp - 1);
             else tc::mbar_arrive(&sm.mb2);
         }
         if (!slow) {
             if (full) {
-                {   // masked G to its tile pair: lanes 0-15 of each sub-partition hold rows
+                {   // masked G^T to its tile pair: lanes 0-15 of each sub-partition hold
+                    // rows m; kept where t' >= m
                     float v[16];
                     tc::tmem_ld16(trow + Cols::G + 16 * q, v);
                     tc::tmem_ld_wait();
@@ -596,9 +609,9 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                         const int row = 16 * s4 + lid;
 #pragma unroll
                         for (int j = 0; j < 16; ++j)
-                            if (16 * q + j > row) v[j] = 0.f;
-                        st8(sm.Gh, sm.Gl, row, 16 * q, kK, v);
-                        st8(sm.Gh, sm.Gl, row, 16 * q + 8, kK, v + 8);
+                            if (16 * q + j < row) v[j] = 0.f;
+                        st8(sm.GTh, sm.GTl, row, 16 * q, kK, v);
+                        st8(sm.GTh, sm.GTl, row, 16 * q + 8, kK, v + 8);
                     }
                 }
                 tc::fence_proxy_async();
@@ -606,11 +619,14 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             }
             if (tid == 0) {
                 if (full) {
-                    // R += W G^T (three terms)
-                    bool fr = false;
-                    prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
-                    prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(Gl), kK, false, kK / 16, idR, fr);
-                    prod(tbase + Cols::R, NAJU_SA(Wl), kP, NAJU_SA(Gh), kK, false, kK / 16, idR, fr);
+                    // [S | R] += W_hi [B | G^T_hi] + W_lo [B | G^T_hi], R += W_hi G^T_lo
+                    // (S starts at zero, R holds X C^T)
+                    constexpr uint32_t idSR = tc::idesc_bf16(128, N + 64, false, true);
+                    constexpr uint32_t idR2 = tc::idesc_bf16(128, 64, false, true);
+                    bool f = false;
+                    prod(tbase + Cols::S, NAJU_SA(Wh), kP, NAJU_SA(Bs), kK, true, kK / 16, idSR, f);
+                    prod(tbase + Cols::S, NAJU_SA(Wl), kP, NAJU_SA(Bs), kK, true, kK / 16, idSR, f);
+                    prod(tbase + Cols::R, NAJU_SA(Wh), kP, NAJU_SA(GTl), kK, true, kK / 16, idR2, f);
                     tc::mma_commit(&sm.mb2);
                 } else {
                     tc::mbar_arrive(&sm.mb2);  // no R in an update-only pass
@@ -636,7 +652,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             tc::tmem_ld16(trow + Cols::SV + 64 + 16 * q, dh);
             tc::tmem_ld_wait();
             if constexpr (kStageY) {
-                __nv_bfloat16* ys = sm.Gh + 16 * q * kP + ch;  // [64 t][128 ch]
+                __nv_bfloat16* ys = sm.Wh + 16 * q * kP + ch;  // [64 t][128 ch] over W
 #pragma unroll
                 for (int kk = 0; kk < 16; ++kk)
                     ys[kk * kP] = __float2bfloat16_rn(fmaf(e[kk], r[kk], dh[kk]));
@@ -662,6 +678,9 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             load_bc(s0, full);
         }
         if (full) state_out(nullptr, true);
+#pragma unroll
+        for (int k = 0; k < NQ; k += 16) tc::tmem_st16(trow + Cols::S + NQ * q + k, kZero16);
+        tc::tmem_st_wait();
         tc::fence_proxy_async();
         sync();
         for (int k = s0; k < s1; ++k) {

@@ -77,9 +77,9 @@ void naju_testing_set_fwd_impl(int32_t impl);
  * sub-chunk kernel, 3 = tensor-core block-form kernel (0 for invalid dims). */
 int32_t naju_testing_fwd_impl(const void* dims);
 
-/* Backward implementation: 0 = automatic (tensor cores for bf16 activations
- * with d_state 64 or 128 and d_inner % 8 == 0: the block-form kernel for
- * d_state 64, the sub-chunk kernel for 128; CUDA cores otherwise),
+/* Backward implementation: 0 = automatic (the tensor-core block-form kernel
+ * for bf16 activations with d_state 64 or 128 and d_inner % 8 == 0, d_state
+ * 128 as two passes over 64-column state halves; CUDA cores otherwise),
  * 1 = always CUDA cores, 2 = the tensor-core sub-chunk kernel, 3 = the
  * block-form kernel (as automatic), where tensor cores apply. */
 void naju_testing_set_bwd_impl(int32_t impl);

@@ -25,7 +25,10 @@
 // The raw inputs of a block (u with its 3-token conv halo, a, b, z) arrive by
 // TMA into one shared buffer as soon as the previous block has read its own;
 // B and C arrive by TMA straight into their swizzled tiles once the previous
-// block's products are done.  Everything per (token, channel) runs on the
+// block's products are done.  With d_state 64 a block's y and fp32 checkpoint
+// leave through staging tiles and TMA stores (a warp's checkpoint rows are 256
+// bytes apart: direct stores would cost one memory transaction per lane).
+// Everything per (token, channel) runs on the
 // CUDA cores, 512 threads: warp w handles channels 32 (w % 4) + lane and
 // tokens [16 q, 16 q + 16) of the block, q = w / 4, and the state columns
 // [q N / 4, (q + 1) N / 4).
@@ -75,6 +78,8 @@ struct alignas(64) FkTmaps {
     CUtensorMap u, a, b, z;  // bf16 [Bt][L][d], plain boxes of 128 channels
     CUtensorMap B, C;        // bf16 [Bt][L][N], swizzled boxes of 64 columns
     CUtensorMap y;           // bf16 output [Bt][L][d] (bf16 outputs only), store boxes
+    CUtensorMap ck;          // fp32 checkpoints [Bt (nck + 1)][d][N], swizzled boxes of
+                             // 128 x 32 (d_state 64 only)
 };
 
 template <int N>
@@ -87,6 +92,12 @@ struct FkSmem {
     alignas(1024) __nv_bfloat16 Cs[kK * N], GTl[kK * kK];  // C: rows t, cols j
     alignas(1024) __nv_bfloat16 ru[(kK + 3) * kP];         // u of tokens tb - 3 ..
     alignas(128) __nv_bfloat16 ra[kK * kP], rb[kK * kP], rz[kK * kP];
+    // d_state 64: a block's fp32 checkpoint (two swizzled 128 x 32 boxes) and
+    // its bf16 y are staged here and leave by TMA stores after the next
+    // block's first barrier (d_state 128: y staged over the W tiles, the
+    // checkpoint stored directly)
+    alignas(1024) float ck[N == 64 ? kP * N : 32];
+    alignas(128) __nv_bfloat16 ys[N == 64 ? kK * kP : 64];
     float xq[4][kP], xe[4][kP];
     uint64_t mb_raw, mb_bc, mb0, mb2;
     uint32_t taddr;
@@ -130,9 +141,12 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     using Cols = FkCols<N>;
     using Sm = FkSmem<N>;
     constexpr int NQ = N / 4;  // state columns per thread
-    // bf16 outputs are staged in the G tiles' bytes (free once R is complete)
-    // and leave by one TMA store per block; fp32 outputs are stored directly
+    // bf16 outputs are staged in shared memory and leave by one TMA store per
+    // block; fp32 outputs are stored directly
     constexpr bool kStageY = std::is_same<Tout, __nv_bfloat16>::value;
+    // d_state 64: own staging buffers for y and the checkpoint (room in shared
+    // memory), so neither waits on the W tiles nor stores 256-byte-strided rows
+    constexpr bool kOwnStage = N == 64;
     static_assert(offsetof(Sm, GTh) == offsetof(Sm, Bs) + sizeof(Sm::Bs) &&
                       sizeof(Sm::Bs) == (size_t)(N / 64) * kK * 128,
                   "B and G^T are one MN-major operand: 64-column blocks kK * 128 bytes apart");
@@ -505,11 +519,11 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         tc::tmem_st_wait();
         sync();
     };
-    // X <- E_63 (X + S) on this thread's columns.
     // After a block: X <- E_63 (X + S) on this thread's columns (the exact
     // path has updated X already), then the new state to a global [d][N] row
-    // (dst != null) and to the X tile pair (tiles), from the same registers.
-    auto advance = [&](bool slow, float* dst, bool tiles) {
+    // (dst != null), to the checkpoint staging tile (stage; d_state 64) and to
+    // the X tile pair (tiles), from the same registers.
+    auto advance = [&](bool slow, float* dst, bool stage, bool tiles) {
 #pragma unroll
         for (int k = 0; k < NQ; k += 16) {
             float v[16], sv[16];
@@ -528,6 +542,18 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                     *reinterpret_cast<float4*>(dst + c * N + NQ * q + k + j) =
                         make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
             }
+            if (kOwnStage && stage) {
+                // box col / 32 of 128 rows x 128 bytes, row ch, 16-byte chunk
+                // (col % 32) / 4 XOR-permuted by ch % 8 (the TMA store's layout)
+#pragma unroll
+                for (int j = 0; j < 16; j += 4) {
+                    const int col = NQ * q + k + j;
+                    const uint32_t o = (uint32_t)((col >> 5) * kP * 128 + ch * 128 +
+                                                  ((((col & 31) >> 2) ^ (ch & 7)) << 4));
+                    *reinterpret_cast<float4*>(reinterpret_cast<char*>(sm.ck) + o) =
+                        make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                }
+            }
             if (tiles) {
                 st8(sm.Xh, sm.Xl, ch, NQ * q + k, kP, v);
                 st8(sm.Xh, sm.Xl, ch, NQ * q + k + 8, kP, v + 8);
@@ -541,46 +567,60 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
     // holds the state entering it; on exit the state in tensor memory is
     // updated and, for next >= 0, block next's loads are issued.
     float logP = 0.f;  // log of the decay product over an update-only pass
-    // The staged y of a block leaves after the next block's first barrier
-    // (no barrier of its own): the block whose y is pending, or -1.
-    int y_pending = -1;
-    auto store_y = [&]() {
-        if (kStageY && tid == 0 && y_pending >= 0) {
-            tma::store_3d(&tm.y, (int)c0, y_pending * kK, bb, sm.Wh);
-            tma::store_commit();
+    // The staged y of a block and its staged checkpoint leave after the next
+    // block's first barrier (no barrier of their own): the block whose y is
+    // pending and the checkpoint index pending, or -1.
+    int y_pending = -1, ck_pending = -1;
+    auto store_out = [&]() {
+        if (tid == 0) {
+            bool any = false;
+            if (kStageY && y_pending >= 0) {
+                tma::store_3d(&tm.y, (int)c0, y_pending * kK, bb, kOwnStage ? sm.ys : sm.Wh);
+                any = true;
+            }
+            if (kOwnStage && ck_pending >= 0) {
+                const int z = bb * (p.nck + 1) + ck_pending;
+#pragma unroll
+                for (int jb = 0; jb < N / 32; ++jb)
+                    tma::store_3d(&tm.ck, 32 * jb, (int)c0, z, sm.ck + jb * kP * 32);
+                any = true;
+            }
+            if (any) tma::store_commit();
         }
         y_pending = -1;
+        ck_pending = -1;
     };
     auto run_block = [&](int k, bool full, int next) {
         const int64_t tb = (int64_t)k * kK;
         const int nv = (int)min64((int64_t)kK, L - tb);
         constexpr uint32_t idR = tc::idesc_bf16(128, 64);
-        // G = C B^T (M = 64; B and C exact) goes to the tensor core as soon as
-        // this block's B and C have landed (thread 0 waits for them) and
-        // overlaps the CUDA-core work below.
-        if (tid == 0) {
+        wait_mb(&sm.mb_raw, ph_raw);
+        store_out();
+        // Once this block's B and C have landed, two threads on different
+        // warps issue the two products that overlap the CUDA-core work below
+        // (each MMA holds its issuing warp for some 50 cycles): thread 32
+        // G^T = B C^T (M = 64: rows m, columns t'; B and C exact), thread 0
+        // R = X C^T (the X tiles hold the state entering the block since the
+        // barrier above; R += W G^T follows on the same thread).  Thread 32
+        // also waits in an update-only pass, whose S reads B.
+        if (tid == 32 || (full && tid == 0)) {
             if (!timed_out && !tc::mbar_wait(&sm.mb_bc, ph_bc, kSpin)) timed_out = true;
-            if (full) {
-                // G^T = B C^T (M = 64: rows m, columns t')
-                bool fg = true;
-                prod(tbase + Cols::G, NAJU_SA(Bs), kK, NAJU_SA(Cs), kK, false, N / 16,
-                     tc::idesc_bf16(64, 64), fg);
-                tc::mma_commit(&sm.mb0);
-            }
         }
         ph_bc ^= 1u;
-        wait_mb(&sm.mb_raw, ph_raw);
-        store_y();
-        // R = X C^T: the X tiles (state entering the block) are in place since
-        // that barrier and C has landed; R += W G^T follows on the same thread
+        if (full && tid == 32) {
+            bool fg = true;
+            prod(tbase + Cols::G, NAJU_SA(Bs), kK, NAJU_SA(Cs), kK, false, N / 16,
+                 tc::idesc_bf16(64, 64), fg);
+            tc::mma_commit(&sm.mb0);
+        }
         if (full && tid == 0) {
             bool fr = true;
             prod(tbase + Cols::R, NAJU_SA(Xh), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
             prod(tbase + Cols::R, NAJU_SA(Xl), kP, NAJU_SA(Cs), kK, false, N / 16, idR, fr);
         }
-        // the previous block's y (staged over W) must have left before unpack
-        // rewrites W (the decays' barrier orders this wait)
-        if (kStageY && tid == 0) tma::store_wait_read();
+        // d_state 128: the previous block's y (staged over W) must have left
+        // before unpack rewrites W (the decays' barrier orders this wait)
+        if (!kOwnStage && kStageY && tid == 0) tma::store_wait_read();
         const bool slow = decays(nv);
         unpack(slow, full);
         tc::tmem_st_wait();
@@ -590,8 +630,6 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         } else {
             sync();
         }
-        // the raw buffer is read (the exact path still needs a)
-        if (tid == 0 && next >= 0 && !slow) load_raw(next, full);
         // update-only pass: S = W B, one 64-column block per issuing thread
         // (a full pass has S in the chain below; those threads arrive)
         if (lid == 0 && warp >= 1 && warp <= N / 64) {
@@ -631,6 +669,12 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                 } else {
                     tc::mbar_arrive(&sm.mb2);  // no R in an update-only pass
                 }
+                // the raw buffer is read: the next block's inputs load while
+                // the products run
+                if (next >= 0) load_raw(next, full);
+                // d_state 64: the staged y and checkpoint of the previous
+                // block have left before this block's are staged
+                if (kOwnStage) tma::store_wait_read();
             }
             wait_mb(&sm.mb2, ph2);
         } else {
@@ -638,6 +682,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             if (tid == 0) {
                 if (full) tc::mma_commit(&sm.mb2);
                 else tc::mbar_arrive(&sm.mb2);
+                if (kOwnStage) tma::store_wait_read();
             }
             wait_mb(&sm.mb2, ph2);
             exact_block(nv, full);
@@ -652,7 +697,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             tc::tmem_ld16(trow + Cols::SV + 64 + 16 * q, dh);
             tc::tmem_ld_wait();
             if constexpr (kStageY) {
-                __nv_bfloat16* ys = sm.Wh + 16 * q * kP + ch;  // [64 t][128 ch] over W
+                // [64 t][128 ch], d_state 128 over W
+                __nv_bfloat16* ys = (kOwnStage ? sm.ys : sm.Wh) + 16 * q * kP + ch;
 #pragma unroll
                 for (int kk = 0; kk < 16; ++kk)
                     ys[kk * kP] = __float2bfloat16_rn(fmaf(e[kk], r[kk], dh[kk]));
@@ -686,14 +732,20 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         for (int k = s0; k < s1; ++k) {
             const bool last = k + 1 == s1;
             const bool slow = run_block(k, full, last ? -1 : k + 1);
-            advance(slow, full && (!last || end_ckpt) ? ck_at(k + 1) : nullptr, full && !last);
-            // X tiles and the staged y -> async proxy; the next block's first
-            // barrier orders them before its MMAs and y's store
+            // checkpoint after every block but the last (and the last when
+            // end_ckpt; that one is stored directly, as a successor may read
+            // it in this launch)
+            const bool ck = full && (!last || end_ckpt);
+            const bool stage = kOwnStage && ck && !last;
+            advance(slow, ck && !stage ? ck_at(k + 1) : nullptr, stage, full && !last);
+            // X tiles and the staged y / checkpoint -> async proxy; the next
+            // block's first barrier orders them before its MMAs and stores
             tc::fence_proxy_async();
             if (full) y_pending = k;
+            if (stage) ck_pending = k + 1;
         }
         sync();
-        store_y();
+        store_out();
     };
     if (sbase & 1023u) {  // the swizzled tiles need 1024-byte alignment
         if (tid == 0) atomicOr(&p.hdr->status, 1 << NAJU_ERR_INVALID_ARG);
@@ -783,7 +835,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         if (last_group && p.x_final) state_out(p.x_final + (int64_t)bb * d * N, false);
     }
 #undef NAJU_SA
-    if (kStageY && tid == 0) tma::store_wait_all();
+    if (tid == 0) tma::store_wait_all();
     if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
     sync();
     if (warp == 0) tc::tmem_dealloc(tbase, Cols::ALLOC);
@@ -801,6 +853,9 @@ static cudaError_t launch_fwd_blk_t(const FwdParams& p, cudaStream_t st) {
               tma_encode_bf16_3d_sw128(&tm.C, p.C, p.Bt, p.L, N, kK);
     if (ok && std::is_same<Tout, __nv_bfloat16>::value)
         ok = tma_encode_bf16_3d(&tm.y, p.y, p.Bt, p.L, p.d, kK, kP);
+    if (ok && N == 64)
+        ok = p.ckpt != nullptr &&
+             tma_encode_f32_3d_sw128(&tm.ck, p.ckpt, p.Bt * (p.nck + 1), p.d, N, kP);
     if (!ok) return cudaErrorInvalidValue;
     const size_t smem = sizeof(FkSmem<N>);
     auto kern = scan_fwd_blk_kernel<Tout, N, CONV, PIECES>;

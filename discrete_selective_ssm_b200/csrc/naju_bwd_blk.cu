@@ -82,7 +82,10 @@ constexpr long long kSpin = 1LL << 24;
 // accumulator per thread, so each chain keeps its order): committing
 // threads per completion barrier.
 constexpr int kIss0 = 2;  // G (warp 0), P (warp 5); the exact path arrives for P
-constexpr int kIss2 = 5;  // dB (0), R (1), GB (2), carry (3), dC (4)
+constexpr int kIss2 = 3;  // R (1), GB (2), carry (3)
+constexpr int kIss3 = 2;  // dB (0), dC (4)
+// the thread that stores a block's staged gradients (not an MMA issuer)
+constexpr int kStoreTid = 7 * 32;
 
 // Tensor-memory columns (lane = channel unless stated).
 struct BkCols {
@@ -125,7 +128,7 @@ struct BkSmem {
     float dph[4][3][kP];          // first three dp of each quarter
     float dnext[2][3][kP];        // first three dp of the later block
     float red6[6][kP];            // per-channel parameter sums
-    uint64_t mb_in, mb_bc, mb_x, mb0, mb2, mb_e;
+    uint64_t mb_in, mb_bc, mb_x, mb0, mb2, mb3, mb_e;
     uint32_t taddr;
     int item, ok;
 };
@@ -233,7 +236,8 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tc::mbar_init(&sm.mb_bc, 1);
         tc::mbar_init(&sm.mb_x, 1);
         tc::mbar_init(&sm.mb0, kIss0);  // G and P
-        tc::mbar_init(&sm.mb2, kIss2);  // every chain of the block
+        tc::mbar_init(&sm.mb2, kIss2);  // the chains the epilogue reads
+        tc::mbar_init(&sm.mb3, kIss3);  // dB and dC
         tc::mbar_init(&sm.mb_e, 1);     // the early pass's carry
         tma::prefetch_map(&tm.X);
         tma::prefetch_map(&tm.u);
@@ -262,7 +266,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     const uint32_t sb4 = sbase >> 4;
     const bool aligned1k = (sbase & 1023u) == 0;  // the swizzled tiles need it
     if (!aligned1k && tid == 0) atomicOr(&p.hdr->status, 1 << NAJU_ERR_INVALID_ARG);
-    uint32_t ph_in = 0, ph_bc = 0, ph_x = 0, ph0 = 0, ph2 = 0, ph_e = 0;  // mbarrier parities
+    uint32_t ph_in = 0, ph_bc = 0, ph_x = 0, ph0 = 0, ph2 = 0, ph3 = 0, ph_e = 0;  // mbarrier parities
     bool timed_out = false;
 
     // This thread's two 16-byte chunks (columns [16 q, 16 q + 8) and
@@ -393,6 +397,20 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             if (has_b) tma::load_3d(rb, &tm.b, x, y, zb, &sm.mb_in);
         }
     };
+    // The same inputs of a full block in two steps: u (its own buffer) with
+    // the expected bytes of all five, then the four in region A.
+    auto load_raw_u = [&](int k) {
+        const uint32_t rows = kK * (2 + (has_z ? 1 : 0) + (has_b ? 1 : 0)) + (kK + 3);
+        tma::expect_tx(&sm.mb_in, rows * kP * 2u);
+        tma::load_3d(sm.ru, &tm.u, (int)c0, k * kK - 3, bb, &sm.mb_in);
+    };
+    auto load_raw_a = [&](int k) {
+        const int x = (int)c0, y = k * kK, zb = bb;
+        tma::load_3d(ra, &tm.a, x, y, zb, &sm.mb_in);
+        tma::load_3d(rdy, &tm.dy, x, y, zb, &sm.mb_in);
+        if (has_z) tma::load_3d(rz, &tm.z, x, y, zb, &sm.mb_in);
+        if (has_b) tma::load_3d(rb, &tm.b, x, y, zb, &sm.mb_in);
+    };
     // C (and B when full) of block k into their tiles (thread 0).
     auto load_bc = [&](int k, bool full) {
         tma::expect_tx(&sm.mb_bc, (uint32_t)(2 * kK * kN * (full ? 2 : 1)));
@@ -451,6 +469,9 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         tc::tmem_st16(trow + Cols::SV + 3 * 64 + 16 * q, qv);
         sm.xq[q][ch] = Qh;
         sm.xe[q][ch] = Eh;
+        // the previous block's staged gradients must have left the W / U bytes
+        // before unpack rewrites them (this barrier orders the wait)
+        if (kStage && tid == kStoreTid) tma::store_wait_read();
         const bool maybe = __syncthreads_or(!(Qh <= kQuarter)) != 0;
         float Qa = 1.f, Ea = 1.f;
         Qb = 1.f;
@@ -687,6 +708,9 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     };
     // Batch 2: R += W G^T, GB += U G (G transposed), dC^T = X^T U + B^T Pm^T
     // (lanes +0), dB^T = H'^T W + C^T Pm (lanes +16), all over the masked tiles.
+    // R, GB (and the carry) complete on mb2, which the epilogue waits for;
+    // dB and dC on mb3, waited for halfway through the epilogue, so these
+    // chains run beside its first pass.
     auto issue_b2 = [&]() {
         if (issuer == 1) {
             bool f = false;
@@ -707,7 +731,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                  tc::idesc_bf16(64, 64, true, false), f);
             prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Pl), false, kK / 16,
                  tc::idesc_bf16(64, 64, true, false), f);
-            tc::mma_commit(&sm.mb2);
+            tc::mma_commit(&sm.mb3);
         } else if (issuer == 0) {
             bool f = true;
             prod3(tbase + lane16 + Cols::BC, NAJU_SA(Hh), NAJU_SA(Hl), true, NAJU_SA(Wh),
@@ -716,7 +740,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                  tc::idesc_bf16(64, 64, true, true), f);
             prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Pl), true, kK / 16,
                  tc::idesc_bf16(64, 64, true, true), f);
-            tc::mma_commit(&sm.mb2);
+            tc::mma_commit(&sm.mb3);
         }
     };
     // G (lanes +0) and P (lanes +16) from tensor memory to their tile pairs,
@@ -944,7 +968,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
         // barrier (no barrier of their own): that block's first token, or -1.
         int out_pending = -1;
         auto store_out = [&]() {
-            if (kStage && tid == 0 && out_pending >= 0) {
+            if (kStage && tid == kStoreTid && out_pending >= 0) {
                 const int x = (int)c0, y = out_pending;
                 if (has_z) tma::store_3d(&tm.oz, x, y, bb, sm.Wh);
                 if (has_b) tma::store_3d(&tm.ob, x, y, bb, sm.Wl);
@@ -1003,8 +1027,6 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             issue_g();    // (the exact path waits for it too, to keep the barrier phases)
             float xr[16];
             read_x(xr);
-            // the staged gradients must have left the W / U bytes before unpack
-            if (kStage && tid == 0) tma::store_wait_read();
             const bool slow = decays(nv);  // (its barriers end the reads of the fp32 checkpoint)
             st8o(sm.Xh, sm.Xl, oc0, xr);
             st8o(sm.Xh, sm.Xl, oc1, xr + 8);
@@ -1035,12 +1057,20 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 exact_block(tb, nv);
             }
             // ------------------------------------------------ phase C
-            // Region A, the u buffer and the B, C tiles are free: the earlier
-            // block's inputs are requested.
-            if (tid == 0 && k > kb0) {
-                load_raw(k - 1, true);
-                load_bc(k - 1, true);
-            }
+            // The u buffer is free: the earlier block's u is requested.
+            if (tid == 0 && k > kb0) load_raw_u(k - 1);
+            // Halfway through the epilogue: dB and dC are complete, so region A,
+            // the B, C tiles and the X tiles (their operands) take the earlier
+            // block's inputs and checkpoint.
+            auto mid_barrier = [&]() {
+                if (!slow) wait_mb(&sm.mb3, ph3);
+                else __syncthreads();
+                if (tid == 0 && k > kb0) {
+                    load_raw_a(k - 1);
+                    load_bc(k - 1, true);
+                    load_x(k - 1);
+                }
+            };
             if constexpr (kImport) {
                 // the first pass's R and GB of this block (state columns 0..63)
                 const float* rp = p.rgb_part + ((int64_t)bb * L + tb + 16 * q) * d + c;
@@ -1094,8 +1124,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                     for (int qq = 0; qq < 4; ++qq) ts += sm.tailp[par][qq][ch];
                     p.tail_part[((int64_t)bb * p.nsub + k) * d + c] = ts;
                 }
-                __syncthreads();
-                if (tid == 0 && k > kb0) load_x(k - 1);
+                mid_barrier();
             } else {
             // The epilogue in four variants (b and z present or not), so no
             // per-token branch tests them.
@@ -1158,9 +1187,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
                 sm.dph[q][0][ch] = dpf0;
                 sm.dph[q][1][ch] = dpf1;
                 sm.dph[q][2][ch] = dpf2;
-                __syncthreads();
-                // the X tiles and the W, U tiles are read: the next checkpoint may land
-                if (tid == 0 && k > kb0) load_x(k - 1);
+                mid_barrier();
                 float base = 0.f;  // dL over the later quarters, plus the tail
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
@@ -1317,7 +1344,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     }
 #undef NAJU_SA
 
-    if (kStage && tid == 0) tma::store_wait_all();
+    if (kStage && tid == kStoreTid) tma::store_wait_all();
     if (timed_out) atomicOr(&p.hdr->status, 1 << NAJU_ERR_TIMEOUT);
     sync();
     if (warp == 0) tc::tmem_dealloc(tbase, 512);

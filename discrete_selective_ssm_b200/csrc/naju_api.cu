@@ -227,7 +227,8 @@ Layout layout(const naju_dims* dm) {
     l.off_carry = off;
     off = up256(off + sizeof(float) * (size_t)groups_n * Bt * d * N);
     l.off_dbc = off;
-    off = up256(off + sizeof(float) * (size_t)parts_n * Bt * L * 2 * N);
+    // (the block backward's accumulator pads the tokens to a multiple of four)
+    off = up256(off + sizeof(float) * (size_t)parts_n * Bt * ((L + 3) / 4 * 4) * 2 * N);
     l.off_chan = off;
     off = up256(off + sizeof(float) * (size_t)Bt * groups_n * d * 8);
     l.off_edge = off;

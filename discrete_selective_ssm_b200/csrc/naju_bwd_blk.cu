@@ -150,6 +150,20 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ void red_add(float* p, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
+// Four consecutive floats (p 16-byte aligned) in one reduction.
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b),
+                 "f"(c), "f"(d)
+                 : "memory");
+}
+// The dB / dC accumulator holds tokens in chunks of four, innermost:
+// [Bt][ceil(L / 4)][2][N][4] (slot 0 dB, 1 dC), so one thread's four
+// consecutive tokens of a state column are one 16-byte reduction.
+__host__ __device__ __forceinline__ int64_t dbc_index(int64_t b, int64_t t, int slot, int64_t col,
+                                                       int64_t L, int64_t N) {
+    const int64_t L4 = (L + 3) >> 2;
+    return (((b * L4 + (t >> 2)) * 2 + slot) * N + col) * 4 + (t & 3);
+}
 // hi = bf16(a, b) (round to nearest), lo = bf16 of the remainders.
 __device__ __forceinline__ void split2(float a, float b, uint32_t& hi, uint32_t& lo) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -783,7 +797,6 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 #pragma unroll
         for (int j = 0; j < 16; j += 4) ld4o(sm.Xh, sm.Xl, (j < 8 ? oc0 : oc1) + (j & 4) * 2, x + j);
         __syncthreads();
-        float* acc = p.dBCp + (int64_t)bb * L * 2 * NS + JH;
         for (int tt = 0; tt < nv; ++tt) {
             const float f = f_at(tt), v = ld1(sm.Wh, sm.Wl, ch, tt), sdy = ld1(sm.Uh, sm.Ul, ch, tt);
             float rp = 0.f;
@@ -796,7 +809,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const float r = warp_sum(sdy * x[j]);
-                if (lid == 0) red_add(acc + (tb + tt) * 2 * NS + NS + 16 * q + j, r);
+                if (lid == 0) red_add(p.dBCp + dbc_index(bb, tb + tt, 1, JH + 16 * q + j, L, NS), r);
             }
         }
         for (int tt = nv - 1; tt >= 0; --tt) {
@@ -811,7 +824,7 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const float r = warp_sum(v * hx[j]);
-                if (lid == 0) red_add(acc + (tb + tt) * 2 * NS + 16 * q + j, r);
+                if (lid == 0) red_add(p.dBCp + dbc_index(bb, tb + tt, 0, JH + 16 * q + j, L, NS), r);
                 hx[j] *= f;
             }
         }
@@ -1296,18 +1309,21 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             }
             }  // (gradients of the per-token inputs)
             // dC^T (lanes +0) and dB^T (lanes +16): this warp's lanes, columns
-            // [16 q, 16 q + 16), added into the accumulator
+            // [16 q, 16 q + 16), added into the accumulator four tokens at a
+            // time (the tokens of a chunk past the end land in its padding)
             if (!slow) {
                 float v[16];
                 tc::tmem_ld16(trow + Cols::BC + 16 * q, v);
                 tc::tmem_ld_wait();
                 const int j = 16 * s4 + (lid & 15);
                 const int slot = lid < 16 ? 1 : 0;  // slot 0 dB, 1 dC
-                float* acc = p.dBCp + ((int64_t)bb * L + tb + 16 * q) * 2 * NS + slot * NS + JH + j;
+                float* acc = p.dBCp + dbc_index(bb, tb + 16 * q, slot, JH + j, L, NS);
                 const int nvq = nv - 16 * q;
 #pragma unroll
-                for (int k2 = 0; k2 < 16; ++k2)
-                    if (k2 < nvq) red_add(acc + k2 * 2 * NS, v[k2]);
+                for (int i = 0; i < 4; ++i)
+                    if (4 * i < nvq)
+                        red_add4(acc + (int64_t)i * 2 * NS * 4, v[4 * i], v[4 * i + 1], v[4 * i + 2],
+                                 v[4 * i + 3]);
             }
             // staged outputs -> async proxy; the next block's first barrier
             // orders them (and this block's reads of tiles and tensor memory)
@@ -1350,20 +1366,27 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     if (warp == 0) tc::tmem_dealloc(tbase, 512);
 }
 
-// dB, dC from the fp32 accumulator [Bt][L][2][N] (slot 0 dB, 1 dC).
+// dB, dC from the fp32 accumulator [Bt][ceil(L / 4)][2][N][4]: one thread per
+// (batch, four-token chunk, state column), consecutive threads on consecutive
+// columns (16-byte loads, coalesced stores).
 template <typename Tout>
-__global__ void finish_dBC_kernel(const float* __restrict__ acc, int64_t BtL, int64_t N,
+__global__ void finish_dBC_kernel(const float* __restrict__ acc, int64_t Bt, int64_t L, int64_t N,
                                   Tout* __restrict__ dB, Tout* __restrict__ dC) {
-    const int64_t n4 = BtL * N / 4;
-    for (int64_t i4 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i4 < n4;
-         i4 += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t i = i4 * 4, row = i / N, j = i % N;
-        const float4 b4 = *reinterpret_cast<const float4*>(acc + row * 2 * N + j);
-        const float4 c4 = *reinterpret_cast<const float4*>(acc + row * 2 * N + N + j);
-        dB[i] = from_f<Tout>(b4.x); dB[i + 1] = from_f<Tout>(b4.y);
-        dB[i + 2] = from_f<Tout>(b4.z); dB[i + 3] = from_f<Tout>(b4.w);
-        dC[i] = from_f<Tout>(c4.x); dC[i + 1] = from_f<Tout>(c4.y);
-        dC[i + 2] = from_f<Tout>(c4.z); dC[i + 3] = from_f<Tout>(c4.w);
+    const int64_t L4 = (L + 3) >> 2, n = Bt * L4 * N;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t j = i % N, row = i / N, b = row / L4, t0 = (row % L4) * 4;
+        const float4 b4 = *reinterpret_cast<const float4*>(acc + (row * 2 * N + j) * 4);
+        const float4 c4 = *reinterpret_cast<const float4*>(acc + (row * 2 * N + N + j) * 4);
+        const float bv[4] = {b4.x, b4.y, b4.z, b4.w}, cv[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+            if (t0 + tt < L) {
+                const int64_t o = (b * L + t0 + tt) * N + j;
+                dB[o] = from_f<Tout>(bv[tt]);
+                dC[o] = from_f<Tout>(cv[tt]);
+            }
+        }
     }
 }
 
@@ -1422,7 +1445,8 @@ static cudaError_t launch_blk_mode(const BwdParams& p, int out_dtype, cudaStream
 
 cudaError_t launch_scan_bwd_blk(const BwdParams& p, int out_dtype, cudaStream_t st) {
     // the dB / dC accumulator starts at zero
-    cudaError_t e = cudaMemsetAsync(p.dBCp, 0, sizeof(float) * (size_t)p.Bt * p.L * 2 * p.N, st);
+    cudaError_t e = cudaMemsetAsync(
+        p.dBCp, 0, sizeof(float) * (size_t)p.Bt * ((p.L + 3) / 4 * 4) * 2 * p.N, st);
     if (e != cudaSuccess) return e;
     if (p.N == kN) return launch_blk_mode<0>(p, out_dtype, st);
     // d_state 128: state columns 0..63, then 64..127 with fresh tickets and flags
@@ -1436,13 +1460,12 @@ cudaError_t launch_scan_bwd_blk(const BwdParams& p, int out_dtype, cudaStream_t 
 
 cudaError_t launch_finish_dBC(const BwdParams& p, int out_dtype, void* dB, void* dC,
                               cudaStream_t st) {
-    const int64_t BtL = p.Bt * p.L;
     if (out_dtype == NAJU_BF16)
         finish_dBC_kernel<__nv_bfloat16><<<592, 256, 0, st>>>(
-            p.dBCp, BtL, p.N, static_cast<__nv_bfloat16*>(dB), static_cast<__nv_bfloat16*>(dC));
+            p.dBCp, p.Bt, p.L, p.N, static_cast<__nv_bfloat16*>(dB), static_cast<__nv_bfloat16*>(dC));
     else
-        finish_dBC_kernel<float><<<592, 256, 0, st>>>(p.dBCp, BtL, p.N, static_cast<float*>(dB),
-                                                       static_cast<float*>(dC));
+        finish_dBC_kernel<float><<<592, 256, 0, st>>>(p.dBCp, p.Bt, p.L, p.N,
+                                                       static_cast<float*>(dB), static_cast<float*>(dC));
     return cudaGetLastError();
 }
 

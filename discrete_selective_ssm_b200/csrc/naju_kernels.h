@@ -67,6 +67,7 @@ struct BwdParams {
     float* carry;          // [ngroups][Bt][d][N] adjoint carries between groups
     int* flags;            // [ngroups][Bt][ntiles]
     float* dBCp;           // [nclus][Bt][L][2][N] partial dB, dC over channel clusters
+                           // (block backward: one accumulator [Bt][ceil(L/4)][2][N][4])
     float* chan_part;      // [Bt*ngroups][d][8] partial dD, dconv_w[4], dconv_b
     float* conv_edge;      // [Bt][ngroups][2][3][d]: first 3 dp / last 3 partial du
     float* rgb_part;       // block backward, d_state 128: [2][Bt][L][d] partial R, GB of
@@ -109,7 +110,7 @@ bool fwd_blk_supported(int dtype, int64_t N, int64_t d, int T_ck);
 cudaError_t launch_scan_fwd_blk(const FwdParams& p, int out_dtype, cudaStream_t st);
 // Block-form tensor-core backward (bf16 activations, d_state 64 or 128; 128 as
 // two passes over 64-column state halves through p.rgb_part / p.tail_part):
-// dB / dC go into an fp32 accumulator [Bt][L][2][N] at p.dBCp (zeroed by the
+// dB / dC go into an fp32 accumulator [Bt][ceil(L/4)][2][N][4] at p.dBCp (zeroed by the
 // launch); launch_bwd_reductions_acc then finishes dB, dC and the per-channel
 // sums.
 bool bwd_blk_supported(int dtype, int64_t N, int64_t d);

@@ -67,7 +67,7 @@ struct FkCols {
     static constexpr uint32_t X = 0;             // state [ch][j]
     static constexpr uint32_t S = N;             // W B   [ch][j]
     static constexpr uint32_t R = 2 * N;         // R     [ch][t]
-    static constexpr uint32_t G = 2 * N + 64;    // G (M = 64)
+    static constexpr uint32_t G = 2 * N + 64;    // G^T (M = 64): t' < 32 at lanes +0, >= 32 at +16
     static constexpr uint32_t SV = 2 * N + 128;  // s E SiLU(z), D h SiLU(z)  [ch][t] x 2
     static constexpr uint32_t USED = 2 * N + 256;
     static constexpr uint32_t ALLOC = USED <= 256 ? 256 : 512;
@@ -599,7 +599,9 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         // Once this block's B and C have landed, two threads on different
         // warps issue the two products that overlap the CUDA-core work below
         // (each MMA holds its issuing warp for some 50 cycles): thread 32
-        // G^T = B C^T (M = 64: rows m, columns t'; B and C exact), thread 0
+        // G^T = B C^T (M = 64: rows m, columns t'; B and C exact) as two
+        // halves of 32 columns t' in the two lane halves of the same tensor
+        // memory columns, so all lanes share the copy below; thread 0
         // R = X C^T (the X tiles hold the state entering the block since the
         // barrier above; R += W G^T follows on the same thread).  Thread 32
         // also waits in an update-only pass, whose S reads B.
@@ -608,9 +610,12 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         }
         ph_bc ^= 1u;
         if (full && tid == 32) {
+            constexpr uint32_t idG = tc::idesc_bf16(64, 32);
             bool fg = true;
-            prod(tbase + Cols::G, NAJU_SA(Bs), kK, NAJU_SA(Cs), kK, false, N / 16,
-                 tc::idesc_bf16(64, 64), fg);
+            prod(tbase + Cols::G, NAJU_SA(Bs), kK, NAJU_SA(Cs), kK, false, N / 16, idG, fg);
+            fg = true;  // rows t' 32.. of C: four 8-row groups (4096 bytes) on
+            prod(tbase + (16u << 16) + Cols::G, NAJU_SA(Bs), kK, NAJU_SA(Cs) + 4096 / 16, kK, false,
+                 N / 16, idG, fg);
             tc::mma_commit(&sm.mb0);
         }
         if (full && tid == 0) {
@@ -638,19 +643,17 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
         }
         if (!slow) {
             if (full) {
-                {   // masked G^T to its tile pair: lanes 0-15 of each sub-partition hold
-                    // rows m; kept where t' >= m
-                    float v[16];
-                    tc::tmem_ld16(trow + Cols::G + 16 * q, v);
+                {   // masked G^T to its tile pair, kept where t' >= m: lane l of
+                    // sub-partition s4 holds row m = 16 s4 + l % 16, columns
+                    // t' = 32 (l / 16) + [0, 32); this warp copies 8 of them
+                    float v[8];
+                    tc::tmem_ld8(trow + Cols::G + 8 * q, v);
                     tc::tmem_ld_wait();
-                    if (lid < 16) {
-                        const int row = 16 * s4 + lid;
+                    const int row = 16 * s4 + (lid & 15), t0 = 32 * (lid >> 4) + 8 * q;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            if (16 * q + j < row) v[j] = 0.f;
-                        st8(sm.GTh, sm.GTl, row, 16 * q, kK, v);
-                        st8(sm.GTh, sm.GTl, row, 16 * q + 8, kK, v + 8);
-                    }
+                    for (int j = 0; j < 8; ++j)
+                        if (t0 + j < row) v[j] = 0.f;
+                    st8(sm.GTh, sm.GTl, row, t0, kK, v);
                 }
                 tc::fence_proxy_async();
                 sync();

@@ -74,6 +74,19 @@ __device__ __forceinline__ float exp2a_(float v) {
 }
 __device__ __forceinline__ float expa_(float v) { return exp2a_(v * 1.4426950408889634f); }
 __device__ __forceinline__ float sigmoidx_(float v) { return rcpa_(1.0f + expa_(-v)); }
+// tanh on the MUFU unit (PTX tanh.approx.f32: relative error about 2^-11) and
+// SiLU through it, v sigma(v) = h + h tanh(h) with h = v / 2 (absolute error
+// at most about 2^-12 |v|).  Used only where the result is rounded to bf16
+// right after (the forward's output gate with bf16 outputs).
+__device__ __forceinline__ float tanha_(float v) {
+    float r;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+__device__ __forceinline__ float siluta_(float v) {
+    const float h = 0.5f * v;
+    return fmaf(h, tanha_(h), h);
+}
 __device__ __forceinline__ float silua_(float v) { return v * sigmoida_(v); }
 __device__ __forceinline__ float sigmoidf_(float v) { return rcpf_(1.0f + __expf(-v)); }
 __device__ __forceinline__ float siluf_(float v) { return v * sigmoidf_(v); }

@@ -367,8 +367,11 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                 // SiLU(conv), sigma(b) and SiLU(z) share one reciprocal:
                 // q = 1 + e^{-v} with e^{-v} capped at 2^36 (the product stays
                 // finite; a sigmoid below 1.5e-11 moves by at most that much),
-                // r = 1 / (qp qb qz), sigma_p = r qb qz and so on.
-                float pv[4], qp[4], qb[4], qz[4], zv[4];
+                // r = 1 / (qp qb qz), sigma_p = r qb qz and so on.  With bf16
+                // outputs SiLU(z), which only scales y, comes from the MUFU tanh
+                // instead (error at most about 2^-12 |z|, below y's own bf16
+                // rounding) and leaves the reciprocal to the other two.
+                float pv[4], qp[4], qb[4], qz[4], zv[4], gz[4];
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
                     const float u3 = bf2f(rup[(kb + k4 + 3) * kP]);
@@ -395,7 +398,12 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         zv[k4] = bf2f(rzp[(kb + k4) * kP]);
-                        qz[k4] = 1.f + exp2a_(fminf(-kLog2e * zv[k4], 36.f));
+                        if (kStageY) {
+                            gz[k4] = siluta_(zv[k4]);
+                            qz[k4] = 1.f;
+                        } else {
+                            qz[k4] = 1.f + exp2a_(fminf(-kLog2e * zv[k4], 36.f));
+                        }
                     }
                 } else {
 #pragma unroll
@@ -418,7 +426,7 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                         const float qq = qv[kb + k4];
                         iw[k4] = qq < 3.0e38f ? (qq - 1.f) * fv[kb + k4] : 1.f;
                     }
-                    gg[k4] = (full && has_z) ? zv[k4] * (rp * qb[k4]) : 1.f;
+                    gg[k4] = (full && has_z) ? (kStageY ? gz[k4] : zv[k4] * (rp * qb[k4])) : 1.f;
                 }
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {

@@ -326,7 +326,8 @@ namespace naju {
 // the forward's shared-reciprocal form for three arguments (x, x / 2, -x):
 // q_i = 1 + min(e^{-v_i}, 2^36), r = 1 / (q0 q1 q2), sigma(x) = r q1 q2.
 __global__ void fast_math_kernel(const float* __restrict__ x, float* __restrict__ ex,
-                                 float* __restrict__ sig, float* __restrict__ sig3, int64_t n) {
+                                 float* __restrict__ sig, float* __restrict__ sig3,
+                                 float* __restrict__ silut, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x) {
         const float v = x[i];
@@ -338,16 +339,17 @@ __global__ void fast_math_kernel(const float* __restrict__ x, float* __restrict_
         const float q2 = 1.f + exp2a_(fminf(kL2e * v, 36.f));
         const float r = rcpa_(q0 * (q1 * q2));
         sig3[i] = r * (q1 * q2);
+        silut[i] = siluta_(v);
     }
 }
 }  // namespace naju
 
 extern "C" naju_status naju_testing_fast_math(const float* x, float* ex, float* sig, float* sig3,
-                                              int64_t n, void* stream) {
-    if (!x || !ex || !sig || !sig3 || n < 0) return NAJU_ERR_INVALID_ARG;
+                                              float* silut, int64_t n, void* stream) {
+    if (!x || !ex || !sig || !sig3 || !silut || n < 0) return NAJU_ERR_INVALID_ARG;
     if (n == 0) return NAJU_OK;
     const int blocks = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
     naju::fast_math_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, ex, sig, sig3,
-                                                                                n);
+                                                                                silut, n);
     return cudaGetLastError() == cudaSuccess ? NAJU_OK : NAJU_ERR_CUDA;
 }

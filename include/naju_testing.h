@@ -126,11 +126,13 @@ naju_status naju_testing_tc_mma_gen(int32_t M, int32_t N, int32_t K, int32_t a_m
 /* The block-form kernels' fast exponential and sigmoids, for n device fp32
  * inputs x: ex = e^x computed as 2^(x log2 e) with the MUFU base-2 unit (PTX
  * ex2.approx.ftz; results below the normal range flush to zero), sig =
- * 1 / (1 + e^{-x}) with the approximate reciprocal, and sig3 = the forward's
+ * 1 / (1 + e^{-x}) with the approximate reciprocal, sig3 = the forward's
  * shared-reciprocal form of sigma(x) taken together with sigma(x / 2) and
- * sigma(-x) (each e^{-v} capped at 2^36).  Device pointers, n >= 0. */
-naju_status naju_testing_fast_math(const float* x, float* ex, float* sig, float* sig3, int64_t n,
-                                   void* stream);
+ * sigma(-x) (each e^{-v} capped at 2^36), and silut = SiLU(x) = x sigma(x) as
+ * h + h tanh(h), h = x / 2, with the MUFU tanh (PTX tanh.approx.f32; the
+ * forward's output gate with bf16 outputs).  Device pointers, n >= 0. */
+naju_status naju_testing_fast_math(const float* x, float* ex, float* sig, float* sig3,
+                                   float* silut, int64_t n, void* stream);
 
 #ifdef __cplusplus
 }

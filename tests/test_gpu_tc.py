@@ -123,10 +123,13 @@ def test_fast_math_against_fp64_and_cuda_expf():
     of at most 88 * 1.4427 * 2^-24 * ln 2 < 5.3e-6 in e^x for |x| <= 88, plus
     the base-2 unit's few ulp; results below the normal range (x < -87.33)
     may flush to zero.  sigma(x) then errs by < 2e-6 absolute; the capped
-    form also moves sigma(x) for x < -24.95 to 1 / (1 + 2^36) < 1.46e-11."""
+    form also moves sigma(x) for x < -24.95 to 1 / (1 + 2^36) < 1.46e-11.
+    The output gate's SiLU(x) = h + h tanh(h), h = x / 2, on the MUFU tanh
+    (PTX tanh.approx.f32, relative error below 2^-10.98): an error of at most
+    |h| |tanh(h)| 2^-10.98 < 2.5e-4 |x| plus the fp32 rounding of h + h t."""
     L = naju.lib()
     f = L.naju_testing_fast_math
-    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_void_p]
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int64, ctypes.c_void_p]
     f.restype = ctypes.c_int
     g = torch.Generator().manual_seed(7)
     x = torch.cat([torch.linspace(-100.0, 100.0, 200001), 5.0 * torch.randn(100000, generator=g),
@@ -136,8 +139,10 @@ def test_fast_math_against_fp64_and_cuda_expf():
     ex = torch.empty_like(dx)
     sig = torch.empty_like(dx)
     sig3 = torch.empty_like(dx)
+    silut = torch.empty_like(dx)
     rc = f(ctypes.c_void_p(dx.data_ptr()), ctypes.c_void_p(ex.data_ptr()),
-           ctypes.c_void_p(sig.data_ptr()), ctypes.c_void_p(sig3.data_ptr()), x.numel(),
+           ctypes.c_void_p(sig.data_ptr()), ctypes.c_void_p(sig3.data_ptr()),
+           ctypes.c_void_p(silut.data_ptr()), x.numel(),
            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert rc == 0
     cuda_exp = torch.exp(dx).cpu().double().numpy()  # CUDA's expf
@@ -162,3 +167,8 @@ def test_fast_math_against_fp64_and_cuda_expf():
     unc = xd > -24.9
     assert np.max(np.abs(s3[unc] - s64[unc]) / s64[unc]) < 2e-5
     assert np.max(np.abs(s3[~unc] - s64[~unc])) < 1.46e-11
+    st = silut.cpu().double().numpy()
+    silu64 = xd * s64
+    err_t = np.abs(st - silu64)
+    assert np.all(err_t <= 2.5e-4 * np.abs(xd) + 2e-7 * np.abs(silu64) + 1e-30), \
+        (err_t / np.maximum(np.abs(xd), 1e-30)).max()

@@ -233,6 +233,16 @@ def run_decode(args, w, rank, world, local):
     for k in range(args.warmup):
         step(k)
     torch.cuda.synchronize()
+    # The K timed steps are captured once in a CUDA graph and replayed: one
+    # launch per step from Python leaves the GPU waiting on the host between
+    # steps (a step is ~50 us of device work).  The first replay uploads the
+    # graph and is not timed.
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for k in range(args.steps):
+            step(args.warmup + k)
+    graph.replay()
+    torch.cuda.synchronize()
     clk = ClockSampler(local)
     clk.start()
     time.sleep(0.3)
@@ -241,8 +251,7 @@ def run_decode(args, w, rank, world, local):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for k in range(args.steps):
-        step(args.warmup + k)
+    graph.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
@@ -297,7 +306,7 @@ def run_decode(args, w, rank, world, local):
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "d_inner": w.d_inner,
                        "d_state": w.d_state, "conv_state": True, "gating": True,
-                       "parallelism": f"replicas{world}",
+                       "parallelism": f"replicas{world}", "cuda_graph": True,
                        "l2": "state (134 MB) and input pool larger than L2 (no flush)"},
             "roofline": {"bound": "hbm", "kernel": "naju_scan_step_conv: step_kernel",
                          "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -128,6 +128,14 @@ __device__ __forceinline__ void st8(__nv_bfloat16* th, __nv_bfloat16* tl, int ro
     *reinterpret_cast<uint4*>(reinterpret_cast<char*>(th) + o) = h;
     *reinterpret_cast<uint4*>(reinterpret_cast<char*>(tl) + o) = l;
 }
+// Eight floats to global memory in one 32-byte store (p 32-byte aligned):
+// a warp's state rows are N * 4 bytes apart, so each lane's store is a
+// transaction of its own, and whole 32-byte sectors halve their count.
+__device__ __forceinline__ void st_v8(float* p, const float* v) {
+    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(v[0]),
+                 "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+                 : "memory");
+}
 __device__ __forceinline__ float ld1(const __nv_bfloat16* t, int row, int col, int R) {
     return bf2f(*reinterpret_cast<const __nv_bfloat16*>(reinterpret_cast<const char*>(t) +
                                                           tc::bf_offset_w(row, col, R)));
@@ -284,10 +292,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
             tc::tmem_ld16(trow + Cols::X + NQ * q + k, v);
             tc::tmem_ld_wait();
             if (dst && cvalid) {
-#pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                    *reinterpret_cast<float4*>(dst + c * N + NQ * q + k + j) =
-                        make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                st_v8(dst + c * N + NQ * q + k, v);
+                st_v8(dst + c * N + NQ * q + k + 8, v + 8);
             }
             if (tiles) {
                 st8(sm.Xh, sm.Xl, ch, NQ * q + k, kP, v);
@@ -545,10 +551,8 @@ scan_fwd_blk_kernel(const FwdParams p, const __grid_constant__ FkTmaps tm) {
                 tc::tmem_st16(trow + Cols::S + NQ * q + k, kZero16);  // S accumulates from zero
             }
             if (dst && cvalid) {
-#pragma unroll
-                for (int j = 0; j < 16; j += 4)
-                    *reinterpret_cast<float4*>(dst + c * N + NQ * q + k + j) =
-                        make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                st_v8(dst + c * N + NQ * q + k, v);
+                st_v8(dst + c * N + NQ * q + k + 8, v + 8);
             }
             if (kOwnStage && stage) {
                 // box col / 32 of 128 rows x 128 bytes, row ch, 16-byte chunk

@@ -83,7 +83,7 @@ constexpr long long kSpin = 1LL << 24;
 // threads per completion barrier.
 constexpr int kIss0 = 2;  // G (warp 0), P (warp 5); the exact path arrives for P
 constexpr int kIss2 = 3;  // R (1), GB (2), carry (3)
-constexpr int kIss3 = 2;  // dB (0), dC (4)
+constexpr int kIss3 = 2;  // dC (1), dB (2)
 // the thread that stores a block's staged gradients (not an MMA issuer)
 constexpr int kStoreTid = 7 * 32;
 
@@ -723,21 +723,17 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
     // Batch 2: R += W G^T, GB += U G (G transposed), dC^T = X^T U + B^T Pm^T
     // (lanes +0), dB^T = H'^T W + C^T Pm (lanes +16), all over the masked tiles.
     // R, GB (and the carry) complete on mb2, which the epilogue waits for;
-    // dB and dC on mb3, waited for halfway through the epilogue, so these
-    // chains run beside its first pass.
+    // dC and dB on mb3, waited for halfway through the epilogue, so these
+    // chains run beside its first pass.  dC follows R on one thread and dB
+    // follows GB on another (two issuing threads measured best: the tensor
+    // core then takes R and GB first).
     auto issue_b2 = [&]() {
         if (issuer == 1) {
             bool f = false;
             prod3(tbase + Cols::R, NAJU_SA(Wh), NAJU_SA(Wl), false, NAJU_SA(Gh), NAJU_SA(Gl), false,
                   kK / 16, tc::idesc_bf16(128, 64), f);
             tc::mma_commit(&sm.mb2);
-        } else if (issuer == 2) {
-            bool f = false;
-            prod3(tbase + Cols::GB, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Gh), NAJU_SA(Gl), true,
-                  kK / 16, tc::idesc_bf16(128, 64, false, true), f);
-            tc::mma_commit(&sm.mb2);
-        } else if (issuer == 4) {
-            bool f = true;
+            f = true;
             prod3(tbase + Cols::BC, NAJU_SA(Xh), NAJU_SA(Xl), true, NAJU_SA(Uh), NAJU_SA(Ul), true,
                   kP / 16, tc::idesc_bf16(64, 64, true, true), f);
             // B^T Pm^T: B (rows m = K) against Pm (rows t, K = m): hi and lo of Pm
@@ -746,8 +742,12 @@ scan_bwd_blk_kernel(const BwdParams p, const __grid_constant__ BkTmaps tm) {
             prod(tbase + Cols::BC, NAJU_SA(Bs), true, NAJU_SA(Pl), false, kK / 16,
                  tc::idesc_bf16(64, 64, true, false), f);
             tc::mma_commit(&sm.mb3);
-        } else if (issuer == 0) {
-            bool f = true;
+        } else if (issuer == 2) {
+            bool f = false;
+            prod3(tbase + Cols::GB, NAJU_SA(Uh), NAJU_SA(Ul), false, NAJU_SA(Gh), NAJU_SA(Gl), true,
+                  kK / 16, tc::idesc_bf16(128, 64, false, true), f);
+            tc::mma_commit(&sm.mb2);
+            f = true;
             prod3(tbase + lane16 + Cols::BC, NAJU_SA(Hh), NAJU_SA(Hl), true, NAJU_SA(Wh),
                   NAJU_SA(Wl), true, kP / 16, tc::idesc_bf16(64, 64, true, true), f);
             prod(tbase + lane16 + Cols::BC, NAJU_SA(Cs), true, NAJU_SA(Ph), true, kK / 16,

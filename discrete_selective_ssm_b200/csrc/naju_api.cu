@@ -93,9 +93,14 @@ bool use_bwd_blk(const naju_dims* dm) {
 // decides the time.  Sequence-group count for `units` blocks' worth of work
 // per group over `nseg` 64-token segments: the g (at most 16) with the least
 // modelled time: waves of units * G blocks, G the groups after rounding to
-// whole segments, each over ceil(nseg / g) segments, plus 17 % for the early
-// (backward) or update-only (forward) pass that all but the last group run.
-int tc_groups(int64_t units, int nseg, int sms) {
+// whole segments, each over ceil(nseg / g) segments, plus `extra` (a share of
+// a full pass) for the early (backward) or update-only (forward) pass that
+// all but the last group run.  Fitted on sweeps of the group count: 0.17 for
+// the backward's early pass, 0.7 for the forward's update-only pass (it runs
+// most of the forward's per-token work); for 8 x 2048 x 1536 x 64 these pick
+// 3 backward groups and 1 forward group, for 2 x 8192 x 2048 x 128 9 and 9.
+constexpr double kBwdEarlyPass = 0.17, kFwdUpdatePass = 0.7;
+int tc_groups(int64_t units, int nseg, int sms, double extra) {
     if (units >= sms) return 1;  // a wave or more: piece mode, or whole waves already
     int best = 1;
     double best_cost = 1e30;
@@ -103,7 +108,7 @@ int tc_groups(int64_t units, int nseg, int sms) {
         const int64_t per = cdiv(nseg, g), groups = cdiv(nseg, per);
         const double waves = (double)cdiv(units * groups, sms);
         const double cost =
-            waves * (double)per / nseg * (1.0 + 0.17 * (double)(groups - 1) / groups);
+            waves * (double)per / nseg * (1.0 + extra * (double)(groups - 1) / groups);
         if (cost < best_cost - 1e-12) {
             best_cost = cost;
             best = g;
@@ -154,7 +159,7 @@ BwdTiling bwd_tiling(const naju_dims* dm, int nsub, bool tc, int sms) {
     if (gb <= 0) {
         const int64_t ctas = dm->batch * (int64_t)b.ntiles;
         if (tc) {
-            gb = tc_groups(ctas, nsub, sms);
+            gb = tc_groups(ctas, nsub, sms, kBwdEarlyPass);
         } else {
             const int64_t want = 4 * (int64_t)sms;
             gb = ctas >= want ? 1 : (int)cdiv(want, ctas);
@@ -171,7 +176,7 @@ int auto_groups(const naju_dims* dm, int nck, int ntiles_f, bool tc, int sms) {
     const int64_t items = dm->batch * (int64_t)ntiles_f;
     // One tensor-core block per SM (its operand stages fill most of the
     // shared memory): the wave model; three CUDA-core blocks per SM.
-    if (tc) return tc_groups(items, nck, sms);
+    if (tc) return tc_groups(items, nck, sms, kFwdUpdatePass);
     const int64_t want = 3 * (int64_t)sms;
     if (items >= want) return 1;
     int64_t g = cdiv(want, items);

@@ -23,13 +23,14 @@
 // as the K-major operand and as the MN-major one (B in S = W B).
 //
 // The raw inputs of a block (u with its 3-token conv halo, a, b, z) arrive by
-// TMA into one shared buffer as soon as the previous block has read its own;
-// B and C arrive by TMA straight into their swizzled tiles once the previous
-// block's products are done.  With d_state 64 a block's y and fp32 checkpoint
-// leave through staging tiles and TMA stores (a warp's checkpoint rows are 256
-// bytes apart: direct stores would cost one memory transaction per lane).
-// Everything per (token, channel) runs on the
-// CUDA cores, 512 threads: warp w handles channels 32 (w % 4) + lane and
+// TMA into one shared buffer, requested once the previous block has read its
+// own and issued its products; B and C arrive by TMA straight into their
+// swizzled tiles once the previous block's products are done.  With d_state
+// 64 a block's y and fp32 checkpoint leave through staging tiles and TMA
+// stores (a warp's checkpoint rows are 256 bytes apart: direct stores would
+// cost one memory transaction per lane); with d_state 128 the checkpoint is
+// stored directly in 32-byte pieces.  Everything per (token, channel) runs on
+// the CUDA cores, 512 threads: warp w handles channels 32 (w % 4) + lane and
 // tokens [16 q, 16 q + 16) of the block, q = w / 4, and the state columns
 // [q N / 4, (q + 1) N / 4).
 //
